@@ -1,0 +1,94 @@
+"""Pins for the oracle's dequantization (with per-block MSE) and W4A4 GEMM reference.
+
+The dequantizer re-derives values from packed codes and scale bytes, a code
+path separate from the quantizers; it must reproduce their fused outputs bit
+for bit.  The GEMM reference (fp64 product of exactly decoded operands) is
+checked against a plain triple loop over ml_dtypes-decoded operands.
+"""
+import ml_dtypes as md
+import numpy as np
+import pytest
+
+from block_scaled_fp4_03_b200 import inputs
+
+
+def _x(kind, rows, cols, seed=0):
+    return inputs.as_f32(inputs.generate(kind, rows, cols, seed=seed))
+
+
+@pytest.mark.parametrize("B", [4, 8, 16, 32])
+@pytest.mark.parametrize("rule", [0, 1, 2, 3])
+def test_dequant_reproduces_nvfp4(O, B, rule):
+    x = _x("gaussian", 24, 128, seed=B + rule)
+    g = O.global_scale(O.amax(x))
+    q = O.nvfp4_quantize(x, B, rule, g=g)
+    d = O.dequant_mse(q["codes"], q["scales"], 24, 128, B, O.SF_E4M3, None, g=g, ref=x)
+    assert np.array_equal(d["deq"].view(np.uint32), q["deq"].view(np.uint32))
+    assert np.array_equal(d["mse"].view(np.uint32), q["mse"].view(np.uint32))
+
+
+@pytest.mark.parametrize("sf,kind,specials", [(1, "razer_weight", [5.0, -5.0, 3.5, -3.5]),
+                                              (0, "razer_act", [5.0, -5.0])])
+def test_dequant_reproduces_razer(O, sf, kind, specials):
+    x = _x(kind, 24, 256, seed=sf)
+    g = O.global_scale(O.amax(x), sf)
+    q = O.razer_quantize(x, sf, specials, g=g)
+    d = O.dequant_mse(q["codes"], q["meta"], 24, 256, 16, sf, specials, g=g, ref=x)
+    assert np.array_equal(d["deq"].view(np.uint32), q["deq"].view(np.uint32))
+    assert np.array_equal(d["mse"].view(np.uint32), q["mse"].view(np.uint32))
+
+
+def test_dequant_reproduces_mxfp4(O):
+    x = _x("mx_act", 24, 256, seed=1)
+    t = inputs.positive_vector(256, seed=4)
+    q = O.mxfp4_quantize(x, t, True, O.RULE_ABSMAX)
+    y = O.mx_transform(x, t, True)
+    d = O.dequant_mse(q["codes"], q["scales"], 24, 256, 32, O.SF_E8M0, None, ref=y)
+    assert np.array_equal(d["deq"].view(np.uint32), q["deq"].view(np.uint32))
+    assert np.array_equal(d["mse"].view(np.uint32), q["mse"].view(np.uint32))
+
+
+def test_dequant_independent_decode(O):
+    """deq = RN32(v * RN32(sc * g)) with v, sc decoded by ml_dtypes."""
+    x = _x("gaussian", 8, 64, seed=3)
+    g = O.global_scale(O.amax(x))
+    q = O.nvfp4_quantize(x, 16, O.RULE_FOUR_OVER_SIX, g=g)
+    lo, hi = q["codes"] & 0xF, q["codes"] >> 4
+    c = np.empty((8, 64), np.uint8)
+    c[:, 0::2], c[:, 1::2] = lo, hi
+    v = c.view(md.float4_e2m1fn).astype(np.float32)
+    S = (q["scales"].view(md.float8_e4m3fn).astype(np.float32) * np.float32(g)).astype(np.float32)
+    deq = (v * np.repeat(S, 16, axis=1)).astype(np.float32)
+    assert np.array_equal(deq.view(np.uint32), q["deq"].view(np.uint32))
+
+
+def test_gemm_reference_matches_triple_loop(O):
+    a = _x("gemm_act", 6, 64, seed=1)
+    w = _x("gemm_weight", 5, 64, seed=1)
+    ga = O.global_scale(O.amax(a))
+    gw = O.global_scale(O.amax(w))
+    qa = O.nvfp4_quantize(a, 16, O.RULE_FOUR_OVER_SIX, g=ga)
+    qw = O.nvfp4_quantize(w, 16, O.RULE_ABSMAX, g=gw)
+    ref = O.gemm_ref(qa["codes"], qa["scales"], ga, qw["codes"], qw["scales"], gw)
+
+    def decode(q, rows):
+        c = np.empty((rows, 64), np.uint8)
+        c[:, 0::2], c[:, 1::2] = q["codes"] & 0xF, q["codes"] >> 4
+        v = c.view(md.float4_e2m1fn).astype(np.float64)
+        s = q["scales"].view(md.float8_e4m3fn).astype(np.float64)
+        return v, s
+
+    va, sa = decode(qa, 6)
+    vw, sw = decode(qw, 5)
+    for m in range(6):
+        for n in range(5):
+            acc = 0.0
+            for k in range(64):
+                acc += (va[m, k] * sa[m, k // 16]) * (vw[n, k] * sw[n, k // 16])
+            assert abs(ref[m, n] - float(ga) * float(gw) * acc) <= 1e-12 * max(1.0, abs(ref[m, n]))
+    # and it approximates the unquantized product at FP4 accuracy
+    exact = a.astype(np.float64) @ w.astype(np.float64).T
+    assert np.linalg.norm(ref - exact) <= 0.2 * np.linalg.norm(exact)
+    sub = O.gemm_ref(qa["codes"], qa["scales"], ga, qw["codes"], qw["scales"], gw,
+                     rows=np.array([1, 4]), cols=np.array([0, 3]))
+    assert np.array_equal(sub, ref[np.ix_([1, 4], [0, 3])])
