@@ -1,0 +1,230 @@
+"""Thin Python binding of the fp4q C ABI (include/fp4q.h).
+
+Argument marshalling only: torch tensors provide device memory and the
+current CUDA stream; every step of the computation runs in the CUDA library
+``libfp4q.so``.  There is no CPU fallback -- if the library is missing or the
+tensors are not on a CUDA device, the call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+from . import build as _build
+
+F32, BF16 = 0, 1
+SF_E4M3, SF_E3M3, SF_E8M0 = 0, 1, 2
+ABSMAX, PREVENT_ZERO, FOUR_OVER_SIX, BRUTE_FORCE, HESSIAN_EXP = range(5)
+GS_NONE, GS_AMAX, GS_GIVEN = 0, 1, 2
+SF_ROWMAJOR, SF_MMA = 0, 1
+OP_QUANTIZE, OP_HESSIAN, OP_CHANNEL_SCALE, OP_GEMM = range(4)
+
+# name -> (restype, argtypes) of every exported entry point
+_vp, _i, _i64, _sz, _fp = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
+SIGNATURES = {
+    "fp4q_workspace_size": (_sz, [_i, _i64, _i64, _i64]),
+    "fp4q_status_str": (ctypes.c_char_p, [_i]),
+    "fp4q_version": (ctypes.c_char_p, []),
+    "nvfp4_quantize": (_i, [_vp, _i, _i64, _i64, _i, _i, _i, _vp, _vp, _vp, _i, _vp, _vp, _vp, _sz, _vp]),
+    "razer_quantize": (_i, [_vp, _i, _i64, _i64, _i, _vp, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "mxfp4_quantize": (_i, [_vp, _i, _i64, _i64, _vp, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "fp4_hessian_blocks": (_i, [_vp, _i, _i64, _i64, _vp, _i, _vp, _vp, _sz, _vp]),
+    "mxfp4_channel_scale": (_i, [_vp, _i, _i64, _vp, _i, _i64, _i64, _fp, _vp, _vp, _vp, _sz, _vp]),
+    "fp4_dequant_mse": (_i, [_vp, _vp, _i64, _i64, _i, _i, _vp, _i, _vp, _vp, _i, _vp, _vp, _vp]),
+}
+
+_lock = threading.Lock()
+_lib = None
+
+
+def library_path() -> str:
+    return _build.LIB
+
+
+def lib(build_if_missing: bool = True):
+    """Load libfp4q.so (compiling it in-tree first if it is missing or stale)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if build_if_missing:
+                _build.build()
+            if not os.path.exists(_build.LIB):
+                raise RuntimeError("fp4q CUDA library not built: %s" % _build.LIB)
+            L = ctypes.CDLL(_build.LIB)
+            for name, (res, args) in SIGNATURES.items():
+                fn = getattr(L, name)
+                fn.restype = res
+                fn.argtypes = args
+            _lib = L
+    return _lib
+
+
+class Fp4qError(RuntimeError):
+    pass
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        msg = lib().fp4q_status_str(status).decode()
+        raise Fp4qError("%s failed: %s (%d)" % (what, msg, status))
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return F32
+    if t.dtype == torch.bfloat16:
+        return BF16
+    raise TypeError("fp4q takes float32 or bfloat16 tensors, got %s" % t.dtype)
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None:
+            if not t.is_cuda:
+                raise ValueError("fp4q needs CUDA tensors (no CPU path)")
+            if not t.is_contiguous():
+                raise ValueError("fp4q needs contiguous tensors")
+
+
+def workspace_size(op: int, rows: int, cols: int, n: int = 0) -> int:
+    return int(lib().fp4q_workspace_size(op, rows, cols, n))
+
+
+def _workspace(op, rows, cols, n, device, ws):
+    need = workspace_size(op, rows, cols, n)
+    if ws is None and need:
+        ws = torch.empty(need, dtype=torch.uint8, device=device)
+    return ws, (0 if ws is None else ws.numel())
+
+
+def nvfp4_quantize(x: torch.Tensor, block: int = 16, rule: int = ABSMAX, gs_mode: int = GS_AMAX,
+                   global_scale: torch.Tensor | None = None, sf_layout: int = SF_ROWMAJOR,
+                   dequant: bool = False, mse: bool = False, out: dict | None = None,
+                   workspace: torch.Tensor | None = None, stream=None) -> dict:
+    """NVFP4 block quantization; returns dict(codes, scales, global_scale, dequant, mse)."""
+    _need_cuda(x)
+    rows, cols = x.shape
+    dev = x.device
+    o = out or {}
+    codes = o.get("codes") if o.get("codes") is not None else torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev)
+    scales = o.get("scales") if o.get("scales") is not None else torch.empty((rows, cols // block), dtype=torch.uint8, device=dev)
+    if global_scale is None and gs_mode != GS_NONE:
+        global_scale = o.get("global_scale") if o.get("global_scale") is not None else torch.empty(1, dtype=torch.float32, device=dev)
+    dq = (o.get("dequant") if o.get("dequant") is not None else torch.empty((rows, cols), dtype=torch.float32, device=dev)) if dequant else None
+    ms = (o.get("mse") if o.get("mse") is not None else torch.empty((rows, cols // block), dtype=torch.float32, device=dev)) if mse else None
+    ws, wsb = (workspace, workspace.numel()) if workspace is not None else (
+        _workspace(OP_QUANTIZE, rows, cols, 0, dev, None) if gs_mode == GS_AMAX else (None, 0))
+    _need_cuda(codes, scales, global_scale, dq, ms, ws)
+    st = lib().nvfp4_quantize(_ptr(x), _dtype_code(x), rows, cols, block, rule, gs_mode,
+                              _ptr(global_scale), _ptr(codes), _ptr(scales), sf_layout, _ptr(dq),
+                              _ptr(ms), _ptr(ws), wsb, _stream(stream))
+    _check(st, "nvfp4_quantize")
+    return dict(codes=codes, scales=scales, global_scale=global_scale, dequant=dq, mse=ms)
+
+
+def razer_quantize(x: torch.Tensor, scale_fmt: int, specials, gs_mode: int = GS_AMAX,
+                   global_scale: torch.Tensor | None = None, dequant: bool = False,
+                   mse: bool = False, out: dict | None = None,
+                   workspace: torch.Tensor | None = None, stream=None) -> dict:
+    """RaZeR quantization (blocks of 16); returns dict(codes, meta, global_scale, dequant, mse)."""
+    _need_cuda(x)
+    rows, cols = x.shape
+    dev = x.device
+    o = out or {}
+    codes = o.get("codes") if o.get("codes") is not None else torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev)
+    meta = o.get("meta") if o.get("meta") is not None else torch.empty((rows, cols // 16), dtype=torch.uint8, device=dev)
+    if global_scale is None and gs_mode != GS_NONE:
+        global_scale = o.get("global_scale") if o.get("global_scale") is not None else torch.empty(1, dtype=torch.float32, device=dev)
+    dq = (o.get("dequant") if o.get("dequant") is not None else torch.empty((rows, cols), dtype=torch.float32, device=dev)) if dequant else None
+    ms = (o.get("mse") if o.get("mse") is not None else torch.empty((rows, cols // 16), dtype=torch.float32, device=dev)) if mse else None
+    ws, wsb = (workspace, workspace.numel()) if workspace is not None else (
+        _workspace(OP_QUANTIZE, rows, cols, 0, dev, None) if gs_mode == GS_AMAX else (None, 0))
+    sp = (ctypes.c_float * len(specials))(*[float(v) for v in specials])
+    st = lib().razer_quantize(_ptr(x), _dtype_code(x), rows, cols, scale_fmt, ctypes.cast(sp, ctypes.c_void_p),
+                              len(specials), gs_mode, _ptr(global_scale), _ptr(codes), _ptr(meta),
+                              _ptr(dq), _ptr(ms), _ptr(ws), wsb, _stream(stream))
+    _check(st, "razer_quantize")
+    return dict(codes=codes, meta=meta, global_scale=global_scale, dequant=dq, mse=ms)
+
+
+def mxfp4_quantize(x: torch.Tensor, chan_scale: torch.Tensor | None = None, hadamard: bool = True,
+                   rule: int = ABSMAX, hess: torch.Tensor | None = None, dequant: bool = False,
+                   mse: bool = False, out: dict | None = None, stream=None) -> dict:
+    """MXFP4 quantization with the online transform; returns dict(codes, scales, dequant, mse)."""
+    _need_cuda(x, chan_scale, hess)
+    rows, cols = x.shape
+    dev = x.device
+    o = out or {}
+    codes = o.get("codes") if o.get("codes") is not None else torch.empty((rows, cols // 2), dtype=torch.uint8, device=dev)
+    scales = o.get("scales") if o.get("scales") is not None else torch.empty((rows, cols // 32), dtype=torch.uint8, device=dev)
+    dq = (o.get("dequant") if o.get("dequant") is not None else torch.empty((rows, cols), dtype=torch.float32, device=dev)) if dequant else None
+    ms = (o.get("mse") if o.get("mse") is not None else torch.empty((rows, cols // 32), dtype=torch.float32, device=dev)) if mse else None
+    st = lib().mxfp4_quantize(_ptr(x), _dtype_code(x), rows, cols, _ptr(chan_scale), int(bool(hadamard)),
+                              rule, _ptr(hess), _ptr(codes), _ptr(scales), _ptr(dq), _ptr(ms),
+                              _stream(stream))
+    _check(st, "mxfp4_quantize")
+    return dict(codes=codes, scales=scales, dequant=dq, mse=ms)
+
+
+def hessian_blocks(x: torch.Tensor, chan_scale: torch.Tensor | None = None, hadamard: bool = True,
+                   out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                   stream=None) -> torch.Tensor:
+    """H'_k = X'_k^T X'_k for every 32-column block; returns [cols/32, 32, 32] fp32."""
+    _need_cuda(x, chan_scale)
+    rows, cols = x.shape
+    dev = x.device
+    h = out if out is not None else torch.empty((cols // 32, 32, 32), dtype=torch.float32, device=dev)
+    ws, wsb = (workspace, workspace.numel()) if workspace is not None else _workspace(OP_HESSIAN, rows, cols, 0, dev, None)
+    st = lib().fp4_hessian_blocks(_ptr(x), _dtype_code(x), rows, cols, _ptr(chan_scale),
+                                  int(bool(hadamard)), _ptr(h), _ptr(ws), wsb, _stream(stream))
+    _check(st, "fp4_hessian_blocks")
+    return h
+
+
+def channel_scale(x: torch.Tensor, w: torch.Tensor, alpha: float = 0.75, out=None,
+                  workspace: torch.Tensor | None = None, stream=None):
+    """Online per-channel scale t and 1/t ([tokens, cols] activations, [n_out, cols] weights)."""
+    _need_cuda(x, w)
+    tokens, cols = x.shape
+    n_out = w.shape[0]
+    dev = x.device
+    t = out[0] if out is not None else torch.empty(cols, dtype=torch.float32, device=dev)
+    ti = out[1] if out is not None else torch.empty(cols, dtype=torch.float32, device=dev)
+    ws, wsb = (workspace, workspace.numel()) if workspace is not None else _workspace(OP_CHANNEL_SCALE, tokens, cols, n_out, dev, None)
+    st = lib().mxfp4_channel_scale(_ptr(x), _dtype_code(x), tokens, _ptr(w), _dtype_code(w), n_out,
+                                   cols, float(alpha), _ptr(t), _ptr(ti), _ptr(ws), wsb,
+                                   _stream(stream))
+    _check(st, "mxfp4_channel_scale")
+    return t, ti
+
+
+def dequant_mse(codes: torch.Tensor, scales: torch.Tensor, rows: int, cols: int, block: int,
+                scale_fmt: int, specials=None, global_scale: torch.Tensor | None = None,
+                ref: torch.Tensor | None = None, want_dequant: bool = True, stream=None) -> dict:
+    _need_cuda(codes, scales, global_scale, ref)
+    dev = codes.device
+    dq = torch.empty((rows, cols), dtype=torch.float32, device=dev) if want_dequant else None
+    ms = torch.empty((rows, cols // block), dtype=torch.float32, device=dev) if ref is not None else None
+    sp = None
+    n_sp = 0
+    if specials is not None:
+        n_sp = len(specials)
+        sp = (ctypes.c_float * n_sp)(*[float(v) for v in specials])
+    st = lib().fp4_dequant_mse(_ptr(codes), _ptr(scales), rows, cols, block, scale_fmt,
+                               None if sp is None else ctypes.cast(sp, ctypes.c_void_p), n_sp,
+                               _ptr(global_scale), _ptr(ref), 0 if ref is None else _dtype_code(ref),
+                               _ptr(dq), _ptr(ms), _stream(stream))
+    _check(st, "fp4_dequant_mse")
+    return dict(dequant=dq, mse=ms)

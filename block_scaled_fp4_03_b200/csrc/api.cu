@@ -1,0 +1,255 @@
+// api.cu -- the C ABI declared in include/fp4q.h: argument checking on the
+// host, then launches on the caller's stream.  No allocation, no state.
+#include <cmath>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/fp4q.h"
+#include "fp4q_internal.h"
+
+using namespace fp4q;
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned_or_null(const void* p) { return p == nullptr || aligned16(p); }
+bool valid_block(int b) { return b == 4 || b == 8 || b == 16 || b == 32; }
+bool valid_dtype(int d) { return d == FP4Q_F32 || d == FP4Q_BF16; }
+cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+int from_cuda(cudaError_t e) { return e == cudaSuccess ? FP4Q_OK : FP4Q_ERR_CUDA; }
+
+constexpr size_t kQuantWs = 4096;   // >= kAmaxPartials floats, rounded up
+static_assert(kAmaxPartials * sizeof(float) <= kQuantWs, "amax partials must fit");
+
+// Resolve a global-scale request into launch arguments (running the amax
+// pre-pass for AMAX).  Returns FP4Q_OK or an error.
+int prepare_gs(int gs_mode, float denom, const void* x, int dtype, int64_t n, float* global_scale,
+               void* ws, size_t ws_bytes, cudaStream_t s, GsArgs& gs)
+{
+    gs = GsArgs{};
+    gs.mode = gs_mode;
+    gs.denom = denom;
+    if (gs_mode == FP4Q_GS_NONE)
+        return FP4Q_OK;
+    if (gs_mode == FP4Q_GS_GIVEN) {
+        if (!global_scale)
+            return FP4Q_ERR_ARG;
+        gs.given = global_scale;
+        return FP4Q_OK;
+    }
+    if (gs_mode != FP4Q_GS_AMAX)
+        return FP4Q_ERR_ARG;
+    if (!ws || ws_bytes < kQuantWs)
+        return FP4Q_ERR_WORKSPACE;
+    if (!aligned16(ws))
+        return FP4Q_ERR_ALIGN;
+    gs.partials = reinterpret_cast<const float*>(ws);
+    gs.n_partials = kAmaxPartials;
+    gs.out = global_scale;
+    return from_cuda(launch_amax(x, dtype, n, reinterpret_cast<float*>(ws), s));
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t fp4q_workspace_size(int op, int64_t rows, int64_t cols, int64_t n)
+{
+    if (rows < 0 || cols < 0 || n < 0)
+        return 0;
+    switch (op) {
+    case FP4Q_OP_QUANTIZE: return kQuantWs;
+    case FP4Q_OP_HESSIAN: return cols % 32 ? 0 : hessian_ws_bytes(rows, cols);
+    case FP4Q_OP_CHANNEL_SCALE: return channel_scale_ws_bytes(rows, n, cols);
+    default: return 0;
+    }
+}
+
+const char* fp4q_status_str(int status)
+{
+    switch (status) {
+    case FP4Q_OK: return "ok";
+    case FP4Q_ERR_ARG: return "invalid argument";
+    case FP4Q_ERR_ALIGN: return "misaligned pointer";
+    case FP4Q_ERR_UNSUPPORTED: return "unsupported";
+    case FP4Q_ERR_CUDA: return "CUDA error";
+    case FP4Q_ERR_TIMEOUT: return "device wait timed out";
+    case FP4Q_ERR_WORKSPACE: return "workspace missing or too small";
+    default: return "unknown status";
+    }
+}
+
+const char* fp4q_version(void) { return "fp4q 0.1.0 sm_100a"; }
+
+int nvfp4_quantize(const void* x, int dtype, int64_t rows, int64_t cols, int block, int rule,
+                   int gs_mode, float* global_scale, uint8_t* codes, uint8_t* scales,
+                   int sf_layout, float* dequant, float* block_mse, void* workspace,
+                   size_t workspace_bytes, void* stream)
+{
+    const bool empty = rows == 0 || cols == 0;   // empty tensors may come with NULL buffers
+    if ((!empty && (!x || !codes || !scales)) || !valid_dtype(dtype) || rows < 0 || cols < 0)
+        return FP4Q_ERR_ARG;
+    if (!valid_block(block) || cols % block != 0)
+        return FP4Q_ERR_ARG;
+    if (rule < FP4Q_ABSMAX || rule > FP4Q_BRUTE_FORCE)
+        return FP4Q_ERR_ARG;
+    if (gs_mode < FP4Q_GS_NONE || gs_mode > FP4Q_GS_GIVEN)
+        return FP4Q_ERR_ARG;
+    if (sf_layout == FP4Q_SFLAYOUT_MMA) {
+        if (block != 16 || rows % 128 != 0 || (cols / 16) % 4 != 0)
+            return FP4Q_ERR_ARG;
+    } else if (sf_layout != FP4Q_SFLAYOUT_ROWMAJOR) {
+        return FP4Q_ERR_ARG;
+    }
+    if (!aligned16(x) || !aligned16(codes) || !aligned_or_null(dequant) ||
+        !aligned_or_null(global_scale) || !aligned_or_null(block_mse))
+        return FP4Q_ERR_ALIGN;
+    cudaStream_t s = as_stream(stream);
+    GsArgs gs;
+    int st = prepare_gs(gs_mode, 2688.0f, x, dtype, rows * cols, global_scale, workspace,
+                        workspace_bytes, s, gs);
+    if (st != FP4Q_OK)
+        return st;
+    return from_cuda(launch_nvfp4_quant(x, dtype, rows, cols, block, rule, gs, codes, scales,
+                                        sf_layout == FP4Q_SFLAYOUT_MMA, dequant, block_mse, s));
+}
+
+int razer_quantize(const void* x, int dtype, int64_t rows, int64_t cols, int scale_fmt,
+                   const float* specials, int n_special, int gs_mode, float* global_scale,
+                   uint8_t* codes, uint8_t* meta, float* dequant, float* block_mse,
+                   void* workspace, size_t workspace_bytes, void* stream)
+{
+    const bool empty = rows == 0 || cols == 0;
+    if ((!empty && (!x || !codes || !meta)) || !specials || !valid_dtype(dtype) || rows < 0 ||
+        cols < 0)
+        return FP4Q_ERR_ARG;
+    if (cols % 16 != 0)
+        return FP4Q_ERR_ARG;
+    if (scale_fmt == FP4Q_SF_E3M3) {
+        if (n_special < 1 || n_special > 4)
+            return FP4Q_ERR_ARG;
+    } else if (scale_fmt == FP4Q_SF_E4M3) {
+        if (n_special < 1 || n_special > 2)
+            return FP4Q_ERR_ARG;
+    } else {
+        return FP4Q_ERR_ARG;
+    }
+    for (int i = 0; i < n_special; ++i) {
+        const float v = specials[i];
+        const float twice = v * 2.0f;
+        if (!(std::fabs(v) <= 32.0f) || v == 0.0f || twice != std::nearbyint(twice))
+            return FP4Q_ERR_ARG;
+    }
+    if (gs_mode < FP4Q_GS_NONE || gs_mode > FP4Q_GS_GIVEN)
+        return FP4Q_ERR_ARG;
+    if (!aligned16(x) || !aligned16(codes) || !aligned_or_null(dequant) ||
+        !aligned_or_null(global_scale) || !aligned_or_null(block_mse))
+        return FP4Q_ERR_ALIGN;
+    cudaStream_t s = as_stream(stream);
+    GsArgs gs;
+    const float denom = scale_fmt == FP4Q_SF_E3M3 ? 180.0f : 2688.0f;
+    int st = prepare_gs(gs_mode, denom, x, dtype, rows * cols, global_scale, workspace,
+                        workspace_bytes, s, gs);
+    if (st != FP4Q_OK)
+        return st;
+    return from_cuda(launch_razer_quant(x, dtype, rows, cols, scale_fmt, specials, n_special, gs,
+                                        codes, meta, dequant, block_mse, s));
+}
+
+int mxfp4_quantize(const void* x, int dtype, int64_t rows, int64_t cols,
+                   const float* chan_scale, int hadamard32, int rule, const float* hess_blocks,
+                   uint8_t* codes, uint8_t* scales, float* dequant, float* block_mse,
+                   void* stream)
+{
+    const bool empty = rows == 0 || cols == 0;
+    if ((!empty && (!x || !codes || !scales)) || !valid_dtype(dtype) || rows < 0 || cols < 0 ||
+        cols % 32 != 0)
+        return FP4Q_ERR_ARG;
+    if (rule != FP4Q_ABSMAX && rule != FP4Q_HESSIAN_EXP)
+        return FP4Q_ERR_ARG;
+    if (rule == FP4Q_HESSIAN_EXP && !hess_blocks)
+        return FP4Q_ERR_ARG;
+    if (!aligned16(x) || !aligned16(codes) || !aligned_or_null(chan_scale) ||
+        !aligned_or_null(hess_blocks) || !aligned_or_null(dequant) || !aligned_or_null(block_mse))
+        return FP4Q_ERR_ALIGN;
+    if (rows == 0 || cols == 0)
+        return FP4Q_OK;
+    return from_cuda(launch_mxfp4_quant(x, dtype, rows, cols, chan_scale, hadamard32 != 0, rule,
+                                        hess_blocks, codes, scales, dequant, block_mse,
+                                        as_stream(stream)));
+}
+
+int fp4_hessian_blocks(const void* x, int dtype, int64_t rows, int64_t cols,
+                       const float* chan_scale, int hadamard32, float* hess_blocks,
+                       void* workspace, size_t workspace_bytes, void* stream)
+{
+    if (!x || !hess_blocks || !valid_dtype(dtype) || rows < 0 || cols < 0 || cols % 32 != 0)
+        return FP4Q_ERR_ARG;
+    if (!aligned16(x) || !aligned16(hess_blocks) || !aligned_or_null(chan_scale))
+        return FP4Q_ERR_ALIGN;
+    if (cols == 0)
+        return FP4Q_OK;
+    const size_t need = hessian_ws_bytes(rows, cols);
+    if (need > 0 && (!workspace || workspace_bytes < need))
+        return FP4Q_ERR_WORKSPACE;
+    if (!aligned_or_null(workspace))
+        return FP4Q_ERR_ALIGN;
+    if (rows == 0)
+        return from_cuda(cudaMemsetAsync(hess_blocks, 0, (size_t)(cols / 32) * 1024 * sizeof(float),
+                                         as_stream(stream)));
+    return from_cuda(launch_hessian_blocks(x, dtype, rows, cols, chan_scale, hadamard32 != 0,
+                                           hess_blocks, workspace, as_stream(stream)));
+}
+
+int mxfp4_channel_scale(const void* x, int x_dtype, int64_t tokens, const void* w,
+                        int w_dtype, int64_t n_out, int64_t cols, float alpha, float* t,
+                        float* t_inv, void* workspace, size_t workspace_bytes, void* stream)
+{
+    if (!x || !w || !t || !valid_dtype(x_dtype) || !valid_dtype(w_dtype))
+        return FP4Q_ERR_ARG;
+    if (tokens <= 0 || n_out <= 0 || cols <= 0 || cols % 8 != 0 || !(std::isfinite(alpha)))
+        return FP4Q_ERR_ARG;
+    if (!aligned16(x) || !aligned16(w) || !aligned16(t) || !aligned_or_null(t_inv))
+        return FP4Q_ERR_ALIGN;
+    const size_t need = channel_scale_ws_bytes(tokens, n_out, cols);
+    if (!workspace || workspace_bytes < need)
+        return FP4Q_ERR_WORKSPACE;
+    if (!aligned16(workspace))
+        return FP4Q_ERR_ALIGN;
+    return from_cuda(launch_mx_channel_scale(x, x_dtype, tokens, w, w_dtype, n_out, cols, alpha, t,
+                                             t_inv, workspace, as_stream(stream)));
+}
+
+int fp4_dequant_mse(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t cols,
+                    int block, int scale_fmt, const float* specials, int n_special,
+                    const float* global_scale, const void* ref, int ref_dtype, float* dequant,
+                    float* block_mse, void* stream)
+{
+    const bool empty = rows == 0 || cols == 0;
+    if ((!empty && (!codes || !scales)) || rows < 0 || cols < 0 || !valid_block(block) ||
+        cols % block != 0)
+        return FP4Q_ERR_ARG;
+    if (scale_fmt < FP4Q_SF_E4M3 || scale_fmt > FP4Q_SF_E8M0)
+        return FP4Q_ERR_ARG;
+    if (scale_fmt == FP4Q_SF_E8M0 && (block != 32 || specials))
+        return FP4Q_ERR_ARG;
+    if (specials) {
+        if (block != 16 || n_special < 1 || n_special > (scale_fmt == FP4Q_SF_E3M3 ? 4 : 2))
+            return FP4Q_ERR_ARG;
+    }
+    if (block_mse && !ref && !empty)
+        return FP4Q_ERR_ARG;
+    if (ref && !valid_dtype(ref_dtype))
+        return FP4Q_ERR_ARG;
+    if (!aligned16(codes) || !aligned_or_null(ref) || !aligned_or_null(dequant) ||
+        !aligned_or_null(block_mse) || !aligned_or_null(global_scale))
+        return FP4Q_ERR_ALIGN;
+    if (rows == 0 || cols == 0)
+        return FP4Q_OK;
+    return from_cuda(launch_dequant_mse(codes, scales, rows, cols, block, scale_fmt, specials,
+                                        specials ? n_special : 0, global_scale, ref, ref_dtype,
+                                        dequant, block_mse, as_stream(stream)));
+}
+
+}  // extern "C"

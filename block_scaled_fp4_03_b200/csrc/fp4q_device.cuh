@@ -1,0 +1,215 @@
+// fp4q_device.cuh -- device-side format conversions shared by the quantizer,
+// dequantizer and GEMM kernels of the fp4q library (sm_100a only).
+//
+// Formats (see the public header for the page citations):
+//   E2M1 element  : sign<<3 | magnitude index, magnitudes {0,.5,1,1.5,2,3,4,6}
+//   E4M3 scale    : OCP E4M3FN, largest finite 448
+//   E3M3 scale    : 6-bit unsigned, bias 3, 2^-5 .. 30
+//   E8M0 scale    : 2^(byte-127)
+//
+// All fp32 arithmetic that decides a code or produces an output goes through
+// explicit round-to-nearest intrinsics (__fmul_rn, __fsub_rn, __fmaf_rn) and
+// the library is compiled with -fmad=false, so no contraction changes a
+// rounding behind our back.
+#pragma once
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+namespace fp4q {
+
+constexpr float kFltMax = 3.402823466e+38f;
+
+// ---------------------------------------------------------------- E2M1
+// Encode 8 fp32 values to 8 E2M1 codes (RNE, saturating, sign kept), value i
+// in nibble i of the result.
+__device__ __forceinline__ uint32_t e2m1x8_encode(float y0, float y1, float y2, float y3,
+                                                  float y4, float y5, float y6, float y7)
+{
+    uint32_t out;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(out)
+        : "f"(y0), "f"(y1), "f"(y2), "f"(y3), "f"(y4), "f"(y5), "f"(y6), "f"(y7));
+    return out;
+}
+
+// Encode 4 values into the low 16 bits.
+__device__ __forceinline__ uint32_t e2m1x4_encode(float y0, float y1, float y2, float y3)
+{
+    uint32_t out;
+    asm("{\n\t.reg .b8 b0, b1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "mov.b32 %0, {b0, b1, b1, b1};\n\t}"
+        : "=r"(out)
+        : "f"(y0), "f"(y1), "f"(y2), "f"(y3));
+    return out & 0xFFFFu;
+}
+
+// Decode the two E2M1 codes of one byte (low nibble first) to fp32; exact.
+// The byte is handed to the conversion as the low half of a zero-extended
+// 16-bit register, one conversion per byte.
+__device__ __forceinline__ float2 e2m1x2_decode(uint32_t byte)
+{
+    uint32_t h2;
+    const unsigned short b16 = (unsigned short)(byte & 0xFFu);
+    asm("{\n\t.reg .b8 lo, hi;\n\t"
+        "mov.b16 {lo, hi}, %1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, lo;\n\t}"
+        : "=r"(h2)
+        : "h"(b16));
+    return __half22float2(*reinterpret_cast<__half2*>(&h2));
+}
+
+// Decode 8 E2M1 codes (nibble i = value i) to fp32; exact.
+__device__ __forceinline__ void e2m1x8_decode(uint32_t w, float (&v)[8])
+{
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const float2 f = e2m1x2_decode(w >> (8 * k));
+        v[2 * k] = f.x;
+        v[2 * k + 1] = f.y;
+    }
+}
+
+// Decode the low 4 nibbles.
+__device__ __forceinline__ void e2m1x4_decode(uint32_t w, float (&v)[4])
+{
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        const float2 f = e2m1x2_decode(w >> (8 * k));
+        v[2 * k] = f.x;
+        v[2 * k + 1] = f.y;
+    }
+}
+
+// ---------------------------------------------------------------- E4M3
+// Non-negative r -> E4M3 code (RNE, saturating at 448).
+__device__ __forceinline__ uint32_t e4m3_encode(float r)
+{
+    uint16_t out;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %2, %1;" : "=h"(out) : "f"(r), "f"(0.0f));
+    return out & 0xFFu;
+}
+
+// E4M3 code (low 8 bits; sign bit honoured) -> fp32; exact.
+__device__ __forceinline__ float e4m3_decode(uint32_t code)
+{
+    uint32_t h;
+    uint16_t c = (uint16_t)(code & 0xFFu);
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(c));
+    return __half2float(__ushort_as_half((unsigned short)(h & 0xFFFFu)));
+}
+
+// ---------------------------------------------------------------- E3M3
+// Non-negative r -> E3M3 code, RNE, saturating at 30.  Below 2^-2 the format
+// is a fixed-point grid of step 2^-5 (rint of r*32, ties to even = even code);
+// from 2^-2 to 30 it has E4M3's 3-bit mantissa, so the E4M3 code shifted by
+// 4 exponent steps is the answer, clamped at 30.
+__device__ __forceinline__ uint32_t e3m3_encode(float r)
+{
+    if (r < 0.25f)
+        return (uint32_t)rintf(__fmul_rn(r, 32.0f));
+    uint32_t c4 = e4m3_encode(r);
+    c4 = c4 > 0x5Fu ? 0x5Fu : c4;     // 0x5F = 30 in E4M3
+    return c4 - 32u;
+}
+
+__device__ __forceinline__ float e3m3_decode(uint32_t code)
+{
+    code &= 0x3Fu;
+    if (code < 8u)
+        return __fmul_rn((float)code, 0.03125f);
+    return e4m3_decode(code + 32u);
+}
+
+// ---------------------------------------------------------------- loads
+// Load N consecutive input elements starting at p (16-byte aligned when the
+// byte count allows) into fp32 registers.
+template <int N>
+__device__ __forceinline__ void load_f32(const float* __restrict__ p, float (&x)[N])
+{
+    static_assert(N % 4 == 0, "fp32 loads come in float4");
+#pragma unroll
+    for (int i = 0; i < N; i += 4) {
+        float4 v = __ldg(reinterpret_cast<const float4*>(p + i));
+        x[i] = v.x; x[i + 1] = v.y; x[i + 2] = v.z; x[i + 3] = v.w;
+    }
+}
+
+__device__ __forceinline__ void bf16x2_to_f32(uint32_t w, float& lo, float& hi)
+{
+    lo = __uint_as_float(w << 16);
+    hi = __uint_as_float(w & 0xFFFF0000u);
+}
+
+template <int N>
+__device__ __forceinline__ void load_bf16(const __nv_bfloat16* __restrict__ p, float (&x)[N])
+{
+    static_assert(N % 4 == 0, "bf16 loads come in groups of 4");
+    if constexpr (N % 8 == 0) {
+#pragma unroll
+        for (int i = 0; i < N; i += 8) {
+            uint4 v = __ldg(reinterpret_cast<const uint4*>(p + i));
+            bf16x2_to_f32(v.x, x[i], x[i + 1]);
+            bf16x2_to_f32(v.y, x[i + 2], x[i + 3]);
+            bf16x2_to_f32(v.z, x[i + 4], x[i + 5]);
+            bf16x2_to_f32(v.w, x[i + 6], x[i + 7]);
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < N; i += 4) {
+            uint2 v = __ldg(reinterpret_cast<const uint2*>(p + i));
+            bf16x2_to_f32(v.x, x[i], x[i + 1]);
+            bf16x2_to_f32(v.y, x[i + 2], x[i + 3]);
+        }
+    }
+}
+
+template <typename T, int N>
+__device__ __forceinline__ void load_elems(const T* __restrict__ p, float (&x)[N])
+{
+    if constexpr (sizeof(T) == 4)
+        load_f32<N>(reinterpret_cast<const float*>(p), x);
+    else
+        load_bf16<N>(reinterpret_cast<const __nv_bfloat16*>(p), x);
+}
+
+template <int N>
+__device__ __forceinline__ void store_f32(float* __restrict__ p, const float (&x)[N])
+{
+#pragma unroll
+    for (int i = 0; i < N; i += 4)
+        *reinterpret_cast<float4*>(p + i) = make_float4(x[i], x[i + 1], x[i + 2], x[i + 3]);
+}
+
+// Store the packed codes of one block: N/2 bytes from the words w[].
+template <int N>
+__device__ __forceinline__ void store_codes(uint8_t* __restrict__ p, const uint32_t (&w)[(N + 7) / 8])
+{
+    if constexpr (N == 4)
+        *reinterpret_cast<uint16_t*>(p) = (uint16_t)w[0];
+    else if constexpr (N == 8)
+        *reinterpret_cast<uint32_t*>(p) = w[0];
+    else if constexpr (N == 16)
+        *reinterpret_cast<uint2*>(p) = make_uint2(w[0], w[1]);
+    else
+        *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// Offset of scale (row r, scale column kb) in the tcgen05 block-scaled MMA
+// scale-factor layout: 128-row x 4-column atoms of 512 bytes, atoms ordered
+// with the scale-column index fastest; inside an atom, row r goes to
+// 16*(r%32) + 4*((r/32)%4) and column kb to kb%4.
+__device__ __forceinline__ int64_t mma_sf_offset(int64_t r, int64_t kb, int64_t kb_atoms)
+{
+    return ((r >> 7) * kb_atoms + (kb >> 2)) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (kb & 3);
+}
+
+}  // namespace fp4q

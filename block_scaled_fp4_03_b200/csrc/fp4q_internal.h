@@ -1,0 +1,59 @@
+// fp4q_internal.h -- launchers behind the C ABI of include/fp4q.h.
+// Every launcher enqueues on `stream` and returns the cudaError_t of its
+// launches; argument checking is done by the C ABI layer before these run.
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace fp4q {
+
+// Global-scale source for a quantizer launch.
+struct GsArgs {
+    int mode;                 // 0 none (g = 1), 1 amax partials in ws, 2 given (device float)
+    const float* partials;    // mode 1: per-CTA block maxima written by launch_amax
+    int n_partials;
+    float denom;              // mode 1: 6 * largest scale of the format (2688 or 180)
+    const float* given;       // mode 2
+    float* out;               // nullable: where to write the g that was used
+};
+
+// Number of partial maxima launch_amax writes (fixed; the workspace holds them).
+constexpr int kAmaxPartials = 592;   // 148 SMs x 4
+
+int num_sms();
+
+cudaError_t launch_amax(const void* x, int dtype, int64_t n, float* partials, cudaStream_t s);
+
+cudaError_t launch_nvfp4_quant(const void* x, int dtype, int64_t rows, int64_t cols, int block,
+                               int rule, const GsArgs& gs, uint8_t* codes, uint8_t* scales,
+                               int mma_layout, float* deq, float* mse, cudaStream_t s);
+
+cudaError_t launch_razer_quant(const void* x, int dtype, int64_t rows, int64_t cols, int sf,
+                               const float* specials_host, int n_special, const GsArgs& gs,
+                               uint8_t* codes, uint8_t* meta, float* deq, float* mse,
+                               cudaStream_t s);
+
+cudaError_t launch_dequant_mse(const uint8_t* codes, const uint8_t* scales, int64_t rows,
+                               int64_t cols, int block, int sf, const float* specials_host,
+                               int n_special, const float* gs_dev, const void* ref, int ref_dt,
+                               float* deq, float* mse, cudaStream_t s);
+
+cudaError_t launch_mx_channel_scale(const void* x, int xdt, int64_t tokens, const void* w, int wdt,
+                                    int64_t n_out, int64_t cols, float alpha, float* t,
+                                    float* t_inv, void* ws, cudaStream_t s);
+
+cudaError_t launch_hessian_blocks(const void* x, int dtype, int64_t rows, int64_t cols,
+                                  const float* chan_scale, int hadamard, float* hess, void* ws,
+                                  cudaStream_t s);
+
+cudaError_t launch_mxfp4_quant(const void* x, int dtype, int64_t rows, int64_t cols,
+                               const float* chan_scale, int hadamard, int rule, const float* hess,
+                               uint8_t* codes, uint8_t* scales, float* deq, float* mse,
+                               cudaStream_t s);
+
+// Workspace (bytes) launch_hessian_blocks / launch_mx_channel_scale need.
+size_t hessian_ws_bytes(int64_t rows, int64_t cols);
+size_t channel_scale_ws_bytes(int64_t tokens, int64_t n_out, int64_t cols);
+
+}  // namespace fp4q

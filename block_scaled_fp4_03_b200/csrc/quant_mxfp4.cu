@@ -1,0 +1,492 @@
+// quant_mxfp4.cu -- the MXFP4 path of MACaQ ("MACaQ: Fast, Model Agnostic
+// Calibrated Quantization ..." review, section 1 Key Terms and section 3
+// Method): per-channel online scale t, size-32 block-Hadamard rotation, OCP
+// E8M0 shared exponent, Hessian-weighted exponent choice among the standard
+// exponent plus {+1, 0, -1}, the 32x32 diagonal Hessian blocks it weights
+// with, and the calibration of t from weight and activation statistics.
+//
+// Layout: row-major tensors, 32-element blocks along the last dimension.
+// Every quantization decision is made by one thread per block in fp32 with
+// explicit round-to-nearest operations, in the same order as the definition.
+#include <cfloat>
+#include <cstdint>
+
+#include "fp4q_device.cuh"
+#include "fp4q_internal.h"
+
+namespace fp4q {
+
+namespace {
+
+constexpr int kThreads = 256;
+
+// fp32 nearest to 1/sqrt(32) (the Hadamard normalisation), bit pattern 0x3E3504F3.
+__device__ __forceinline__ float had_norm() { return __uint_as_float(0x3E3504F3u); }
+
+// 2^e as fp32 for e in [-127, 127] (2^-127 is the subnormal 0x00400000).
+__device__ __forceinline__ float pow2f(int e)
+{
+    return e <= -127 ? __uint_as_float(0x00400000u) : __uint_as_float((uint32_t)(e + 127) << 23);
+}
+
+// u <- (u * t) then the in-register Sylvester butterflies for strides 1..16
+// and the 1/sqrt(32) normalisation.
+__device__ __forceinline__ void online_transform(float (&u)[32], const float* __restrict__ t,
+                                                 bool had)
+{
+    if (t) {
+#pragma unroll
+        for (int i = 0; i < 32; i += 4) {
+            float4 tv = __ldg(reinterpret_cast<const float4*>(t + i));
+            u[i] = __fmul_rn(u[i], tv.x);
+            u[i + 1] = __fmul_rn(u[i + 1], tv.y);
+            u[i + 2] = __fmul_rn(u[i + 2], tv.z);
+            u[i + 3] = __fmul_rn(u[i + 3], tv.w);
+        }
+    }
+    if (had) {
+#pragma unroll
+        for (int h = 1; h < 32; h <<= 1) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                if ((i & h) == 0) {
+                    const float p = u[i], q = u[i + h];
+                    u[i] = __fadd_rn(p, q);
+                    u[i + h] = __fsub_rn(p, q);
+                }
+            }
+        }
+        const float c = had_norm();
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            u[i] = __fmul_rn(u[i], c);
+    }
+}
+
+// OCP MX shared exponent: floor(log2 a) - 2, clamped to [-127, 127]; a
+// subnormal or zero block maximum gives -127.
+__device__ __forceinline__ int mx_exponent(float a)
+{
+    const uint32_t E = __float_as_uint(a) >> 23;   // a >= 0
+    if (E == 0u)
+        return -127;
+    const int e = (int)E - 129;
+    return e < -127 ? -127 : e;
+}
+
+// Quantize one 32-block at exponent e: codes, deq, ordered squared error.
+__device__ __forceinline__ float mx_eval(const float (&u)[32], int e, uint32_t (&cw)[4],
+                                         float (&dq)[32])
+{
+    const float down = pow2f(-e);
+    const float up = pow2f(e);
+    float acc = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int o = 8 * j;
+        uint32_t w = e2m1x8_encode(__fmul_rn(u[o], down), __fmul_rn(u[o + 1], down),
+                                   __fmul_rn(u[o + 2], down), __fmul_rn(u[o + 3], down),
+                                   __fmul_rn(u[o + 4], down), __fmul_rn(u[o + 5], down),
+                                   __fmul_rn(u[o + 6], down), __fmul_rn(u[o + 7], down));
+        float v[8];
+        e2m1x8_decode(w, v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float d = __fmul_rn(v[i], up);
+            const float er = __fsub_rn(u[o + i], d);
+            acc = __fmaf_rn(er, er, acc);
+            dq[o + i] = d;
+        }
+        cw[j] = w;
+    }
+    return acc;
+}
+
+template <typename T>
+__device__ __forceinline__ void load32(const T* __restrict__ p, float (&u)[32])
+{
+    load_elems<T, 32>(p, u);
+}
+
+// ------------------------------------------------- OCP exponent (activations)
+template <typename T>
+__global__ void __launch_bounds__(kThreads)
+mx_quant_absmax_kernel(const T* __restrict__ x, int64_t nblk, int64_t kb,
+                       const float* __restrict__ t, int had, uint8_t* __restrict__ codes,
+                       uint8_t* __restrict__ scales, float* __restrict__ deq,
+                       float* __restrict__ mse)
+{
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblk; b += stride) {
+        float u[32];
+        load32<T>(x + b * 32, u);
+        online_transform(u, t ? t + (b % kb) * 32 : nullptr, had != 0);
+        float a = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            a = fmaxf(a, fabsf(u[i]));
+        const int e = mx_exponent(a);
+        uint32_t cw[4];
+        float dq[32];
+        const float sse = mx_eval(u, e, cw, dq);
+        *reinterpret_cast<uint4*>(codes + b * 16) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+        scales[b] = (uint8_t)(e + 127);
+        if (deq)
+            store_f32<32>(deq + b * 32, dq);
+        if (mse)
+            mse[b] = __fmul_rn(sse, 1.0f / 32.0f);
+    }
+}
+
+// d^T H d for the block error d = u - deq(u, e): v_i = sum_j H_ij d_j and the
+// outer sum, each accumulated with fma in index order.  Ht holds H transposed
+// (row j of Ht = column j of H, one 128-byte broadcast read); ds is this
+// thread's slice of a [32][kThreads] shared buffer through which d_j is read
+// inside a rolled j loop, keeping one H row in flight at a time.
+__device__ __forceinline__ float hess_cost(const float (&u)[32], int e, const float* Ht, float* ds)
+{
+    const float down = pow2f(-e);
+    const float up = pow2f(e);
+    float d[32];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int o = 8 * j;
+        uint32_t w = e2m1x8_encode(__fmul_rn(u[o], down), __fmul_rn(u[o + 1], down),
+                                   __fmul_rn(u[o + 2], down), __fmul_rn(u[o + 3], down),
+                                   __fmul_rn(u[o + 4], down), __fmul_rn(u[o + 5], down),
+                                   __fmul_rn(u[o + 6], down), __fmul_rn(u[o + 7], down));
+        float v[8];
+        e2m1x8_decode(w, v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            d[o + i] = __fsub_rn(u[o + i], __fmul_rn(v[i], up));
+            ds[(o + i) * kThreads] = d[o + i];
+        }
+    }
+    float v[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+        v[i] = 0.0f;
+#pragma unroll 1
+    for (int j = 0; j < 32; ++j) {
+        const float dj = ds[j * kThreads];
+#pragma unroll
+        for (int i = 0; i < 32; i += 4) {
+            const float4 h = *reinterpret_cast<const float4*>(&Ht[j * 32 + i]);
+            v[i] = __fmaf_rn(h.x, dj, v[i]);
+            v[i + 1] = __fmaf_rn(h.y, dj, v[i + 1]);
+            v[i + 2] = __fmaf_rn(h.z, dj, v[i + 2]);
+            v[i + 3] = __fmaf_rn(h.w, dj, v[i + 3]);
+        }
+    }
+    float cost = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+        cost = __fmaf_rn(d[i], v[i], cost);
+    return cost;
+}
+
+// --------------------------------------------- Hessian-weighted exponent
+// One CTA = one 32-column block k and kThreads rows; H'_k staged in shared
+// memory and read as broadcasts.  Candidates in the order 0, +1, -1 around
+// the OCP exponent; the winner has the strictly smallest d^T H'_k d with
+// d = u - deq, each product sum accumulated with fma in index order.
+template <typename T>
+__global__ void __launch_bounds__(kThreads)
+mx_quant_hessian_kernel(const T* __restrict__ x, int64_t rows, int64_t kb,
+                        const float* __restrict__ t, int had, const float* __restrict__ hess,
+                        uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
+                        float* __restrict__ deq, float* __restrict__ mse)
+{
+    __shared__ __align__(16) float Hs[32 * 32];   // H'_k transposed
+    __shared__ float Ds[32 * kThreads];          // per-thread error staging
+    const int64_t k = blockIdx.y;
+    for (int i = threadIdx.x; i < 32 * 32; i += blockDim.x)
+        Hs[(i & 31) * 32 + (i >> 5)] = __ldg(hess + k * 1024 + i);
+    __syncthreads();
+    const int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (r >= rows)
+        return;
+    const int64_t b = r * kb + k;
+    float u[32];
+    load32<T>(x + b * 32, u);
+    online_transform(u, t ? t + k * 32 : nullptr, had != 0);
+    float a = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+        a = fmaxf(a, fabsf(u[i]));
+    const int e0 = mx_exponent(a);
+    int best_e = e0;
+    float best = hess_cost(u, e0, Hs, Ds + threadIdx.x);
+#pragma unroll 1
+    for (int o = 1; o < 3; ++o) {
+        const int ec = o == 1 ? e0 + 1 : e0 - 1;
+        if (ec < -127 || ec > 127)
+            continue;
+        const float cost = hess_cost(u, ec, Hs, Ds + threadIdx.x);
+        if (cost < best) {
+            best = cost;
+            best_e = ec;
+        }
+    }
+    uint32_t cw[4];
+    float dq[32];
+    const float sse = mx_eval(u, best_e, cw, dq);
+    *reinterpret_cast<uint4*>(codes + b * 16) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+    scales[b] = (uint8_t)(best_e + 127);
+    if (deq)
+        store_f32<32>(deq + b * 32, dq);
+    if (mse)
+        mse[b] = __fmul_rn(sse, 1.0f / 32.0f);
+}
+
+// ------------------------------------------------------- Hessian blocks
+// Partial H'_k over a chunk of kTok tokens: the chunk's transformed rows are
+// staged in shared memory, then each thread accumulates 4 of the 1024
+// entries over the chunk.  Partials go to ws[chunk][k][32][32] and are summed
+// in chunk order by hessian_reduce_kernel.
+constexpr int kTok = 256;
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads)
+hessian_partial_kernel(const T* __restrict__ x, int64_t rows, int64_t cols,
+                       const float* __restrict__ t, int had, float* __restrict__ part)
+{
+    __shared__ __align__(16) float Xs[kTok][33];
+    const int64_t k = blockIdx.y;
+    const int64_t chunk = blockIdx.x;
+    const int64_t r0 = chunk * kTok;
+    // stage: one thread per token row of this chunk
+    for (int rr = threadIdx.x; rr < kTok; rr += blockDim.x) {
+        const int64_t r = r0 + rr;
+        float u[32];
+        if (r < rows) {
+            load32<T>(x + r * cols + k * 32, u);
+            online_transform(u, t ? t + k * 32 : nullptr, had != 0);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                u[i] = 0.0f;
+        }
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            Xs[rr][i] = u[i];
+    }
+    __syncthreads();
+    // thread -> entries (i, j0..j0+3): i = tid / 8, j0 = 4 * (tid % 8)
+    const int i = threadIdx.x >> 3;
+    const int j0 = (threadIdx.x & 7) * 4;
+    float acc0 = 0.0f, acc1 = 0.0f, acc2 = 0.0f, acc3 = 0.0f;
+    const int nr = (int)((rows - r0) < kTok ? (rows - r0) : kTok);
+    for (int rr = 0; rr < nr; ++rr) {
+        const float xi = Xs[rr][i];
+        acc0 = __fmaf_rn(xi, Xs[rr][j0], acc0);
+        acc1 = __fmaf_rn(xi, Xs[rr][j0 + 1], acc1);
+        acc2 = __fmaf_rn(xi, Xs[rr][j0 + 2], acc2);
+        acc3 = __fmaf_rn(xi, Xs[rr][j0 + 3], acc3);
+    }
+    float* o = part + (chunk * (cols / 32) + k) * 1024 + i * 32 + j0;
+    *reinterpret_cast<float4*>(o) = make_float4(acc0, acc1, acc2, acc3);
+}
+
+__global__ void __launch_bounds__(kThreads)
+hessian_reduce_kernel(const float* __restrict__ part, int64_t nchunk, int64_t total,
+                      float* __restrict__ hess)
+{
+    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= total)
+        return;
+    float s = 0.0f;
+    for (int64_t c = 0; c < nchunk; ++c)
+        s = __fadd_rn(s, __ldg(part + c * total + idx));
+    hess[idx] = s;
+}
+
+// ------------------------------------------------------- channel scale
+// Column statistics in fp64 over a chunk of rows: sum and sum of squares.
+// One thread owns 8 consecutive columns (one 16-byte bf16 vector or two fp32
+// vectors) for every row of the chunk.
+constexpr int kStatRows = 128;
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads)
+column_stats_kernel(const T* __restrict__ x, int64_t rows, int64_t cols, double* __restrict__ sum,
+                    double* __restrict__ sumsq)
+{
+    const int64_t c0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 8;
+    if (c0 >= cols)
+        return;
+    const int64_t r0 = (int64_t)blockIdx.y * kStatRows;
+    const int64_t r1 = (r0 + kStatRows) < rows ? (r0 + kStatRows) : rows;
+    double s[8], q[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        s[i] = 0.0;
+        q[i] = 0.0;
+    }
+    for (int64_t r = r0; r < r1; ++r) {
+        float v[8];
+        load_elems<T, 8>(x + r * cols + c0, v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const double d = (double)v[i];
+            s[i] += d;
+            q[i] = fma(d, d, q[i]);
+        }
+    }
+    const int64_t o = (int64_t)blockIdx.y * cols + c0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        if (sum)
+            sum[o + i] = s[i];
+        sumsq[o + i] = q[i];
+    }
+}
+
+// t_j = (sigma_j^W / rms_j^X)^alpha, t = 1 where a factor is zero; fp64, then
+// rounded to fp32; t_inv = 1/t in fp32.
+__global__ void __launch_bounds__(kThreads)
+channel_scale_kernel(const double* __restrict__ wsum, const double* __restrict__ wsq,
+                     int64_t wchunks, int64_t n_out, const double* __restrict__ xsq,
+                     int64_t xchunks, int64_t tokens, int64_t cols, double alpha,
+                     float* __restrict__ t, float* __restrict__ t_inv)
+{
+    const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (j >= cols)
+        return;
+    double s = 0.0, q = 0.0, h = 0.0;
+    for (int64_t c = 0; c < wchunks; ++c) {
+        s += wsum[c * cols + j];
+        q += wsq[c * cols + j];
+    }
+    for (int64_t c = 0; c < xchunks; ++c)
+        h += xsq[c * cols + j];
+    const double n = (double)n_out;
+    const double mean = s / n;
+    double var = q / n - mean * mean;
+    var = var > 0.0 ? var : 0.0;
+    const double sigma = sqrt(var);
+    const double rms = sqrt(h / (double)tokens);
+    double tj = 1.0;
+    if (sigma > 0.0 && rms > 0.0)
+        tj = pow(sigma / rms, alpha);
+    const float t32 = (float)tj;
+    t[j] = t32;
+    if (t_inv)
+        t_inv[j] = __frcp_rn(t32);
+}
+
+int grid_for(int64_t work, const void* kernel)
+{
+    int per_sm = 0;
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, 0);
+    if (per_sm < 1)
+        per_sm = 1;
+    int64_t want = (work + kThreads - 1) / kThreads;
+    const int64_t cap = (int64_t)num_sms() * per_sm;
+    want = want > cap ? cap : want;
+    return (int)(want < 1 ? 1 : want);
+}
+
+}  // namespace
+
+size_t hessian_ws_bytes(int64_t rows, int64_t cols)
+{
+    const int64_t nchunk = (rows + kTok - 1) / kTok;
+    return (size_t)nchunk * (size_t)(cols / 32) * 1024 * sizeof(float);
+}
+
+size_t channel_scale_ws_bytes(int64_t tokens, int64_t n_out, int64_t cols)
+{
+    const int64_t wch = (n_out + kStatRows - 1) / kStatRows;
+    const int64_t xch = (tokens + kStatRows - 1) / kStatRows;
+    return (size_t)(2 * wch + xch) * (size_t)cols * sizeof(double);
+}
+
+cudaError_t launch_mxfp4_quant(const void* x, int dtype, int64_t rows, int64_t cols,
+                               const float* chan_scale, int hadamard, int rule, const float* hess,
+                               uint8_t* codes, uint8_t* scales, float* deq, float* mse,
+                               cudaStream_t s)
+{
+    const int64_t kb = cols / 32;
+    const int64_t nblk = rows * kb;
+    if (rule == 4) {
+        dim3 grid((unsigned)((rows + kThreads - 1) / kThreads), (unsigned)kb);
+        if (dtype == 1)
+            mx_quant_hessian_kernel<__nv_bfloat16><<<grid, kThreads, 0, s>>>(
+                reinterpret_cast<const __nv_bfloat16*>(x), rows, kb, chan_scale, hadamard, hess,
+                codes, scales, deq, mse);
+        else
+            mx_quant_hessian_kernel<float><<<grid, kThreads, 0, s>>>(
+                reinterpret_cast<const float*>(x), rows, kb, chan_scale, hadamard, hess, codes,
+                scales, deq, mse);
+        return cudaGetLastError();
+    }
+    if (dtype == 1) {
+        auto k = mx_quant_absmax_kernel<__nv_bfloat16>;
+        k<<<grid_for(nblk, (const void*)k), kThreads, 0, s>>>(
+            reinterpret_cast<const __nv_bfloat16*>(x), nblk, kb, chan_scale, hadamard, codes,
+            scales, deq, mse);
+    } else {
+        auto k = mx_quant_absmax_kernel<float>;
+        k<<<grid_for(nblk, (const void*)k), kThreads, 0, s>>>(reinterpret_cast<const float*>(x),
+                                                               nblk, kb, chan_scale, hadamard,
+                                                               codes, scales, deq, mse);
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_hessian_blocks(const void* x, int dtype, int64_t rows, int64_t cols,
+                                  const float* chan_scale, int hadamard, float* hess, void* ws,
+                                  cudaStream_t s)
+{
+    const int64_t kb = cols / 32;
+    const int64_t nchunk = (rows + kTok - 1) / kTok;
+    float* part = reinterpret_cast<float*>(ws);
+    dim3 grid((unsigned)nchunk, (unsigned)kb);
+    if (dtype == 1)
+        hessian_partial_kernel<__nv_bfloat16><<<grid, kThreads, 0, s>>>(
+            reinterpret_cast<const __nv_bfloat16*>(x), rows, cols, chan_scale, hadamard, part);
+    else
+        hessian_partial_kernel<float><<<grid, kThreads, 0, s>>>(
+            reinterpret_cast<const float*>(x), rows, cols, chan_scale, hadamard, part);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return e;
+    const int64_t total = kb * 1024;
+    hessian_reduce_kernel<<<(unsigned)((total + kThreads - 1) / kThreads), kThreads, 0, s>>>(
+        part, nchunk, total, hess);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_mx_channel_scale(const void* x, int xdt, int64_t tokens, const void* w, int wdt,
+                                    int64_t n_out, int64_t cols, float alpha, float* t,
+                                    float* t_inv, void* ws, cudaStream_t s)
+{
+    const int64_t wch = (n_out + kStatRows - 1) / kStatRows;
+    const int64_t xch = (tokens + kStatRows - 1) / kStatRows;
+    double* wsum = reinterpret_cast<double*>(ws);
+    double* wsq = wsum + wch * cols;
+    double* xsq = wsq + wch * cols;
+    const unsigned gx = (unsigned)((cols / 8 + kThreads - 1) / kThreads);
+    if (wdt == 1)
+        column_stats_kernel<__nv_bfloat16><<<dim3(gx, (unsigned)wch), kThreads, 0, s>>>(
+            reinterpret_cast<const __nv_bfloat16*>(w), n_out, cols, wsum, wsq);
+    else
+        column_stats_kernel<float><<<dim3(gx, (unsigned)wch), kThreads, 0, s>>>(
+            reinterpret_cast<const float*>(w), n_out, cols, wsum, wsq);
+    if (xdt == 1)
+        column_stats_kernel<__nv_bfloat16><<<dim3(gx, (unsigned)xch), kThreads, 0, s>>>(
+            reinterpret_cast<const __nv_bfloat16*>(x), tokens, cols, nullptr, xsq);
+    else
+        column_stats_kernel<float><<<dim3(gx, (unsigned)xch), kThreads, 0, s>>>(
+            reinterpret_cast<const float*>(x), tokens, cols, nullptr, xsq);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess)
+        return e;
+    channel_scale_kernel<<<(unsigned)((cols + kThreads - 1) / kThreads), kThreads, 0, s>>>(
+        wsum, wsq, wch, n_out, xsq, xch, tokens, cols, (double)alpha, t, t_inv);
+    return cudaGetLastError();
+}
+
+}  // namespace fp4q

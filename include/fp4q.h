@@ -1,0 +1,235 @@
+/*
+ * fp4q.h -- C ABI of the block-scaled 4-bit quantization library for NVIDIA
+ * B200 (sm_100a).  Plain pointers and sizes only.
+ *
+ * Sources (web pages; cited by title and section):
+ *   [NVFP4] "Why Gated DeltaNet Survives 4-Bit Quantization: NVFP4 W4A4 for the
+ *           Recurrent Half of a Hybrid 27B LLM" review, section 1 (NVFP4: E2M1
+ *           values with one E4M3 scale per 16 elements; W4A4) and section 3
+ *           (one global scale shared across fused GEMMs).
+ *   [RaZeR] "RaZeR: Redundant Zero Remapping" technical summary, section 1
+ *           (E2M1 value set; the always-positive E4M3 scale wastes its sign
+ *           bit), section 2.1 (E3M3 weight scale frees 2 bits, E4M3
+ *           activation scale frees 1), section 2.2 (the -0 code is remapped to
+ *           a per-block special value picked for least squared error).
+ *   [MACaQ] "MACaQ: Fast, Model Agnostic Calibrated Quantization for
+ *           Low-Precision Weights and Activations" review, section 1 (MXFP4 =
+ *           E2M1 + E8M0 per 32 elements; online per-channel scale and size-32
+ *           block-Hadamard; Hessian-weighted exponent among {+1, 0, -1}) and
+ *           section 3 (t_j ~ (sigma_j^W / rms_j^X)^0.75, H = X^T X).
+ *   [Finer] "Finer is Better (with the Right Scaling)" summary, Methodology
+ *           1-2 (block sizes 4..32; abs-max, prevent-zero, 4-over-6, brute
+ *           force and hierarchical scaling).
+ *
+ * Conventions for every entry point:
+ *  - Tensors are row-major.  Blocks are contiguous runs along the last
+ *    dimension; cols must be a multiple of the block size.
+ *  - Packed codes: byte i holds element 2i in bits 3:0 and element 2i+1 in
+ *    bits 7:4; an E2M1 code is sign<<3 | magnitude index (0, .5, 1, 1.5, 2, 3,
+ *    4, 6).  rows * cols / 2 bytes.
+ *  - Scale bytes, one per block, row-major [rows][cols/block] unless an MMA
+ *    layout is requested.
+ *  - "device" pointers are CUDA device memory owned by the caller; the library
+ *    allocates and frees nothing and keeps no state between calls.  "host"
+ *    pointers are read during the call only.
+ *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream) and is asynchronous: outputs are valid once the stream reaches
+ *    the call.  Argument errors are found on the host before anything is
+ *    launched and leave all outputs untouched.
+ *  - Pointers to vectors of 4-byte or wider elements and code buffers must
+ *    be 16-byte aligned (FP4Q_ERR_ALIGN otherwise).
+ *  - Inputs must be finite; scales/global scales passed in must be positive
+ *    and finite.  Results for other inputs are unspecified.
+ *  - Every fp32 decision (scale choice, special value, exponent) is computed
+ *    with IEEE round-to-nearest operations in a fixed order and is
+ *    reproducible bit for bit.
+ */
+#ifndef FP4Q_H
+#define FP4Q_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define FP4Q_API __attribute__((visibility("default")))
+#else
+#define FP4Q_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FP4Q_OK = 0,
+    FP4Q_ERR_ARG = 1,          /* a size, enum or pointer argument is invalid */
+    FP4Q_ERR_ALIGN = 2,        /* a pointer is not aligned as required */
+    FP4Q_ERR_UNSUPPORTED = 3,  /* valid request this build does not implement */
+    FP4Q_ERR_CUDA = 4,         /* a CUDA launch or runtime call failed */
+    FP4Q_ERR_TIMEOUT = 5,      /* a device-side bounded wait gave up */
+    FP4Q_ERR_WORKSPACE = 6     /* the workspace is missing or too small */
+} fp4q_status;
+
+typedef enum { FP4Q_F32 = 0, FP4Q_BF16 = 1 } fp4q_dtype;
+
+/* Block-scale formats: E4M3 = OCP FP8 E4M3FN (NVFP4 and RaZeR activations),
+ * E3M3 = 6-bit unsigned, bias 3, 2^-5..30 (RaZeR weights, [RaZeR] 2.1),
+ * E8M0 = 2^(byte-127) (MXFP4, [MACaQ] 1). */
+typedef enum { FP4Q_SF_E4M3 = 0, FP4Q_SF_E3M3 = 1, FP4Q_SF_E8M0 = 2 } fp4q_scale_fmt;
+
+/* Block-scale selection rules ([Finer] Methodology 2; [MACaQ] 1):
+ *  ABSMAX        scale = E4M3(amax_b / (6 g)), ties to even, saturating at 448
+ *  PREVENT_ZERO  ABSMAX, but a zero scale becomes the smallest positive E4M3 (2^-9)
+ *  FOUR_OVER_SIX the 6-mapping scale or the 4-mapping scale E4M3(amax_b / (4 g)),
+ *                whichever gives the strictly smaller block squared error
+ *  BRUTE_FORCE   every finite positive E4M3 scale; least squared error, ties to
+ *                the smallest scale
+ *  HESSIAN_EXP   MXFP4 only: OCP exponent plus offset 0, +1 or -1 (tried in that
+ *                order), least H'-weighted error d^T H'_k d, ties to the earlier */
+typedef enum {
+    FP4Q_ABSMAX = 0,
+    FP4Q_PREVENT_ZERO = 1,
+    FP4Q_FOUR_OVER_SIX = 2,
+    FP4Q_BRUTE_FORCE = 3,
+    FP4Q_HESSIAN_EXP = 4
+} fp4q_rule;
+
+/* Per-tensor FP32 global scale g of hierarchical scaling ([Finer] Methodology 2):
+ *  NONE   g = 1
+ *  AMAX   g = amax(x) / (6 * S_max), S_max = 448 (E4M3) or 30 (E3M3); g = 1 for
+ *         an all-zero tensor.  Computed on the device by a pre-pass; needs a
+ *         workspace; the g used is written to *global_scale if non-NULL.
+ *  GIVEN  g read from *global_scale (device) -- e.g. one g shared by fused
+ *         projections, the global-scale mismatch fix of [NVFP4] 3. */
+typedef enum { FP4Q_GS_NONE = 0, FP4Q_GS_AMAX = 1, FP4Q_GS_GIVEN = 2 } fp4q_gs_mode;
+
+/* Scale-byte layouts: ROWMAJOR [rows][cols/block]; MMA = the tcgen05 block-scaled
+ * MMA scale-factor layout (128-row x 4-scale atoms of 512 bytes, atoms ordered
+ * with the scale column fastest, row r of an atom at 16*(r%32) + 4*((r/32)%4),
+ * scale column c at c%4).  MMA needs block 16, rows % 128 == 0 and
+ * (cols/16) % 4 == 0. */
+typedef enum { FP4Q_SFLAYOUT_ROWMAJOR = 0, FP4Q_SFLAYOUT_MMA = 1 } fp4q_sf_layout;
+
+/* Workspace queries for fp4q_workspace_size(). */
+typedef enum {
+    FP4Q_OP_QUANTIZE = 0,       /* nvfp4_quantize / razer_quantize with GS_AMAX */
+    FP4Q_OP_HESSIAN = 1,        /* fp4_hessian_blocks (rows, cols) */
+    FP4Q_OP_CHANNEL_SCALE = 2,  /* mxfp4_channel_scale (tokens=rows, cols, n_out=n) */
+    FP4Q_OP_GEMM = 3            /* w4a4_gemm with bf16 A (M=rows, K=cols, N=n) */
+} fp4q_op;
+
+/* Bytes of device workspace an entry point needs (0 if none). */
+FP4Q_API size_t fp4q_workspace_size(int op, int64_t rows, int64_t cols, int64_t n);
+
+/* Human-readable name of a status code (static storage). */
+FP4Q_API const char* fp4q_status_str(int status);
+
+/* Library version, e.g. "fp4q 0.1.0 sm_100a". */
+FP4Q_API const char* fp4q_version(void);
+
+/*
+ * NVFP4 quantization with a choice of block size and scale rule.
+ * [NVFP4] 1 (format), [Finer] Methodology 1-2 (block sizes, rules, hierarchical).
+ *
+ *  x            device, rows x cols, dtype FP4Q_F32 or FP4Q_BF16, 16-byte aligned
+ *  block        4, 8, 16 or 32 (cols % block == 0)
+ *  rule         ABSMAX, PREVENT_ZERO, FOUR_OVER_SIX or BRUTE_FORCE
+ *  gs_mode      NONE / AMAX / GIVEN; global_scale: device float, out for AMAX
+ *               (nullable), in for GIVEN (required), ignored for NONE
+ *  codes        device, rows*cols/2 bytes (out), 16-byte aligned
+ *  scales       device, rows*cols/block E4M3 bytes (out), layout per sf_layout
+ *  dequant      device fp32 rows x cols (out, nullable): v * (sc * g)
+ *  block_mse    device fp32 rows x cols/block (out, nullable): sum((x-deq)^2)/block
+ *  workspace    device, >= fp4q_workspace_size(FP4Q_OP_QUANTIZE, ...) bytes when
+ *               gs_mode == AMAX (else may be NULL), 16-byte aligned
+ * Errors: ERR_ARG (bad enum/size/null), ERR_ALIGN, ERR_WORKSPACE, ERR_CUDA.
+ */
+FP4Q_API int nvfp4_quantize(const void* x, int dtype, int64_t rows, int64_t cols, int block, int rule,
+                   int gs_mode, float* global_scale, uint8_t* codes, uint8_t* scales,
+                   int sf_layout, float* dequant, float* block_mse, void* workspace,
+                   size_t workspace_bytes, void* stream);
+
+/*
+ * RaZeR quantization, blocks of 16 ([RaZeR] 2.1-2.2).  The block scale is the
+ * abs-max scale in `scale_fmt`; for each special value the block is quantized
+ * with the -0 code standing for that value (an element takes it when the
+ * value, of the same sign, is strictly nearer than its E2M1 neighbour;
+ * elements that round to zero take +0); the least squared error wins, ties to
+ * the earlier table entry.
+ *
+ *  scale_fmt    FP4Q_SF_E3M3 (weights: meta = sel<<6 | e3m3, up to 4 specials)
+ *               or FP4Q_SF_E4M3 (activations: meta = sel<<7 | e4m3, up to 2)
+ *  specials     host, n_special values, each a non-zero multiple of 0.5 with
+ *               magnitude <= 32
+ *  meta         device, rows*cols/16 bytes (out)
+ *  other arguments as nvfp4_quantize (g = amax / (6 * S_max) for AMAX).
+ */
+FP4Q_API int razer_quantize(const void* x, int dtype, int64_t rows, int64_t cols, int scale_fmt,
+                   const float* specials, int n_special, int gs_mode, float* global_scale,
+                   uint8_t* codes, uint8_t* meta, float* dequant, float* block_mse,
+                   void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * MXFP4 quantization with the online transform of [MACaQ] 1: u = x * t (per
+ * column, if chan_scale != NULL), then for each 32-column block the
+ * normalised Sylvester Hadamard rotation (if hadamard32), then E2M1 codes
+ * with an E8M0 shared exponent.  rule ABSMAX: OCP exponent
+ * floor(log2 amax_b) - 2; rule HESSIAN_EXP: that exponent plus 0, +1 or -1,
+ * least d^T H'_k d.
+ *
+ *  chan_scale   device fp32 [cols] (nullable), 16-byte aligned
+ *  hess_blocks  device fp32 [cols/32][32][32] (HESSIAN_EXP only)
+ *  codes        device rows*cols/2 (out); scales: device rows*cols/32 E8M0 bytes
+ *  dequant / block_mse  nullable; both refer to the transformed values u'
+ * Errors: ERR_ARG (cols % 32, rule, missing hess), ERR_ALIGN, ERR_CUDA.
+ */
+FP4Q_API int mxfp4_quantize(const void* x, int dtype, int64_t rows, int64_t cols,
+                   const float* chan_scale, int hadamard32, int rule, const float* hess_blocks,
+                   uint8_t* codes, uint8_t* scales, float* dequant, float* block_mse,
+                   void* stream);
+
+/*
+ * Diagonal 32x32 blocks of the Hessian of the transformed activations,
+ * H'_k = X'_k^T X'_k with X' = transform(x) as in mxfp4_quantize ([MACaQ] 1,
+ * H = X^T X).  fp32 accumulation (tolerance, not bit-exact).
+ *  hess_blocks  device fp32 [cols/32][32][32] (out)
+ *  workspace    >= fp4q_workspace_size(FP4Q_OP_HESSIAN, rows, cols, 0)
+ */
+FP4Q_API int fp4_hessian_blocks(const void* x, int dtype, int64_t rows, int64_t cols,
+                       const float* chan_scale, int hadamard32, float* hess_blocks,
+                       void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Online per-channel scale of [MACaQ] 3: t_j = (sigma_j^W / rms_j^X)^alpha,
+ * sigma_j^W the population std of weight column j over n_out rows, rms_j^X =
+ * sqrt(sum_t x_tj^2 / tokens) (the Hessian diagonal); t_j = 1 where either is
+ * zero.  fp64 statistics, t rounded to fp32, t_inv = 1/t in fp32.
+ *  x  device [tokens][cols]; w  device [n_out][cols]; cols % 8 == 0
+ *  t, t_inv  device fp32 [cols] (out; t_inv nullable)
+ *  workspace >= fp4q_workspace_size(FP4Q_OP_CHANNEL_SCALE, tokens, cols, n_out)
+ */
+FP4Q_API int mxfp4_channel_scale(const void* x, int x_dtype, int64_t tokens, const void* w,
+                        int w_dtype, int64_t n_out, int64_t cols, float alpha, float* t,
+                        float* t_inv, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Dequantization with per-block MSE (the selection criterion of [RaZeR] 2.2
+ * and [Finer] Methodology 2, as a standalone pass).
+ *  codes, scales  as produced by the quantizers (row-major scale bytes)
+ *  block          4/8/16/32 (E8M0: 32; RaZeR: 16)
+ *  scale_fmt      E4M3 / E3M3: deq = v * (sc * g); E8M0: deq = v * 2^(byte-127)
+ *  specials       host, nullable: RaZeR tables (selector in the scale byte's top bits)
+ *  global_scale   device float g, nullable (= 1); ignored for E8M0
+ *  ref            device reference tensor (ref_dtype), nullable; needed for block_mse
+ *  dequant        device fp32 (out, nullable); block_mse device fp32 (out, nullable)
+ */
+FP4Q_API int fp4_dequant_mse(const uint8_t* codes, const uint8_t* scales, int64_t rows, int64_t cols,
+                    int block, int scale_fmt, const float* specials, int n_special,
+                    const float* global_scale, const void* ref, int ref_dtype, float* dequant,
+                    float* block_mse, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP4Q_H */

@@ -1,0 +1,88 @@
+"""The C-ABI library builds for sm_100a, loads, and exports every symbol the
+public headers declare; host-side argument checks reject bad calls before any
+CUDA work (so these run without a GPU)."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    names = []
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        src = open(h).read()
+        names += re.findall(r"FP4Q_API\s+[\w\s\*]+?\b(\w+)\s*\(", src)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from block_scaled_fp4_03_b200 import binding
+    return binding.lib()
+
+
+def test_every_declared_symbol_is_exported(L):
+    from block_scaled_fp4_03_b200 import binding
+    names = declared_symbols()
+    assert len(names) >= 9
+    for n in names:
+        assert hasattr(L, n), n
+        assert n in binding.SIGNATURES, n
+
+
+def test_version_and_status_strings(L):
+    assert b"sm_100a" in L.fp4q_version()
+    assert L.fp4q_status_str(0) == b"ok"
+    assert L.fp4q_status_str(1) == b"invalid argument"
+    assert L.fp4q_status_str(99) == b"unknown status"
+
+
+def test_workspace_sizes(L):
+    assert L.fp4q_workspace_size(0, 4096, 4096, 0) >= 592 * 4
+    h = L.fp4q_workspace_size(1, 8192, 4096, 0)
+    assert h == (8192 // 256) * (4096 // 32) * 1024 * 4
+    assert L.fp4q_workspace_size(1, 8192, 100, 0) == 0
+    assert L.fp4q_workspace_size(2, 8192, 4096, 4096) > 0
+
+
+FAKE = ctypes.c_void_p(0x10000)          # aligned, never dereferenced: calls fail before launch
+MIS = ctypes.c_void_p(0x10004)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(block=5), 1), (dict(block=16, cols=24), 1), (dict(rule=7), 1), (dict(dtype=3), 1),
+    (dict(gs_mode=9), 1), (dict(rows=-1), 1), (dict(sf_layout=1, rows=100), 1),
+    (dict(x=MIS), 2), (dict(codes=MIS), 2), (dict(gs_mode=1, ws=None), 6),
+    (dict(gs_mode=2, gs=None), 1),
+])
+def test_nvfp4_argument_errors(L, kw, expect):
+    a = dict(x=FAKE, dtype=0, rows=128, cols=64, block=16, rule=0, gs_mode=0, gs=FAKE, codes=FAKE,
+             scales=FAKE, sf_layout=0, deq=None, mse=None, ws=FAKE, wsb=4096)
+    a.update(kw)
+    st = L.nvfp4_quantize(a["x"], a["dtype"], a["rows"], a["cols"], a["block"], a["rule"], a["gs_mode"],
+                          a["gs"], a["codes"], a["scales"], a["sf_layout"], a["deq"], a["mse"], a["ws"],
+                          a["wsb"], None)
+    assert st == expect
+
+
+def test_razer_rejects_bad_specials(L):
+    for sp, n, sf in (([5.3], 1, 0), ([0.0], 1, 0), ([5, -5, 3.5], 3, 0), ([5, -5, 3.5, -3.5, 1], 5, 1),
+                      ([100.0], 1, 1)):
+        arr = (ctypes.c_float * len(sp))(*sp)
+        st = L.razer_quantize(FAKE, 0, 16, 32, sf, ctypes.cast(arr, ctypes.c_void_p), n, 0, None,
+                              FAKE, FAKE, None, None, None, 0, None)
+        assert st == 1, sp
+
+
+def test_mx_and_dequant_argument_errors(L):
+    assert L.mxfp4_quantize(FAKE, 0, 4, 48, None, 1, 0, None, FAKE, FAKE, None, None, None) == 1
+    assert L.mxfp4_quantize(FAKE, 0, 4, 64, None, 1, 4, None, FAKE, FAKE, None, None, None) == 1
+    assert L.mxfp4_quantize(FAKE, 0, 4, 64, None, 1, 2, None, FAKE, FAKE, None, None, None) == 1
+    assert L.fp4_dequant_mse(FAKE, FAKE, 4, 64, 16, 2, None, 0, None, None, 0, FAKE, None, None) == 1
+    assert L.fp4_dequant_mse(FAKE, FAKE, 4, 64, 16, 0, None, 0, None, None, 0, FAKE, FAKE, None) == 1
+    assert L.fp4_hessian_blocks(FAKE, 0, 64, 64, None, 1, FAKE, None, 0, None) == 6
+    assert L.mxfp4_channel_scale(FAKE, 0, 64, FAKE, 0, 64, 12, 0.75, FAKE, None, FAKE, 1 << 20, None) == 1
