@@ -1,0 +1,479 @@
+"""Benchmark of the block-scaled FP4 hot path on B200.
+
+One step = one pass over every hot-path row at its workload size:
+  c1  NVFP4 prevent-zero quantize, 4096x4096 fp32 N(0,1), block 16,
+      hierarchical scale, with dequant + per-block MSE        (amax, quantize)
+  c2  block sizes {4,8,16,32} x rules {abs-max, prevent-zero, 4-over-6,
+      brute force} on 8192x8192 fp32 Student-t(3)*1e-3, g = 1, codes +
+      scales + per-block MSE                                  (16 quantizations)
+  c3  RaZeR: 8192x8192 bf16 weights (E3M3 + 4 specials) and 16384x4096 bf16
+      activations (E4M3 + 2 specials), hierarchical scale
+  c4  MXFP4 prep: channel scale t from 8192x4096 bf16 activations and
+      4096x4096 bf16 weights, Hessian blocks H', activation quantize (t,
+      Hadamard-32, E8M0), weight quantize with the Hessian-weighted exponent
+  c5  dynamic 4-over-6 NVFP4 activation quantize of 8192x4096 bf16 into the
+      MMA scale layout
+Inputs are synthetic and seeded (block_scaled_fp4_03_b200.inputs), resident in
+HBM when timing starts; L2 is flushed (a 512 MiB write) before every step.
+
+The JSON line's value is elements quantized per second over the whole step
+(Gelem/s, all ranks); per-row times, bandwidths and roofline fractions are in
+"rows".  `--impl reference` times the plain CPU oracle on a bounded sample of
+the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "FP4 quantize Gelem/s & % of HBM roofline; W4A4 GEMM TFLOP/s & % FP4 peak"
+WORKLOAD = "hot path: one pass of every row (NVFP4 4096^2 PZ; 8192^2 block-size x rule sweep; RaZeR W 8192^2 + A 16384x4096; MXFP4 prep 8192x4096 + 4096^2; 4-over-6 act quant 8192x4096)"
+SM_COUNT = 148
+FP32_LANES_PER_SM = 128
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d.get("sm_max_mhz", 1965.0)), "measured"
+    except Exception:
+        return 6650.0, 1965.0, "fallback"
+
+
+# ----------------------------------------------------------------------------- rows
+class Row:
+    """One hot-path row: how to launch it on device buffers and what it moves."""
+
+    def __init__(self, name, kernel, units, bytes_, launches, fn, out, bound="hbm", flops=0.0, evals=0.0):
+        self.name, self.kernel, self.units, self.bytes, self.launches = name, kernel, units, bytes_, launches
+        self.fn, self.out, self.bound, self.flops, self.evals = fn, out, bound, flops, evals
+
+
+def build_rows(torch, fq, inputs, dev, host_copies=None):
+    """Create the step's device buffers and rows.  host_copies (dict) receives
+    the host arrays that an end-to-end run copies in each step."""
+    def to_dev(a, key):
+        if host_copies is not None:
+            host_copies[key] = a
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+        return torch.from_numpy(a).to(dev)
+
+    rows = []
+    X = {}
+    # c1
+    a1 = inputs.generate("gaussian")
+    X["c1"] = to_dev(a1, "c1")
+    n1 = a1.size
+    o1 = {}
+    ws1 = torch.empty(fq.workspace_size(fq.OP_QUANTIZE, *a1.shape), dtype=torch.uint8, device=dev)
+
+    def c1():
+        o1.update(fq.nvfp4_quantize(X["c1"], 16, fq.PREVENT_ZERO, gs_mode=fq.GS_AMAX, dequant=True,
+                                    mse=True, out=o1, workspace=ws1))
+    rows.append(Row("c1_nvfp4_pz_deq_mse", "nvfp4_quant_kernel<16, float, 1>", n1, n1 * (4 + 0.5 + 1 / 16 + 4 + 4 / 16), 2, c1, o1))
+    # c2
+    a2 = inputs.generate("student_t")
+    X["c2"] = to_dev(a2, "c2")
+    n2 = a2.size
+    names = {fq.ABSMAX: "absmax", fq.PREVENT_ZERO: "pz", fq.FOUR_OVER_SIX: "4o6", fq.BRUTE_FORCE: "bf"}
+    for B in (4, 8, 16, 32):
+        for rule in (fq.ABSMAX, fq.PREVENT_ZERO, fq.FOUR_OVER_SIX, fq.BRUTE_FORCE):
+            o = {}
+
+            def c2(B=B, rule=rule, o=o):
+                o.update(fq.nvfp4_quantize(X["c2"], B, rule, gs_mode=fq.GS_NONE, mse=True, out=o))
+            rows.append(Row("c2_B%d_%s" % (B, names[rule]), "nvfp4_quant_kernel<%d, float, %d>" % (B, rule),
+                            n2, n2 * (4 + 0.5 + 1 / B + 4 / B), 1, c2, o,
+                            bound="alu" if rule == fq.BRUTE_FORCE else "hbm",
+                            evals=n2 * 126.0 if rule == fq.BRUTE_FORCE else 0.0))
+    # c3
+    w3 = inputs.generate("razer_weight")
+    X["c3w"] = to_dev(w3, "c3w")
+    a3 = inputs.generate("razer_act")
+    X["c3a"] = to_dev(a3, "c3a")
+    ws3 = torch.empty(fq.workspace_size(fq.OP_QUANTIZE, 1, 1), dtype=torch.uint8, device=dev)
+    o3w, o3a = {}, {}
+
+    def c3w():
+        o3w.update(fq.razer_quantize(X["c3w"], fq.SF_E3M3, [5.0, -5.0, 3.5, -3.5], gs_mode=fq.GS_AMAX, out=o3w, workspace=ws3))
+
+    def c3a():
+        o3a.update(fq.razer_quantize(X["c3a"], fq.SF_E4M3, [5.0, -5.0], gs_mode=fq.GS_AMAX, out=o3a, workspace=ws3))
+    rows.append(Row("c3_razer_weight", "razer_quant_kernel<__nv_bfloat16, 1>", w3.size, w3.size * (2 + 0.5 + 1 / 16), 2, c3w, o3w))
+    rows.append(Row("c3_razer_act", "razer_quant_kernel<__nv_bfloat16, 0>", a3.size, a3.size * (2 + 0.5 + 1 / 16), 2, c3a, o3a))
+    # c4
+    x4 = inputs.generate("mx_act")
+    w4 = inputs.generate("mx_weight")
+    X["c4x"] = to_dev(x4, "c4x")
+    X["c4w"] = to_dev(w4, "c4w")
+    T, C = x4.shape
+    N4 = w4.shape[0]
+    t4 = torch.empty(C, dtype=torch.float32, device=dev)
+    ti4 = torch.empty(C, dtype=torch.float32, device=dev)
+    h4 = torch.empty((C // 32, 32, 32), dtype=torch.float32, device=dev)
+    wsc = torch.empty(fq.workspace_size(fq.OP_CHANNEL_SCALE, T, C, N4), dtype=torch.uint8, device=dev)
+    wsh = torch.empty(fq.workspace_size(fq.OP_HESSIAN, T, C), dtype=torch.uint8, device=dev)
+    o4a, o4w = {}, {}
+
+    def c4s():
+        fq.channel_scale(X["c4x"], X["c4w"], 0.75, out=(t4, ti4), workspace=wsc)
+
+    def c4h():
+        fq.hessian_blocks(X["c4x"], t4, True, out=h4, workspace=wsh)
+
+    def c4a():
+        o4a.update(fq.mxfp4_quantize(X["c4x"], t4, True, fq.ABSMAX, out=o4a))
+
+    def c4w():
+        o4w.update(fq.mxfp4_quantize(X["c4w"], ti4, True, fq.HESSIAN_EXP, hess=h4, out=o4w))
+    rows.append(Row("c4_channel_scale", "column_stats_kernel", 0, x4.size * 2 + w4.size * 2, 3, c4s, {"t": t4, "t_inv": ti4}))
+    rows.append(Row("c4_hessian_blocks", "hessian_partial_kernel", 0, x4.size * 2 + C * 32 * 4, 2, c4h,
+                    {"hess": h4}, flops=2.0 * T * C * 32))
+    rows.append(Row("c4_mx_act", "mx_quant_absmax_kernel", x4.size, x4.size * (2 + 0.5 + 1 / 32), 1, c4a, o4a))
+    rows.append(Row("c4_mx_weight_hessian", "mx_quant_hessian_kernel", w4.size, w4.size * (2 + 0.5 + 1 / 32) + C * 32 * 4,
+                    1, c4w, o4w, bound="alu", flops=2.0 * 3 * N4 * (C // 32) * 32 * 32))
+    # c5
+    a5 = inputs.generate("gemm_act")
+    X["c5"] = to_dev(a5, "c5")
+    ws5 = torch.empty(fq.workspace_size(fq.OP_QUANTIZE, 1, 1), dtype=torch.uint8, device=dev)
+    o5 = {}
+
+    def c5():
+        o5.update(fq.nvfp4_quantize(X["c5"], 16, fq.FOUR_OVER_SIX, gs_mode=fq.GS_AMAX, sf_layout=fq.SF_MMA,
+                                    out=o5, workspace=ws5))
+    rows.append(Row("c5_act_quant_4o6_mma", "nvfp4_quant_kernel<16, __nv_bfloat16, 2>", a5.size, a5.size * (2 + 0.5 + 1 / 16), 2, c5, o5))
+    return rows, X
+
+
+# ------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = "index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap"
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        self.t0 = time.perf_counter()
+        try:
+            fd, self.path = tempfile.mkstemp(prefix="fp4q_clocks_", suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.FIELDS,
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            p = [v.strip() for v in line.split(",")]
+            if len(p) < 9:
+                continue
+            try:
+                sm.append(float(p[1]))
+                smax.append(float(p[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, p[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        os.unlink(self.path)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(max(smax)), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------- reference arm
+def oracle_sample_inputs(inputs, frac_rows):
+    """Leading rows of every input (a bounded sample of the step's workload), fp32."""
+    def sub(kind, frac):
+        a = inputs.as_f32(inputs.generate(kind))
+        r = max(1, int(round(a.shape[0] * frac)))
+        return np.ascontiguousarray(a[:r])
+
+    return {"c1": sub("gaussian", frac_rows["c1"]), "c2": sub("student_t", frac_rows["c2"]),
+            "c3w": sub("razer_weight", frac_rows["c3"]), "c3a": sub("razer_act", frac_rows["c3"]),
+            "c4x": sub("mx_act", frac_rows["c4"]), "c4w": sub("mx_weight", frac_rows["c4"]),
+            "c5": sub("gemm_act", frac_rows["c5"])}
+
+
+def oracle_sample_run(O, S):
+    """One step of the CPU oracle over the sampled rows; returns (elements, seconds).
+    Global scales come from the sample itself (the sample is the workload)."""
+    t0 = time.perf_counter()
+    O.nvfp4_quantize(S["c1"], 16, O.RULE_PREVENT_ZERO, g=O.global_scale(O.amax(S["c1"])))
+    for B in (4, 8, 16, 32):
+        for rule in range(4):
+            O.nvfp4_quantize(S["c2"], B, rule, g=1.0, want_deq=False)
+    O.razer_quantize(S["c3w"], O.SF_E3M3, [5.0, -5.0, 3.5, -3.5], g=O.global_scale(O.amax(S["c3w"]), O.SF_E3M3),
+                     want_deq=False)
+    O.razer_quantize(S["c3a"], O.SF_E4M3, [5.0, -5.0], g=O.global_scale(O.amax(S["c3a"]), O.SF_E4M3), want_deq=False)
+    t, ti = O.channel_scale(S["c4x"], S["c4w"], 0.75)
+    hb = O.hessian_blocks(S["c4x"], t, True).astype(np.float32)
+    O.mxfp4_quantize(S["c4x"], t, True, O.RULE_ABSMAX, want_deq=False)
+    O.mxfp4_quantize(S["c4w"], ti, True, O.RULE_HESSIAN_EXP, hb, want_deq=False)
+    O.nvfp4_quantize(S["c5"], 16, O.RULE_FOUR_OVER_SIX, g=O.global_scale(O.amax(S["c5"])), want_deq=False)
+    elems = (S["c1"].size + 16 * S["c2"].size + S["c3w"].size + S["c3a"].size + S["c4x"].size + S["c4w"].size
+             + S["c5"].size)
+    return elems, time.perf_counter() - t0
+
+
+FULL_ELEMS = 4096 * 4096 + 16 * 8192 * 8192 + 8192 * 8192 + 16384 * 4096 + 8192 * 4096 + 4096 * 4096 + 8192 * 4096
+SAMPLE_ROWS = {"c1": 1 / 4, "c2": 1 / 4, "c3": 1 / 4, "c4": 1 / 4, "c5": 1 / 4}
+
+
+def run_reference(args, rank, world):
+    """The reference arm: the plain CPU oracle, bounded sample, on host cores."""
+    if rank != 0:
+        return
+    from block_scaled_fp4_03_b200 import inputs
+    from oracle import oracle as O
+    O.build()
+    cores = O.get_threads()
+    S = oracle_sample_inputs(inputs, SAMPLE_ROWS)
+    for _ in range(args.warmup):
+        oracle_sample_run(O, S)
+    times, elems = [], 0
+    for _ in range(args.steps):
+        elems, dt = oracle_sample_run(O, S)
+        times.append(dt)
+    sec = float(np.mean(times))
+    value = elems / sec / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "Gelem/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "sample": "the first quarter of the rows of every input"},
+        "cpu_baseline": {"value": value, "unit": "Gelem/s", "cores": cores, "kind": "oracle",
+                         "sample": "each step quantizes %d of the %d elements of a full step (row prefixes)" % (elems, FULL_ELEMS)},
+        "e2e": {"value": value, "unit": "Gelem/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ main arm
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import torch
+    import torch.distributed as dist
+    from block_scaled_fp4_03_b200 import binding as fq
+    from block_scaled_fp4_03_b200 import inputs
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    fq.lib(build_if_missing=True)
+    hbm_peak, sm_max_mhz, peak_src = load_peaks()
+
+    host = {}
+    rows, X = build_rows(torch, fq, inputs, dev, host)
+    flush = torch.empty(512 * 2 ** 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(times=None):
+        for r in rows:
+            if times is not None:
+                e0, e1 = torch.cuda.Event(True), torch.cuda.Event(True)
+                e0.record(stream)
+                r.fn()
+                e1.record(stream)
+                times[r.name].append((e0, e1))
+            else:
+                r.fn()
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    clocks = ClockSampler(local)
+    per_row = {r.name: [] for r in rows}
+    step_ev = []
+    barrier()
+    clocks.start()
+    for _ in range(args.steps):
+        flush.zero_()
+        s0, s1 = torch.cuda.Event(True), torch.cuda.Event(True)
+        s0.record(stream)
+        step(per_row)
+        s1.record(stream)
+        step_ev.append((s0, s1))
+    barrier()
+    # nvidia-smi samples every 100 ms; a step takes a few ms, so the sampling
+    # window extends past the K timed steps with untimed repeats of the same
+    # step until it has lasted at least 1.5 s
+    extra = 0
+    while time.perf_counter() - clocks.t0 < 1.5:
+        step()
+        torch.cuda.synchronize()
+        extra += 1
+    clk = clocks.stop()
+    if clk is not None:
+        clk["window"] = "the %d timed steps plus %d untimed repeats of the same step" % (args.steps, extra)
+    step_ms = float(np.mean([a.elapsed_time(b) for a, b in step_ev]))
+    if world > 1:
+        t = torch.tensor([step_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        step_ms = float(t.item())
+    units = sum(r.units for r in rows)
+    value = units * world / (step_ms * 1e-3) / 1e9
+
+    row_out = {}
+    for r in rows:
+        ms = float(np.mean([a.elapsed_time(b) for a, b in per_row[r.name]]))
+        d = {"ms": ms, "GB_s": r.bytes / (ms * 1e-3) / 1e9, "hbm_frac": r.bytes / (ms * 1e-3) / 1e9 / hbm_peak,
+             "launches": r.launches, "bound": r.bound}
+        if r.units:
+            d["Gelem_s"] = r.units / (ms * 1e-3) / 1e9
+        if r.flops:
+            d["TFLOP_s"] = r.flops / (ms * 1e-3) / 1e12
+        row_out[r.name] = d
+    dom = max(rows, key=lambda r: row_out[r.name]["ms"])
+    dms = row_out[dom.name]["ms"]
+    # fp32 pipe: 148 SMs x 128 lanes x clock; one element-candidate evaluation of
+    # a scale search is 6 issue slots (scale multiply, e2m1 encode and decode,
+    # dequant multiply, subtract, fma)
+    eval_peak = SM_COUNT * FP32_LANES_PER_SM * sm_max_mhz * 1e6 / 6.0 / 1e9
+    for r in rows:
+        if r.evals:
+            row_out[r.name]["Geval_s"] = r.evals / (row_out[r.name]["ms"] * 1e-3) / 1e9
+            row_out[r.name]["alu_frac"] = row_out[r.name]["Geval_s"] / eval_peak
+    if dom.bound == "alu" and dom.evals:
+        ach = dom.evals / (dms * 1e-3) / 1e9
+        roof = {"bound": "alu", "achieved": ach, "peak": eval_peak, "unit": "Geval/s", "frac": ach / eval_peak,
+                "traffic": None, "kernel": dom.kernel, "row": dom.name,
+                "note": "brute force: 126 candidate scales x elements per launch; exact shortcuts skip provably "
+                        "losing candidates, so frac can exceed 1"}
+    else:
+        ach = dom.bytes / (dms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": ach, "peak": hbm_peak, "unit": "GB/s", "frac": ach / hbm_peak,
+                "traffic": None, "kernel": dom.kernel, "row": dom.name}
+    roof["peak_source"] = peak_src
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(torch, rows, X, host, stream, args, barrier, world, dist if world > 1 else None, dev)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        from oracle import oracle as O
+        O.build()
+        S = oracle_sample_inputs(inputs, SAMPLE_ROWS)
+        secs = []
+        for _ in range(3):
+            elems, sec = oracle_sample_run(O, S)
+            secs.append(sec)
+        sec = float(np.mean(secs))
+        cpu = {"value": elems / sec / 1e9, "unit": "Gelem/s", "cores": O.get_threads(), "kind": "oracle",
+               "sample": "the first quarter of the rows of every input (%d of the %d elements of a step), "
+                         "3 repeats, %.1f s each" % (elems, FULL_ELEMS, sec)}
+
+    launches = sum(r.launches for r in rows) * args.steps
+    line = {
+        "metric": METRIC, "value": value, "unit": "Gelem/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "elements_per_step_per_gpu": units, "l2": "flushed before every step (512 MiB write)",
+                   "parallelism": "replicas: every rank runs the full step on its own inputs"},
+        "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clk,
+        "rows": row_out,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def run_e2e(torch, rows, X, host, stream, args, barrier, world, dist, dev):
+    """Same step through the public API with host buffers: pinned host -> device
+    copies of every input, the step, and device -> host copies of every output."""
+    pinned = {k: torch.from_numpy(v.view(np.int16) if v.dtype == np.uint16 else v).pin_memory() for k, v in host.items()}
+    h2d = sum(p.numel() * p.element_size() for p in pinned.values())
+
+    outs_dev = []
+    for r in rows:
+        for t in r.out.values():
+            if torch.is_tensor(t) and all(t.data_ptr() != u.data_ptr() for u in outs_dev):
+                outs_dev.append(t)
+    outs_host = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs_dev]
+    d2h = sum(t.numel() * t.element_size() for t in outs_dev)
+
+    def one():
+        for k, p in pinned.items():
+            dst = X[k]
+            dst.view(torch.int16 if dst.dtype == torch.bfloat16 else dst.dtype).copy_(p, non_blocking=True)
+        for r in rows:
+            r.fn()
+        for d, h in zip(outs_dev, outs_host):
+            h.copy_(d, non_blocking=True)
+
+    for _ in range(2):
+        one()
+    barrier()
+    e0, e1 = torch.cuda.Event(True), torch.cuda.Event(True)
+    e0.record(stream)
+    n = max(1, min(args.steps, 3))
+    for _ in range(n):
+        one()
+    e1.record(stream)
+    barrier()
+    ms = e0.elapsed_time(e1) / n
+    if dist is not None:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    units = sum(r.units for r in rows)
+    return {"value": units * world / (ms * 1e-3) / 1e9, "unit": "Gelem/s", "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms}
+
+
+if __name__ == "__main__":
+    main()
