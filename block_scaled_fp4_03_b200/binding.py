@@ -32,6 +32,7 @@ SIGNATURES = {
     "razer_quantize": (_i, [_vp, _i, _i64, _i64, _i, _vp, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "mxfp4_quantize": (_i, [_vp, _i, _i64, _i64, _vp, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
     "fp4_hessian_blocks": (_i, [_vp, _i, _i64, _i64, _vp, _i, _vp, _vp, _sz, _vp]),
+    "fp4_hessian_blocks_noalloc": (_i, [_vp, _i, _i64, _i64, _vp, _i, _vp, _vp]),
     "mxfp4_channel_scale": (_i, [_vp, _i, _i64, _vp, _i, _i64, _i64, _fp, _vp, _vp, _vp, _sz, _vp]),
     "fp4_dequant_mse": (_i, [_vp, _vp, _i64, _i64, _i, _i, _vp, _i, _vp, _vp, _i, _vp, _vp, _vp]),
 }

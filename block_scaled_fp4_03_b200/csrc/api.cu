@@ -76,6 +76,7 @@ const char* fp4q_status_str(int status)
     case FP4Q_ERR_CUDA: return "CUDA error";
     case FP4Q_ERR_TIMEOUT: return "device wait timed out";
     case FP4Q_ERR_WORKSPACE: return "workspace missing or too small";
+    case FP4Q_ERR_TOO_LARGE: return "problem exceeds the library's built-in scratch";
     default: return "unknown status";
     }
 }

@@ -67,7 +67,8 @@ typedef enum {
     FP4Q_ERR_UNSUPPORTED = 3,  /* valid request this build does not implement */
     FP4Q_ERR_CUDA = 4,         /* a CUDA launch or runtime call failed */
     FP4Q_ERR_TIMEOUT = 5,      /* a device-side bounded wait gave up */
-    FP4Q_ERR_WORKSPACE = 6     /* the workspace is missing or too small */
+    FP4Q_ERR_WORKSPACE = 6,    /* the workspace is missing or too small */
+    FP4Q_ERR_TOO_LARGE = 7     /* the problem needs more than the library's built-in scratch */
 } fp4q_status;
 
 typedef enum { FP4Q_F32 = 0, FP4Q_BF16 = 1 } fp4q_dtype;
@@ -198,6 +199,28 @@ FP4Q_API int mxfp4_quantize(const void* x, int dtype, int64_t rows, int64_t cols
 FP4Q_API int fp4_hessian_blocks(const void* x, int dtype, int64_t rows, int64_t cols,
                        const float* chan_scale, int hadamard32, float* hess_blocks,
                        void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * fp4_hessian_blocks for callers that cannot allocate device memory.  No page
+ * has a counterpart: this is a packaging of the same computation.
+ *
+ * Same arguments, layout and result as fp4_hessian_blocks, minus the
+ * workspace: the per-chunk partial sums go to a 16 MiB scratch array that
+ * the library keeps in device memory (held on every GPU that loads the
+ * library, until the process exits).  Meant for code that owns no allocator
+ * -- e.g. a plugin living in another framework's fixed memory plan, or a
+ * path that must not call cudaMalloc because it can synchronize the device.
+ * The scratch needed is ceil(rows/256) * (cols/32) * 4 KiB; problems above
+ * 16 MiB of it (e.g. more than 8192 rows at 4096 columns) return
+ * FP4Q_ERR_TOO_LARGE before anything runs.  Nothing is allocated or freed.
+ * All calls share the one scratch array: calls whose work overlaps on the
+ * GPU (other streams, other threads) race -- order them on one stream.  The
+ * first call on a device looks up the scratch's device address on that
+ * device; make that first call before any stream capture begins.
+ */
+FP4Q_API int fp4_hessian_blocks_noalloc(const void* x, int dtype, int64_t rows, int64_t cols,
+                                        const float* chan_scale, int hadamard32,
+                                        float* hess_blocks, void* stream);
 
 /*
  * Online per-channel scale of [MACaQ] 3: t_j = (sigma_j^W / rms_j^X)^alpha,
