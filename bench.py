@@ -11,14 +11,16 @@ One step = one pass over every hot-path row at its workload size:
   c4  MXFP4 prep: channel scale t from 8192x4096 bf16 activations and
       4096x4096 bf16 weights, Hessian blocks H', activation quantize (t,
       Hadamard-32, E8M0), weight quantize with the Hessian-weighted exponent
-  c5  dynamic 4-over-6 NVFP4 activation quantize of 8192x4096 bf16 into the
-      MMA scale layout
+  c5  W4A4 GEMM M=8192 x K=4096 x N=14336 -> bf16: dynamic 4-over-6 NVFP4
+      quantize of the bf16 activations into the MMA scale layout, then the
+      tcgen05 block-scaled GEMM on weights quantized once beforehand
 Inputs are synthetic and seeded (block_scaled_fp4_03_b200.inputs), resident in
 HBM when timing starts; L2 is flushed (a 512 MiB write) before every step.
 
 The JSON line's value is elements quantized per second over the whole step
-(Gelem/s, all ranks); per-row times, bandwidths and roofline fractions are in
-"rows".  `--impl reference` times the plain CPU oracle on a bounded sample of
+(Gelem/s, all ranks; the GEMM's time is part of the step); per-row times,
+bandwidths, TFLOP/s and roofline fractions are in "rows", the GEMM's
+TFLOP/s and FP4-peak fraction also under "gemm".  `--impl reference` times the plain CPU oracle on a bounded sample of
 the same workload instead.
 """
 from __future__ import annotations
@@ -37,7 +39,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "FP4 quantize Gelem/s & % of HBM roofline; W4A4 GEMM TFLOP/s & % FP4 peak"
-WORKLOAD = "hot path: one pass of every row (NVFP4 4096^2 PZ; 8192^2 block-size x rule sweep; RaZeR W 8192^2 + A 16384x4096; MXFP4 prep 8192x4096 + 4096^2; 4-over-6 act quant 8192x4096)"
+WORKLOAD = "hot path: one pass of every row (NVFP4 4096^2 PZ; 8192^2 block-size x rule sweep; RaZeR W 8192^2 + A 16384x4096; MXFP4 prep 8192x4096 + 4096^2; W4A4 GEMM 8192x14336x4096 with 4-over-6 activation quant)"
 SM_COUNT = 148
 FP32_LANES_PER_SM = 128
 
@@ -47,9 +49,10 @@ def load_peaks():
     try:
         with open(p) as f:
             d = json.load(f)
-        return float(d["hbm_gbs"]), float(d.get("sm_max_mhz", 1965.0)), "measured"
+        return (float(d["hbm_gbs"]), float(d.get("sm_max_mhz", 1965.0)), float(d["bf16_tflops"]),
+                float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured")
     except Exception:
-        return 6650.0, 1965.0, "fallback"
+        return 6650.0, 1965.0, 1590.0, 1400.0, "fallback"
 
 
 # ----------------------------------------------------------------------------- rows
@@ -145,16 +148,32 @@ def build_rows(torch, fq, inputs, dev, host_copies=None):
     rows.append(Row("c4_mx_act", "mx_quant_absmax_kernel", x4.size, x4.size * (2 + 0.5 + 1 / 32), 1, c4a, o4a))
     rows.append(Row("c4_mx_weight_hessian", "mx_quant_hessian_kernel", w4.size, w4.size * (2 + 0.5 + 1 / 32) + C * 32 * 4,
                     1, c4w, o4w, bound="alu", flops=2.0 * 3 * N4 * (C // 32) * 32 * 32))
-    # c5
+    # c5: weights pre-quantized once (abs-max NVFP4, hierarchical scale, MMA
+    # scale layout) outside the timed step; the step quantizes the activations
+    # (4-over-6, MMA layout) and runs the tcgen05 GEMM on the packed operands
     a5 = inputs.generate("gemm_act")
     X["c5"] = to_dev(a5, "c5")
+    w5 = inputs.generate("gemm_weight")
+    w5d = torch.from_numpy(w5.view(np.int16)).to(dev).view(torch.bfloat16)
+    M5, K5 = a5.shape
+    N5 = w5.shape[0]
+    qw5 = fq.nvfp4_quantize(w5d, 16, fq.ABSMAX, gs_mode=fq.GS_AMAX, sf_layout=fq.SF_MMA)
+    del w5d
     ws5 = torch.empty(fq.workspace_size(fq.OP_QUANTIZE, 1, 1), dtype=torch.uint8, device=dev)
+    wsg = torch.empty(fq.workspace_size(fq.OP_GEMM, 128, 256, 256), dtype=torch.uint8, device=dev)
     o5 = {}
+    y5 = torch.empty((M5, N5), dtype=torch.bfloat16, device=dev)
 
     def c5():
         o5.update(fq.nvfp4_quantize(X["c5"], 16, fq.FOUR_OVER_SIX, gs_mode=fq.GS_AMAX, sf_layout=fq.SF_MMA,
                                     out=o5, workspace=ws5))
+
+    def c5g():
+        fq.w4a4_gemm(o5["codes"], qw5["codes"], qw5["scales"], qw5["global_scale"], a_scales=o5["scales"],
+                     a_global_scale=o5["global_scale"], K=K5, out=y5, workspace=wsg)
     rows.append(Row("c5_act_quant_4o6_mma", "nvfp4_quant_kernel<16, __nv_bfloat16, 2>", a5.size, a5.size * (2 + 0.5 + 1 / 16), 2, c5, o5))
+    rows.append(Row("c5_w4a4_gemm", "w4a4_gemm_kernel", 0, M5 * K5 * (0.5 + 1 / 16) + N5 * K5 * (0.5 + 1 / 16) + M5 * N5 * 2,
+                    1, c5g, {"out": y5}, bound="tensor", flops=2.0 * M5 * N5 * K5))
     return rows, X
 
 
@@ -220,7 +239,15 @@ def oracle_sample_inputs(inputs, frac_rows):
     return {"c1": sub("gaussian", frac_rows["c1"]), "c2": sub("student_t", frac_rows["c2"]),
             "c3w": sub("razer_weight", frac_rows["c3"]), "c3a": sub("razer_act", frac_rows["c3"]),
             "c4x": sub("mx_act", frac_rows["c4"]), "c4w": sub("mx_weight", frac_rows["c4"]),
-            "c5": sub("gemm_act", frac_rows["c5"])}
+            "c5": sub("gemm_act", frac_rows["c5"]), "c5w": inputs.as_f32(inputs.generate("gemm_weight"))}
+
+
+def oracle_prepare(O, S):
+    """Weights of the GEMM row quantized once (abs-max, hierarchical), outside the timed step."""
+    if "c5q" not in S:
+        gw = O.global_scale(O.amax(S["c5w"]))
+        S["c5q"] = (O.nvfp4_quantize(S["c5w"], 16, O.RULE_ABSMAX, g=gw, want_deq=False, want_mse=False), gw)
+    return S
 
 
 def oracle_sample_run(O, S):
@@ -238,7 +265,10 @@ def oracle_sample_run(O, S):
     hb = O.hessian_blocks(S["c4x"], t, True).astype(np.float32)
     O.mxfp4_quantize(S["c4x"], t, True, O.RULE_ABSMAX, want_deq=False)
     O.mxfp4_quantize(S["c4w"], ti, True, O.RULE_HESSIAN_EXP, hb, want_deq=False)
-    O.nvfp4_quantize(S["c5"], 16, O.RULE_FOUR_OVER_SIX, g=O.global_scale(O.amax(S["c5"])), want_deq=False)
+    ga = O.global_scale(O.amax(S["c5"]))
+    qa = O.nvfp4_quantize(S["c5"], 16, O.RULE_FOUR_OVER_SIX, g=ga, want_deq=False, want_mse=False)
+    qw, gw = S["c5q"]
+    O.gemm_ref(qa["codes"], qa["scales"], ga, qw["codes"], qw["scales"], gw)
     elems = (S["c1"].size + 16 * S["c2"].size + S["c3w"].size + S["c3a"].size + S["c4x"].size + S["c4w"].size
              + S["c5"].size)
     return elems, time.perf_counter() - t0
@@ -256,7 +286,7 @@ def run_reference(args, rank, world):
     from oracle import oracle as O
     O.build()
     cores = O.get_threads()
-    S = oracle_sample_inputs(inputs, SAMPLE_ROWS)
+    S = oracle_prepare(O, oracle_sample_inputs(inputs, SAMPLE_ROWS))
     for _ in range(args.warmup):
         oracle_sample_run(O, S)
     times, elems = [], 0
@@ -306,7 +336,7 @@ def main():
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     fq.lib(build_if_missing=True)
-    hbm_peak, sm_max_mhz, peak_src = load_peaks()
+    hbm_peak, sm_max_mhz, bf16_peak, bf16_sust, peak_src = load_peaks()
 
     host = {}
     rows, X = build_rows(torch, fq, inputs, dev, host)
@@ -386,7 +416,17 @@ def main():
         if r.evals:
             row_out[r.name]["Geval_s"] = r.evals / (row_out[r.name]["ms"] * 1e-3) / 1e9
             row_out[r.name]["alu_frac"] = row_out[r.name]["Geval_s"] / eval_peak
-    if dom.bound == "alu" and dom.evals:
+    fp4_peak = bf16_peak * 4.0     # dense FP4 = 4 x dense bf16 (nominal 9 / 2.25 PFLOP/s)
+    for r in rows:
+        if r.bound == "tensor":
+            row_out[r.name]["tensor_frac"] = row_out[r.name]["TFLOP_s"] / fp4_peak
+    if dom.bound == "tensor":
+        ach = dom.flops / (dms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": ach, "peak": fp4_peak, "unit": "TFLOP/s", "frac": ach / fp4_peak,
+                "traffic": None, "kernel": dom.kernel, "row": dom.name,
+                "note": "FP4 peak = measured bf16 burst x 4 (nominal fp4/bf16 ratio); sustained-based: %.3f"
+                        % (ach / (bf16_sust * 4.0))}
+    elif dom.bound == "alu" and dom.evals:
         ach = dom.evals / (dms * 1e-3) / 1e9
         roof = {"bound": "alu", "achieved": ach, "peak": eval_peak, "unit": "Geval/s", "frac": ach / eval_peak,
                 "traffic": None, "kernel": dom.kernel, "row": dom.name,
@@ -406,7 +446,7 @@ def main():
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         from oracle import oracle as O
         O.build()
-        S = oracle_sample_inputs(inputs, SAMPLE_ROWS)
+        S = oracle_prepare(O, oracle_sample_inputs(inputs, SAMPLE_ROWS))
         secs = []
         for _ in range(3):
             elems, sec = oracle_sample_run(O, S)
@@ -417,13 +457,19 @@ def main():
                          "3 repeats, %.1f s each" % (elems, FULL_ELEMS, sec)}
 
     launches = sum(r.launches for r in rows) * args.steps
+    gem = next((r for r in rows if r.bound == "tensor"), None)
+    gemm = None
+    if gem is not None:
+        g = row_out[gem.name]
+        gemm = {"TFLOP_s": g["TFLOP_s"], "frac_of_fp4_peak": g["tensor_frac"], "fp4_peak_TFLOP_s": fp4_peak,
+                "ms": g["ms"], "shape": "M=8192 N=14336 K=4096"}
     line = {
         "metric": METRIC, "value": value, "unit": "Gelem/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": WORKLOAD, "elements_per_step_per_gpu": units, "l2": "flushed before every step (512 MiB write)",
                    "parallelism": "replicas: every rank runs the full step on its own inputs"},
-        "roofline": roof, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clk,
+        "roofline": roof, "gemm": gemm, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clk,
         "rows": row_out,
     }
     if rank == 0:

@@ -15,7 +15,7 @@ import torch
 
 from . import build as _build
 
-F32, BF16 = 0, 1
+F32, BF16, NVFP4_PACKED = 0, 1, 2
 SF_E4M3, SF_E3M3, SF_E8M0 = 0, 1, 2
 ABSMAX, PREVENT_ZERO, FOUR_OVER_SIX, BRUTE_FORCE, HESSIAN_EXP = range(5)
 GS_NONE, GS_AMAX, GS_GIVEN = 0, 1, 2
@@ -35,6 +35,8 @@ SIGNATURES = {
     "fp4_hessian_blocks_noalloc": (_i, [_vp, _i, _i64, _i64, _vp, _i, _vp, _vp]),
     "mxfp4_channel_scale": (_i, [_vp, _i, _i64, _vp, _i, _i64, _i64, _fp, _vp, _vp, _vp, _sz, _vp]),
     "fp4_dequant_mse": (_i, [_vp, _vp, _i64, _i64, _i, _i, _vp, _i, _vp, _vp, _i, _vp, _vp, _vp]),
+    "w4a4_gemm": (_i, [_vp, _i, _i, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _sz, _vp]),
+    "fp4q_gemm_status": (_i, [_vp, _vp]),
 }
 
 _lock = threading.Lock()
@@ -229,3 +231,34 @@ def dequant_mse(codes: torch.Tensor, scales: torch.Tensor, rows: int, cols: int,
                                _ptr(dq), _ptr(ms), _stream(stream))
     _check(st, "fp4_dequant_mse")
     return dict(dequant=dq, mse=ms)
+
+
+def w4a4_gemm(a: torch.Tensor, w_codes: torch.Tensor, w_scales: torch.Tensor, w_global_scale: torch.Tensor,
+              a_scales: torch.Tensor | None = None, a_global_scale: torch.Tensor | None = None,
+              a_rule: int = FOUR_OVER_SIX, K: int | None = None, out: torch.Tensor | None = None,
+              workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """out = A . W^T in bf16.  `a` is either a dense fp32/bf16 [M, K] tensor (quantized on the
+    fly with `a_rule`) or packed NVFP4 codes [M, K/2] uint8 with `a_scales` (MMA layout) and
+    `a_global_scale`.  W is packed codes [N, K/2] with MMA-layout scales."""
+    _need_cuda(a, w_codes, w_scales, w_global_scale, a_scales, a_global_scale)
+    if a.dtype == torch.uint8:
+        fmt = NVFP4_PACKED
+        M = a.shape[0]
+        K = a.shape[1] * 2 if K is None else K
+    else:
+        fmt = _dtype_code(a)
+        M, K = a.shape
+    N = w_codes.shape[0]
+    dev = a.device
+    o = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    ws, wsb = (workspace, workspace.numel()) if workspace is not None else _workspace(OP_GEMM, M, K, N, dev, None)
+    st = lib().w4a4_gemm(_ptr(a), fmt, a_rule, _ptr(a_scales), _ptr(a_global_scale), _ptr(w_codes),
+                         _ptr(w_scales), _ptr(w_global_scale), M, N, K, _ptr(o), _ptr(ws), wsb,
+                         _stream(stream))
+    _check(st, "w4a4_gemm")
+    return o
+
+
+def gemm_status(workspace: torch.Tensor, stream=None) -> int:
+    """Synchronize and return the device-side status word of the last GEMM on `workspace`."""
+    return int(lib().fp4q_gemm_status(_ptr(workspace), _stream(stream)))

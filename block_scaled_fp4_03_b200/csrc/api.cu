@@ -20,6 +20,12 @@ cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 int from_cuda(cudaError_t e) { return e == cudaSuccess ? FP4Q_OK : FP4Q_ERR_CUDA; }
 
 constexpr size_t kQuantWs = 4096;   // >= kAmaxPartials floats, rounded up
+// GEMM workspace: [0, 4096) amax partials, 4096 g_a, 4160 error word, then the
+// quantized A (codes, then MMA-layout scales) from 8192 on.
+constexpr size_t kGemmHeader = 8192;
+constexpr size_t kGemmGa = 4096;
+constexpr size_t kGemmErr = 4160;
+size_t gemm_ws_bytes(int64_t M, int64_t K) { return kGemmHeader + (size_t)M * (size_t)K / 2 + (size_t)M * (size_t)K / 16; }
 static_assert(kAmaxPartials * sizeof(float) <= kQuantWs, "amax partials must fit");
 
 // Resolve a global-scale request into launch arguments (running the amax
@@ -62,6 +68,7 @@ size_t fp4q_workspace_size(int op, int64_t rows, int64_t cols, int64_t n)
     case FP4Q_OP_QUANTIZE: return kQuantWs;
     case FP4Q_OP_HESSIAN: return cols % 32 ? 0 : hessian_ws_bytes(rows, cols);
     case FP4Q_OP_CHANNEL_SCALE: return channel_scale_ws_bytes(rows, n, cols);
+    case FP4Q_OP_GEMM: return gemm_ws_bytes(rows, cols);
     default: return 0;
     }
 }
@@ -251,6 +258,75 @@ int fp4_dequant_mse(const uint8_t* codes, const uint8_t* scales, int64_t rows, i
     return from_cuda(launch_dequant_mse(codes, scales, rows, cols, block, scale_fmt, specials,
                                         specials ? n_special : 0, global_scale, ref, ref_dtype,
                                         dequant, block_mse, as_stream(stream)));
+}
+
+int w4a4_gemm(const void* a, int a_format, int a_rule, const uint8_t* a_scales,
+              const float* a_global_scale, const uint8_t* w_codes, const uint8_t* w_scales,
+              const float* w_global_scale, int64_t M, int64_t N, int64_t K, void* out,
+              void* workspace, size_t workspace_bytes, void* stream)
+{
+    if (!a || !w_codes || !w_scales || !w_global_scale || !out || !workspace)
+        return FP4Q_ERR_ARG;
+    if (a_format != FP4Q_F32 && a_format != FP4Q_BF16 && a_format != FP4Q_NVFP4_PACKED)
+        return FP4Q_ERR_ARG;
+    if (a_format == FP4Q_NVFP4_PACKED && (!a_scales || !a_global_scale))
+        return FP4Q_ERR_ARG;
+    if (a_format != FP4Q_NVFP4_PACKED && (a_rule < FP4Q_ABSMAX || a_rule > FP4Q_BRUTE_FORCE))
+        return FP4Q_ERR_ARG;
+    if (M <= 0 || N <= 0 || K <= 0)
+        return FP4Q_ERR_ARG;
+    if (!gemm_shape_supported(M, N, K))
+        return FP4Q_ERR_UNSUPPORTED;
+    if (!aligned16(a) || !aligned16(w_codes) || !aligned16(w_scales) || !aligned16(out) ||
+        !aligned16(workspace) || !aligned_or_null(a_scales) || !aligned16(w_global_scale) ||
+        !aligned_or_null(a_global_scale))
+        return FP4Q_ERR_ALIGN;
+    const size_t need = a_format == FP4Q_NVFP4_PACKED ? kGemmHeader : gemm_ws_bytes(M, K);
+    if (workspace_bytes < need)
+        return FP4Q_ERR_WORKSPACE;
+    cudaStream_t s = as_stream(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    int* err = reinterpret_cast<int*>(ws + kGemmErr);
+    if (cudaMemsetAsync(err, 0, sizeof(int), s) != cudaSuccess)
+        return FP4Q_ERR_CUDA;
+    const uint8_t* a_codes = static_cast<const uint8_t*>(a);
+    const uint8_t* a_sf = a_scales;
+    const float* ga = a_global_scale;
+    if (a_format != FP4Q_NVFP4_PACKED) {
+        uint8_t* qcodes = ws + kGemmHeader;
+        uint8_t* qsf = qcodes + (size_t)M * (size_t)K / 2;
+        float* g = reinterpret_cast<float*>(ws + kGemmGa);
+        GsArgs gs{};
+        gs.mode = FP4Q_GS_AMAX;
+        gs.denom = 2688.0f;
+        gs.partials = reinterpret_cast<const float*>(ws);
+        gs.n_partials = kAmaxPartials;
+        gs.out = g;
+        cudaError_t e = launch_amax(a, a_format, M * K, reinterpret_cast<float*>(ws), s);
+        if (e == cudaSuccess)
+            e = launch_nvfp4_quant(a, a_format, M, K, 16, a_rule, gs, qcodes, qsf, 1, nullptr,
+                                   nullptr, s);
+        if (e != cudaSuccess)
+            return FP4Q_ERR_CUDA;
+        a_codes = qcodes;
+        a_sf = qsf;
+        ga = g;
+    }
+    return from_cuda(launch_w4a4_gemm(a_codes, a_sf, ga, w_codes, w_scales, w_global_scale, M, N, K,
+                                      out, err, s));
+}
+
+int fp4q_gemm_status(const void* workspace, void* stream)
+{
+    if (!workspace)
+        return FP4Q_ERR_ARG;
+    int flag = 0;
+    cudaStream_t s = as_stream(stream);
+    if (cudaMemcpyAsync(&flag, static_cast<const uint8_t*>(workspace) + kGemmErr, sizeof(int),
+                        cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return FP4Q_ERR_CUDA;
+    return flag ? FP4Q_ERR_TIMEOUT : FP4Q_OK;
 }
 
 }  // extern "C"

@@ -52,6 +52,12 @@ cudaError_t launch_mxfp4_quant(const void* x, int dtype, int64_t rows, int64_t c
                                uint8_t* codes, uint8_t* scales, float* deq, float* mse,
                                cudaStream_t s);
 
+bool gemm_shape_supported(int64_t M, int64_t N, int64_t K);
+
+cudaError_t launch_w4a4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* ga,
+                             const uint8_t* w_codes, const uint8_t* w_sf, const float* gw, int64_t M,
+                             int64_t N, int64_t K, void* out, int* err, cudaStream_t s);
+
 // Workspace (bytes) launch_hessian_blocks / launch_mx_channel_scale need.
 size_t hessian_ws_bytes(int64_t rows, int64_t cols);
 size_t channel_scale_ws_bytes(int64_t tokens, int64_t n_out, int64_t cols);

@@ -71,7 +71,7 @@ typedef enum {
     FP4Q_ERR_TOO_LARGE = 7     /* the problem needs more than the library's built-in scratch */
 } fp4q_status;
 
-typedef enum { FP4Q_F32 = 0, FP4Q_BF16 = 1 } fp4q_dtype;
+typedef enum { FP4Q_F32 = 0, FP4Q_BF16 = 1, FP4Q_NVFP4_PACKED = 2 } fp4q_dtype;
 
 /* Block-scale formats: E4M3 = OCP FP8 E4M3FN (NVFP4 and RaZeR activations),
  * E3M3 = 6-bit unsigned, bias 3, 2^-5..30 (RaZeR weights, [RaZeR] 2.1),
@@ -250,6 +250,39 @@ FP4Q_API int fp4_dequant_mse(const uint8_t* codes, const uint8_t* scales, int64_
                     int block, int scale_fmt, const float* specials, int n_special,
                     const float* global_scale, const void* ref, int ref_dtype, float* dequant,
                     float* block_mse, void* stream);
+
+/*
+ * W4A4 GEMM on NVFP4 operands ([NVFP4] 1: W4A4 inference with E2M1 values and
+ * E4M3 scales per 16 elements; [NVFP4] 3: per-tensor global scales).
+ *
+ *   out[m][n] = bf16( g_a * g_w * sum_k (v_a sc_a)[m][k] * (v_w sc_w)[n][k] ),
+ *   i.e. out = A . W^T, A: M x K, W: N x K, out: M x N bf16 row-major.
+ *
+ *  a, a_format    FP4Q_F32 / FP4Q_BF16: A is a dense M x K tensor quantized here
+ *                 (block 16, rule a_rule of ABSMAX/PREVENT_ZERO/FOUR_OVER_SIX/BRUTE_FORCE,
+ *                 g_a = amax(A)/2688) into the workspace, then multiplied;
+ *                 FP4Q_NVFP4_PACKED: a = packed codes (M*K/2 bytes), a_scales = E4M3
+ *                 bytes in the MMA layout (FP4Q_SFLAYOUT_MMA), a_global_scale = device g_a
+ *  w_codes        device N*K/2 packed codes; w_scales E4M3 bytes in the MMA layout;
+ *                 w_global_scale device g_w
+ *  M % 128 == 0, N % 256 == 0, K % 256 == 0 (FP4Q_ERR_UNSUPPORTED otherwise)
+ *  workspace      >= fp4q_workspace_size(FP4Q_OP_GEMM, M, K, N) bytes (at least 8 KiB
+ *                 for packed A), 16-byte aligned; it also holds the error word read by
+ *                 fp4q_gemm_status
+ * The product runs on tcgen05 tensor cores with fp32 accumulation in TMEM.
+ */
+FP4Q_API int w4a4_gemm(const void* a, int a_format, int a_rule, const uint8_t* a_scales,
+                       const float* a_global_scale, const uint8_t* w_codes,
+                       const uint8_t* w_scales, const float* w_global_scale, int64_t M,
+                       int64_t N, int64_t K, void* out, void* workspace,
+                       size_t workspace_bytes, void* stream);
+
+/*
+ * Synchronizes `stream` and reports whether the last w4a4_gemm that used this
+ * workspace finished normally (FP4Q_OK) or gave up a bounded device-side wait
+ * (FP4Q_ERR_TIMEOUT; its output is then incomplete).
+ */
+FP4Q_API int fp4q_gemm_status(const void* workspace, void* stream);
 
 #ifdef __cplusplus
 }
