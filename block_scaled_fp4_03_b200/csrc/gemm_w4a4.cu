@@ -6,9 +6,9 @@
 // "Why Gated DeltaNet Survives 4-Bit Quantization" review, section 1.
 //
 // Kernel shape (one CTA per SM, persistent over 128 x 256 output tiles):
-//   warp 0     TMA producer: FP4 code tiles (128B-swizzled, K-major) by
-//              cp.async.bulk.tensor, scale-factor atoms (512 contiguous bytes
-//              each, already in the MMA layout) by cp.async.bulk
+//   warp 0     TMA producer: FP4 code tiles (128B-swizzled, K-major) and
+//              scale-factor atoms (512 contiguous bytes each, already in the
+//              MMA layout) by cp.async.bulk.tensor
 //   warp 1     TMEM owner + MMA issuer: tcgen05.cp moves the scale atoms into
 //              TMEM, tcgen05.mma.kind::mxf4nvf4.block_scale.block16 (M=128,
 //              N=256, K=64) accumulates in TMEM, tcgen05.commit frees stages
@@ -49,6 +49,8 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSfCol0 = 256;              // accumulator uses columns [0, 256)
 constexpr uint32_t kSfColsPerStage = 48;       // SFA 4 k-steps x 4 + SFB 4 k-steps x 8
 constexpr long long kWaitCycles = 4000000000LL;   // about 2 s at the boost clock
+// The pair teardown outlasts a peer's own quiesce waits.
+constexpr long long kTeardownCycles = 3 * kWaitCycles;
 
 static_assert(kStageBytes % 1024 == 0, "stage bases must keep the 1024-byte swizzle alignment");
 static_assert(kSfCol0 + kStages * kSfColsPerStage <= kTmemCols, "TMEM budget");
@@ -93,14 +95,56 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
     return ok != 0;
 }
 
-// Wait for the phase with the given parity; false if it did not complete in time.
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity)
+// Wait for the phase with the given parity.  False if it did not complete
+// in time or, while waiting, this CTA's abort flag was raised.
+__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const volatile int* abort_flag)
+{
+    if (mbar_try_wait(bar, parity))
+        return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        if (*abort_flag || clock64() - t0 > kWaitCycles)
+            return false;
+    }
+    return true;
+}
+
+// Time-bounded wait that ignores the abort flag: used to let this CTA's own
+// copies and MMAs finish before its resources go away.
+__device__ __noinline__ bool mbar_quiesce(uint32_t bar, uint32_t parity)
 {
     if (mbar_try_wait(bar, parity))
         return true;
     const long long t0 = clock64();
     while (!mbar_try_wait(bar, parity)) {
         if (clock64() - t0 > kWaitCycles)
+            return false;
+    }
+    return true;
+}
+
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok)
+                 : "r"(bar), "r"(parity)
+                 : "memory");
+    return ok != 0;
+}
+
+// Bounded wait with cluster-scope acquire, for barriers that other CTAs arrive
+// on; gives up after `limit` cycles or when the abort flag (if any) is raised.
+__device__ __noinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, const volatile int* abort_flag,
+                                               long long limit = kWaitCycles)
+{
+    if (mbar_try_wait_cluster(bar, parity))
+        return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait_cluster(bar, parity)) {
+        if ((abort_flag && *abort_flag) || clock64() - t0 > limit)
             return false;
     }
     return true;
@@ -116,10 +160,12 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
                  : "memory");
 }
 
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar)
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y, int z,
+                                            uint32_t bar)
 {
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
-                 "l"(src), "r"(bytes), "r"(bar)
+    asm volatile("cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+                 " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+                 "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
                  : "memory");
 }
 
@@ -192,8 +238,9 @@ struct GemmParams {
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
-w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                 const GemmParams p)
+w4a4_gemm_1sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
+                     const GemmParams p)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -249,7 +296,7 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 const int mt = tile % p.tiles_m;
                 const int nt = tile / p.tiles_m;
                 for (int kb = 0; kb < p.kblocks; ++kb) {
-                    if (!mbar_wait(empty_bar(stage), phase ^ 1u) || *abort_flag) {
+                    if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag) || *abort_flag) {
                         give_up();
                         break;
                     }
@@ -258,13 +305,10 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                     uint8_t* st = smem + stage * kStageBytes;
                     tma_load_2d(smem_u32(st), &tmA, kb * (kBK / 2), mt * kBM, fb);
                     tma_load_2d(smem_u32(st + kAStage), &tmB, kb * (kBK / 2), nt * kBN, fb);
-                    const uint8_t* sa = p.sfa + ((int64_t)mt * p.kb_atoms + (int64_t)kb * 4) * 512;
-                    const uint8_t* sb0 = p.sfb + ((int64_t)(2 * nt) * p.kb_atoms + (int64_t)kb * 4) * 512;
-                    const uint8_t* sb1 = p.sfb + ((int64_t)(2 * nt + 1) * p.kb_atoms + (int64_t)kb * 4) * 512;
-                    bulk_load(smem_u32(st + kAStage + kBStage), sa, kSfaStage, fb);
-                    bulk_load(smem_u32(st + kAStage + kBStage + kSfaStage), sb0, kSfbStage / 2, fb);
-                    bulk_load(smem_u32(st + kAStage + kBStage + kSfaStage + kSfbStage / 2), sb1,
-                              kSfbStage / 2, fb);
+                    // scale atoms: 4 consecutive K atoms of row atom mt (A), of row
+                    // atoms 2nt and 2nt+1 (B)
+                    tma_load_3d(smem_u32(st + kAStage + kBStage), &tmSA, 0, kb * 4, mt, fb);
+                    tma_load_3d(smem_u32(st + kAStage + kBStage + kSfaStage), &tmSB, 0, kb * 4, 2 * nt, fb);
                     issued |= 1u << stage;
                     issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
                     if (++stage == kStages) {
@@ -277,7 +321,7 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                 // let the copies this thread started land before the CTA exits
                 for (int s = 0; s < kStages; ++s)
                     if (issued & (1u << s))
-                        mbar_wait(full_bar(s), (issued_parity >> s) & 1u);
+                        mbar_quiesce(full_bar(s), (issued_parity >> s) & 1u);
             }
         }
     } else if (warp == 1) {
@@ -287,14 +331,14 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             uint32_t phase = 0, acc_phase = 0;
             bool issued_any = false;
             for (int tile = blockIdx.x; tile < num_tiles && !*abort_flag; tile += gridDim.x) {
-                if (!mbar_wait(acc_empty, acc_phase ^ 1u) || *abort_flag) {
+                if (!mbar_wait(acc_empty, acc_phase ^ 1u, abort_flag) || *abort_flag) {
                     give_up();
                     break;
                 }
                 tc_fence_after();
                 bool ok = true;
                 for (int kb = 0; kb < p.kblocks; ++kb) {
-                    if (!mbar_wait(full_bar(stage), phase) || *abort_flag) {
+                    if (!mbar_wait(full_bar(stage), phase, abort_flag) || *abort_flag) {
                         give_up();
                         ok = false;
                         break;
@@ -332,7 +376,7 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
             if (issued_any) {
                 // every MMA and copy this thread issued has finished once this arrives
                 tc_commit(drain);
-                if (!mbar_wait(drain, 0))
+                if (!mbar_quiesce(drain, 0))
                     give_up();
             }
         }
@@ -342,7 +386,7 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
         uint32_t acc_phase = 0;
         const float scale = __fmul_rn(__ldg(p.ga), __ldg(p.gw));
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-            bool ok = !*abort_flag && mbar_wait(acc_full, acc_phase);
+            bool ok = !*abort_flag && mbar_wait(acc_full, acc_phase, abort_flag);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) {
                 if (lane == 0)
@@ -385,6 +429,352 @@ w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant_
                      : "memory");
 }
 
+// ===================================================== CTA-pair (cta_group::2)
+// Two CTAs of a cluster compute a 256 x 256 output tile with M=256, N=256,
+// K=64 pair MMAs issued by the leader (cluster rank 0).  Each CTA stages its
+// own 128 rows of A, its own 128 rows of B (the MMA reads the two halves of
+// B from the two CTAs), its own A scale atom and both B scale atoms, and
+// signals its own barrier; the follower forwards "stage ready" to the leader
+// with one remote arrive.  The leader's commits are multicast to both CTAs.
+// The epilogue stages bf16 32 x 64 boxes in 128B-swizzled shared memory (two
+// boxes, half a tile row, at a time) and writes them with TMA stores, handing
+// the accumulator back as soon as its TMEM reads are done, so the stores
+// overlap the next tile's main loop.  Five 38 KiB stages keep ~190 KiB of
+// operands in flight per SM.
+constexpr int k2Stages = 5;
+constexpr int k2AStage = 128 * kBK / 2;        // 16 KiB
+constexpr int k2BStage = 128 * kBK / 2;        // 16 KiB (this CTA's half of B)
+constexpr int k2SfaStage = 128 * kBK / 16;     // 2 KiB
+constexpr int k2SfbStage = 256 * kBK / 16;     // 4 KiB (both B row atoms)
+constexpr int k2StageBytes = k2AStage + k2BStage + k2SfaStage + k2SfbStage;
+constexpr int k2EpiWarpBytes = 32 * 128 * 2;   // 32 rows x 128 bf16 per epilogue warp (half a tile row)
+constexpr int k2EpiBytes = 4 * k2EpiWarpBytes;
+constexpr int k2SmemBytes = k2Stages * k2StageBytes + k2EpiBytes + 1024 + kBarBytes;
+static_assert(k2StageBytes % 1024 == 0 && (k2Stages * k2StageBytes) % 1024 == 0, "swizzle alignment");
+static_assert(k2SmemBytes <= 232448, "shared memory budget");
+static_assert(kSfCol0 + k2Stages * kSfColsPerStage <= kTmemCols, "TMEM budget");
+
+// Pair instruction descriptor: E2M1 x E2M1, K-major, UE4M3 scales, N = 256, M = 256.
+constexpr uint32_t k2Idesc = (1u << 7) | (1u << 10) | ((uint32_t)(256 >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
+
+__device__ __forceinline__ uint32_t cluster_rank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// Address of the same shared-memory offset in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t mapa_rank(uint32_t saddr, uint32_t rank)
+{
+    uint32_t d;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(d) : "r"(saddr), "r"(rank));
+    return d;
+}
+
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr)
+{
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+__device__ __forceinline__ void tc2_commit_mc(uint32_t bar, uint16_t mask)
+{
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+                 "h"(mask)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc2_cp_sf(uint32_t taddr, uint64_t sdesc)
+{
+    asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+__device__ __forceinline__ void tc2_mma(uint32_t tacc, uint64_t da, uint64_t db, uint32_t idesc,
+                                        uint32_t accumulate, uint32_t tsfa, uint32_t tsfb)
+{
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "setp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(tacc),
+                 "l"(da), "l"(db), "r"(idesc), "r"(accumulate), "r"(tsfa), "r"(tsfb)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int x, int y)
+{
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(src), "r"(x), "r"(y)
+                 : "memory");
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+w4a4_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
+                     const __grid_constant__ CUtensorMap tmOut, const GemmParams p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* epi = smem + k2Stages * k2StageBytes;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(epi + k2EpiBytes);
+    // bars: [0,S) full, [S,2S) empty, [2S,3S) peer-ready (leader), 3S acc_full,
+    // 3S+1 acc_empty (leader), 3S+2 drain, 3S+3 teardown handshake
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 3 * k2Stages + 4);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();
+    const bool leader = rank == 0;
+    const uint32_t bar0 = smem_u32(bars);
+    auto full_bar = [&](int s) { return bar0 + 8u * (uint32_t)s; };
+    auto empty_bar = [&](int s) { return bar0 + 8u * (uint32_t)(k2Stages + s); };
+    auto peer_bar = [&](int s) { return bar0 + 8u * (uint32_t)(2 * k2Stages + s); };
+    const uint32_t acc_full = bar0 + 8u * (3 * k2Stages);
+    const uint32_t acc_empty = bar0 + 8u * (3 * k2Stages + 1);
+    const uint32_t drain = bar0 + 8u * (3 * k2Stages + 2);
+    const uint32_t bye = bar0 + 8u * (3 * k2Stages + 3);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < k2Stages; ++s) {
+            mbar_init(full_bar(s), 1);
+            mbar_init(empty_bar(s), 1);
+            mbar_init(peer_bar(s), 1);
+        }
+        mbar_init(acc_full, 1);
+        mbar_init(acc_empty, 2 * 128);
+        mbar_init(drain, 1);
+        mbar_init(bye, 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_holder)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    // both CTAs' barriers exist before either touches the other's
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+    const int cluster = blockIdx.x >> 1;
+    const int nclusters = gridDim.x >> 1;
+    const int num_tiles = p.tiles_m * p.tiles_n;
+    const uint32_t peer_abort = mapa_rank(smem_u32(const_cast<int*>(abort_flag)), rank ^ 1u);
+
+    // A failed wait stops both CTAs of the pair: every role polls its own
+    // abort flag, so all of them head for the teardown handshake at once.
+    auto give_up = [&]() {
+        *abort_flag = 1;
+        asm volatile("st.relaxed.cluster.shared::cluster.u32 [%0], %1;" ::"r"(peer_abort), "r"(1) : "memory");
+        atomicExch(p.err, 1);
+    };
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // -------------------------------------------- producer (both CTAs)
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t issued = 0, issued_parity = 0;
+            for (int tile = cluster; tile < num_tiles && !*abort_flag; tile += nclusters) {
+                const int mt = tile % p.tiles_m;
+                const int nt = tile / p.tiles_m;
+                for (int kb = 0; kb < p.kblocks; ++kb) {
+                    if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag) || *abort_flag) {
+                        give_up();
+                        break;
+                    }
+                    const uint32_t fb = full_bar(stage);
+                    mbar_expect_tx(fb, k2StageBytes);
+                    uint8_t* st = smem + stage * k2StageBytes;
+                    tma_load_2d(smem_u32(st), &tmA, kb * (kBK / 2), mt * 256 + (int)rank * 128, fb);
+                    tma_load_2d(smem_u32(st + k2AStage), &tmB, kb * (kBK / 2), nt * 256 + (int)rank * 128, fb);
+                    tma_load_3d(smem_u32(st + k2AStage + k2BStage), &tmSA, 0, kb * 4, 2 * mt + (int)rank, fb);
+                    tma_load_3d(smem_u32(st + k2AStage + k2BStage + k2SfaStage), &tmSB, 0, kb * 4, 2 * nt, fb);
+                    issued |= 1u << stage;
+                    issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+                    if (++stage == k2Stages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (*abort_flag)
+                for (int s = 0; s < k2Stages; ++s)
+                    if (issued & (1u << s))
+                        mbar_quiesce(full_bar(s), (issued_parity >> s) & 1u);
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && leader) {
+            // ------------------------------------------- MMA issuer (leader)
+            int stage = 0;
+            uint32_t phase = 0, acc_phase = 0;
+            bool issued_any = false;
+            for (int tile = cluster; tile < num_tiles && !*abort_flag; tile += nclusters) {
+                if (!mbar_wait_cluster(acc_empty, acc_phase ^ 1u, abort_flag) || *abort_flag) {
+                    give_up();
+                    break;
+                }
+                tc_fence_after();
+                bool ok = true;
+                for (int kb = 0; kb < p.kblocks; ++kb) {
+                    if (!mbar_wait(full_bar(stage), phase, abort_flag) ||
+                        !mbar_wait_cluster(peer_bar(stage), phase, abort_flag) || *abort_flag) {
+                        give_up();
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    uint8_t* st = smem + stage * k2StageBytes;
+                    const uint32_t sa_s = smem_u32(st + k2AStage + k2BStage);
+                    const uint32_t sb_s = sa_s + k2SfaStage;
+                    const uint32_t tsfa = tmem + kSfCol0 + (uint32_t)stage * kSfColsPerStage;
+                    const uint32_t tsfb = tsfa + 16;
+#pragma unroll
+                    for (int s = 0; s < 4; ++s) {
+                        tc2_cp_sf(tsfa + 4 * s, sdesc_sf(sa_s + 512 * s));
+                        tc2_cp_sf(tsfb + 8 * s, sdesc_sf(sb_s + 512 * s));
+                        tc2_cp_sf(tsfb + 8 * s + 4, sdesc_sf(sb_s + k2SfbStage / 2 + 512 * s));
+                    }
+                    const uint32_t a_s = smem_u32(st);
+                    const uint32_t b_s = a_s + k2AStage;
+#pragma unroll
+                    for (int s = 0; s < 4; ++s)
+                        tc2_mma(tmem, sdesc_sw128(a_s + 32 * s), sdesc_sw128(b_s + 32 * s), k2Idesc,
+                                (kb | s) != 0, tsfa + 4 * s, tsfb + 8 * s);
+                    issued_any = true;
+                    tc2_commit_mc(empty_bar(stage), (uint16_t)0x3);
+                    if (++stage == k2Stages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok)
+                    break;
+                tc2_commit_mc(acc_full, (uint16_t)0x3);
+                acc_phase ^= 1u;
+            }
+            if (issued_any) {
+                tc2_commit_mc(drain, (uint16_t)0x1);
+                if (!mbar_quiesce(drain, 0))
+                    give_up();
+            }
+        } else if (lane == 0) {
+            // --------------------- follower: forward "stage ready" to the leader
+            int stage = 0;
+            uint32_t phase = 0;
+            for (int tile = cluster; tile < num_tiles && !*abort_flag; tile += nclusters) {
+                bool ok = true;
+                for (int kb = 0; kb < p.kblocks; ++kb) {
+                    if (!mbar_wait(full_bar(stage), phase, abort_flag) || *abort_flag) {
+                        give_up();
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_cluster(mapa_rank(peer_bar(stage), 0));
+                    if (++stage == k2Stages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok)
+                    break;
+            }
+        }
+    } else {
+        // ------------------------------------------------ epilogue (both CTAs)
+        const int q = warp & 3;
+        uint8_t* stg = epi + q * k2EpiWarpBytes;
+        const uint32_t leader_acc_empty = mapa_rank(acc_empty, 0);
+        uint32_t acc_phase = 0;
+        const float scale = __fmul_rn(__ldg(p.ga), __ldg(p.gw));
+        for (int tile = cluster; tile < num_tiles; tile += nclusters) {
+            bool ok = !*abort_flag && mbar_wait(acc_full, acc_phase, abort_flag);
+            ok = __all_sync(0xffffffffu, ok);
+            if (!ok) {
+                if (lane == 0)
+                    give_up();
+                break;
+            }
+            tc_fence_after();
+            // the previous tile's stores have finished reading the staging buffer
+            if (lane == 0)
+                asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+            __syncwarp();
+            const int mt = tile % p.tiles_m;
+            const int nt = tile / p.tiles_m;
+            const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16);
+#pragma unroll 1
+            for (int c = 0; c < 8; ++c) {
+                if (c == 4) {
+                    // second half of the row: reuse the staging buffer once the
+                    // first half's stores have read it
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    __syncwarp();
+                    if (lane == 0) {
+                        const int y = mt * 256 + (int)rank * 128 + q * 32;
+                        tma_store_2d(&tmOut, smem_u32(stg), nt * 256, y);
+                        tma_store_2d(&tmOut, smem_u32(stg + 4096), nt * 256 + 64, y);
+                        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+                        asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+                    }
+                    __syncwarp();
+                }
+                uint32_t r[32];
+                tmem_ld32(tq + 32 * c, r);
+                uint32_t pk[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[2 * j]), scale),
+                                                             __fmul_rn(__uint_as_float(r[2 * j + 1]), scale));
+                    pk[j] = *reinterpret_cast<uint32_t*>(&h);
+                }
+                // box (c/2)%2 of the staging holds columns [64 (c/2), +64); row
+                // `lane` of a box is 128 bytes whose 16-byte chunks sit at
+                // (chunk ^ (row % 8))
+                uint8_t* rowp = stg + ((c >> 1) & 1) * 4096 + lane * 128;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int chunk = (c & 1) * 4 + j;
+                    *reinterpret_cast<uint4*>(rowp + ((chunk ^ (lane & 7)) << 4)) =
+                        make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+                }
+            }
+            tc_fence_before();
+            mbar_arrive_cluster(leader_acc_empty);
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) {
+                const int y = mt * 256 + (int)rank * 128 + q * 32;
+                tma_store_2d(&tmOut, smem_u32(stg), nt * 256 + 128, y);
+                tma_store_2d(&tmOut, smem_u32(stg + 4096), nt * 256 + 192, y);
+                asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+            }
+            acc_phase ^= 1u;
+        }
+        if (lane == 0)
+            asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+        __syncwarp();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    // neither CTA leaves while the other may still read its shared memory or
+    // write its tensor memory
+    if (threadIdx.x == 0) {
+        mbar_arrive_cluster(mapa_rank(bye, rank ^ 1u));
+        if (!mbar_wait_cluster(bye, 0, nullptr, kTeardownCycles))
+            give_up();
+    }
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1)
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+                     : "memory");
+}
+
 // ------------------------------------------------------------ host side
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
 {
@@ -415,6 +805,39 @@ bool make_code_map(CUtensorMap* m, const void* base, int64_t rows, int64_t kbyte
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 3-D map over MMA-layout scale bytes viewed as [row atom][K atom][128 words]
+// (each 128-row x 4-scale atom is 512 contiguous bytes, K atoms fastest); a
+// box is 4 K atoms of `row_atoms` consecutive row atoms.
+bool make_sf_map(CUtensorMap* m, const void* base, int64_t rows, int64_t K, int row_atoms)
+{
+    auto fn = encode_fn();
+    if (!fn)
+        return false;
+    const int64_t kb_atoms = K / 64;
+    cuuint64_t dims[3] = {128u, (cuuint64_t)kb_atoms, (cuuint64_t)(rows / 128)};
+    cuuint64_t strides[2] = {512u, (cuuint64_t)kb_atoms * 512u};
+    cuuint32_t box[3] = {128u, 4u, (cuuint32_t)row_atoms};
+    cuuint32_t estr[3] = {1u, 1u, 1u};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2-D map over the bf16 output: rows x cols, box 32 rows x 64 columns (128 B), 128B swizzle.
+bool make_out_map(CUtensorMap* m, void* base, int64_t rows, int64_t cols)
+{
+    auto fn = encode_fn();
+    if (!fn)
+        return false;
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+    cuuint32_t box[2] = {64u, 32u};
+    cuuint32_t estr[2] = {1u, 1u};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 bool gemm_shape_supported(int64_t M, int64_t N, int64_t K)
@@ -427,17 +850,6 @@ cudaError_t launch_w4a4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const 
                              const uint8_t* w_codes, const uint8_t* w_sf, const float* gw, int64_t M,
                              int64_t N, int64_t K, void* out, int* err, cudaStream_t s)
 {
-    CUtensorMap ta, tb;
-    if (!make_code_map(&ta, a_codes, M, K / 2, kBM) || !make_code_map(&tb, w_codes, N, K / 2, kBN))
-        return cudaErrorInvalidValue;
-    static std::once_flag attr_once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(w4a4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        kSmemBytes);
-    });
-    if (attr_err != cudaSuccess)
-        return attr_err;
     GemmParams p;
     p.sfa = a_sf;
     p.sfb = w_sf;
@@ -445,14 +857,48 @@ cudaError_t launch_w4a4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const 
     p.gw = gw;
     p.out = reinterpret_cast<__nv_bfloat16*>(out);
     p.err = err;
-    p.tiles_m = (int)(M / kBM);
     p.tiles_n = (int)(N / kBN);
     p.kblocks = (int)(K / kBK);
     p.kb_atoms = (int)(K / 64);
     p.N = (int)N;
+    if (M % 256 == 0) {
+        // CTA pairs: 256 x 256 tiles
+        CUtensorMap ta, tb, tsa, tsb, to;
+        if (!make_code_map(&ta, a_codes, M, K / 2, 128) || !make_code_map(&tb, w_codes, N, K / 2, 128) ||
+            !make_sf_map(&tsa, a_sf, M, K, 1) || !make_sf_map(&tsb, w_sf, N, K, 2) ||
+            !make_out_map(&to, out, M, N))
+            return cudaErrorInvalidValue;
+        static std::once_flag attr2_once;
+        static cudaError_t attr2_err = cudaSuccess;
+        std::call_once(attr2_once, [] {
+            attr2_err = cudaFuncSetAttribute(w4a4_gemm_2sm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             k2SmemBytes);
+        });
+        if (attr2_err != cudaSuccess)
+            return attr2_err;
+        p.tiles_m = (int)(M / 256);
+        const int tiles = p.tiles_m * p.tiles_n;
+        const int pairs = num_sms() / 2;
+        const int grid = 2 * (tiles < pairs ? tiles : pairs);
+        w4a4_gemm_2sm_kernel<<<grid, kThreads, k2SmemBytes, s>>>(ta, tb, tsa, tsb, to, p);
+        return cudaGetLastError();
+    }
+    CUtensorMap ta, tb, tsa, tsb;
+    if (!make_code_map(&ta, a_codes, M, K / 2, kBM) || !make_code_map(&tb, w_codes, N, K / 2, kBN) ||
+        !make_sf_map(&tsa, a_sf, M, K, 1) || !make_sf_map(&tsb, w_sf, N, K, 2))
+        return cudaErrorInvalidValue;
+    static std::once_flag attr_once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(attr_once, [] {
+        attr_err = cudaFuncSetAttribute(w4a4_gemm_1sm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        kSmemBytes);
+    });
+    if (attr_err != cudaSuccess)
+        return attr_err;
+    p.tiles_m = (int)(M / kBM);
     const int tiles = p.tiles_m * p.tiles_n;
     const int grid = tiles < num_sms() ? tiles : num_sms();
-    w4a4_gemm_kernel<<<grid, kThreads, kSmemBytes, s>>>(ta, tb, p);
+    w4a4_gemm_1sm_kernel<<<grid, kThreads, kSmemBytes, s>>>(ta, tb, tsa, tsb, p);
     return cudaGetLastError();
 }
 
