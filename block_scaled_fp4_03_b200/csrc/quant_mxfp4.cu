@@ -109,17 +109,18 @@ __device__ __forceinline__ void load32(const T* __restrict__ p, float (&u)[32])
 }
 
 // ------------------------------------------------- OCP exponent (activations)
-template <typename T>
+// ERR: also produce the dequantized values / block errors (only when asked).
+template <typename T, bool ERR>
 __global__ void __launch_bounds__(kThreads)
-mx_quant_absmax_kernel(const T* __restrict__ x, int64_t nblk, int64_t kb,
+mx_quant_absmax_kernel(const T* __restrict__ x, uint32_t nblk, uint32_t kb,
                        const float* __restrict__ t, int had, uint8_t* __restrict__ codes,
                        uint8_t* __restrict__ scales, float* __restrict__ deq,
                        float* __restrict__ mse)
 {
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblk; b += stride) {
+    const uint32_t stride = gridDim.x * blockDim.x;
+    for (uint32_t b = blockIdx.x * blockDim.x + threadIdx.x; b < nblk; b += stride) {
         float u[32];
-        load32<T>(x + b * 32, u);
+        load32<T>(x + (size_t)b * 32, u);
         online_transform(u, t ? t + (b % kb) * 32 : nullptr, had != 0);
         float a = 0.0f;
 #pragma unroll
@@ -127,14 +128,26 @@ mx_quant_absmax_kernel(const T* __restrict__ x, int64_t nblk, int64_t kb,
             a = fmaxf(a, fabsf(u[i]));
         const int e = mx_exponent(a);
         uint32_t cw[4];
-        float dq[32];
-        const float sse = mx_eval(u, e, cw, dq);
-        *reinterpret_cast<uint4*>(codes + b * 16) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+        if constexpr (ERR) {
+            float dq[32];
+            const float sse = mx_eval(u, e, cw, dq);
+            if (deq)
+                store_f32<32>(deq + (size_t)b * 32, dq);
+            if (mse)
+                mse[b] = __fmul_rn(sse, 1.0f / 32.0f);
+        } else {
+            const float down = pow2f(-e);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int o = 8 * j;
+                cw[j] = e2m1x8_encode(__fmul_rn(u[o], down), __fmul_rn(u[o + 1], down),
+                                      __fmul_rn(u[o + 2], down), __fmul_rn(u[o + 3], down),
+                                      __fmul_rn(u[o + 4], down), __fmul_rn(u[o + 5], down),
+                                      __fmul_rn(u[o + 6], down), __fmul_rn(u[o + 7], down));
+            }
+        }
+        *reinterpret_cast<uint4*>(codes + (size_t)b * 16) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
         scales[b] = (uint8_t)(e + 127);
-        if (deq)
-            store_f32<32>(deq + b * 32, dq);
-        if (mse)
-            mse[b] = __fmul_rn(sse, 1.0f / 32.0f);
     }
 }
 
@@ -252,11 +265,12 @@ __global__ void __launch_bounds__(kThreads)
 hessian_partial_kernel(const T* __restrict__ x, int64_t rows, int64_t cols,
                        const float* __restrict__ t, int had, float* __restrict__ part)
 {
-    __shared__ __align__(16) float Xs[kTok][33];
+    __shared__ __align__(16) float Xs[kTok][32];
+    __shared__ __align__(16) float red[3][64][16];
     const int64_t k = blockIdx.y;
     const int64_t chunk = blockIdx.x;
     const int64_t r0 = chunk * kTok;
-    // stage: one thread per token row of this chunk
+    // stage: one thread per token row of this chunk, transformed in registers
     for (int rr = threadIdx.x; rr < kTok; rr += blockDim.x) {
         const int64_t r = r0 + rr;
         float u[32];
@@ -269,24 +283,57 @@ hessian_partial_kernel(const T* __restrict__ x, int64_t rows, int64_t cols,
                 u[i] = 0.0f;
         }
 #pragma unroll
-        for (int i = 0; i < 32; ++i)
-            Xs[rr][i] = u[i];
+        for (int i = 0; i < 32; i += 4)
+            *reinterpret_cast<float4*>(&Xs[rr][i]) = make_float4(u[i], u[i + 1], u[i + 2], u[i + 3]);
     }
     __syncthreads();
-    // thread -> entries (i, j0..j0+3): i = tid / 8, j0 = 4 * (tid % 8)
-    const int i = threadIdx.x >> 3;
-    const int j0 = (threadIdx.x & 7) * 4;
-    float acc0 = 0.0f, acc1 = 0.0f, acc2 = 0.0f, acc3 = 0.0f;
+    // thread -> 4x4 entries (4 ti + [0,4), 4 tj + [0,4)) over tokens tg, tg+4, ...
+    const int tg = threadIdx.x >> 6;
+    const int ti = (threadIdx.x >> 3) & 7;
+    const int tj = threadIdx.x & 7;
+    float acc[4][4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+            acc[a][c] = 0.0f;
     const int nr = (int)((rows - r0) < kTok ? (rows - r0) : kTok);
-    for (int rr = 0; rr < nr; ++rr) {
-        const float xi = Xs[rr][i];
-        acc0 = __fmaf_rn(xi, Xs[rr][j0], acc0);
-        acc1 = __fmaf_rn(xi, Xs[rr][j0 + 1], acc1);
-        acc2 = __fmaf_rn(xi, Xs[rr][j0 + 2], acc2);
-        acc3 = __fmaf_rn(xi, Xs[rr][j0 + 3], acc3);
+    for (int rr = tg; rr < nr; rr += 4) {
+        const float4 xi = *reinterpret_cast<const float4*>(&Xs[rr][4 * ti]);
+        const float4 xj = *reinterpret_cast<const float4*>(&Xs[rr][4 * tj]);
+        const float vi[4] = {xi.x, xi.y, xi.z, xi.w};
+        const float vj[4] = {xj.x, xj.y, xj.z, xj.w};
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                acc[a][c] = __fmaf_rn(vi[a], vj[c], acc[a][c]);
     }
-    float* o = part + (chunk * (cols / 32) + k) * 1024 + i * 32 + j0;
-    *reinterpret_cast<float4*>(o) = make_float4(acc0, acc1, acc2, acc3);
+    // sum the four token groups in a fixed order
+    if (tg > 0) {
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                red[tg - 1][threadIdx.x & 63][4 * a + c] = acc[a][c];
+    }
+    __syncthreads();
+    if (tg == 0) {
+        float* o = part + (chunk * (cols / 32) + k) * 1024;
+#pragma unroll
+        for (int a = 0; a < 4; ++a) {
+            float v4[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                float v = acc[a][c];
+                v = __fadd_rn(v, red[0][threadIdx.x][4 * a + c]);
+                v = __fadd_rn(v, red[1][threadIdx.x][4 * a + c]);
+                v = __fadd_rn(v, red[2][threadIdx.x][4 * a + c]);
+                v4[c] = v;
+            }
+            *reinterpret_cast<float4*>(o + (4 * ti + a) * 32 + 4 * tj) = make_float4(v4[0], v4[1], v4[2], v4[3]);
+        }
+    }
 }
 
 __global__ void __launch_bounds__(kThreads)
@@ -306,7 +353,7 @@ hessian_reduce_kernel(const float* __restrict__ part, int64_t nchunk, int64_t to
 // Column statistics in fp64 over a chunk of rows: sum and sum of squares.
 // One thread owns 8 consecutive columns (one 16-byte bf16 vector or two fp32
 // vectors) for every row of the chunk.
-constexpr int kStatRows = 128;
+constexpr int kStatRows = 32;
 
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
@@ -422,16 +469,19 @@ cudaError_t launch_mxfp4_quant(const void* x, int dtype, int64_t rows, int64_t c
                 scales, deq, mse);
         return cudaGetLastError();
     }
+    if (nblk > (int64_t)0xFFFFFFFFu)
+        return cudaErrorInvalidValue;
+    const bool err = deq || mse;
     if (dtype == 1) {
-        auto k = mx_quant_absmax_kernel<__nv_bfloat16>;
+        auto k = err ? mx_quant_absmax_kernel<__nv_bfloat16, true> : mx_quant_absmax_kernel<__nv_bfloat16, false>;
         k<<<grid_for(nblk, (const void*)k), kThreads, 0, s>>>(
-            reinterpret_cast<const __nv_bfloat16*>(x), nblk, kb, chan_scale, hadamard, codes,
-            scales, deq, mse);
+            reinterpret_cast<const __nv_bfloat16*>(x), (uint32_t)nblk, (uint32_t)kb, chan_scale, hadamard,
+            codes, scales, deq, mse);
     } else {
-        auto k = mx_quant_absmax_kernel<float>;
+        auto k = err ? mx_quant_absmax_kernel<float, true> : mx_quant_absmax_kernel<float, false>;
         k<<<grid_for(nblk, (const void*)k), kThreads, 0, s>>>(reinterpret_cast<const float*>(x),
-                                                               nblk, kb, chan_scale, hadamard,
-                                                               codes, scales, deq, mse);
+                                                               (uint32_t)nblk, (uint32_t)kb, chan_scale,
+                                                               hadamard, codes, scales, deq, mse);
     }
     return cudaGetLastError();
 }

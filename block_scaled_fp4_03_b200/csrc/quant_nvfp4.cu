@@ -70,7 +70,31 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const T* __restrict__ x,
     const int64_t nvec = n / V;
     float m = 0.0f;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nvec; i += stride) {
+    const int64_t i0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    // four independent 16-byte loads in flight per thread
+    int64_t i = i0;
+    for (; i + 3 * stride < nvec; i += 4 * stride) {
+        uint4 w[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+            w[u] = __ldg(reinterpret_cast<const uint4*>(x) + i + u * stride);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            if constexpr (sizeof(T) == 4) {
+                m = fmaxf(m, fmaxf(fmaxf(fabsf(__uint_as_float(w[u].x)), fabsf(__uint_as_float(w[u].y))),
+                                   fmaxf(fabsf(__uint_as_float(w[u].z)), fabsf(__uint_as_float(w[u].w)))));
+            } else {
+                const uint32_t ww[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    float lo, hi;
+                    bf16x2_to_f32(ww[q], lo, hi);
+                    m = fmaxf(m, fmaxf(fabsf(lo), fabsf(hi)));
+                }
+            }
+        }
+    }
+    for (; i < nvec; i += stride) {
         uint4 v = __ldg(reinterpret_cast<const uint4*>(x) + i);
         if constexpr (sizeof(T) == 4) {
             m = fmaxf(m, fmaxf(fmaxf(fabsf(__uint_as_float(v.x)), fabsf(__uint_as_float(v.y))),
@@ -153,13 +177,42 @@ __device__ __forceinline__ float quant_eval(const float (&x)[B], float sc, float
     return acc;
 }
 
-// Squared error only (brute-force search).
+// Squared error only (brute-force search); t = (S, inv) of the candidate,
+// precomputed exactly as quant_eval computes them.
 template <int B>
-__device__ __forceinline__ float quant_sse(const float (&x)[B], float sc, float g)
+__device__ __forceinline__ float quant_sse(const float (&x)[B], float, float, float2 t)
 {
-    uint32_t cw[(B + 7) / 8];
-    float dq[B];
-    return quant_eval<B>(x, sc, g, cw, dq);
+    const float S = t.x;
+    const float inv = t.y;
+    float acc = 0.0f;
+    if constexpr (B == 4) {
+        uint32_t w = e2m1x4_encode(__fmul_rn(x[0], inv), __fmul_rn(x[1], inv),
+                                   __fmul_rn(x[2], inv), __fmul_rn(x[3], inv));
+        float v[4];
+        e2m1x4_decode(w, v);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float e = __fsub_rn(x[i], __fmul_rn(v[i], S));
+            acc = __fmaf_rn(e, e, acc);
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < B / 8; ++j) {
+            const int o = 8 * j;
+            uint32_t w = e2m1x8_encode(__fmul_rn(x[o], inv), __fmul_rn(x[o + 1], inv),
+                                       __fmul_rn(x[o + 2], inv), __fmul_rn(x[o + 3], inv),
+                                       __fmul_rn(x[o + 4], inv), __fmul_rn(x[o + 5], inv),
+                                       __fmul_rn(x[o + 6], inv), __fmul_rn(x[o + 7], inv));
+            float v[8];
+            e2m1x8_decode(w, v);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float e = __fsub_rn(x[o + i], __fmul_rn(v[i], S));
+                acc = __fmaf_rn(e, e, acc);
+            }
+        }
+    }
+    return acc;
 }
 
 // Error of one element of magnitude a under scale S / reciprocal inv.
@@ -186,6 +239,17 @@ nvfp4_quant_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs
     const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
     const int64_t kb_atoms = (bpr + 3) >> 2;
+    // brute force: every code's effective scale S = sc * g and reciprocal
+    // inv = min(1/S, FLT_MAX) (0 for S = 0), computed once per CTA
+    __shared__ float2 bf_tab[128];
+    const bool g_one = g == 1.0f;
+    if constexpr (RULE == R_BF) {
+        for (int c = threadIdx.x; c < 128; c += blockDim.x) {
+            const float S = __fmul_rn(e4m3_decode((uint32_t)(c < 127 ? c : 126)), g);
+            bf_tab[c] = make_float2(S, (S == 0.0f) ? 0.0f : fminf(__frcp_rn(S), kFltMax));
+        }
+        __syncthreads();
+    }
 
     for (int64_t base = warp0 * 32; base < nblk; base += nwarps * 32) {
         const int64_t b = base + lane;
@@ -229,49 +293,75 @@ nvfp4_quant_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs
             for (int i = 0; i < B; ++i)
                 dq[i] = take4 ? dq4[i] : dq[i];
         } else {
-            // Brute force over E4M3 codes 1..126 in ascending order, keeping the
-            // lowest code among equal errors.  Exact shortcuts:
-            //  * once the largest element rounds to zero (|y| <= 0.25) every
-            //    element does, and every larger scale gives the same error, so
-            //    the scan stops there;
-            //  * the squared error of the largest element alone is a lower bound
-            //    of the in-order fma sum, so a candidate whose bound already
-            //    loses is skipped.
+            // Brute force over E4M3 codes 1..126: the least error, ties to the
+            // lowest code.  Exact shortcuts (each provably skips only losers):
+            //  * from the first code at which the largest element rounds to
+            //    zero (|y| <= 0.25, found by bisection: |y| falls as the code
+            //    grows) every element does, so that code gives the all-zero
+            //    error and every higher code ties it with a higher code;
+            //  * below the abs-max code the largest element clips to 6, its
+            //    error a - 6S grows as the code falls, and its square alone
+            //    bounds the in-order fma chain from below: the downward scan
+            //    stops at the first code whose bound already loses;
+            //  * in between, the same single-element bound skips candidates.
+            // Each lane walks its own range, so lanes of a warp stay busy.
             float sse0 = 0.0f;
 #pragma unroll
             for (int i = 0; i < B; ++i)
                 sse0 = __fmaf_rn(xv[i], xv[i], sse0);
-            uint32_t c0 = e4m3_encode(__fdiv_rn(a, g6));
-            c0 = c0 == 0u ? 1u : c0;
-            float best = quant_sse<B>(xv, e4m3_decode(c0), g);
-            uint32_t bc = c0;
-            bool done = !valid;
-            for (uint32_t c = 1; c <= 0x7Eu; ++c) {
-                if (!done) {
-                    const float scv = e4m3_decode(c);
-                    const float S = __fmul_rn(scv, g);
-                    const float inv = (S == 0.0f) ? 0.0f : fminf(__frcp_rn(S), kFltMax);
-                    const float ym = __fmul_rn(a, inv);
-                    if (ym <= 0.25f) {
-                        done = true;
-                        if (c != c0 && (sse0 < best || (sse0 == best && c < bc))) {
-                            best = sse0;
+            uint32_t c6 = e4m3_encode(__fdiv_rn(a, g6));
+            uint32_t c4 = e4m3_encode(__fdiv_rn(a, g4));
+            c6 = c6 == 0u ? 1u : c6;
+            c4 = c4 == 0u ? 1u : c4;
+            float best = quant_sse<B>(xv, bf_tab[c6].x, g_one ? 1.0f : g, bf_tab[c6]);
+            uint32_t bc = c6;
+            if (c4 != c6) {
+                const float s4 = quant_sse<B>(xv, bf_tab[c4].x, g_one ? 1.0f : g, bf_tab[c4]);
+                if (s4 < best || (s4 == best && c4 < bc)) {
+                    best = s4;
+                    bc = c4;
+                }
+            }
+            // first all-zero code (127 = none)
+            uint32_t lo = 1u, hi = 127u;
+            while (lo < hi) {
+                const uint32_t mid = (lo + hi) >> 1;
+                if (__fmul_rn(a, bf_tab[mid].y) <= 0.25f)
+                    hi = mid;
+                else
+                    lo = mid + 1u;
+            }
+            const uint32_t cz = lo;
+            if (cz < 127u && (sse0 < best || (sse0 == best && cz < bc))) {
+                best = sse0;
+                bc = cz;
+            }
+            // downward: codes below c6 while the clipped bound can still win
+            uint32_t clo = c6;
+            while (clo > 1u) {
+                const float2 t = bf_tab[clo - 1u];
+                const float em = elem_err(a, t.x, t.y);
+                if (__fmul_rn(em, em) > best)
+                    break;
+                --clo;
+            }
+            const uint32_t chi = (cz < 127u ? cz : 127u) - 1u;   // last code to evaluate
+            const int span = valid ? (int)chi - (int)clo + 1 : 0;
+            const int wspan = __reduce_max_sync(0xffffffffu, span > 0 ? span : 0);
+            for (int it = 0; it < wspan; ++it) {
+                const uint32_t c = clo + (uint32_t)it;
+                if (it < span && c != c6 && c != c4) {
+                    const float2 t = bf_tab[c];
+                    const float em = elem_err(a, t.x, t.y);
+                    const float lb = __fmul_rn(em, em);
+                    if (lb < best || (lb == best && c < bc)) {
+                        const float sc_ = quant_sse<B>(xv, t.x, g_one ? 1.0f : g, t);
+                        if (sc_ < best || (sc_ == best && c < bc)) {
+                            best = sc_;
                             bc = c;
-                        }
-                    } else if (c != c0) {
-                        const float em = elem_err(a, S, inv);
-                        const float lb = __fmul_rn(em, em);
-                        if (lb < best || (lb == best && c < bc)) {
-                            const float s = quant_sse<B>(xv, scv, g);
-                            if (s < best || (s == best && c < bc)) {
-                                best = s;
-                                bc = c;
-                            }
                         }
                     }
                 }
-                if (__all_sync(0xffffffffu, done))
-                    break;
             }
             sc = bc;
             sse = quant_eval<B>(xv, e4m3_decode(bc), g, cw, dq);
@@ -291,14 +381,26 @@ nvfp4_quant_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs
 
 // ------------------------------------------------------------------ RaZeR
 struct SpecialArgs {
-    float v[4];
+    float v[4];        // table in order
     int n;
+    float mag[4];      // distinct magnitudes |v|
+    int nmag;
+    int mag_of[4];     // magnitude index of each table entry
+    int neg[4];        // 1 if the table entry is negative
 };
 
 // SF = 0: E4M3 scale, selector in bit 7 (activations); SF = 1: E3M3 scale,
 // selector in bits 7..6 (weights).  Block size 16.
+//
+// Per block: the plain E2M1 error e_i of every element is computed once.  For
+// each distinct special magnitude a 16-bit mask marks the elements that are
+// not zero-coded and for which that magnitude is strictly nearer than their
+// grid neighbour; a signed table entry takes the elements of its magnitude
+// mask whose sign matches.  Its in-order fma error chain then uses
+// RN(|x| - RN(|v| S)) at the masked positions (the square equals that of
+// x - RN(v S) for a same-signed v) and e_i elsewhere.
 template <typename T, int SF>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 3)
 razer_quant_kernel(const T* __restrict__ x, int64_t nblk, GsArgs gs, SpecialArgs sp,
                    uint8_t* __restrict__ codes, uint8_t* __restrict__ meta,
                    float* __restrict__ deq, float* __restrict__ mse)
@@ -331,9 +433,11 @@ razer_quant_kernel(const T* __restrict__ x, int64_t nblk, GsArgs gs, SpecialArgs
         const float S = __fmul_rn(scv, g);
         const float inv = (S == 0.0f) ? 0.0f : fminf(__frcp_rn(S), kFltMax);
 
-        // plain E2M1 quantization of every element
-        float ay[B], vs[B], dstd[B];
+        // plain E2M1 quantization, its errors and the per-magnitude masks
+        float e[B];
         uint32_t cw[2];
+        uint32_t negm = 0u, zerom = 0u;
+        uint32_t magm[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
             float y[8];
@@ -345,63 +449,82 @@ razer_quant_kernel(const T* __restrict__ x, int64_t nblk, GsArgs gs, SpecialArgs
             e2m1x8_decode(cw[j], v);
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                ay[8 * j + i] = fabsf(y[i]);
-                vs[8 * j + i] = v[i];
-                dstd[8 * j + i] = __fmul_rn(v[i], S);
+                const int idx = 8 * j + i;
+                e[idx] = __fsub_rn(xv[idx], __fmul_rn(v[i], S));
+                const float ay = fabsf(y[i]);
+                const float dg = fabsf(__fsub_rn(ay, fabsf(v[i])));
+                const bool nz = v[i] != 0.0f;
+                negm |= (uint32_t)signbit(y[i]) << idx;
+                zerom |= (uint32_t)(!nz) << idx;
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    if (k < sp.nmag) {
+                        const bool near = nz && (fabsf(__fsub_rn(ay, sp.mag[k])) < dg);
+                        magm[k] |= (uint32_t)near << idx;
+                    }
+                }
             }
         }
-        // score each special value in table order
+        // score each table entry in order; strict < keeps the earliest minimum
         float best = 0.0f;
         int sel = 0;
+        uint32_t best_mask = 0u;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             if (k >= sp.n)
                 break;
-            const float spv = sp.v[k];
-            const float spa = fabsf(spv);
-            const bool spneg = signbit(spv);
-            const float dsp = __fmul_rn(spv, S);
+            const int mi = sp.mag_of[k];
+            const uint32_t mm = mi == 0 ? magm[0] : mi == 1 ? magm[1] : mi == 2 ? magm[2] : magm[3];
+            const uint32_t use = mm & (sp.neg[k] ? negm : ~negm);
+            const float D = __fmul_rn(sp.mag[mi == 0 ? 0 : mi == 1 ? 1 : mi == 2 ? 2 : 3], S);
             float acc = 0.0f;
 #pragma unroll
             for (int i = 0; i < B; ++i) {
-                const uint32_t code = (cw[i >> 3] >> (4 * (i & 7))) & 0xFu;
-                const bool nz = (code & 7u) != 0u;
-                const bool neg = (code & 8u) != 0u;
-                const float dg = fabsf(__fsub_rn(ay[i], fabsf(vs[i])));
-                const float ds = fabsf(__fsub_rn(ay[i], spa));
-                const bool use = nz && (neg == spneg) && (ds < dg);
-                const float e = __fsub_rn(xv[i], use ? dsp : dstd[i]);
-                acc = __fmaf_rn(e, e, acc);
+                const float es = __fsub_rn(fabsf(xv[i]), D);
+                const float ei = ((use >> i) & 1u) ? es : e[i];
+                acc = __fmaf_rn(ei, ei, acc);
             }
             if (k == 0 || acc < best) {
                 best = acc;
                 sel = k;
+                best_mask = use;
             }
         }
-        // outputs for the chosen special
-        const float spv = sel == 0 ? sp.v[0] : sel == 1 ? sp.v[1] : sel == 2 ? sp.v[2] : sp.v[3];
-        const float spa = fabsf(spv);
-        const bool spneg = signbit(spv);
-        const float dsp = __fmul_rn(spv, S);
-        float dq[B];
-        uint32_t ow[2] = {0u, 0u};
-#pragma unroll
-        for (int i = 0; i < B; ++i) {
-            const uint32_t code = (cw[i >> 3] >> (4 * (i & 7))) & 0xFu;
-            const bool nz = (code & 7u) != 0u;
-            const bool neg = (code & 8u) != 0u;
-            const float dg = fabsf(__fsub_rn(ay[i], fabsf(vs[i])));
-            const float ds = fabsf(__fsub_rn(ay[i], spa));
-            const bool use = nz && (neg == spneg) && (ds < dg);
-            const uint32_t oc = !nz ? 0u : (use ? 8u : code);
-            dq[i] = !nz ? 0.0f : (use ? dsp : dstd[i]);
-            ow[i >> 3] |= oc << (4 * (i & 7));
-        }
         if (valid) {
+            // codes: zero-coded elements take +0, the chosen elements the -0 code
+            uint32_t ow[2];
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                uint32_t w = cw[j];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int idx = 8 * j + i;
+                    const uint32_t clr = ((zerom >> idx) & 1u) | ((best_mask >> idx) & 1u);
+                    w &= ~(clr * (0xFu << (4 * i)));
+                    w |= ((best_mask >> idx) & 1u) << (4 * i + 3);
+                }
+                ow[j] = w;
+            }
             *reinterpret_cast<uint2*>(codes + b * 8) = make_uint2(ow[0], ow[1]);
             meta[b] = (uint8_t)(SF == 1 ? ((uint32_t)sel << 6) | scc : ((uint32_t)sel << 7) | scc);
-            if (deq)
+            if (deq) {
+                // dequantized values from the final codes: the chosen special at
+                // its positions, v * S (+0 for zero codes) elsewhere
+                const float spv = sel == 0 ? sp.v[0] : sel == 1 ? sp.v[1] : sel == 2 ? sp.v[2] : sp.v[3];
+                const float dsp = __fmul_rn(spv, S);
+                float dq[B];
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    float vv[8];
+                    e2m1x8_decode(ow[j], vv);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int idx = 8 * j + i;
+                        dq[idx] = ((best_mask >> idx) & 1u) ? dsp : __fmul_rn(vv[i], S);
+                    }
+                }
                 store_f32<B>(deq + b * B, dq);
+            }
             if (mse)
                 mse[b] = __fmul_rn(best, 1.0f / 16.0f);
         }
@@ -622,8 +745,18 @@ cudaError_t launch_razer_quant(const void* x, int dtype, int64_t rows, int64_t c
                                cudaStream_t s)
 {
     SpecialArgs sp{};
-    for (int i = 0; i < n_special && i < 4; ++i)
-        sp.v[i] = specials_host[i];
+    for (int i = 0; i < n_special && i < 4; ++i) {
+        const float v = specials_host[i];
+        const float m = v < 0.0f ? -v : v;
+        sp.v[i] = v;
+        sp.neg[i] = v < 0.0f;
+        int mi = 0;
+        while (mi < sp.nmag && sp.mag[mi] != m)
+            ++mi;
+        if (mi == sp.nmag)
+            sp.mag[sp.nmag++] = m;
+        sp.mag_of[i] = mi;
+    }
     sp.n = n_special;
     const int64_t nblk = rows * (cols / 16);
     if (dtype == 1) {
