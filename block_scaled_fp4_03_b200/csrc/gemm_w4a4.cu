@@ -507,6 +507,22 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t sr
                  : "memory");
 }
 
+// Write 32 bf16 columns (chunk c of 8 across the 256-column row half-pair)
+// of row `lane` into the epilogue staging: box (c/2)%2 holds columns
+// [64 (c/2 % 2), +64) of a 128-column half; row `lane` of a box is 128 bytes
+// whose 16-byte chunks sit at (chunk ^ (row % 8)), the 128-byte swizzle the
+// output tensor map expects.
+__device__ __forceinline__ void stage_row_chunk(uint8_t* stg, int c, int lane, const uint32_t (&h)[16])
+{
+    uint8_t* rowp = stg + ((c >> 1) & 1) * 4096 + lane * 128;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const int chunk = (c & 1) * 4 + j;
+        *reinterpret_cast<uint4*>(rowp + ((chunk ^ (lane & 7)) << 4)) =
+            make_uint4(h[4 * j], h[4 * j + 1], h[4 * j + 2], h[4 * j + 3]);
+    }
+}
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 w4a4_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
@@ -699,55 +715,54 @@ w4a4_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                 break;
             }
             tc_fence_after();
+            const int mt = tile % p.tiles_m;
+            const int nt = tile / p.tiles_m;
+            const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16);
             // the previous tile's stores have finished reading the staging buffer
             if (lane == 0)
                 asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
             __syncwarp();
-            const int mt = tile % p.tiles_m;
-            const int nt = tile / p.tiles_m;
-            const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16);
-#pragma unroll 1
+            // columns [0, 128) of the accumulator row go to the staging buffer,
+            // columns [128, 256) stay in registers as bf16: the accumulator
+            // goes back to the MMA issuer before any store is waited for
+            uint32_t pk[4][16];
+#pragma unroll
             for (int c = 0; c < 8; ++c) {
-                if (c == 4) {
-                    // second half of the row: reuse the staging buffer once the
-                    // first half's stores have read it
-                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                    __syncwarp();
-                    if (lane == 0) {
-                        const int y = mt * 256 + (int)rank * 128 + q * 32;
-                        tma_store_2d(&tmOut, smem_u32(stg), nt * 256, y);
-                        tma_store_2d(&tmOut, smem_u32(stg + 4096), nt * 256 + 64, y);
-                        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-                        asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-                    }
-                    __syncwarp();
-                }
                 uint32_t r[32];
                 tmem_ld32(tq + 32 * c, r);
-                uint32_t pk[16];
+                uint32_t h16[16];
 #pragma unroll
                 for (int j = 0; j < 16; ++j) {
                     __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[2 * j]), scale),
                                                              __fmul_rn(__uint_as_float(r[2 * j + 1]), scale));
-                    pk[j] = *reinterpret_cast<uint32_t*>(&h);
+                    h16[j] = *reinterpret_cast<uint32_t*>(&h);
                 }
-                // box (c/2)%2 of the staging holds columns [64 (c/2), +64); row
-                // `lane` of a box is 128 bytes whose 16-byte chunks sit at
-                // (chunk ^ (row % 8))
-                uint8_t* rowp = stg + ((c >> 1) & 1) * 4096 + lane * 128;
+                if (c < 4) {
+                    stage_row_chunk(stg, c, lane, h16);
+                } else {
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int chunk = (c & 1) * 4 + j;
-                    *reinterpret_cast<uint4*>(rowp + ((chunk ^ (lane & 7)) << 4)) =
-                        make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
+                    for (int j = 0; j < 16; ++j)
+                        pk[c - 4][j] = h16[j];
                 }
             }
             tc_fence_before();
             mbar_arrive_cluster(leader_acc_empty);
+            const int y = mt * 256 + (int)rank * 128 + q * 32;
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             __syncwarp();
             if (lane == 0) {
-                const int y = mt * 256 + (int)rank * 128 + q * 32;
+                tma_store_2d(&tmOut, smem_u32(stg), nt * 256, y);
+                tma_store_2d(&tmOut, smem_u32(stg + 4096), nt * 256 + 64, y);
+                asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+                asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+            }
+            __syncwarp();
+#pragma unroll
+            for (int c = 4; c < 8; ++c)
+                stage_row_chunk(stg, c, lane, pk[c - 4]);
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) {
                 tma_store_2d(&tmOut, smem_u32(stg), nt * 256 + 128, y);
                 tma_store_2d(&tmOut, smem_u32(stg + 4096), nt * 256 + 192, y);
                 asm volatile("cp.async.bulk.commit_group;" ::: "memory");

@@ -109,32 +109,127 @@ __device__ __forceinline__ void load32(const T* __restrict__ p, float (&u)[32])
 }
 
 // ------------------------------------------------- OCP exponent (activations)
+// One lane per 32-block, but the loads are cooperative: a warp reads its 32
+// consecutive blocks (and their 32 channel-scale slices) as whole 512-byte
+// rows, parks them in shared memory, and each lane reads its own block back.
+// A lane reading 64-128 contiguous bytes straight from global memory would
+// touch 16-32 cache lines per warp instruction; the L1 would then serve many
+// times the wavefronts the bytes need and cap the kernel far below HBM rate.
+// Shared-memory slots are XOR-swizzled so that both the row-wise stores and
+// the block-wise loads are free of bank conflicts.
+constexpr int kMxWarps = kThreads / 32;
+
+__device__ __forceinline__ uint4 ldg_stream(const uint4* p)
+{
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+// slot of 16-byte chunk p of block i, CPB chunks per block (8 or 4)
+template <int CPB>
+__device__ __forceinline__ int mx_slot(int i, int p)
+{
+    if constexpr (CPB == 8)
+        return i * 8 + (p ^ (i & 7));
+    else
+        return i * 4 + (p ^ ((i >> 1) & 3));
+}
+
 // ERR: also produce the dequantized values / block errors (only when asked).
 template <typename T, bool ERR>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 2)
 mx_quant_absmax_kernel(const T* __restrict__ x, uint32_t nblk, uint32_t kb,
                        const float* __restrict__ t, int had, uint8_t* __restrict__ codes,
                        uint8_t* __restrict__ scales, float* __restrict__ deq,
                        float* __restrict__ mse)
 {
-    const uint32_t stride = gridDim.x * blockDim.x;
-    for (uint32_t b = blockIdx.x * blockDim.x + threadIdx.x; b < nblk; b += stride) {
+    constexpr int CPB = 32 * (int)sizeof(T) / 16;   // 16-byte chunks per block
+    // one 4 KB buffer per warp: first the warp's blocks, then their t slices
+    __shared__ uint4 buf[kMxWarps][32 * 8];
+    const int lane = threadIdx.x & 31;
+    const int w = threadIdx.x >> 5;
+    uint4* bw = buf[w];
+    const uint64_t warp0 = ((uint64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const uint64_t nwarps = ((uint64_t)gridDim.x * blockDim.x) >> 5;
+    for (uint64_t base = warp0 * 32; base < nblk; base += nwarps * 32) {
+        const uint32_t nb = (uint32_t)((nblk - base) < 32 ? (nblk - base) : 32);
+        const uint4* src = reinterpret_cast<const uint4*>(x + base * 32);
+        {
+            uint4 v[CPB];
+#pragma unroll
+            for (int k = 0; k < CPB; ++k) {
+                const int c = lane + 32 * k;
+                v[k] = (uint32_t)(c / CPB) < nb ? ldg_stream(src + c) : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int k = 0; k < CPB; ++k) {
+                const int c = lane + 32 * k;
+                bw[mx_slot<CPB>(c / CPB, c % CPB)] = v[k];
+            }
+        }
+        __syncwarp();
         float u[32];
-        load32<T>(x + (size_t)b * 32, u);
-        online_transform(u, t ? t + (b % kb) * 32 : nullptr, had != 0);
+#pragma unroll
+        for (int p = 0; p < CPB; ++p) {
+            const uint4 q = bw[mx_slot<CPB>(lane, p)];
+            if constexpr (CPB == 8) {
+                u[4 * p] = __uint_as_float(q.x);
+                u[4 * p + 1] = __uint_as_float(q.y);
+                u[4 * p + 2] = __uint_as_float(q.z);
+                u[4 * p + 3] = __uint_as_float(q.w);
+            } else {
+                bf16x2_to_f32(q.x, u[8 * p], u[8 * p + 1]);
+                bf16x2_to_f32(q.y, u[8 * p + 2], u[8 * p + 3]);
+                bf16x2_to_f32(q.z, u[8 * p + 4], u[8 * p + 5]);
+                bf16x2_to_f32(q.w, u[8 * p + 6], u[8 * p + 7]);
+            }
+        }
+        if (t) {
+            const uint32_t kb0 = (uint32_t)(base % kb);
+            uint4 tv[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const int c = lane + 32 * k;
+                const uint32_t kbi = (kb0 + (uint32_t)(c >> 3)) % kb;
+                tv[k] = __ldg(reinterpret_cast<const uint4*>(t + (size_t)kbi * 32) + (c & 7));
+            }
+            __syncwarp();   // every lane has read its block
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const int c = lane + 32 * k;
+                bw[mx_slot<8>(c >> 3, c & 7)] = tv[k];
+            }
+            __syncwarp();
+#pragma unroll
+            for (int p = 0; p < 8; ++p) {
+                const uint4 q = bw[mx_slot<8>(lane, p)];
+                u[4 * p] = __fmul_rn(u[4 * p], __uint_as_float(q.x));
+                u[4 * p + 1] = __fmul_rn(u[4 * p + 1], __uint_as_float(q.y));
+                u[4 * p + 2] = __fmul_rn(u[4 * p + 2], __uint_as_float(q.z));
+                u[4 * p + 3] = __fmul_rn(u[4 * p + 3], __uint_as_float(q.w));
+            }
+        }
+        __syncwarp();   // the buffers are refilled next iteration
+        online_transform(u, nullptr, had != 0);
         float a = 0.0f;
 #pragma unroll
         for (int i = 0; i < 32; ++i)
             a = fmaxf(a, fabsf(u[i]));
         const int e = mx_exponent(a);
         uint32_t cw[4];
+        const uint64_t b = base + (uint64_t)lane;
         if constexpr (ERR) {
             float dq[32];
             const float sse = mx_eval(u, e, cw, dq);
-            if (deq)
-                store_f32<32>(deq + (size_t)b * 32, dq);
-            if (mse)
-                mse[b] = __fmul_rn(sse, 1.0f / 32.0f);
+            if ((uint32_t)lane < nb) {
+                if (deq)
+                    store_f32<32>(deq + b * 32, dq);
+                if (mse)
+                    mse[b] = __fmul_rn(sse, 1.0f / 32.0f);
+            }
         } else {
             const float down = pow2f(-e);
 #pragma unroll
@@ -146,21 +241,18 @@ mx_quant_absmax_kernel(const T* __restrict__ x, uint32_t nblk, uint32_t kb,
                                       __fmul_rn(u[o + 6], down), __fmul_rn(u[o + 7], down));
             }
         }
-        *reinterpret_cast<uint4*>(codes + (size_t)b * 16) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-        scales[b] = (uint8_t)(e + 127);
+        if ((uint32_t)lane < nb) {
+            *reinterpret_cast<uint4*>(codes + b * 16) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+            scales[b] = (uint8_t)(e + 127);
+        }
     }
 }
 
-// d^T H d for the block error d = u - deq(u, e): v_i = sum_j H_ij d_j and the
-// outer sum, each accumulated with fma in index order.  Ht holds H transposed
-// (row j of Ht = column j of H, one 128-byte broadcast read); ds is this
-// thread's slice of a [32][kThreads] shared buffer through which d_j is read
-// inside a rolled j loop, keeping one H row in flight at a time.
-__device__ __forceinline__ float hess_cost(const float (&u)[32], int e, const float* Ht, float* ds)
+// Block error d = u - deq(u, e) at exponent e.
+__device__ __forceinline__ void mx_err(const float (&u)[32], int e, float (&d)[32])
 {
     const float down = pow2f(-e);
     const float up = pow2f(e);
-    float d[32];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
         const int o = 8 * j;
@@ -171,51 +263,31 @@ __device__ __forceinline__ float hess_cost(const float (&u)[32], int e, const fl
         float v[8];
         e2m1x8_decode(w, v);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
+        for (int i = 0; i < 8; ++i)
             d[o + i] = __fsub_rn(u[o + i], __fmul_rn(v[i], up));
-            ds[(o + i) * kThreads] = d[o + i];
-        }
     }
-    float v[32];
-#pragma unroll
-    for (int i = 0; i < 32; ++i)
-        v[i] = 0.0f;
-#pragma unroll 1
-    for (int j = 0; j < 32; ++j) {
-        const float dj = ds[j * kThreads];
-#pragma unroll
-        for (int i = 0; i < 32; i += 4) {
-            const float4 h = *reinterpret_cast<const float4*>(&Ht[j * 32 + i]);
-            v[i] = __fmaf_rn(h.x, dj, v[i]);
-            v[i + 1] = __fmaf_rn(h.y, dj, v[i + 1]);
-            v[i + 2] = __fmaf_rn(h.z, dj, v[i + 2]);
-            v[i + 3] = __fmaf_rn(h.w, dj, v[i + 3]);
-        }
-    }
-    float cost = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 32; ++i)
-        cost = __fmaf_rn(d[i], v[i], cost);
-    return cost;
 }
 
-// --------------------------------------------- Hessian-weighted exponent
-// One CTA = one 32-column block k and kThreads rows; H'_k staged in shared
-// memory and read as broadcasts.  Candidates in the order 0, +1, -1 around
-// the OCP exponent; the winner has the strictly smallest d^T H'_k d with
-// d = u - deq, each product sum accumulated with fma in index order.
+// Hessian-weighted exponent (weights): among e0, e0 + 1, e0 - 1 (in that
+// order, strict improvement only) the exponent with the least d^T H'_k d.
+// For each candidate, v_i = sum_j H_ij d_j is an fma chain over j in order and
+// the cost an fma chain of d_i v_i over i in order.  The three candidates'
+// errors stay in registers and every row of H'_k (one broadcast 128-byte
+// shared-memory read) feeds all three chains, so the kernel runs on the FMA
+// pipe rather than on shared-memory bandwidth.
+constexpr int kHessThreads = 128;
+
 template <typename T>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kHessThreads, 3)
 mx_quant_hessian_kernel(const T* __restrict__ x, int64_t rows, int64_t kb,
                         const float* __restrict__ t, int had, const float* __restrict__ hess,
                         uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
                         float* __restrict__ deq, float* __restrict__ mse)
 {
-    __shared__ __align__(16) float Hs[32 * 32];   // H'_k transposed
-    __shared__ float Ds[32 * kThreads];          // per-thread error staging
+    __shared__ __align__(16) float Hs[32 * 32];   // H'_k, row-major
     const int64_t k = blockIdx.y;
     for (int i = threadIdx.x; i < 32 * 32; i += blockDim.x)
-        Hs[(i & 31) * 32 + (i >> 5)] = __ldg(hess + k * 1024 + i);
+        Hs[i] = __ldg(hess + k * 1024 + i);
     __syncthreads();
     const int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (r >= rows)
@@ -229,18 +301,48 @@ mx_quant_hessian_kernel(const T* __restrict__ x, int64_t rows, int64_t kb,
     for (int i = 0; i < 32; ++i)
         a = fmaxf(a, fabsf(u[i]));
     const int e0 = mx_exponent(a);
-    int best_e = e0;
-    float best = hess_cost(u, e0, Hs, Ds + threadIdx.x);
-#pragma unroll 1
-    for (int o = 1; o < 3; ++o) {
-        const int ec = o == 1 ? e0 + 1 : e0 - 1;
-        if (ec < -127 || ec > 127)
-            continue;
-        const float cost = hess_cost(u, ec, Hs, Ds + threadIdx.x);
-        if (cost < best) {
-            best = cost;
-            best_e = ec;
+    // an exponent outside [-127, 127] is not a candidate; its chain runs on
+    // the e0 error and is ignored
+    const int eu = e0 + 1 <= 127 ? e0 + 1 : e0;
+    const int ed = e0 - 1 >= -127 ? e0 - 1 : e0;
+    float d0[32], d1[32], d2[32];
+    mx_err(u, e0, d0);
+    mx_err(u, eu, d1);
+    mx_err(u, ed, d2);
+    float c0 = 0.0f, c1 = 0.0f, c2 = 0.0f;
+    const float4* H4 = reinterpret_cast<const float4*>(Hs);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        float v0 = 0.0f, v1 = 0.0f, v2 = 0.0f;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const float4 h = H4[i * 8 + q];
+            v0 = __fmaf_rn(h.x, d0[4 * q], v0);
+            v1 = __fmaf_rn(h.x, d1[4 * q], v1);
+            v2 = __fmaf_rn(h.x, d2[4 * q], v2);
+            v0 = __fmaf_rn(h.y, d0[4 * q + 1], v0);
+            v1 = __fmaf_rn(h.y, d1[4 * q + 1], v1);
+            v2 = __fmaf_rn(h.y, d2[4 * q + 1], v2);
+            v0 = __fmaf_rn(h.z, d0[4 * q + 2], v0);
+            v1 = __fmaf_rn(h.z, d1[4 * q + 2], v1);
+            v2 = __fmaf_rn(h.z, d2[4 * q + 2], v2);
+            v0 = __fmaf_rn(h.w, d0[4 * q + 3], v0);
+            v1 = __fmaf_rn(h.w, d1[4 * q + 3], v1);
+            v2 = __fmaf_rn(h.w, d2[4 * q + 3], v2);
         }
+        c0 = __fmaf_rn(d0[i], v0, c0);
+        c1 = __fmaf_rn(d1[i], v1, c1);
+        c2 = __fmaf_rn(d2[i], v2, c2);
+    }
+    int best_e = e0;
+    float best = c0;
+    if (eu != e0 && c1 < best) {
+        best = c1;
+        best_e = eu;
+    }
+    if (ed != e0 && c2 < best) {
+        best = c2;
+        best_e = ed;
     }
     uint32_t cw[4];
     float dq[32];
@@ -353,7 +455,7 @@ hessian_reduce_kernel(const float* __restrict__ part, int64_t nchunk, int64_t to
 // Column statistics in fp64 over a chunk of rows: sum and sum of squares.
 // One thread owns 8 consecutive columns (one 16-byte bf16 vector or two fp32
 // vectors) for every row of the chunk.
-constexpr int kStatRows = 32;
+constexpr int kStatRows = 64;
 
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
@@ -371,7 +473,25 @@ column_stats_kernel(const T* __restrict__ x, int64_t rows, int64_t cols, double*
         s[i] = 0.0;
         q[i] = 0.0;
     }
-    for (int64_t r = r0; r < r1; ++r) {
+    // rows in groups of 8 with all 8 loads issued before the sums, so each
+    // thread keeps 8 vectors in flight
+    int64_t r = r0;
+    for (; r + 8 <= r1; r += 8) {
+        float v[8][8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            load_elems<T, 8>(x + (r + k) * cols + c0, v[k]);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const double d = (double)v[k][i];
+                s[i] += d;
+                q[i] = fma(d, d, q[i]);
+            }
+        }
+    }
+    for (; r < r1; ++r) {
         float v[8];
         load_elems<T, 8>(x + r * cols + c0, v);
 #pragma unroll
@@ -391,23 +511,45 @@ column_stats_kernel(const T* __restrict__ x, int64_t rows, int64_t cols, double*
 }
 
 // t_j = (sigma_j^W / rms_j^X)^alpha, t = 1 where a factor is zero; fp64, then
-// rounded to fp32; t_inv = 1/t in fp32.
+// rounded to fp32; t_inv = 1/t in fp32.  A CTA owns 32 columns; its 8 warps
+// split the chunk partials (warp w sums chunks w, w + 8, ...), then one warp
+// adds the 8 slices in a fixed order.
+constexpr int kScaleSlices = kThreads / 32;
+
 __global__ void __launch_bounds__(kThreads)
 channel_scale_kernel(const double* __restrict__ wsum, const double* __restrict__ wsq,
                      int64_t wchunks, int64_t n_out, const double* __restrict__ xsq,
                      int64_t xchunks, int64_t tokens, int64_t cols, double alpha,
                      float* __restrict__ t, float* __restrict__ t_inv)
 {
-    const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (j >= cols)
-        return;
+    __shared__ double red[3][kScaleSlices][32];
+    const int lane = threadIdx.x & 31;
+    const int slice = threadIdx.x >> 5;
+    const int64_t j = (int64_t)blockIdx.x * 32 + lane;
     double s = 0.0, q = 0.0, h = 0.0;
-    for (int64_t c = 0; c < wchunks; ++c) {
-        s += wsum[c * cols + j];
-        q += wsq[c * cols + j];
+    if (j < cols) {
+        for (int64_t c = slice; c < wchunks; c += kScaleSlices) {
+            s += __ldg(wsum + c * cols + j);
+            q += __ldg(wsq + c * cols + j);
+        }
+        for (int64_t c = slice; c < xchunks; c += kScaleSlices)
+            h += __ldg(xsq + c * cols + j);
     }
-    for (int64_t c = 0; c < xchunks; ++c)
-        h += xsq[c * cols + j];
+    red[0][slice][lane] = s;
+    red[1][slice][lane] = q;
+    red[2][slice][lane] = h;
+    __syncthreads();
+    if (slice != 0 || j >= cols)
+        return;
+    s = red[0][0][lane];
+    q = red[1][0][lane];
+    h = red[2][0][lane];
+#pragma unroll
+    for (int k = 1; k < kScaleSlices; ++k) {
+        s += red[0][k][lane];
+        q += red[1][k][lane];
+        h += red[2][k][lane];
+    }
     const double n = (double)n_out;
     const double mean = s / n;
     double var = q / n - mean * mean;
@@ -458,13 +600,13 @@ cudaError_t launch_mxfp4_quant(const void* x, int dtype, int64_t rows, int64_t c
     const int64_t kb = cols / 32;
     const int64_t nblk = rows * kb;
     if (rule == 4) {
-        dim3 grid((unsigned)((rows + kThreads - 1) / kThreads), (unsigned)kb);
+        dim3 grid((unsigned)((rows + kHessThreads - 1) / kHessThreads), (unsigned)kb);
         if (dtype == 1)
-            mx_quant_hessian_kernel<__nv_bfloat16><<<grid, kThreads, 0, s>>>(
+            mx_quant_hessian_kernel<__nv_bfloat16><<<grid, kHessThreads, 0, s>>>(
                 reinterpret_cast<const __nv_bfloat16*>(x), rows, kb, chan_scale, hadamard, hess,
                 codes, scales, deq, mse);
         else
-            mx_quant_hessian_kernel<float><<<grid, kThreads, 0, s>>>(
+            mx_quant_hessian_kernel<float><<<grid, kHessThreads, 0, s>>>(
                 reinterpret_cast<const float*>(x), rows, kb, chan_scale, hadamard, hess, codes,
                 scales, deq, mse);
         return cudaGetLastError();
@@ -534,7 +676,7 @@ cudaError_t launch_mx_channel_scale(const void* x, int xdt, int64_t tokens, cons
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess)
         return e;
-    channel_scale_kernel<<<(unsigned)((cols + kThreads - 1) / kThreads), kThreads, 0, s>>>(
+    channel_scale_kernel<<<(unsigned)((cols + 31) / 32), kThreads, 0, s>>>(
         wsum, wsq, wch, n_out, xsq, xch, tokens, cols, (double)alpha, t, t_inv);
     return cudaGetLastError();
 }

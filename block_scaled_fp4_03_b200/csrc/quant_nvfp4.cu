@@ -226,6 +226,7 @@ __device__ __forceinline__ float elem_err(float a, float S, float inv)
 
 enum { R_ABSMAX = 0, R_PZ = 1, R_46 = 2, R_BF = 3 };
 
+// Abs-max, prevent-zero and 4-over-6 (brute force has its own kernel below).
 template <int B, typename T, int RULE>
 __global__ void __launch_bounds__(kThreads)
 nvfp4_quant_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs,
@@ -239,16 +240,16 @@ nvfp4_quant_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs
     const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
     const int64_t kb_atoms = (bpr + 3) >> 2;
-    // brute force: every code's effective scale S = sc * g and reciprocal
-    // inv = min(1/S, FLT_MAX) (0 for S = 0), computed once per CTA
-    __shared__ float2 bf_tab[128];
-    const bool g_one = g == 1.0f;
-    if constexpr (RULE == R_BF) {
-        for (int c = threadIdx.x; c < 128; c += blockDim.x) {
-            const float S = __fmul_rn(e4m3_decode((uint32_t)(c < 127 ? c : 126)), g);
-            bf_tab[c] = make_float2(S, (S == 0.0f) ? 0.0f : fminf(__frcp_rn(S), kFltMax));
-        }
-        __syncthreads();
+    // MMA-layout scale position: (row, k-block) of this lane's block, advanced
+    // by the grid stride without a per-block 64-bit division
+    int64_t r_cur = 0, kb_cur = 0, step_r = 0, step_kb = 0;
+    if (mma_layout) {
+        const int64_t b0 = warp0 * 32 + lane;
+        const int64_t step = nwarps * 32;
+        r_cur = b0 / bpr;
+        kb_cur = b0 % bpr;
+        step_r = step / bpr;
+        step_kb = step % bpr;
     }
 
     for (int64_t base = warp0 * 32; base < nblk; base += nwarps * 32) {
@@ -292,89 +293,24 @@ nvfp4_quant_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs
 #pragma unroll
             for (int i = 0; i < B; ++i)
                 dq[i] = take4 ? dq4[i] : dq[i];
-        } else {
-            // Brute force over E4M3 codes 1..126: the least error, ties to the
-            // lowest code.  Exact shortcuts (each provably skips only losers):
-            //  * from the first code at which the largest element rounds to
-            //    zero (|y| <= 0.25, found by bisection: |y| falls as the code
-            //    grows) every element does, so that code gives the all-zero
-            //    error and every higher code ties it with a higher code;
-            //  * below the abs-max code the largest element clips to 6, its
-            //    error a - 6S grows as the code falls, and its square alone
-            //    bounds the in-order fma chain from below: the downward scan
-            //    stops at the first code whose bound already loses;
-            //  * in between, the same single-element bound skips candidates.
-            // Each lane walks its own range, so lanes of a warp stay busy.
-            float sse0 = 0.0f;
-#pragma unroll
-            for (int i = 0; i < B; ++i)
-                sse0 = __fmaf_rn(xv[i], xv[i], sse0);
-            uint32_t c6 = e4m3_encode(__fdiv_rn(a, g6));
-            uint32_t c4 = e4m3_encode(__fdiv_rn(a, g4));
-            c6 = c6 == 0u ? 1u : c6;
-            c4 = c4 == 0u ? 1u : c4;
-            float best = quant_sse<B>(xv, bf_tab[c6].x, g_one ? 1.0f : g, bf_tab[c6]);
-            uint32_t bc = c6;
-            if (c4 != c6) {
-                const float s4 = quant_sse<B>(xv, bf_tab[c4].x, g_one ? 1.0f : g, bf_tab[c4]);
-                if (s4 < best || (s4 == best && c4 < bc)) {
-                    best = s4;
-                    bc = c4;
-                }
-            }
-            // first all-zero code (127 = none)
-            uint32_t lo = 1u, hi = 127u;
-            while (lo < hi) {
-                const uint32_t mid = (lo + hi) >> 1;
-                if (__fmul_rn(a, bf_tab[mid].y) <= 0.25f)
-                    hi = mid;
-                else
-                    lo = mid + 1u;
-            }
-            const uint32_t cz = lo;
-            if (cz < 127u && (sse0 < best || (sse0 == best && cz < bc))) {
-                best = sse0;
-                bc = cz;
-            }
-            // downward: codes below c6 while the clipped bound can still win
-            uint32_t clo = c6;
-            while (clo > 1u) {
-                const float2 t = bf_tab[clo - 1u];
-                const float em = elem_err(a, t.x, t.y);
-                if (__fmul_rn(em, em) > best)
-                    break;
-                --clo;
-            }
-            const uint32_t chi = (cz < 127u ? cz : 127u) - 1u;   // last code to evaluate
-            const int span = valid ? (int)chi - (int)clo + 1 : 0;
-            const int wspan = __reduce_max_sync(0xffffffffu, span > 0 ? span : 0);
-            for (int it = 0; it < wspan; ++it) {
-                const uint32_t c = clo + (uint32_t)it;
-                if (it < span && c != c6 && c != c4) {
-                    const float2 t = bf_tab[c];
-                    const float em = elem_err(a, t.x, t.y);
-                    const float lb = __fmul_rn(em, em);
-                    if (lb < best || (lb == best && c < bc)) {
-                        const float sc_ = quant_sse<B>(xv, t.x, g_one ? 1.0f : g, t);
-                        if (sc_ < best || (sc_ == best && c < bc)) {
-                            best = sc_;
-                            bc = c;
-                        }
-                    }
-                }
-            }
-            sc = bc;
-            sse = quant_eval<B>(xv, e4m3_decode(bc), g, cw, dq);
         }
 
         if (valid) {
             store_codes<B>(codes + b * (B / 2), cw);
-            const int64_t so = mma_layout ? mma_sf_offset(b / bpr, b % bpr, kb_atoms) : b;
+            const int64_t so = mma_layout ? mma_sf_offset(r_cur, kb_cur, kb_atoms) : b;
             scales[so] = (uint8_t)sc;
             if (deq)
                 store_f32<B>(deq + b * B, dq);
             if (mse)
                 mse[b] = __fmul_rn(sse, 1.0f / (float)B);
+        }
+        if (mma_layout) {
+            kb_cur += step_kb;
+            r_cur += step_r;
+            if (kb_cur >= bpr) {
+                kb_cur -= bpr;
+                ++r_cur;
+            }
         }
     }
 }
@@ -531,6 +467,385 @@ razer_quant_kernel(const T* __restrict__ x, int64_t nblk, GsArgs gs, SpecialArgs
     }
 }
 
+// Paired tables (+v0, -v0, +v1, -v1, ...), NPAIR pairs, v > 0.  An element
+// can only take the table entry whose sign matches its own (its grid value v
+// is then nonzero with that sign), so with d = |y - v|:
+//   +m candidate: special iff v > 0 and |y - m| < d
+//   -m candidate: special iff v < 0 and |y + m| < d
+// (|y -/+ m| is the |(|y|) - m| of the general rule, written without |y|).
+// Each candidate's in-order fma chain takes either the grid error e or the
+// special error es; the choice is a predicated fma pair on the FMA pipe
+// rather than a select on the integer pipe, and the element's bit enters
+// that candidate's mask under the same predicate.
+// One pair's two candidates; operands: %0/%1 the +/- chains, %2/%3 their
+// masks, %4 y, %5 e, %6 m, %7 es, %8 the element's bit; d, pp, pn shared.
+#define FP4Q_RAZER_PAIR_PTX(A0, A1, M0, M1, Y, E, MAG, ES, BIT)        \
+    "sub.rn.f32 t, " Y ", " MAG ";\n\t"                                \
+    "abs.f32 t, t;\n\t"                                                \
+    "setp.lt.and.f32 q, t, d, pp;\n\t"                                 \
+    "@!q fma.rn.f32 " A0 ", " E ", " E ", " A0 ";\n\t"                 \
+    "@q fma.rn.f32 " A0 ", " ES ", " ES ", " A0 ";\n\t"                \
+    "@q or.b32 " M0 ", " M0 ", " BIT ";\n\t"                           \
+    "add.rn.f32 t, " Y ", " MAG ";\n\t"                                \
+    "abs.f32 t, t;\n\t"                                                \
+    "setp.lt.and.f32 q, t, d, pn;\n\t"                                 \
+    "@!q fma.rn.f32 " A1 ", " E ", " E ", " A1 ";\n\t"                 \
+    "@q fma.rn.f32 " A1 ", " ES ", " ES ", " A1 ";\n\t"                \
+    "@q or.b32 " M1 ", " M1 ", " BIT ";\n\t"
+
+template <int NPAIR>
+__device__ __forceinline__ void razer_pair_step(float y, float v, float e, const float (&mag)[NPAIR],
+                                                const float (&es)[NPAIR], uint32_t bit,
+                                                float (&acc)[2 * NPAIR], uint32_t (&mask)[2 * NPAIR])
+{
+    static_assert(NPAIR == 1 || NPAIR == 2, "one or two pairs");
+    if constexpr (NPAIR == 1) {
+        asm("{\n\t"
+            ".reg .pred pp, pn, q;\n\t"
+            ".reg .f32 d, t;\n\t"
+            "setp.gt.f32 pp, %5, 0f00000000;\n\t"
+            "setp.lt.f32 pn, %5, 0f00000000;\n\t"
+            "sub.rn.f32 d, %4, %5;\n\t"
+            "abs.f32 d, d;\n\t"
+            FP4Q_RAZER_PAIR_PTX("%0", "%1", "%2", "%3", "%4", "%6", "%7", "%8", "%9")
+            "}"
+            : "+f"(acc[0]), "+f"(acc[1]), "+r"(mask[0]), "+r"(mask[1])
+            : "f"(y), "f"(v), "f"(e), "f"(mag[0]), "f"(es[0]), "r"(bit));
+    } else {
+        asm("{\n\t"
+            ".reg .pred pp, pn, q;\n\t"
+            ".reg .f32 d, t;\n\t"
+            "setp.gt.f32 pp, %9, 0f00000000;\n\t"
+            "setp.lt.f32 pn, %9, 0f00000000;\n\t"
+            "sub.rn.f32 d, %8, %9;\n\t"
+            "abs.f32 d, d;\n\t"
+            FP4Q_RAZER_PAIR_PTX("%0", "%1", "%4", "%5", "%8", "%10", "%11", "%13", "%15")
+            FP4Q_RAZER_PAIR_PTX("%2", "%3", "%6", "%7", "%8", "%10", "%12", "%14", "%15")
+            "}"
+            : "+f"(acc[0]), "+f"(acc[1]), "+f"(acc[2]), "+f"(acc[3]), "+r"(mask[0]), "+r"(mask[1]),
+              "+r"(mask[2]), "+r"(mask[3])
+            : "f"(y), "f"(v), "f"(e), "f"(mag[0]), "f"(mag[1]), "f"(es[0]), "f"(es[1]), "r"(bit));
+    }
+}
+#undef FP4Q_RAZER_PAIR_PTX
+
+// Spread the 8 bits of b to bit 0 of the 8 nibbles of a word.
+__device__ __forceinline__ uint32_t spread_bits_to_nibbles(uint32_t b)
+{
+    b = (b | (b << 12)) & 0x000F000Fu;
+    b = (b | (b << 6)) & 0x03030303u;
+    b = (b | (b << 3)) & 0x11111111u;
+    return b;
+}
+
+template <typename T, int SF, int NPAIR>
+__global__ void __launch_bounds__(kThreads, 3)
+razer_paired_kernel(const T* __restrict__ x, int64_t nblk, GsArgs gs, SpecialArgs sp,
+                    uint8_t* __restrict__ codes, uint8_t* __restrict__ meta,
+                    float* __restrict__ deq, float* __restrict__ mse)
+{
+    constexpr int B = 16;
+    const float g = resolve_global_scale(gs);
+    const float g6 = __fmul_rn(6.0f, g);
+    const int lane = threadIdx.x & 31;
+    const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    float mag[NPAIR];
+#pragma unroll
+    for (int m = 0; m < NPAIR; ++m)
+        mag[m] = sp.v[2 * m];
+
+    for (int64_t base = warp0 * 32; base < nblk; base += nwarps * 32) {
+        const int64_t b = base + lane;
+        const bool valid = b < nblk;
+        float xv[B];
+        if (valid) {
+            load_elems<T, B>(x + b * B, xv);
+        } else {
+#pragma unroll
+            for (int i = 0; i < B; ++i)
+                xv[i] = 0.0f;
+        }
+        float a = 0.0f;
+#pragma unroll
+        for (int i = 0; i < B; ++i)
+            a = fmaxf(a, fabsf(xv[i]));
+        const float r = __fdiv_rn(a, g6);
+        const uint32_t scc = SF == 1 ? e3m3_encode(r) : e4m3_encode(r);
+        const float scv = SF == 1 ? e3m3_decode(scc) : e4m3_decode(scc);
+        const float S = __fmul_rn(scv, g);
+        const float inv = (S == 0.0f) ? 0.0f : fminf(__frcp_rn(S), kFltMax);
+        float D[NPAIR];
+#pragma unroll
+        for (int m = 0; m < NPAIR; ++m)
+            D[m] = __fmul_rn(mag[m], S);
+
+        float acc[2 * NPAIR];
+        uint32_t mask[2 * NPAIR];
+#pragma unroll
+        for (int k = 0; k < 2 * NPAIR; ++k) {
+            acc[k] = 0.0f;
+            mask[k] = 0u;
+        }
+        uint32_t cw[2];
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            float y[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                y[i] = __fmul_rn(xv[8 * j + i], inv);
+            cw[j] = e2m1x8_encode(y[0], y[1], y[2], y[3], y[4], y[5], y[6], y[7]);
+            float v[8];
+            e2m1x8_decode(cw[j], v);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int idx = 8 * j + i;
+                const float e = __fsub_rn(xv[idx], __fmul_rn(v[i], S));
+                const float ax = fabsf(xv[idx]);
+                float es[NPAIR];
+#pragma unroll
+                for (int m = 0; m < NPAIR; ++m)
+                    es[m] = __fsub_rn(ax, D[m]);
+                razer_pair_step<NPAIR>(y[i], v[i], e, mag, es, 1u << idx, acc, mask);
+            }
+        }
+        float best = acc[0];
+        int sel = 0;
+#pragma unroll
+        for (int k = 1; k < 2 * NPAIR; ++k) {
+            if (acc[k] < best) {
+                best = acc[k];
+                sel = k;
+            }
+        }
+        if (valid) {
+            uint32_t chosen = mask[0];
+#pragma unroll
+            for (int k = 1; k < 2 * NPAIR; ++k)
+                if (sel == k)
+                    chosen = mask[k];
+            uint32_t ow[2];
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                uint32_t w = cw[j];
+                // -0 (0x8) is the special code: grid zeros take +0
+                const uint32_t t = w ^ 0x88888888u;
+                const uint32_t not8 = (((t & 0x77777777u) + 0x77777777u) | t) & 0x88888888u;
+                w &= ~(~not8 & 0x88888888u);
+                // chosen elements take -0
+                const uint32_t ones = spread_bits_to_nibbles((chosen >> (8 * j)) & 0xFFu);
+                w = (w & ~(ones * 0xFu)) | (ones << 3);
+                ow[j] = w;
+            }
+            *reinterpret_cast<uint2*>(codes + b * 8) = make_uint2(ow[0], ow[1]);
+            meta[b] = (uint8_t)(SF == 1 ? ((uint32_t)sel << 6) | scc : ((uint32_t)sel << 7) | scc);
+            if (deq) {
+                float spv = 0.0f;
+#pragma unroll
+                for (int k = 0; k < 2 * NPAIR; ++k)
+                    if (sel == k)
+                        spv = (k & 1) ? -mag[k >> 1] : mag[k >> 1];
+                const float dsp = __fmul_rn(spv, S);
+                float dq[B];
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    float vv[8];
+                    e2m1x8_decode(ow[j], vv);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int idx = 8 * j + i;
+                        dq[idx] = ((chosen >> idx) & 1u) ? dsp : __fmul_rn(vv[i], S);
+                    }
+                }
+                store_f32<B>(deq + b * B, dq);
+            }
+            if (mse)
+                mse[b] = __fmul_rn(best, 1.0f / 16.0f);
+        }
+    }
+}
+
+// ------------------------------------------------------- brute-force scale
+// Brute force over E4M3 codes 1..126: the least in-order squared error, ties
+// to the lowest code.  Exact shortcuts (each provably skips only losers):
+//  * from the first code at which the largest element rounds to zero
+//    (|y| <= 0.25; |y| falls as the code grows) every element does, so that
+//    code gives the all-zero error (the in-order sum of x^2) and every higher
+//    code ties it with a higher code;
+//  * below the abs-max code c6 the largest element clips to 6, its error
+//    a - 6S grows as the code falls, and its square alone bounds the in-order
+//    fma chain from below (the chain only adds non-negative terms and
+//    rounding is monotone): the downward scan from c6 stops at the first
+//    code whose bound already loses against c6 or the all-zero code.
+// Every code left in between is evaluated in full.  Load balance: the ranges
+// of a warp's 32 blocks differ widely (a heavy-tailed block spans far more
+// codes), so the warp lays all (block, code) pairs end to end and every lane
+// takes every 32nd pair, reading the block from shared memory.  A block's
+// best (error, code) is one 64-bit key -- error bits (non-negative floats
+// order like their bits) above the code -- lowered with a shared-memory
+// atomic minimum, so the lowest code wins ties exactly as in a sequential
+// scan.
+constexpr int kWarps = kThreads / 32;
+
+template <int B, typename T>
+__global__ void __launch_bounds__(kThreads)
+nvfp4_bf_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs,
+                uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, int mma_layout,
+                float* __restrict__ deq, float* __restrict__ mse)
+{
+    // (S, inv) of every code: S = sc * g, inv = min(1/S, FLT_MAX), 0 for S = 0
+    __shared__ float2 tab[128];
+    __shared__ __align__(16) float xs[kWarps][32 * B];
+    __shared__ unsigned long long key[kWarps][32];
+    __shared__ int pre[kWarps][32];
+    __shared__ uint32_t meta[kWarps][32];   // clo | c6 << 8
+
+    const float g = resolve_global_scale(gs);
+    const float g6 = __fmul_rn(6.0f, g);
+    // only a starting point for the exact all-zero search below
+    const float four_over_g = __fmul_rn(4.0f, __frcp_rn(g));
+    for (int c = threadIdx.x; c < 128; c += blockDim.x) {
+        const float S = __fmul_rn(e4m3_decode((uint32_t)(c < 127 ? c : 126)), g);
+        tab[c] = make_float2(S, (S == 0.0f) ? 0.0f : fminf(__frcp_rn(S), kFltMax));
+    }
+    __syncthreads();
+
+    const int lane = threadIdx.x & 31;
+    const int w = threadIdx.x >> 5;
+    const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    const int64_t kb_atoms = (bpr + 3) >> 2;
+    int64_t r_cur = 0, kb_cur = 0, step_r = 0, step_kb = 0;
+    if (mma_layout) {
+        const int64_t b0 = warp0 * 32 + lane;
+        const int64_t step = nwarps * 32;
+        r_cur = b0 / bpr;
+        kb_cur = b0 % bpr;
+        step_r = step / bpr;
+        step_kb = step % bpr;
+    }
+    float* xw = xs[w];
+
+    for (int64_t base = warp0 * 32; base < nblk; base += nwarps * 32) {
+        const int64_t b = base + lane;
+        const bool valid = b < nblk;
+        float xv[B];
+        if (valid) {
+            load_elems<T, B>(x + b * B, xv);
+        } else {
+#pragma unroll
+            for (int i = 0; i < B; ++i)
+                xv[i] = 0.0f;
+        }
+        float a = 0.0f;
+        float sse0 = 0.0f;
+#pragma unroll
+        for (int i = 0; i < B; ++i) {
+            a = fmaxf(a, fabsf(xv[i]));
+            sse0 = __fmaf_rn(xv[i], xv[i], sse0);
+        }
+        uint32_t c6 = e4m3_encode(__fdiv_rn(a, g6));
+        c6 = c6 == 0u ? 1u : c6;
+        float best = quant_sse<B>(xv, 0.0f, 0.0f, tab[c6]);
+        uint32_t bc = c6;
+        // first all-zero code (127 = none): step from a nearby code to the
+        // boundary (|y| is monotone in the code)
+        uint32_t cz = e4m3_encode(__fmul_rn(a, four_over_g));
+        cz = cz == 0u ? 1u : cz;
+        if (__fmul_rn(a, tab[cz].y) <= 0.25f) {
+            while (cz > 1u && __fmul_rn(a, tab[cz - 1u].y) <= 0.25f)
+                --cz;
+        } else {
+            do {
+                ++cz;
+            } while (cz < 127u && __fmul_rn(a, tab[cz].y) > 0.25f);
+        }
+        if (cz < 127u && (sse0 < best || (sse0 == best && cz < bc))) {
+            best = sse0;
+            bc = cz;
+        }
+        // downward: codes below c6 while the clipped bound can still win
+        uint32_t clo = c6;
+        while (clo > 1u) {
+            const float2 t = tab[clo - 1u];
+            const float em = elem_err(a, t.x, t.y);
+            if (__fmul_rn(em, em) > best)
+                break;
+            --clo;
+        }
+        const int chi = (int)(cz < 127u ? cz : 127u) - 1;   // last code to evaluate
+        int span = chi - (int)clo + 1;
+        span = (valid && span > 0) ? span : 0;
+
+        // lay the warp's candidates end to end
+        int incl = span;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, d);
+            if (lane >= d)
+                incl += v;
+        }
+        const int total = __shfl_sync(0xffffffffu, incl, 31);
+        if (total > 0) {
+#pragma unroll
+            for (int i = 0; i < B; i += 4)
+                *reinterpret_cast<float4*>(&xw[lane * B + i]) =
+                    make_float4(xv[i], xv[i + 1], xv[i + 2], xv[i + 3]);
+            key[w][lane] = ((unsigned long long)__float_as_uint(best) << 32) | bc;
+            pre[w][lane] = incl - span;
+            meta[w][lane] = clo | (c6 << 8);
+            __syncwarp();
+            for (int t = lane; t < total; t += 32) {
+                // owner: the last block whose range starts at or before t
+                int j = 0;
+#pragma unroll
+                for (int st = 16; st > 0; st >>= 1)
+                    if (pre[w][j + st] <= t)
+                        j += st;
+                const uint32_t m = meta[w][j];
+                const uint32_t c = (m & 0xFFu) + (uint32_t)(t - pre[w][j]);
+                if (c == (m >> 8))
+                    continue;
+                float xj[B];
+#pragma unroll
+                for (int i = 0; i < B; i += 4) {
+                    const float4 q = *reinterpret_cast<const float4*>(&xw[j * B + i]);
+                    xj[i] = q.x;
+                    xj[i + 1] = q.y;
+                    xj[i + 2] = q.z;
+                    xj[i + 3] = q.w;
+                }
+                const float sc_ = quant_sse<B>(xj, 0.0f, 0.0f, tab[c]);
+                atomicMin(&key[w][j], ((unsigned long long)__float_as_uint(sc_) << 32) | c);
+            }
+            __syncwarp();
+            bc = (uint32_t)key[w][lane];
+            __syncwarp();
+        }
+
+        uint32_t cw[(B + 7) / 8];
+        float dq[B];
+        const float sse = quant_eval<B>(xv, e4m3_decode(bc), g, cw, dq);
+        if (valid) {
+            store_codes<B>(codes + b * (B / 2), cw);
+            const int64_t so = mma_layout ? mma_sf_offset(r_cur, kb_cur, kb_atoms) : b;
+            scales[so] = (uint8_t)bc;
+            if (deq)
+                store_f32<B>(deq + b * B, dq);
+            if (mse)
+                mse[b] = __fmul_rn(sse, 1.0f / (float)B);
+        }
+        if (mma_layout) {
+            kb_cur += step_kb;
+            r_cur += step_r;
+            if (kb_cur >= bpr) {
+                kb_cur -= bpr;
+                ++r_cur;
+            }
+        }
+    }
+}
+
 // ------------------------------------------------------ dequant + MSE
 // SF: 0 E4M3, 1 E3M3, 2 E8M0.  RAZ: the -0 code decodes to the block's
 // special value (selector in the scale byte's top bits).
@@ -636,10 +951,17 @@ cudaError_t nvfp4_launch_t(const void* x, int64_t rows, int64_t cols, const GsAr
                            cudaStream_t s)
 {
     const int64_t nblk = rows * (cols / B);
-    auto k = nvfp4_quant_kernel<B, T, RULE>;
-    const int grid = grid_for(nblk, (const void*)k);
-    k<<<grid, kThreads, 0, s>>>(reinterpret_cast<const T*>(x), nblk, cols / B, gs, codes, scales,
-                                 mma, deq, mse);
+    if constexpr (RULE == R_BF) {
+        auto k = nvfp4_bf_kernel<B, T>;
+        k<<<grid_for(nblk, (const void*)k), kThreads, 0, s>>>(reinterpret_cast<const T*>(x), nblk,
+                                                               cols / B, gs, codes, scales, mma,
+                                                               deq, mse);
+    } else {
+        auto k = nvfp4_quant_kernel<B, T, RULE>;
+        k<<<grid_for(nblk, (const void*)k), kThreads, 0, s>>>(reinterpret_cast<const T*>(x), nblk,
+                                                               cols / B, gs, codes, scales, mma,
+                                                               deq, mse);
+    }
     return cudaGetLastError();
 }
 
@@ -759,6 +1081,34 @@ cudaError_t launch_razer_quant(const void* x, int dtype, int64_t rows, int64_t c
     }
     sp.n = n_special;
     const int64_t nblk = rows * (cols / 16);
+    // (+v, -v) pairs in table order take the single-pass kernel
+    bool paired = n_special % 2 == 0;
+    for (int i = 0; paired && i < n_special; i += 2)
+        paired = specials_host[i] > 0.0f && specials_host[i + 1] == -specials_host[i];
+    if (paired) {
+        const int np = n_special / 2;
+#define FP4Q_RAZER_PAIRED(TT, SFV, NP)                                                                  \
+    {                                                                                                \
+        auto k = razer_paired_kernel<TT, SFV, NP>;                                                   \
+        k<<<grid_for(nblk, (const void*)k), kThreads, 0, s>>>(reinterpret_cast<const TT*>(x), nblk, gs, \
+                                                               sp, codes, meta, deq, mse);           \
+    }
+        if (dtype == 1) {
+            if (sf == 1) {
+                if (np == 1) FP4Q_RAZER_PAIRED(__nv_bfloat16, 1, 1) else FP4Q_RAZER_PAIRED(__nv_bfloat16, 1, 2)
+            } else {
+                FP4Q_RAZER_PAIRED(__nv_bfloat16, 0, 1)
+            }
+        } else {
+            if (sf == 1) {
+                if (np == 1) FP4Q_RAZER_PAIRED(float, 1, 1) else FP4Q_RAZER_PAIRED(float, 1, 2)
+            } else {
+                FP4Q_RAZER_PAIRED(float, 0, 1)
+            }
+        }
+#undef FP4Q_RAZER_PAIRED
+        return cudaGetLastError();
+    }
     if (dtype == 1) {
         if (sf == 1) {
             auto k = razer_quant_kernel<__nv_bfloat16, 1>;
