@@ -51,6 +51,8 @@ constexpr uint32_t kSfColsPerStage = 48;       // SFA 4 k-steps x 4 + SFB 4 k-st
 constexpr long long kWaitCycles = 4000000000LL;   // about 2 s at the boost clock
 // The pair teardown outlasts a peer's own quiesce waits.
 constexpr long long kTeardownCycles = 3 * kWaitCycles;
+// Grace period for copies whose completion this CTA cannot observe (about 1 ms).
+constexpr long long kDrainCycles = 2000000LL;
 
 static_assert(kStageBytes % 1024 == 0, "stage bases must keep the 1024-byte swizzle alignment");
 static_assert(kSfCol0 + kStages * kSfColsPerStage <= kTmemCols, "TMEM budget");
@@ -164,6 +166,27 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
                                             uint32_t bar)
 {
     asm volatile("cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+                 " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
+                 "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+                 : "memory");
+}
+
+// Pair loads: the copy lands in this CTA's shared memory and completes its
+// bytes on an mbarrier that may sit in either CTA of the pair (here: the
+// leader's), so the leader sees both halves of a stage on one barrier.
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                                 uint32_t bar)
+{
+    asm volatile("cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.cta_group::2"
+                 " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+                 "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap* map, int x, int y, int z,
+                                                 uint32_t bar)
+{
+    asm volatile("cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.cta_group::2"
                  " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(dst),
                  "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
                  : "memory");
@@ -433,9 +456,10 @@ w4a4_gemm_1sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
 // Two CTAs of a cluster compute a 256 x 256 output tile with M=256, N=256,
 // K=64 pair MMAs issued by the leader (cluster rank 0).  Each CTA stages its
 // own 128 rows of A, its own 128 rows of B (the MMA reads the two halves of
-// B from the two CTAs), its own A scale atom and both B scale atoms, and
-// signals its own barrier; the follower forwards "stage ready" to the leader
-// with one remote arrive.  The leader's commits are multicast to both CTAs.
+// B from the two CTAs), its own A scale atom and both B scale atoms; both
+// CTAs' copies complete on the leader's stage barrier (pair-form TMA loads),
+// so the MMA issuer waits on one barrier per stage.  The leader's commits are
+// multicast to both CTAs.
 // The epilogue stages bf16 32 x 64 boxes in 128B-swizzled shared memory (two
 // boxes, half a tile row, at a time) and writes them with TMA stores, handing
 // the accumulator back as soon as its TMEM reads are done, so the stores
@@ -532,8 +556,9 @@ w4a4_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* epi = smem + k2Stages * k2StageBytes;
     uint64_t* bars = reinterpret_cast<uint64_t*>(epi + k2EpiBytes);
-    // bars: [0,S) full, [S,2S) empty, [2S,3S) peer-ready (leader), 3S acc_full,
-    // 3S+1 acc_empty (leader), 3S+2 drain, 3S+3 teardown handshake
+    // bars: [0,S) full (the leader's counts both CTAs' bytes), [S,2S) empty,
+    // [2S,3S) unused, 3S acc_full, 3S+1 acc_empty (leader), 3S+2 drain,
+    // 3S+3 teardown handshake
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 3 * k2Stages + 4);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
@@ -544,7 +569,6 @@ w4a4_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
     const uint32_t bar0 = smem_u32(bars);
     auto full_bar = [&](int s) { return bar0 + 8u * (uint32_t)s; };
     auto empty_bar = [&](int s) { return bar0 + 8u * (uint32_t)(k2Stages + s); };
-    auto peer_bar = [&](int s) { return bar0 + 8u * (uint32_t)(2 * k2Stages + s); };
     const uint32_t acc_full = bar0 + 8u * (3 * k2Stages);
     const uint32_t acc_empty = bar0 + 8u * (3 * k2Stages + 1);
     const uint32_t drain = bar0 + 8u * (3 * k2Stages + 2);
@@ -554,7 +578,6 @@ w4a4_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
         for (int s = 0; s < k2Stages; ++s) {
             mbar_init(full_bar(s), 1);
             mbar_init(empty_bar(s), 1);
-            mbar_init(peer_bar(s), 1);
         }
         mbar_init(acc_full, 1);
         mbar_init(acc_empty, 2 * 128);
@@ -602,13 +625,16 @@ w4a4_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                         give_up();
                         break;
                     }
-                    const uint32_t fb = full_bar(stage);
-                    mbar_expect_tx(fb, k2StageBytes);
+                    // the leader expects both CTAs' bytes of this stage
+                    const uint32_t fb = mapa_rank(full_bar(stage), 0);
+                    if (leader)
+                        mbar_expect_tx(full_bar(stage), 2 * k2StageBytes);
                     uint8_t* st = smem + stage * k2StageBytes;
-                    tma_load_2d(smem_u32(st), &tmA, kb * (kBK / 2), mt * 256 + (int)rank * 128, fb);
-                    tma_load_2d(smem_u32(st + k2AStage), &tmB, kb * (kBK / 2), nt * 256 + (int)rank * 128, fb);
-                    tma_load_3d(smem_u32(st + k2AStage + k2BStage), &tmSA, 0, kb * 4, 2 * mt + (int)rank, fb);
-                    tma_load_3d(smem_u32(st + k2AStage + k2BStage + k2SfaStage), &tmSB, 0, kb * 4, 2 * nt, fb);
+                    tma_load_2d_pair(smem_u32(st), &tmA, kb * (kBK / 2), mt * 256 + (int)rank * 128, fb);
+                    tma_load_2d_pair(smem_u32(st + k2AStage), &tmB, kb * (kBK / 2), nt * 256 + (int)rank * 128, fb);
+                    tma_load_3d_pair(smem_u32(st + k2AStage + k2BStage), &tmSA, 0, kb * 4, 2 * mt + (int)rank, fb);
+                    tma_load_3d_pair(smem_u32(st + k2AStage + k2BStage + k2SfaStage), &tmSB, 0, kb * 4, 2 * nt,
+                                     fb);
                     issued |= 1u << stage;
                     issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
                     if (++stage == k2Stages) {
@@ -617,10 +643,21 @@ w4a4_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                     }
                 }
             }
-            if (*abort_flag)
-                for (int s = 0; s < k2Stages; ++s)
-                    if (issued & (1u << s))
-                        mbar_quiesce(full_bar(s), (issued_parity >> s) & 1u);
+            if (*abort_flag && issued) {
+                if (leader) {
+                    // a stage's barrier completes once both CTAs' copies landed
+                    for (int s = 0; s < k2Stages; ++s)
+                        if (issued & (1u << s))
+                            mbar_quiesce(full_bar(s), (issued_parity >> s) & 1u);
+                } else {
+                    // the follower's copies complete on the leader's barrier,
+                    // which it cannot poll: give them a bounded grace period
+                    // (orders of magnitude above a copy's latency)
+                    const long long t0 = clock64();
+                    while (clock64() - t0 < kDrainCycles) {
+                    }
+                }
+            }
         }
     } else if (warp == 1) {
         if (lane == 0 && leader) {
@@ -636,8 +673,7 @@ w4a4_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                 tc_fence_after();
                 bool ok = true;
                 for (int kb = 0; kb < p.kblocks; ++kb) {
-                    if (!mbar_wait(full_bar(stage), phase, abort_flag) ||
-                        !mbar_wait_cluster(peer_bar(stage), phase, abort_flag) || *abort_flag) {
+                    if (!mbar_wait_cluster(full_bar(stage), phase, abort_flag) || *abort_flag) {
                         give_up();
                         ok = false;
                         break;
@@ -676,27 +712,6 @@ w4a4_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                 tc2_commit_mc(drain, (uint16_t)0x1);
                 if (!mbar_quiesce(drain, 0))
                     give_up();
-            }
-        } else if (lane == 0) {
-            // --------------------- follower: forward "stage ready" to the leader
-            int stage = 0;
-            uint32_t phase = 0;
-            for (int tile = cluster; tile < num_tiles && !*abort_flag; tile += nclusters) {
-                bool ok = true;
-                for (int kb = 0; kb < p.kblocks; ++kb) {
-                    if (!mbar_wait(full_bar(stage), phase, abort_flag) || *abort_flag) {
-                        give_up();
-                        ok = false;
-                        break;
-                    }
-                    mbar_arrive_cluster(mapa_rank(peer_bar(stage), 0));
-                    if (++stage == k2Stages) {
-                        stage = 0;
-                        phase ^= 1u;
-                    }
-                }
-                if (!ok)
-                    break;
             }
         }
     } else {
