@@ -59,9 +59,13 @@ def load_peaks():
 class Row:
     """One hot-path row: how to launch it on device buffers and what it moves."""
 
-    def __init__(self, name, kernel, units, bytes_, launches, fn, out, bound="hbm", flops=0.0, evals=0.0):
+    def __init__(self, name, kernel, units, bytes_, launches, fn, out, bound="hbm", flops=0.0, evals=0.0,
+                 eval_ws=None, block=0):
         self.name, self.kernel, self.units, self.bytes, self.launches = name, kernel, units, bytes_, launches
         self.fn, self.out, self.bound, self.flops, self.evals = fn, out, bound, flops, evals
+        # brute force: workspace whose counter at FP4Q_WS_BF_EVALS receives the
+        # number of (block, candidate) error evaluations a call performs
+        self.eval_ws, self.block = eval_ws, block
 
 
 def build_rows(torch, fq, inputs, dev, host_copies=None):
@@ -95,13 +99,15 @@ def build_rows(torch, fq, inputs, dev, host_copies=None):
     for B in (4, 8, 16, 32):
         for rule in (fq.ABSMAX, fq.PREVENT_ZERO, fq.FOUR_OVER_SIX, fq.BRUTE_FORCE):
             o = {}
+            bf = rule == fq.BRUTE_FORCE
+            wsr = torch.zeros(fq.workspace_size(fq.OP_QUANTIZE, 1, 1), dtype=torch.uint8, device=dev) if bf else None
 
-            def c2(B=B, rule=rule, o=o):
-                o.update(fq.nvfp4_quantize(X["c2"], B, rule, gs_mode=fq.GS_NONE, mse=True, out=o))
-            rows.append(Row("c2_B%d_%s" % (B, names[rule]), "nvfp4_quant_kernel<%d, float, %d>" % (B, rule),
+            def c2(B=B, rule=rule, o=o, wsr=wsr):
+                o.update(fq.nvfp4_quantize(X["c2"], B, rule, gs_mode=fq.GS_NONE, mse=True, out=o, workspace=wsr))
+            kern = ("nvfp4_bf_kernel<%d, float>" % B) if bf else ("nvfp4_quant_kernel<%d, float, %d>" % (B, rule))
+            rows.append(Row("c2_B%d_%s" % (B, names[rule]), kern,
                             n2, n2 * (4 + 0.5 + 1 / B + 4 / B), 1, c2, o,
-                            bound="alu" if rule == fq.BRUTE_FORCE else "hbm",
-                            evals=n2 * 126.0 if rule == fq.BRUTE_FORCE else 0.0))
+                            bound="alu" if bf else "hbm", eval_ws=wsr, block=B))
     # c3
     w3 = inputs.generate("razer_weight")
     X["c3w"] = to_dev(w3, "c3w")
@@ -358,6 +364,15 @@ def main():
         flush.zero_()
         step()
     torch.cuda.synchronize()
+    # brute force: the exact number of error evaluations one call performs
+    # (deterministic for a given input), read from the library's counter
+    for r in rows:
+        if r.eval_ws is not None:
+            r.eval_ws.zero_()
+            r.fn()
+            torch.cuda.synchronize()
+            n_eval = int(r.eval_ws[fq.WS_BF_EVALS:fq.WS_BF_EVALS + 8].cpu().numpy().view(np.uint64)[0])
+            r.evals = float(n_eval) * r.block
 
     def barrier():
         if world > 1:
@@ -410,12 +425,16 @@ def main():
     dms = row_out[dom.name]["ms"]
     # fp32 pipe: 148 SMs x 128 lanes x clock; one element-candidate evaluation of
     # a scale search is 6 issue slots (scale multiply, e2m1 encode and decode,
-    # dequant multiply, subtract, fma)
+    # dequant multiply, subtract, fma).  Brute-force rows count the element
+    # evaluations the call actually performed (the exact shortcuts skip most of
+    # the 126 candidates); the overhead around them (seeds, bounds, the warp's
+    # work sharing) is what keeps the fraction below 1.
     eval_peak = SM_COUNT * FP32_LANES_PER_SM * sm_max_mhz * 1e6 / 6.0 / 1e9
     for r in rows:
         if r.evals:
             row_out[r.name]["Geval_s"] = r.evals / (row_out[r.name]["ms"] * 1e-3) / 1e9
             row_out[r.name]["alu_frac"] = row_out[r.name]["Geval_s"] / eval_peak
+            row_out[r.name]["evals_per_block"] = r.evals / r.block / (r.units / r.block)
     fp4_peak = bf16_peak * 4.0     # dense FP4 = 4 x dense bf16 (nominal 9 / 2.25 PFLOP/s)
     for r in rows:
         if r.bound == "tensor":
@@ -430,8 +449,10 @@ def main():
         ach = dom.evals / (dms * 1e-3) / 1e9
         roof = {"bound": "alu", "achieved": ach, "peak": eval_peak, "unit": "Geval/s", "frac": ach / eval_peak,
                 "traffic": None, "kernel": dom.kernel, "row": dom.name,
-                "note": "brute force: 126 candidate scales x elements per launch; exact shortcuts skip provably "
-                        "losing candidates, so frac can exceed 1"}
+                "note": "brute force: element-candidate error evaluations the launch performed (counted by the "
+                        "library; %.2f per block of the 126 a naive scan does) / time, against 148 SMs x 128 "
+                        "fp32 lanes x clock / 6 issue slots per evaluation"
+                        % row_out[dom.name]["evals_per_block"]}
     else:
         ach = dom.bytes / (dms * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": ach, "peak": hbm_peak, "unit": "GB/s", "frac": ach / hbm_peak,

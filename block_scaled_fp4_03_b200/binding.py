@@ -21,6 +21,9 @@ ABSMAX, PREVENT_ZERO, FOUR_OVER_SIX, BRUTE_FORCE, HESSIAN_EXP = range(5)
 GS_NONE, GS_AMAX, GS_GIVEN = 0, 1, 2
 SF_ROWMAJOR, SF_MMA = 0, 1
 OP_QUANTIZE, OP_HESSIAN, OP_CHANNEL_SCALE, OP_GEMM = range(4)
+# byte offset, in a quantize workspace, of the uint64 that brute force adds its
+# evaluation count to (FP4Q_WS_BF_EVALS)
+WS_BF_EVALS = 3072
 
 # name -> (restype, argtypes) of every exported entry point
 _vp, _i, _i64, _sz, _fp = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float

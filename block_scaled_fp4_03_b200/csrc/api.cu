@@ -26,7 +26,8 @@ constexpr size_t kGemmHeader = 8192;
 constexpr size_t kGemmGa = 4096;
 constexpr size_t kGemmErr = 4160;
 size_t gemm_ws_bytes(int64_t M, int64_t K) { return kGemmHeader + (size_t)M * (size_t)K / 2 + (size_t)M * (size_t)K / 16; }
-static_assert(kAmaxPartials * sizeof(float) <= kQuantWs, "amax partials must fit");
+static_assert(kAmaxPartials * sizeof(float) <= FP4Q_WS_BF_EVALS && FP4Q_WS_BF_EVALS + 8 <= kQuantWs,
+              "amax partials and the evaluation counter must fit");
 
 // Resolve a global-scale request into launch arguments (running the amax
 // pre-pass for AMAX).  Returns FP4Q_OK or an error.
@@ -119,8 +120,12 @@ int nvfp4_quantize(const void* x, int dtype, int64_t rows, int64_t cols, int blo
                         workspace_bytes, s, gs);
     if (st != FP4Q_OK)
         return st;
+    unsigned long long* evals =
+        (workspace && workspace_bytes >= kQuantWs)
+            ? reinterpret_cast<unsigned long long*>(static_cast<uint8_t*>(workspace) + FP4Q_WS_BF_EVALS)
+            : nullptr;
     return from_cuda(launch_nvfp4_quant(x, dtype, rows, cols, block, rule, gs, codes, scales,
-                                        sf_layout == FP4Q_SFLAYOUT_MMA, dequant, block_mse, s));
+                                        sf_layout == FP4Q_SFLAYOUT_MMA, dequant, block_mse, evals, s));
 }
 
 int razer_quantize(const void* x, int dtype, int64_t rows, int64_t cols, int scale_fmt,
@@ -305,7 +310,7 @@ int w4a4_gemm(const void* a, int a_format, int a_rule, const uint8_t* a_scales,
         cudaError_t e = launch_amax(a, a_format, M * K, reinterpret_cast<float*>(ws), s);
         if (e == cudaSuccess)
             e = launch_nvfp4_quant(a, a_format, M, K, 16, a_rule, gs, qcodes, qsf, 1, nullptr,
-                                   nullptr, s);
+                                   nullptr, nullptr, s);
         if (e != cudaSuccess)
             return FP4Q_ERR_CUDA;
         a_codes = qcodes;

@@ -25,9 +25,11 @@ int num_sms();
 
 cudaError_t launch_amax(const void* x, int dtype, int64_t n, float* partials, cudaStream_t s);
 
+// evals (nullable): brute force adds its number of block-candidate evaluations
 cudaError_t launch_nvfp4_quant(const void* x, int dtype, int64_t rows, int64_t cols, int block,
                                int rule, const GsArgs& gs, uint8_t* codes, uint8_t* scales,
-                               int mma_layout, float* deq, float* mse, cudaStream_t s);
+                               int mma_layout, float* deq, float* mse, unsigned long long* evals,
+                               cudaStream_t s);
 
 cudaError_t launch_razer_quant(const void* x, int dtype, int64_t rows, int64_t cols, int sf,
                                const float* specials_host, int n_special, const GsArgs& gs,

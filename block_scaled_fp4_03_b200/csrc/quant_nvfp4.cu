@@ -691,8 +691,9 @@ template <int B, typename T>
 __global__ void __launch_bounds__(kThreads)
 nvfp4_bf_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs,
                 uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, int mma_layout,
-                float* __restrict__ deq, float* __restrict__ mse)
+                float* __restrict__ deq, float* __restrict__ mse, unsigned long long* evals)
 {
+    uint32_t n_eval = 0;   // this lane's error evaluations (seed, all-zero, scan)
     // (S, inv) of every code: S = sc * g, inv = min(1/S, FLT_MAX), 0 for S = 0
     __shared__ float2 tab[128];
     __shared__ __align__(16) float xs[kWarps][32 * B];
@@ -748,6 +749,7 @@ nvfp4_bf_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs,
         c6 = c6 == 0u ? 1u : c6;
         float best = quant_sse<B>(xv, 0.0f, 0.0f, tab[c6]);
         uint32_t bc = c6;
+        n_eval += valid ? 1u : 0u;
         // first all-zero code (127 = none): step from a nearby code to the
         // boundary (|y| is monotone in the code)
         uint32_t cz = e4m3_encode(__fmul_rn(a, four_over_g));
@@ -760,6 +762,7 @@ nvfp4_bf_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs,
                 ++cz;
             } while (cz < 127u && __fmul_rn(a, tab[cz].y) > 0.25f);
         }
+        n_eval += (valid && cz < 127u) ? 1u : 0u;
         if (cz < 127u && (sse0 < best || (sse0 == best && cz < bc))) {
             best = sse0;
             bc = cz;
@@ -817,6 +820,7 @@ nvfp4_bf_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs,
                 }
                 const float sc_ = quant_sse<B>(xj, 0.0f, 0.0f, tab[c]);
                 atomicMin(&key[w][j], ((unsigned long long)__float_as_uint(sc_) << 32) | c);
+                ++n_eval;
             }
             __syncwarp();
             bc = (uint32_t)key[w][lane];
@@ -843,6 +847,11 @@ nvfp4_bf_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs,
                 ++r_cur;
             }
         }
+    }
+    if (evals) {
+        const uint32_t wsum = __reduce_add_sync(0xffffffffu, n_eval);
+        if (lane == 0 && wsum)
+            atomicAdd(evals, (unsigned long long)wsum);
     }
 }
 
@@ -948,14 +957,14 @@ int grid_for(int64_t work_threads, const void* kernel)
 template <int B, typename T, int RULE>
 cudaError_t nvfp4_launch_t(const void* x, int64_t rows, int64_t cols, const GsArgs& gs,
                            uint8_t* codes, uint8_t* scales, int mma, float* deq, float* mse,
-                           cudaStream_t s)
+                           unsigned long long* evals, cudaStream_t s)
 {
     const int64_t nblk = rows * (cols / B);
     if constexpr (RULE == R_BF) {
         auto k = nvfp4_bf_kernel<B, T>;
         k<<<grid_for(nblk, (const void*)k), kThreads, 0, s>>>(reinterpret_cast<const T*>(x), nblk,
                                                                cols / B, gs, codes, scales, mma,
-                                                               deq, mse);
+                                                               deq, mse, evals);
     } else {
         auto k = nvfp4_quant_kernel<B, T, RULE>;
         k<<<grid_for(nblk, (const void*)k), kThreads, 0, s>>>(reinterpret_cast<const T*>(x), nblk,
@@ -968,13 +977,13 @@ cudaError_t nvfp4_launch_t(const void* x, int64_t rows, int64_t cols, const GsAr
 template <int B, typename T>
 cudaError_t nvfp4_launch_rule(int rule, const void* x, int64_t rows, int64_t cols,
                               const GsArgs& gs, uint8_t* codes, uint8_t* scales, int mma,
-                              float* deq, float* mse, cudaStream_t s)
+                              float* deq, float* mse, unsigned long long* evals, cudaStream_t s)
 {
     switch (rule) {
-    case R_ABSMAX: return nvfp4_launch_t<B, T, R_ABSMAX>(x, rows, cols, gs, codes, scales, mma, deq, mse, s);
-    case R_PZ: return nvfp4_launch_t<B, T, R_PZ>(x, rows, cols, gs, codes, scales, mma, deq, mse, s);
-    case R_46: return nvfp4_launch_t<B, T, R_46>(x, rows, cols, gs, codes, scales, mma, deq, mse, s);
-    case R_BF: return nvfp4_launch_t<B, T, R_BF>(x, rows, cols, gs, codes, scales, mma, deq, mse, s);
+    case R_ABSMAX: return nvfp4_launch_t<B, T, R_ABSMAX>(x, rows, cols, gs, codes, scales, mma, deq, mse, evals, s);
+    case R_PZ: return nvfp4_launch_t<B, T, R_PZ>(x, rows, cols, gs, codes, scales, mma, deq, mse, evals, s);
+    case R_46: return nvfp4_launch_t<B, T, R_46>(x, rows, cols, gs, codes, scales, mma, deq, mse, evals, s);
+    case R_BF: return nvfp4_launch_t<B, T, R_BF>(x, rows, cols, gs, codes, scales, mma, deq, mse, evals, s);
     default: return cudaErrorInvalidValue;
     }
 }
@@ -982,13 +991,13 @@ cudaError_t nvfp4_launch_rule(int rule, const void* x, int64_t rows, int64_t col
 template <typename T>
 cudaError_t nvfp4_launch_b(int block, int rule, const void* x, int64_t rows, int64_t cols,
                            const GsArgs& gs, uint8_t* codes, uint8_t* scales, int mma, float* deq,
-                           float* mse, cudaStream_t s)
+                           float* mse, unsigned long long* evals, cudaStream_t s)
 {
     switch (block) {
-    case 4: return nvfp4_launch_rule<4, T>(rule, x, rows, cols, gs, codes, scales, mma, deq, mse, s);
-    case 8: return nvfp4_launch_rule<8, T>(rule, x, rows, cols, gs, codes, scales, mma, deq, mse, s);
-    case 16: return nvfp4_launch_rule<16, T>(rule, x, rows, cols, gs, codes, scales, mma, deq, mse, s);
-    case 32: return nvfp4_launch_rule<32, T>(rule, x, rows, cols, gs, codes, scales, mma, deq, mse, s);
+    case 4: return nvfp4_launch_rule<4, T>(rule, x, rows, cols, gs, codes, scales, mma, deq, mse, evals, s);
+    case 8: return nvfp4_launch_rule<8, T>(rule, x, rows, cols, gs, codes, scales, mma, deq, mse, evals, s);
+    case 16: return nvfp4_launch_rule<16, T>(rule, x, rows, cols, gs, codes, scales, mma, deq, mse, evals, s);
+    case 32: return nvfp4_launch_rule<32, T>(rule, x, rows, cols, gs, codes, scales, mma, deq, mse, evals, s);
     default: return cudaErrorInvalidValue;
     }
 }
@@ -1052,13 +1061,14 @@ cudaError_t launch_amax(const void* x, int dtype, int64_t n, float* partials, cu
 
 cudaError_t launch_nvfp4_quant(const void* x, int dtype, int64_t rows, int64_t cols, int block,
                                int rule, const GsArgs& gs, uint8_t* codes, uint8_t* scales,
-                               int mma_layout, float* deq, float* mse, cudaStream_t s)
+                               int mma_layout, float* deq, float* mse, unsigned long long* evals,
+                               cudaStream_t s)
 {
     if (dtype == 1)
         return nvfp4_launch_b<__nv_bfloat16>(block, rule, x, rows, cols, gs, codes, scales,
-                                             mma_layout, deq, mse, s);
+                                             mma_layout, deq, mse, evals, s);
     return nvfp4_launch_b<float>(block, rule, x, rows, cols, gs, codes, scales, mma_layout, deq,
-                                 mse, s);
+                                 mse, evals, s);
 }
 
 cudaError_t launch_razer_quant(const void* x, int dtype, int64_t rows, int64_t cols, int sf,

@@ -143,8 +143,13 @@ FP4Q_API const char* fp4q_version(void);
  *  block_mse    device fp32 rows x cols/block (out, nullable): sum((x-deq)^2)/block
  *  workspace    device, >= fp4q_workspace_size(FP4Q_OP_QUANTIZE, ...) bytes when
  *               gs_mode == AMAX (else may be NULL), 16-byte aligned
+ * Brute force with a workspace also ADDS to the uint64 at workspace byte
+ * offset FP4Q_WS_BF_EVALS the number of (block, candidate scale) error
+ * evaluations the call performed (the exact shortcuts skip the rest); the
+ * caller zeroes it to start a count.  Nothing else reads or resets it.
  * Errors: ERR_ARG (bad enum/size/null), ERR_ALIGN, ERR_WORKSPACE, ERR_CUDA.
  */
+#define FP4Q_WS_BF_EVALS 3072
 FP4Q_API int nvfp4_quantize(const void* x, int dtype, int64_t rows, int64_t cols, int block, int rule,
                    int gs_mode, float* global_scale, uint8_t* codes, uint8_t* scales,
                    int sf_layout, float* dequant, float* block_mse, void* workspace,

@@ -34,6 +34,14 @@ def test_every_declared_symbol_is_exported(L):
         assert n in binding.SIGNATURES, n
 
 
+def test_header_constants_match_binding():
+    from block_scaled_fp4_03_b200 import binding
+    src = open(os.path.join(ROOT, "include", "fp4q.h")).read()
+    m = re.search(r"#define\s+FP4Q_WS_BF_EVALS\s+(\d+)", src)
+    assert m and int(m.group(1)) == binding.WS_BF_EVALS
+    assert binding.WS_BF_EVALS % 8 == 0
+
+
 def test_version_and_status_strings(L):
     assert b"sm_100a" in L.fp4q_version()
     assert L.fp4q_status_str(0) == b"ok"

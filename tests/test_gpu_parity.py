@@ -133,6 +133,35 @@ def test_nvfp4_empty_and_zero(O):
     assert np.all(host(r["mse"]) == 0) and np.all(host(r["codes"]) == 0)
 
 
+def test_brute_force_evaluation_counter(O):
+    """The evaluation count a brute-force call adds to its workspace counter:
+    at least the one seed per block, at most all 126 codes plus the all-zero
+    candidate per block, identical across repeated calls, and added to
+    (not reset) by each call."""
+    x, x32 = make("student_t", 96, 512, seed=3, dtype="f32")
+    ws = torch.zeros(fq.workspace_size(fq.OP_QUANTIZE, 1, 1), dtype=torch.uint8, device="cuda")
+    counts = []
+    for B in (4, 16):
+        ws.zero_()
+        r = fq.nvfp4_quantize(x, B, fq.BRUTE_FORCE, gs_mode=fq.GS_NONE, workspace=ws)
+        torch.cuda.synchronize()
+        n1 = int(host(ws)[fq.WS_BF_EVALS:fq.WS_BF_EVALS + 8].view(np.uint64)[0])
+        fq.nvfp4_quantize(x, B, fq.BRUTE_FORCE, gs_mode=fq.GS_NONE, workspace=ws)
+        torch.cuda.synchronize()
+        n2 = int(host(ws)[fq.WS_BF_EVALS:fq.WS_BF_EVALS + 8].view(np.uint64)[0])
+        nblk = x32.size // B
+        assert nblk <= n1 <= 127 * nblk, (B, n1, nblk)
+        assert n2 == 2 * n1
+        ref = O.nvfp4_quantize(x32, B, O.RULE_BRUTE_FORCE, g=1.0)
+        assert_bits(r["scales"], ref["scales"], "scales B=%d" % B)
+        counts.append(n1)
+    # other rules leave the counter alone
+    ws.zero_()
+    fq.nvfp4_quantize(x, 16, fq.FOUR_OVER_SIX, gs_mode=fq.GS_NONE, workspace=ws)
+    torch.cuda.synchronize()
+    assert int(host(ws)[fq.WS_BF_EVALS:fq.WS_BF_EVALS + 8].view(np.uint64)[0]) == 0
+
+
 # ------------------------------------------------------------------ RaZeR
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("sf,kind,specials", [(fq.SF_E3M3, "razer_weight", [5.0, -5.0, 3.5, -3.5]),
