@@ -17,7 +17,8 @@
  *            by minimum mean squared error).
  *   [MACaQ]  "MACaQ: Fast, Model Agnostic Calibrated Quantization ..."
  *            review, section 1 (MXFP4, online scaling and micro-rotation,
- *            Hessian-weighted exponent selection) and section 3 (Method).
+ *            Hessian-weighted exponent selection, Flip-Refinement) and
+ *            section 3 (Method).
  *   [Finer]  "Finer is Better (with the Right Scaling)" summary,
  *            Methodology items 1-2 (abs-max, prevent-zero, 4-over-6,
  *            brute force, hierarchical scaling).
@@ -485,6 +486,129 @@ int oracle_mxfp4_quantize(const float *x, int64_t rows, int64_t cols, const floa
                 mse[b] = sse * (1.0f / 32.0f);
         }
         free(u);
+    }
+    return bad ? -1 : 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* Flip-Refinement ([MACaQ] section 1 Key Terms, section 3 Method)      */
+/* ------------------------------------------------------------------ */
+
+/* The E2M1 values in increasing order as one ladder of 15 levels (+0 and
+ * -0 are the same level, index 7).  A move takes one element to the
+ * neighbouring level below or above. */
+static int e2m1_level(int code)
+{
+    int m = code & 7;
+    return (code & 8) ? 7 - m : 7 + m;
+}
+
+static int e2m1_code_of_level(int level)
+{
+    return level >= 7 ? level - 7 : (8 | (7 - level));
+}
+
+/* Starting from the codes of an MX quantization (exponents fixed), each
+ * output row runs a greedy coordinate descent on
+ *   f = sum_k d_k^T H'_k d_k,   d = u - deq(codes),
+ * u the transformed row and H'_k the 32x32 diagonal blocks of the layer
+ * Hessian.  A step evaluates, for every element i and both neighbouring
+ * levels, the closed-form decrease of f when the element's dequantized value
+ * moves by D = (v' - v) 2^e:
+ *   gain = 2 D g_i - D^2 H_ii,   g = H' d   (the block's gradient / 2),
+ * takes the largest gain if it is positive (ties: lowest element, then the
+ * downward move), updates the code, and updates the block's g in place:
+ *   g_j <- g_j - D H_ji.
+ * A row stops after max_moves accepted moves or when no move has a
+ * positive gain.  g starts as the fma chain v_i = sum_j H_ij d_j in j order
+ * (the exponent selection's order); gain = 2*(D*g_i) - (D*D)*H_ii with each
+ * product and the difference rounded to fp32.  codes are updated in place;
+ * moves (nullable) receives the accepted move count per row. */
+int oracle_mxfp4_flip_refine(const float *x, int64_t rows, int64_t cols, const float *t,
+                             int hadamard, const float *hess, int max_moves, uint8_t *codes,
+                             const uint8_t *scales, int32_t *moves)
+{
+    if (cols % 32 != 0 || !hess || max_moves < 0)
+        return -1;
+    const int64_t kb = cols / 32;
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < rows; ++r) {
+        float *u = (float *)malloc((size_t)cols * sizeof(float));
+        float *g = (float *)malloc((size_t)cols * sizeof(float));
+        uint8_t *c = (uint8_t *)malloc((size_t)cols);
+        if (!u || !g || !c) {
+#pragma omp atomic write
+            bad = 1;
+            free(u);
+            free(g);
+            free(c);
+            continue;
+        }
+        transform_row(x + r * cols, cols, t, hadamard, u);
+        for (int64_t j = 0; j < cols; ++j) {
+            uint8_t byte = codes[(r * cols + j) / 2];
+            c[j] = (uint8_t)((j & 1) ? (byte >> 4) : (byte & 15));
+        }
+        /* g = H'_k d per block */
+        for (int64_t k = 0; k < kb; ++k) {
+            const int e = (int)scales[r * kb + k] - 127;
+            float d[32];
+            for (int j = 0; j < 32; ++j)
+                d[j] = u[k * 32 + j] - ldexpf(oracle_e2m1_value(c[k * 32 + j]), e);
+            const float *H = hess + k * 1024;
+            for (int i = 0; i < 32; ++i) {
+                float v = 0.0f;
+                for (int j = 0; j < 32; ++j)
+                    v = fmaf(H[i * 32 + j], d[j], v);
+                g[k * 32 + i] = v;
+            }
+        }
+        int32_t n = 0;
+        while (n < max_moves) {
+            float best = 0.0f;
+            int64_t bi = -1;
+            int blevel = 0;
+            for (int64_t i = 0; i < cols; ++i) {
+                const int64_t k = i / 32;
+                const int e = (int)scales[r * kb + k] - 127;
+                const float Hii = hess[k * 1024 + (i % 32) * 33];
+                const int level = e2m1_level(c[i]);
+                const float v = oracle_e2m1_value(c[i]);
+                for (int dir = -1; dir <= 1; dir += 2) {
+                    const int nl = level + dir;
+                    if (nl < 0 || nl > 14)
+                        continue;
+                    const float vn = oracle_e2m1_value(e2m1_code_of_level(nl));
+                    const float D = ldexpf(vn - v, e);
+                    const float gain = 2.0f * (D * g[i]) - (D * D) * Hii;
+                    if (gain > best) {
+                        best = gain;
+                        bi = i;
+                        blevel = nl;
+                    }
+                }
+            }
+            if (bi < 0)
+                break;
+            const int64_t k = bi / 32;
+            const int e = (int)scales[r * kb + k] - 127;
+            const float D = ldexpf(oracle_e2m1_value(e2m1_code_of_level(blevel)) -
+                                       oracle_e2m1_value(c[bi]), e);
+            c[bi] = (uint8_t)e2m1_code_of_level(blevel);
+            const float *H = hess + k * 1024;
+            const int i = (int)(bi % 32);
+            for (int j = 0; j < 32; ++j)
+                g[k * 32 + j] = fmaf(-D, H[j * 32 + i], g[k * 32 + j]);
+            ++n;
+        }
+        for (int64_t j = 0; j < cols; j += 2)
+            codes[(r * cols + j) / 2] = (uint8_t)(c[j] | (c[j + 1] << 4));
+        if (moves)
+            moves[r] = n;
+        free(u);
+        free(g);
+        free(c);
     }
     return bad ? -1 : 0;
 }

@@ -8,6 +8,8 @@ are plain library calls:
 * ``hessian_blocks``  -- H'_k = X'_k^T X'_k for every 32-column block of the
   transformed activations ("MACaQ" review, section 1: Hessian-weighted
   exponent selection uses H = X^T X);
+* ``mxfp4_flip_refine`` -- greedy adjacent-level code moves by closed-form
+  Hessian-weighted gain ("MACaQ" review, sections 1 and 3: Flip-Refinement);
 * ``channel_scale``   -- t_j = (sigma_j^W / rms_j^X)^alpha ("MACaQ" review,
   section 3: online scaling, alpha = 0.75, rms from the Hessian diagonal);
 * ``gemm_ref``        -- the W4A4 product of the dequantized operands in fp64
@@ -82,6 +84,9 @@ def lib():
             L.oracle_mxfp4_quantize.restype = ctypes.c_int
             L.oracle_mxfp4_quantize.argtypes = [f32p, i64, i64, f32p, ctypes.c_int, ctypes.c_int,
                                                 f32p, u8p, u8p, f32p, f32p]
+            L.oracle_mxfp4_flip_refine.restype = ctypes.c_int
+            L.oracle_mxfp4_flip_refine.argtypes = [f32p, i64, i64, f32p, ctypes.c_int, f32p, ctypes.c_int,
+                                                   u8p, u8p, ctypes.POINTER(ctypes.c_int32)]
             L.oracle_dequant_mse.restype = ctypes.c_int
             L.oracle_dequant_mse.argtypes = [u8p, u8p, i64, i64, ctypes.c_int, ctypes.c_int,
                                              f32p, ctypes.c_int, ctypes.c_float, f32p, f32p, f32p]
@@ -215,6 +220,30 @@ def mxfp4_quantize(x, t=None, hadamard: bool = True, rule: int = RULE_ABSMAX, he
     if rc != 0:
         raise ValueError("oracle_mxfp4_quantize rejected its arguments")
     return dict(codes=codes, scales=scales, deq=deq, mse=mse)
+
+
+def mxfp4_flip_refine(x, t, hadamard: bool, hess, codes, scales, max_moves: int = 128):
+    """Flip-Refinement of MXFP4 codes ("MACaQ" review, section 1 Key Terms and
+    section 3 Method): per output row, greedy moves of single codes to a
+    neighbouring E2M1 level by the largest closed-form decrease of
+    sum_k d_k^T H'_k d_k, at most max_moves per row.  x: weights [rows, cols]
+    (the transform with t and the Hadamard flag is applied as in
+    mxfp4_quantize); codes / scales: the MX quantization to refine (exponents
+    stay fixed).  Returns (refined codes, accepted moves per row)."""
+    x = _f32(x)
+    rows, cols = x.shape
+    tt = None if t is None else _f32(t)
+    hh = _f32(hess)
+    out = np.array(codes, np.uint8, copy=True, order="C")
+    sc = np.ascontiguousarray(scales, np.uint8)
+    moves = np.zeros(rows, np.int32)
+    rc = lib().oracle_mxfp4_flip_refine(_p(x, ctypes.c_float), rows, cols, _p(tt, ctypes.c_float),
+                                        int(bool(hadamard)), _p(hh, ctypes.c_float), int(max_moves),
+                                        _p(out, ctypes.c_uint8), _p(sc, ctypes.c_uint8),
+                                        moves.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)))
+    if rc != 0:
+        raise ValueError("oracle_mxfp4_flip_refine rejected its arguments")
+    return out, moves
 
 
 def dequant_mse(codes, scales, rows: int, cols: int, block: int, sf: int, specials=None,
