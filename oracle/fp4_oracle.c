@@ -124,16 +124,37 @@ static int nearest_code(float r, float (*value)(int), int last)
 int oracle_e4m3_encode(float r) { return nearest_code(r, oracle_e4m3_value, 0x7E); }
 int oracle_e3m3_encode(float r) { return nearest_code(r, oracle_e3m3_value, 63); }
 
+/* UE5M3, the wide-exponent block scale [Finer] compares E4M3 + 4-over-6 +
+ * hierarchical scaling against (findings: format compatibility; the page
+ * gives no bit layout).  Read as an unsigned 8-bit float: 5 exponent bits
+ * with bias 15 over 3 mantissa bits, subnormals at exponent 0, and -- as in
+ * the OCP E4M3FN convention -- the all-ones code not a number, so codes
+ * 0..254 span 0, 2^-17 .. 1.75 * 2^16 = 114688. */
+float oracle_ue5m3_value(int code)
+{
+    int e = (code >> 3) & 31, m = code & 7;
+    if (e == 0)
+        return ldexpf((float)m, -17);
+    return ldexpf(1.0f + (float)m / 8.0f, e - 15);
+}
+
+int oracle_ue5m3_encode(float r) { return nearest_code(r, oracle_ue5m3_value, 0xFE); }
+
 /* ------------------------------------------------------------------ */
 /* Shared pieces of the NVFP4 / RaZeR quantizers                        */
 /* ------------------------------------------------------------------ */
 
-enum { SF_E4M3 = 0, SF_E3M3 = 1, SF_E8M0 = 2 };
+enum { SF_E4M3 = 0, SF_E3M3 = 1, SF_E8M0 = 2, SF_UE5M3 = 3 };
 enum { RULE_ABSMAX = 0, RULE_PREVENT_ZERO = 1, RULE_FOUR_OVER_SIX = 2,
        RULE_BRUTE_FORCE = 3, RULE_HESSIAN_EXP = 4 };
 
 /* Largest finite scale of each format (448 for E4M3, 30 for E3M3). */
-static float scale_max(int sf) { return sf == SF_E3M3 ? 30.0f : 448.0f; }
+static float scale_max(int sf)
+{
+    if (sf == SF_UE5M3)
+        return 114688.0f;
+    return sf == SF_E3M3 ? 30.0f : 448.0f;
+}
 
 /* Per-tensor FP32 global scale of hierarchical scaling ([Finer] method 2):
  * g = amax / (6 * S_max), so that the largest block maps to the largest
@@ -210,11 +231,15 @@ static float block_absmax(const float *x, int n)
 static int absmax_scale_code(float a, float M, float g, int sf)
 {
     float r = a / (M * g);
+    if (sf == SF_UE5M3)
+        return oracle_ue5m3_encode(r);
     return sf == SF_E3M3 ? oracle_e3m3_encode(r) : oracle_e4m3_encode(r);
 }
 
 static float scale_value(int code, int sf)
 {
+    if (sf == SF_UE5M3)
+        return oracle_ue5m3_value(code);
     return sf == SF_E3M3 ? oracle_e3m3_value(code) : oracle_e4m3_value(code);
 }
 
@@ -232,12 +257,30 @@ static void pack_codes(const uint8_t *c, int n, uint8_t *out)
  * a row.  Outputs: codes (rows*cols/2 bytes, element 2i in the low nibble),
  * scales (rows*cols/block E4M3 bytes, row-major), deq and mse (nullable).
  * Returns 0, or -1 on a bad argument. */
+int oracle_block_fp4_quantize(const float *x, int64_t rows, int64_t cols, int block, int rule,
+                              int sf, float g, uint8_t *codes, uint8_t *scales, float *deq,
+                              float *mse);
+
 int oracle_nvfp4_quantize(const float *x, int64_t rows, int64_t cols, int block,
                           int rule, float g, uint8_t *codes, uint8_t *scales,
                           float *deq, float *mse)
 {
+    return oracle_block_fp4_quantize(x, rows, cols, block, rule, SF_E4M3, g, codes, scales, deq,
+                                     mse);
+}
+
+/* The same with the scale format as a parameter: SF_E4M3 (NVFP4) or
+ * SF_UE5M3; the rules are unchanged, brute force runs over every finite
+ * positive code of the format in ascending order. */
+int oracle_block_fp4_quantize(const float *x, int64_t rows, int64_t cols, int block, int rule,
+                              int sf, float g, uint8_t *codes, uint8_t *scales, float *deq,
+                              float *mse)
+{
     if (block != 4 && block != 8 && block != 16 && block != 32)
         return -1;
+    if (sf != SF_E4M3 && sf != SF_UE5M3)
+        return -1;
+    const int last = sf == SF_UE5M3 ? 0xFE : 0x7E;
     if (cols % block != 0 || rule < RULE_ABSMAX || rule > RULE_BRUTE_FORCE)
         return -1;
     const int64_t nblk = rows * (cols / block);
@@ -250,15 +293,15 @@ int oracle_nvfp4_quantize(const float *x, int64_t rows, int64_t cols, int block,
         int sc_code;
         float sse;
         if (rule == RULE_ABSMAX || rule == RULE_PREVENT_ZERO) {
-            sc_code = absmax_scale_code(a, 6.0f, g, SF_E4M3);
+            sc_code = absmax_scale_code(a, 6.0f, g, sf);
             if (rule == RULE_PREVENT_ZERO && sc_code == 0)
-                sc_code = 1;     /* smallest positive E4M3, 2^-9 */
-            sse = quantize_block(xb, block, oracle_e4m3_value(sc_code), g, NULL, cbest, dbest);
+                sc_code = 1;     /* smallest positive scale (E4M3: 2^-9) */
+            sse = quantize_block(xb, block, scale_value(sc_code, sf), g, NULL, cbest, dbest);
         } else if (rule == RULE_FOUR_OVER_SIX) {
-            int c6 = absmax_scale_code(a, 6.0f, g, SF_E4M3);
-            int c4 = absmax_scale_code(a, 4.0f, g, SF_E4M3);
-            float sse6 = quantize_block(xb, block, oracle_e4m3_value(c6), g, NULL, cbest, dbest);
-            float sse4 = quantize_block(xb, block, oracle_e4m3_value(c4), g, NULL, ctry, dtry);
+            int c6 = absmax_scale_code(a, 6.0f, g, sf);
+            int c4 = absmax_scale_code(a, 4.0f, g, sf);
+            float sse6 = quantize_block(xb, block, scale_value(c6, sf), g, NULL, cbest, dbest);
+            float sse4 = quantize_block(xb, block, scale_value(c4, sf), g, NULL, ctry, dtry);
             sc_code = c6;
             sse = sse6;
             if (sse4 < sse6) {
@@ -267,11 +310,11 @@ int oracle_nvfp4_quantize(const float *x, int64_t rows, int64_t cols, int block,
                 memcpy(cbest, ctry, sizeof cbest);
                 memcpy(dbest, dtry, sizeof dbest);
             }
-        } else { /* brute force: every finite positive E4M3 value, ascending */
+        } else { /* brute force: every finite positive scale, ascending */
             sc_code = -1;
             sse = 0.0f;
-            for (int c = 1; c <= 0x7E; ++c) {
-                float s = quantize_block(xb, block, oracle_e4m3_value(c), g, NULL, ctry, dtry);
+            for (int c = 1; c <= last; ++c) {
+                float s = quantize_block(xb, block, scale_value(c, sf), g, NULL, ctry, dtry);
                 if (sc_code < 0 || s < sse) {
                     sc_code = c;
                     sse = s;
@@ -629,7 +672,7 @@ int oracle_dequant_mse(const uint8_t *codes, const uint8_t *scales, int64_t rows
         return -1;
     if (sf == SF_E8M0 && (block != 32 || specials))
         return -1;
-    if (specials && block != 16)
+    if (specials && (block != 16 || sf == SF_UE5M3))
         return -1;
     if (mse && !ref)
         return -1;

@@ -33,7 +33,7 @@ _LIB_PATH = os.path.join(_HERE, "liboracle.so")
 _CFLAGS = ["-O2", "-std=gnu99", "-ffp-contract=off", "-fno-fast-math", "-fopenmp",
            "-shared", "-fPIC"]
 
-SF_E4M3, SF_E3M3, SF_E8M0 = 0, 1, 2
+SF_E4M3, SF_E3M3, SF_E8M0, SF_UE5M3 = 0, 1, 2, 3
 RULE_ABSMAX, RULE_PREVENT_ZERO, RULE_FOUR_OVER_SIX, RULE_BRUTE_FORCE, RULE_HESSIAN_EXP = range(5)
 
 _lock = threading.Lock()
@@ -61,10 +61,10 @@ def lib():
             L.oracle_e2m1_value.argtypes = [ctypes.c_int]
             L.oracle_e2m1_encode.restype = ctypes.c_int
             L.oracle_e2m1_encode.argtypes = [ctypes.c_float]
-            for name in ("oracle_e4m3_value", "oracle_e3m3_value"):
+            for name in ("oracle_e4m3_value", "oracle_e3m3_value", "oracle_ue5m3_value"):
                 getattr(L, name).restype = ctypes.c_float
                 getattr(L, name).argtypes = [ctypes.c_int]
-            for name in ("oracle_e4m3_encode", "oracle_e3m3_encode"):
+            for name in ("oracle_e4m3_encode", "oracle_e3m3_encode", "oracle_ue5m3_encode"):
                 getattr(L, name).restype = ctypes.c_int
                 getattr(L, name).argtypes = [ctypes.c_float]
             L.oracle_e8m0_value.restype = ctypes.c_double
@@ -76,6 +76,9 @@ def lib():
             L.oracle_nvfp4_quantize.restype = ctypes.c_int
             L.oracle_nvfp4_quantize.argtypes = [f32p, i64, i64, ctypes.c_int, ctypes.c_int,
                                                 ctypes.c_float, u8p, u8p, f32p, f32p]
+            L.oracle_block_fp4_quantize.restype = ctypes.c_int
+            L.oracle_block_fp4_quantize.argtypes = [f32p, i64, i64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                                    ctypes.c_float, u8p, u8p, f32p, f32p]
             L.oracle_razer_quantize.restype = ctypes.c_int
             L.oracle_razer_quantize.argtypes = [f32p, i64, i64, ctypes.c_int, f32p, ctypes.c_int,
                                                 ctypes.c_float, u8p, u8p, f32p, f32p]
@@ -119,6 +122,14 @@ def get_threads() -> int:
 # ---------------------------------------------------------------- formats
 def e2m1_value(code: int) -> float:
     return float(lib().oracle_e2m1_value(int(code)))
+
+
+def ue5m3_value(code: int) -> float:
+    return float(lib().oracle_ue5m3_value(int(code)))
+
+
+def ue5m3_encode(r: float) -> int:
+    return int(lib().oracle_ue5m3_encode(float(np.float32(r))))
 
 
 def e2m1_encode(y: float) -> int:
@@ -169,6 +180,25 @@ def nvfp4_quantize(x, block: int, rule: int, g: float = 1.0, want_deq=True, want
                                      _p(mse, ctypes.c_float))
     if rc != 0:
         raise ValueError("oracle_nvfp4_quantize rejected its arguments")
+    return dict(codes=codes, scales=scales, deq=deq, mse=mse)
+
+
+def block_fp4_quantize(x, block: int, rule: int, sf: int = SF_E4M3, g: float = 1.0, want_deq=True,
+                       want_mse=True):
+    """nvfp4_quantize with the block-scale format as a parameter (SF_E4M3 or
+    SF_UE5M3, the wide-exponent scale of the "Finer is Better" summary)."""
+    x = _f32(x)
+    rows, cols = x.shape
+    codes = np.zeros((rows, cols // 2), np.uint8)
+    scales = np.zeros((rows, cols // block), np.uint8)
+    deq = np.zeros((rows, cols), np.float32) if want_deq else None
+    mse = np.zeros((rows, cols // block), np.float32) if want_mse else None
+    rc = lib().oracle_block_fp4_quantize(_p(x, ctypes.c_float), rows, cols, block, rule, sf,
+                                         float(np.float32(g)), _p(codes, ctypes.c_uint8),
+                                         _p(scales, ctypes.c_uint8), _p(deq, ctypes.c_float),
+                                         _p(mse, ctypes.c_float))
+    if rc != 0:
+        raise ValueError("oracle_block_fp4_quantize rejected its arguments")
     return dict(codes=codes, scales=scales, deq=deq, mse=mse)
 
 
