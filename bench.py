@@ -5,12 +5,15 @@ One step = one pass over every hot-path row at its workload size:
       hierarchical scale, with dequant + per-block MSE        (amax, quantize)
   c2  block sizes {4,8,16,32} x rules {abs-max, prevent-zero, 4-over-6,
       brute force} on 8192x8192 fp32 Student-t(3)*1e-3, g = 1, codes +
-      scales + per-block MSE                                  (16 quantizations)
+      scales + per-block MSE                                  (16 quantizations),
+      and per block size the scale-format comparison: UE5M3 abs-max and
+      4-over-6 (g = 1) against E4M3 4-over-6 with hierarchical scaling (12)
   c3  RaZeR: 8192x8192 bf16 weights (E3M3 + 4 specials) and 16384x4096 bf16
       activations (E4M3 + 2 specials), hierarchical scale
   c4  MXFP4 prep: channel scale t from 8192x4096 bf16 activations and
       4096x4096 bf16 weights, Hessian blocks H', activation quantize (t,
-      Hadamard-32, E8M0), weight quantize with the Hessian-weighted exponent
+      Hadamard-32, E8M0), weight quantize with the Hessian-weighted exponent,
+      Flip-Refinement of the weight codes (128 moves per row)
   c5  W4A4 GEMM M=8192 x K=4096 x N=14336 -> bf16: dynamic 4-over-6 NVFP4
       quantize of the bf16 activations into the MMA scale layout, then the
       tcgen05 block-scaled GEMM on weights quantized once beforehand
@@ -39,7 +42,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "FP4 quantize Gelem/s & % of HBM roofline; W4A4 GEMM TFLOP/s & % FP4 peak"
-WORKLOAD = "hot path: one pass of every row (NVFP4 4096^2 PZ; 8192^2 block-size x rule sweep; RaZeR W 8192^2 + A 16384x4096; MXFP4 prep 8192x4096 + 4096^2; W4A4 GEMM 8192x14336x4096 with 4-over-6 activation quant)"
+WORKLOAD = "hot path: one pass of every row (NVFP4 4096^2 PZ; 8192^2 block-size x rule sweep + UE5M3 / hierarchical-E4M3 comparison; RaZeR W 8192^2 + A 16384x4096; MXFP4 prep 8192x4096 + 4096^2 with Flip-Refinement; W4A4 GEMM 8192x14336x4096 with 4-over-6 activation quant)"
 SM_COUNT = 148
 FP32_LANES_PER_SM = 128
 
@@ -68,9 +71,10 @@ class Row:
         self.eval_ws, self.block = eval_ws, block
 
 
-def build_rows(torch, fq, inputs, dev, host_copies=None):
+def build_rows(torch, fq, inputs, dev, host_copies=None, groups=None):
     """Create the step's device buffers and rows.  host_copies (dict) receives
-    the host arrays that an end-to-end run copies in each step."""
+    the host arrays that an end-to-end run copies in each step; groups (a set
+    of "c1".."c5", default all) limits which workloads are built."""
     def to_dev(a, key):
         if host_copies is not None:
             host_copies[key] = a
@@ -80,106 +84,133 @@ def build_rows(torch, fq, inputs, dev, host_copies=None):
 
     rows = []
     X = {}
-    # c1
-    a1 = inputs.generate("gaussian")
-    X["c1"] = to_dev(a1, "c1")
-    n1 = a1.size
-    o1 = {}
-    ws1 = torch.empty(fq.workspace_size(fq.OP_QUANTIZE, *a1.shape), dtype=torch.uint8, device=dev)
+    if groups is None or "c1" in groups:
+        # c1
+        a1 = inputs.generate("gaussian")
+        X["c1"] = to_dev(a1, "c1")
+        n1 = a1.size
+        o1 = {}
+        ws1 = torch.empty(fq.workspace_size(fq.OP_QUANTIZE, *a1.shape), dtype=torch.uint8, device=dev)
 
-    def c1():
-        o1.update(fq.nvfp4_quantize(X["c1"], 16, fq.PREVENT_ZERO, gs_mode=fq.GS_AMAX, dequant=True,
-                                    mse=True, out=o1, workspace=ws1))
-    rows.append(Row("c1_nvfp4_pz_deq_mse", "nvfp4_quant_kernel<16, float, 1>", n1, n1 * (4 + 0.5 + 1 / 16 + 4 + 4 / 16), 2, c1, o1))
-    # c2
-    a2 = inputs.generate("student_t")
-    X["c2"] = to_dev(a2, "c2")
-    n2 = a2.size
-    names = {fq.ABSMAX: "absmax", fq.PREVENT_ZERO: "pz", fq.FOUR_OVER_SIX: "4o6", fq.BRUTE_FORCE: "bf"}
-    for B in (4, 8, 16, 32):
-        for rule in (fq.ABSMAX, fq.PREVENT_ZERO, fq.FOUR_OVER_SIX, fq.BRUTE_FORCE):
-            o = {}
-            bf = rule == fq.BRUTE_FORCE
-            wsr = torch.zeros(fq.workspace_size(fq.OP_QUANTIZE, 1, 1), dtype=torch.uint8, device=dev) if bf else None
+        def c1():
+            o1.update(fq.nvfp4_quantize(X["c1"], 16, fq.PREVENT_ZERO, gs_mode=fq.GS_AMAX, dequant=True,
+                                        mse=True, out=o1, workspace=ws1))
+        rows.append(Row("c1_nvfp4_pz_deq_mse", "nvfp4_quant_kernel<16, float, 1>", n1, n1 * (4 + 0.5 + 1 / 16 + 4 + 4 / 16), 2, c1, o1))
+    if groups is None or "c2" in groups:
+        # c2
+        a2 = inputs.generate("student_t")
+        X["c2"] = to_dev(a2, "c2")
+        n2 = a2.size
+        names = {fq.ABSMAX: "absmax", fq.PREVENT_ZERO: "pz", fq.FOUR_OVER_SIX: "4o6", fq.BRUTE_FORCE: "bf"}
+        for B in (4, 8, 16, 32):
+            for rule in (fq.ABSMAX, fq.PREVENT_ZERO, fq.FOUR_OVER_SIX, fq.BRUTE_FORCE):
+                o = {}
+                bf = rule == fq.BRUTE_FORCE
+                wsr = torch.zeros(fq.workspace_size(fq.OP_QUANTIZE, 1, 1), dtype=torch.uint8, device=dev) if bf else None
 
-            def c2(B=B, rule=rule, o=o, wsr=wsr):
-                o.update(fq.nvfp4_quantize(X["c2"], B, rule, gs_mode=fq.GS_NONE, mse=True, out=o, workspace=wsr))
-            kern = ("nvfp4_bf_kernel<%d, float>" % B) if bf else ("nvfp4_quant_kernel<%d, float, %d>" % (B, rule))
-            rows.append(Row("c2_B%d_%s" % (B, names[rule]), kern,
-                            n2, n2 * (4 + 0.5 + 1 / B + 4 / B), 1, c2, o,
-                            bound="alu" if bf else "hbm", eval_ws=wsr, block=B))
-    # c3
-    w3 = inputs.generate("razer_weight")
-    X["c3w"] = to_dev(w3, "c3w")
-    a3 = inputs.generate("razer_act")
-    X["c3a"] = to_dev(a3, "c3a")
-    ws3 = torch.empty(fq.workspace_size(fq.OP_QUANTIZE, 1, 1), dtype=torch.uint8, device=dev)
-    o3w, o3a = {}, {}
+                def c2(B=B, rule=rule, o=o, wsr=wsr):
+                    o.update(fq.nvfp4_quantize(X["c2"], B, rule, gs_mode=fq.GS_NONE, mse=True, out=o, workspace=wsr))
+                kern = ("nvfp4_bf_kernel<%d, float>" % B) if bf else ("nvfp4_quant_kernel<%d, float, %d>" % (B, rule))
+                rows.append(Row("c2_B%d_%s" % (B, names[rule]), kern,
+                                n2, n2 * (4 + 0.5 + 1 / B + 4 / B), 1, c2, o,
+                                bound="alu" if bf else "hbm", eval_ws=wsr, block=B))
+        # the summary's comparison: UE5M3 block scales without a global scale
+        # against E4M3 with 4-over-6 and hierarchical (global) scaling
+        wsh2 = torch.empty(fq.workspace_size(fq.OP_QUANTIZE, 1, 1), dtype=torch.uint8, device=dev)
+        for B in (4, 8, 16, 32):
+            for tag, rule, sfmt, gsm in (("ue5m3_absmax", fq.ABSMAX, fq.SF_UE5M3, fq.GS_NONE),
+                                         ("ue5m3_4o6", fq.FOUR_OVER_SIX, fq.SF_UE5M3, fq.GS_NONE),
+                                         ("e4m3_4o6_hier", fq.FOUR_OVER_SIX, fq.SF_E4M3, fq.GS_AMAX)):
+                o = {}
 
-    def c3w():
-        o3w.update(fq.razer_quantize(X["c3w"], fq.SF_E3M3, [5.0, -5.0, 3.5, -3.5], gs_mode=fq.GS_AMAX, out=o3w, workspace=ws3))
+                def c2x(B=B, rule=rule, sfmt=sfmt, gsm=gsm, o=o):
+                    o.update(fq.nvfp4_quantize(X["c2"], B, rule, gs_mode=gsm, mse=True, out=o, scale_fmt=sfmt,
+                                               workspace=wsh2 if gsm == fq.GS_AMAX else None))
+                rows.append(Row("c2_B%d_%s" % (B, tag),
+                                "nvfp4_quant_kernel<%d, float, %d, %d>" % (B, rule, 1 if sfmt == fq.SF_UE5M3 else 0),
+                                n2, n2 * (4 + 0.5 + 1 / B + 4 / B), 2 if gsm == fq.GS_AMAX else 1, c2x, o))
+    if groups is None or "c3" in groups:
+        # c3
+        w3 = inputs.generate("razer_weight")
+        X["c3w"] = to_dev(w3, "c3w")
+        a3 = inputs.generate("razer_act")
+        X["c3a"] = to_dev(a3, "c3a")
+        ws3 = torch.empty(fq.workspace_size(fq.OP_QUANTIZE, 1, 1), dtype=torch.uint8, device=dev)
+        o3w, o3a = {}, {}
 
-    def c3a():
-        o3a.update(fq.razer_quantize(X["c3a"], fq.SF_E4M3, [5.0, -5.0], gs_mode=fq.GS_AMAX, out=o3a, workspace=ws3))
-    rows.append(Row("c3_razer_weight", "razer_quant_kernel<__nv_bfloat16, 1>", w3.size, w3.size * (2 + 0.5 + 1 / 16), 2, c3w, o3w))
-    rows.append(Row("c3_razer_act", "razer_quant_kernel<__nv_bfloat16, 0>", a3.size, a3.size * (2 + 0.5 + 1 / 16), 2, c3a, o3a))
-    # c4
-    x4 = inputs.generate("mx_act")
-    w4 = inputs.generate("mx_weight")
-    X["c4x"] = to_dev(x4, "c4x")
-    X["c4w"] = to_dev(w4, "c4w")
-    T, C = x4.shape
-    N4 = w4.shape[0]
-    t4 = torch.empty(C, dtype=torch.float32, device=dev)
-    ti4 = torch.empty(C, dtype=torch.float32, device=dev)
-    h4 = torch.empty((C // 32, 32, 32), dtype=torch.float32, device=dev)
-    wsc = torch.empty(fq.workspace_size(fq.OP_CHANNEL_SCALE, T, C, N4), dtype=torch.uint8, device=dev)
-    wsh = torch.empty(fq.workspace_size(fq.OP_HESSIAN, T, C), dtype=torch.uint8, device=dev)
-    o4a, o4w = {}, {}
+        def c3w():
+            o3w.update(fq.razer_quantize(X["c3w"], fq.SF_E3M3, [5.0, -5.0, 3.5, -3.5], gs_mode=fq.GS_AMAX, out=o3w, workspace=ws3))
 
-    def c4s():
-        fq.channel_scale(X["c4x"], X["c4w"], 0.75, out=(t4, ti4), workspace=wsc)
+        def c3a():
+            o3a.update(fq.razer_quantize(X["c3a"], fq.SF_E4M3, [5.0, -5.0], gs_mode=fq.GS_AMAX, out=o3a, workspace=ws3))
+        rows.append(Row("c3_razer_weight", "razer_quant_kernel<__nv_bfloat16, 1>", w3.size, w3.size * (2 + 0.5 + 1 / 16), 2, c3w, o3w))
+        rows.append(Row("c3_razer_act", "razer_quant_kernel<__nv_bfloat16, 0>", a3.size, a3.size * (2 + 0.5 + 1 / 16), 2, c3a, o3a))
+    if groups is None or "c4" in groups:
+        # c4
+        x4 = inputs.generate("mx_act")
+        w4 = inputs.generate("mx_weight")
+        X["c4x"] = to_dev(x4, "c4x")
+        X["c4w"] = to_dev(w4, "c4w")
+        T, C = x4.shape
+        N4 = w4.shape[0]
+        t4 = torch.empty(C, dtype=torch.float32, device=dev)
+        ti4 = torch.empty(C, dtype=torch.float32, device=dev)
+        h4 = torch.empty((C // 32, 32, 32), dtype=torch.float32, device=dev)
+        wsc = torch.empty(fq.workspace_size(fq.OP_CHANNEL_SCALE, T, C, N4), dtype=torch.uint8, device=dev)
+        wsh = torch.empty(fq.workspace_size(fq.OP_HESSIAN, T, C), dtype=torch.uint8, device=dev)
+        o4a, o4w = {}, {}
 
-    def c4h():
-        fq.hessian_blocks(X["c4x"], t4, True, out=h4, workspace=wsh)
+        def c4s():
+            fq.channel_scale(X["c4x"], X["c4w"], 0.75, out=(t4, ti4), workspace=wsc)
 
-    def c4a():
-        o4a.update(fq.mxfp4_quantize(X["c4x"], t4, True, fq.ABSMAX, out=o4a))
+        def c4h():
+            fq.hessian_blocks(X["c4x"], t4, True, out=h4, workspace=wsh)
 
-    def c4w():
-        o4w.update(fq.mxfp4_quantize(X["c4w"], ti4, True, fq.HESSIAN_EXP, hess=h4, out=o4w))
-    rows.append(Row("c4_channel_scale", "column_stats_kernel", 0, x4.size * 2 + w4.size * 2, 3, c4s, {"t": t4, "t_inv": ti4}))
-    rows.append(Row("c4_hessian_blocks", "hessian_partial_kernel", 0, x4.size * 2 + C * 32 * 4, 2, c4h,
-                    {"hess": h4}, flops=2.0 * T * C * 32))
-    rows.append(Row("c4_mx_act", "mx_quant_absmax_kernel", x4.size, x4.size * (2 + 0.5 + 1 / 32), 1, c4a, o4a))
-    rows.append(Row("c4_mx_weight_hessian", "mx_quant_hessian_kernel", w4.size, w4.size * (2 + 0.5 + 1 / 32) + C * 32 * 4,
-                    1, c4w, o4w, bound="alu", flops=2.0 * 3 * N4 * (C // 32) * 32 * 32))
-    # c5: weights pre-quantized once (abs-max NVFP4, hierarchical scale, MMA
-    # scale layout) outside the timed step; the step quantizes the activations
-    # (4-over-6, MMA layout) and runs the tcgen05 GEMM on the packed operands
-    a5 = inputs.generate("gemm_act")
-    X["c5"] = to_dev(a5, "c5")
-    w5 = inputs.generate("gemm_weight")
-    w5d = torch.from_numpy(w5.view(np.int16)).to(dev).view(torch.bfloat16)
-    M5, K5 = a5.shape
-    N5 = w5.shape[0]
-    qw5 = fq.nvfp4_quantize(w5d, 16, fq.ABSMAX, gs_mode=fq.GS_AMAX, sf_layout=fq.SF_MMA)
-    del w5d
-    ws5 = torch.empty(fq.workspace_size(fq.OP_QUANTIZE, 1, 1), dtype=torch.uint8, device=dev)
-    wsg = torch.empty(fq.workspace_size(fq.OP_GEMM, 128, 256, 256), dtype=torch.uint8, device=dev)
-    o5 = {}
-    y5 = torch.empty((M5, N5), dtype=torch.bfloat16, device=dev)
+        def c4a():
+            o4a.update(fq.mxfp4_quantize(X["c4x"], t4, True, fq.ABSMAX, out=o4a))
 
-    def c5():
-        o5.update(fq.nvfp4_quantize(X["c5"], 16, fq.FOUR_OVER_SIX, gs_mode=fq.GS_AMAX, sf_layout=fq.SF_MMA,
-                                    out=o5, workspace=ws5))
+        def c4w():
+            o4w.update(fq.mxfp4_quantize(X["c4w"], ti4, True, fq.HESSIAN_EXP, hess=h4, out=o4w))
+        rows.append(Row("c4_channel_scale", "column_stats_kernel", 0, x4.size * 2 + w4.size * 2, 3, c4s, {"t": t4, "t_inv": ti4}))
+        rows.append(Row("c4_hessian_blocks", "hessian_partial_kernel", 0, x4.size * 2 + C * 32 * 4, 2, c4h,
+                        {"hess": h4}, flops=2.0 * T * C * 32))
+        rows.append(Row("c4_mx_act", "mx_quant_absmax_kernel", x4.size, x4.size * (2 + 0.5 + 1 / 32), 1, c4a, o4a))
+        rows.append(Row("c4_mx_weight_hessian", "mx_quant_hessian_kernel", w4.size, w4.size * (2 + 0.5 + 1 / 32) + C * 32 * 4,
+                        1, c4w, o4w, bound="alu", flops=2.0 * 3 * N4 * (C // 32) * 32 * 32))
+        # Flip-Refinement of those weight codes, the pages' K = 128 moves per row
+        mv4 = torch.empty(N4, dtype=torch.int32, device=dev)
 
-    def c5g():
-        fq.w4a4_gemm(o5["codes"], qw5["codes"], qw5["scales"], qw5["global_scale"], a_scales=o5["scales"],
-                     a_global_scale=o5["global_scale"], K=K5, out=y5, workspace=wsg)
-    rows.append(Row("c5_act_quant_4o6_mma", "nvfp4_quant_kernel<16, __nv_bfloat16, 2>", a5.size, a5.size * (2 + 0.5 + 1 / 16), 2, c5, o5))
-    rows.append(Row("c5_w4a4_gemm", "w4a4_gemm_kernel", 0, M5 * K5 * (0.5 + 1 / 16) + N5 * K5 * (0.5 + 1 / 16) + M5 * N5 * 2,
-                    1, c5g, {"out": y5}, bound="tensor", flops=2.0 * M5 * N5 * K5))
+        def c4f():
+            fq.mxfp4_flip_refine(X["c4w"], o4w["codes"], o4w["scales"], h4, chan_scale=ti4, max_moves=128, moves=mv4)
+        rows.append(Row("c4_mx_weight_flip", "flip_refine_kernel", 0, w4.size * (2 + 0.5 + 0.5 + 1 / 32) + C * 32 * 4,
+                        1, c4f, {"moves": mv4}, bound="alu", flops=2.0 * N4 * (C // 32) * 32 * 32))
+    if groups is None or "c5" in groups:
+        # c5: weights pre-quantized once (abs-max NVFP4, hierarchical scale, MMA
+        # scale layout) outside the timed step; the step quantizes the activations
+        # (4-over-6, MMA layout) and runs the tcgen05 GEMM on the packed operands
+        a5 = inputs.generate("gemm_act")
+        X["c5"] = to_dev(a5, "c5")
+        w5 = inputs.generate("gemm_weight")
+        w5d = torch.from_numpy(w5.view(np.int16)).to(dev).view(torch.bfloat16)
+        M5, K5 = a5.shape
+        N5 = w5.shape[0]
+        qw5 = fq.nvfp4_quantize(w5d, 16, fq.ABSMAX, gs_mode=fq.GS_AMAX, sf_layout=fq.SF_MMA)
+        del w5d
+        ws5 = torch.empty(fq.workspace_size(fq.OP_QUANTIZE, 1, 1), dtype=torch.uint8, device=dev)
+        wsg = torch.empty(fq.workspace_size(fq.OP_GEMM, 128, 256, 256), dtype=torch.uint8, device=dev)
+        o5 = {}
+        y5 = torch.empty((M5, N5), dtype=torch.bfloat16, device=dev)
+
+        def c5():
+            o5.update(fq.nvfp4_quantize(X["c5"], 16, fq.FOUR_OVER_SIX, gs_mode=fq.GS_AMAX, sf_layout=fq.SF_MMA,
+                                        out=o5, workspace=ws5))
+
+        def c5g():
+            fq.w4a4_gemm(o5["codes"], qw5["codes"], qw5["scales"], qw5["global_scale"], a_scales=o5["scales"],
+                         a_global_scale=o5["global_scale"], K=K5, out=y5, workspace=wsg)
+        rows.append(Row("c5_act_quant_4o6_mma", "nvfp4_quant_kernel<16, __nv_bfloat16, 2>", a5.size, a5.size * (2 + 0.5 + 1 / 16), 2, c5, o5))
+        rows.append(Row("c5_w4a4_gemm", "w4a4_gemm_kernel", 0, M5 * K5 * (0.5 + 1 / 16) + N5 * K5 * (0.5 + 1 / 16) + M5 * N5 * 2,
+                        1, c5g, {"out": y5}, bound="tensor", flops=2.0 * M5 * N5 * K5))
     return rows, X
 
 
@@ -264,23 +295,29 @@ def oracle_sample_run(O, S):
     for B in (4, 8, 16, 32):
         for rule in range(4):
             O.nvfp4_quantize(S["c2"], B, rule, g=1.0, want_deq=False)
+    g2 = O.global_scale(O.amax(S["c2"]))
+    for B in (4, 8, 16, 32):
+        O.block_fp4_quantize(S["c2"], B, O.RULE_ABSMAX, O.SF_UE5M3, 1.0, want_deq=False)
+        O.block_fp4_quantize(S["c2"], B, O.RULE_FOUR_OVER_SIX, O.SF_UE5M3, 1.0, want_deq=False)
+        O.nvfp4_quantize(S["c2"], B, O.RULE_FOUR_OVER_SIX, g=g2, want_deq=False)
     O.razer_quantize(S["c3w"], O.SF_E3M3, [5.0, -5.0, 3.5, -3.5], g=O.global_scale(O.amax(S["c3w"]), O.SF_E3M3),
                      want_deq=False)
     O.razer_quantize(S["c3a"], O.SF_E4M3, [5.0, -5.0], g=O.global_scale(O.amax(S["c3a"]), O.SF_E4M3), want_deq=False)
     t, ti = O.channel_scale(S["c4x"], S["c4w"], 0.75)
     hb = O.hessian_blocks(S["c4x"], t, True).astype(np.float32)
     O.mxfp4_quantize(S["c4x"], t, True, O.RULE_ABSMAX, want_deq=False)
-    O.mxfp4_quantize(S["c4w"], ti, True, O.RULE_HESSIAN_EXP, hb, want_deq=False)
+    qw4 = O.mxfp4_quantize(S["c4w"], ti, True, O.RULE_HESSIAN_EXP, hb, want_deq=False)
+    O.mxfp4_flip_refine(S["c4w"], ti, True, hb, qw4["codes"], qw4["scales"], 128)
     ga = O.global_scale(O.amax(S["c5"]))
     qa = O.nvfp4_quantize(S["c5"], 16, O.RULE_FOUR_OVER_SIX, g=ga, want_deq=False, want_mse=False)
     qw, gw = S["c5q"]
     O.gemm_ref(qa["codes"], qa["scales"], ga, qw["codes"], qw["scales"], gw)
-    elems = (S["c1"].size + 16 * S["c2"].size + S["c3w"].size + S["c3a"].size + S["c4x"].size + S["c4w"].size
+    elems = (S["c1"].size + 28 * S["c2"].size + S["c3w"].size + S["c3a"].size + S["c4x"].size + S["c4w"].size
              + S["c5"].size)
     return elems, time.perf_counter() - t0
 
 
-FULL_ELEMS = 4096 * 4096 + 16 * 8192 * 8192 + 8192 * 8192 + 16384 * 4096 + 8192 * 4096 + 4096 * 4096 + 8192 * 4096
+FULL_ELEMS = 4096 * 4096 + 28 * 8192 * 8192 + 8192 * 8192 + 16384 * 4096 + 8192 * 4096 + 4096 * 4096 + 8192 * 4096
 SAMPLE_ROWS = {"c1": 1 / 4, "c2": 1 / 4, "c3": 1 / 4, "c4": 1 / 4, "c5": 1 / 4}
 
 
@@ -322,6 +359,10 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-row", default=None,
+                    help="for profiler captures: build only this row's workload group, run the group once, "
+                         "then the row --reps times; prints no JSON")
+    ap.add_argument("--reps", type=int, default=2)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -343,6 +384,19 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     fq.lib(build_if_missing=True)
     hbm_peak, sm_max_mhz, bf16_peak, bf16_sust, peak_src = load_peaks()
+
+    if args.profile_row:
+        rows, X = build_rows(torch, fq, inputs, dev, None, groups={args.profile_row[:2]})
+        target = [r for r in rows if r.name == args.profile_row]
+        if not target:
+            raise SystemExit("unknown row %s; rows: %s" % (args.profile_row, [r.name for r in rows]))
+        for r in rows:
+            r.fn()
+        for _ in range(args.reps):
+            target[0].fn()
+        torch.cuda.synchronize()
+        print("profiled row", args.profile_row, "x", args.reps)
+        return 0
 
     host = {}
     rows, X = build_rows(torch, fq, inputs, dev, host)

@@ -16,7 +16,7 @@ import torch
 from . import build as _build
 
 F32, BF16, NVFP4_PACKED = 0, 1, 2
-SF_E4M3, SF_E3M3, SF_E8M0 = 0, 1, 2
+SF_E4M3, SF_E3M3, SF_E8M0, SF_UE5M3 = 0, 1, 2, 3
 ABSMAX, PREVENT_ZERO, FOUR_OVER_SIX, BRUTE_FORCE, HESSIAN_EXP = range(5)
 GS_NONE, GS_AMAX, GS_GIVEN = 0, 1, 2
 SF_ROWMAJOR, SF_MMA = 0, 1
@@ -32,8 +32,10 @@ SIGNATURES = {
     "fp4q_status_str": (ctypes.c_char_p, [_i]),
     "fp4q_version": (ctypes.c_char_p, []),
     "nvfp4_quantize": (_i, [_vp, _i, _i64, _i64, _i, _i, _i, _vp, _vp, _vp, _i, _vp, _vp, _vp, _sz, _vp]),
+    "fp4_block_quantize": (_i, [_vp, _i, _i64, _i64, _i, _i, _i, _i, _vp, _vp, _vp, _i, _vp, _vp, _vp, _sz, _vp]),
     "razer_quantize": (_i, [_vp, _i, _i64, _i64, _i, _vp, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "mxfp4_quantize": (_i, [_vp, _i, _i64, _i64, _vp, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "mxfp4_flip_refine": (_i, [_vp, _i, _i64, _i64, _vp, _i, _vp, _i, _vp, _vp, _vp, _vp]),
     "fp4_hessian_blocks": (_i, [_vp, _i, _i64, _i64, _vp, _i, _vp, _vp, _sz, _vp]),
     "fp4_hessian_blocks_noalloc": (_i, [_vp, _i, _i64, _i64, _vp, _i, _vp, _vp]),
     "mxfp4_channel_scale": (_i, [_vp, _i, _i64, _vp, _i, _i64, _i64, _fp, _vp, _vp, _vp, _sz, _vp]),
@@ -118,8 +120,10 @@ def _workspace(op, rows, cols, n, device, ws):
 def nvfp4_quantize(x: torch.Tensor, block: int = 16, rule: int = ABSMAX, gs_mode: int = GS_AMAX,
                    global_scale: torch.Tensor | None = None, sf_layout: int = SF_ROWMAJOR,
                    dequant: bool = False, mse: bool = False, out: dict | None = None,
-                   workspace: torch.Tensor | None = None, stream=None) -> dict:
-    """NVFP4 block quantization; returns dict(codes, scales, global_scale, dequant, mse)."""
+                   workspace: torch.Tensor | None = None, stream=None, scale_fmt: int = SF_E4M3) -> dict:
+    """NVFP4 block quantization; returns dict(codes, scales, global_scale, dequant, mse).
+    scale_fmt=SF_UE5M3 runs the same rules with UE5M3 block scales
+    (fp4_block_quantize)."""
     _need_cuda(x)
     rows, cols = x.shape
     dev = x.device
@@ -133,10 +137,16 @@ def nvfp4_quantize(x: torch.Tensor, block: int = 16, rule: int = ABSMAX, gs_mode
     ws, wsb = (workspace, workspace.numel()) if workspace is not None else (
         _workspace(OP_QUANTIZE, rows, cols, 0, dev, None) if gs_mode == GS_AMAX else (None, 0))
     _need_cuda(codes, scales, global_scale, dq, ms, ws)
-    st = lib().nvfp4_quantize(_ptr(x), _dtype_code(x), rows, cols, block, rule, gs_mode,
-                              _ptr(global_scale), _ptr(codes), _ptr(scales), sf_layout, _ptr(dq),
-                              _ptr(ms), _ptr(ws), wsb, _stream(stream))
-    _check(st, "nvfp4_quantize")
+    if scale_fmt == SF_E4M3:
+        st = lib().nvfp4_quantize(_ptr(x), _dtype_code(x), rows, cols, block, rule, gs_mode,
+                                  _ptr(global_scale), _ptr(codes), _ptr(scales), sf_layout, _ptr(dq),
+                                  _ptr(ms), _ptr(ws), wsb, _stream(stream))
+        _check(st, "nvfp4_quantize")
+    else:
+        st = lib().fp4_block_quantize(_ptr(x), _dtype_code(x), rows, cols, block, rule, scale_fmt, gs_mode,
+                                      _ptr(global_scale), _ptr(codes), _ptr(scales), sf_layout, _ptr(dq),
+                                      _ptr(ms), _ptr(ws), wsb, _stream(stream))
+        _check(st, "fp4_block_quantize")
     return dict(codes=codes, scales=scales, global_scale=global_scale, dequant=dq, mse=ms)
 
 
@@ -182,6 +192,20 @@ def mxfp4_quantize(x: torch.Tensor, chan_scale: torch.Tensor | None = None, hada
                               _stream(stream))
     _check(st, "mxfp4_quantize")
     return dict(codes=codes, scales=scales, dequant=dq, mse=ms)
+
+
+def mxfp4_flip_refine(w: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, hess: torch.Tensor,
+                      chan_scale: torch.Tensor | None = None, hadamard: bool = True, max_moves: int = 128,
+                      moves: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Flip-Refinement of MXFP4 codes in place (exponents fixed); returns the
+    int32 [rows] count of moves each row took."""
+    _need_cuda(w, codes, scales, hess, chan_scale)
+    rows, cols = w.shape
+    mv = moves if moves is not None else torch.empty(rows, dtype=torch.int32, device=w.device)
+    st = lib().mxfp4_flip_refine(_ptr(w), _dtype_code(w), rows, cols, _ptr(chan_scale), int(bool(hadamard)),
+                                 _ptr(hess), int(max_moves), _ptr(codes), _ptr(scales), _ptr(mv), _stream(stream))
+    _check(st, "mxfp4_flip_refine")
+    return mv
 
 
 def hessian_blocks(x: torch.Tensor, chan_scale: torch.Tensor | None = None, hadamard: bool = True,

@@ -20,6 +20,10 @@ cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 int from_cuda(cudaError_t e) { return e == cudaSuccess ? FP4Q_OK : FP4Q_ERR_CUDA; }
 
 constexpr size_t kQuantWs = 4096;   // >= kAmaxPartials floats, rounded up
+// Flip-Refinement: a row's state lives in shared memory (5 bytes per column
+// per row, 4 rows per CTA), and a row's move budget is bounded
+constexpr int64_t kFlipMaxCols = 8192;
+constexpr int kFlipMaxMoves = 1 << 20;
 // GEMM workspace: [0, 4096) amax partials, 4096 g_a, 4160 error word, then the
 // quantized A (codes, then MMA-layout scales) from 8192 on.
 constexpr size_t kGemmHeader = 8192;
@@ -91,11 +95,14 @@ const char* fp4q_status_str(int status)
 
 const char* fp4q_version(void) { return "fp4q 0.1.0 sm_100a"; }
 
-int nvfp4_quantize(const void* x, int dtype, int64_t rows, int64_t cols, int block, int rule,
-                   int gs_mode, float* global_scale, uint8_t* codes, uint8_t* scales,
-                   int sf_layout, float* dequant, float* block_mse, void* workspace,
-                   size_t workspace_bytes, void* stream)
+int fp4_block_quantize(const void* x, int dtype, int64_t rows, int64_t cols, int block, int rule,
+                       int scale_fmt, int gs_mode, float* global_scale, uint8_t* codes,
+                       uint8_t* scales, int sf_layout, float* dequant, float* block_mse,
+                       void* workspace, size_t workspace_bytes, void* stream)
 {
+    if (scale_fmt != FP4Q_SF_E4M3 && scale_fmt != FP4Q_SF_UE5M3)
+        return FP4Q_ERR_ARG;
+    const bool ue5m3 = scale_fmt == FP4Q_SF_UE5M3;
     const bool empty = rows == 0 || cols == 0;   // empty tensors may come with NULL buffers
     if ((!empty && (!x || !codes || !scales)) || !valid_dtype(dtype) || rows < 0 || cols < 0)
         return FP4Q_ERR_ARG;
@@ -106,7 +113,7 @@ int nvfp4_quantize(const void* x, int dtype, int64_t rows, int64_t cols, int blo
     if (gs_mode < FP4Q_GS_NONE || gs_mode > FP4Q_GS_GIVEN)
         return FP4Q_ERR_ARG;
     if (sf_layout == FP4Q_SFLAYOUT_MMA) {
-        if (block != 16 || rows % 128 != 0 || (cols / 16) % 4 != 0)
+        if (ue5m3 || block != 16 || rows % 128 != 0 || (cols / 16) % 4 != 0)
             return FP4Q_ERR_ARG;
     } else if (sf_layout != FP4Q_SFLAYOUT_ROWMAJOR) {
         return FP4Q_ERR_ARG;
@@ -116,7 +123,7 @@ int nvfp4_quantize(const void* x, int dtype, int64_t rows, int64_t cols, int blo
         return FP4Q_ERR_ALIGN;
     cudaStream_t s = as_stream(stream);
     GsArgs gs;
-    int st = prepare_gs(gs_mode, 2688.0f, x, dtype, rows * cols, global_scale, workspace,
+    int st = prepare_gs(gs_mode, ue5m3 ? 6.0f * 114688.0f : 2688.0f, x, dtype, rows * cols, global_scale, workspace,
                         workspace_bytes, s, gs);
     if (st != FP4Q_OK)
         return st;
@@ -125,7 +132,18 @@ int nvfp4_quantize(const void* x, int dtype, int64_t rows, int64_t cols, int blo
             ? reinterpret_cast<unsigned long long*>(static_cast<uint8_t*>(workspace) + FP4Q_WS_BF_EVALS)
             : nullptr;
     return from_cuda(launch_nvfp4_quant(x, dtype, rows, cols, block, rule, gs, codes, scales,
-                                        sf_layout == FP4Q_SFLAYOUT_MMA, dequant, block_mse, evals, s));
+                                        sf_layout == FP4Q_SFLAYOUT_MMA, dequant, block_mse, evals, s,
+                                        ue5m3 ? 1 : 0));
+}
+
+int nvfp4_quantize(const void* x, int dtype, int64_t rows, int64_t cols, int block, int rule,
+                   int gs_mode, float* global_scale, uint8_t* codes, uint8_t* scales,
+                   int sf_layout, float* dequant, float* block_mse, void* workspace,
+                   size_t workspace_bytes, void* stream)
+{
+    return fp4_block_quantize(x, dtype, rows, cols, block, rule, FP4Q_SF_E4M3, gs_mode,
+                              global_scale, codes, scales, sf_layout, dequant, block_mse, workspace,
+                              workspace_bytes, stream);
 }
 
 int razer_quantize(const void* x, int dtype, int64_t rows, int64_t cols, int scale_fmt,
@@ -193,6 +211,26 @@ int mxfp4_quantize(const void* x, int dtype, int64_t rows, int64_t cols,
                                         as_stream(stream)));
 }
 
+int mxfp4_flip_refine(const void* w, int dtype, int64_t rows, int64_t cols, const float* chan_scale,
+                      int hadamard32, const float* hess_blocks, int max_moves, uint8_t* codes,
+                      const uint8_t* scales, int32_t* moves, void* stream)
+{
+    const bool empty = rows == 0 || cols == 0;
+    if ((!empty && (!w || !codes || !scales || !hess_blocks)) || !valid_dtype(dtype) || rows < 0 ||
+        cols < 0 || cols % 32 != 0 || max_moves < 0 || max_moves > kFlipMaxMoves)
+        return FP4Q_ERR_ARG;
+    if (!aligned16(w) || !aligned16(codes) || !aligned_or_null(chan_scale) ||
+        !aligned_or_null(hess_blocks) || !aligned_or_null(moves))
+        return FP4Q_ERR_ALIGN;
+    if (cols > kFlipMaxCols)
+        return FP4Q_ERR_UNSUPPORTED;
+    if (empty)
+        return FP4Q_OK;
+    return from_cuda(launch_mxfp4_flip_refine(w, dtype, rows, cols, chan_scale, hadamard32 != 0,
+                                              hess_blocks, max_moves, codes, scales, moves,
+                                              as_stream(stream)));
+}
+
 int fp4_hessian_blocks(const void* x, int dtype, int64_t rows, int64_t cols,
                        const float* chan_scale, int hadamard32, float* hess_blocks,
                        void* workspace, size_t workspace_bytes, void* stream)
@@ -243,7 +281,9 @@ int fp4_dequant_mse(const uint8_t* codes, const uint8_t* scales, int64_t rows, i
     if ((!empty && (!codes || !scales)) || rows < 0 || cols < 0 || !valid_block(block) ||
         cols % block != 0)
         return FP4Q_ERR_ARG;
-    if (scale_fmt < FP4Q_SF_E4M3 || scale_fmt > FP4Q_SF_E8M0)
+    if (scale_fmt < FP4Q_SF_E4M3 || scale_fmt > FP4Q_SF_UE5M3)
+        return FP4Q_ERR_ARG;
+    if (scale_fmt == FP4Q_SF_UE5M3 && specials)
         return FP4Q_ERR_ARG;
     if (scale_fmt == FP4Q_SF_E8M0 && (block != 32 || specials))
         return FP4Q_ERR_ARG;

@@ -129,6 +129,50 @@ __device__ __forceinline__ float e3m3_decode(uint32_t code)
     return e4m3_decode(code + 32u);
 }
 
+// UE5M3 ("Finer is Better" summary, findings: the wide-exponent block scale):
+// unsigned, 5 exponent bits with bias 15 over 3 mantissa bits, subnormals at
+// exponent 0, codes 0..254 finite (0xFF is not a number and never produced).
+// Encode: nearest value, ties to the even code, saturating at 0xFE = 114688.
+__device__ __forceinline__ uint32_t ue5m3_encode(float r)
+{
+    if (!(r < 114688.0f))
+        return 0xFEu;
+    if (r < 6.103515625e-05f) {   // below 2^-14: multiples of 2^-17, 8 -> the first normal
+        return (uint32_t)rintf(__fmul_rn(r, 131072.0f));
+    }
+    const uint32_t bits = __float_as_uint(r);
+    const uint32_t rounded = bits + 0x7FFFFu + ((bits >> 20) & 1u);   // to 3 mantissa bits, ties even
+    const uint32_t code = (rounded >> 20) - (112u << 3);               // exponent bias 127 -> 15
+    return code > 0xFEu ? 0xFEu : code;
+}
+
+__device__ __forceinline__ float ue5m3_decode(uint32_t code)
+{
+    const uint32_t e = (code >> 3) & 31u, m = code & 7u;
+    if (e == 0u)
+        return __fmul_rn((float)m, 7.62939453125e-06f);   // m * 2^-17
+    return __uint_as_float(((e + 112u) << 23) | (m << 20));
+}
+
+// Block-scale format of the NVFP4-style quantizers: 0 = E4M3 (NVFP4), 1 = UE5M3.
+template <int SFMT>
+__device__ __forceinline__ uint32_t sf_encode(float r)
+{
+    if constexpr (SFMT == 1)
+        return ue5m3_encode(r);
+    else
+        return e4m3_encode(r);
+}
+
+template <int SFMT>
+__device__ __forceinline__ float sf_decode(uint32_t code)
+{
+    if constexpr (SFMT == 1)
+        return ue5m3_decode(code);
+    else
+        return e4m3_decode(code);
+}
+
 // ---------------------------------------------------------------- loads
 // Load N consecutive input elements starting at p (16-byte aligned when the
 // byte count allows) into fp32 registers.
@@ -179,6 +223,79 @@ __device__ __forceinline__ void load_elems(const T* __restrict__ p, float (&x)[N
         load_f32<N>(reinterpret_cast<const float*>(p), x);
     else
         load_bf16<N>(reinterpret_cast<const __nv_bfloat16*>(p), x);
+}
+
+// ------------------------------------------------ warp-staged block loads
+// 16-byte streaming load that does not allocate in L1.
+__device__ __forceinline__ uint4 ldg_stream(const uint4* p)
+{
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+// Shared-memory slot of 16-byte chunk p of block i when a block is CPB chunks
+// (2, 4 or 8): XOR-swizzled so that a warp's row-wise stores (8 consecutive
+// lanes = consecutive chunks) and its block-wise loads (8 consecutive lanes =
+// the same chunk of consecutive blocks) both hit 8 distinct 16-byte bank
+// groups per phase.
+template <int CPB>
+__device__ __forceinline__ int staged_slot(int i, int p)
+{
+    static_assert(CPB == 2 || CPB == 4 || CPB == 8, "2, 4 or 8 chunks per block");
+    if constexpr (CPB == 8)
+        return i * 8 + (p ^ (i & 7));
+    else if constexpr (CPB == 4)
+        return i * 4 + (p ^ ((i >> 1) & 3));
+    else
+        return i * 2 + (p ^ ((i >> 2) & 1));
+}
+
+// A warp loads its 32 consecutive blocks of B elements (block `base` + lane
+// for each lane; blocks at or past nblk read as zero) as whole 512-byte rows
+// and hands each lane its own block, via `buf` (this warp's 32 * B *
+// sizeof(T) bytes of shared memory).  A lane reading its 64-128 contiguous
+// bytes straight from global memory would touch 16-32 cache lines per warp
+// instruction.
+template <typename T, int B>
+__device__ __forceinline__ void warp_load_blocks(const T* __restrict__ x, int64_t base, int64_t nblk,
+                                                 uint4* buf, float (&xv)[B])
+{
+    constexpr int CPB = B * (int)sizeof(T) / 16;
+    const int lane = threadIdx.x & 31;
+    const int64_t left = nblk - base;
+    const int nb = left < 32 ? (int)left : 32;
+    const uint4* src = reinterpret_cast<const uint4*>(x + base * B);
+    uint4 v[CPB];
+#pragma unroll
+    for (int k = 0; k < CPB; ++k) {
+        const int c = lane + 32 * k;
+        v[k] = c / CPB < nb ? ldg_stream(src + c) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    __syncwarp();   // the previous blocks have been read back
+#pragma unroll
+    for (int k = 0; k < CPB; ++k) {
+        const int c = lane + 32 * k;
+        buf[staged_slot<CPB>(c / CPB, c % CPB)] = v[k];
+    }
+    __syncwarp();
+#pragma unroll
+    for (int p = 0; p < CPB; ++p) {
+        const uint4 q = buf[staged_slot<CPB>(lane, p)];
+        if constexpr (sizeof(T) == 4) {
+            xv[4 * p] = __uint_as_float(q.x);
+            xv[4 * p + 1] = __uint_as_float(q.y);
+            xv[4 * p + 2] = __uint_as_float(q.z);
+            xv[4 * p + 3] = __uint_as_float(q.w);
+        } else {
+            bf16x2_to_f32(q.x, xv[8 * p], xv[8 * p + 1]);
+            bf16x2_to_f32(q.y, xv[8 * p + 2], xv[8 * p + 3]);
+            bf16x2_to_f32(q.z, xv[8 * p + 4], xv[8 * p + 5]);
+            bf16x2_to_f32(q.w, xv[8 * p + 6], xv[8 * p + 7]);
+        }
+    }
 }
 
 template <int N>

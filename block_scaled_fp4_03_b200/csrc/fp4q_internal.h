@@ -25,11 +25,12 @@ int num_sms();
 
 cudaError_t launch_amax(const void* x, int dtype, int64_t n, float* partials, cudaStream_t s);
 
-// evals (nullable): brute force adds its number of block-candidate evaluations
+// evals (nullable): brute force adds its number of block-candidate evaluations;
+// ue5m3: the block scales are UE5M3 instead of E4M3
 cudaError_t launch_nvfp4_quant(const void* x, int dtype, int64_t rows, int64_t cols, int block,
                                int rule, const GsArgs& gs, uint8_t* codes, uint8_t* scales,
                                int mma_layout, float* deq, float* mse, unsigned long long* evals,
-                               cudaStream_t s);
+                               cudaStream_t s, int ue5m3 = 0);
 
 cudaError_t launch_razer_quant(const void* x, int dtype, int64_t rows, int64_t cols, int sf,
                                const float* specials_host, int n_special, const GsArgs& gs,
@@ -53,6 +54,12 @@ cudaError_t launch_mxfp4_quant(const void* x, int dtype, int64_t rows, int64_t c
                                const float* chan_scale, int hadamard, int rule, const float* hess,
                                uint8_t* codes, uint8_t* scales, float* deq, float* mse,
                                cudaStream_t s);
+
+// Flip-Refinement of MX codes in place (exponents fixed); moves nullable.
+cudaError_t launch_mxfp4_flip_refine(const void* w, int dtype, int64_t rows, int64_t cols,
+                                     const float* tinv, int hadamard, const float* hess, int max_moves,
+                                     uint8_t* codes, const uint8_t* scales, int32_t* moves, cudaStream_t s);
+size_t flip_refine_smem_bytes(int64_t cols);
 
 bool gemm_shape_supported(int64_t M, int64_t N, int64_t K);
 

@@ -119,25 +119,6 @@ __device__ __forceinline__ void load32(const T* __restrict__ p, float (&u)[32])
 // the block-wise loads are free of bank conflicts.
 constexpr int kMxWarps = kThreads / 32;
 
-__device__ __forceinline__ uint4 ldg_stream(const uint4* p)
-{
-    uint4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "l"(p));
-    return v;
-}
-
-// slot of 16-byte chunk p of block i, CPB chunks per block (8 or 4)
-template <int CPB>
-__device__ __forceinline__ int mx_slot(int i, int p)
-{
-    if constexpr (CPB == 8)
-        return i * 8 + (p ^ (i & 7));
-    else
-        return i * 4 + (p ^ ((i >> 1) & 3));
-}
-
 // ERR: also produce the dequantized values / block errors (only when asked).
 template <typename T, bool ERR>
 __global__ void __launch_bounds__(kThreads, 2)
@@ -167,14 +148,14 @@ mx_quant_absmax_kernel(const T* __restrict__ x, uint32_t nblk, uint32_t kb,
 #pragma unroll
             for (int k = 0; k < CPB; ++k) {
                 const int c = lane + 32 * k;
-                bw[mx_slot<CPB>(c / CPB, c % CPB)] = v[k];
+                bw[staged_slot<CPB>(c / CPB, c % CPB)] = v[k];
             }
         }
         __syncwarp();
         float u[32];
 #pragma unroll
         for (int p = 0; p < CPB; ++p) {
-            const uint4 q = bw[mx_slot<CPB>(lane, p)];
+            const uint4 q = bw[staged_slot<CPB>(lane, p)];
             if constexpr (CPB == 8) {
                 u[4 * p] = __uint_as_float(q.x);
                 u[4 * p + 1] = __uint_as_float(q.y);
@@ -200,12 +181,12 @@ mx_quant_absmax_kernel(const T* __restrict__ x, uint32_t nblk, uint32_t kb,
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
                 const int c = lane + 32 * k;
-                bw[mx_slot<8>(c >> 3, c & 7)] = tv[k];
+                bw[staged_slot<8>(c >> 3, c & 7)] = tv[k];
             }
             __syncwarp();
 #pragma unroll
             for (int p = 0; p < 8; ++p) {
-                const uint4 q = bw[mx_slot<8>(lane, p)];
+                const uint4 q = bw[staged_slot<8>(lane, p)];
                 u[4 * p] = __fmul_rn(u[4 * p], __uint_as_float(q.x));
                 u[4 * p + 1] = __fmul_rn(u[4 * p + 1], __uint_as_float(q.y));
                 u[4 * p + 2] = __fmul_rn(u[4 * p + 2], __uint_as_float(q.z));

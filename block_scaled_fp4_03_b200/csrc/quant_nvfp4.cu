@@ -227,7 +227,8 @@ __device__ __forceinline__ float elem_err(float a, float S, float inv)
 enum { R_ABSMAX = 0, R_PZ = 1, R_46 = 2, R_BF = 3 };
 
 // Abs-max, prevent-zero and 4-over-6 (brute force has its own kernel below).
-template <int B, typename T, int RULE>
+// SFMT: the block-scale format, 0 = E4M3 (NVFP4), 1 = UE5M3.
+template <int B, typename T, int RULE, int SFMT>
 __global__ void __launch_bounds__(kThreads)
 nvfp4_quant_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs,
                    uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, int mma_layout,
@@ -240,6 +241,23 @@ nvfp4_quant_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs
     const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
     const int64_t kb_atoms = (bpr + 3) >> 2;
+    // blocks of 128 bytes or more are loaded warp-cooperatively through shared memory
+    constexpr bool kStaged = B * sizeof(T) >= 128;
+    __shared__ uint4 stage_buf[kStaged ? kThreads / 32 : 1][kStaged ? 2 * B * (int)sizeof(T) : 1];
+    // small blocks (one or two 16-byte loads per lane): keep the next block's
+    // load in flight while this one is quantized
+    constexpr bool kPrefetch = !kStaged && B * sizeof(T) <= 32;
+    float xn[B];
+    if constexpr (kPrefetch) {
+        const int64_t b0 = warp0 * 32 + lane;
+        if (b0 < nblk) {
+            load_elems<T, B>(x + b0 * B, xn);
+        } else {
+#pragma unroll
+            for (int i = 0; i < B; ++i)
+                xn[i] = 0.0f;
+        }
+    }
     // MMA-layout scale position: (row, k-block) of this lane's block, advanced
     // by the grid stride without a per-block 64-bit division
     int64_t r_cur = 0, kb_cur = 0, step_r = 0, step_kb = 0;
@@ -256,7 +274,18 @@ nvfp4_quant_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs
         const int64_t b = base + lane;
         const bool valid = b < nblk;
         float xv[B];
-        if (valid) {
+        if constexpr (kStaged) {
+            warp_load_blocks<T, B>(x, base, nblk, stage_buf[threadIdx.x >> 5], xv);
+        } else if constexpr (kPrefetch) {
+            // this iteration's block was loaded last iteration; start the next one
+#pragma unroll
+            for (int i = 0; i < B; ++i)
+                xv[i] = xn[i];
+            const int64_t bn = b + nwarps * 32;
+            if (bn < nblk) {
+                load_elems<T, B>(x + bn * B, xn);
+            }
+        } else if (valid) {
             load_elems<T, B>(x + b * B, xv);
         } else {
 #pragma unroll
@@ -273,26 +302,32 @@ nvfp4_quant_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs
         float sse;
         uint32_t sc;
         if constexpr (RULE == R_ABSMAX || RULE == R_PZ) {
-            sc = e4m3_encode(__fdiv_rn(a, g6));
+            sc = sf_encode<SFMT>(__fdiv_rn(a, g6));
             if (RULE == R_PZ && sc == 0u)
                 sc = 1u;
-            sse = quant_eval<B>(xv, e4m3_decode(sc), g, cw, dq);
+            sse = quant_eval<B>(xv, sf_decode<SFMT>(sc), g, cw, dq);
         } else if constexpr (RULE == R_46) {
-            const uint32_t c6 = e4m3_encode(__fdiv_rn(a, g6));
-            const uint32_t c4 = e4m3_encode(__fdiv_rn(a, g4));
-            uint32_t cw4[(B + 7) / 8];
-            float dq4[B];
-            const float s6 = quant_eval<B>(xv, e4m3_decode(c6), g, cw, dq);
-            const float s4 = quant_eval<B>(xv, e4m3_decode(c4), g, cw4, dq4);
-            const bool take4 = s4 < s6;
-            sc = take4 ? c4 : c6;
-            sse = take4 ? s4 : s6;
+            const uint32_t c6 = sf_encode<SFMT>(__fdiv_rn(a, g6));
+            const uint32_t c4 = sf_encode<SFMT>(__fdiv_rn(a, g4));
+            const float s6 = quant_eval<B>(xv, sf_decode<SFMT>(c6), g, cw, dq);
+            sc = c6;
+            sse = s6;
+            // equal codes give equal errors, and a tie keeps the 6-mapping
+            if (c4 != c6) {
+                uint32_t cw4[(B + 7) / 8];
+                float dq4[B];
+                const float s4 = quant_eval<B>(xv, sf_decode<SFMT>(c4), g, cw4, dq4);
+                if (s4 < s6) {
+                    sc = c4;
+                    sse = s4;
 #pragma unroll
-            for (int j = 0; j < (B + 7) / 8; ++j)
-                cw[j] = take4 ? cw4[j] : cw[j];
+                    for (int j = 0; j < (B + 7) / 8; ++j)
+                        cw[j] = cw4[j];
 #pragma unroll
-            for (int i = 0; i < B; ++i)
-                dq[i] = take4 ? dq4[i] : dq[i];
+                    for (int i = 0; i < B; ++i)
+                        dq[i] = dq4[i];
+                }
+            }
         }
 
         if (valid) {
@@ -666,7 +701,8 @@ razer_paired_kernel(const T* __restrict__ x, int64_t nblk, GsArgs gs, SpecialArg
 }
 
 // ------------------------------------------------------- brute-force scale
-// Brute force over E4M3 codes 1..126: the least in-order squared error, ties
+// Brute force over the scale format's codes (E4M3 1..126, UE5M3 1..254): the
+// least in-order squared error, ties
 // to the lowest code.  Exact shortcuts (each provably skips only losers):
 //  * from the first code at which the largest element rounds to zero
 //    (|y| <= 0.25; |y| falls as the code grows) every element does, so that
@@ -687,15 +723,18 @@ razer_paired_kernel(const T* __restrict__ x, int64_t nblk, GsArgs gs, SpecialArg
 // scan.
 constexpr int kWarps = kThreads / 32;
 
-template <int B, typename T>
+template <int B, typename T, int SFMT>
 __global__ void __launch_bounds__(kThreads)
 nvfp4_bf_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs,
                 uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, int mma_layout,
                 float* __restrict__ deq, float* __restrict__ mse, unsigned long long* evals)
 {
     uint32_t n_eval = 0;   // this lane's error evaluations (seed, all-zero, scan)
+    // the format's largest finite code, and the "no all-zero code" marker
+    constexpr uint32_t kLast = SFMT == 1 ? 254u : 126u;
+    constexpr uint32_t kNone = kLast + 1u;
     // (S, inv) of every code: S = sc * g, inv = min(1/S, FLT_MAX), 0 for S = 0
-    __shared__ float2 tab[128];
+    __shared__ float2 tab[kNone + 1];
     __shared__ __align__(16) float xs[kWarps][32 * B];
     __shared__ unsigned long long key[kWarps][32];
     __shared__ int pre[kWarps][32];
@@ -705,8 +744,8 @@ nvfp4_bf_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs,
     const float g6 = __fmul_rn(6.0f, g);
     // only a starting point for the exact all-zero search below
     const float four_over_g = __fmul_rn(4.0f, __frcp_rn(g));
-    for (int c = threadIdx.x; c < 128; c += blockDim.x) {
-        const float S = __fmul_rn(e4m3_decode((uint32_t)(c < 127 ? c : 126)), g);
+    for (int c = threadIdx.x; c <= (int)kNone; c += blockDim.x) {
+        const float S = __fmul_rn(sf_decode<SFMT>((uint32_t)c < kNone ? (uint32_t)c : kLast), g);
         tab[c] = make_float2(S, (S == 0.0f) ? 0.0f : fminf(__frcp_rn(S), kFltMax));
     }
     __syncthreads();
@@ -745,14 +784,14 @@ nvfp4_bf_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs,
             a = fmaxf(a, fabsf(xv[i]));
             sse0 = __fmaf_rn(xv[i], xv[i], sse0);
         }
-        uint32_t c6 = e4m3_encode(__fdiv_rn(a, g6));
+        uint32_t c6 = sf_encode<SFMT>(__fdiv_rn(a, g6));
         c6 = c6 == 0u ? 1u : c6;
         float best = quant_sse<B>(xv, 0.0f, 0.0f, tab[c6]);
         uint32_t bc = c6;
         n_eval += valid ? 1u : 0u;
-        // first all-zero code (127 = none): step from a nearby code to the
+        // first all-zero code (kNone = none): step from a nearby code to the
         // boundary (|y| is monotone in the code)
-        uint32_t cz = e4m3_encode(__fmul_rn(a, four_over_g));
+        uint32_t cz = sf_encode<SFMT>(__fmul_rn(a, four_over_g));
         cz = cz == 0u ? 1u : cz;
         if (__fmul_rn(a, tab[cz].y) <= 0.25f) {
             while (cz > 1u && __fmul_rn(a, tab[cz - 1u].y) <= 0.25f)
@@ -760,10 +799,10 @@ nvfp4_bf_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs,
         } else {
             do {
                 ++cz;
-            } while (cz < 127u && __fmul_rn(a, tab[cz].y) > 0.25f);
+            } while (cz < kNone && __fmul_rn(a, tab[cz].y) > 0.25f);
         }
-        n_eval += (valid && cz < 127u) ? 1u : 0u;
-        if (cz < 127u && (sse0 < best || (sse0 == best && cz < bc))) {
+        n_eval += (valid && cz < kNone) ? 1u : 0u;
+        if (cz < kNone && (sse0 < best || (sse0 == best && cz < bc))) {
             best = sse0;
             bc = cz;
         }
@@ -776,7 +815,7 @@ nvfp4_bf_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs,
                 break;
             --clo;
         }
-        const int chi = (int)(cz < 127u ? cz : 127u) - 1;   // last code to evaluate
+        const int chi = (int)(cz < kNone ? cz : kNone) - 1;   // last code to evaluate
         int span = chi - (int)clo + 1;
         span = (valid && span > 0) ? span : 0;
 
@@ -829,7 +868,7 @@ nvfp4_bf_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs,
 
         uint32_t cw[(B + 7) / 8];
         float dq[B];
-        const float sse = quant_eval<B>(xv, e4m3_decode(bc), g, cw, dq);
+        const float sse = quant_eval<B>(xv, sf_decode<SFMT>(bc), g, cw, dq);
         if (valid) {
             store_codes<B>(codes + b * (B / 2), cw);
             const int64_t so = mma_layout ? mma_sf_offset(r_cur, kb_cur, kb_atoms) : b;
@@ -856,7 +895,7 @@ nvfp4_bf_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs,
 }
 
 // ------------------------------------------------------ dequant + MSE
-// SF: 0 E4M3, 1 E3M3, 2 E8M0.  RAZ: the -0 code decodes to the block's
+// SF: 0 E4M3, 1 E3M3, 2 E8M0, 3 UE5M3.  RAZ: the -0 code decodes to the block's
 // special value (selector in the scale byte's top bits).
 template <int B, int SF, bool RAZ, typename TR>
 __global__ void __launch_bounds__(kThreads)
@@ -913,7 +952,7 @@ dequant_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ sc
                 const uint32_t k = (int)sel < sp.n ? sel : 0u;
                 spv = k == 0u ? sp.v[0] : k == 1u ? sp.v[1] : k == 2u ? sp.v[2] : sp.v[3];
             }
-            const float scv = SF == 1 ? e3m3_decode(scc) : e4m3_decode(scc);
+            const float scv = SF == 1 ? e3m3_decode(scc) : SF == 3 ? ue5m3_decode(scc) : e4m3_decode(scc);
             const float S = __fmul_rn(scv, g);
 #pragma unroll
             for (int i = 0; i < B; ++i) {
@@ -954,19 +993,19 @@ int grid_for(int64_t work_threads, const void* kernel)
     return (int)(want < 1 ? 1 : want);
 }
 
-template <int B, typename T, int RULE>
+template <int B, typename T, int RULE, int SFMT>
 cudaError_t nvfp4_launch_t(const void* x, int64_t rows, int64_t cols, const GsArgs& gs,
                            uint8_t* codes, uint8_t* scales, int mma, float* deq, float* mse,
                            unsigned long long* evals, cudaStream_t s)
 {
     const int64_t nblk = rows * (cols / B);
     if constexpr (RULE == R_BF) {
-        auto k = nvfp4_bf_kernel<B, T>;
+        auto k = nvfp4_bf_kernel<B, T, SFMT>;
         k<<<grid_for(nblk, (const void*)k), kThreads, 0, s>>>(reinterpret_cast<const T*>(x), nblk,
                                                                cols / B, gs, codes, scales, mma,
                                                                deq, mse, evals);
     } else {
-        auto k = nvfp4_quant_kernel<B, T, RULE>;
+        auto k = nvfp4_quant_kernel<B, T, RULE, SFMT>;
         k<<<grid_for(nblk, (const void*)k), kThreads, 0, s>>>(reinterpret_cast<const T*>(x), nblk,
                                                                cols / B, gs, codes, scales, mma,
                                                                deq, mse);
@@ -974,30 +1013,30 @@ cudaError_t nvfp4_launch_t(const void* x, int64_t rows, int64_t cols, const GsAr
     return cudaGetLastError();
 }
 
-template <int B, typename T>
+template <int B, typename T, int SFMT>
 cudaError_t nvfp4_launch_rule(int rule, const void* x, int64_t rows, int64_t cols,
                               const GsArgs& gs, uint8_t* codes, uint8_t* scales, int mma,
                               float* deq, float* mse, unsigned long long* evals, cudaStream_t s)
 {
     switch (rule) {
-    case R_ABSMAX: return nvfp4_launch_t<B, T, R_ABSMAX>(x, rows, cols, gs, codes, scales, mma, deq, mse, evals, s);
-    case R_PZ: return nvfp4_launch_t<B, T, R_PZ>(x, rows, cols, gs, codes, scales, mma, deq, mse, evals, s);
-    case R_46: return nvfp4_launch_t<B, T, R_46>(x, rows, cols, gs, codes, scales, mma, deq, mse, evals, s);
-    case R_BF: return nvfp4_launch_t<B, T, R_BF>(x, rows, cols, gs, codes, scales, mma, deq, mse, evals, s);
+    case R_ABSMAX: return nvfp4_launch_t<B, T, R_ABSMAX, SFMT>(x, rows, cols, gs, codes, scales, mma, deq, mse, evals, s);
+    case R_PZ: return nvfp4_launch_t<B, T, R_PZ, SFMT>(x, rows, cols, gs, codes, scales, mma, deq, mse, evals, s);
+    case R_46: return nvfp4_launch_t<B, T, R_46, SFMT>(x, rows, cols, gs, codes, scales, mma, deq, mse, evals, s);
+    case R_BF: return nvfp4_launch_t<B, T, R_BF, SFMT>(x, rows, cols, gs, codes, scales, mma, deq, mse, evals, s);
     default: return cudaErrorInvalidValue;
     }
 }
 
-template <typename T>
+template <typename T, int SFMT>
 cudaError_t nvfp4_launch_b(int block, int rule, const void* x, int64_t rows, int64_t cols,
                            const GsArgs& gs, uint8_t* codes, uint8_t* scales, int mma, float* deq,
                            float* mse, unsigned long long* evals, cudaStream_t s)
 {
     switch (block) {
-    case 4: return nvfp4_launch_rule<4, T>(rule, x, rows, cols, gs, codes, scales, mma, deq, mse, evals, s);
-    case 8: return nvfp4_launch_rule<8, T>(rule, x, rows, cols, gs, codes, scales, mma, deq, mse, evals, s);
-    case 16: return nvfp4_launch_rule<16, T>(rule, x, rows, cols, gs, codes, scales, mma, deq, mse, evals, s);
-    case 32: return nvfp4_launch_rule<32, T>(rule, x, rows, cols, gs, codes, scales, mma, deq, mse, evals, s);
+    case 4: return nvfp4_launch_rule<4, T, SFMT>(rule, x, rows, cols, gs, codes, scales, mma, deq, mse, evals, s);
+    case 8: return nvfp4_launch_rule<8, T, SFMT>(rule, x, rows, cols, gs, codes, scales, mma, deq, mse, evals, s);
+    case 16: return nvfp4_launch_rule<16, T, SFMT>(rule, x, rows, cols, gs, codes, scales, mma, deq, mse, evals, s);
+    case 32: return nvfp4_launch_rule<32, T, SFMT>(rule, x, rows, cols, gs, codes, scales, mma, deq, mse, evals, s);
     default: return cudaErrorInvalidValue;
     }
 }
@@ -1062,13 +1101,20 @@ cudaError_t launch_amax(const void* x, int dtype, int64_t n, float* partials, cu
 cudaError_t launch_nvfp4_quant(const void* x, int dtype, int64_t rows, int64_t cols, int block,
                                int rule, const GsArgs& gs, uint8_t* codes, uint8_t* scales,
                                int mma_layout, float* deq, float* mse, unsigned long long* evals,
-                               cudaStream_t s)
+                               cudaStream_t s, int ue5m3)
 {
+    if (ue5m3) {
+        if (dtype == 1)
+            return nvfp4_launch_b<__nv_bfloat16, 1>(block, rule, x, rows, cols, gs, codes, scales,
+                                                    mma_layout, deq, mse, evals, s);
+        return nvfp4_launch_b<float, 1>(block, rule, x, rows, cols, gs, codes, scales, mma_layout,
+                                        deq, mse, evals, s);
+    }
     if (dtype == 1)
-        return nvfp4_launch_b<__nv_bfloat16>(block, rule, x, rows, cols, gs, codes, scales,
-                                             mma_layout, deq, mse, evals, s);
-    return nvfp4_launch_b<float>(block, rule, x, rows, cols, gs, codes, scales, mma_layout, deq,
-                                 mse, evals, s);
+        return nvfp4_launch_b<__nv_bfloat16, 0>(block, rule, x, rows, cols, gs, codes, scales,
+                                                mma_layout, deq, mse, evals, s);
+    return nvfp4_launch_b<float, 0>(block, rule, x, rows, cols, gs, codes, scales, mma_layout, deq,
+                                    mse, evals, s);
 }
 
 cudaError_t launch_razer_quant(const void* x, int dtype, int64_t rows, int64_t cols, int sf,
@@ -1156,6 +1202,8 @@ cudaError_t launch_dequant_mse(const uint8_t* codes, const uint8_t* scales, int6
     const bool raz = specials_host != nullptr && n_special > 0;
     if (sf == 2)
         return dequant_launch_b<2, false>(block, codes, scales, nblk, sp, nullptr, ref, ref_dt, deq, mse, s);
+    if (sf == 3)
+        return dequant_launch_b<3, false>(block, codes, scales, nblk, sp, gs_dev, ref, ref_dt, deq, mse, s);
     if (sf == 1)
         return raz ? dequant_launch_b<1, true>(block, codes, scales, nblk, sp, gs_dev, ref, ref_dt, deq, mse, s)
                    : dequant_launch_b<1, false>(block, codes, scales, nblk, sp, gs_dev, ref, ref_dt, deq, mse, s);

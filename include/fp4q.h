@@ -76,7 +76,7 @@ typedef enum { FP4Q_F32 = 0, FP4Q_BF16 = 1, FP4Q_NVFP4_PACKED = 2 } fp4q_dtype;
 /* Block-scale formats: E4M3 = OCP FP8 E4M3FN (NVFP4 and RaZeR activations),
  * E3M3 = 6-bit unsigned, bias 3, 2^-5..30 (RaZeR weights, [RaZeR] 2.1),
  * E8M0 = 2^(byte-127) (MXFP4, [MACaQ] 1). */
-typedef enum { FP4Q_SF_E4M3 = 0, FP4Q_SF_E3M3 = 1, FP4Q_SF_E8M0 = 2 } fp4q_scale_fmt;
+typedef enum { FP4Q_SF_E4M3 = 0, FP4Q_SF_E3M3 = 1, FP4Q_SF_E8M0 = 2, FP4Q_SF_UE5M3 = 3 } fp4q_scale_fmt;
 
 /* Block-scale selection rules ([Finer] Methodology 2; [MACaQ] 1):
  *  ABSMAX        scale = E4M3(amax_b / (6 g)), ties to even, saturating at 448
@@ -156,6 +156,21 @@ FP4Q_API int nvfp4_quantize(const void* x, int dtype, int64_t rows, int64_t cols
                    size_t workspace_bytes, void* stream);
 
 /*
+ * nvfp4_quantize with the block-scale format as a parameter: FP4Q_SF_E4M3
+ * (NVFP4, identical to nvfp4_quantize) or FP4Q_SF_UE5M3, the wide-exponent
+ * scale of [Finer] (findings: E4M3 with 4-over-6 and hierarchical scaling
+ * reaches UE5M3's quality).  UE5M3 is read as an unsigned 8-bit float with 5
+ * exponent bits (bias 15), 3 mantissa bits and subnormals, codes 0..254
+ * finite (0 .. 114688); the rules are unchanged, brute force searches codes
+ * 1..254, prevent-zero uses code 1 (2^-17), AMAX mode g = amax / (6 * 114688).
+ * UE5M3 scales are row-major only (the GEMM consumes E4M3).
+ */
+FP4Q_API int fp4_block_quantize(const void* x, int dtype, int64_t rows, int64_t cols, int block,
+                   int rule, int scale_fmt, int gs_mode, float* global_scale, uint8_t* codes,
+                   uint8_t* scales, int sf_layout, float* dequant, float* block_mse,
+                   void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * RaZeR quantization, blocks of 16 ([RaZeR] 2.1-2.2).  The block scale is the
  * abs-max scale in `scale_fmt`; for each special value the block is quantized
  * with the -0 code standing for that value (an element takes it when the
@@ -192,6 +207,31 @@ FP4Q_API int razer_quantize(const void* x, int dtype, int64_t rows, int64_t cols
 FP4Q_API int mxfp4_quantize(const void* x, int dtype, int64_t rows, int64_t cols,
                    const float* chan_scale, int hadamard32, int rule, const float* hess_blocks,
                    uint8_t* codes, uint8_t* scales, float* dequant, float* block_mse,
+                   void* stream);
+
+/*
+ * Flip-Refinement of MXFP4 weight codes ([MACaQ] 1 "Flip-Refinement", 3
+ * "Exponent selection and Flip-Refinement"): starting from the codes of an
+ * mxfp4_quantize call (round to nearest at the chosen exponents, which stay
+ * fixed), each row repeatedly moves the one code whose shift to the
+ * neighbouring E2M1 level below or above gives the largest decrease of
+ * sum_k d_k^T H'_k d_k (d = u - deq, u the transformed row), computed in
+ * closed form as 2 D g_i - D^2 H_ii with g = H' d updated incrementally
+ * (g_j -= D H_ji); ties go to the lowest element, then the downward move.
+ * A row stops when no move decreases the objective or after max_moves moves.
+ *
+ *  w            device rows x cols (F32 or BF16), the weights given to
+ *               mxfp4_quantize; chan_scale / hadamard32 as there
+ *  hess_blocks  device fp32 [cols/32][32][32] (H'_k, as fp4_hessian_blocks)
+ *  max_moves    0 .. 2^20 accepted moves per row (the pages' setting: 128)
+ *  codes        device rows*cols/2, in/out; scales: device E8M0 bytes (in)
+ *  moves        device int32 [rows] (out, nullable): moves taken per row
+ * Errors: ERR_ARG, ERR_ALIGN, ERR_UNSUPPORTED (cols > 8192: the per-row state
+ * is kept in shared memory), ERR_CUDA.
+ */
+FP4Q_API int mxfp4_flip_refine(const void* w, int dtype, int64_t rows, int64_t cols,
+                   const float* chan_scale, int hadamard32, const float* hess_blocks,
+                   int max_moves, uint8_t* codes, const uint8_t* scales, int32_t* moves,
                    void* stream);
 
 /*
@@ -245,7 +285,8 @@ FP4Q_API int mxfp4_channel_scale(const void* x, int x_dtype, int64_t tokens, con
  * and [Finer] Methodology 2, as a standalone pass).
  *  codes, scales  as produced by the quantizers (row-major scale bytes)
  *  block          4/8/16/32 (E8M0: 32; RaZeR: 16)
- *  scale_fmt      E4M3 / E3M3: deq = v * (sc * g); E8M0: deq = v * 2^(byte-127)
+ *  scale_fmt      E4M3 / E3M3 / UE5M3: deq = v * (sc * g); E8M0: deq = v * 2^(byte-127)
+ *                 (UE5M3 takes no specials)
  *  specials       host, nullable: RaZeR tables (selector in the scale byte's top bits)
  *  global_scale   device float g, nullable (= 1); ignored for E8M0
  *  ref            device reference tensor (ref_dtype), nullable; needed for block_mse

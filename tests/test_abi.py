@@ -77,6 +77,18 @@ def test_nvfp4_argument_errors(L, kw, expect):
     assert st == expect
 
 
+def test_block_quantize_scale_formats(L):
+    args = lambda sf, layout: (FAKE, 0, 128, 64, 16, 0, sf, 0, None, FAKE, FAKE, layout, None, None, None, 0, None)
+    assert L.fp4_block_quantize(*args(1, 0)) == 1          # E3M3 is RaZeR's, not a block-quantizer format
+    assert L.fp4_block_quantize(*args(2, 0)) == 1
+    assert L.fp4_block_quantize(*args(9, 0)) == 1
+    assert L.fp4_block_quantize(*args(3, 1)) == 1          # UE5M3 scales are row-major only
+    # UE5M3 dequant takes no specials
+    sp = (ctypes.c_float * 2)(5.0, -5.0)
+    assert L.fp4_dequant_mse(FAKE, FAKE, 4, 64, 16, 3, ctypes.cast(sp, ctypes.c_void_p), 2, None, None, 0,
+                             FAKE, None, None) == 1
+
+
 def test_razer_rejects_bad_specials(L):
     for sp, n, sf in (([5.3], 1, 0), ([0.0], 1, 0), ([5, -5, 3.5], 3, 0), ([5, -5, 3.5, -3.5, 1], 5, 1),
                       ([100.0], 1, 1)):
@@ -94,3 +106,11 @@ def test_mx_and_dequant_argument_errors(L):
     assert L.fp4_dequant_mse(FAKE, FAKE, 4, 64, 16, 0, None, 0, None, None, 0, FAKE, FAKE, None) == 1
     assert L.fp4_hessian_blocks(FAKE, 0, 64, 64, None, 1, FAKE, None, 0, None) == 6
     assert L.mxfp4_channel_scale(FAKE, 0, 64, FAKE, 0, 64, 12, 0.75, FAKE, None, FAKE, 1 << 20, None) == 1
+    # Flip-Refinement: bad width, budget, missing Hessian, misalignment, too wide, empty
+    assert L.mxfp4_flip_refine(FAKE, 0, 4, 48, None, 1, FAKE, 8, FAKE, FAKE, None, None) == 1
+    assert L.mxfp4_flip_refine(FAKE, 0, 4, 64, None, 1, FAKE, -1, FAKE, FAKE, None, None) == 1
+    assert L.mxfp4_flip_refine(FAKE, 0, 4, 64, None, 1, FAKE, (1 << 20) + 1, FAKE, FAKE, None, None) == 1
+    assert L.mxfp4_flip_refine(FAKE, 0, 4, 64, None, 1, None, 8, FAKE, FAKE, None, None) == 1
+    assert L.mxfp4_flip_refine(MIS, 0, 4, 64, None, 1, FAKE, 8, FAKE, FAKE, None, None) == 2
+    assert L.mxfp4_flip_refine(FAKE, 0, 4, 8224, None, 1, FAKE, 8, FAKE, FAKE, None, None) == 3
+    assert L.mxfp4_flip_refine(None, 0, 0, 64, None, 1, None, 8, None, None, None, None) == 0

@@ -86,6 +86,54 @@ def test_nvfp4_small(O, B, rule, dtype, gs_mode):
     assert_bits(r["mse"], ref["mse"], "mse")
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("rule", RULES)
+@pytest.mark.parametrize("B", [4, 8, 16, 32])
+@pytest.mark.parametrize("gs_mode", [fq.GS_NONE, fq.GS_AMAX])
+def test_ue5m3_small(O, B, rule, dtype, gs_mode):
+    """The same rules with UE5M3 block scales (fp4_block_quantize)."""
+    kind = "student_t" if gs_mode == fq.GS_NONE else "gaussian"
+    x, x32 = make(kind, 67, 320, seed=B * 10 + rule + 5, dtype=dtype)
+    r = fq.nvfp4_quantize(x, block=B, rule=rule, gs_mode=gs_mode, dequant=True, mse=True,
+                          scale_fmt=fq.SF_UE5M3)
+    torch.cuda.synchronize()
+    g = np.float32(1.0) if gs_mode == fq.GS_NONE else O.global_scale(O.amax(x32), O.SF_UE5M3)
+    if gs_mode == fq.GS_AMAX:
+        assert_bits(r["global_scale"], np.array([g], np.float32), "global scale")
+    ref = O.block_fp4_quantize(x32, B, rule, O.SF_UE5M3, g=g)
+    assert_bits(r["codes"], ref["codes"], "codes")
+    assert_bits(r["scales"], ref["scales"], "scales")
+    assert_bits(r["dequant"], ref["deq"], "dequant")
+    assert_bits(r["mse"], ref["mse"], "mse")
+
+
+def test_ue5m3_edge_values(O):
+    """Scales at the ends of the UE5M3 range: tiny blocks (subnormal scales),
+    huge blocks (saturation), zeros, and midpoints between scale values."""
+    rng = np.random.default_rng(5)
+    x32 = (rng.standard_normal((8, 64)) * np.float32(1e-5)).astype(np.float32)
+    x32[1] *= np.float32(1e-3)
+    x32[2] = 0
+    x32[3] *= np.float32(3e10)
+    x32[4, :16] = np.float32(6 * 1.0625)      # a/6 at the midpoint between 1 and 1.125
+    for rule in RULES:
+        r = fq.nvfp4_quantize(dev(x32), block=16, rule=rule, gs_mode=fq.GS_NONE, dequant=True, mse=True,
+                              scale_fmt=fq.SF_UE5M3)
+        torch.cuda.synchronize()
+        ref = O.block_fp4_quantize(x32, 16, rule, O.SF_UE5M3, g=1.0)
+        for k, rk in (("codes", "codes"), ("scales", "scales"), ("dequant", "deq"), ("mse", "mse")):
+            assert_bits(r[k], ref[rk], "%s rule=%d" % (k, rule))
+
+
+def test_dequant_ue5m3(O):
+    x, x32 = make("student_t", 33, 128, seed=4, dtype="f32")
+    q = O.block_fp4_quantize(x32, 16, O.RULE_FOUR_OVER_SIX, O.SF_UE5M3, g=1.0)
+    r = fq.dequant_mse(dev(q["codes"]), dev(q["scales"]), 33, 128, 16, fq.SF_UE5M3, None, None, ref=x)
+    torch.cuda.synchronize()
+    assert_bits(r["dequant"], q["deq"], "dequant")
+    assert_bits(r["mse"], q["mse"], "mse")
+
+
 def test_nvfp4_mma_scale_layout(O):
     x, x32 = make("gemm_act", 256, 512, seed=3, dtype="bf16")
     rm = fq.nvfp4_quantize(x, 16, fq.FOUR_OVER_SIX)
@@ -235,6 +283,40 @@ def test_channel_scale(O):
     assert_bits(ti, (np.float32(1) / host(t)).astype(np.float32), "t_inv is the fp32 reciprocal of t")
 
 
+# ------------------------------------------------------- Flip-Refinement
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("K", [0, 1, 7, 128, 100000])
+def test_flip_refine_small(O, dtype, K):
+    """37 rows (ragged against the 4 rows of a CTA) x 256 columns: refined
+    codes and per-row move counts equal the oracle's."""
+    w, w32 = make("mx_weight", 37, 256, seed=11, dtype=dtype)
+    xa, xa32 = make("mx_act", 300, 256, seed=12, dtype="f32")
+    t, ti = O.channel_scale(xa32, w32, 0.75)
+    hin = O.hessian_blocks(xa32, t, True).astype(np.float32)
+    q = O.mxfp4_quantize(w32, ti, True, O.RULE_HESSIAN_EXP, hin, want_deq=False)
+    codes = dev(q["codes"].copy())
+    mv = fq.mxfp4_flip_refine(w, codes, dev(q["scales"]), dev(hin), chan_scale=dev(ti), max_moves=K)
+    torch.cuda.synchronize()
+    rc, rm = O.mxfp4_flip_refine(w32, ti, True, hin, q["codes"], q["scales"], K)
+    assert_bits(host(mv), rm, "moves per row")
+    assert_bits(codes, rc, "refined codes")
+    if K >= 7:
+        assert np.all(rm > 0)
+
+
+def test_flip_refine_without_transform(O):
+    w, w32 = make("mx_weight", 9, 128, seed=13, dtype="f32")
+    xa, xa32 = make("mx_act", 200, 128, seed=14, dtype="f32")
+    hin = O.hessian_blocks(xa32, None, False).astype(np.float32)
+    q = O.mxfp4_quantize(w32, None, False, O.RULE_HESSIAN_EXP, hin, want_deq=False)
+    codes = dev(q["codes"].copy())
+    mv = fq.mxfp4_flip_refine(w, codes, dev(q["scales"]), dev(hin), hadamard=False, max_moves=64)
+    torch.cuda.synchronize()
+    rc, rm = O.mxfp4_flip_refine(w32, None, False, hin, q["codes"], q["scales"], 64)
+    assert_bits(host(mv), rm, "moves per row")
+    assert_bits(codes, rc, "refined codes")
+
+
 # ------------------------------------------------------------- dequant
 @pytest.mark.parametrize("B", [4, 8, 16, 32])
 def test_dequant_nvfp4(O, B):
@@ -350,3 +432,11 @@ def test_full_mxfp4_prep_sampled(O):
     assert_bits(host(qw["codes"])[wrows], refw["codes"], "weight codes")
     assert_bits(host(qw["scales"])[wrows], refw["scales"], "weight scales")
     assert_bits(host(qw["mse"])[wrows], refw["mse"], "weight mse")
+    # Flip-Refinement of the whole weight tensor (128 moves per row), sampled rows
+    codes = qw["codes"].clone()
+    mv = fq.mxfp4_flip_refine(w, codes, qw["scales"], dev(hin), chan_scale=ti, max_moves=128)
+    torch.cuda.synchronize()
+    rc, rm = O.mxfp4_flip_refine(w32[wrows], tig, True, hin, host(qw["codes"])[wrows],
+                                 host(qw["scales"])[wrows], 128)
+    assert_bits(host(codes)[wrows], rc, "refined weight codes")
+    assert_bits(host(mv)[wrows], rm, "moves per row")
