@@ -20,7 +20,7 @@ SF_E4M3, SF_E3M3, SF_E8M0, SF_UE5M3 = 0, 1, 2, 3
 ABSMAX, PREVENT_ZERO, FOUR_OVER_SIX, BRUTE_FORCE, HESSIAN_EXP = range(5)
 GS_NONE, GS_AMAX, GS_GIVEN = 0, 1, 2
 SF_ROWMAJOR, SF_MMA = 0, 1
-OP_QUANTIZE, OP_HESSIAN, OP_CHANNEL_SCALE, OP_GEMM = range(4)
+OP_QUANTIZE, OP_HESSIAN, OP_CHANNEL_SCALE, OP_GEMM, OP_FLIP = range(5)
 # byte offset, in a quantize workspace, of the uint64 that brute force adds its
 # evaluation count to (FP4Q_WS_BF_EVALS)
 WS_BF_EVALS = 3072
@@ -35,7 +35,7 @@ SIGNATURES = {
     "fp4_block_quantize": (_i, [_vp, _i, _i64, _i64, _i, _i, _i, _i, _vp, _vp, _vp, _i, _vp, _vp, _vp, _sz, _vp]),
     "razer_quantize": (_i, [_vp, _i, _i64, _i64, _i, _vp, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "mxfp4_quantize": (_i, [_vp, _i, _i64, _i64, _vp, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp]),
-    "mxfp4_flip_refine": (_i, [_vp, _i, _i64, _i64, _vp, _i, _vp, _i, _vp, _vp, _vp, _vp]),
+    "mxfp4_flip_refine": (_i, [_vp, _i, _i64, _i64, _vp, _i, _vp, _i, _vp, _vp, _vp, _vp, _sz, _vp]),
     "fp4_hessian_blocks": (_i, [_vp, _i, _i64, _i64, _vp, _i, _vp, _vp, _sz, _vp]),
     "fp4_hessian_blocks_noalloc": (_i, [_vp, _i, _i64, _i64, _vp, _i, _vp, _vp]),
     "mxfp4_channel_scale": (_i, [_vp, _i, _i64, _vp, _i, _i64, _i64, _fp, _vp, _vp, _vp, _sz, _vp]),
@@ -196,14 +196,17 @@ def mxfp4_quantize(x: torch.Tensor, chan_scale: torch.Tensor | None = None, hada
 
 def mxfp4_flip_refine(w: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, hess: torch.Tensor,
                       chan_scale: torch.Tensor | None = None, hadamard: bool = True, max_moves: int = 128,
-                      moves: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+                      moves: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                      stream=None) -> torch.Tensor:
     """Flip-Refinement of MXFP4 codes in place (exponents fixed); returns the
     int32 [rows] count of moves each row took."""
-    _need_cuda(w, codes, scales, hess, chan_scale)
+    _need_cuda(w, codes, scales, hess, chan_scale, workspace)
     rows, cols = w.shape
     mv = moves if moves is not None else torch.empty(rows, dtype=torch.int32, device=w.device)
+    ws, wsb = (workspace, workspace.numel()) if workspace is not None else _workspace(OP_FLIP, rows, cols, 0, w.device, None)
     st = lib().mxfp4_flip_refine(_ptr(w), _dtype_code(w), rows, cols, _ptr(chan_scale), int(bool(hadamard)),
-                                 _ptr(hess), int(max_moves), _ptr(codes), _ptr(scales), _ptr(mv), _stream(stream))
+                                 _ptr(hess), int(max_moves), _ptr(codes), _ptr(scales), _ptr(mv), _ptr(ws), wsb,
+                                 _stream(stream))
     _check(st, "mxfp4_flip_refine")
     return mv
 

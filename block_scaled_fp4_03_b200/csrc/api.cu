@@ -71,6 +71,7 @@ size_t fp4q_workspace_size(int op, int64_t rows, int64_t cols, int64_t n)
         return 0;
     switch (op) {
     case FP4Q_OP_QUANTIZE: return kQuantWs;
+    case FP4Q_OP_FLIP: return (rows <= 0 || cols <= 0 || cols % 32) ? 0 : flip_refine_ws_bytes(rows, cols);
     case FP4Q_OP_HESSIAN: return cols % 32 ? 0 : hessian_ws_bytes(rows, cols);
     case FP4Q_OP_CHANNEL_SCALE: return channel_scale_ws_bytes(rows, n, cols);
     case FP4Q_OP_GEMM: return gemm_ws_bytes(rows, cols);
@@ -213,7 +214,8 @@ int mxfp4_quantize(const void* x, int dtype, int64_t rows, int64_t cols,
 
 int mxfp4_flip_refine(const void* w, int dtype, int64_t rows, int64_t cols, const float* chan_scale,
                       int hadamard32, const float* hess_blocks, int max_moves, uint8_t* codes,
-                      const uint8_t* scales, int32_t* moves, void* stream)
+                      const uint8_t* scales, int32_t* moves, void* workspace, size_t workspace_bytes,
+                      void* stream)
 {
     const bool empty = rows == 0 || cols == 0;
     if ((!empty && (!w || !codes || !scales || !hess_blocks)) || !valid_dtype(dtype) || rows < 0 ||
@@ -226,8 +228,12 @@ int mxfp4_flip_refine(const void* w, int dtype, int64_t rows, int64_t cols, cons
         return FP4Q_ERR_UNSUPPORTED;
     if (empty)
         return FP4Q_OK;
+    if (!workspace || workspace_bytes < flip_refine_ws_bytes(rows, cols))
+        return FP4Q_ERR_WORKSPACE;
+    if (!aligned16(workspace))
+        return FP4Q_ERR_ALIGN;
     return from_cuda(launch_mxfp4_flip_refine(w, dtype, rows, cols, chan_scale, hadamard32 != 0,
-                                              hess_blocks, max_moves, codes, scales, moves,
+                                              hess_blocks, max_moves, codes, scales, moves, workspace,
                                               as_stream(stream)));
 }
 

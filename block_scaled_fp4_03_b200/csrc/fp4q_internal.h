@@ -58,8 +58,10 @@ cudaError_t launch_mxfp4_quant(const void* x, int dtype, int64_t rows, int64_t c
 // Flip-Refinement of MX codes in place (exponents fixed); moves nullable.
 cudaError_t launch_mxfp4_flip_refine(const void* w, int dtype, int64_t rows, int64_t cols,
                                      const float* tinv, int hadamard, const float* hess, int max_moves,
-                                     uint8_t* codes, const uint8_t* scales, int32_t* moves, cudaStream_t s);
+                                     uint8_t* codes, const uint8_t* scales, int32_t* moves, void* ws,
+                                     cudaStream_t s);
 size_t flip_refine_smem_bytes(int64_t cols);
+size_t flip_refine_ws_bytes(int64_t rows, int64_t cols);
 
 bool gemm_shape_supported(int64_t M, int64_t N, int64_t K);
 

@@ -116,7 +116,8 @@ typedef enum {
     FP4Q_OP_QUANTIZE = 0,       /* nvfp4_quantize / razer_quantize with GS_AMAX */
     FP4Q_OP_HESSIAN = 1,        /* fp4_hessian_blocks (rows, cols) */
     FP4Q_OP_CHANNEL_SCALE = 2,  /* mxfp4_channel_scale (tokens=rows, cols, n_out=n) */
-    FP4Q_OP_GEMM = 3            /* w4a4_gemm with bf16 A (M=rows, K=cols, N=n) */
+    FP4Q_OP_GEMM = 3,           /* w4a4_gemm with bf16 A (M=rows, K=cols, N=n) */
+    FP4Q_OP_FLIP = 4            /* mxfp4_flip_refine (rows, cols) */
 } fp4q_op;
 
 /* Bytes of device workspace an entry point needs (0 if none). */
@@ -226,13 +227,15 @@ FP4Q_API int mxfp4_quantize(const void* x, int dtype, int64_t rows, int64_t cols
  *  max_moves    0 .. 2^20 accepted moves per row (the pages' setting: 128)
  *  codes        device rows*cols/2, in/out; scales: device E8M0 bytes (in)
  *  moves        device int32 [rows] (out, nullable): moves taken per row
- * Errors: ERR_ARG, ERR_ALIGN, ERR_UNSUPPORTED (cols > 8192: the per-row state
- * is kept in shared memory), ERR_CUDA.
+ *  workspace    device, >= fp4q_workspace_size(FP4Q_OP_FLIP, rows, cols, 0)
+ *               bytes, 16-byte aligned (each block's first moves, a row list)
+ * Errors: ERR_ARG, ERR_ALIGN, ERR_WORKSPACE, ERR_UNSUPPORTED (cols > 8192:
+ * a row's state is kept in shared memory), ERR_CUDA.
  */
 FP4Q_API int mxfp4_flip_refine(const void* w, int dtype, int64_t rows, int64_t cols,
                    const float* chan_scale, int hadamard32, const float* hess_blocks,
                    int max_moves, uint8_t* codes, const uint8_t* scales, int32_t* moves,
-                   void* stream);
+                   void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Diagonal 32x32 blocks of the Hessian of the transformed activations,

@@ -106,11 +106,17 @@ def test_mx_and_dequant_argument_errors(L):
     assert L.fp4_dequant_mse(FAKE, FAKE, 4, 64, 16, 0, None, 0, None, None, 0, FAKE, FAKE, None) == 1
     assert L.fp4_hessian_blocks(FAKE, 0, 64, 64, None, 1, FAKE, None, 0, None) == 6
     assert L.mxfp4_channel_scale(FAKE, 0, 64, FAKE, 0, 64, 12, 0.75, FAKE, None, FAKE, 1 << 20, None) == 1
-    # Flip-Refinement: bad width, budget, missing Hessian, misalignment, too wide, empty
-    assert L.mxfp4_flip_refine(FAKE, 0, 4, 48, None, 1, FAKE, 8, FAKE, FAKE, None, None) == 1
-    assert L.mxfp4_flip_refine(FAKE, 0, 4, 64, None, 1, FAKE, -1, FAKE, FAKE, None, None) == 1
-    assert L.mxfp4_flip_refine(FAKE, 0, 4, 64, None, 1, FAKE, (1 << 20) + 1, FAKE, FAKE, None, None) == 1
-    assert L.mxfp4_flip_refine(FAKE, 0, 4, 64, None, 1, None, 8, FAKE, FAKE, None, None) == 1
-    assert L.mxfp4_flip_refine(MIS, 0, 4, 64, None, 1, FAKE, 8, FAKE, FAKE, None, None) == 2
-    assert L.mxfp4_flip_refine(FAKE, 0, 4, 8224, None, 1, FAKE, 8, FAKE, FAKE, None, None) == 3
-    assert L.mxfp4_flip_refine(None, 0, 0, 64, None, 1, None, 8, None, None, None, None) == 0
+    # Flip-Refinement: bad width, budget, missing Hessian, misalignment, too wide,
+    # missing workspace, empty
+    big = 1 << 30
+    assert L.mxfp4_flip_refine(FAKE, 0, 4, 48, None, 1, FAKE, 8, FAKE, FAKE, None, FAKE, big, None) == 1
+    assert L.mxfp4_flip_refine(FAKE, 0, 4, 64, None, 1, FAKE, -1, FAKE, FAKE, None, FAKE, big, None) == 1
+    assert L.mxfp4_flip_refine(FAKE, 0, 4, 64, None, 1, FAKE, (1 << 20) + 1, FAKE, FAKE, None, FAKE, big, None) == 1
+    assert L.mxfp4_flip_refine(FAKE, 0, 4, 64, None, 1, None, 8, FAKE, FAKE, None, FAKE, big, None) == 1
+    assert L.mxfp4_flip_refine(MIS, 0, 4, 64, None, 1, FAKE, 8, FAKE, FAKE, None, FAKE, big, None) == 2
+    assert L.mxfp4_flip_refine(FAKE, 0, 4, 8224, None, 1, FAKE, 8, FAKE, FAKE, None, FAKE, big, None) == 3
+    need = L.fp4q_workspace_size(4, 4, 64, 0)
+    assert need > 0
+    assert L.mxfp4_flip_refine(FAKE, 0, 4, 64, None, 1, FAKE, 8, FAKE, FAKE, None, FAKE, need - 1, None) == 6
+    assert L.mxfp4_flip_refine(FAKE, 0, 4, 64, None, 1, FAKE, 8, FAKE, FAKE, None, None, 0, None) == 6
+    assert L.mxfp4_flip_refine(None, 0, 0, 64, None, 1, None, 8, None, None, None, None, 0, None) == 0

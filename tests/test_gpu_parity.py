@@ -304,6 +304,29 @@ def test_flip_refine_small(O, dtype, K):
         assert np.all(rm > 0)
 
 
+@pytest.mark.parametrize("K", [5, 10, 100000])
+def test_flip_refine_long_block_sequences(O, K):
+    """Blocks whose own greedy runs for many moves (every element just below a
+    rounding midpoint, H' dominated by the all-ones direction): past the moves
+    precomputed per block the rows take the direct per-row path; results are
+    the same either way."""
+    rng = np.random.default_rng(3)
+    w32 = np.zeros((6, 64), np.float32)
+    for r in range(6):
+        for k in range(2):
+            w32[r, 32 * k:32 * k + 32] = (np.float32(4.9 * 2.0 ** (r - 2)) *
+                                          (1 + 0.001 * rng.standard_normal(32)).astype(np.float32))
+    H = np.tile((np.ones((32, 32), np.float32) + 0.05 * np.eye(32, dtype=np.float32))[None], (2, 1, 1))
+    q = O.mxfp4_quantize(w32, None, False, O.RULE_HESSIAN_EXP, H, want_deq=False)
+    codes = dev(q["codes"].copy())
+    mv = fq.mxfp4_flip_refine(dev(w32), codes, dev(q["scales"]), dev(H), hadamard=False, max_moves=K)
+    torch.cuda.synchronize()
+    rc, rm = O.mxfp4_flip_refine(w32, None, False, H, q["codes"], q["scales"], K)
+    assert_bits(host(mv), rm, "moves per row")
+    assert_bits(codes, rc, "refined codes")
+    assert np.all(rm == min(K, 28))
+
+
 def test_flip_refine_without_transform(O):
     w, w32 = make("mx_weight", 9, 128, seed=13, dtype="f32")
     xa, xa32 = make("mx_act", 200, 128, seed=14, dtype="f32")
