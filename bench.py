@@ -60,6 +60,37 @@ def load_peaks():
         return 6650.0, 1965.0, 1590.0, 1400.0, "fallback"
 
 
+# Per-launch DRAM traffic of a row's kernel, from the committed ncu summary of
+# that kernel on the same workload (profiles/*.md); rows without one report null.
+PROFILE_OF_ROW = {
+    "c2_B4_bf": "nvfp4_bf_kernel_B4_student_t_8192x8192.md",
+    "c2_B4_4o6": "nvfp4_quant_kernel_B4_4o6_student_t_8192x8192.md",
+    "c2_B16_absmax": "nvfp4_quant_kernel_B16_absmax_student_t_8192x8192.md",
+    "c3_razer_weight": "razer_paired_kernel_weights_8192x8192_bf16.md",
+    "c3_razer_act": "razer_paired_kernel_acts_16384x4096_bf16.md",
+    "c4_mx_act": "mx_quant_absmax_kernel_acts_8192x4096_bf16.md",
+    "c4_mx_weight_hessian": "mx_quant_hessian_kernel_weights_4096x4096_bf16.md",
+    "c4_hessian_blocks": "hessian_partial_kernel_acts_8192x4096_bf16.md",
+    "c5_act_quant_4o6_mma": "nvfp4_quant_kernel_B16_4o6_bf16_mma_layout_8192x4096.md",
+    "c5_w4a4_gemm": "w4a4_gemm_2sm_kernel_M8192_N14336_K4096.md",
+    "c1_nvfp4_pz_deq_mse": "nvfp4_quant_kernel_B16_pz_deq_mse_gaussian_4096x4096.md",
+}
+
+
+def profiled_traffic(row_name):
+    """DRAM bytes per launch recorded in the row's ncu summary, or None."""
+    import re
+    f = PROFILE_OF_ROW.get(row_name)
+    if not f:
+        return None
+    try:
+        with open(os.path.join(ROOT, "profiles", f)) as fh:
+            m = re.search(r"DRAM traffic \(read \+ write\): ([0-9.]+) MB per launch", fh.read())
+        return float(m.group(1)) * 1e6 if m else None
+    except OSError:
+        return None
+
+
 # ----------------------------------------------------------------------------- rows
 class Row:
     """One hot-path row: how to launch it on device buffers and what it moves."""
@@ -100,7 +131,7 @@ def build_rows(torch, fq, inputs, dev, host_copies=None, groups=None):
         def c1():
             o1.update(fq.nvfp4_quantize(X["c1"], 16, fq.PREVENT_ZERO, gs_mode=fq.GS_AMAX, dequant=True,
                                         mse=True, out=o1, workspace=ws1))
-        rows.append(Row("c1_nvfp4_pz_deq_mse", "nvfp4_quant_kernel<16, float, 1>", n1, n1 * (4 + 0.5 + 1 / 16 + 4 + 4 / 16), 2, c1, o1))
+        rows.append(Row("c1_nvfp4_pz_deq_mse", "nvfp4_quant_kernel<16, float, 1, 0>", n1, n1 * (4 + 0.5 + 1 / 16 + 4 + 4 / 16), 2, c1, o1))
     if groups is None or "c2" in groups:
         # c2
         a2 = inputs.generate("student_t")
@@ -115,7 +146,7 @@ def build_rows(torch, fq, inputs, dev, host_copies=None, groups=None):
 
                 def c2(B=B, rule=rule, o=o, wsr=wsr):
                     o.update(fq.nvfp4_quantize(X["c2"], B, rule, gs_mode=fq.GS_NONE, mse=True, out=o, workspace=wsr))
-                kern = ("nvfp4_bf_kernel<%d, float>" % B) if bf else ("nvfp4_quant_kernel<%d, float, %d>" % (B, rule))
+                kern = ("nvfp4_bf_kernel<%d, float, 0>" % B) if bf else ("nvfp4_quant_kernel<%d, float, %d, 0>" % (B, rule))
                 rows.append(Row("c2_B%d_%s" % (B, names[rule]), kern,
                                 n2, n2 * (4 + 0.5 + 1 / B + 4 / B), 1, c2, o,
                                 bound="alu" if bf else "hbm", eval_ws=wsr, block=B))
@@ -148,8 +179,8 @@ def build_rows(torch, fq, inputs, dev, host_copies=None, groups=None):
 
         def c3a():
             o3a.update(fq.razer_quantize(X["c3a"], fq.SF_E4M3, [5.0, -5.0], gs_mode=fq.GS_AMAX, out=o3a, workspace=ws3))
-        rows.append(Row("c3_razer_weight", "razer_quant_kernel<__nv_bfloat16, 1>", w3.size, w3.size * (2 + 0.5 + 1 / 16), 2, c3w, o3w))
-        rows.append(Row("c3_razer_act", "razer_quant_kernel<__nv_bfloat16, 0>", a3.size, a3.size * (2 + 0.5 + 1 / 16), 2, c3a, o3a))
+        rows.append(Row("c3_razer_weight", "razer_paired_kernel<__nv_bfloat16, 1, 2>", w3.size, w3.size * (2 + 0.5 + 1 / 16), 2, c3w, o3w))
+        rows.append(Row("c3_razer_act", "razer_paired_kernel<__nv_bfloat16, 0, 1>", a3.size, a3.size * (2 + 0.5 + 1 / 16), 2, c3a, o3a))
     if groups is None or "c4" in groups:
         # c4
         x4 = inputs.generate("mx_act")
@@ -215,8 +246,8 @@ def build_rows(torch, fq, inputs, dev, host_copies=None, groups=None):
         def c5g():
             fq.w4a4_gemm(o5["codes"], qw5["codes"], qw5["scales"], qw5["global_scale"], a_scales=o5["scales"],
                          a_global_scale=o5["global_scale"], K=K5, out=y5, workspace=wsg)
-        rows.append(Row("c5_act_quant_4o6_mma", "nvfp4_quant_kernel<16, __nv_bfloat16, 2>", a5.size, a5.size * (2 + 0.5 + 1 / 16), 2, c5, o5))
-        rows.append(Row("c5_w4a4_gemm", "w4a4_gemm_kernel", 0, M5 * K5 * (0.5 + 1 / 16) + N5 * K5 * (0.5 + 1 / 16) + M5 * N5 * 2,
+        rows.append(Row("c5_act_quant_4o6_mma", "nvfp4_quant_kernel<16, __nv_bfloat16, 2, 0>", a5.size, a5.size * (2 + 0.5 + 1 / 16), 2, c5, o5))
+        rows.append(Row("c5_w4a4_gemm", "w4a4_gemm_2sm_kernel", 0, M5 * K5 * (0.5 + 1 / 16) + N5 * K5 * (0.5 + 1 / 16) + M5 * N5 * 2,
                         1, c5g, {"out": y5}, bound="tensor", flops=2.0 * M5 * N5 * K5))
     return rows, X
 
@@ -525,6 +556,7 @@ def main():
         roof = {"bound": "hbm", "achieved": ach, "peak": hbm_peak, "unit": "GB/s", "frac": ach / hbm_peak,
                 "traffic": None, "kernel": dom.kernel, "row": dom.name}
     roof["peak_source"] = peak_src
+    roof["traffic"] = profiled_traffic(dom.name)
 
     e2e = None
     if not args.no_e2e:
@@ -550,7 +582,7 @@ def main():
     if gem is not None:
         g = row_out[gem.name]
         gemm = {"TFLOP_s": g["TFLOP_s"], "frac_of_fp4_peak": g["tensor_frac"], "fp4_peak_TFLOP_s": fp4_peak,
-                "ms": g["ms"], "shape": "M=8192 N=14336 K=4096"}
+                "ms": g["ms"], "shape": "M=8192 N=14336 K=4096", "traffic": profiled_traffic("c5_w4a4_gemm")}
     line = {
         "metric": METRIC, "value": value, "unit": "Gelem/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",

@@ -27,6 +27,7 @@
 // best is the largest positive gain, ties to the lowest element and, within
 // an element, to the downward move; after a move g_j <- fma(-D, H_ji, g_j).
 #include <cstdint>
+#include <mutex>
 
 #include "fp4q_device.cuh"
 #include "fp4q_internal.h"
@@ -154,7 +155,7 @@ __device__ __forceinline__ void stage_hess_block(const float* __restrict__ hess,
 }
 
 // ------------------------------------------------------ 1: block sequences
-constexpr int kSeq = 7;             // moves precomputed per block; heads 0..kSeq stored
+constexpr int kSeq = 15;            // moves precomputed per block; heads 0..kSeq stored
 constexpr int kBlocksWarps = 8;
 
 __device__ __forceinline__ uint2 pack_move(const Move& m)
@@ -407,6 +408,28 @@ size_t flip_refine_smem_bytes(int64_t cols)
     return (size_t)(32 * 33 + cols) * sizeof(float) + (size_t)kFlipWarps * ((size_t)cols * 5 + (size_t)kb * 8);
 }
 
+// Opt the direct-greedy kernel into its largest shared-memory footprint
+// (8192 columns) once per device.
+cudaError_t flip_refine_opt_in()
+{
+    static std::mutex mu;
+    static bool done[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess || dev < 0 || dev >= 64)
+        return e != cudaSuccess ? e : cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (done[dev])
+        return cudaSuccess;
+    const int smem = (int)flip_refine_smem_bytes(8192);
+    e = cudaFuncSetAttribute(flip_refine_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(flip_refine_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess)
+        done[dev] = true;
+    return e;
+}
+
 size_t flip_refine_ws_bytes(int64_t rows, int64_t cols)
 {
     const int64_t kb = cols / 32;
@@ -463,21 +486,18 @@ cudaError_t launch_mxfp4_flip_refine(const void* w, int dtype, int64_t rows, int
     int64_t ctas = (rows + kFlipWarps - 1) / kFlipWarps;
     const int64_t cap = (int64_t)num_sms() * 2;
     ctas = ctas < cap ? ctas : cap;
-    if (dtype == 1) {
-        auto k = flip_refine_kernel<__nv_bfloat16>;
-        e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess)
-            return e;
-        k<<<(unsigned)ctas, kFlipThreads, smem, s>>>(reinterpret_cast<const __nv_bfloat16*>(w), cols, tinv, hadamard,
-                                                      hess, max_moves, codes, scales, moves, fb_list, fb_count);
-    } else {
-        auto k = flip_refine_kernel<float>;
-        e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess)
-            return e;
-        k<<<(unsigned)ctas, kFlipThreads, smem, s>>>(reinterpret_cast<const float*>(w), cols, tinv, hadamard, hess,
-                                                      max_moves, codes, scales, moves, fb_list, fb_count);
-    }
+    // the shared-memory opt-in is set once per device for the largest width
+    e = flip_refine_opt_in();
+    if (e != cudaSuccess)
+        return e;
+    if (dtype == 1)
+        flip_refine_kernel<__nv_bfloat16><<<(unsigned)ctas, kFlipThreads, smem, s>>>(
+            reinterpret_cast<const __nv_bfloat16*>(w), cols, tinv, hadamard, hess, max_moves, codes, scales, moves,
+            fb_list, fb_count);
+    else
+        flip_refine_kernel<float><<<(unsigned)ctas, kFlipThreads, smem, s>>>(
+            reinterpret_cast<const float*>(w), cols, tinv, hadamard, hess, max_moves, codes, scales, moves, fb_list,
+            fb_count);
     return cudaGetLastError();
 }
 

@@ -732,6 +732,8 @@ nvfp4_bf_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs,
     uint32_t n_eval = 0;   // this lane's error evaluations (seed, all-zero, scan)
     // the format's largest finite code, and the "no all-zero code" marker
     constexpr uint32_t kLast = SFMT == 1 ? 254u : 126u;
+    // codes each lane evaluates itself before the warp shares out the rest
+    constexpr int kDirect = B <= 8 ? 3 : 2;
     constexpr uint32_t kNone = kLast + 1u;
     // (S, inv) of every code: S = sc * g, inv = min(1/S, FLT_MAX), 0 for S = 0
     __shared__ float2 tab[kNone + 1];
@@ -815,7 +817,22 @@ nvfp4_bf_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs,
                 break;
             --clo;
         }
-        const int chi = (int)(cz < kNone ? cz : kNone) - 1;   // last code to evaluate
+        int chi = (int)(cz < kNone ? cz : kNone) - 1;   // last code to evaluate
+        // the first kDirect codes of the range straight from registers (most
+        // blocks need no more); the rest is shared out across the warp
+#pragma unroll
+        for (int s = 0; s < kDirect; ++s) {
+            const uint32_t c = clo + (uint32_t)s;
+            if (valid && (int)c <= chi && c != c6) {
+                const float sc_ = quant_sse<B>(xv, 0.0f, 0.0f, tab[c]);
+                n_eval += 1u;
+                if (sc_ < best || (sc_ == best && c < bc)) {
+                    best = sc_;
+                    bc = c;
+                }
+            }
+        }
+        clo = min(clo + (uint32_t)kDirect, (uint32_t)(chi + 1));   // <= kNone: fits the 8-bit field
         int span = chi - (int)clo + 1;
         span = (valid && span > 0) ? span : 0;
 
