@@ -460,6 +460,12 @@ w4a4_gemm_1sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
 // CTAs' copies complete on the leader's stage barrier (pair-form TMA loads),
 // so the MMA issuer waits on one barrier per stage.  The leader's commits are
 // multicast to both CTAs.
+// The scale atoms of a stage go to TMEM from three scale-copy warps of the
+// leader (SFA, SFB rows 0-127, SFB rows 128-255), each waiting for the stage
+// and committing its copies to the stage's "scales ready" barrier; the MMA
+// issuer waits on that barrier and issues only the four MMAs.  One thread
+// issuing 12 copies and 4 MMAs per stage was the bound: the copies cost as
+// much issue time as the MMAs, and split across warps they overlap.
 // The epilogue stages bf16 32 x 64 boxes in 128B-swizzled shared memory (two
 // boxes, half a tile row, at a time) and writes them with TMA stores, handing
 // the accumulator back as soon as its TMEM reads are done, so the stores
@@ -474,6 +480,9 @@ constexpr int k2StageBytes = k2AStage + k2BStage + k2SfaStage + k2SfbStage;
 constexpr int k2EpiWarpBytes = 32 * 128 * 2;   // 32 rows x 128 bf16 per epilogue warp (half a tile row)
 constexpr int k2EpiBytes = 4 * k2EpiWarpBytes;
 constexpr int k2SmemBytes = k2Stages * k2StageBytes + k2EpiBytes + 1024 + kBarBytes;
+// warp 0 producer, warp 1 MMA issuer, warps 2-5 epilogue, warps 6-8 scale copies
+constexpr int k2Threads = 288;
+static_assert(8 * (3 * k2Stages + 7) + 8 <= kBarBytes, "barrier area");
 static_assert(k2StageBytes % 1024 == 0 && (k2Stages * k2StageBytes) % 1024 == 0, "swizzle alignment");
 static_assert(k2SmemBytes <= 232448, "shared memory budget");
 static_assert(kSfCol0 + k2Stages * kSfColsPerStage <= kTmemCols, "TMEM budget");
@@ -547,7 +556,7 @@ __device__ __forceinline__ void stage_row_chunk(uint8_t* stg, int c, int lane, c
     }
 }
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(k2Threads, 1)
 w4a4_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
                      const __grid_constant__ CUtensorMap tmOut, const GemmParams p)
@@ -557,9 +566,9 @@ w4a4_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
     uint8_t* epi = smem + k2Stages * k2StageBytes;
     uint64_t* bars = reinterpret_cast<uint64_t*>(epi + k2EpiBytes);
     // bars: [0,S) full (the leader's counts both CTAs' bytes), [S,2S) empty,
-    // [2S,3S) unused, 3S acc_full, 3S+1 acc_empty (leader), 3S+2 drain,
-    // 3S+3 teardown handshake
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 3 * k2Stages + 4);
+    // [2S,3S) scales ready (leader), 3S acc_full, 3S+1 acc_empty (leader),
+    // 3S+2 drain, 3S+3 teardown handshake, [3S+4, 3S+7) scale-copy drains
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 3 * k2Stages + 7);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5;
@@ -569,6 +578,7 @@ w4a4_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
     const uint32_t bar0 = smem_u32(bars);
     auto full_bar = [&](int s) { return bar0 + 8u * (uint32_t)s; };
     auto empty_bar = [&](int s) { return bar0 + 8u * (uint32_t)(k2Stages + s); };
+    auto sf_ready_bar = [&](int s) { return bar0 + 8u * (uint32_t)(2 * k2Stages + s); };
     const uint32_t acc_full = bar0 + 8u * (3 * k2Stages);
     const uint32_t acc_empty = bar0 + 8u * (3 * k2Stages + 1);
     const uint32_t drain = bar0 + 8u * (3 * k2Stages + 2);
@@ -578,11 +588,14 @@ w4a4_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
         for (int s = 0; s < k2Stages; ++s) {
             mbar_init(full_bar(s), 1);
             mbar_init(empty_bar(s), 1);
+            mbar_init(sf_ready_bar(s), 3);
         }
         mbar_init(acc_full, 1);
         mbar_init(acc_empty, 2 * 128);
         mbar_init(drain, 1);
         mbar_init(bye, 1);
+        for (int w = 0; w < 3; ++w)
+            mbar_init(bar0 + 8u * (uint32_t)(3 * k2Stages + 4 + w), 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -673,23 +686,18 @@ w4a4_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                 tc_fence_after();
                 bool ok = true;
                 for (int kb = 0; kb < p.kblocks; ++kb) {
-                    if (!mbar_wait_cluster(full_bar(stage), phase, abort_flag) || *abort_flag) {
+                    // the scale warps observed the stage's full barrier (cluster
+                    // acquire) before their copies; their commits complete this
+                    // barrier only after the copies, so the stage is in place
+                    if (!mbar_wait(sf_ready_bar(stage), phase, abort_flag) || *abort_flag) {
                         give_up();
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     uint8_t* st = smem + stage * k2StageBytes;
-                    const uint32_t sa_s = smem_u32(st + k2AStage + k2BStage);
-                    const uint32_t sb_s = sa_s + k2SfaStage;
                     const uint32_t tsfa = tmem + kSfCol0 + (uint32_t)stage * kSfColsPerStage;
                     const uint32_t tsfb = tsfa + 16;
-#pragma unroll
-                    for (int s = 0; s < 4; ++s) {
-                        tc2_cp_sf(tsfa + 4 * s, sdesc_sf(sa_s + 512 * s));
-                        tc2_cp_sf(tsfb + 8 * s, sdesc_sf(sb_s + 512 * s));
-                        tc2_cp_sf(tsfb + 8 * s + 4, sdesc_sf(sb_s + k2SfbStage / 2 + 512 * s));
-                    }
                     const uint32_t a_s = smem_u32(st);
                     const uint32_t b_s = a_s + k2AStage;
 #pragma unroll
@@ -711,6 +719,50 @@ w4a4_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
             if (issued_any) {
                 tc2_commit_mc(drain, (uint16_t)0x1);
                 if (!mbar_quiesce(drain, 0))
+                    give_up();
+            }
+        }
+    } else if (warp >= 6) {
+        if (lane == 0 && leader) {
+            // ------------------------------- scale-copy warps (leader), one
+            // atom column each: 0 SFA, 1 SFB rows 0-127, 2 SFB rows 128-255
+            const int which = warp - 6;
+            const uint32_t sf_off = which == 0 ? 0u : which == 1 ? (uint32_t)k2SfaStage
+                                                                 : (uint32_t)(k2SfaStage + k2SfbStage / 2);
+            const uint32_t col_off = which == 0 ? 0u : which == 1 ? 16u : 20u;
+            const uint32_t col_step = which == 0 ? 4u : 8u;
+            int stage = 0;
+            uint32_t phase = 0;
+            bool issued_any = false;
+            for (int tile = cluster; tile < num_tiles && !*abort_flag; tile += nclusters) {
+                bool ok = true;
+                for (int kb = 0; kb < p.kblocks; ++kb) {
+                    if (!mbar_wait_cluster(full_bar(stage), phase, abort_flag) || *abort_flag) {
+                        give_up();
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t src = smem_u32(smem + stage * k2StageBytes + k2AStage + k2BStage) + sf_off;
+                    const uint32_t dst = tmem + kSfCol0 + (uint32_t)stage * kSfColsPerStage + col_off;
+#pragma unroll
+                    for (int s = 0; s < 4; ++s)
+                        tc2_cp_sf(dst + col_step * (uint32_t)s, sdesc_sf(src + 512 * s));
+                    issued_any = true;
+                    tc2_commit_mc(sf_ready_bar(stage), (uint16_t)0x1);
+                    if (++stage == k2Stages) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok)
+                    break;
+            }
+            if (issued_any) {
+                // this warp's copies have landed before the TMEM can go away
+                const uint32_t own_drain = bar0 + 8u * (uint32_t)(3 * k2Stages + 4 + which);
+                tc2_commit_mc(own_drain, (uint16_t)0x1);
+                if (!mbar_quiesce(own_drain, 0))
                     give_up();
             }
         }
@@ -910,7 +962,7 @@ cudaError_t launch_w4a4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const 
         const int tiles = p.tiles_m * p.tiles_n;
         const int pairs = num_sms() / 2;
         const int grid = 2 * (tiles < pairs ? tiles : pairs);
-        w4a4_gemm_2sm_kernel<<<grid, kThreads, k2SmemBytes, s>>>(ta, tb, tsa, tsb, to, p);
+        w4a4_gemm_2sm_kernel<<<grid, k2Threads, k2SmemBytes, s>>>(ta, tb, tsa, tsb, to, p);
         return cudaGetLastError();
     }
     CUtensorMap ta, tb, tsa, tsb;
