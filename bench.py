@@ -249,6 +249,46 @@ def build_rows(torch, fq, inputs, dev, host_copies=None, groups=None):
         rows.append(Row("c5_act_quant_4o6_mma", "nvfp4_quant_kernel<16, __nv_bfloat16, 2, 0>", a5.size, a5.size * (2 + 0.5 + 1 / 16), 2, c5, o5))
         rows.append(Row("c5_w4a4_gemm", "w4a4_gemm_2sm_kernel", 0, M5 * K5 * (0.5 + 1 / 16) + N5 * K5 * (0.5 + 1 / 16) + M5 * N5 * 2,
                         1, c5g, {"out": y5}, bound="tensor", flops=2.0 * M5 * N5 * K5))
+
+        # RaZeR-aware GEMM (next rows): the same weights quantized with RaZeR
+        # (E3M3 scale, +-5 / +-3.5) and split into two E2M1 tensors once, offline;
+        # (a) with the step's 4-over-6 NVFP4 activations: 2 passes over K;
+        # (b) with RaZeR activations (E4M3, +-5) quantized and split per call: 4 passes
+        spw, spa = [5.0, -5.0, 3.5, -3.5], [5.0, -5.0]
+        w5d = torch.from_numpy(w5.view(np.int16)).to(dev).view(torch.bfloat16)
+        rw5 = fq.razer_quantize(w5d, fq.SF_E3M3, spw, gs_mode=fq.GS_AMAX)
+        del w5d
+        pw5 = fq.razer_gemm_prepare(rw5["codes"], rw5["meta"], fq.SF_E3M3, spw)
+        pwo = {"main": pw5["main"], "extra": pw5["extra"], "scales": pw5["scales"]}
+        wsr = torch.empty(8192, dtype=torch.uint8, device=dev)
+        ra5, pa5 = {}, {}
+
+        def f2p():
+            fq.razer_gemm_prepare(rw5["codes"], rw5["meta"], fq.SF_E3M3, spw, out=pwo)
+
+        def f2w():
+            fq.razer_w4a4_gemm(o5["codes"], o5["scales"], o5["global_scale"], pw5["main"], pw5["scales"],
+                               rw5["global_scale"], w_extra=pw5["extra"], out=y5, workspace=wsr)
+
+        def f2aq():
+            ra5.update(fq.razer_quantize(X["c5"], fq.SF_E4M3, spa, gs_mode=fq.GS_AMAX, out=ra5, workspace=ws5))
+            pa5.update(fq.razer_gemm_prepare(ra5["codes"], ra5["meta"], fq.SF_E4M3, spa, out=pa5))
+
+        def f2wa():
+            fq.razer_w4a4_gemm(pa5["main"], pa5["scales"], ra5["global_scale"], pw5["main"], pw5["scales"],
+                               rw5["global_scale"], a_extra=pa5["extra"], w_extra=pw5["extra"], out=y5,
+                               workspace=wsr)
+        rows.append(Row("f2_razer_prepare_weights", "razer_prepare_kernel<1>", N5 * K5,
+                        N5 * K5 * (0.5 + 1 / 16) + N5 * K5 * (0.5 + 0.5 + 1 / 16), 1, f2p, pwo, extra=True))
+        rows.append(Row("f2_razer_gemm_w_2pass", "w4a4_gemm_2sm_kernel", 0,
+                        M5 * K5 * (0.5 + 1 / 16) + N5 * K5 * (1.0 + 1 / 16) + M5 * N5 * 2, 1, f2w, {"out": y5},
+                        bound="tensor", flops=2.0 * M5 * N5 * K5, extra=True))
+        rows.append(Row("f2_razer_act_quant_prep", "razer_paired_kernel<__nv_bfloat16, 0, 1>", a5.size,
+                        a5.size * (2 + 0.5 + 1 / 16) + a5.size * (0.5 + 1 / 16 + 1.0 + 1 / 16), 3, f2aq, pa5,
+                        extra=True))
+        rows.append(Row("f2_razer_gemm_wa_4pass", "w4a4_gemm_2sm_kernel", 0,
+                        M5 * K5 * (1.0 + 1 / 16) + N5 * K5 * (1.0 + 1 / 16) + M5 * N5 * 2, 1, f2wa, {"out": y5},
+                        bound="tensor", flops=2.0 * M5 * N5 * K5, extra=True))
     return rows, X
 
 

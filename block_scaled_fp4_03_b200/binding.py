@@ -42,6 +42,8 @@ SIGNATURES = {
     "fp4_dequant_mse": (_i, [_vp, _vp, _i64, _i64, _i, _i, _vp, _i, _vp, _vp, _i, _vp, _vp, _vp]),
     "w4a4_gemm": (_i, [_vp, _i, _i, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _sz, _vp]),
     "fp4q_gemm_status": (_i, [_vp, _vp]),
+    "razer_gemm_prepare": (_i, [_vp, _vp, _i64, _i64, _i, _vp, _i, _vp, _vp, _vp, _vp]),
+    "razer_w4a4_gemm": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _sz, _vp]),
 }
 
 _lock = threading.Lock()
@@ -286,6 +288,45 @@ def w4a4_gemm(a: torch.Tensor, w_codes: torch.Tensor, w_scales: torch.Tensor, w_
                          _ptr(w_scales), _ptr(w_global_scale), M, N, K, _ptr(o), _ptr(ws), wsb,
                          _stream(stream))
     _check(st, "w4a4_gemm")
+    return o
+
+
+def razer_gemm_prepare(codes: torch.Tensor, meta: torch.Tensor, scale_fmt: int, specials,
+                       out: dict | None = None, stream=None) -> dict:
+    """Split RaZeR codes into (main, extra) E2M1 tensors sharing E4M3 scales in the MMA layout;
+    returns dict(main, extra, scales)."""
+    _need_cuda(codes, meta)
+    rows, half = codes.shape
+    cols = half * 2
+    dev = codes.device
+    o = out or {}
+    main = o.get("main") if o.get("main") is not None else torch.empty((rows, half), dtype=torch.uint8, device=dev)
+    extra = o.get("extra") if o.get("extra") is not None else torch.empty((rows, half), dtype=torch.uint8, device=dev)
+    scales = o.get("scales") if o.get("scales") is not None else torch.empty((rows * cols // 16,), dtype=torch.uint8, device=dev)
+    sp = (ctypes.c_float * len(specials))(*[float(v) for v in specials])
+    st = lib().razer_gemm_prepare(_ptr(codes), _ptr(meta), rows, cols, scale_fmt, ctypes.cast(sp, ctypes.c_void_p),
+                                  len(specials), _ptr(main), _ptr(extra), _ptr(scales), _stream(stream))
+    _check(st, "razer_gemm_prepare")
+    return dict(main=main, extra=extra, scales=scales)
+
+
+def razer_w4a4_gemm(a_codes: torch.Tensor, a_scales: torch.Tensor, a_global_scale: torch.Tensor,
+                    w_codes: torch.Tensor, w_scales: torch.Tensor, w_global_scale: torch.Tensor,
+                    a_extra: torch.Tensor | None = None, w_extra: torch.Tensor | None = None,
+                    out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                    stream=None) -> torch.Tensor:
+    """out = bf16(g_a g_w (A + A_extra) . (W + W_extra)^T): each operand a packed code tensor
+    plus an optional extra code tensor sharing its MMA-layout E4M3 scales."""
+    _need_cuda(a_codes, a_scales, a_global_scale, w_codes, w_scales, w_global_scale, a_extra, w_extra)
+    M, K = a_codes.shape[0], a_codes.shape[1] * 2
+    N = w_codes.shape[0]
+    dev = a_codes.device
+    o = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    ws = workspace if workspace is not None else torch.empty(8192, dtype=torch.uint8, device=dev)
+    st = lib().razer_w4a4_gemm(_ptr(a_codes), _ptr(a_extra), _ptr(a_scales), _ptr(a_global_scale),
+                               _ptr(w_codes), _ptr(w_extra), _ptr(w_scales), _ptr(w_global_scale),
+                               M, N, K, _ptr(o), _ptr(ws), ws.numel(), _stream(stream))
+    _check(st, "razer_w4a4_gemm")
     return o
 
 

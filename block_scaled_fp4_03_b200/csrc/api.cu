@@ -380,4 +380,90 @@ int fp4q_gemm_status(const void* workspace, void* stream)
     return flag ? FP4Q_ERR_TIMEOUT : FP4Q_OK;
 }
 
+// E2M1 codes (p, q) with value(p) + value(q) == v exactly: p the largest
+// magnitude of the special's sign that leaves an E2M1 remainder.  False when
+// no such pair exists.
+static bool split_special(float v, uint8_t* p, uint8_t* q)
+{
+    static const float kMag[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+    const uint8_t sign = v < 0.0f ? 8u : 0u;
+    const float m = std::fabs(v);
+    for (int i = 7; i >= 1; --i) {
+        if (kMag[i] > m)
+            continue;
+        const float r = m - kMag[i];
+        for (int j = 0; j < 8; ++j) {
+            if (kMag[j] == r) {
+                *p = (uint8_t)(sign | i);
+                *q = (uint8_t)(j == 0 ? 0 : (sign | j));
+                return true;
+            }
+        }
+    }
+    return false;
+}
+
+int razer_gemm_prepare(const uint8_t* codes, const uint8_t* meta, int64_t rows, int64_t cols,
+                       int scale_fmt, const float* specials, int n_special, uint8_t* main_codes,
+                       uint8_t* extra_codes, uint8_t* scales_mma, void* stream)
+{
+    const bool empty = rows == 0 || cols == 0;
+    if (rows < 0 || cols < 0 || !specials)
+        return FP4Q_ERR_ARG;
+    if (!empty && (!codes || !meta || !main_codes || !extra_codes || !scales_mma))
+        return FP4Q_ERR_ARG;
+    if (scale_fmt == FP4Q_SF_E3M3) {
+        if (n_special < 1 || n_special > 4)
+            return FP4Q_ERR_ARG;
+    } else if (scale_fmt == FP4Q_SF_E4M3) {
+        if (n_special < 1 || n_special > 2)
+            return FP4Q_ERR_ARG;
+    } else {
+        return FP4Q_ERR_ARG;
+    }
+    uint8_t pc[4] = {0, 0, 0, 0}, qc[4] = {0, 0, 0, 0};
+    for (int i = 0; i < n_special; ++i) {
+        const float v = specials[i];
+        const float twice = v * 2.0f;
+        if (!(std::fabs(v) <= 32.0f) || v == 0.0f || twice != std::nearbyint(twice))
+            return FP4Q_ERR_ARG;
+        if (!split_special(v, &pc[i], &qc[i]))
+            return FP4Q_ERR_UNSUPPORTED;
+    }
+    if (rows % 128 != 0 || cols % 64 != 0)
+        return FP4Q_ERR_ARG;
+    if (!aligned_or_null(codes) || !aligned_or_null(main_codes) || !aligned_or_null(extra_codes))
+        return FP4Q_ERR_ALIGN;
+    if (empty)
+        return FP4Q_OK;
+    return from_cuda(launch_razer_gemm_prepare(codes, meta, rows, cols, scale_fmt, pc, qc, main_codes,
+                                               extra_codes, scales_mma, as_stream(stream)));
+}
+
+int razer_w4a4_gemm(const uint8_t* a_codes, const uint8_t* a_extra, const uint8_t* a_scales,
+                    const float* a_global_scale, const uint8_t* w_codes, const uint8_t* w_extra,
+                    const uint8_t* w_scales, const float* w_global_scale, int64_t M, int64_t N,
+                    int64_t K, void* out, void* workspace, size_t workspace_bytes, void* stream)
+{
+    if (!a_codes || !a_scales || !a_global_scale || !w_codes || !w_scales || !w_global_scale || !out ||
+        !workspace)
+        return FP4Q_ERR_ARG;
+    if (M <= 0 || N <= 0 || K <= 0)
+        return FP4Q_ERR_ARG;
+    if (!gemm_shape_supported(M, N, K))
+        return FP4Q_ERR_UNSUPPORTED;
+    if (!aligned16(a_codes) || !aligned_or_null(a_extra) || !aligned16(a_scales) || !aligned16(w_codes) ||
+        !aligned_or_null(w_extra) || !aligned16(w_scales) || !aligned16(out) || !aligned16(workspace) ||
+        !aligned16(a_global_scale) || !aligned16(w_global_scale))
+        return FP4Q_ERR_ALIGN;
+    if (workspace_bytes < kGemmHeader)
+        return FP4Q_ERR_WORKSPACE;
+    cudaStream_t s = as_stream(stream);
+    int* err = reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) + kGemmErr);
+    if (cudaMemsetAsync(err, 0, sizeof(int), s) != cudaSuccess)
+        return FP4Q_ERR_CUDA;
+    return from_cuda(launch_w4a4_gemm(a_codes, a_scales, a_global_scale, w_codes, w_scales, w_global_scale,
+                                      M, N, K, out, err, s, a_extra, w_extra));
+}
+
 }  // extern "C"

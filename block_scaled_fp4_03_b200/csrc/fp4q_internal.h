@@ -65,9 +65,21 @@ size_t flip_refine_ws_bytes(int64_t rows, int64_t cols);
 
 bool gemm_shape_supported(int64_t M, int64_t N, int64_t K);
 
+// a1_codes / w1_codes (nullable): second code tensors sharing the scales of
+// A / W; the GEMM then sums the products of every pair of present tensors,
+// out = (A + A1) . (W + W1)^T, as extra passes over K into one accumulator.
 cudaError_t launch_w4a4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* ga,
                              const uint8_t* w_codes, const uint8_t* w_sf, const float* gw, int64_t M,
-                             int64_t N, int64_t K, void* out, int* err, cudaStream_t s);
+                             int64_t N, int64_t K, void* out, int* err, cudaStream_t s,
+                             const uint8_t* a1_codes = nullptr, const uint8_t* w1_codes = nullptr);
+
+// RaZeR codes + meta -> (main codes, extra codes, E4M3 scale bytes in the MMA
+// layout) with main + extra = the RaZeR values exactly.  p_code / q_code:
+// per selector, the E2M1 codes whose values sum to the special value.
+cudaError_t launch_razer_gemm_prepare(const uint8_t* codes, const uint8_t* meta, int64_t rows,
+                                      int64_t cols, int sf, const uint8_t* p_code,
+                                      const uint8_t* q_code, uint8_t* main_codes,
+                                      uint8_t* extra_codes, uint8_t* scales_mma, cudaStream_t s);
 
 // Workspace (bytes) launch_hessian_blocks / launch_mx_channel_scale need.
 size_t hessian_ws_bytes(int64_t rows, int64_t cols);

@@ -258,11 +258,24 @@ struct GemmParams {
     __nv_bfloat16* out;       // M x N row-major
     int* err;                 // error word (workspace)
     int tiles_m, tiles_n, kblocks, kb_atoms, N;
+    // Passes: the K loop runs kiters = kblocks << pass_shift steps; step j
+    // covers K block j >> pass_shift with operand pair (pass_sel >> 2*(j %
+    // passes)) & 3: bit 0 takes A's second code tensor, bit 1 W's.  All passes
+    // share the scales and accumulate into one accumulator (one pass: the
+    // plain GEMM).
+    int kiters, pass_shift, pass_sel;
 };
+
+// Code tensors of step j (see GemmParams).
+__device__ __forceinline__ int pass_operands(const GemmParams& p, int j)
+{
+    return (p.pass_sel >> (2 * (j & ((1 << p.pass_shift) - 1)))) & 3;
+}
 
 __global__ void __launch_bounds__(kThreads, 1)
 w4a4_gemm_1sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
+                     const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
                      const GemmParams p)
 {
     extern __shared__ uint8_t smem_raw[];
@@ -318,16 +331,18 @@ w4a4_gemm_1sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
             for (int tile = blockIdx.x; tile < num_tiles && !*abort_flag; tile += gridDim.x) {
                 const int mt = tile % p.tiles_m;
                 const int nt = tile / p.tiles_m;
-                for (int kb = 0; kb < p.kblocks; ++kb) {
+                for (int j = 0; j < p.kiters; ++j) {
                     if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag) || *abort_flag) {
                         give_up();
                         break;
                     }
+                    const int kb = j >> p.pass_shift;
+                    const int sel = pass_operands(p, j);
                     const uint32_t fb = full_bar(stage);
                     mbar_expect_tx(fb, kStageBytes);
                     uint8_t* st = smem + stage * kStageBytes;
-                    tma_load_2d(smem_u32(st), &tmA, kb * (kBK / 2), mt * kBM, fb);
-                    tma_load_2d(smem_u32(st + kAStage), &tmB, kb * (kBK / 2), nt * kBN, fb);
+                    tma_load_2d(smem_u32(st), (sel & 1) ? &tmA1 : &tmA, kb * (kBK / 2), mt * kBM, fb);
+                    tma_load_2d(smem_u32(st + kAStage), (sel & 2) ? &tmB1 : &tmB, kb * (kBK / 2), nt * kBN, fb);
                     // scale atoms: 4 consecutive K atoms of row atom mt (A), of row
                     // atoms 2nt and 2nt+1 (B)
                     tma_load_3d(smem_u32(st + kAStage + kBStage), &tmSA, 0, kb * 4, mt, fb);
@@ -360,7 +375,7 @@ w4a4_gemm_1sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                 }
                 tc_fence_after();
                 bool ok = true;
-                for (int kb = 0; kb < p.kblocks; ++kb) {
+                for (int kb = 0; kb < p.kiters; ++kb) {
                     if (!mbar_wait(full_bar(stage), phase, abort_flag) || *abort_flag) {
                         give_up();
                         ok = false;
@@ -559,7 +574,8 @@ __device__ __forceinline__ void stage_row_chunk(uint8_t* stg, int c, int lane, c
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(k2Threads, 1)
 w4a4_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
-                     const __grid_constant__ CUtensorMap tmOut, const GemmParams p)
+                     const __grid_constant__ CUtensorMap tmOut, const __grid_constant__ CUtensorMap tmA1,
+                     const __grid_constant__ CUtensorMap tmB1, const GemmParams p)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -633,18 +649,22 @@ w4a4_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
             for (int tile = cluster; tile < num_tiles && !*abort_flag; tile += nclusters) {
                 const int mt = tile % p.tiles_m;
                 const int nt = tile / p.tiles_m;
-                for (int kb = 0; kb < p.kblocks; ++kb) {
+                for (int j = 0; j < p.kiters; ++j) {
                     if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag) || *abort_flag) {
                         give_up();
                         break;
                     }
+                    const int kb = j >> p.pass_shift;
+                    const int sel = pass_operands(p, j);
                     // the leader expects both CTAs' bytes of this stage
                     const uint32_t fb = mapa_rank(full_bar(stage), 0);
                     if (leader)
                         mbar_expect_tx(full_bar(stage), 2 * k2StageBytes);
                     uint8_t* st = smem + stage * k2StageBytes;
-                    tma_load_2d_pair(smem_u32(st), &tmA, kb * (kBK / 2), mt * 256 + (int)rank * 128, fb);
-                    tma_load_2d_pair(smem_u32(st + k2AStage), &tmB, kb * (kBK / 2), nt * 256 + (int)rank * 128, fb);
+                    tma_load_2d_pair(smem_u32(st), (sel & 1) ? &tmA1 : &tmA, kb * (kBK / 2),
+                                     mt * 256 + (int)rank * 128, fb);
+                    tma_load_2d_pair(smem_u32(st + k2AStage), (sel & 2) ? &tmB1 : &tmB, kb * (kBK / 2),
+                                     nt * 256 + (int)rank * 128, fb);
                     tma_load_3d_pair(smem_u32(st + k2AStage + k2BStage), &tmSA, 0, kb * 4, 2 * mt + (int)rank, fb);
                     tma_load_3d_pair(smem_u32(st + k2AStage + k2BStage + k2SfaStage), &tmSB, 0, kb * 4, 2 * nt,
                                      fb);
@@ -685,7 +705,7 @@ w4a4_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                 }
                 tc_fence_after();
                 bool ok = true;
-                for (int kb = 0; kb < p.kblocks; ++kb) {
+                for (int kb = 0; kb < p.kiters; ++kb) {
                     // the scale warps observed the stage's full barrier (cluster
                     // acquire) before their copies; their commits complete this
                     // barrier only after the copies, so the stage is in place
@@ -736,7 +756,7 @@ w4a4_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
             bool issued_any = false;
             for (int tile = cluster; tile < num_tiles && !*abort_flag; tile += nclusters) {
                 bool ok = true;
-                for (int kb = 0; kb < p.kblocks; ++kb) {
+                for (int kb = 0; kb < p.kiters; ++kb) {
                     if (!mbar_wait_cluster(full_bar(stage), phase, abort_flag) || *abort_flag) {
                         give_up();
                         ok = false;
@@ -930,9 +950,25 @@ bool gemm_shape_supported(int64_t M, int64_t N, int64_t K)
 
 cudaError_t launch_w4a4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* ga,
                              const uint8_t* w_codes, const uint8_t* w_sf, const float* gw, int64_t M,
-                             int64_t N, int64_t K, void* out, int* err, cudaStream_t s)
+                             int64_t N, int64_t K, void* out, int* err, cudaStream_t s,
+                             const uint8_t* a1_codes, const uint8_t* w1_codes)
 {
     GemmParams p;
+    // passes in K-block order: (A, W), then (A, W1), (A1, W), (A1, W1) as present
+    {
+        int sels[4], n = 0;
+        sels[n++] = 0;
+        if (w1_codes)
+            sels[n++] = 2;
+        if (a1_codes)
+            sels[n++] = 1;
+        if (a1_codes && w1_codes)
+            sels[n++] = 3;
+        p.pass_shift = n == 1 ? 0 : n == 2 ? 1 : 2;
+        p.pass_sel = 0;
+        for (int i = 0; i < n; ++i)
+            p.pass_sel |= sels[i] << (2 * i);
+    }
     p.sfa = a_sf;
     p.sfb = w_sf;
     p.ga = ga;
@@ -943,12 +979,16 @@ cudaError_t launch_w4a4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const 
     p.kblocks = (int)(K / kBK);
     p.kb_atoms = (int)(K / 64);
     p.N = (int)N;
+    p.kiters = p.kblocks << p.pass_shift;
+    const uint8_t* a1 = a1_codes ? a1_codes : a_codes;
+    const uint8_t* w1 = w1_codes ? w1_codes : w_codes;
     if (M % 256 == 0) {
         // CTA pairs: 256 x 256 tiles
-        CUtensorMap ta, tb, tsa, tsb, to;
+        CUtensorMap ta, tb, tsa, tsb, to, ta1, tb1;
         if (!make_code_map(&ta, a_codes, M, K / 2, 128) || !make_code_map(&tb, w_codes, N, K / 2, 128) ||
             !make_sf_map(&tsa, a_sf, M, K, 1) || !make_sf_map(&tsb, w_sf, N, K, 2) ||
-            !make_out_map(&to, out, M, N))
+            !make_out_map(&to, out, M, N) || !make_code_map(&ta1, a1, M, K / 2, 128) ||
+            !make_code_map(&tb1, w1, N, K / 2, 128))
             return cudaErrorInvalidValue;
         static std::once_flag attr2_once;
         static cudaError_t attr2_err = cudaSuccess;
@@ -962,12 +1002,13 @@ cudaError_t launch_w4a4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const 
         const int tiles = p.tiles_m * p.tiles_n;
         const int pairs = num_sms() / 2;
         const int grid = 2 * (tiles < pairs ? tiles : pairs);
-        w4a4_gemm_2sm_kernel<<<grid, k2Threads, k2SmemBytes, s>>>(ta, tb, tsa, tsb, to, p);
+        w4a4_gemm_2sm_kernel<<<grid, k2Threads, k2SmemBytes, s>>>(ta, tb, tsa, tsb, to, ta1, tb1, p);
         return cudaGetLastError();
     }
-    CUtensorMap ta, tb, tsa, tsb;
+    CUtensorMap ta, tb, tsa, tsb, ta1, tb1;
     if (!make_code_map(&ta, a_codes, M, K / 2, kBM) || !make_code_map(&tb, w_codes, N, K / 2, kBN) ||
-        !make_sf_map(&tsa, a_sf, M, K, 1) || !make_sf_map(&tsb, w_sf, N, K, 2))
+        !make_sf_map(&tsa, a_sf, M, K, 1) || !make_sf_map(&tsb, w_sf, N, K, 2) ||
+        !make_code_map(&ta1, a1, M, K / 2, kBM) || !make_code_map(&tb1, w1, N, K / 2, kBN))
         return cudaErrorInvalidValue;
     static std::once_flag attr_once;
     static cudaError_t attr_err = cudaSuccess;
@@ -980,7 +1021,7 @@ cudaError_t launch_w4a4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const 
     p.tiles_m = (int)(M / kBM);
     const int tiles = p.tiles_m * p.tiles_n;
     const int grid = tiles < num_sms() ? tiles : num_sms();
-    w4a4_gemm_1sm_kernel<<<grid, kThreads, kSmemBytes, s>>>(ta, tb, tsa, tsb, p);
+    w4a4_gemm_1sm_kernel<<<grid, kThreads, kSmemBytes, s>>>(ta, tb, tsa, tsb, ta1, tb1, p);
     return cudaGetLastError();
 }
 

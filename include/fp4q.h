@@ -327,6 +327,57 @@ FP4Q_API int w4a4_gemm(const void* a, int a_format, int a_rule, const uint8_t* a
                        size_t workspace_bytes, void* stream);
 
 /*
+ * RaZeR operands for the tensor-core GEMM ([RaZeR] 2.2: the -0 code of a
+ * block stands for the block's special value; [RaZeR] 2.3: the Blackwell
+ * kernels handle the remapping in two passes on the existing tensor cores).
+ * Splits RaZeR codes into two E2M1 tensors that share one set of E4M3 block
+ * scales: every special value v is written as p + q with p, q E2M1 values
+ * (p the largest magnitude of v's sign leaving an E2M1 remainder: +-5 =
+ * +-(4 + 1), +-3.5 = +-(3 + 0.5)),
+ *   main_codes   the codes with each -0 replaced by p of the block's selector
+ *   extra_codes  q at the -0 positions, +0 everywhere else
+ * so v_main * sc + v_extra * sc equals the RaZeR value v * sc exactly.
+ *
+ *  codes, meta    device, razer_quantize output: rows*cols/2 code bytes
+ *                 (16-byte aligned) and rows*cols/16 meta bytes
+ *  scale_fmt      FP4Q_SF_E3M3 (meta = sel<<6 | e3m3, up to 4 specials) or
+ *                 FP4Q_SF_E4M3 (meta = sel<<7 | e4m3, up to 2)
+ *  specials       host, the table razer_quantize was given
+ *  main_codes, extra_codes   device, rows*cols/2 bytes each (out), 16-byte aligned
+ *  scales_mma     device, rows*cols/16 E4M3 bytes in FP4Q_SFLAYOUT_MMA (out)
+ *                 (E3M3 values are E4M3 values: the conversion is exact)
+ *  rows % 128 == 0, cols % 64 == 0 (FP4Q_ERR_ARG otherwise).
+ * Errors: ERR_ARG (sizes, format, table), ERR_UNSUPPORTED (a special that is
+ * not the sum of two E2M1 values, e.g. 5.5 = 4 + 1.5 is fine, 11 is not),
+ * ERR_ALIGN, ERR_CUDA.  Weights are prepared once, offline.
+ */
+FP4Q_API int razer_gemm_prepare(const uint8_t* codes, const uint8_t* meta, int64_t rows, int64_t cols,
+                                int scale_fmt, const float* specials, int n_special,
+                                uint8_t* main_codes, uint8_t* extra_codes, uint8_t* scales_mma,
+                                void* stream);
+
+/*
+ * RaZeR-aware W4A4 GEMM: out = bf16(g_a * g_w * (A + A1) . (W + W1)^T) where
+ * A, A1 (and W, W1) are E2M1 code tensors sharing the block scales a_scales
+ * (w_scales) -- the razer_gemm_prepare split of a RaZeR operand, or a plain
+ * NVFP4 operand with its extra tensor NULL.  Each present pair of tensors is
+ * one pass over K into the same fp32 TMEM accumulator (2 passes for RaZeR
+ * weights, 4 when both operands are RaZeR).
+ *
+ *  a_codes, a_extra (nullable)   device M*K/2 bytes; a_scales E4M3 MMA layout;
+ *                                a_global_scale device g_a
+ *  w_codes, w_extra (nullable)   device N*K/2 bytes; w_scales E4M3 MMA layout;
+ *                                w_global_scale device g_w
+ *  shapes, out, workspace (>= 8 KiB) and errors as w4a4_gemm; fp4q_gemm_status
+ *  reports a device timeout.
+ */
+FP4Q_API int razer_w4a4_gemm(const uint8_t* a_codes, const uint8_t* a_extra, const uint8_t* a_scales,
+                             const float* a_global_scale, const uint8_t* w_codes,
+                             const uint8_t* w_extra, const uint8_t* w_scales,
+                             const float* w_global_scale, int64_t M, int64_t N, int64_t K, void* out,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Synchronizes `stream` and reports whether the last w4a4_gemm that used this
  * workspace finished normally (FP4Q_OK) or gave up a bounded device-side wait
  * (FP4Q_ERR_TIMEOUT; its output is then incomplete).

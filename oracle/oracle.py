@@ -346,6 +346,38 @@ def nvfp4_decode_exact(codes, scales, block: int = 16):
     return v * np.repeat(sc, block, axis=1)
 
 
+def razer_decode_exact(codes, meta, sf: int, specials):
+    """RaZeR values in fp64 (exact), "RaZeR: Redundant Zero Remapping" section
+    2.2: every code decodes to its E2M1 value except -0 (code 8), which takes the
+    block's special value specials[sel]; times the block scale (E3M3 for
+    weights, meta = sel<<6 | code; E4M3 for activations, meta = sel<<7 | code)."""
+    codes = np.asarray(codes, np.uint8)
+    meta = np.asarray(meta, np.uint8)
+    rows, cols = codes.shape[0], codes.shape[1] * 2
+    e2 = np.array([e2m1_value(c) for c in range(16)], np.float64)
+    c = np.empty((rows, cols), np.int64)
+    c[:, 0::2] = codes & 0xF
+    c[:, 1::2] = codes >> 4
+    if sf == SF_E3M3:
+        sel, sc_code = meta >> 6, meta & 0x3F
+        sc = np.array([e3m3_value(int(k)) for k in range(64)], np.float64)[sc_code]
+    elif sf == SF_E4M3:
+        sel, sc_code = meta >> 7, meta & 0x7F
+        sc = np.array([e4m3_value(int(k)) for k in range(128)], np.float64)[sc_code]
+    else:
+        raise ValueError("RaZeR scales are E3M3 or E4M3")
+    sp = np.asarray(specials, np.float64)
+    v = e2[c]
+    special = np.repeat(sp[sel], 16, axis=1)
+    v = np.where(c == 8, special, v)
+    return v * np.repeat(sc, 16, axis=1)
+
+
+def gemm_values(da, dw, g_a, g_w):
+    """out = g_a * g_w * (da @ dw^T) in fp64 for exactly decoded operands."""
+    return (float(g_a) * float(g_w)) * (np.asarray(da, np.float64) @ np.asarray(dw, np.float64).T)
+
+
 def gemm_ref(a_codes, a_scales, g_a, w_codes, w_scales, g_w, rows=None, cols=None):
     """out = g_a * g_w * (deqA @ deqW^T) in fp64, optionally for a subset of rows / cols."""
     if rows is not None:

@@ -92,3 +92,39 @@ def test_gemm_reference_matches_triple_loop(O):
     sub = O.gemm_ref(qa["codes"], qa["scales"], ga, qw["codes"], qw["scales"], gw,
                      rows=np.array([1, 4]), cols=np.array([0, 3]))
     assert np.array_equal(sub, ref[np.ix_([1, 4], [0, 3])])
+
+
+@pytest.mark.parametrize("sf,kind,specials", [(1, "razer_weight", [5.0, -5.0, 3.5, -3.5]),
+                                              (0, "razer_act", [5.0, -5.0])])
+def test_razer_decode_exact_matches_quantizer(O, sf, kind, specials):
+    """With g = 1 every RaZeR value v * sc is exact in fp32, so the exact decode
+    equals the quantizer's own fused dequantization (separate C code path)."""
+    x = _x(kind, 16, 256, seed=7 + sf)
+    q = O.razer_quantize(x, sf, specials, g=1.0)
+    d = O.razer_decode_exact(q["codes"], q["meta"], sf, specials)
+    assert np.array_equal(d, q["deq"].astype(np.float64))
+    lo, hi = q["codes"] & 0xF, q["codes"] >> 4
+    assert ((lo == 8) | (hi == 8)).any()           # specials do occur
+
+
+def test_razer_gemm_reference_matches_triple_loop(O):
+    a = _x("razer_act", 6, 64, seed=2)
+    w = _x("razer_weight", 5, 64, seed=2)
+    spa, spw = [5.0, -5.0], [5.0, -5.0, 3.5, -3.5]
+    ga = O.global_scale(O.amax(a), O.SF_E4M3)
+    gw = O.global_scale(O.amax(w), O.SF_E3M3)
+    qa = O.razer_quantize(a, O.SF_E4M3, spa, g=ga)
+    qw = O.razer_quantize(w, O.SF_E3M3, spw, g=gw)
+    ref = O.gemm_values(O.razer_decode_exact(qa["codes"], qa["meta"], O.SF_E4M3, spa),
+                        O.razer_decode_exact(qw["codes"], qw["meta"], O.SF_E3M3, spw), ga, gw)
+    # operand values from the C dequantizer at g = 1 (exact v * sc)
+    va = O.dequant_mse(qa["codes"], qa["meta"], 6, 64, 16, O.SF_E4M3, spa)["deq"].astype(np.float64)
+    vw = O.dequant_mse(qw["codes"], qw["meta"], 5, 64, 16, O.SF_E3M3, spw)["deq"].astype(np.float64)
+    for m in range(6):
+        for n in range(5):
+            acc = 0.0
+            for k in range(64):
+                acc += va[m, k] * vw[n, k]
+            assert abs(ref[m, n] - float(ga) * float(gw) * acc) <= 1e-12 * max(1.0, abs(ref[m, n]))
+    exact = a.astype(np.float64) @ w.astype(np.float64).T
+    assert np.linalg.norm(ref - exact) <= 0.2 * np.linalg.norm(exact)
