@@ -733,7 +733,8 @@ nvfp4_bf_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs,
     // the format's largest finite code, and the "no all-zero code" marker
     constexpr uint32_t kLast = SFMT == 1 ? 254u : 126u;
     // codes each lane evaluates itself before the warp shares out the rest
-    constexpr int kDirect = B <= 8 ? 3 : 2;
+    // (measured on the Student-t block sweep: 3 for B <= 8, 5 above)
+    constexpr int kDirect = B <= 8 ? 3 : 5;
     constexpr uint32_t kNone = kLast + 1u;
     // (S, inv) of every code: S = sc * g, inv = min(1/S, FLT_MAX), 0 for S = 0
     __shared__ float2 tab[kNone + 1];
@@ -795,13 +796,24 @@ nvfp4_bf_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs,
         // boundary (|y| is monotone in the code)
         uint32_t cz = sf_encode<SFMT>(__fmul_rn(a, four_over_g));
         cz = cz == 0u ? 1u : cz;
-        if (__fmul_rn(a, tab[cz].y) <= 0.25f) {
-            while (cz > 1u && __fmul_rn(a, tab[cz - 1u].y) <= 0.25f)
-                --cz;
-        } else {
-            do {
+        {
+            // usually the boundary is cz or cz + 1: test both without a loop
+            const bool f0 = cz > 1u && __fmul_rn(a, tab[cz - 1u].y) <= 0.25f;
+            const bool f1 = __fmul_rn(a, tab[cz].y) <= 0.25f;
+            const bool f2 = cz + 1u >= kNone || __fmul_rn(a, tab[cz + 1u].y) <= 0.25f;
+            if (f1 && !f0) {
+            } else if (!f1 && f2) {
                 ++cz;
-            } while (cz < kNone && __fmul_rn(a, tab[cz].y) > 0.25f);
+            } else if (f1) {
+                --cz;
+                while (cz > 1u && __fmul_rn(a, tab[cz - 1u].y) <= 0.25f)
+                    --cz;
+            } else {
+                ++cz;
+                do {
+                    ++cz;
+                } while (cz < kNone && __fmul_rn(a, tab[cz].y) > 0.25f);
+            }
         }
         n_eval += (valid && cz < kNone) ? 1u : 0u;
         if (cz < kNone && (sse0 < best || (sse0 == best && cz < bc))) {
@@ -818,12 +830,14 @@ nvfp4_bf_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs,
             --clo;
         }
         int chi = (int)(cz < kNone ? cz : kNone) - 1;   // last code to evaluate
-        // the first kDirect codes of the range straight from registers (most
-        // blocks need no more); the rest is shared out across the warp
+        // the first kDirect codes of the range other than c6 straight from
+        // registers (most blocks need no more); the rest is shared out across
+        // the warp.  Code list: clo, clo + 1, ... with c6 left out.
 #pragma unroll
         for (int s = 0; s < kDirect; ++s) {
-            const uint32_t c = clo + (uint32_t)s;
-            if (valid && (int)c <= chi && c != c6) {
+            uint32_t c = clo + (uint32_t)s;
+            c += c >= c6 ? 1u : 0u;
+            if (valid && (int)c <= chi) {
                 const float sc_ = quant_sse<B>(xv, 0.0f, 0.0f, tab[c]);
                 n_eval += 1u;
                 if (sc_ < best || (sc_ == best && c < bc)) {
@@ -832,8 +846,8 @@ nvfp4_bf_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs,
                 }
             }
         }
-        clo = min(clo + (uint32_t)kDirect, (uint32_t)(chi + 1));   // <= kNone: fits the 8-bit field
-        int span = chi - (int)clo + 1;
+        // codes left after the direct ones (c6 <= chi unless the block is all zero)
+        int span = chi - (int)clo + 1 - ((int)c6 <= chi ? 1 : 0) - kDirect;
         span = (valid && span > 0) ? span : 0;
 
         // lay the warp's candidates end to end
@@ -852,7 +866,7 @@ nvfp4_bf_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs,
                     make_float4(xv[i], xv[i + 1], xv[i + 2], xv[i + 3]);
             key[w][lane] = ((unsigned long long)__float_as_uint(best) << 32) | bc;
             pre[w][lane] = incl - span;
-            meta[w][lane] = clo | (c6 << 8);
+            meta[w][lane] = clo | (c6 << 8);   // clo <= c6 <= kLast: 8 bits each
             __syncwarp();
             for (int t = lane; t < total; t += 32) {
                 // owner: the last block whose range starts at or before t
@@ -862,9 +876,8 @@ nvfp4_bf_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs,
                     if (pre[w][j + st] <= t)
                         j += st;
                 const uint32_t m = meta[w][j];
-                const uint32_t c = (m & 0xFFu) + (uint32_t)(t - pre[w][j]);
-                if (c == (m >> 8))
-                    continue;
+                uint32_t c = (m & 0xFFu) + (uint32_t)(kDirect + t - pre[w][j]);
+                c += c >= (m >> 8) ? 1u : 0u;
                 float xj[B];
 #pragma unroll
                 for (int i = 0; i < B; i += 4) {
