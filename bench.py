@@ -222,6 +222,36 @@ def build_rows(torch, fq, inputs, dev, host_copies=None, groups=None):
                                  workspace=wsf)
         rows.append(Row("c4_mx_weight_flip", "flip_refine_kernel", 0, w4.size * (2 + 0.5 + 0.5 + 1 / 32) + C * 32 * 4,
                         1, c4f, {"moves": mv4}, bound="alu", flops=2.0 * N4 * (C // 32) * 32 * 32, extra=True))
+
+        # MXFP4 GEMM (next rows) at the size the MACaQ review quotes the online
+        # transform's overhead at: these activations (8192 x 4096) against
+        # 16384 x 4096 MXFP4 weights (1/t, rotation, quantized once, offline).
+        # (a) packed activations: the GEMM alone; (b) dense bf16 activations:
+        # the prologue (x * t, rotation, E8M0, the GEMM's scale layout) + GEMM.
+        N3 = 16384
+        w3d = torch.from_numpy(inputs.generate("mx_weight", N3, C, seed=3).view(np.int16)).to(dev).view(torch.bfloat16)
+        t3 = torch.from_numpy(inputs.positive_vector(C, seed=3)).to(dev)
+        ti3 = 1.0 / t3.double()
+        ti3 = ti3.float()
+        qw3 = fq.mxfp4_quantize(w3d, ti3, True, fq.ABSMAX)
+        del w3d
+        w3sc = fq.scales_to_mma(qw3["scales"])
+        qa3 = fq.mxfp4_quantize(X["c4x"], t3, True, fq.ABSMAX)
+        a3sc = fq.scales_to_mma(qa3["scales"])
+        y3 = torch.empty((T, N3), dtype=torch.bfloat16, device=dev)
+        ws3 = torch.empty(fq.workspace_size(fq.OP_MX_GEMM, T, C, N3), dtype=torch.uint8, device=dev)
+
+        def f3p():
+            fq.mxfp4_gemm(qa3["codes"], qw3["codes"], w3sc, a_scales=a3sc, out=y3, workspace=ws3)
+
+        def f3d():
+            fq.mxfp4_gemm(X["c4x"], qw3["codes"], w3sc, chan_scale=t3, out=y3, workspace=ws3)
+        mxg_bytes = T * C * (0.5 + 1 / 32) + N3 * C * (0.5 + 1 / 32) + T * N3 * 2
+        rows.append(Row("f3_mx_gemm_packed", "w4a4_gemm_2sm_kernel<true>", 0, mxg_bytes, 1, f3p, {"out": y3},
+                        bound="tensor", flops=2.0 * T * N3 * C, extra=True))
+        rows.append(Row("f3_mx_gemm_with_prologue", "mx_quant_absmax_kernel + w4a4_gemm_2sm_kernel<true>", 0,
+                        mxg_bytes + T * C * 2, 2, f3d, {"out": y3}, bound="tensor", flops=2.0 * T * N3 * C,
+                        extra=True))
     if groups is None or "c5" in groups:
         # c5: weights pre-quantized once (abs-max NVFP4, hierarchical scale, MMA
         # scale layout) outside the timed step; the step quantizes the activations
@@ -247,7 +277,7 @@ def build_rows(torch, fq, inputs, dev, host_copies=None, groups=None):
             fq.w4a4_gemm(o5["codes"], qw5["codes"], qw5["scales"], qw5["global_scale"], a_scales=o5["scales"],
                          a_global_scale=o5["global_scale"], K=K5, out=y5, workspace=wsg)
         rows.append(Row("c5_act_quant_4o6_mma", "nvfp4_quant_kernel<16, __nv_bfloat16, 2, 0>", a5.size, a5.size * (2 + 0.5 + 1 / 16), 2, c5, o5))
-        rows.append(Row("c5_w4a4_gemm", "w4a4_gemm_2sm_kernel", 0, M5 * K5 * (0.5 + 1 / 16) + N5 * K5 * (0.5 + 1 / 16) + M5 * N5 * 2,
+        rows.append(Row("c5_w4a4_gemm", "w4a4_gemm_2sm_kernel<false>", 0, M5 * K5 * (0.5 + 1 / 16) + N5 * K5 * (0.5 + 1 / 16) + M5 * N5 * 2,
                         1, c5g, {"out": y5}, bound="tensor", flops=2.0 * M5 * N5 * K5))
 
         # RaZeR-aware GEMM (next rows): the same weights quantized with RaZeR
@@ -280,13 +310,13 @@ def build_rows(torch, fq, inputs, dev, host_copies=None, groups=None):
                                workspace=wsr)
         rows.append(Row("f2_razer_prepare_weights", "razer_prepare_kernel<1>", N5 * K5,
                         N5 * K5 * (0.5 + 1 / 16) + N5 * K5 * (0.5 + 0.5 + 1 / 16), 1, f2p, pwo, extra=True))
-        rows.append(Row("f2_razer_gemm_w_2pass", "w4a4_gemm_2sm_kernel", 0,
+        rows.append(Row("f2_razer_gemm_w_2pass", "w4a4_gemm_2sm_kernel<false>", 0,
                         M5 * K5 * (0.5 + 1 / 16) + N5 * K5 * (1.0 + 1 / 16) + M5 * N5 * 2, 1, f2w, {"out": y5},
                         bound="tensor", flops=2.0 * M5 * N5 * K5, extra=True))
         rows.append(Row("f2_razer_act_quant_prep", "razer_paired_kernel<__nv_bfloat16, 0, 1>", a5.size,
                         a5.size * (2 + 0.5 + 1 / 16) + a5.size * (0.5 + 1 / 16 + 1.0 + 1 / 16), 3, f2aq, pa5,
                         extra=True))
-        rows.append(Row("f2_razer_gemm_wa_4pass", "w4a4_gemm_2sm_kernel", 0,
+        rows.append(Row("f2_razer_gemm_wa_4pass", "w4a4_gemm_2sm_kernel<false>", 0,
                         M5 * K5 * (1.0 + 1 / 16) + N5 * K5 * (1.0 + 1 / 16) + M5 * N5 * 2, 1, f2wa, {"out": y5},
                         bound="tensor", flops=2.0 * M5 * N5 * K5, extra=True))
     return rows, X
@@ -458,7 +488,9 @@ def main():
     hbm_peak, sm_max_mhz, bf16_peak, bf16_sust, peak_src = load_peaks()
 
     if args.profile_row:
-        rows, X = build_rows(torch, fq, inputs, dev, None, groups={args.profile_row[:2]})
+        # the next rows f2 / f3 are built with the workloads they extend
+        grp = {"f2": "c5", "f3": "c4"}.get(args.profile_row[:2], args.profile_row[:2])
+        rows, X = build_rows(torch, fq, inputs, dev, None, groups={grp})
         target = [r for r in rows if r.name == args.profile_row]
         if not target:
             raise SystemExit("unknown row %s; rows: %s" % (args.profile_row, [r.name for r in rows]))
@@ -617,7 +649,7 @@ def main():
                          "3 repeats, %.1f s each" % (elems, FULL_ELEMS, sec)}
 
     launches = sum(r.launches for r in hot) * args.steps
-    gem = next((r for r in rows if r.bound == "tensor"), None)
+    gem = next((r for r in rows if r.name == "c5_w4a4_gemm"), None)
     gemm = None
     if gem is not None:
         g = row_out[gem.name]

@@ -15,12 +15,12 @@ import torch
 
 from . import build as _build
 
-F32, BF16, NVFP4_PACKED = 0, 1, 2
+F32, BF16, NVFP4_PACKED, MXFP4_PACKED = 0, 1, 2, 3
 SF_E4M3, SF_E3M3, SF_E8M0, SF_UE5M3 = 0, 1, 2, 3
 ABSMAX, PREVENT_ZERO, FOUR_OVER_SIX, BRUTE_FORCE, HESSIAN_EXP = range(5)
 GS_NONE, GS_AMAX, GS_GIVEN = 0, 1, 2
 SF_ROWMAJOR, SF_MMA = 0, 1
-OP_QUANTIZE, OP_HESSIAN, OP_CHANNEL_SCALE, OP_GEMM, OP_FLIP = range(5)
+OP_QUANTIZE, OP_HESSIAN, OP_CHANNEL_SCALE, OP_GEMM, OP_FLIP, OP_MX_GEMM = range(6)
 # byte offset, in a quantize workspace, of the uint64 that brute force adds its
 # evaluation count to (FP4Q_WS_BF_EVALS)
 WS_BF_EVALS = 3072
@@ -44,6 +44,8 @@ SIGNATURES = {
     "fp4q_gemm_status": (_i, [_vp, _vp]),
     "razer_gemm_prepare": (_i, [_vp, _vp, _i64, _i64, _i, _vp, _i, _vp, _vp, _vp, _vp]),
     "razer_w4a4_gemm": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _sz, _vp]),
+    "fp4_scales_to_mma": (_i, [_vp, _i64, _i64, _vp, _vp]),
+    "mxfp4_gemm": (_i, [_vp, _i, _vp, _vp, _i, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _sz, _vp]),
 }
 
 _lock = threading.Lock()
@@ -327,6 +329,44 @@ def razer_w4a4_gemm(a_codes: torch.Tensor, a_scales: torch.Tensor, a_global_scal
                                _ptr(w_codes), _ptr(w_extra), _ptr(w_scales), _ptr(w_global_scale),
                                M, N, K, _ptr(o), _ptr(ws), ws.numel(), _stream(stream))
     _check(st, "razer_w4a4_gemm")
+    return o
+
+
+def scales_to_mma(scales: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Row-major scale bytes [rows, nscales] -> the MMA scale layout (flat uint8)."""
+    _need_cuda(scales, out)
+    rows, n = scales.shape
+    o = out if out is not None else torch.empty((rows * n,), dtype=torch.uint8, device=scales.device)
+    _check(lib().fp4_scales_to_mma(_ptr(scales), rows, n, _ptr(o), _stream(stream)), "fp4_scales_to_mma")
+    return o
+
+
+def mxfp4_gemm(a: torch.Tensor, w_codes: torch.Tensor, w_scales: torch.Tensor,
+               a_scales: torch.Tensor | None = None, chan_scale: torch.Tensor | None = None,
+               hadamard: bool = True, K: int | None = None, out: torch.Tensor | None = None,
+               workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """out = A' . W'^T in bf16 with MXFP4 operands.  `a` is a dense fp32/bf16 [M, K] tensor
+    (transformed with chan_scale and the 32-block rotation and quantized in the call) or packed
+    MXFP4 codes [M, K/2] uint8 with `a_scales` (E8M0, MMA layout).  W: codes [N, K/2] with
+    E8M0 scales in the MMA layout."""
+    _need_cuda(a, w_codes, w_scales, a_scales, chan_scale)
+    if a.dtype == torch.uint8:
+        fmt = MXFP4_PACKED
+        M = a.shape[0]
+        K = a.shape[1] * 2 if K is None else K
+    else:
+        fmt = _dtype_code(a)
+        M, K = a.shape
+    N = w_codes.shape[0]
+    dev = a.device
+    o = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    ws, wsb = (workspace, workspace.numel()) if workspace is not None else _workspace(OP_MX_GEMM, M, K, N, dev, None)
+    if fmt == MXFP4_PACKED and ws is None:
+        ws = torch.empty(8192, dtype=torch.uint8, device=dev)
+        wsb = ws.numel()
+    st = lib().mxfp4_gemm(_ptr(a), fmt, _ptr(a_scales), _ptr(chan_scale), int(bool(hadamard)), _ptr(w_codes),
+                          _ptr(w_scales), M, N, K, _ptr(o), _ptr(ws), wsb, _stream(stream))
+    _check(st, "mxfp4_gemm")
     return o
 
 

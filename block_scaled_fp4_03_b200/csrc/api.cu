@@ -30,6 +30,7 @@ constexpr size_t kGemmHeader = 8192;
 constexpr size_t kGemmGa = 4096;
 constexpr size_t kGemmErr = 4160;
 size_t gemm_ws_bytes(int64_t M, int64_t K) { return kGemmHeader + (size_t)M * (size_t)K / 2 + (size_t)M * (size_t)K / 16; }
+size_t mx_gemm_ws_bytes(int64_t M, int64_t K) { return kGemmHeader + (size_t)M * (size_t)K / 2 + (size_t)M * (size_t)K / 32; }
 static_assert(kAmaxPartials * sizeof(float) <= FP4Q_WS_BF_EVALS && FP4Q_WS_BF_EVALS + 8 <= kQuantWs,
               "amax partials and the evaluation counter must fit");
 
@@ -75,6 +76,7 @@ size_t fp4q_workspace_size(int op, int64_t rows, int64_t cols, int64_t n)
     case FP4Q_OP_HESSIAN: return cols % 32 ? 0 : hessian_ws_bytes(rows, cols);
     case FP4Q_OP_CHANNEL_SCALE: return channel_scale_ws_bytes(rows, n, cols);
     case FP4Q_OP_GEMM: return gemm_ws_bytes(rows, cols);
+    case FP4Q_OP_MX_GEMM: return mx_gemm_ws_bytes(rows, cols);
     default: return 0;
     }
 }
@@ -464,6 +466,61 @@ int razer_w4a4_gemm(const uint8_t* a_codes, const uint8_t* a_extra, const uint8_
         return FP4Q_ERR_CUDA;
     return from_cuda(launch_w4a4_gemm(a_codes, a_scales, a_global_scale, w_codes, w_scales, w_global_scale,
                                       M, N, K, out, err, s, a_extra, w_extra));
+}
+
+int fp4_scales_to_mma(const uint8_t* scales, int64_t rows, int64_t nscales, uint8_t* out, void* stream)
+{
+    if (rows < 0 || nscales < 0 || rows % 128 != 0 || nscales % 4 != 0)
+        return FP4Q_ERR_ARG;
+    if (rows == 0 || nscales == 0)
+        return FP4Q_OK;
+    if (!scales || !out)
+        return FP4Q_ERR_ARG;
+    if (!aligned16(scales) || !aligned16(out))
+        return FP4Q_ERR_ALIGN;
+    return from_cuda(launch_scales_to_mma(scales, rows, nscales, out, as_stream(stream)));
+}
+
+int mxfp4_gemm(const void* a, int a_format, const uint8_t* a_scales, const float* chan_scale,
+               int hadamard32, const uint8_t* w_codes, const uint8_t* w_scales, int64_t M, int64_t N,
+               int64_t K, void* out, void* workspace, size_t workspace_bytes, void* stream)
+{
+    if (!a || !w_codes || !w_scales || !out || !workspace)
+        return FP4Q_ERR_ARG;
+    if (a_format != FP4Q_F32 && a_format != FP4Q_BF16 && a_format != FP4Q_MXFP4_PACKED)
+        return FP4Q_ERR_ARG;
+    if (a_format == FP4Q_MXFP4_PACKED && (!a_scales || chan_scale))
+        return FP4Q_ERR_ARG;
+    if (M <= 0 || N <= 0 || K <= 0)
+        return FP4Q_ERR_ARG;
+    if (!gemm_shape_supported(M, N, K))
+        return FP4Q_ERR_UNSUPPORTED;
+    if (!aligned16(a) || !aligned16(w_codes) || !aligned16(w_scales) || !aligned16(out) ||
+        !aligned16(workspace) || !aligned_or_null(a_scales) || !aligned_or_null(chan_scale))
+        return FP4Q_ERR_ALIGN;
+    const size_t need = a_format == FP4Q_MXFP4_PACKED ? kGemmHeader : mx_gemm_ws_bytes(M, K);
+    if (workspace_bytes < need)
+        return FP4Q_ERR_WORKSPACE;
+    cudaStream_t s = as_stream(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    int* err = reinterpret_cast<int*>(ws + kGemmErr);
+    if (cudaMemsetAsync(err, 0, sizeof(int), s) != cudaSuccess)
+        return FP4Q_ERR_CUDA;
+    const uint8_t* a_codes = static_cast<const uint8_t*>(a);
+    const uint8_t* a_sf = a_scales;
+    if (a_format != FP4Q_MXFP4_PACKED) {
+        // the prologue: u = a * t, block rotation, E8M0 quantization, scales
+        // written straight into the GEMM's layout
+        uint8_t* qcodes = ws + kGemmHeader;
+        uint8_t* qsf = qcodes + (size_t)M * (size_t)K / 2;
+        if (launch_mxfp4_quant(a, a_format, M, K, chan_scale, hadamard32 != 0, FP4Q_ABSMAX, nullptr, qcodes,
+                               qsf, nullptr, nullptr, s, 1) != cudaSuccess)
+            return FP4Q_ERR_CUDA;
+        a_codes = qcodes;
+        a_sf = qsf;
+    }
+    return from_cuda(launch_w4a4_gemm(a_codes, a_sf, nullptr, w_codes, w_scales, nullptr, M, N, K, out, err, s,
+                                      nullptr, nullptr, 1));
 }
 
 }  // extern "C"

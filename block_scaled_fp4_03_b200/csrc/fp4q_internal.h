@@ -50,10 +50,11 @@ cudaError_t launch_hessian_blocks(const void* x, int dtype, int64_t rows, int64_
                                   const float* chan_scale, int hadamard, float* hess, void* ws,
                                   cudaStream_t s);
 
+// mma_layout: scales in the MMA scale layout (rows % 128 == 0, cols % 128 == 0)
 cudaError_t launch_mxfp4_quant(const void* x, int dtype, int64_t rows, int64_t cols,
                                const float* chan_scale, int hadamard, int rule, const float* hess,
                                uint8_t* codes, uint8_t* scales, float* deq, float* mse,
-                               cudaStream_t s);
+                               cudaStream_t s, int mma_layout = 0);
 
 // Flip-Refinement of MX codes in place (exponents fixed); moves nullable.
 cudaError_t launch_mxfp4_flip_refine(const void* w, int dtype, int64_t rows, int64_t cols,
@@ -68,10 +69,18 @@ bool gemm_shape_supported(int64_t M, int64_t N, int64_t K);
 // a1_codes / w1_codes (nullable): second code tensors sharing the scales of
 // A / W; the GEMM then sums the products of every pair of present tensors,
 // out = (A + A1) . (W + W1)^T, as extra passes over K into one accumulator.
+// mx: MXFP4 operands (E8M0 scales per 32 elements in the MMA layout; ga, gw
+// NULL = no global scale).
 cudaError_t launch_w4a4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* ga,
                              const uint8_t* w_codes, const uint8_t* w_sf, const float* gw, int64_t M,
                              int64_t N, int64_t K, void* out, int* err, cudaStream_t s,
-                             const uint8_t* a1_codes = nullptr, const uint8_t* w1_codes = nullptr);
+                             const uint8_t* a1_codes = nullptr, const uint8_t* w1_codes = nullptr,
+                             int mx = 0);
+
+// Row-major scale bytes [rows][nscales] -> the MMA scale layout (rows % 128 == 0,
+// nscales % 4 == 0).
+cudaError_t launch_scales_to_mma(const uint8_t* scales, int64_t rows, int64_t nscales, uint8_t* out,
+                                 cudaStream_t s);
 
 // RaZeR codes + meta -> (main codes, extra codes, E4M3 scale bytes in the MMA
 // layout) with main + extra = the RaZeR values exactly.  p_code / q_code:

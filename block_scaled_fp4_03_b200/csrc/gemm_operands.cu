@@ -1,6 +1,10 @@
-// razer_gemm.cu -- RaZeR operands for the tensor-core GEMM.
+// gemm_operands.cu -- operand preparation for the tensor-core GEMM.
 //
-// A RaZeR block ("RaZeR: Redundant Zero Remapping" summary, section 2.2)
+// (1) Scale bytes from the row-major layout to the tcgen05 scale layout
+// (for operands quantized row-major, e.g. MXFP4 weights after
+// Flip-Refinement, which reads its exponents row-major).
+//
+// (2) RaZeR operands.  A RaZeR block ("RaZeR: Redundant Zero Remapping" summary, section 2.2)
 // decodes its -0 code to the block's special value sv (a multiple of 0.5,
 // section 2.2 value constraint) times the block scale; the tensor core decodes
 // -0 as zero.  The summary's Blackwell kernels handle the remapping in two
@@ -65,7 +69,34 @@ razer_prepare_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restric
     }
 }
 
+// One thread per 4 scale bytes of a row (one 32-bit word of an atom row).
+__global__ void __launch_bounds__(kPrepThreads)
+scales_to_mma_kernel(const uint8_t* __restrict__ scales, int64_t rows, int64_t nscales,
+                     uint8_t* __restrict__ out)
+{
+    const int64_t words = nscales >> 2;
+    const int64_t n = rows * words;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
+        const int64_t r = i / words;
+        const int64_t c = (i - r * words) * 4;
+        const uint32_t v = __ldg(reinterpret_cast<const uint32_t*>(scales + r * nscales + c));
+        *reinterpret_cast<uint32_t*>(out + mma_sf_offset(r, c, words)) = v;
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_scales_to_mma(const uint8_t* scales, int64_t rows, int64_t nscales, uint8_t* out,
+                                 cudaStream_t s)
+{
+    const int64_t n = rows * (nscales / 4);
+    int64_t want = (n + kPrepThreads - 1) / kPrepThreads;
+    const int64_t cap = (int64_t)num_sms() * 8;
+    const int grid = (int)(want < 1 ? 1 : (want > cap ? cap : want));
+    scales_to_mma_kernel<<<grid, kPrepThreads, 0, s>>>(scales, rows, nscales, out);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_razer_gemm_prepare(const uint8_t* codes, const uint8_t* meta, int64_t rows,
                                       int64_t cols, int sf, const uint8_t* p_code,

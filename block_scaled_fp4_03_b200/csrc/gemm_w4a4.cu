@@ -62,6 +62,38 @@ static_assert(kSmemBytes <= 232448, "shared memory budget");
 // mxf4nvf4 kind), K-major, UE4M3 scales, N = 256, M = 128, dense K = 64.
 constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | ((uint32_t)(kBN >> 3) << 17) |
                             ((uint32_t)(kBM >> 4) << 24);
+// Bit 23 of the descriptor selects UE8M0 scales (MXFP4: one E8M0 per 32).
+constexpr uint32_t kScaleUE8M0 = 1u << 23;
+
+// Scale atoms (128 rows x 4 scale bytes, 512 B) per row atom in one 256-wide
+// K stage: NVFP4 has 16 scales per row there (4 atoms), MXFP4 8 (2 atoms).
+template <bool MX>
+struct SfGeom {
+    static constexpr int kAtoms = MX ? 2 : 4;
+};
+
+// Scale-factor operands of MMA k-step s (K = 64 elements) of a stage, given
+// the TMEM columns of the stage's A and B scale atoms.  NVFP4: one atom per
+// k-step (4 scales per row).  MXFP4: one atom per two k-steps (2 scales per
+// row each), the second k-step reading bytes 2-3 of every 32-bit cell: the
+// byte offset goes into bits 31:30 of the scale address and the scale-factor
+// id fields of the instruction descriptor (bits 30:29 for A, 5:4 for B).
+template <bool MX>
+__device__ __forceinline__ void mma_scale_operands(int s, uint32_t tsfa, uint32_t tsfb, uint32_t idesc,
+                                                   uint32_t& sfa, uint32_t& sfb, uint32_t& id_out)
+{
+    if constexpr (MX) {
+        const uint32_t a = (uint32_t)s >> 1;
+        const uint32_t id = ((uint32_t)s & 1u) * 2u;
+        sfa = (tsfa + 4u * a) | (id << 30);
+        sfb = (tsfb + 8u * a) | (id << 30);
+        id_out = idesc | (id << 29) | (id << 4);
+    } else {
+        sfa = tsfa + 4u * (uint32_t)s;
+        sfb = tsfb + 8u * (uint32_t)s;
+        id_out = idesc;
+    }
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p)
 {
@@ -209,14 +241,22 @@ __device__ __forceinline__ void tc_cp_sf(uint32_t taddr, uint64_t sdesc)
     asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
+template <bool MX>
 __device__ __forceinline__ void tc_mma(uint32_t tacc, uint64_t da, uint64_t db, uint32_t idesc,
                                        uint32_t accumulate, uint32_t tsfa, uint32_t tsfb)
 {
-    asm volatile("{\n\t.reg .pred p;\n\t"
-                 "setp.ne.b32 p, %4, 0;\n\t"
-                 "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(tacc),
-                 "l"(da), "l"(db), "r"(idesc), "r"(accumulate), "r"(tsfa), "r"(tsfb)
-                 : "memory");
+    if constexpr (MX)
+        asm volatile("{\n\t.reg .pred p;\n\t"
+                     "setp.ne.b32 p, %4, 0;\n\t"
+                     "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(tacc),
+                     "l"(da), "l"(db), "r"(idesc), "r"(accumulate), "r"(tsfa), "r"(tsfb)
+                     : "memory");
+    else
+        asm volatile("{\n\t.reg .pred p;\n\t"
+                     "setp.ne.b32 p, %4, 0;\n\t"
+                     "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(tacc),
+                     "l"(da), "l"(db), "r"(idesc), "r"(accumulate), "r"(tsfa), "r"(tsfb)
+                     : "memory");
 }
 
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32])
@@ -272,6 +312,7 @@ __device__ __forceinline__ int pass_operands(const GemmParams& p, int j)
     return (p.pass_sel >> (2 * (j & ((1 << p.pass_shift) - 1)))) & 3;
 }
 
+template <bool MX>
 __global__ void __launch_bounds__(kThreads, 1)
 w4a4_gemm_1sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
@@ -339,14 +380,15 @@ w4a4_gemm_1sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                     const int kb = j >> p.pass_shift;
                     const int sel = pass_operands(p, j);
                     const uint32_t fb = full_bar(stage);
-                    mbar_expect_tx(fb, kStageBytes);
+                    mbar_expect_tx(fb, kAStage + kBStage + 3 * 512 * SfGeom<MX>::kAtoms);
                     uint8_t* st = smem + stage * kStageBytes;
                     tma_load_2d(smem_u32(st), (sel & 1) ? &tmA1 : &tmA, kb * (kBK / 2), mt * kBM, fb);
                     tma_load_2d(smem_u32(st + kAStage), (sel & 2) ? &tmB1 : &tmB, kb * (kBK / 2), nt * kBN, fb);
                     // scale atoms: 4 consecutive K atoms of row atom mt (A), of row
                     // atoms 2nt and 2nt+1 (B)
-                    tma_load_3d(smem_u32(st + kAStage + kBStage), &tmSA, 0, kb * 4, mt, fb);
-                    tma_load_3d(smem_u32(st + kAStage + kBStage + kSfaStage), &tmSB, 0, kb * 4, 2 * nt, fb);
+                    tma_load_3d(smem_u32(st + kAStage + kBStage), &tmSA, 0, kb * SfGeom<MX>::kAtoms, mt, fb);
+                    tma_load_3d(smem_u32(st + kAStage + kBStage + kSfaStage), &tmSB, 0, kb * SfGeom<MX>::kAtoms,
+                                2 * nt, fb);
                     issued |= 1u << stage;
                     issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
                     if (++stage == kStages) {
@@ -387,18 +429,22 @@ w4a4_gemm_1sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                     const uint32_t sb_s = sa_s + kSfaStage;
                     const uint32_t tsfa = tmem + kSfCol0 + (uint32_t)stage * kSfColsPerStage;
                     const uint32_t tsfb = tsfa + 16;
+                    constexpr int kAt = SfGeom<MX>::kAtoms;
 #pragma unroll
-                    for (int s = 0; s < 4; ++s) {
+                    for (int s = 0; s < kAt; ++s) {
                         tc_cp_sf(tsfa + 4 * s, sdesc_sf(sa_s + 512 * s));
                         tc_cp_sf(tsfb + 8 * s, sdesc_sf(sb_s + 512 * s));
-                        tc_cp_sf(tsfb + 8 * s + 4, sdesc_sf(sb_s + kSfbStage / 2 + 512 * s));
+                        tc_cp_sf(tsfb + 8 * s + 4, sdesc_sf(sb_s + 512 * kAt + 512 * s));
                     }
                     const uint32_t a_s = smem_u32(st);
                     const uint32_t b_s = a_s + kAStage;
 #pragma unroll
-                    for (int s = 0; s < 4; ++s)
-                        tc_mma(tmem, sdesc_sw128(a_s + 32 * s), sdesc_sw128(b_s + 32 * s), kIdesc,
-                               (kb | s) != 0, tsfa + 4 * s, tsfb + 8 * s);
+                    for (int s = 0; s < 4; ++s) {
+                        uint32_t sfa, sfb, id;
+                        mma_scale_operands<MX>(s, tsfa, tsfb, MX ? (kIdesc | kScaleUE8M0) : kIdesc, sfa, sfb, id);
+                        tc_mma<MX>(tmem, sdesc_sw128(a_s + 32 * s), sdesc_sw128(b_s + 32 * s), id, (kb | s) != 0,
+                                   sfa, sfb);
+                    }
                     issued_any = true;
                     tc_commit(empty_bar(stage));
                     if (++stage == kStages) {
@@ -422,7 +468,7 @@ w4a4_gemm_1sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
         // ---------------------------------------------------- epilogue
         const int q = warp & 3;                      // TMEM lane quarter of this warp
         uint32_t acc_phase = 0;
-        const float scale = __fmul_rn(__ldg(p.ga), __ldg(p.gw));
+        const float scale = p.ga ? __fmul_rn(__ldg(p.ga), __ldg(p.gw)) : 1.0f;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
             bool ok = !*abort_flag && mbar_wait(acc_full, acc_phase, abort_flag);
             ok = __all_sync(0xffffffffu, ok);
@@ -537,14 +583,22 @@ __device__ __forceinline__ void tc2_cp_sf(uint32_t taddr, uint64_t sdesc)
     asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
+template <bool MX>
 __device__ __forceinline__ void tc2_mma(uint32_t tacc, uint64_t da, uint64_t db, uint32_t idesc,
                                         uint32_t accumulate, uint32_t tsfa, uint32_t tsfb)
 {
-    asm volatile("{\n\t.reg .pred p;\n\t"
-                 "setp.ne.b32 p, %4, 0;\n\t"
-                 "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(tacc),
-                 "l"(da), "l"(db), "r"(idesc), "r"(accumulate), "r"(tsfa), "r"(tsfb)
-                 : "memory");
+    if constexpr (MX)
+        asm volatile("{\n\t.reg .pred p;\n\t"
+                     "setp.ne.b32 p, %4, 0;\n\t"
+                     "tcgen05.mma.cta_group::2.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(tacc),
+                     "l"(da), "l"(db), "r"(idesc), "r"(accumulate), "r"(tsfa), "r"(tsfb)
+                     : "memory");
+    else
+        asm volatile("{\n\t.reg .pred p;\n\t"
+                     "setp.ne.b32 p, %4, 0;\n\t"
+                     "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(tacc),
+                     "l"(da), "l"(db), "r"(idesc), "r"(accumulate), "r"(tsfa), "r"(tsfb)
+                     : "memory");
 }
 
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int x, int y)
@@ -571,6 +625,7 @@ __device__ __forceinline__ void stage_row_chunk(uint8_t* stg, int c, int lane, c
     }
 }
 
+template <bool MX>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(k2Threads, 1)
 w4a4_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
@@ -659,15 +714,16 @@ w4a4_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                     // the leader expects both CTAs' bytes of this stage
                     const uint32_t fb = mapa_rank(full_bar(stage), 0);
                     if (leader)
-                        mbar_expect_tx(full_bar(stage), 2 * k2StageBytes);
+                        mbar_expect_tx(full_bar(stage), 2 * (k2AStage + k2BStage + 3 * 512 * SfGeom<MX>::kAtoms));
                     uint8_t* st = smem + stage * k2StageBytes;
                     tma_load_2d_pair(smem_u32(st), (sel & 1) ? &tmA1 : &tmA, kb * (kBK / 2),
                                      mt * 256 + (int)rank * 128, fb);
                     tma_load_2d_pair(smem_u32(st + k2AStage), (sel & 2) ? &tmB1 : &tmB, kb * (kBK / 2),
                                      nt * 256 + (int)rank * 128, fb);
-                    tma_load_3d_pair(smem_u32(st + k2AStage + k2BStage), &tmSA, 0, kb * 4, 2 * mt + (int)rank, fb);
-                    tma_load_3d_pair(smem_u32(st + k2AStage + k2BStage + k2SfaStage), &tmSB, 0, kb * 4, 2 * nt,
-                                     fb);
+                    tma_load_3d_pair(smem_u32(st + k2AStage + k2BStage), &tmSA, 0, kb * SfGeom<MX>::kAtoms,
+                                     2 * mt + (int)rank, fb);
+                    tma_load_3d_pair(smem_u32(st + k2AStage + k2BStage + k2SfaStage), &tmSB, 0,
+                                     kb * SfGeom<MX>::kAtoms, 2 * nt, fb);
                     issued |= 1u << stage;
                     issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
                     if (++stage == k2Stages) {
@@ -721,9 +777,12 @@ w4a4_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                     const uint32_t a_s = smem_u32(st);
                     const uint32_t b_s = a_s + k2AStage;
 #pragma unroll
-                    for (int s = 0; s < 4; ++s)
-                        tc2_mma(tmem, sdesc_sw128(a_s + 32 * s), sdesc_sw128(b_s + 32 * s), k2Idesc,
-                                (kb | s) != 0, tsfa + 4 * s, tsfb + 8 * s);
+                    for (int s = 0; s < 4; ++s) {
+                        uint32_t sfa, sfb, id;
+                        mma_scale_operands<MX>(s, tsfa, tsfb, MX ? (k2Idesc | kScaleUE8M0) : k2Idesc, sfa, sfb, id);
+                        tc2_mma<MX>(tmem, sdesc_sw128(a_s + 32 * s), sdesc_sw128(b_s + 32 * s), id, (kb | s) != 0,
+                                    sfa, sfb);
+                    }
                     issued_any = true;
                     tc2_commit_mc(empty_bar(stage), (uint16_t)0x3);
                     if (++stage == k2Stages) {
@@ -747,8 +806,9 @@ w4a4_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
             // ------------------------------- scale-copy warps (leader), one
             // atom column each: 0 SFA, 1 SFB rows 0-127, 2 SFB rows 128-255
             const int which = warp - 6;
+            constexpr int kAt = SfGeom<MX>::kAtoms;
             const uint32_t sf_off = which == 0 ? 0u : which == 1 ? (uint32_t)k2SfaStage
-                                                                 : (uint32_t)(k2SfaStage + k2SfbStage / 2);
+                                                                 : (uint32_t)(k2SfaStage + 512 * kAt);
             const uint32_t col_off = which == 0 ? 0u : which == 1 ? 16u : 20u;
             const uint32_t col_step = which == 0 ? 4u : 8u;
             int stage = 0;
@@ -766,7 +826,7 @@ w4a4_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                     const uint32_t src = smem_u32(smem + stage * k2StageBytes + k2AStage + k2BStage) + sf_off;
                     const uint32_t dst = tmem + kSfCol0 + (uint32_t)stage * kSfColsPerStage + col_off;
 #pragma unroll
-                    for (int s = 0; s < 4; ++s)
+                    for (int s = 0; s < kAt; ++s)
                         tc2_cp_sf(dst + col_step * (uint32_t)s, sdesc_sf(src + 512 * s));
                     issued_any = true;
                     tc2_commit_mc(sf_ready_bar(stage), (uint16_t)0x1);
@@ -792,7 +852,7 @@ w4a4_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
         uint8_t* stg = epi + q * k2EpiWarpBytes;
         const uint32_t leader_acc_empty = mapa_rank(acc_empty, 0);
         uint32_t acc_phase = 0;
-        const float scale = __fmul_rn(__ldg(p.ga), __ldg(p.gw));
+        const float scale = p.ga ? __fmul_rn(__ldg(p.ga), __ldg(p.gw)) : 1.0f;
         for (int tile = cluster; tile < num_tiles; tile += nclusters) {
             bool ok = !*abort_flag && mbar_wait(acc_full, acc_phase, abort_flag);
             ok = __all_sync(0xffffffffu, ok);
@@ -909,16 +969,17 @@ bool make_code_map(CUtensorMap* m, const void* base, int64_t rows, int64_t kbyte
 
 // 3-D map over MMA-layout scale bytes viewed as [row atom][K atom][128 words]
 // (each 128-row x 4-scale atom is 512 contiguous bytes, K atoms fastest); a
-// box is 4 K atoms of `row_atoms` consecutive row atoms.
-bool make_sf_map(CUtensorMap* m, const void* base, int64_t rows, int64_t K, int row_atoms)
+// box is the K atoms of one 256-wide K stage (4 for NVFP4's 16-element
+// blocks, 2 for MXFP4's 32-element blocks) of `row_atoms` consecutive row atoms.
+bool make_sf_map(CUtensorMap* m, const void* base, int64_t rows, int64_t K, int row_atoms, bool mx)
 {
     auto fn = encode_fn();
     if (!fn)
         return false;
-    const int64_t kb_atoms = K / 64;
+    const int64_t kb_atoms = K / (mx ? 128 : 64);
     cuuint64_t dims[3] = {128u, (cuuint64_t)kb_atoms, (cuuint64_t)(rows / 128)};
     cuuint64_t strides[2] = {512u, (cuuint64_t)kb_atoms * 512u};
-    cuuint32_t box[3] = {128u, 4u, (cuuint32_t)row_atoms};
+    cuuint32_t box[3] = {128u, mx ? 2u : 4u, (cuuint32_t)row_atoms};
     cuuint32_t estr[3] = {1u, 1u, 1u};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<void*>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
@@ -948,10 +1009,58 @@ bool gemm_shape_supported(int64_t M, int64_t N, int64_t K)
            N / kBN < (1 << 20);
 }
 
+template <bool MX>
+cudaError_t launch_gemm_t(const uint8_t* a_codes, const uint8_t* a_sf, const uint8_t* w_codes,
+                          const uint8_t* w_sf, const uint8_t* a1, const uint8_t* w1, int64_t M, int64_t N,
+                          int64_t K, void* out, GemmParams& p, cudaStream_t s)
+{
+    if (M % 256 == 0) {
+        // CTA pairs: 256 x 256 tiles
+        CUtensorMap ta, tb, tsa, tsb, to, ta1, tb1;
+        if (!make_code_map(&ta, a_codes, M, K / 2, 128) || !make_code_map(&tb, w_codes, N, K / 2, 128) ||
+            !make_sf_map(&tsa, a_sf, M, K, 1, MX) || !make_sf_map(&tsb, w_sf, N, K, 2, MX) ||
+            !make_out_map(&to, out, M, N) || !make_code_map(&ta1, a1, M, K / 2, 128) ||
+            !make_code_map(&tb1, w1, N, K / 2, 128))
+            return cudaErrorInvalidValue;
+        static std::once_flag attr2_once;
+        static cudaError_t attr2_err = cudaSuccess;
+        std::call_once(attr2_once, [] {
+            attr2_err = cudaFuncSetAttribute(w4a4_gemm_2sm_kernel<MX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             k2SmemBytes);
+        });
+        if (attr2_err != cudaSuccess)
+            return attr2_err;
+        p.tiles_m = (int)(M / 256);
+        const int tiles = p.tiles_m * p.tiles_n;
+        const int pairs = num_sms() / 2;
+        const int grid = 2 * (tiles < pairs ? tiles : pairs);
+        w4a4_gemm_2sm_kernel<MX><<<grid, k2Threads, k2SmemBytes, s>>>(ta, tb, tsa, tsb, to, ta1, tb1, p);
+        return cudaGetLastError();
+    }
+    CUtensorMap ta, tb, tsa, tsb, ta1, tb1;
+    if (!make_code_map(&ta, a_codes, M, K / 2, kBM) || !make_code_map(&tb, w_codes, N, K / 2, kBN) ||
+        !make_sf_map(&tsa, a_sf, M, K, 1, MX) || !make_sf_map(&tsb, w_sf, N, K, 2, MX) ||
+        !make_code_map(&ta1, a1, M, K / 2, kBM) || !make_code_map(&tb1, w1, N, K / 2, kBN))
+        return cudaErrorInvalidValue;
+    static std::once_flag attr_once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(attr_once, [] {
+        attr_err = cudaFuncSetAttribute(w4a4_gemm_1sm_kernel<MX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        kSmemBytes);
+    });
+    if (attr_err != cudaSuccess)
+        return attr_err;
+    p.tiles_m = (int)(M / kBM);
+    const int tiles = p.tiles_m * p.tiles_n;
+    const int grid = tiles < num_sms() ? tiles : num_sms();
+    w4a4_gemm_1sm_kernel<MX><<<grid, kThreads, kSmemBytes, s>>>(ta, tb, tsa, tsb, ta1, tb1, p);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_w4a4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* ga,
                              const uint8_t* w_codes, const uint8_t* w_sf, const float* gw, int64_t M,
                              int64_t N, int64_t K, void* out, int* err, cudaStream_t s,
-                             const uint8_t* a1_codes, const uint8_t* w1_codes)
+                             const uint8_t* a1_codes, const uint8_t* w1_codes, int mx)
 {
     GemmParams p;
     // passes in K-block order: (A, W), then (A, W1), (A1, W), (A1, W1) as present
@@ -977,52 +1086,14 @@ cudaError_t launch_w4a4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const 
     p.err = err;
     p.tiles_n = (int)(N / kBN);
     p.kblocks = (int)(K / kBK);
-    p.kb_atoms = (int)(K / 64);
+    p.kb_atoms = (int)(K / (mx ? 128 : 64));
     p.N = (int)N;
     p.kiters = p.kblocks << p.pass_shift;
     const uint8_t* a1 = a1_codes ? a1_codes : a_codes;
     const uint8_t* w1 = w1_codes ? w1_codes : w_codes;
-    if (M % 256 == 0) {
-        // CTA pairs: 256 x 256 tiles
-        CUtensorMap ta, tb, tsa, tsb, to, ta1, tb1;
-        if (!make_code_map(&ta, a_codes, M, K / 2, 128) || !make_code_map(&tb, w_codes, N, K / 2, 128) ||
-            !make_sf_map(&tsa, a_sf, M, K, 1) || !make_sf_map(&tsb, w_sf, N, K, 2) ||
-            !make_out_map(&to, out, M, N) || !make_code_map(&ta1, a1, M, K / 2, 128) ||
-            !make_code_map(&tb1, w1, N, K / 2, 128))
-            return cudaErrorInvalidValue;
-        static std::once_flag attr2_once;
-        static cudaError_t attr2_err = cudaSuccess;
-        std::call_once(attr2_once, [] {
-            attr2_err = cudaFuncSetAttribute(w4a4_gemm_2sm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             k2SmemBytes);
-        });
-        if (attr2_err != cudaSuccess)
-            return attr2_err;
-        p.tiles_m = (int)(M / 256);
-        const int tiles = p.tiles_m * p.tiles_n;
-        const int pairs = num_sms() / 2;
-        const int grid = 2 * (tiles < pairs ? tiles : pairs);
-        w4a4_gemm_2sm_kernel<<<grid, k2Threads, k2SmemBytes, s>>>(ta, tb, tsa, tsb, to, ta1, tb1, p);
-        return cudaGetLastError();
-    }
-    CUtensorMap ta, tb, tsa, tsb, ta1, tb1;
-    if (!make_code_map(&ta, a_codes, M, K / 2, kBM) || !make_code_map(&tb, w_codes, N, K / 2, kBN) ||
-        !make_sf_map(&tsa, a_sf, M, K, 1) || !make_sf_map(&tsb, w_sf, N, K, 2) ||
-        !make_code_map(&ta1, a1, M, K / 2, kBM) || !make_code_map(&tb1, w1, N, K / 2, kBN))
-        return cudaErrorInvalidValue;
-    static std::once_flag attr_once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(w4a4_gemm_1sm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        kSmemBytes);
-    });
-    if (attr_err != cudaSuccess)
-        return attr_err;
-    p.tiles_m = (int)(M / kBM);
-    const int tiles = p.tiles_m * p.tiles_n;
-    const int grid = tiles < num_sms() ? tiles : num_sms();
-    w4a4_gemm_1sm_kernel<<<grid, kThreads, kSmemBytes, s>>>(ta, tb, tsa, tsb, ta1, tb1, p);
-    return cudaGetLastError();
+    if (mx)
+        return launch_gemm_t<true>(a_codes, a_sf, w_codes, w_sf, a1, w1, M, N, K, out, p, s);
+    return launch_gemm_t<false>(a_codes, a_sf, w_codes, w_sf, a1, w1, M, N, K, out, p, s);
 }
 
 }  // namespace fp4q

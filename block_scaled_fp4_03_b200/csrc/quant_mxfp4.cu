@@ -125,7 +125,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 mx_quant_absmax_kernel(const T* __restrict__ x, uint32_t nblk, uint32_t kb,
                        const float* __restrict__ t, int had, uint8_t* __restrict__ codes,
                        uint8_t* __restrict__ scales, float* __restrict__ deq,
-                       float* __restrict__ mse)
+                       float* __restrict__ mse, int mma)
 {
     constexpr int CPB = 32 * (int)sizeof(T) / 16;   // 16-byte chunks per block
     // one 4 KB buffer per warp: first the warp's blocks, then their t slices
@@ -224,7 +224,9 @@ mx_quant_absmax_kernel(const T* __restrict__ x, uint32_t nblk, uint32_t kb,
         }
         if ((uint32_t)lane < nb) {
             *reinterpret_cast<uint4*>(codes + b * 16) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-            scales[b] = (uint8_t)(e + 127);
+            const uint64_t r = b / kb;
+            scales[mma ? mma_sf_offset((int64_t)r, (int64_t)(b - r * kb), kb >> 2) : (int64_t)b] =
+                (uint8_t)(e + 127);
         }
     }
 }
@@ -263,7 +265,7 @@ __global__ void __launch_bounds__(kHessThreads, 3)
 mx_quant_hessian_kernel(const T* __restrict__ x, int64_t rows, int64_t kb,
                         const float* __restrict__ t, int had, const float* __restrict__ hess,
                         uint8_t* __restrict__ codes, uint8_t* __restrict__ scales,
-                        float* __restrict__ deq, float* __restrict__ mse)
+                        float* __restrict__ deq, float* __restrict__ mse, int mma)
 {
     __shared__ __align__(16) float Hs[32 * 32];   // H'_k, row-major
     const int64_t k = blockIdx.y;
@@ -329,7 +331,7 @@ mx_quant_hessian_kernel(const T* __restrict__ x, int64_t rows, int64_t kb,
     float dq[32];
     const float sse = mx_eval(u, best_e, cw, dq);
     *reinterpret_cast<uint4*>(codes + b * 16) = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-    scales[b] = (uint8_t)(best_e + 127);
+    scales[mma ? mma_sf_offset(r, k, kb >> 2) : b] = (uint8_t)(best_e + 127);
     if (deq)
         store_f32<32>(deq + b * 32, dq);
     if (mse)
@@ -576,7 +578,7 @@ size_t channel_scale_ws_bytes(int64_t tokens, int64_t n_out, int64_t cols)
 cudaError_t launch_mxfp4_quant(const void* x, int dtype, int64_t rows, int64_t cols,
                                const float* chan_scale, int hadamard, int rule, const float* hess,
                                uint8_t* codes, uint8_t* scales, float* deq, float* mse,
-                               cudaStream_t s)
+                               cudaStream_t s, int mma_layout)
 {
     const int64_t kb = cols / 32;
     const int64_t nblk = rows * kb;
@@ -585,11 +587,11 @@ cudaError_t launch_mxfp4_quant(const void* x, int dtype, int64_t rows, int64_t c
         if (dtype == 1)
             mx_quant_hessian_kernel<__nv_bfloat16><<<grid, kHessThreads, 0, s>>>(
                 reinterpret_cast<const __nv_bfloat16*>(x), rows, kb, chan_scale, hadamard, hess,
-                codes, scales, deq, mse);
+                codes, scales, deq, mse, mma_layout);
         else
             mx_quant_hessian_kernel<float><<<grid, kHessThreads, 0, s>>>(
                 reinterpret_cast<const float*>(x), rows, kb, chan_scale, hadamard, hess, codes,
-                scales, deq, mse);
+                scales, deq, mse, mma_layout);
         return cudaGetLastError();
     }
     if (nblk > (int64_t)0xFFFFFFFFu)
@@ -599,12 +601,13 @@ cudaError_t launch_mxfp4_quant(const void* x, int dtype, int64_t rows, int64_t c
         auto k = err ? mx_quant_absmax_kernel<__nv_bfloat16, true> : mx_quant_absmax_kernel<__nv_bfloat16, false>;
         k<<<grid_for(nblk, (const void*)k), kThreads, 0, s>>>(
             reinterpret_cast<const __nv_bfloat16*>(x), (uint32_t)nblk, (uint32_t)kb, chan_scale, hadamard,
-            codes, scales, deq, mse);
+            codes, scales, deq, mse, mma_layout);
     } else {
         auto k = err ? mx_quant_absmax_kernel<float, true> : mx_quant_absmax_kernel<float, false>;
         k<<<grid_for(nblk, (const void*)k), kThreads, 0, s>>>(reinterpret_cast<const float*>(x),
                                                                (uint32_t)nblk, (uint32_t)kb, chan_scale,
-                                                               hadamard, codes, scales, deq, mse);
+                                                               hadamard, codes, scales, deq, mse,
+                                                               mma_layout);
     }
     return cudaGetLastError();
 }

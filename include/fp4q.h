@@ -71,7 +71,7 @@ typedef enum {
     FP4Q_ERR_TOO_LARGE = 7     /* the problem needs more than the library's built-in scratch */
 } fp4q_status;
 
-typedef enum { FP4Q_F32 = 0, FP4Q_BF16 = 1, FP4Q_NVFP4_PACKED = 2 } fp4q_dtype;
+typedef enum { FP4Q_F32 = 0, FP4Q_BF16 = 1, FP4Q_NVFP4_PACKED = 2, FP4Q_MXFP4_PACKED = 3 } fp4q_dtype;
 
 /* Block-scale formats: E4M3 = OCP FP8 E4M3FN (NVFP4 and RaZeR activations),
  * E3M3 = 6-bit unsigned, bias 3, 2^-5..30 (RaZeR weights, [RaZeR] 2.1),
@@ -117,7 +117,8 @@ typedef enum {
     FP4Q_OP_HESSIAN = 1,        /* fp4_hessian_blocks (rows, cols) */
     FP4Q_OP_CHANNEL_SCALE = 2,  /* mxfp4_channel_scale (tokens=rows, cols, n_out=n) */
     FP4Q_OP_GEMM = 3,           /* w4a4_gemm with bf16 A (M=rows, K=cols, N=n) */
-    FP4Q_OP_FLIP = 4            /* mxfp4_flip_refine (rows, cols) */
+    FP4Q_OP_FLIP = 4,           /* mxfp4_flip_refine (rows, cols) */
+    FP4Q_OP_MX_GEMM = 5         /* mxfp4_gemm with bf16/fp32 A (M=rows, K=cols) */
 } fp4q_op;
 
 /* Bytes of device workspace an entry point needs (0 if none). */
@@ -376,6 +377,46 @@ FP4Q_API int razer_w4a4_gemm(const uint8_t* a_codes, const uint8_t* a_extra, con
                              const uint8_t* w_extra, const uint8_t* w_scales,
                              const float* w_global_scale, int64_t M, int64_t N, int64_t K, void* out,
                              void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Scale bytes from the row-major layout [rows][nscales] to FP4Q_SFLAYOUT_MMA
+ * (the tcgen05 scale layout; works for E4M3 scales per 16 and E8M0 scales per
+ * 32 alike), e.g. for MXFP4 weights quantized row-major and refined by
+ * mxfp4_flip_refine.  rows % 128 == 0, nscales % 4 == 0; both pointers device,
+ * 16-byte aligned, rows*nscales bytes.  Errors: ERR_ARG, ERR_ALIGN, ERR_CUDA.
+ */
+FP4Q_API int fp4_scales_to_mma(const uint8_t* scales, int64_t rows, int64_t nscales, uint8_t* out,
+                               void* stream);
+
+/*
+ * MXFP4 W4A4 GEMM ([MACaQ] 1: W4A4 inference with MXFP4 operands, E2M1 values
+ * and one E8M0 exponent per 32 elements, the activations rotated online):
+ *
+ *   out[m][n] = bf16( sum_k (v_a 2^(ea - 127))[m][k] * (v_w 2^(ew - 127))[n][k] ),
+ *
+ * on tcgen05 tensor cores (kind::mxf4, block 32).  With the online transform
+ * X' = (X * t) B (t per channel, B the normalised 32-block Hadamard) and the
+ * weights prepared as W' = (W / t) B (mxfp4_quantize with 1/t), out
+ * approximates X W^T.
+ *
+ *  a, a_format  FP4Q_F32 / FP4Q_BF16: A is a dense M x K tensor; the prologue
+ *               (a * chan_scale, the 32-block rotation if hadamard32, OCP E8M0
+ *               exponent, E2M1 codes) runs here into the workspace, scales
+ *               written in the GEMM's layout; FP4Q_MXFP4_PACKED: a = codes
+ *               (M*K/2 bytes), a_scales = E8M0 bytes in FP4Q_SFLAYOUT_MMA
+ *               (chan_scale must be NULL)
+ *  chan_scale   device fp32 [K] (nullable): t for the dense A
+ *  w_codes      device N*K/2 bytes; w_scales E8M0 bytes in FP4Q_SFLAYOUT_MMA
+ *               (mxfp4_quantize + fp4_scales_to_mma)
+ *  M % 128 == 0, N % 256 == 0, K % 256 == 0 (FP4Q_ERR_UNSUPPORTED otherwise)
+ *  workspace    >= fp4q_workspace_size(FP4Q_OP_MX_GEMM, M, K, N) for dense A,
+ *               8 KiB for packed A; 16-byte aligned; holds the error word read
+ *               by fp4q_gemm_status
+ */
+FP4Q_API int mxfp4_gemm(const void* a, int a_format, const uint8_t* a_scales, const float* chan_scale,
+                        int hadamard32, const uint8_t* w_codes, const uint8_t* w_scales, int64_t M,
+                        int64_t N, int64_t K, void* out, void* workspace, size_t workspace_bytes,
+                        void* stream);
 
 /*
  * Synchronizes `stream` and reports whether the last w4a4_gemm that used this

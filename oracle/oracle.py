@@ -373,6 +373,19 @@ def razer_decode_exact(codes, meta, sf: int, specials):
     return v * np.repeat(sc, 16, axis=1)
 
 
+def mx_decode_exact(codes, scales):
+    """MXFP4 values in fp64 (exact), "MACaQ" review section 1: each E2M1 code
+    times 2^(byte - 127) of its 32-element block."""
+    codes = np.asarray(codes, np.uint8)
+    rows, cols = codes.shape[0], codes.shape[1] * 2
+    e2 = np.array([e2m1_value(c) for c in range(16)], np.float64)
+    v = np.empty((rows, cols), np.float64)
+    v[:, 0::2] = e2[codes & 0xF]
+    v[:, 1::2] = e2[codes >> 4]
+    p2 = np.ldexp(1.0, np.asarray(scales, np.int64) - 127)
+    return v * np.repeat(p2, 32, axis=1)
+
+
 def gemm_values(da, dw, g_a, g_w):
     """out = g_a * g_w * (da @ dw^T) in fp64 for exactly decoded operands."""
     return (float(g_a) * float(g_w)) * (np.asarray(da, np.float64) @ np.asarray(dw, np.float64).T)

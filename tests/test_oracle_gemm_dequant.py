@@ -128,3 +128,27 @@ def test_razer_gemm_reference_matches_triple_loop(O):
             assert abs(ref[m, n] - float(ga) * float(gw) * acc) <= 1e-12 * max(1.0, abs(ref[m, n]))
     exact = a.astype(np.float64) @ w.astype(np.float64).T
     assert np.linalg.norm(ref - exact) <= 0.2 * np.linalg.norm(exact)
+
+
+def test_mx_decode_exact_matches_dequantizer(O):
+    """v * 2^e is exact in fp32 here, so the fp64 decode equals the C
+    dequantizer's E8M0 output; and the MX product of the transformed operands
+    approximates X W^T (the rotation and 1/t cancel)."""
+    x = _x("mx_act", 64, 256, seed=5)
+    w = _x("mx_weight", 48, 256, seed=6)
+    t = inputs.positive_vector(256, seed=7)
+    qa = O.mxfp4_quantize(x, t, True, O.RULE_ABSMAX)
+    d = O.mx_decode_exact(qa["codes"], qa["scales"])
+    deq = O.dequant_mse(qa["codes"], qa["scales"], 64, 256, 32, O.SF_E8M0, None)["deq"]
+    assert np.array_equal(d, deq.astype(np.float64))
+    tinv = (1.0 / t.astype(np.float64)).astype(np.float32)
+    qw = O.mxfp4_quantize(w, tinv, True, O.RULE_ABSMAX)
+    ref = O.gemm_values(d, O.mx_decode_exact(qw["codes"], qw["scales"]), 1.0, 1.0)
+    exact = x.astype(np.float64) @ w.astype(np.float64).T
+    e_ref = np.linalg.norm(ref - exact) / np.linalg.norm(exact)
+    # without the matching 1/t on the weights the product is far off (t spans
+    # [1/4, 4], which also makes 4-bit blocks coarse: e_ref is about 0.46)
+    qw_bad = O.mxfp4_quantize(w, None, True, O.RULE_ABSMAX)
+    bad = O.gemm_values(d, O.mx_decode_exact(qw_bad["codes"], qw_bad["scales"]), 1.0, 1.0)
+    e_bad = np.linalg.norm(bad - exact) / np.linalg.norm(exact)
+    assert e_ref <= 0.6 and e_bad >= 2 * e_ref, (e_ref, e_bad)
