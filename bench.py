@@ -461,6 +461,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-next-rows", action="store_true",
+                    help="time the hot-path step only (skip the rows built on top of it)")
     ap.add_argument("--profile-row", default=None,
                     help="for profiler captures: build only this row's workload group, run the group once, "
                          "then the row --reps times; prints no JSON")
@@ -508,7 +510,9 @@ def main():
     stream = torch.cuda.current_stream()
 
     hot = [r for r in rows if not r.extra]
-    extra = [r for r in rows if r.extra]
+    extra = [] if args.no_next_rows else [r for r in rows if r.extra]
+    if args.no_next_rows:
+        rows = hot
 
     def run_rows(rs, times=None):
         for r in rs:
