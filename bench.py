@@ -105,6 +105,8 @@ class Row:
         # rows beyond the hot path proper (the next rows built on it): timed
         # and reported per row, outside the step and its value
         self.extra = extra
+        # the step's input tensors (keys of X) this row reads; set per workload
+        self.inputs = []
 
 
 def build_rows(torch, fq, inputs, dev, host_copies=None, groups=None):
@@ -120,6 +122,11 @@ def build_rows(torch, fq, inputs, dev, host_copies=None, groups=None):
 
     rows = []
     X = {}
+
+    def tag(start, keys):
+        for r in rows[start:]:
+            r.inputs = list(keys)
+    n0 = len(rows)
     if groups is None or "c1" in groups:
         # c1
         a1 = inputs.generate("gaussian")
@@ -132,6 +139,8 @@ def build_rows(torch, fq, inputs, dev, host_copies=None, groups=None):
             o1.update(fq.nvfp4_quantize(X["c1"], 16, fq.PREVENT_ZERO, gs_mode=fq.GS_AMAX, dequant=True,
                                         mse=True, out=o1, workspace=ws1))
         rows.append(Row("c1_nvfp4_pz_deq_mse", "nvfp4_quant_kernel<16, float, 1, 0>", n1, n1 * (4 + 0.5 + 1 / 16 + 4 + 4 / 16), 2, c1, o1))
+    tag(n0, [k for k in ("c1",) if k in X])
+    n0 = len(rows)
     if groups is None or "c2" in groups:
         # c2
         a2 = inputs.generate("student_t")
@@ -165,6 +174,8 @@ def build_rows(torch, fq, inputs, dev, host_copies=None, groups=None):
                 rows.append(Row("c2_B%d_%s" % (B, tag),
                                 "nvfp4_quant_kernel<%d, float, %d, %d>" % (B, rule, 1 if sfmt == fq.SF_UE5M3 else 0),
                                 n2, n2 * (4 + 0.5 + 1 / B + 4 / B), 2 if gsm == fq.GS_AMAX else 1, c2x, o, extra=True))
+    tag(n0, [k for k in ("c2",) if k in X])
+    n0 = len(rows)
     if groups is None or "c3" in groups:
         # c3
         w3 = inputs.generate("razer_weight")
@@ -181,6 +192,9 @@ def build_rows(torch, fq, inputs, dev, host_copies=None, groups=None):
             o3a.update(fq.razer_quantize(X["c3a"], fq.SF_E4M3, [5.0, -5.0], gs_mode=fq.GS_AMAX, out=o3a, workspace=ws3))
         rows.append(Row("c3_razer_weight", "razer_paired_kernel<__nv_bfloat16, 1, 2>", w3.size, w3.size * (2 + 0.5 + 1 / 16), 2, c3w, o3w))
         rows.append(Row("c3_razer_act", "razer_paired_kernel<__nv_bfloat16, 0, 1>", a3.size, a3.size * (2 + 0.5 + 1 / 16), 2, c3a, o3a))
+    for r in rows[n0:]:
+        r.inputs = ["c3w"] if "weight" in r.name else ["c3a"]
+    n0 = len(rows)
     if groups is None or "c4" in groups:
         # c4
         x4 = inputs.generate("mx_act")
@@ -252,6 +266,8 @@ def build_rows(torch, fq, inputs, dev, host_copies=None, groups=None):
         rows.append(Row("f3_mx_gemm_with_prologue", "mx_quant_absmax_kernel + w4a4_gemm_2sm_kernel<true>", 0,
                         mxg_bytes + T * C * 2, 2, f3d, {"out": y3}, bound="tensor", flops=2.0 * T * N3 * C,
                         extra=True))
+    tag(n0, [k for k in ("c4x", "c4w") if k in X])
+    n0 = len(rows)
     if groups is None or "c5" in groups:
         # c5: weights pre-quantized once (abs-max NVFP4, hierarchical scale, MMA
         # scale layout) outside the timed step; the step quantizes the activations
@@ -319,6 +335,7 @@ def build_rows(torch, fq, inputs, dev, host_copies=None, groups=None):
         rows.append(Row("f2_razer_gemm_wa_4pass", "w4a4_gemm_2sm_kernel<false>", 0,
                         M5 * K5 * (1.0 + 1 / 16) + N5 * K5 * (1.0 + 1 / 16) + M5 * N5 * 2, 1, f2wa, {"out": y5},
                         bound="tensor", flops=2.0 * M5 * N5 * K5, extra=True))
+    tag(n0, [k for k in ("c5",) if k in X])
     return rows, X
 
 
@@ -676,36 +693,77 @@ def main():
 
 def run_e2e(torch, rows, X, host, stream, args, barrier, world, dist, dev):
     """Same step through the public API with host buffers: pinned host -> device
-    copies of every input, the step, and device -> host copies of every output."""
+    copies of every input, the step, and device -> host copies of every output.
+    The copies run on two copy streams, overlapped with the rows' compute: a row
+    starts once its inputs have landed, its outputs go back as soon as it is
+    done, and the next step's copies wait only for the buffers they overwrite."""
     pinned = {k: torch.from_numpy(v.view(np.int16) if v.dtype == np.uint16 else v).pin_memory() for k, v in host.items()}
     h2d = sum(p.numel() * p.element_size() for p in pinned.values())
 
-    outs_dev = []
+    outs_of = []          # per row: the output tensors it is the first to list
+    seen = []
     for r in rows:
+        mine = []
         for t in r.out.values():
-            if torch.is_tensor(t) and all(t.data_ptr() != u.data_ptr() for u in outs_dev):
-                outs_dev.append(t)
-    outs_host = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs_dev]
-    d2h = sum(t.numel() * t.element_size() for t in outs_dev)
+            if torch.is_tensor(t) and all(t.data_ptr() != u.data_ptr() for u in seen):
+                seen.append(t)
+                mine.append(t)
+        outs_of.append(mine)
+    host_of = {t.data_ptr(): torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in seen}
+    d2h = sum(t.numel() * t.element_size() for t in seen)
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    last_use = {}         # input key -> event after the last row that read it
+    out_done = {}         # output pointer -> event after its copy back
+    order = []
+    for r in rows:
+        for k in r.inputs:
+            if k not in order:
+                order.append(k)
+    order += [k for k in pinned if k not in order]
 
     def one():
-        for k, p in pinned.items():
-            dst = X[k]
-            dst.view(torch.int16 if dst.dtype == torch.bfloat16 else dst.dtype).copy_(p, non_blocking=True)
-        for r in rows:
+        ev_in = {}
+        for k in order:
+            if k in last_use:
+                s_in.wait_event(last_use[k])
+            with torch.cuda.stream(s_in):
+                dst = X[k]
+                dst.view(torch.int16 if dst.dtype == torch.bfloat16 else dst.dtype).copy_(pinned[k], non_blocking=True)
+                ev_in[k] = torch.cuda.Event()
+                ev_in[k].record(s_in)
+        for r, mine in zip(rows, outs_of):
+            for k in r.inputs:
+                stream.wait_event(ev_in[k])
+            for t in mine:
+                if t.data_ptr() in out_done:
+                    stream.wait_event(out_done[t.data_ptr()])
             r.fn()
-        for d, h in zip(outs_dev, outs_host):
-            h.copy_(d, non_blocking=True)
+            ev = torch.cuda.Event()
+            ev.record(stream)
+            for k in r.inputs:
+                last_use[k] = ev
+            if mine:
+                s_out.wait_event(ev)
+                with torch.cuda.stream(s_out):
+                    for t in mine:
+                        host_of[t.data_ptr()].copy_(t, non_blocking=True)
+                    done = torch.cuda.Event()
+                    done.record(s_out)
+                for t in mine:
+                    out_done[t.data_ptr()] = done
 
     for _ in range(2):
         one()
     barrier()
     e0, e1 = torch.cuda.Event(True), torch.cuda.Event(True)
-    e0.record(stream)
+    e0.record(s_in)
     n = max(1, min(args.steps, 3))
     for _ in range(n):
         one()
-    e1.record(stream)
+    # the last copy back is the end of the step's work
+    s_out.wait_event(_record(torch, stream))
+    s_out.wait_event(_record(torch, s_in))
+    e1.record(s_out)
     barrier()
     ms = e0.elapsed_time(e1) / n
     if dist is not None:
@@ -714,7 +772,14 @@ def run_e2e(torch, rows, X, host, stream, args, barrier, world, dist, dev):
         ms = float(t.item())
     units = sum(r.units for r in rows)
     return {"value": units * world / (ms * 1e-3) / 1e9, "unit": "Gelem/s", "h2d_bytes_per_step": h2d,
-            "d2h_bytes_per_step": d2h, "ms_per_step": ms}
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms,
+            "overlap": "inputs in and outputs back on two copy streams, overlapped with the rows' compute"}
+
+
+def _record(torch, s):
+    ev = torch.cuda.Event()
+    ev.record(s)
+    return ev
 
 
 if __name__ == "__main__":

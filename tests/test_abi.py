@@ -120,3 +120,39 @@ def test_mx_and_dequant_argument_errors(L):
     assert L.mxfp4_flip_refine(FAKE, 0, 4, 64, None, 1, FAKE, 8, FAKE, FAKE, None, FAKE, need - 1, None) == 6
     assert L.mxfp4_flip_refine(FAKE, 0, 4, 64, None, 1, FAKE, 8, FAKE, FAKE, None, None, 0, None) == 6
     assert L.mxfp4_flip_refine(None, 0, 0, 64, None, 1, None, 8, None, None, None, None, 0, None) == 0
+
+
+def test_gemm_family_argument_errors(L):
+    """RaZeR split, RaZeR / MXFP4 GEMMs and the scale relayout reject bad calls on the host."""
+    def table(*v):
+        arr = (ctypes.c_float * len(v))(*v)
+        return ctypes.cast(arr, ctypes.c_void_p), arr
+    sp, keep = table(5.0, -5.0, 3.5, -3.5)
+    bad, keep2 = table(11.0)
+    # razer_gemm_prepare: shapes, format, table, alignment, empty
+    assert L.razer_gemm_prepare(FAKE, FAKE, 120, 64, 1, sp, 4, FAKE, FAKE, FAKE, None) == 1
+    assert L.razer_gemm_prepare(FAKE, FAKE, 128, 96, 1, sp, 4, FAKE, FAKE, FAKE, None) == 1
+    assert L.razer_gemm_prepare(FAKE, FAKE, 128, 64, 0, sp, 4, FAKE, FAKE, FAKE, None) == 1
+    assert L.razer_gemm_prepare(FAKE, FAKE, 128, 64, 1, bad, 1, FAKE, FAKE, FAKE, None) == 3
+    assert L.razer_gemm_prepare(MIS, FAKE, 128, 64, 1, sp, 4, FAKE, FAKE, FAKE, None) == 2
+    assert L.razer_gemm_prepare(None, None, 0, 64, 1, sp, 4, None, None, None, None) == 0
+    # razer_w4a4_gemm: missing operands, shapes, alignment, workspace
+    assert L.razer_w4a4_gemm(None, None, FAKE, FAKE, FAKE, None, FAKE, FAKE, 128, 256, 256, FAKE, FAKE, 8192, None) == 1
+    assert L.razer_w4a4_gemm(FAKE, None, FAKE, FAKE, FAKE, None, FAKE, FAKE, 100, 256, 256, FAKE, FAKE, 8192, None) == 3
+    assert L.razer_w4a4_gemm(FAKE, MIS, FAKE, FAKE, FAKE, None, FAKE, FAKE, 128, 256, 256, FAKE, FAKE, 8192, None) == 2
+    assert L.razer_w4a4_gemm(FAKE, None, FAKE, FAKE, FAKE, None, FAKE, FAKE, 128, 256, 256, FAKE, FAKE, 100, None) == 6
+    # mxfp4_gemm: format, packed A without scales or with a channel scale, shapes, workspace
+    assert L.mxfp4_gemm(FAKE, 2, FAKE, None, 1, FAKE, FAKE, 128, 256, 256, FAKE, FAKE, 1 << 20, None) == 1
+    assert L.mxfp4_gemm(FAKE, 3, None, None, 1, FAKE, FAKE, 128, 256, 256, FAKE, FAKE, 1 << 20, None) == 1
+    assert L.mxfp4_gemm(FAKE, 3, FAKE, FAKE, 1, FAKE, FAKE, 128, 256, 256, FAKE, FAKE, 1 << 20, None) == 1
+    assert L.mxfp4_gemm(FAKE, 1, None, None, 1, FAKE, FAKE, 128, 256, 100, FAKE, FAKE, 1 << 20, None) == 3
+    assert L.mxfp4_gemm(FAKE, 1, None, None, 1, FAKE, FAKE, 0, 256, 256, FAKE, FAKE, 1 << 20, None) == 1
+    need = L.fp4q_workspace_size(5, 128, 256, 256)
+    assert need == 8192 + 128 * 256 // 2 + 128 * 256 // 32
+    assert L.mxfp4_gemm(FAKE, 1, None, None, 1, FAKE, FAKE, 128, 256, 256, FAKE, FAKE, need - 1, None) == 6
+    assert L.mxfp4_gemm(FAKE, 3, FAKE, None, 1, FAKE, FAKE, 128, 256, 256, FAKE, FAKE, 8191, None) == 6
+    # fp4_scales_to_mma
+    assert L.fp4_scales_to_mma(FAKE, 100, 8, FAKE, None) == 1
+    assert L.fp4_scales_to_mma(FAKE, 128, 6, FAKE, None) == 1
+    assert L.fp4_scales_to_mma(MIS, 128, 8, FAKE, None) == 2
+    assert L.fp4_scales_to_mma(None, 0, 8, None, None) == 0
