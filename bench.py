@@ -123,7 +123,7 @@ def build_rows(torch, fq, inputs, dev, host_copies=None, groups=None):
     rows = []
     X = {}
 
-    def tag(start, keys):
+    def set_inputs(start, keys):
         for r in rows[start:]:
             r.inputs = list(keys)
     n0 = len(rows)
@@ -139,7 +139,7 @@ def build_rows(torch, fq, inputs, dev, host_copies=None, groups=None):
             o1.update(fq.nvfp4_quantize(X["c1"], 16, fq.PREVENT_ZERO, gs_mode=fq.GS_AMAX, dequant=True,
                                         mse=True, out=o1, workspace=ws1))
         rows.append(Row("c1_nvfp4_pz_deq_mse", "nvfp4_quant_kernel<16, float, 1, 0>", n1, n1 * (4 + 0.5 + 1 / 16 + 4 + 4 / 16), 2, c1, o1))
-    tag(n0, [k for k in ("c1",) if k in X])
+    set_inputs(n0, [k for k in ("c1",) if k in X])
     n0 = len(rows)
     if groups is None or "c2" in groups:
         # c2
@@ -174,7 +174,7 @@ def build_rows(torch, fq, inputs, dev, host_copies=None, groups=None):
                 rows.append(Row("c2_B%d_%s" % (B, tag),
                                 "nvfp4_quant_kernel<%d, float, %d, %d>" % (B, rule, 1 if sfmt == fq.SF_UE5M3 else 0),
                                 n2, n2 * (4 + 0.5 + 1 / B + 4 / B), 2 if gsm == fq.GS_AMAX else 1, c2x, o, extra=True))
-    tag(n0, [k for k in ("c2",) if k in X])
+    set_inputs(n0, [k for k in ("c2",) if k in X])
     n0 = len(rows)
     if groups is None or "c3" in groups:
         # c3
@@ -266,7 +266,7 @@ def build_rows(torch, fq, inputs, dev, host_copies=None, groups=None):
         rows.append(Row("f3_mx_gemm_with_prologue", "mx_quant_absmax_kernel + w4a4_gemm_2sm_kernel<true>", 0,
                         mxg_bytes + T * C * 2, 2, f3d, {"out": y3}, bound="tensor", flops=2.0 * T * N3 * C,
                         extra=True))
-    tag(n0, [k for k in ("c4x", "c4w") if k in X])
+    set_inputs(n0, [k for k in ("c4x", "c4w") if k in X])
     n0 = len(rows)
     if groups is None or "c5" in groups:
         # c5: weights pre-quantized once (abs-max NVFP4, hierarchical scale, MMA
@@ -335,7 +335,7 @@ def build_rows(torch, fq, inputs, dev, host_copies=None, groups=None):
         rows.append(Row("f2_razer_gemm_wa_4pass", "w4a4_gemm_2sm_kernel<false>", 0,
                         M5 * K5 * (1.0 + 1 / 16) + N5 * K5 * (1.0 + 1 / 16) + M5 * N5 * 2, 1, f2wa, {"out": y5},
                         bound="tensor", flops=2.0 * M5 * N5 * K5, extra=True))
-    tag(n0, [k for k in ("c5",) if k in X])
+    set_inputs(n0, [k for k in ("c5",) if k in X])
     return rows, X
 
 

@@ -340,10 +340,15 @@ mx_quant_hessian_kernel(const T* __restrict__ x, int64_t rows, int64_t kb,
 
 // ------------------------------------------------------- Hessian blocks
 // Partial H'_k over a chunk of kTok tokens: the chunk's transformed rows are
-// staged in shared memory, then each thread accumulates 4 of the 1024
-// entries over the chunk.  Partials go to ws[chunk][k][32][32] and are summed
-// in chunk order by hessian_reduce_kernel.
+// staged in shared memory, then each thread accumulates one 4x4 tile of the
+// upper triangle of H'_k (36 tiles, the diagonal ones included) over every
+// 7th token of the chunk; the lower triangle is written as the transpose
+// (H'_k is symmetric, and x_i * x_j rounds exactly as x_j * x_i).  The seven
+// token groups are summed in a fixed order.  Partials go to
+// ws[chunk][k][32][32] and are summed in chunk order by hessian_reduce_kernel.
 constexpr int kTok = 256;
+constexpr int kHessTiles = 36;                  // 4x4 tiles with ti <= tj
+constexpr int kHessGroups = kThreads / kHessTiles;   // 7 token groups
 
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
@@ -351,7 +356,7 @@ hessian_partial_kernel(const T* __restrict__ x, int64_t rows, int64_t cols,
                        const float* __restrict__ t, int had, float* __restrict__ part)
 {
     __shared__ __align__(16) float Xs[kTok][32];
-    __shared__ __align__(16) float red[3][64][16];
+    __shared__ __align__(16) float red[kHessGroups - 1][kHessTiles][16];
     const int64_t k = blockIdx.y;
     const int64_t chunk = blockIdx.x;
     const int64_t r0 = chunk * kTok;
@@ -372,10 +377,15 @@ hessian_partial_kernel(const T* __restrict__ x, int64_t rows, int64_t cols,
             *reinterpret_cast<float4*>(&Xs[rr][i]) = make_float4(u[i], u[i + 1], u[i + 2], u[i + 3]);
     }
     __syncthreads();
-    // thread -> 4x4 entries (4 ti + [0,4), 4 tj + [0,4)) over tokens tg, tg+4, ...
-    const int tg = threadIdx.x >> 6;
-    const int ti = (threadIdx.x >> 3) & 7;
-    const int tj = threadIdx.x & 7;
+    const int tile = threadIdx.x % kHessTiles;
+    const int g = threadIdx.x / kHessTiles;       // token group; kHessGroups is idle
+    // tile -> (ti, tj), ti <= tj, row by row of the upper triangle
+    int ti = 0, tj = tile;
+    while (tj >= 8 - ti) {
+        tj -= 8 - ti;
+        ++ti;
+    }
+    tj += ti;
     float acc[4][4];
 #pragma unroll
     for (int a = 0; a < 4; ++a)
@@ -383,40 +393,49 @@ hessian_partial_kernel(const T* __restrict__ x, int64_t rows, int64_t cols,
         for (int c = 0; c < 4; ++c)
             acc[a][c] = 0.0f;
     const int nr = (int)((rows - r0) < kTok ? (rows - r0) : kTok);
-    for (int rr = tg; rr < nr; rr += 4) {
-        const float4 xi = *reinterpret_cast<const float4*>(&Xs[rr][4 * ti]);
-        const float4 xj = *reinterpret_cast<const float4*>(&Xs[rr][4 * tj]);
-        const float vi[4] = {xi.x, xi.y, xi.z, xi.w};
-        const float vj[4] = {xj.x, xj.y, xj.z, xj.w};
+    if (g < kHessGroups) {
+        for (int rr = g; rr < nr; rr += kHessGroups) {
+            const float4 xi = *reinterpret_cast<const float4*>(&Xs[rr][4 * ti]);
+            const float4 xj = *reinterpret_cast<const float4*>(&Xs[rr][4 * tj]);
+            const float vi[4] = {xi.x, xi.y, xi.z, xi.w};
+            const float vj[4] = {xj.x, xj.y, xj.z, xj.w};
 #pragma unroll
-        for (int a = 0; a < 4; ++a)
+            for (int a = 0; a < 4; ++a)
 #pragma unroll
-            for (int c = 0; c < 4; ++c)
-                acc[a][c] = __fmaf_rn(vi[a], vj[c], acc[a][c]);
+                for (int c = 0; c < 4; ++c)
+                    acc[a][c] = __fmaf_rn(vi[a], vj[c], acc[a][c]);
+        }
     }
-    // sum the four token groups in a fixed order
-    if (tg > 0) {
+    // sum the token groups in a fixed order
+    if (g > 0 && g < kHessGroups) {
 #pragma unroll
         for (int a = 0; a < 4; ++a)
 #pragma unroll
             for (int c = 0; c < 4; ++c)
-                red[tg - 1][threadIdx.x & 63][4 * a + c] = acc[a][c];
+                red[g - 1][tile][4 * a + c] = acc[a][c];
     }
     __syncthreads();
-    if (tg == 0) {
+    if (g == 0) {
         float* o = part + (chunk * (cols / 32) + k) * 1024;
+        float v[4][4];
 #pragma unroll
-        for (int a = 0; a < 4; ++a) {
-            float v4[4];
+        for (int a = 0; a < 4; ++a)
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
-                float v = acc[a][c];
-                v = __fadd_rn(v, red[0][threadIdx.x][4 * a + c]);
-                v = __fadd_rn(v, red[1][threadIdx.x][4 * a + c]);
-                v = __fadd_rn(v, red[2][threadIdx.x][4 * a + c]);
-                v4[c] = v;
+                float s = acc[a][c];
+#pragma unroll
+                for (int q = 0; q < kHessGroups - 1; ++q)
+                    s = __fadd_rn(s, red[q][tile][4 * a + c]);
+                v[a][c] = s;
             }
-            *reinterpret_cast<float4*>(o + (4 * ti + a) * 32 + 4 * tj) = make_float4(v4[0], v4[1], v4[2], v4[3]);
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+            *reinterpret_cast<float4*>(o + (4 * ti + a) * 32 + 4 * tj) = make_float4(v[a][0], v[a][1], v[a][2], v[a][3]);
+        if (ti != tj) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                *reinterpret_cast<float4*>(o + (4 * tj + c) * 32 + 4 * ti) =
+                    make_float4(v[0][c], v[1][c], v[2][c], v[3][c]);
         }
     }
 }
