@@ -437,6 +437,21 @@ def oracle_sample_run(O, S):
 
 
 FULL_ELEMS = 4096 * 4096 + 16 * 8192 * 8192 + 8192 * 8192 + 16384 * 4096 + 8192 * 4096 + 4096 * 4096 + 8192 * 4096
+def max_over_ranks(torch, dist, ms, device):
+    """The slowest rank's time: every rank contributes its own device-timed
+    milliseconds and all get the maximum (one all-reduce, same order on every
+    rank)."""
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank, world, ms):
+    """Whole-job throughput in G units/s: every rank processed units_per_rank
+    in the (max-over-ranks) time ms."""
+    return units_per_rank * world / (ms * 1e-3) / 1e9
+
+
 SAMPLE_ROWS = {"c1": 1 / 4, "c2": 1 / 4, "c3": 1 / 4, "c4": 1 / 4, "c5": 1 / 4}
 
 
@@ -594,11 +609,9 @@ def main():
         clk["window"] = "the %d timed steps plus %d untimed repeats of the same step" % (args.steps, n_repeats)
     step_ms = float(np.mean([a.elapsed_time(b) for a, b in step_ev]))
     if world > 1:
-        t = torch.tensor([step_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        step_ms = float(t.item())
+        step_ms = max_over_ranks(torch, dist, step_ms, dev)
     units = sum(r.units for r in hot)
-    value = units * world / (step_ms * 1e-3) / 1e9
+    value = whole_job_rate(units, world, step_ms)
 
     row_out = {}
     for r in rows:
@@ -767,11 +780,9 @@ def run_e2e(torch, rows, X, host, stream, args, barrier, world, dist, dev):
     barrier()
     ms = e0.elapsed_time(e1) / n
     if dist is not None:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+        ms = max_over_ranks(torch, dist, ms, dev)
     units = sum(r.units for r in rows)
-    return {"value": units * world / (ms * 1e-3) / 1e9, "unit": "Gelem/s", "h2d_bytes_per_step": h2d,
+    return {"value": whole_job_rate(units, world, ms), "unit": "Gelem/s", "h2d_bytes_per_step": h2d,
             "d2h_bytes_per_step": d2h, "ms_per_step": ms,
             "overlap": "inputs in and outputs back on two copy streams, overlapped with the rows' compute"}
 
