@@ -437,6 +437,18 @@ def oracle_sample_run(O, S):
 
 
 FULL_ELEMS = 4096 * 4096 + 16 * 8192 * 8192 + 8192 * 8192 + 16384 * 4096 + 8192 * 4096 + 4096 * 4096 + 8192 * 4096
+def cpu_model():
+    """The host CPU's model name (first entry of /proc/cpuinfo), or None."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
 def max_over_ranks(torch, dist, ms, device):
     """The slowest rank's time: every rank contributes its own device-timed
     milliseconds and all get the maximum (one all-reduce, same order on every
@@ -477,7 +489,7 @@ def run_reference(args, rank, world):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": WORKLOAD, "sample": "the first quarter of the rows of every input"},
-        "cpu_baseline": {"value": value, "unit": "Gelem/s", "cores": cores, "kind": "oracle",
+        "cpu_baseline": {"value": value, "unit": "Gelem/s", "cores": cores, "kind": "oracle", "cpu_model": cpu_model(),
                          "sample": "each step quantizes %d of the %d elements of a full step (row prefixes)" % (elems, FULL_ELEMS)},
         "e2e": {"value": value, "unit": "Gelem/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -617,6 +629,7 @@ def main():
     for r in rows:
         ms = float(np.mean([a.elapsed_time(b) for a, b in per_row[r.name]]))
         d = {"ms": ms, "GB_s": r.bytes / (ms * 1e-3) / 1e9, "hbm_frac": r.bytes / (ms * 1e-3) / 1e9 / hbm_peak,
+             "hbm_frac_of_8000": r.bytes / (ms * 1e-3) / 1e9 / 8000.0,
              "launches": r.launches, "bound": r.bound}
         if r.units:
             d["Gelem_s"] = r.units / (ms * 1e-3) / 1e9
@@ -679,6 +692,7 @@ def main():
             secs.append(sec)
         sec = float(np.mean(secs))
         cpu = {"value": elems / sec / 1e9, "unit": "Gelem/s", "cores": O.get_threads(), "kind": "oracle",
+               "cpu_model": cpu_model(),
                "sample": "the first quarter of the rows of every input (%d of the %d elements of a step), "
                          "3 repeats, %.1f s each" % (elems, FULL_ELEMS, sec)}
 
@@ -688,6 +702,7 @@ def main():
     if gem is not None:
         g = row_out[gem.name]
         gemm = {"TFLOP_s": g["TFLOP_s"], "frac_of_fp4_peak": g["tensor_frac"], "fp4_peak_TFLOP_s": fp4_peak,
+                "frac_of_9000_spec": g["TFLOP_s"] / 9000.0,
                 "ms": g["ms"], "shape": "M=8192 N=14336 K=4096", "traffic": profiled_traffic("c5_w4a4_gemm")}
     line = {
         "metric": METRIC, "value": value, "unit": "Gelem/s", "n_gpus": world, "steps": args.steps,
