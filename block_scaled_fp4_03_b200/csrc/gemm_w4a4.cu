@@ -275,6 +275,17 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32])
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// 64 consecutive accumulator columns of this warp's 32 lanes, one load and one wait.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64])
+{
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x64.b32 "
+                 "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%64];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+                 : "r"(taddr)
+                 : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
 // Shared-memory matrix descriptor, K-major, 128-byte swizzle: 8-row groups
 // 1024 bytes apart (leading offset unused, encoded 1), sm100 version 1.
 __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr)
@@ -874,22 +885,28 @@ w4a4_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
             // goes back to the MMA issuer before any store is waited for
             uint32_t pk[4][16];
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                uint32_t r[32];
-                tmem_ld32(tq + 32 * c, r);
-                uint32_t h16[16];
+            for (int c2 = 0; c2 < 4; ++c2) {
+                // two 32-column chunks per TMEM load: half the load round trips
+                uint32_t r[64];
+                tmem_ld64(tq + 64 * c2, r);
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[2 * j]), scale),
-                                                             __fmul_rn(__uint_as_float(r[2 * j + 1]), scale));
-                    h16[j] = *reinterpret_cast<uint32_t*>(&h);
-                }
-                if (c < 4) {
-                    stage_row_chunk(stg, c, lane, h16);
-                } else {
+                for (int h = 0; h < 2; ++h) {
+                    const int c = 2 * c2 + h;
+                    uint32_t h16[16];
 #pragma unroll
-                    for (int j = 0; j < 16; ++j)
-                        pk[c - 4][j] = h16[j];
+                    for (int j = 0; j < 16; ++j) {
+                        __nv_bfloat162 b = __floats2bfloat162_rn(
+                            __fmul_rn(__uint_as_float(r[32 * h + 2 * j]), scale),
+                            __fmul_rn(__uint_as_float(r[32 * h + 2 * j + 1]), scale));
+                        h16[j] = *reinterpret_cast<uint32_t*>(&b);
+                    }
+                    if (c < 4) {
+                        stage_row_chunk(stg, c, lane, h16);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 16; ++j)
+                            pk[c - 4][j] = h16[j];
+                    }
                 }
             }
             tc_fence_before();
