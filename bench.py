@@ -505,6 +505,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="launch the timed step eagerly, not as a CUDA graph")
     ap.add_argument("--no-next-rows", action="store_true",
                     help="time the hot-path step only (skip the rows built on top of it)")
     ap.add_argument("--profile-row", default=None,
@@ -592,6 +593,28 @@ def main():
             dist.barrier()
         torch.cuda.synchronize()
 
+    # the hot step as one CUDA graph: its launches replay back to back with no
+    # host launch overhead between them (every buffer the rows touch already
+    # exists after the warm-up, so the capture allocates nothing)
+    graph, graph_note = None, "eager launches (--no-graph)"
+    if not args.no_graph:
+        try:
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                run_rows(hot)
+            torch.cuda.synchronize()
+            graph, graph_note = g, "one CUDA graph replay of the step's launches"
+        except Exception as e:    # report and time the eager step instead
+            graph_note = "eager launches (graph capture failed: %s)" % str(e).splitlines()[0][:160]
+            torch.cuda.synchronize()
+
+    def hot_step():
+        if graph is not None:
+            graph.replay()
+        else:
+            run_rows(hot)
+
     clocks = ClockSampler(local)
     per_row = {r.name: [] for r in rows}
     step_ev = []
@@ -601,10 +624,13 @@ def main():
         flush.zero_()
         s0, s1 = torch.cuda.Event(True), torch.cuda.Event(True)
         s0.record(stream)
-        run_rows(hot, per_row)
+        hot_step()
         s1.record(stream)
         step_ev.append((s0, s1))
-        # the next rows, outside the step (their inputs may share L2 with it)
+        # per-row times: the same rows launched one by one, each between two
+        # events, after another flush; then the next rows, outside the step
+        flush.zero_()
+        run_rows(hot, per_row)
         flush.zero_()
         run_rows(extra, per_row)
     barrier()
@@ -613,7 +639,7 @@ def main():
     # step until it has lasted at least 1.5 s
     n_repeats = 0
     while time.perf_counter() - clocks.t0 < 1.5:
-        run_rows(hot)
+        hot_step()
         torch.cuda.synchronize()
         n_repeats += 1
     clk = clocks.stop()
@@ -709,6 +735,7 @@ def main():
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": WORKLOAD, "elements_per_step_per_gpu": units, "l2": "flushed before every step (512 MiB write)",
+                   "step_launch": graph_note,
                    "parallelism": "replicas: every rank runs the full step on its own inputs"},
         "roofline": roof, "gemm": gemm, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clk,
         "rows": row_out,

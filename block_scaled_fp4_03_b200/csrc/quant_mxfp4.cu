@@ -10,6 +10,7 @@
 // explicit round-to-nearest operations, in the same order as the definition.
 #include <cfloat>
 #include <cstdint>
+#include <mutex>
 
 #include "fp4q_device.cuh"
 #include "fp4q_internal.h"
@@ -339,106 +340,9 @@ mx_quant_hessian_kernel(const T* __restrict__ x, int64_t rows, int64_t kb,
 }
 
 // ------------------------------------------------------- Hessian blocks
-// Partial H'_k over a chunk of kTok tokens: the chunk's transformed rows are
-// staged in shared memory, then each thread accumulates one 4x4 tile of the
-// upper triangle of H'_k (36 tiles, the diagonal ones included) over every
-// 7th token of the chunk; the lower triangle is written as the transpose
-// (H'_k is symmetric, and x_i * x_j rounds exactly as x_j * x_i).  The seven
-// token groups are summed in a fixed order.  Partials go to
-// ws[chunk][k][32][32] and are summed in chunk order by hessian_reduce_kernel.
+// H'_k partial sums are taken over chunks of kTok tokens (hessian_partial_tc_kernel
+// below) and summed in chunk order by hessian_reduce_kernel.
 constexpr int kTok = 256;
-constexpr int kHessTiles = 36;                  // 4x4 tiles with ti <= tj
-constexpr int kHessGroups = kThreads / kHessTiles;   // 7 token groups
-
-template <typename T>
-__global__ void __launch_bounds__(kThreads)
-hessian_partial_kernel(const T* __restrict__ x, int64_t rows, int64_t cols,
-                       const float* __restrict__ t, int had, float* __restrict__ part)
-{
-    __shared__ __align__(16) float Xs[kTok][32];
-    __shared__ __align__(16) float red[kHessGroups - 1][kHessTiles][16];
-    const int64_t k = blockIdx.y;
-    const int64_t chunk = blockIdx.x;
-    const int64_t r0 = chunk * kTok;
-    // stage: one thread per token row of this chunk, transformed in registers
-    for (int rr = threadIdx.x; rr < kTok; rr += blockDim.x) {
-        const int64_t r = r0 + rr;
-        float u[32];
-        if (r < rows) {
-            load32<T>(x + r * cols + k * 32, u);
-            online_transform(u, t ? t + k * 32 : nullptr, had != 0);
-        } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-                u[i] = 0.0f;
-        }
-#pragma unroll
-        for (int i = 0; i < 32; i += 4)
-            *reinterpret_cast<float4*>(&Xs[rr][i]) = make_float4(u[i], u[i + 1], u[i + 2], u[i + 3]);
-    }
-    __syncthreads();
-    const int tile = threadIdx.x % kHessTiles;
-    const int g = threadIdx.x / kHessTiles;       // token group; kHessGroups is idle
-    // tile -> (ti, tj), ti <= tj, row by row of the upper triangle
-    int ti = 0, tj = tile;
-    while (tj >= 8 - ti) {
-        tj -= 8 - ti;
-        ++ti;
-    }
-    tj += ti;
-    float acc[4][4];
-#pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-            acc[a][c] = 0.0f;
-    const int nr = (int)((rows - r0) < kTok ? (rows - r0) : kTok);
-    if (g < kHessGroups) {
-        for (int rr = g; rr < nr; rr += kHessGroups) {
-            const float4 xi = *reinterpret_cast<const float4*>(&Xs[rr][4 * ti]);
-            const float4 xj = *reinterpret_cast<const float4*>(&Xs[rr][4 * tj]);
-            const float vi[4] = {xi.x, xi.y, xi.z, xi.w};
-            const float vj[4] = {xj.x, xj.y, xj.z, xj.w};
-#pragma unroll
-            for (int a = 0; a < 4; ++a)
-#pragma unroll
-                for (int c = 0; c < 4; ++c)
-                    acc[a][c] = __fmaf_rn(vi[a], vj[c], acc[a][c]);
-        }
-    }
-    // sum the token groups in a fixed order
-    if (g > 0 && g < kHessGroups) {
-#pragma unroll
-        for (int a = 0; a < 4; ++a)
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-                red[g - 1][tile][4 * a + c] = acc[a][c];
-    }
-    __syncthreads();
-    if (g == 0) {
-        float* o = part + (chunk * (cols / 32) + k) * 1024;
-        float v[4][4];
-#pragma unroll
-        for (int a = 0; a < 4; ++a)
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                float s = acc[a][c];
-#pragma unroll
-                for (int q = 0; q < kHessGroups - 1; ++q)
-                    s = __fadd_rn(s, red[q][tile][4 * a + c]);
-                v[a][c] = s;
-            }
-#pragma unroll
-        for (int a = 0; a < 4; ++a)
-            *reinterpret_cast<float4*>(o + (4 * ti + a) * 32 + 4 * tj) = make_float4(v[a][0], v[a][1], v[a][2], v[a][3]);
-        if (ti != tj) {
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-                *reinterpret_cast<float4*>(o + (4 * tj + c) * 32 + 4 * ti) =
-                    make_float4(v[0][c], v[1][c], v[2][c], v[3][c]);
-        }
-    }
-}
 
 __global__ void __launch_bounds__(kThreads)
 hessian_reduce_kernel(const float* __restrict__ part, int64_t nchunk, int64_t total,
@@ -579,6 +483,266 @@ int grid_for(int64_t work, const void* kernel)
     return (int)(want < 1 ? 1 : want);
 }
 
+// ------------------------------------------- Hessian blocks on tensor cores
+// The same partial sums H'_k over a chunk of kTok tokens, as tcgen05 MMAs.
+// Four column blocks k0..k0+3 of the transformed chunk X' (tokens x 128
+// columns) are staged transposed, X'^T (128 rows = columns, K = tokens), in
+// the K-major 128B-swizzled layout; the same tile is both MMA operands, so
+// D = X'^T X' (128 x 128) holds the four wanted 32 x 32 blocks H'_k on its
+// diagonal.  tf32 operands carry 11 significant bits, so every value is split
+// x = hi + lo (hi = x rounded to tf32, lo = the remainder rounded to tf32) and
+//   D = hi^T hi + hi^T lo + lo^T hi
+// (lo^T lo, about 2^-22 relative, is dropped): three MMAs per k-step into one
+// 128-column TMEM accumulator, so three CTAs share an SM.  Warps 0-3 stage
+// (one token per lane, one column block per warp; the next K block's loads are
+// in flight while the current one is transformed and stored) and then read
+// back the diagonal block of their TMEM lane quarter; warp 4 owns the TMEM and
+// issues the MMAs.  Waits are bounded; a CTA that gives up writes NaN into its
+// partial blocks, which the reduction carries into H'.
+constexpr int kHxKB = 32;                       // tokens per K block (128 B of tf32 per tile row)
+constexpr int kHxTile = 128 * 128;              // bytes of one operand tile
+constexpr int kHxThreads = 160;
+// dynamic shared memory: 2 stages x (hi, lo) tiles, barriers, alignment slack;
+// at most three CTAs fit an SM (each holds 128 of its 512 TMEM columns)
+constexpr int kHxSmem = 4 * kHxTile + 2048;
+constexpr int kHxCols = 128;
+constexpr long long kHxWaitCycles = 4000000000LL;
+// kind::tf32, fp32 accumulate, K-major A and B, N = 128, M = 128
+constexpr uint32_t kHxIdesc = (1u << 4) | (2u << 7) | (2u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+
+__device__ __forceinline__ uint32_t hx_smem(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ bool hx_try_wait(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok)
+                 : "r"(bar), "r"(parity)
+                 : "memory");
+    return ok != 0;
+}
+
+// False if the phase did not complete in time or the CTA's abort flag rose.
+__device__ __noinline__ bool hx_wait(uint32_t bar, uint32_t parity, const volatile int* abort_flag)
+{
+    const long long t0 = clock64();
+    while (!hx_try_wait(bar, parity)) {
+        if ((abort_flag && *abort_flag) || clock64() - t0 > kHxWaitCycles)
+            return false;
+    }
+    return true;
+}
+
+__device__ __forceinline__ uint64_t hx_sdesc(uint32_t saddr)
+{
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+__device__ __forceinline__ void hx_mma(uint32_t tacc, uint64_t da, uint64_t db, uint32_t accumulate)
+{
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "setp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(tacc),
+                 "l"(da), "l"(db), "r"(kHxIdesc), "r"(accumulate)
+                 : "memory");
+}
+
+__device__ __forceinline__ void hx_commit(uint32_t bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+
+__device__ __forceinline__ void hx_ld32(uint32_t taddr, float (&v)[32])
+{
+    uint32_t r[32];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+                 "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+                 "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+                   "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+                   "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+                   "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+                   "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+                   "=r"(r[31])
+                 : "r"(taddr)
+                 : "memory");
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int j = 0; j < 32; ++j)
+        v[j] = __uint_as_float(r[j]);
+}
+
+__device__ __forceinline__ float hx_tf32(float a)
+{
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(a));
+    return __uint_as_float(r);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kHxThreads, 1)
+hessian_partial_tc_kernel(const T* __restrict__ x, int64_t rows, int64_t cols, const float* __restrict__ t,
+                          int had, float* __restrict__ part)
+{
+    extern __shared__ uint8_t hx_raw[];
+    uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(hx_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + 4 * kHxTile);
+    // bars: full[0], full[1] (128 stagers), empty[0], empty[1] (MMA commit),
+    // acc_full, drain
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 6);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+    const uint32_t bar0 = hx_smem(bars);
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int64_t kb = cols / 32;
+    const int64_t chunk = blockIdx.x;
+    const int64_t k0 = 4 * (int64_t)blockIdx.y;
+    const int nblk = (int)((kb - k0) < 4 ? (kb - k0) : 4);
+    const int64_t r0 = chunk * kTok;
+    constexpr int kSteps = kTok / kHxKB;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < 2; ++i) {
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar0 + 8u * i), "r"(128) : "memory");
+            asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar0 + 8u * (2 + i)), "r"(1) : "memory");
+        }
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar0 + 32u), "r"(1) : "memory");
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar0 + 40u), "r"(1) : "memory");
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 4) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(hx_smem(tmem_holder)),
+                     "r"(kHxCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    const uint32_t tmem = *tmem_holder;
+
+    if (warp < 4) {
+        // ---------------- staging: lane = token of the K block, warp = column block
+        const int b = warp;
+        const int64_t col0 = (k0 + b) * 32;
+        constexpr int kRaw = 32 * (int)sizeof(T) / 16;     // 16-byte vectors per token row
+        uint4 raw[kRaw];
+        auto fetch = [&](int s) {
+            const int64_t r = r0 + (int64_t)s * kHxKB + lane;
+            if (b < nblk && r < rows) {
+                const uint4* p = reinterpret_cast<const uint4*>(x + r * cols + col0);
+#pragma unroll
+                for (int v = 0; v < kRaw; ++v)
+                    raw[v] = __ldg(p + v);
+            } else {
+#pragma unroll
+                for (int v = 0; v < kRaw; ++v)
+                    raw[v] = make_uint4(0u, 0u, 0u, 0u);
+            }
+        };
+        fetch(0);
+        for (int s = 0; s < kSteps && !*abort_flag; ++s) {
+            const int st = s & 1;
+            const uint32_t use = (uint32_t)(s >> 1);
+            float u[32];
+#pragma unroll
+            for (int v = 0; v < kRaw; ++v) {
+                if constexpr (sizeof(T) == 4) {
+                    u[4 * v] = __uint_as_float(raw[v].x);
+                    u[4 * v + 1] = __uint_as_float(raw[v].y);
+                    u[4 * v + 2] = __uint_as_float(raw[v].z);
+                    u[4 * v + 3] = __uint_as_float(raw[v].w);
+                } else {
+                    bf16x2_to_f32(raw[v].x, u[8 * v], u[8 * v + 1]);
+                    bf16x2_to_f32(raw[v].y, u[8 * v + 2], u[8 * v + 3]);
+                    bf16x2_to_f32(raw[v].z, u[8 * v + 4], u[8 * v + 5]);
+                    bf16x2_to_f32(raw[v].w, u[8 * v + 6], u[8 * v + 7]);
+                }
+            }
+            if (s + 1 < kSteps)
+                fetch(s + 1);          // in flight while this block is transformed
+            if (use > 0 && !hx_wait(bar0 + 8u * (2 + st), (use - 1u) & 1u, abort_flag)) {
+                *abort_flag = 1;
+                break;
+            }
+            uint8_t* hi = sm + st * 2 * kHxTile;
+            uint8_t* lo = hi + kHxTile;
+            online_transform(u, t ? t + col0 : nullptr, had != 0);
+            // X'^T: row m = 32 b + i, K position = lane; 16-byte chunk (lane/4)
+            // XOR (m % 8) of the 128-byte row
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const int m = 32 * b + i;
+                const uint32_t off = (uint32_t)m * 128u + ((((uint32_t)lane >> 2) ^ ((uint32_t)m & 7u)) << 4) +
+                                     ((uint32_t)lane & 3u) * 4u;
+                const float h = hx_tf32(u[i]);
+                *reinterpret_cast<float*>(hi + off) = h;
+                *reinterpret_cast<float*>(lo + off) = hx_tf32(__fsub_rn(u[i], h));
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar0 + 8u * st) : "memory");
+        }
+        // ---------------- epilogue: the diagonal 32 x 32 block of this lane quarter
+        const bool ok = __all_sync(0xffffffffu, !*abort_flag && hx_wait(bar0 + 32u, 0u, abort_flag));
+        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        if (b < nblk) {
+            float h[32];
+            if (ok) {
+                hx_ld32(tmem + ((uint32_t)(32 * b) << 16) + (uint32_t)(32 * b), h);
+            } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    h[j] = __uint_as_float(0x7FC00000u);
+            }
+            float* o = part + (chunk * kb + k0 + b) * 1024 + lane * 32;
+#pragma unroll
+            for (int j = 0; j < 32; j += 4)
+                *reinterpret_cast<float4*>(o + j) = make_float4(h[j], h[j + 1], h[j + 2], h[j + 3]);
+        }
+    } else if (lane == 0) {
+        // ---------------- MMA issuer: D += hi hi^T + hi lo^T + lo hi^T per k-step
+        bool issued = false;
+        for (int s = 0; s < kSteps; ++s) {
+            const int st = s & 1;
+            if (!hx_wait(bar0 + 8u * st, (uint32_t)(s >> 1) & 1u, abort_flag)) {
+                *abort_flag = 1;
+                break;
+            }
+            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+            const uint32_t hi = hx_smem(sm + st * 2 * kHxTile);
+            const uint32_t lo = hi + kHxTile;
+#pragma unroll
+            for (int k = 0; k < kHxKB / 8; ++k) {
+                const uint64_t dh = hx_sdesc(hi + 32u * k);
+                const uint64_t dl = hx_sdesc(lo + 32u * k);
+                hx_mma(tmem, dh, dh, (s | k) != 0);
+                hx_mma(tmem, dh, dl, 1u);
+                hx_mma(tmem, dl, dh, 1u);
+            }
+            issued = true;
+            hx_commit(bar0 + 8u * (2 + st));
+        }
+        if (!*abort_flag)
+            hx_commit(bar0 + 32u);
+        if (issued) {
+            // every MMA of this CTA has finished before the TMEM goes away
+            hx_commit(bar0 + 40u);
+            if (!hx_wait(bar0 + 40u, 0u, nullptr))
+                *abort_flag = 1;
+        }
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    if (warp == 4)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kHxCols) : "memory");
+}
+
 }  // namespace
 
 size_t hessian_ws_bytes(int64_t rows, int64_t cols)
@@ -638,12 +802,23 @@ cudaError_t launch_hessian_blocks(const void* x, int dtype, int64_t rows, int64_
     const int64_t kb = cols / 32;
     const int64_t nchunk = (rows + kTok - 1) / kTok;
     float* part = reinterpret_cast<float*>(ws);
-    dim3 grid((unsigned)nchunk, (unsigned)kb);
+    static std::once_flag hx_once;
+    static cudaError_t hx_attr = cudaSuccess;
+    std::call_once(hx_once, [] {
+        hx_attr = cudaFuncSetAttribute(hessian_partial_tc_kernel<__nv_bfloat16>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kHxSmem);
+        if (hx_attr == cudaSuccess)
+            hx_attr = cudaFuncSetAttribute(hessian_partial_tc_kernel<float>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, kHxSmem);
+    });
+    if (hx_attr != cudaSuccess)
+        return hx_attr;
+    dim3 grid((unsigned)nchunk, (unsigned)((kb + 3) / 4));
     if (dtype == 1)
-        hessian_partial_kernel<__nv_bfloat16><<<grid, kThreads, 0, s>>>(
+        hessian_partial_tc_kernel<__nv_bfloat16><<<grid, kHxThreads, kHxSmem, s>>>(
             reinterpret_cast<const __nv_bfloat16*>(x), rows, cols, chan_scale, hadamard, part);
     else
-        hessian_partial_kernel<float><<<grid, kThreads, 0, s>>>(
+        hessian_partial_tc_kernel<float><<<grid, kHxThreads, kHxSmem, s>>>(
             reinterpret_cast<const float*>(x), rows, cols, chan_scale, hadamard, part);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess)
