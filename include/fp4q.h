@@ -241,7 +241,10 @@ FP4Q_API int mxfp4_flip_refine(const void* w, int dtype, int64_t rows, int64_t c
 /*
  * Diagonal 32x32 blocks of the Hessian of the transformed activations,
  * H'_k = X'_k^T X'_k with X' = transform(x) as in mxfp4_quantize ([MACaQ] 1,
- * H = X^T X).  fp32 accumulation (tolerance, not bit-exact).
+ * H = X^T X).  Computed on the tcgen05 tensor cores in tf32 with every value
+ * split into two tf32 parts (hi + lo) and fp32 accumulation: about fp32
+ * accuracy (tolerance, not bit-exact); partial sums per 256 tokens are added
+ * in a fixed order, so the result is deterministic.
  *  hess_blocks  device fp32 [cols/32][32][32] (out)
  *  workspace    >= fp4q_workspace_size(FP4Q_OP_HESSIAN, rows, cols, 0)
  */
