@@ -70,7 +70,7 @@ PROFILE_OF_ROW = {
     "c3_razer_act": "razer_paired_kernel_acts_16384x4096_bf16.md",
     "c4_mx_act": "mx_quant_absmax_kernel_acts_8192x4096_bf16.md",
     "c4_mx_weight_hessian": "mx_quant_hessian_kernel_weights_4096x4096_bf16.md",
-    "c4_hessian_blocks": "hessian_partial_kernel_acts_8192x4096_bf16.md",
+    "c4_hessian_blocks": "hessian_partial_tc_kernel_acts_8192x4096_bf16.md",
     "c5_act_quant_4o6_mma": "nvfp4_quant_kernel_B16_4o6_bf16_mma_layout_8192x4096.md",
     "c5_w4a4_gemm": "w4a4_gemm_2sm_kernel_M8192_N14336_K4096.md",
     "c1_nvfp4_pz_deq_mse": "nvfp4_quant_kernel_B16_pz_deq_mse_gaussian_4096x4096.md",
