@@ -28,6 +28,7 @@
 
 #include "fp4q_device.cuh"
 #include "fp4q_internal.h"
+#include "tc05_common.cuh"
 
 namespace fp4q {
 
@@ -48,9 +49,8 @@ constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSfCol0 = 256;              // accumulator uses columns [0, 256)
 constexpr uint32_t kSfColsPerStage = 48;       // SFA 4 k-steps x 4 + SFB 4 k-steps x 8
-constexpr long long kWaitCycles = 4000000000LL;   // about 2 s at the boost clock
 // The pair teardown outlasts a peer's own quiesce waits.
-constexpr long long kTeardownCycles = 3 * kWaitCycles;
+constexpr long long kTeardownCycles = 3 * kTcWaitCycles;
 // Grace period for copies whose completion this CTA cannot observe (about 1 ms).
 constexpr long long kDrainCycles = 2000000LL;
 
@@ -95,66 +95,11 @@ __device__ __forceinline__ void mma_scale_operands(int s, uint32_t tsfa, uint32_
     }
 }
 
-__device__ __forceinline__ uint32_t smem_u32(const void* p)
-{
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
 // ---------------------------------------------------------------- mbarrier
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
-{
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-
 __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes)
 {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
                  : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint32_t bar)
-{
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
-{
-    uint32_t ok;
-    asm volatile("{\n\t.reg .pred p;\n\t"
-                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-                 "selp.u32 %0, 1, 0, p;\n\t}"
-                 : "=r"(ok)
-                 : "r"(bar), "r"(parity)
-                 : "memory");
-    return ok != 0;
-}
-
-// Wait for the phase with the given parity.  False if it did not complete
-// in time or, while waiting, this CTA's abort flag was raised.
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const volatile int* abort_flag)
-{
-    if (mbar_try_wait(bar, parity))
-        return true;
-    const long long t0 = clock64();
-    while (!mbar_try_wait(bar, parity)) {
-        if (*abort_flag || clock64() - t0 > kWaitCycles)
-            return false;
-    }
-    return true;
-}
-
-// Time-bounded wait that ignores the abort flag: used to let this CTA's own
-// copies and MMAs finish before its resources go away.
-__device__ __noinline__ bool mbar_quiesce(uint32_t bar, uint32_t parity)
-{
-    if (mbar_try_wait(bar, parity))
-        return true;
-    const long long t0 = clock64();
-    while (!mbar_try_wait(bar, parity)) {
-        if (clock64() - t0 > kWaitCycles)
-            return false;
-    }
-    return true;
 }
 
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity)
@@ -172,7 +117,7 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
 // Bounded wait with cluster-scope acquire, for barriers that other CTAs arrive
 // on; gives up after `limit` cycles or when the abort flag (if any) is raised.
 __device__ __noinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, const volatile int* abort_flag,
-                                               long long limit = kWaitCycles)
+                                               long long limit = kTcWaitCycles)
 {
     if (mbar_try_wait_cluster(bar, parity))
         return true;
@@ -225,14 +170,6 @@ __device__ __forceinline__ void tma_load_3d_pair(uint32_t dst, const CUtensorMap
 }
 
 // ---------------------------------------------------------------- tcgen05
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-__device__ __forceinline__ void tc_commit(uint32_t bar)
-{
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-                 : "memory");
-}
 
 // Copy one 512-byte scale atom (32 rows x 16 bytes in shared memory) into 4
 // TMEM columns, replicated into the four 32-lane quarters.
@@ -259,21 +196,6 @@ __device__ __forceinline__ void tc_mma(uint32_t tacc, uint64_t da, uint64_t db, 
                      : "memory");
 }
 
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32])
-{
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-                 "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-                 "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-                   "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-                   "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
-                   "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-                   "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
-                   "=r"(r[31])
-                 : "r"(taddr)
-                 : "memory");
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
 
 // 64 consecutive accumulator columns of this warp's 32 lanes, one load and one wait.
 __device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64])
@@ -286,13 +208,6 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64])
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
-// Shared-memory matrix descriptor, K-major, 128-byte swizzle: 8-row groups
-// 1024 bytes apart (leading offset unused, encoded 1), sm100 version 1.
-__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr)
-{
-    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
-           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
-}
 
 // Descriptor of a scale atom for tcgen05.cp: 32 rows of 16 bytes, no
 // swizzle, 8-row core matrices 128 bytes apart.

@@ -14,6 +14,7 @@
 
 #include "fp4q_device.cuh"
 #include "fp4q_internal.h"
+#include "tc05_common.cuh"
 
 namespace fp4q {
 
@@ -506,40 +507,11 @@ constexpr int kHxThreads = 160;
 // at most three CTAs fit an SM (each holds 128 of its 512 TMEM columns)
 constexpr int kHxSmem = 4 * kHxTile + 2048;
 constexpr int kHxCols = 128;
-constexpr long long kHxWaitCycles = 4000000000LL;
 // kind::tf32, fp32 accumulate, K-major A and B, N = 128, M = 128
 constexpr uint32_t kHxIdesc = (1u << 4) | (2u << 7) | (2u << 10) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
 
-__device__ __forceinline__ uint32_t hx_smem(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
-__device__ __forceinline__ bool hx_try_wait(uint32_t bar, uint32_t parity)
-{
-    uint32_t ok;
-    asm volatile("{\n\t.reg .pred p;\n\t"
-                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-                 "selp.u32 %0, 1, 0, p;\n\t}"
-                 : "=r"(ok)
-                 : "r"(bar), "r"(parity)
-                 : "memory");
-    return ok != 0;
-}
 
-// False if the phase did not complete in time or the CTA's abort flag rose.
-__device__ __noinline__ bool hx_wait(uint32_t bar, uint32_t parity, const volatile int* abort_flag)
-{
-    const long long t0 = clock64();
-    while (!hx_try_wait(bar, parity)) {
-        if ((abort_flag && *abort_flag) || clock64() - t0 > kHxWaitCycles)
-            return false;
-    }
-    return true;
-}
-
-__device__ __forceinline__ uint64_t hx_sdesc(uint32_t saddr)
-{
-    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
-           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
-}
 
 __device__ __forceinline__ void hx_mma(uint32_t tacc, uint64_t da, uint64_t db, uint32_t accumulate)
 {
@@ -550,31 +522,7 @@ __device__ __forceinline__ void hx_mma(uint32_t tacc, uint64_t da, uint64_t db, 
                  : "memory");
 }
 
-__device__ __forceinline__ void hx_commit(uint32_t bar)
-{
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-                 : "memory");
-}
 
-__device__ __forceinline__ void hx_ld32(uint32_t taddr, float (&v)[32])
-{
-    uint32_t r[32];
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-                 "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-                 "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-                   "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
-                   "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
-                   "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
-                   "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
-                   "=r"(r[31])
-                 : "r"(taddr)
-                 : "memory");
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int j = 0; j < 32; ++j)
-        v[j] = __uint_as_float(r[j]);
-}
 
 __device__ __forceinline__ float hx_tf32(float a)
 {
@@ -595,7 +543,7 @@ hessian_partial_tc_kernel(const T* __restrict__ x, int64_t rows, int64_t cols, c
     // acc_full, drain
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 6);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-    const uint32_t bar0 = hx_smem(bars);
+    const uint32_t bar0 = smem_u32(bars);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int64_t kb = cols / 32;
@@ -607,23 +555,23 @@ hessian_partial_tc_kernel(const T* __restrict__ x, int64_t rows, int64_t cols, c
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < 2; ++i) {
-            asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar0 + 8u * i), "r"(128) : "memory");
-            asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar0 + 8u * (2 + i)), "r"(1) : "memory");
+            mbar_init(bar0 + 8u * i, 128);
+            mbar_init(bar0 + 8u * (2 + i), 1);
         }
-        asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar0 + 32u), "r"(1) : "memory");
-        asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar0 + 40u), "r"(1) : "memory");
+        mbar_init(bar0 + 32u, 1);
+        mbar_init(bar0 + 40u, 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 4) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(hx_smem(tmem_holder)),
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_holder)),
                      "r"(kHxCols)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
-    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    tc_fence_before();
     __syncthreads();
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    tc_fence_after();
     const uint32_t tmem = *tmem_holder;
 
     if (warp < 4) {
@@ -666,7 +614,7 @@ hessian_partial_tc_kernel(const T* __restrict__ x, int64_t rows, int64_t cols, c
             }
             if (s + 1 < kSteps)
                 fetch(s + 1);          // in flight while this block is transformed
-            if (use > 0 && !hx_wait(bar0 + 8u * (2 + st), (use - 1u) & 1u, abort_flag)) {
+            if (use > 0 && !mbar_wait(bar0 + 8u * (2 + st), (use - 1u) & 1u, abort_flag)) {
                 *abort_flag = 1;
                 break;
             }
@@ -685,15 +633,19 @@ hessian_partial_tc_kernel(const T* __restrict__ x, int64_t rows, int64_t cols, c
                 *reinterpret_cast<float*>(lo + off) = hx_tf32(__fsub_rn(u[i], h));
             }
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar0 + 8u * st) : "memory");
+            mbar_arrive(bar0 + 8u * st);
         }
         // ---------------- epilogue: the diagonal 32 x 32 block of this lane quarter
-        const bool ok = __all_sync(0xffffffffu, !*abort_flag && hx_wait(bar0 + 32u, 0u, abort_flag));
-        asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+        const bool ok = __all_sync(0xffffffffu, !*abort_flag && mbar_wait(bar0 + 32u, 0u, abort_flag));
+        tc_fence_after();
         if (b < nblk) {
             float h[32];
             if (ok) {
-                hx_ld32(tmem + ((uint32_t)(32 * b) << 16) + (uint32_t)(32 * b), h);
+                uint32_t r[32];
+                tmem_ld32(tmem + ((uint32_t)(32 * b) << 16) + (uint32_t)(32 * b), r);
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    h[j] = __uint_as_float(r[j]);
             } else {
 #pragma unroll
                 for (int j = 0; j < 32; ++j)
@@ -709,36 +661,36 @@ hessian_partial_tc_kernel(const T* __restrict__ x, int64_t rows, int64_t cols, c
         bool issued = false;
         for (int s = 0; s < kSteps; ++s) {
             const int st = s & 1;
-            if (!hx_wait(bar0 + 8u * st, (uint32_t)(s >> 1) & 1u, abort_flag)) {
+            if (!mbar_wait(bar0 + 8u * st, (uint32_t)(s >> 1) & 1u, abort_flag)) {
                 *abort_flag = 1;
                 break;
             }
-            asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-            const uint32_t hi = hx_smem(sm + st * 2 * kHxTile);
+            tc_fence_after();
+            const uint32_t hi = smem_u32(sm + st * 2 * kHxTile);
             const uint32_t lo = hi + kHxTile;
 #pragma unroll
             for (int k = 0; k < kHxKB / 8; ++k) {
-                const uint64_t dh = hx_sdesc(hi + 32u * k);
-                const uint64_t dl = hx_sdesc(lo + 32u * k);
+                const uint64_t dh = sdesc_sw128(hi + 32u * k);
+                const uint64_t dl = sdesc_sw128(lo + 32u * k);
                 hx_mma(tmem, dh, dh, (s | k) != 0);
                 hx_mma(tmem, dh, dl, 1u);
                 hx_mma(tmem, dl, dh, 1u);
             }
             issued = true;
-            hx_commit(bar0 + 8u * (2 + st));
+            tc_commit(bar0 + 8u * (2 + st));
         }
         if (!*abort_flag)
-            hx_commit(bar0 + 32u);
+            tc_commit(bar0 + 32u);
         if (issued) {
             // every MMA of this CTA has finished before the TMEM goes away
-            hx_commit(bar0 + 40u);
-            if (!hx_wait(bar0 + 40u, 0u, nullptr))
+            tc_commit(bar0 + 40u);
+            if (!mbar_wait(bar0 + 40u, 0u, nullptr))
                 *abort_flag = 1;
         }
     }
-    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+    tc_fence_before();
     __syncthreads();
-    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    tc_fence_after();
     if (warp == 4)
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kHxCols) : "memory");
 }
