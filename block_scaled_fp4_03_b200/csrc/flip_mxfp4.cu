@@ -27,7 +27,6 @@
 // best is the largest positive gain, ties to the lowest element and, within
 // an element, to the downward move; after a move g_j <- fma(-D, H_ji, g_j).
 #include <cstdint>
-#include <mutex>
 
 #include "fp4q_device.cuh"
 #include "fp4q_internal.h"
@@ -412,21 +411,10 @@ size_t flip_refine_smem_bytes(int64_t cols)
 // (8192 columns) once per device.
 cudaError_t flip_refine_opt_in()
 {
-    static std::mutex mu;
-    static bool done[64] = {};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess || dev < 0 || dev >= 64)
-        return e != cudaSuccess ? e : cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(mu);
-    if (done[dev])
-        return cudaSuccess;
     const int smem = (int)flip_refine_smem_bytes(8192);
-    e = cudaFuncSetAttribute(flip_refine_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = smem_opt_in((const void*)flip_refine_kernel<__nv_bfloat16>, smem);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(flip_refine_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    if (e == cudaSuccess)
-        done[dev] = true;
+        e = smem_opt_in((const void*)flip_refine_kernel<float>, smem);
     return e;
 }
 

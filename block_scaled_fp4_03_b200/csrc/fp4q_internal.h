@@ -21,7 +21,12 @@ struct GsArgs {
 // Number of partial maxima launch_amax writes (fixed; the workspace holds them).
 constexpr int kAmaxPartials = 592;   // 148 SMs x 4
 
+// SM count of the current device (cached per device).
 int num_sms();
+
+// Raise `kernel`'s dynamic shared-memory limit to `bytes` on the current
+// device, once per (kernel, device); thread-safe.
+cudaError_t smem_opt_in(const void* kernel, int bytes);
 
 cudaError_t launch_amax(const void* x, int dtype, int64_t n, float* partials, cudaStream_t s);
 

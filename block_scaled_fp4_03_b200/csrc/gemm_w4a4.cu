@@ -954,12 +954,7 @@ cudaError_t launch_gemm_t(const uint8_t* a_codes, const uint8_t* a_sf, const uin
             !make_out_map(&to, out, M, N) || !make_code_map(&ta1, a1, M, K / 2, 128) ||
             !make_code_map(&tb1, w1, N, K / 2, 128))
             return cudaErrorInvalidValue;
-        static std::once_flag attr2_once;
-        static cudaError_t attr2_err = cudaSuccess;
-        std::call_once(attr2_once, [] {
-            attr2_err = cudaFuncSetAttribute(w4a4_gemm_2sm_kernel<MX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             k2SmemBytes);
-        });
+        const cudaError_t attr2_err = smem_opt_in((const void*)w4a4_gemm_2sm_kernel<MX>, k2SmemBytes);
         if (attr2_err != cudaSuccess)
             return attr2_err;
         p.tiles_m = (int)(M / 256);
@@ -974,12 +969,7 @@ cudaError_t launch_gemm_t(const uint8_t* a_codes, const uint8_t* a_sf, const uin
         !make_sf_map(&tsa, a_sf, M, K, 1, MX) || !make_sf_map(&tsb, w_sf, N, K, 2, MX) ||
         !make_code_map(&ta1, a1, M, K / 2, kBM) || !make_code_map(&tb1, w1, N, K / 2, kBN))
         return cudaErrorInvalidValue;
-    static std::once_flag attr_once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(attr_once, [] {
-        attr_err = cudaFuncSetAttribute(w4a4_gemm_1sm_kernel<MX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        kSmemBytes);
-    });
+    const cudaError_t attr_err = smem_opt_in((const void*)w4a4_gemm_1sm_kernel<MX>, kSmemBytes);
     if (attr_err != cudaSuccess)
         return attr_err;
     p.tiles_m = (int)(M / kBM);

@@ -10,7 +10,6 @@
 // explicit round-to-nearest operations, in the same order as the definition.
 #include <cfloat>
 #include <cstdint>
-#include <mutex>
 
 #include "fp4q_device.cuh"
 #include "fp4q_internal.h"
@@ -754,15 +753,9 @@ cudaError_t launch_hessian_blocks(const void* x, int dtype, int64_t rows, int64_
     const int64_t kb = cols / 32;
     const int64_t nchunk = (rows + kTok - 1) / kTok;
     float* part = reinterpret_cast<float*>(ws);
-    static std::once_flag hx_once;
-    static cudaError_t hx_attr = cudaSuccess;
-    std::call_once(hx_once, [] {
-        hx_attr = cudaFuncSetAttribute(hessian_partial_tc_kernel<__nv_bfloat16>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, kHxSmem);
-        if (hx_attr == cudaSuccess)
-            hx_attr = cudaFuncSetAttribute(hessian_partial_tc_kernel<float>,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize, kHxSmem);
-    });
+    const cudaError_t hx_attr =
+        dtype == 1 ? smem_opt_in((const void*)hessian_partial_tc_kernel<__nv_bfloat16>, kHxSmem)
+                   : smem_opt_in((const void*)hessian_partial_tc_kernel<float>, kHxSmem);
     if (hx_attr != cudaSuccess)
         return hx_attr;
     dim3 grid((unsigned)nchunk, (unsigned)((kb + 3) / 4));

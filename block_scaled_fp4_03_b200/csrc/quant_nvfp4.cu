@@ -1104,19 +1104,6 @@ cudaError_t dequant_launch_b(int block, const uint8_t* codes, const uint8_t* sca
 
 }  // namespace
 
-int num_sms()
-{
-    static int n = 0;
-    if (n == 0) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        if (n <= 0)
-            n = 148;
-    }
-    return n;
-}
-
 cudaError_t launch_amax(const void* x, int dtype, int64_t n, float* partials, cudaStream_t s)
 {
     if (dtype == 1)

@@ -1,0 +1,52 @@
+// runtime.cu -- per-device host-side state of the library: the SM count used to
+// size persistent grids, and the shared-memory opt-in of kernels that need more
+// than the default 48 KiB of dynamic shared memory.  Both are per device, so a
+// process that drives several GPUs gets each one right.
+#include <atomic>
+#include <mutex>
+#include <set>
+#include <utility>
+
+#include "fp4q_internal.h"
+
+namespace fp4q {
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::atomic<int> g_sms[kMaxDevices];
+std::mutex g_opt_mu;
+std::set<std::pair<const void*, int>> g_opted;   // (kernel, device) pairs already opted in
+
+}  // namespace
+
+int num_sms()
+{
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
+        return 148;
+    int n = g_sms[dev].load(std::memory_order_relaxed);
+    if (n == 0) {
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        g_sms[dev].store(n, std::memory_order_relaxed);
+    }
+    return n;
+}
+
+cudaError_t smem_opt_in(const void* kernel, int bytes)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    std::lock_guard<std::mutex> lock(g_opt_mu);
+    if (g_opted.count({kernel, dev}))
+        return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess)
+        g_opted.insert({kernel, dev});
+    return e;
+}
+
+}  // namespace fp4q
