@@ -64,3 +64,17 @@ def test_reference_arm_runs_on_rank_zero_only():
         warmup, steps, gpus = 1, 1, 2
     # a rank other than 0 returns at once, without touching the oracle
     assert bench.run_reference(Args, rank=1, world=2) is None
+
+
+def test_every_profiled_row_has_a_committed_summary():
+    """The bench reads a row's DRAM traffic from its committed ncu summary; each
+    mapped file must exist, carry its command and parse to a positive number."""
+    sys.path.insert(0, ROOT)
+    import bench
+    for row, fname in bench.PROFILE_OF_ROW.items():
+        path = os.path.join(ROOT, "profiles", fname)
+        assert os.path.exists(path), (row, fname)
+        text = open(path).read()
+        assert "ncu " in text and "--clock-control none" in text, fname
+        t = bench.profiled_traffic(row)
+        assert t is not None and t > 0, (row, fname)
