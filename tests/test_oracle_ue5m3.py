@@ -106,3 +106,37 @@ def test_page_claim_e4m3_recipe_matches_ue5m3(O, B):
     assert e4_abs1 > 20 * ue_abs
     zero_scales = (O.block_fp4_quantize(x, B, O.RULE_ABSMAX, O.SF_UE5M3, 1.0)["scales"] == 0).mean()
     assert zero_scales < 1e-3
+
+
+def _exact_block_sse(xb, s):
+    """Exact SSE of block xb at scale s: RNE to the E2M1 grid (ties to the even
+    code), saturating at 6 -- written out with rationals, independent of the
+    oracle's fp32 arithmetic."""
+    grid = [Fraction(v) for v in (0, 0.5, 1, 1.5, 2, 3, 4, 6)]
+    tot = Fraction(0)
+    for v in xb:
+        a = abs(Fraction(float(v)))
+        y = a / s
+        if y >= 6:
+            q = grid[-1]
+        else:
+            q = min(range(8), key=lambda i: (abs(y - grid[i]), i % 2))
+            q = grid[q]
+        tot += (a - q * s) ** 2
+    return tot
+
+
+@pytest.mark.parametrize("B,mag", [(4, 1e-5), (8, 1.0), (16, 3e3), (4, 40.0)])
+def test_brute_force_tiny_exhaustive_exact(O, B, mag):
+    """UE5M3 brute force: over all 254 finite positive scales, the chosen one's
+    exact block error is the minimum (to fp32 rounding of the search)."""
+    rng = np.random.default_rng(int(B * 7 + mag * 3) % 1000)
+    x = (rng.standard_normal((1, 2 * B)) * mag).astype(np.float32)
+    r = O.block_fp4_quantize(x, B, O.RULE_BRUTE_FORCE, O.SF_UE5M3, 1.0)
+    scales = [Fraction(O.ue5m3_value(c)) for c in range(1, 255)]
+    for b in range(2):
+        xb = x[0, b * B:(b + 1) * B]
+        exact = [_exact_block_sse(xb, s) for s in scales]
+        best = min(exact)
+        chosen = exact[int(r["scales"][0, b]) - 1]
+        assert float(chosen) <= float(best) * (1 + 1e-5) + 1e-45, (b, float(chosen), float(best))
