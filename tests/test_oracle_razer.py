@@ -96,3 +96,45 @@ def test_plus_minus_five_is_the_best_pair(O):
         tot = {v: O.razer_quantize(x, sf, [v, -v], g=g)["mse"].astype(np.float64).mean()
                for v in (2.5, 3.5, 4.5, 5.0, 5.5)}
         assert min(tot, key=tot.get) == 5.0
+
+
+def _exact_razer_block(xb, S, v):
+    """Exact rational SSE of one block under the RaZeR encode of section 2.2 as
+    read here: each element takes the nearest E2M1 grid value (ties to the
+    even code, saturating at 6) unless it has v's sign, the grid value is not
+    zero, and |y| is strictly nearer to |v| than to the grid value -- then it
+    takes v.  Written with Fractions, independent of the oracle's fp32 code."""
+    from fractions import Fraction
+    grid = [Fraction(g) for g in (0, 0.5, 1, 1.5, 2, 3, 4, 6)]
+    v = Fraction(v)
+    tot = Fraction(0)
+    for x in xb:
+        xf = Fraction(float(x))
+        y = xf / S
+        ay = abs(y)
+        m = 7 if ay >= 6 else min(range(8), key=lambda i: (abs(ay - grid[i]), i % 2))
+        q = grid[m] * (1 if y >= 0 else -1)
+        if m != 0 and (y > 0) == (v > 0) and abs(ay - abs(v)) < abs(ay - grid[m]):
+            q = v
+        tot += (xf - q * S) ** 2
+    return tot
+
+
+@pytest.mark.parametrize("sf,specials", [(0, A_SPECIALS), (1, W_SPECIALS)])
+def test_selection_matches_exact_rational_search(O, sf, specials):
+    """On tiny inputs whose scaled values are exact (g = 1, scale = block max / 6
+    rounded to the format), the chosen special is the exact-arithmetic minimum
+    over the table (ties to the earlier entry) and the reported MSE is its error."""
+    from fractions import Fraction
+    rng = np.random.default_rng(17 + sf)
+    x = (rng.standard_normal((6, 16)) * 2.0).astype(np.float32)
+    r = O.razer_quantize(x, sf, specials, g=1.0)
+    val = O.e3m3_value if sf == 1 else O.e4m3_value
+    for b in range(6):
+        meta = int(r["meta"][b, 0])
+        sel, code = (meta >> 6, meta & 0x3F) if sf == 1 else (meta >> 7, meta & 0x7F)
+        S = Fraction(val(code))
+        errs = [_exact_razer_block(x[b], S, v) for v in specials]
+        best = min(errs)
+        assert errs[sel] <= best * (1 + Fraction(1, 10 ** 5)) + Fraction(1, 10 ** 40), (b, sel, errs)
+        assert abs(float(r["mse"][b, 0]) - float(errs[sel]) / 16) <= 1e-5 * float(errs[sel]) / 16 + 1e-30
