@@ -156,3 +156,22 @@ def test_gemm_family_argument_errors(L):
     assert L.fp4_scales_to_mma(FAKE, 128, 6, FAKE, None) == 1
     assert L.fp4_scales_to_mma(MIS, 128, 8, FAKE, None) == 2
     assert L.fp4_scales_to_mma(None, 0, 8, None, None) == 0
+
+
+def test_header_is_plain_c(tmp_path):
+    """include/fp4q.h compiles as C99 on its own (a C-ABI header, no C++ or CUDA types)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use.c"
+    src.write_text('#include "fp4q.h"\n'
+                   'int main(void) {\n'
+                   '    size_t n = fp4q_workspace_size(FP4Q_OP_GEMM, 128, 256, 256);\n'
+                   '    const char* s = fp4q_status_str(FP4Q_ERR_ARG);\n'
+                   '    return (int)(n == 0) + (s == 0);\n'
+                   '}\n')
+    r = subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-pedantic", "-fsyntax-only",
+                        "-I", os.path.join(ROOT, "include"), str(src)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
