@@ -4,8 +4,13 @@
 // i.e. A . W^T with both operands NVFP4 (E2M1 codes, one E4M3 scale per 16
 // elements along K, an FP32 global scale each): the W4A4 inference of the
 // "Why Gated DeltaNet Survives 4-Bit Quantization" review, section 1.
+// The same kernels also run (template argument MX) MXFP4 operands -- one E8M0
+// scale per 32 elements, no global scale, kind::mxf4 -- for the MACaQ W4A4
+// path, and (GemmParams passes) the RaZeR operands split in two E2M1 tensors,
+// one pass over K per operand pair into the same accumulator.
 //
-// Kernel shape (one CTA per SM, persistent over 128 x 256 output tiles):
+// The CTA-pair kernel (M % 256 == 0) is described at its definition below.
+// The single-CTA kernel (one CTA per SM, persistent over 128 x 256 tiles):
 //   warp 0     TMA producer: FP4 code tiles (128B-swizzled, K-major) and
 //              scale-factor atoms (512 contiguous bytes each, already in the
 //              MMA layout) by cp.async.bulk.tensor
