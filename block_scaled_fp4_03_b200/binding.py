@@ -42,6 +42,7 @@ SIGNATURES = {
     "fp4_dequant_mse": (_i, [_vp, _vp, _i64, _i64, _i, _i, _vp, _i, _vp, _vp, _i, _vp, _vp, _vp]),
     "w4a4_gemm": (_i, [_vp, _i, _i, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _sz, _vp]),
     "fp4q_gemm_status": (_i, [_vp, _vp]),
+    "fp4q_sync_status": (_i, [_vp, _vp]),
     "razer_gemm_prepare": (_i, [_vp, _vp, _i64, _i64, _i, _vp, _i, _vp, _vp, _vp, _vp]),
     "razer_w4a4_gemm": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _sz, _vp]),
     "fp4_scales_to_mma": (_i, [_vp, _i64, _i64, _vp, _vp]),

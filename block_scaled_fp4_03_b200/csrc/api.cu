@@ -382,6 +382,11 @@ int fp4q_gemm_status(const void* workspace, void* stream)
     return flag ? FP4Q_ERR_TIMEOUT : FP4Q_OK;
 }
 
+int fp4q_sync_status(const void* workspace, void* stream)
+{
+    return fp4q_gemm_status(workspace, stream);
+}
+
 // E2M1 codes (p, q) with value(p) + value(q) == v exactly: p the largest
 // magnitude of the special's sign that leaves an E2M1 remainder.  False when
 // no such pair exists.

@@ -428,6 +428,13 @@ FP4Q_API int mxfp4_gemm(const void* a, int a_format, const uint8_t* a_scales, co
  */
 FP4Q_API int fp4q_gemm_status(const void* workspace, void* stream);
 
+/*
+ * The same report for any call that takes a GEMM workspace (w4a4_gemm,
+ * razer_w4a4_gemm, mxfp4_gemm): synchronizes `stream`, then FP4Q_OK or
+ * FP4Q_ERR_TIMEOUT.  Same semantics as fp4q_gemm_status.
+ */
+FP4Q_API int fp4q_sync_status(const void* workspace, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

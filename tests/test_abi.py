@@ -175,3 +175,8 @@ def test_header_is_plain_c(tmp_path):
     r = subprocess.run([cc, "-std=c99", "-Wall", "-Werror", "-pedantic", "-fsyntax-only",
                         "-I", os.path.join(ROOT, "include"), str(src)], capture_output=True, text=True)
     assert r.returncode == 0, r.stderr
+
+
+def test_status_calls_reject_a_missing_workspace(L):
+    assert L.fp4q_gemm_status(None, None) == 1
+    assert L.fp4q_sync_status(None, None) == 1
