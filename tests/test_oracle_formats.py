@@ -10,7 +10,6 @@ from fractions import Fraction
 
 import ml_dtypes as md
 import numpy as np
-import pytest
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "page_facts.json")
 

@@ -9,7 +9,6 @@ rms from the Hessian diagonal).
 """
 import ml_dtypes as md
 import numpy as np
-import pytest
 
 from block_scaled_fp4_03_b200 import inputs
 
