@@ -5,10 +5,16 @@ arch=compute_100a,code=sm_100a), with -fmad=false so that no fp32 multiply-add
 is contracted behind the explicit round-to-nearest intrinsics, and links a
 shared object with the CUDA runtime statically (the stream handles passed in
 are driver-level and shared with PyTorch's runtime).
+
+A build is reused only when the SHA-256 of every source, header, this script
+and the compiler flags equals the one recorded beside the library when it was
+built (file times are not trusted: a copied tree can carry a stale library
+with a fresh time stamp).
 """
 from __future__ import annotations
 
 import concurrent.futures as cf
+import hashlib
 import os
 import shutil
 import subprocess
@@ -19,6 +25,7 @@ CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libfp4q.so")
+STAMP = os.path.join(BUILD, "libfp4q.sha256")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-fmad=false", "-Xcompiler", "-fPIC",
@@ -46,11 +53,22 @@ def _deps() -> list[str]:
     return out
 
 
+def source_digest() -> str:
+    """SHA-256 over the flags and the name and bytes of every input of the build."""
+    h = hashlib.sha256()
+    h.update(" ".join(ARCH + NVCC_FLAGS[:-4]).encode())
+    for p in sorted(_deps()) + [os.path.abspath(__file__)]:
+        h.update(os.path.basename(p).encode())
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+    if not (os.path.exists(LIB) and os.path.exists(STAMP)):
         return False
-    t = os.path.getmtime(LIB)
-    return all(os.path.getmtime(p) <= t for p in _deps() + [os.path.abspath(__file__)])
+    with open(STAMP) as f:
+        return f.read().strip() == source_digest()
 
 
 def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) -> str:
@@ -78,6 +96,8 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
     if r.returncode != 0:
         raise RuntimeError("link failed:\n%s%s" % (r.stdout, r.stderr))
     os.replace(tmp, LIB)
+    with open(STAMP, "w") as f:
+        f.write(source_digest() + "\n")
     return LIB
 
 
