@@ -40,13 +40,14 @@ SIGNATURES = {
     "fp4_hessian_blocks_noalloc": (_i, [_vp, _i, _i64, _i64, _vp, _i, _vp, _vp]),
     "mxfp4_channel_scale": (_i, [_vp, _i, _i64, _vp, _i, _i64, _i64, _fp, _vp, _vp, _vp, _sz, _vp]),
     "fp4_dequant_mse": (_i, [_vp, _vp, _i64, _i64, _i, _i, _vp, _i, _vp, _vp, _i, _vp, _vp, _vp]),
-    "w4a4_gemm": (_i, [_vp, _i, _i, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _sz, _vp]),
+    "w4a4_gemm": (_i, [_vp, _i, _i, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _i, _vp, _sz, _vp]),
     "fp4q_gemm_status": (_i, [_vp, _vp]),
-    "fp4q_sync_status": (_i, [_vp, _vp]),
+    "fp4q_hessian_status": (_i, [_vp, _vp]),
+    "fp4q_debug_set_wait_cycles": (_i64, [_i64]),
     "razer_gemm_prepare": (_i, [_vp, _vp, _i64, _i64, _i, _vp, _i, _vp, _vp, _vp, _vp]),
-    "razer_w4a4_gemm": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _sz, _vp]),
+    "razer_w4a4_gemm": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _i, _vp, _sz, _vp]),
     "fp4_scales_to_mma": (_i, [_vp, _i64, _i64, _vp, _vp]),
-    "mxfp4_gemm": (_i, [_vp, _i, _vp, _vp, _i, _vp, _vp, _i64, _i64, _i64, _vp, _vp, _sz, _vp]),
+    "mxfp4_gemm": (_i, [_vp, _i, _vp, _vp, _i, _vp, _vp, _i64, _i64, _i64, _vp, _i, _vp, _sz, _vp]),
 }
 
 _lock = threading.Lock()
@@ -100,6 +101,14 @@ def _dtype_code(t: torch.Tensor) -> int:
     if t.dtype == torch.bfloat16:
         return BF16
     raise TypeError("fp4q takes float32 or bfloat16 tensors, got %s" % t.dtype)
+
+
+def _out_tensor(out, M, N, out_dtype, device):
+    """The GEMM output tensor and its fp4q dtype code (bf16 unless fp32 is asked for)."""
+    if out is not None:
+        return out, _dtype_code(out)
+    dt = torch.float32 if out_dtype == F32 else torch.bfloat16
+    return torch.empty((M, N), dtype=dt, device=device), (F32 if out_dtype == F32 else BF16)
 
 
 def _need_cuda(*ts):
@@ -271,10 +280,11 @@ def dequant_mse(codes: torch.Tensor, scales: torch.Tensor, rows: int, cols: int,
 def w4a4_gemm(a: torch.Tensor, w_codes: torch.Tensor, w_scales: torch.Tensor, w_global_scale: torch.Tensor,
               a_scales: torch.Tensor | None = None, a_global_scale: torch.Tensor | None = None,
               a_rule: int = FOUR_OVER_SIX, K: int | None = None, out: torch.Tensor | None = None,
-              workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
-    """out = A . W^T in bf16.  `a` is either a dense fp32/bf16 [M, K] tensor (quantized on the
-    fly with `a_rule`) or packed NVFP4 codes [M, K/2] uint8 with `a_scales` (MMA layout) and
-    `a_global_scale`.  W is packed codes [N, K/2] with MMA-layout scales."""
+              workspace: torch.Tensor | None = None, stream=None, out_dtype: int = BF16) -> torch.Tensor:
+    """out = A . W^T in bf16 (or fp32 with out_dtype=F32, or an fp32 `out`).  `a` is either a
+    dense fp32/bf16 [M, K] tensor (quantized on the fly with `a_rule`) or packed NVFP4 codes
+    [M, K/2] uint8 with `a_scales` (MMA layout) and `a_global_scale`.  W is packed codes
+    [N, K/2] with MMA-layout scales."""
     _need_cuda(a, w_codes, w_scales, w_global_scale, a_scales, a_global_scale)
     if a.dtype == torch.uint8:
         fmt = NVFP4_PACKED
@@ -285,10 +295,10 @@ def w4a4_gemm(a: torch.Tensor, w_codes: torch.Tensor, w_scales: torch.Tensor, w_
         M, K = a.shape
     N = w_codes.shape[0]
     dev = a.device
-    o = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    o, odt = _out_tensor(out, M, N, out_dtype, dev)
     ws, wsb = (workspace, workspace.numel()) if workspace is not None else _workspace(OP_GEMM, M, K, N, dev, None)
     st = lib().w4a4_gemm(_ptr(a), fmt, a_rule, _ptr(a_scales), _ptr(a_global_scale), _ptr(w_codes),
-                         _ptr(w_scales), _ptr(w_global_scale), M, N, K, _ptr(o), _ptr(ws), wsb,
+                         _ptr(w_scales), _ptr(w_global_scale), M, N, K, _ptr(o), odt, _ptr(ws), wsb,
                          _stream(stream))
     _check(st, "w4a4_gemm")
     return o
@@ -317,18 +327,18 @@ def razer_w4a4_gemm(a_codes: torch.Tensor, a_scales: torch.Tensor, a_global_scal
                     w_codes: torch.Tensor, w_scales: torch.Tensor, w_global_scale: torch.Tensor,
                     a_extra: torch.Tensor | None = None, w_extra: torch.Tensor | None = None,
                     out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
-                    stream=None) -> torch.Tensor:
+                    stream=None, out_dtype: int = BF16) -> torch.Tensor:
     """out = bf16(g_a g_w (A + A_extra) . (W + W_extra)^T): each operand a packed code tensor
     plus an optional extra code tensor sharing its MMA-layout E4M3 scales."""
     _need_cuda(a_codes, a_scales, a_global_scale, w_codes, w_scales, w_global_scale, a_extra, w_extra)
     M, K = a_codes.shape[0], a_codes.shape[1] * 2
     N = w_codes.shape[0]
     dev = a_codes.device
-    o = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    o, odt = _out_tensor(out, M, N, out_dtype, dev)
     ws = workspace if workspace is not None else torch.empty(8192, dtype=torch.uint8, device=dev)
     st = lib().razer_w4a4_gemm(_ptr(a_codes), _ptr(a_extra), _ptr(a_scales), _ptr(a_global_scale),
                                _ptr(w_codes), _ptr(w_extra), _ptr(w_scales), _ptr(w_global_scale),
-                               M, N, K, _ptr(o), _ptr(ws), ws.numel(), _stream(stream))
+                               M, N, K, _ptr(o), odt, _ptr(ws), ws.numel(), _stream(stream))
     _check(st, "razer_w4a4_gemm")
     return o
 
@@ -345,7 +355,7 @@ def scales_to_mma(scales: torch.Tensor, out: torch.Tensor | None = None, stream=
 def mxfp4_gemm(a: torch.Tensor, w_codes: torch.Tensor, w_scales: torch.Tensor,
                a_scales: torch.Tensor | None = None, chan_scale: torch.Tensor | None = None,
                hadamard: bool = True, K: int | None = None, out: torch.Tensor | None = None,
-               workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+               workspace: torch.Tensor | None = None, stream=None, out_dtype: int = BF16) -> torch.Tensor:
     """out = A' . W'^T in bf16 with MXFP4 operands.  `a` is a dense fp32/bf16 [M, K] tensor
     (transformed with chan_scale and the 32-block rotation and quantized in the call) or packed
     MXFP4 codes [M, K/2] uint8 with `a_scales` (E8M0, MMA layout).  W: codes [N, K/2] with
@@ -360,13 +370,13 @@ def mxfp4_gemm(a: torch.Tensor, w_codes: torch.Tensor, w_scales: torch.Tensor,
         M, K = a.shape
     N = w_codes.shape[0]
     dev = a.device
-    o = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    o, odt = _out_tensor(out, M, N, out_dtype, dev)
     ws, wsb = (workspace, workspace.numel()) if workspace is not None else _workspace(OP_MX_GEMM, M, K, N, dev, None)
     if fmt == MXFP4_PACKED and ws is None:
         ws = torch.empty(8192, dtype=torch.uint8, device=dev)
         wsb = ws.numel()
     st = lib().mxfp4_gemm(_ptr(a), fmt, _ptr(a_scales), _ptr(chan_scale), int(bool(hadamard)), _ptr(w_codes),
-                          _ptr(w_scales), M, N, K, _ptr(o), _ptr(ws), wsb, _stream(stream))
+                          _ptr(w_scales), M, N, K, _ptr(o), odt, _ptr(ws), wsb, _stream(stream))
     _check(st, "mxfp4_gemm")
     return o
 
@@ -374,3 +384,15 @@ def mxfp4_gemm(a: torch.Tensor, w_codes: torch.Tensor, w_scales: torch.Tensor,
 def gemm_status(workspace: torch.Tensor, stream=None) -> int:
     """Synchronize and return the device-side status word of the last GEMM on `workspace`."""
     return int(lib().fp4q_gemm_status(_ptr(workspace), _stream(stream)))
+
+
+def hessian_status(workspace: torch.Tensor | None, stream=None) -> int:
+    """Synchronize and return the status of the last fp4_hessian_blocks call on `workspace`
+    (None: the last fp4_hessian_blocks_noalloc call on the current device)."""
+    return int(lib().fp4q_hessian_status(_ptr(workspace), _stream(stream)))
+
+
+def debug_set_wait_cycles(cycles: int) -> int:
+    """Process-wide limit of the tensor-core kernels' bounded waits (0: the default);
+    returns the previous setting.  For tests of the timeout path."""
+    return int(lib().fp4q_debug_set_wait_cycles(int(cycles)))

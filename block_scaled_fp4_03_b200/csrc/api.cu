@@ -29,6 +29,9 @@ constexpr int kFlipMaxMoves = 1 << 20;
 constexpr size_t kGemmHeader = 8192;
 constexpr size_t kGemmGa = 4096;
 constexpr size_t kGemmErr = 4160;
+// Hessian workspace: [0, 256) header (error word at 0), then the partial sums.
+constexpr size_t kHessHeader = 256;
+bool valid_out_dtype(int d) { return d == FP4Q_BF16 || d == FP4Q_F32; }
 size_t gemm_ws_bytes(int64_t M, int64_t K) { return kGemmHeader + (size_t)M * (size_t)K / 2 + (size_t)M * (size_t)K / 16; }
 size_t mx_gemm_ws_bytes(int64_t M, int64_t K) { return kGemmHeader + (size_t)M * (size_t)K / 2 + (size_t)M * (size_t)K / 32; }
 static_assert(kAmaxPartials * sizeof(float) <= FP4Q_WS_BF_EVALS && FP4Q_WS_BF_EVALS + 8 <= kQuantWs,
@@ -73,7 +76,7 @@ size_t fp4q_workspace_size(int op, int64_t rows, int64_t cols, int64_t n)
     switch (op) {
     case FP4Q_OP_QUANTIZE: return kQuantWs;
     case FP4Q_OP_FLIP: return (rows <= 0 || cols <= 0 || cols % 32) ? 0 : flip_refine_ws_bytes(rows, cols);
-    case FP4Q_OP_HESSIAN: return cols % 32 ? 0 : hessian_ws_bytes(rows, cols);
+    case FP4Q_OP_HESSIAN: return cols % 32 ? 0 : kHessHeader + hessian_ws_bytes(rows, cols);
     case FP4Q_OP_CHANNEL_SCALE: return channel_scale_ws_bytes(rows, n, cols);
     case FP4Q_OP_GEMM: return gemm_ws_bytes(rows, cols);
     case FP4Q_OP_MX_GEMM: return mx_gemm_ws_bytes(rows, cols);
@@ -249,16 +252,20 @@ int fp4_hessian_blocks(const void* x, int dtype, int64_t rows, int64_t cols,
         return FP4Q_ERR_ALIGN;
     if (cols == 0)
         return FP4Q_OK;
-    const size_t need = hessian_ws_bytes(rows, cols);
-    if (need > 0 && (!workspace || workspace_bytes < need))
+    const size_t need = kHessHeader + hessian_ws_bytes(rows, cols);
+    if (!workspace || workspace_bytes < need)
         return FP4Q_ERR_WORKSPACE;
-    if (!aligned_or_null(workspace))
+    if (!aligned16(workspace))
         return FP4Q_ERR_ALIGN;
+    cudaStream_t s = as_stream(stream);
+    int* err = static_cast<int*>(workspace);
+    if (cudaMemsetAsync(err, 0, sizeof(int), s) != cudaSuccess)
+        return FP4Q_ERR_CUDA;
     if (rows == 0)
-        return from_cuda(cudaMemsetAsync(hess_blocks, 0, (size_t)(cols / 32) * 1024 * sizeof(float),
-                                         as_stream(stream)));
+        return from_cuda(cudaMemsetAsync(hess_blocks, 0, (size_t)(cols / 32) * 1024 * sizeof(float), s));
+    float* part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kHessHeader);
     return from_cuda(launch_hessian_blocks(x, dtype, rows, cols, chan_scale, hadamard32 != 0,
-                                           hess_blocks, workspace, as_stream(stream)));
+                                           hess_blocks, part, err, s));
 }
 
 int mxfp4_channel_scale(const void* x, int x_dtype, int64_t tokens, const void* w,
@@ -316,9 +323,9 @@ int fp4_dequant_mse(const uint8_t* codes, const uint8_t* scales, int64_t rows, i
 int w4a4_gemm(const void* a, int a_format, int a_rule, const uint8_t* a_scales,
               const float* a_global_scale, const uint8_t* w_codes, const uint8_t* w_scales,
               const float* w_global_scale, int64_t M, int64_t N, int64_t K, void* out,
-              void* workspace, size_t workspace_bytes, void* stream)
+              int out_dtype, void* workspace, size_t workspace_bytes, void* stream)
 {
-    if (!a || !w_codes || !w_scales || !w_global_scale || !out || !workspace)
+    if (!a || !w_codes || !w_scales || !w_global_scale || !out || !workspace || !valid_out_dtype(out_dtype))
         return FP4Q_ERR_ARG;
     if (a_format != FP4Q_F32 && a_format != FP4Q_BF16 && a_format != FP4Q_NVFP4_PACKED)
         return FP4Q_ERR_ARG;
@@ -366,7 +373,7 @@ int w4a4_gemm(const void* a, int a_format, int a_rule, const uint8_t* a_scales,
         ga = g;
     }
     return from_cuda(launch_w4a4_gemm(a_codes, a_sf, ga, w_codes, w_scales, w_global_scale, M, N, K,
-                                      out, err, s));
+                                      out, out_dtype == FP4Q_F32, err, s));
 }
 
 int fp4q_gemm_status(const void* workspace, void* stream)
@@ -382,9 +389,18 @@ int fp4q_gemm_status(const void* workspace, void* stream)
     return flag ? FP4Q_ERR_TIMEOUT : FP4Q_OK;
 }
 
-int fp4q_sync_status(const void* workspace, void* stream)
+int fp4q_hessian_status(const void* workspace, void* stream)
 {
-    return fp4q_gemm_status(workspace, stream);
+    // NULL: the error word of fp4_hessian_blocks_noalloc on the current device
+    const void* word = workspace ? workspace : noalloc_hessian_error_word();
+    if (!word)
+        return FP4Q_ERR_CUDA;
+    int flag = 0;
+    cudaStream_t s = as_stream(stream);
+    if (cudaMemcpyAsync(&flag, word, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+        return FP4Q_ERR_CUDA;
+    return flag ? FP4Q_ERR_TIMEOUT : FP4Q_OK;
 }
 
 // E2M1 codes (p, q) with value(p) + value(q) == v exactly: p the largest
@@ -450,10 +466,10 @@ int razer_gemm_prepare(const uint8_t* codes, const uint8_t* meta, int64_t rows, 
 int razer_w4a4_gemm(const uint8_t* a_codes, const uint8_t* a_extra, const uint8_t* a_scales,
                     const float* a_global_scale, const uint8_t* w_codes, const uint8_t* w_extra,
                     const uint8_t* w_scales, const float* w_global_scale, int64_t M, int64_t N,
-                    int64_t K, void* out, void* workspace, size_t workspace_bytes, void* stream)
+                    int64_t K, void* out, int out_dtype, void* workspace, size_t workspace_bytes, void* stream)
 {
     if (!a_codes || !a_scales || !a_global_scale || !w_codes || !w_scales || !w_global_scale || !out ||
-        !workspace)
+        !workspace || !valid_out_dtype(out_dtype))
         return FP4Q_ERR_ARG;
     if (M <= 0 || N <= 0 || K <= 0)
         return FP4Q_ERR_ARG;
@@ -470,7 +486,7 @@ int razer_w4a4_gemm(const uint8_t* a_codes, const uint8_t* a_extra, const uint8_
     if (cudaMemsetAsync(err, 0, sizeof(int), s) != cudaSuccess)
         return FP4Q_ERR_CUDA;
     return from_cuda(launch_w4a4_gemm(a_codes, a_scales, a_global_scale, w_codes, w_scales, w_global_scale,
-                                      M, N, K, out, err, s, a_extra, w_extra));
+                                      M, N, K, out, out_dtype == FP4Q_F32, err, s, a_extra, w_extra));
 }
 
 int fp4_scales_to_mma(const uint8_t* scales, int64_t rows, int64_t nscales, uint8_t* out, void* stream)
@@ -488,9 +504,9 @@ int fp4_scales_to_mma(const uint8_t* scales, int64_t rows, int64_t nscales, uint
 
 int mxfp4_gemm(const void* a, int a_format, const uint8_t* a_scales, const float* chan_scale,
                int hadamard32, const uint8_t* w_codes, const uint8_t* w_scales, int64_t M, int64_t N,
-               int64_t K, void* out, void* workspace, size_t workspace_bytes, void* stream)
+               int64_t K, void* out, int out_dtype, void* workspace, size_t workspace_bytes, void* stream)
 {
-    if (!a || !w_codes || !w_scales || !out || !workspace)
+    if (!a || !w_codes || !w_scales || !out || !workspace || !valid_out_dtype(out_dtype))
         return FP4Q_ERR_ARG;
     if (a_format != FP4Q_F32 && a_format != FP4Q_BF16 && a_format != FP4Q_MXFP4_PACKED)
         return FP4Q_ERR_ARG;
@@ -524,8 +540,8 @@ int mxfp4_gemm(const void* a, int a_format, const uint8_t* a_scales, const float
         a_codes = qcodes;
         a_sf = qsf;
     }
-    return from_cuda(launch_w4a4_gemm(a_codes, a_sf, nullptr, w_codes, w_scales, nullptr, M, N, K, out, err, s,
-                                      nullptr, nullptr, 1));
+    return from_cuda(launch_w4a4_gemm(a_codes, a_sf, nullptr, w_codes, w_scales, nullptr, M, N, K, out,
+                                      out_dtype == FP4Q_F32, err, s, nullptr, nullptr, 1));
 }
 
 }  // extern "C"

@@ -8,6 +8,14 @@
 
 namespace fp4q {
 
+// Default limit of the bounded device-side waits (SM clock cycles, about 2 s
+// at the boost clock).
+constexpr long long kDefaultWaitCycles = 4000000000LL;
+
+// The limit the next launch gives its main-loop waits: the process-wide
+// setting of fp4q_debug_set_wait_cycles, or kDefaultWaitCycles.
+long long wait_limit_cycles();
+
 // Global-scale source for a quantizer launch.
 struct GsArgs {
     int mode;                 // 0 none (g = 1), 1 amax partials in ws, 2 given (device float)
@@ -51,9 +59,11 @@ cudaError_t launch_mx_channel_scale(const void* x, int xdt, int64_t tokens, cons
                                     int64_t n_out, int64_t cols, float alpha, float* t,
                                     float* t_inv, void* ws, cudaStream_t s);
 
+// part: the partial-sum area (hessian_ws_bytes(rows, cols) bytes); err: a
+// device int set to 1 when a bounded wait gave up (the caller clears it)
 cudaError_t launch_hessian_blocks(const void* x, int dtype, int64_t rows, int64_t cols,
-                                  const float* chan_scale, int hadamard, float* hess, void* ws,
-                                  cudaStream_t s);
+                                  const float* chan_scale, int hadamard, float* hess, float* part,
+                                  int* err, cudaStream_t s);
 
 // mma_layout: scales in the MMA scale layout (rows % 128 == 0, cols % 128 == 0)
 cudaError_t launch_mxfp4_quant(const void* x, int dtype, int64_t rows, int64_t cols,
@@ -76,9 +86,10 @@ bool gemm_shape_supported(int64_t M, int64_t N, int64_t K);
 // out = (A + A1) . (W + W1)^T, as extra passes over K into one accumulator.
 // mx: MXFP4 operands (E8M0 scales per 32 elements in the MMA layout; ga, gw
 // NULL = no global scale).
+// out_f32: fp32 output instead of bf16 (same layout, M x N row-major).
 cudaError_t launch_w4a4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* ga,
                              const uint8_t* w_codes, const uint8_t* w_sf, const float* gw, int64_t M,
-                             int64_t N, int64_t K, void* out, int* err, cudaStream_t s,
+                             int64_t N, int64_t K, void* out, int out_f32, int* err, cudaStream_t s,
                              const uint8_t* a1_codes = nullptr, const uint8_t* w1_codes = nullptr,
                              int mx = 0);
 
@@ -94,6 +105,10 @@ cudaError_t launch_razer_gemm_prepare(const uint8_t* codes, const uint8_t* meta,
                                       int64_t cols, int sf, const uint8_t* p_code,
                                       const uint8_t* q_code, uint8_t* main_codes,
                                       uint8_t* extra_codes, uint8_t* scales_mma, cudaStream_t s);
+
+// Device address of fp4_hessian_blocks_noalloc's error word on the current
+// device (NULL if it cannot be looked up).
+const int* noalloc_hessian_error_word();
 
 // Workspace (bytes) launch_hessian_blocks / launch_mx_channel_scale need.
 size_t hessian_ws_bytes(int64_t rows, int64_t cols);

@@ -119,19 +119,33 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
     return ok != 0;
 }
 
+__device__ __forceinline__ bool mbar_test_wait_cluster(uint32_t bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok)
+                 : "r"(bar), "r"(parity)
+                 : "memory");
+    return ok != 0;
+}
+
 // Bounded wait with cluster-scope acquire, for barriers that other CTAs arrive
 // on; gives up after `limit` cycles or when the abort flag (if any) is raised.
+// A short (test) limit makes the first probe non-blocking, as in mbar_wait.
 __device__ __noinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, const volatile int* abort_flag,
                                                long long limit = kTcWaitCycles)
 {
-    if (mbar_try_wait_cluster(bar, parity))
+    if (limit >= kShortWaitCycles ? mbar_try_wait_cluster(bar, parity) : mbar_test_wait_cluster(bar, parity))
         return true;
     const long long t0 = clock64();
-    while (!mbar_try_wait_cluster(bar, parity)) {
+    for (;;) {
         if ((abort_flag && *abort_flag) || clock64() - t0 > limit)
             return false;
+        if (mbar_try_wait_cluster(bar, parity))
+            return true;
     }
-    return true;
 }
 
 // ---------------------------------------------------------------- copies
@@ -226,8 +240,9 @@ struct GemmParams {
     const uint8_t* sfb;       // W scales, MMA layout
     const float* ga;          // A global scale (device)
     const float* gw;          // W global scale (device)
-    __nv_bfloat16* out;       // M x N row-major
+    void* out;                // M x N row-major, bf16 (or fp32 when the kernel's OUTF32 is set)
     int* err;                 // error word (workspace)
+    long long wait_limit;     // cycles after which a main-loop wait gives up
     int tiles_m, tiles_n, kblocks, kb_atoms, N;
     // Passes: the K loop runs kiters = kblocks << pass_shift steps; step j
     // covers K block j >> pass_shift with operand pair (pass_sel >> 2*(j %
@@ -243,7 +258,7 @@ __device__ __forceinline__ int pass_operands(const GemmParams& p, int j)
     return (p.pass_sel >> (2 * (j & ((1 << p.pass_shift) - 1)))) & 3;
 }
 
-template <bool MX>
+template <bool MX, bool OUTF32>
 __global__ void __launch_bounds__(kThreads, 1)
 w4a4_gemm_1sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
@@ -304,7 +319,7 @@ w4a4_gemm_1sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                 const int mt = tile % p.tiles_m;
                 const int nt = tile / p.tiles_m;
                 for (int j = 0; j < p.kiters; ++j) {
-                    if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag) || *abort_flag) {
+                    if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, p.wait_limit) || *abort_flag) {
                         give_up();
                         break;
                     }
@@ -342,14 +357,14 @@ w4a4_gemm_1sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
             uint32_t phase = 0, acc_phase = 0;
             bool issued_any = false;
             for (int tile = blockIdx.x; tile < num_tiles && !*abort_flag; tile += gridDim.x) {
-                if (!mbar_wait(acc_empty, acc_phase ^ 1u, abort_flag) || *abort_flag) {
+                if (!mbar_wait(acc_empty, acc_phase ^ 1u, abort_flag, p.wait_limit) || *abort_flag) {
                     give_up();
                     break;
                 }
                 tc_fence_after();
                 bool ok = true;
                 for (int kb = 0; kb < p.kiters; ++kb) {
-                    if (!mbar_wait(full_bar(stage), phase, abort_flag) || *abort_flag) {
+                    if (!mbar_wait(full_bar(stage), phase, abort_flag, p.wait_limit) || *abort_flag) {
                         give_up();
                         ok = false;
                         break;
@@ -401,7 +416,7 @@ w4a4_gemm_1sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
         uint32_t acc_phase = 0;
         const float scale = p.ga ? __fmul_rn(__ldg(p.ga), __ldg(p.gw)) : 1.0f;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-            bool ok = !*abort_flag && mbar_wait(acc_full, acc_phase, abort_flag);
+            bool ok = !*abort_flag && mbar_wait(acc_full, acc_phase, abort_flag, p.wait_limit);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) {
                 if (lane == 0)
@@ -412,23 +427,33 @@ w4a4_gemm_1sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
             const int mt = tile % p.tiles_m;
             const int nt = tile / p.tiles_m;
             const int64_t row = (int64_t)mt * kBM + q * 32 + lane;
-            __nv_bfloat16* orow = p.out + row * p.N + (int64_t)nt * kBN;
+            const int64_t orow_off = row * p.N + (int64_t)nt * kBN;
             const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16);
 #pragma unroll 1
             for (int c = 0; c < kBN / 32; ++c) {
                 uint32_t r[32];
                 tmem_ld32(tq + 32 * c, r);
-                uint32_t pk[16];
+                if constexpr (OUTF32) {
+                    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.out) + orow_off + 32 * c);
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[2 * j]), scale),
-                                                             __fmul_rn(__uint_as_float(r[2 * j + 1]), scale));
-                    pk[j] = *reinterpret_cast<uint32_t*>(&h);
+                    for (int j = 0; j < 8; ++j)
+                        dst[j] = make_float4(__fmul_rn(__uint_as_float(r[4 * j]), scale),
+                                             __fmul_rn(__uint_as_float(r[4 * j + 1]), scale),
+                                             __fmul_rn(__uint_as_float(r[4 * j + 2]), scale),
+                                             __fmul_rn(__uint_as_float(r[4 * j + 3]), scale));
+                } else {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        __nv_bfloat162 h = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[2 * j]), scale),
+                                                                 __fmul_rn(__uint_as_float(r[2 * j + 1]), scale));
+                        pk[j] = *reinterpret_cast<uint32_t*>(&h);
+                    }
+                    uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.out) + orow_off + 32 * c);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
                 }
-                uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    dst[j] = make_uint4(pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
             }
             tc_fence_before();
             mbar_arrive(acc_empty);
@@ -556,7 +581,7 @@ __device__ __forceinline__ void stage_row_chunk(uint8_t* stg, int c, int lane, c
     }
 }
 
-template <bool MX>
+template <bool MX, bool OUTF32>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(k2Threads, 1)
 w4a4_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmSA, const __grid_constant__ CUtensorMap tmSB,
@@ -636,7 +661,7 @@ w4a4_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                 const int mt = tile % p.tiles_m;
                 const int nt = tile / p.tiles_m;
                 for (int j = 0; j < p.kiters; ++j) {
-                    if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag) || *abort_flag) {
+                    if (!mbar_wait(empty_bar(stage), phase ^ 1u, abort_flag, p.wait_limit) || *abort_flag) {
                         give_up();
                         break;
                     }
@@ -686,7 +711,7 @@ w4a4_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
             uint32_t phase = 0, acc_phase = 0;
             bool issued_any = false;
             for (int tile = cluster; tile < num_tiles && !*abort_flag; tile += nclusters) {
-                if (!mbar_wait_cluster(acc_empty, acc_phase ^ 1u, abort_flag) || *abort_flag) {
+                if (!mbar_wait_cluster(acc_empty, acc_phase ^ 1u, abort_flag, p.wait_limit) || *abort_flag) {
                     give_up();
                     break;
                 }
@@ -696,7 +721,7 @@ w4a4_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                     // the scale warps observed the stage's full barrier (cluster
                     // acquire) before their copies; their commits complete this
                     // barrier only after the copies, so the stage is in place
-                    if (!mbar_wait(sf_ready_bar(stage), phase, abort_flag) || *abort_flag) {
+                    if (!mbar_wait(sf_ready_bar(stage), phase, abort_flag, p.wait_limit) || *abort_flag) {
                         give_up();
                         ok = false;
                         break;
@@ -748,7 +773,7 @@ w4a4_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
             for (int tile = cluster; tile < num_tiles && !*abort_flag; tile += nclusters) {
                 bool ok = true;
                 for (int kb = 0; kb < p.kiters; ++kb) {
-                    if (!mbar_wait_cluster(full_bar(stage), phase, abort_flag) || *abort_flag) {
+                    if (!mbar_wait_cluster(full_bar(stage), phase, abort_flag, p.wait_limit) || *abort_flag) {
                         give_up();
                         ok = false;
                         break;
@@ -785,7 +810,7 @@ w4a4_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
         uint32_t acc_phase = 0;
         const float scale = p.ga ? __fmul_rn(__ldg(p.ga), __ldg(p.gw)) : 1.0f;
         for (int tile = cluster; tile < num_tiles; tile += nclusters) {
-            bool ok = !*abort_flag && mbar_wait(acc_full, acc_phase, abort_flag);
+            bool ok = !*abort_flag && mbar_wait(acc_full, acc_phase, abort_flag, p.wait_limit);
             ok = __all_sync(0xffffffffu, ok);
             if (!ok) {
                 if (lane == 0)
@@ -796,6 +821,27 @@ w4a4_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
             const int mt = tile % p.tiles_m;
             const int nt = tile / p.tiles_m;
             const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16);
+            if constexpr (OUTF32) {
+                // fp32 output: each lane writes its own accumulator row directly
+                float* orow = static_cast<float*>(p.out) +
+                              (int64_t)(mt * 256 + (int)rank * 128 + q * 32 + lane) * p.N + (int64_t)nt * 256;
+#pragma unroll 1
+                for (int c2 = 0; c2 < 4; ++c2) {
+                    uint32_t r[64];
+                    tmem_ld64(tq + 64 * c2, r);
+                    float4* dst = reinterpret_cast<float4*>(orow + 64 * c2);
+#pragma unroll
+                    for (int j = 0; j < 16; ++j)
+                        dst[j] = make_float4(__fmul_rn(__uint_as_float(r[4 * j]), scale),
+                                             __fmul_rn(__uint_as_float(r[4 * j + 1]), scale),
+                                             __fmul_rn(__uint_as_float(r[4 * j + 2]), scale),
+                                             __fmul_rn(__uint_as_float(r[4 * j + 3]), scale));
+                }
+                tc_fence_before();
+                mbar_arrive_cluster(leader_acc_empty);
+                acc_phase ^= 1u;
+                continue;
+            }
             // the previous tile's stores have finished reading the staging buffer
             if (lane == 0)
                 asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
@@ -946,27 +992,27 @@ bool gemm_shape_supported(int64_t M, int64_t N, int64_t K)
            N / kBN < (1 << 20);
 }
 
-template <bool MX>
+template <bool MX, bool OUTF32>
 cudaError_t launch_gemm_t(const uint8_t* a_codes, const uint8_t* a_sf, const uint8_t* w_codes,
                           const uint8_t* w_sf, const uint8_t* a1, const uint8_t* w1, int64_t M, int64_t N,
                           int64_t K, void* out, GemmParams& p, cudaStream_t s)
 {
     if (M % 256 == 0) {
         // CTA pairs: 256 x 256 tiles
-        CUtensorMap ta, tb, tsa, tsb, to, ta1, tb1;
+        CUtensorMap ta, tb, tsa, tsb, to{}, ta1, tb1;
         if (!make_code_map(&ta, a_codes, M, K / 2, 128) || !make_code_map(&tb, w_codes, N, K / 2, 128) ||
             !make_sf_map(&tsa, a_sf, M, K, 1, MX) || !make_sf_map(&tsb, w_sf, N, K, 2, MX) ||
-            !make_out_map(&to, out, M, N) || !make_code_map(&ta1, a1, M, K / 2, 128) ||
+            (!OUTF32 && !make_out_map(&to, out, M, N)) || !make_code_map(&ta1, a1, M, K / 2, 128) ||
             !make_code_map(&tb1, w1, N, K / 2, 128))
             return cudaErrorInvalidValue;
-        const cudaError_t attr2_err = smem_opt_in((const void*)w4a4_gemm_2sm_kernel<MX>, k2SmemBytes);
+        const cudaError_t attr2_err = smem_opt_in((const void*)w4a4_gemm_2sm_kernel<MX, OUTF32>, k2SmemBytes);
         if (attr2_err != cudaSuccess)
             return attr2_err;
         p.tiles_m = (int)(M / 256);
         const int tiles = p.tiles_m * p.tiles_n;
         const int pairs = num_sms() / 2;
         const int grid = 2 * (tiles < pairs ? tiles : pairs);
-        w4a4_gemm_2sm_kernel<MX><<<grid, k2Threads, k2SmemBytes, s>>>(ta, tb, tsa, tsb, to, ta1, tb1, p);
+        w4a4_gemm_2sm_kernel<MX, OUTF32><<<grid, k2Threads, k2SmemBytes, s>>>(ta, tb, tsa, tsb, to, ta1, tb1, p);
         return cudaGetLastError();
     }
     CUtensorMap ta, tb, tsa, tsb, ta1, tb1;
@@ -974,19 +1020,19 @@ cudaError_t launch_gemm_t(const uint8_t* a_codes, const uint8_t* a_sf, const uin
         !make_sf_map(&tsa, a_sf, M, K, 1, MX) || !make_sf_map(&tsb, w_sf, N, K, 2, MX) ||
         !make_code_map(&ta1, a1, M, K / 2, kBM) || !make_code_map(&tb1, w1, N, K / 2, kBN))
         return cudaErrorInvalidValue;
-    const cudaError_t attr_err = smem_opt_in((const void*)w4a4_gemm_1sm_kernel<MX>, kSmemBytes);
+    const cudaError_t attr_err = smem_opt_in((const void*)w4a4_gemm_1sm_kernel<MX, OUTF32>, kSmemBytes);
     if (attr_err != cudaSuccess)
         return attr_err;
     p.tiles_m = (int)(M / kBM);
     const int tiles = p.tiles_m * p.tiles_n;
     const int grid = tiles < num_sms() ? tiles : num_sms();
-    w4a4_gemm_1sm_kernel<MX><<<grid, kThreads, kSmemBytes, s>>>(ta, tb, tsa, tsb, ta1, tb1, p);
+    w4a4_gemm_1sm_kernel<MX, OUTF32><<<grid, kThreads, kSmemBytes, s>>>(ta, tb, tsa, tsb, ta1, tb1, p);
     return cudaGetLastError();
 }
 
 cudaError_t launch_w4a4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* ga,
                              const uint8_t* w_codes, const uint8_t* w_sf, const float* gw, int64_t M,
-                             int64_t N, int64_t K, void* out, int* err, cudaStream_t s,
+                             int64_t N, int64_t K, void* out, int out_f32, int* err, cudaStream_t s,
                              const uint8_t* a1_codes, const uint8_t* w1_codes, int mx)
 {
     GemmParams p;
@@ -1009,8 +1055,9 @@ cudaError_t launch_w4a4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const 
     p.sfb = w_sf;
     p.ga = ga;
     p.gw = gw;
-    p.out = reinterpret_cast<__nv_bfloat16*>(out);
+    p.out = out;
     p.err = err;
+    p.wait_limit = wait_limit_cycles();
     p.tiles_n = (int)(N / kBN);
     p.kblocks = (int)(K / kBK);
     p.kb_atoms = (int)(K / (mx ? 128 : 64));
@@ -1019,8 +1066,10 @@ cudaError_t launch_w4a4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const 
     const uint8_t* a1 = a1_codes ? a1_codes : a_codes;
     const uint8_t* w1 = w1_codes ? w1_codes : w_codes;
     if (mx)
-        return launch_gemm_t<true>(a_codes, a_sf, w_codes, w_sf, a1, w1, M, N, K, out, p, s);
-    return launch_gemm_t<false>(a_codes, a_sf, w_codes, w_sf, a1, w1, M, N, K, out, p, s);
+        return out_f32 ? launch_gemm_t<true, true>(a_codes, a_sf, w_codes, w_sf, a1, w1, M, N, K, out, p, s)
+                       : launch_gemm_t<true, false>(a_codes, a_sf, w_codes, w_sf, a1, w1, M, N, K, out, p, s);
+    return out_f32 ? launch_gemm_t<false, true>(a_codes, a_sf, w_codes, w_sf, a1, w1, M, N, K, out, p, s)
+                   : launch_gemm_t<false, false>(a_codes, a_sf, w_codes, w_sf, a1, w1, M, N, K, out, p, s);
 }
 
 }  // namespace fp4q

@@ -12,14 +12,17 @@
 //
 // The scratch array is file-scope device memory of kScratchFloats floats
 // (16 MiB); every GPU that loads the library holds it until the process
-// exits.  The first call on each device looks up the array's device address
-// on that device (cudaGetSymbolAddress); make that first call before any
-// stream capture begins.  All calls share the array, so two calls whose
-// kernels overlap on the GPU (different streams, or different host threads)
-// race on it; order them on one stream.  Each call overwrites every partial
-// it later reads, so nothing needs clearing between calls.
+// exits.  Every call looks up the array's device address on the current
+// device (cudaGetSymbolAddress; nothing is cached, so a device reset that
+// reloads the module at another address is picked up).  The first lookup on
+// a device loads the library's device code there; make that first call
+// before any stream capture begins.  All calls share the array, so two calls
+// whose kernels overlap on the GPU (different streams, or different host
+// threads) race on it; order them on one stream.  Each call overwrites every
+// partial it later reads, so the partials need no clearing; the error word
+// beside them (set when a bounded device wait gives up, read by
+// fp4q_hessian_status(NULL, stream)) is cleared at the start of every call.
 #include <cstdint>
-#include <mutex>
 #include <cuda_runtime.h>
 
 #include "../../include/fp4q.h"
@@ -33,27 +36,20 @@ constexpr size_t kScratchBlocks = 4096;
 constexpr size_t kScratchFloats = kScratchBlocks * 1024;
 
 static __device__ __align__(256) float g_hessian_scratch[kScratchFloats];
+static __device__ __align__(16) int g_hessian_err;
 
-constexpr int kMaxDevices = 64;
-std::mutex g_setup_mutex;
-float* g_scratch_ptr[kMaxDevices] = {};
-
-// Device address of the scratch array on the current device, looked up once
-// per device (the host-side symbol is only a stand-in, not a device address).
-int scratch_for_current_device(float** out)
+// Device addresses of the scratch array and of the error word on the current
+// device (in host code the symbols are only stand-ins, not device addresses).
+bool lookup_scratch(float** scratch, int** err)
 {
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
-        return FP4Q_ERR_CUDA;
-    std::lock_guard<std::mutex> lock(g_setup_mutex);
-    if (!g_scratch_ptr[dev]) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_hessian_scratch) != cudaSuccess || !p)
-            return FP4Q_ERR_CUDA;
-        g_scratch_ptr[dev] = static_cast<float*>(p);
-    }
-    *out = g_scratch_ptr[dev];
-    return FP4Q_OK;
+    void* p = nullptr;
+    void* e = nullptr;
+    if (cudaGetSymbolAddress(&p, g_hessian_scratch) != cudaSuccess || !p ||
+        cudaGetSymbolAddress(&e, g_hessian_err) != cudaSuccess || !e)
+        return false;
+    *scratch = static_cast<float*>(p);
+    *err = static_cast<int*>(e);
+    return true;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -78,19 +74,30 @@ int fp4_hessian_blocks_noalloc(const void* x, int dtype, int64_t rows, int64_t c
     if (need > kScratchFloats * sizeof(float))
         return FP4Q_ERR_TOO_LARGE;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    float* scratch = nullptr;
+    int* err = nullptr;
+    if (!lookup_scratch(&scratch, &err) || cudaMemsetAsync(err, 0, sizeof(int), s) != cudaSuccess)
+        return FP4Q_ERR_CUDA;
     if (rows == 0)
         return cudaMemsetAsync(hess_blocks, 0, (size_t)(cols / 32) * 1024 * sizeof(float), s) ==
                        cudaSuccess
                    ? FP4Q_OK
                    : FP4Q_ERR_CUDA;
-    float* scratch = nullptr;
-    const int st = scratch_for_current_device(&scratch);
-    if (st != FP4Q_OK)
-        return st;
     return fp4q::launch_hessian_blocks(x, dtype, rows, cols, chan_scale, hadamard32 != 0,
-                                       hess_blocks, scratch, s) == cudaSuccess
+                                       hess_blocks, scratch, err, s) == cudaSuccess
                ? FP4Q_OK
                : FP4Q_ERR_CUDA;
 }
 
 }  // extern "C"
+
+namespace fp4q {
+
+const int* noalloc_hessian_error_word()
+{
+    float* scratch = nullptr;
+    int* err = nullptr;
+    return lookup_scratch(&scratch, &err) ? err : nullptr;
+}
+
+}  // namespace fp4q

@@ -497,8 +497,9 @@ int grid_for(int64_t work, const void* kernel)
 // (one token per lane, one column block per warp; the next K block's loads are
 // in flight while the current one is transformed and stored) and then read
 // back the diagonal block of their TMEM lane quarter; warp 4 owns the TMEM and
-// issues the MMAs.  Waits are bounded; a CTA that gives up writes NaN into its
-// partial blocks, which the reduction carries into H'.
+// issues the MMAs.  Waits are bounded (main-loop waits by `wait_limit` cycles);
+// a CTA that gives up writes NaN into its partial blocks, which the reduction
+// carries into H', and sets the caller's error word *err to 1.
 constexpr int kHxKB = 32;                       // tokens per K block (128 B of tf32 per tile row)
 constexpr int kHxTile = 128 * 128;              // bytes of one operand tile
 constexpr int kHxThreads = 160;
@@ -533,7 +534,7 @@ __device__ __forceinline__ float hx_tf32(float a)
 template <typename T>
 __global__ void __launch_bounds__(kHxThreads, 1)
 hessian_partial_tc_kernel(const T* __restrict__ x, int64_t rows, int64_t cols, const float* __restrict__ t,
-                          int had, float* __restrict__ part)
+                          int had, float* __restrict__ part, long long wait_limit, int* err)
 {
     extern __shared__ uint8_t hx_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(hx_raw) + 1023) & ~uintptr_t(1023));
@@ -613,7 +614,7 @@ hessian_partial_tc_kernel(const T* __restrict__ x, int64_t rows, int64_t cols, c
             }
             if (s + 1 < kSteps)
                 fetch(s + 1);          // in flight while this block is transformed
-            if (use > 0 && !mbar_wait(bar0 + 8u * (2 + st), (use - 1u) & 1u, abort_flag)) {
+            if (use > 0 && !mbar_wait(bar0 + 8u * (2 + st), (use - 1u) & 1u, abort_flag, wait_limit)) {
                 *abort_flag = 1;
                 break;
             }
@@ -635,7 +636,8 @@ hessian_partial_tc_kernel(const T* __restrict__ x, int64_t rows, int64_t cols, c
             mbar_arrive(bar0 + 8u * st);
         }
         // ---------------- epilogue: the diagonal 32 x 32 block of this lane quarter
-        const bool ok = __all_sync(0xffffffffu, !*abort_flag && mbar_wait(bar0 + 32u, 0u, abort_flag));
+        const bool ok =
+            __all_sync(0xffffffffu, !*abort_flag && mbar_wait(bar0 + 32u, 0u, abort_flag, wait_limit));
         tc_fence_after();
         if (b < nblk) {
             float h[32];
@@ -660,7 +662,7 @@ hessian_partial_tc_kernel(const T* __restrict__ x, int64_t rows, int64_t cols, c
         bool issued = false;
         for (int s = 0; s < kSteps; ++s) {
             const int st = s & 1;
-            if (!mbar_wait(bar0 + 8u * st, (uint32_t)(s >> 1) & 1u, abort_flag)) {
+            if (!mbar_wait(bar0 + 8u * st, (uint32_t)(s >> 1) & 1u, abort_flag, wait_limit)) {
                 *abort_flag = 1;
                 break;
             }
@@ -690,6 +692,8 @@ hessian_partial_tc_kernel(const T* __restrict__ x, int64_t rows, int64_t cols, c
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+    if (threadIdx.x == 0 && *abort_flag)
+        atomicExch(err, 1);
     if (warp == 4)
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kHxCols) : "memory");
 }
@@ -747,12 +751,12 @@ cudaError_t launch_mxfp4_quant(const void* x, int dtype, int64_t rows, int64_t c
 }
 
 cudaError_t launch_hessian_blocks(const void* x, int dtype, int64_t rows, int64_t cols,
-                                  const float* chan_scale, int hadamard, float* hess, void* ws,
-                                  cudaStream_t s)
+                                  const float* chan_scale, int hadamard, float* hess, float* part,
+                                  int* err, cudaStream_t s)
 {
     const int64_t kb = cols / 32;
     const int64_t nchunk = (rows + kTok - 1) / kTok;
-    float* part = reinterpret_cast<float*>(ws);
+    const long long limit = wait_limit_cycles();
     const cudaError_t hx_attr =
         dtype == 1 ? smem_opt_in((const void*)hessian_partial_tc_kernel<__nv_bfloat16>, kHxSmem)
                    : smem_opt_in((const void*)hessian_partial_tc_kernel<float>, kHxSmem);
@@ -761,10 +765,10 @@ cudaError_t launch_hessian_blocks(const void* x, int dtype, int64_t rows, int64_
     dim3 grid((unsigned)nchunk, (unsigned)((kb + 3) / 4));
     if (dtype == 1)
         hessian_partial_tc_kernel<__nv_bfloat16><<<grid, kHxThreads, kHxSmem, s>>>(
-            reinterpret_cast<const __nv_bfloat16*>(x), rows, cols, chan_scale, hadamard, part);
+            reinterpret_cast<const __nv_bfloat16*>(x), rows, cols, chan_scale, hadamard, part, limit, err);
     else
         hessian_partial_tc_kernel<float><<<grid, kHxThreads, kHxSmem, s>>>(
-            reinterpret_cast<const float*>(x), rows, cols, chan_scale, hadamard, part);
+            reinterpret_cast<const float*>(x), rows, cols, chan_scale, hadamard, part, limit, err);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess)
         return e;

@@ -1,12 +1,14 @@
-// runtime.cu -- per-device host-side state of the library: the SM count used to
-// size persistent grids, and the shared-memory opt-in of kernels that need more
-// than the default 48 KiB of dynamic shared memory.  Both are per device, so a
-// process that drives several GPUs gets each one right.
+// runtime.cu -- host-side state of the library: the SM count used to size
+// persistent grids and the shared-memory opt-in of kernels that need more than
+// the default 48 KiB of dynamic shared memory (both per device, so a process
+// that drives several GPUs gets each one right), and the process-wide limit of
+// the tensor-core kernels' bounded waits (fp4q_debug_set_wait_cycles).
 #include <atomic>
 #include <mutex>
 #include <set>
 #include <utility>
 
+#include "../../include/fp4q.h"
 #include "fp4q_internal.h"
 
 namespace fp4q {
@@ -17,8 +19,15 @@ constexpr int kMaxDevices = 64;
 std::atomic<int> g_sms[kMaxDevices];
 std::mutex g_opt_mu;
 std::set<std::pair<const void*, int>> g_opted;   // (kernel, device) pairs already opted in
+std::atomic<long long> g_wait_cycles{0};         // 0: kDefaultWaitCycles
 
 }  // namespace
+
+long long wait_limit_cycles()
+{
+    const long long v = g_wait_cycles.load(std::memory_order_relaxed);
+    return v > 0 ? v : kDefaultWaitCycles;
+}
 
 int num_sms()
 {
@@ -50,3 +59,8 @@ cudaError_t smem_opt_in(const void* kernel, int bytes)
 }
 
 }  // namespace fp4q
+
+extern "C" int64_t fp4q_debug_set_wait_cycles(int64_t cycles)
+{
+    return fp4q::g_wait_cycles.exchange(cycles > 0 ? cycles : 0, std::memory_order_relaxed);
+}

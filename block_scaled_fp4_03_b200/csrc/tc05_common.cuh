@@ -3,11 +3,16 @@
 #pragma once
 #include <cstdint>
 
+#include "fp4q_internal.h"
+
 namespace fp4q {
 namespace {
 
-// About 2 s at the boost clock: every wait on a barrier gives up after this.
-constexpr long long kTcWaitCycles = 4000000000LL;
+// About 2 s at the boost clock: every wait on a barrier gives up after this
+// (the default; a kernel's main-loop waits may be given a shorter limit, see
+// fp4q_debug_set_wait_cycles, but the waits that let a CTA's own copies and
+// MMAs finish before it exits always use this one).
+constexpr long long kTcWaitCycles = kDefaultWaitCycles;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p)
 {
@@ -37,18 +42,38 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity)
     return ok != 0;
 }
 
-// Wait for the phase with the given parity.  False if it did not complete
-// within kTcWaitCycles or, while waiting, the abort flag (if any) was raised.
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const volatile int* abort_flag)
+// Non-blocking test of the phase with the given parity.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity)
 {
-    if (mbar_try_wait(bar, parity))
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok)
+                 : "r"(bar), "r"(parity)
+                 : "memory");
+    return ok != 0;
+}
+
+// Limits below this are test settings: the first probe of such a wait does
+// not block (a blocking probe may sleep in hardware until the phase
+// completes), so a wait whose phase is not already complete gives up.
+constexpr long long kShortWaitCycles = 1LL << 20;
+
+// Wait for the phase with the given parity.  False if it did not complete
+// within `limit` cycles or, while waiting, the abort flag (if any) was raised.
+__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const volatile int* abort_flag,
+                                       long long limit = kTcWaitCycles)
+{
+    if (limit >= kShortWaitCycles ? mbar_try_wait(bar, parity) : mbar_test_wait(bar, parity))
         return true;
     const long long t0 = clock64();
-    while (!mbar_try_wait(bar, parity)) {
-        if ((abort_flag && *abort_flag) || clock64() - t0 > kTcWaitCycles)
+    for (;;) {
+        if ((abort_flag && *abort_flag) || clock64() - t0 > limit)
             return false;
+        if (mbar_try_wait(bar, parity))
+            return true;
     }
-    return true;
 }
 
 // Time-bounded wait that ignores any abort flag: lets this CTA's own copies

@@ -30,8 +30,10 @@
  *  - Scale bytes, one per block, row-major [rows][cols/block] unless an MMA
  *    layout is requested.
  *  - "device" pointers are CUDA device memory owned by the caller; the library
- *    allocates and frees nothing and keeps no state between calls.  "host"
- *    pointers are read during the call only.
+ *    allocates and frees nothing and keeps no state between calls (apart from
+ *    the debug wait limit of fp4q_debug_set_wait_cycles and the fixed scratch
+ *    of fp4_hessian_blocks_noalloc).  "host" pointers are read during the call
+ *    only.
  *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
  *    stream) and is asynchronous: outputs are valid once the stream reaches
  *    the call.  Argument errors are found on the host before anything is
@@ -246,7 +248,13 @@ FP4Q_API int mxfp4_flip_refine(const void* w, int dtype, int64_t rows, int64_t c
  * accuracy (tolerance, not bit-exact); partial sums per 256 tokens are added
  * in a fixed order, so the result is deterministic.
  *  hess_blocks  device fp32 [cols/32][32][32] (out)
- *  workspace    >= fp4q_workspace_size(FP4Q_OP_HESSIAN, rows, cols, 0)
+ *  workspace    >= fp4q_workspace_size(FP4Q_OP_HESSIAN, rows, cols, 0) bytes
+ *               (cols > 0), 16-byte aligned: an error word, then the partials
+ * The kernel's waits on its own barriers are bounded.  If one gives up, the
+ * blocks of the CTAs concerned come out NaN and the workspace's error word is
+ * set: fp4q_hessian_status(workspace, stream) then returns FP4Q_ERR_TIMEOUT
+ * (the call itself has already returned FP4Q_OK, having only enqueued work).
+ * Errors: ERR_ARG, ERR_ALIGN, ERR_WORKSPACE, ERR_CUDA.
  */
 FP4Q_API int fp4_hessian_blocks(const void* x, int dtype, int64_t rows, int64_t cols,
                        const float* chan_scale, int hadamard32, float* hess_blocks,
@@ -266,13 +274,25 @@ FP4Q_API int fp4_hessian_blocks(const void* x, int dtype, int64_t rows, int64_t 
  * 16 MiB of it (e.g. more than 8192 rows at 4096 columns) return
  * FP4Q_ERR_TOO_LARGE before anything runs.  Nothing is allocated or freed.
  * All calls share the one scratch array: calls whose work overlaps on the
- * GPU (other streams, other threads) race -- order them on one stream.  The
- * first call on a device looks up the scratch's device address on that
- * device; make that first call before any stream capture begins.
+ * GPU (other streams, other threads) race -- order them on one stream.  Every
+ * call looks up the scratch's device address on the current device (the
+ * first lookup on a device loads the library's device code there: make that
+ * first call before any stream capture begins).  A bounded device wait that
+ * gives up is reported by fp4q_hessian_status(NULL, stream) (FP4Q_ERR_TIMEOUT,
+ * blocks NaN); the error word is cleared by every call.
  */
 FP4Q_API int fp4_hessian_blocks_noalloc(const void* x, int dtype, int64_t rows, int64_t cols,
                                         const float* chan_scale, int hadamard32,
                                         float* hess_blocks, void* stream);
+
+/*
+ * Synchronizes `stream` and reports whether the last fp4_hessian_blocks call
+ * that used `workspace` (or, for workspace == NULL, the last
+ * fp4_hessian_blocks_noalloc call on the current device) finished normally
+ * (FP4Q_OK) or had a bounded device-side wait give up (FP4Q_ERR_TIMEOUT: the
+ * blocks of the CTAs concerned are NaN).  ERR_CUDA if the word cannot be read.
+ */
+FP4Q_API int fp4q_hessian_status(const void* workspace, void* stream);
 
 /*
  * Online per-channel scale of [MACaQ] 3: t_j = (sigma_j^W / rms_j^X)^alpha,
@@ -309,7 +329,7 @@ FP4Q_API int fp4_dequant_mse(const uint8_t* codes, const uint8_t* scales, int64_
  * E4M3 scales per 16 elements; [NVFP4] 3: per-tensor global scales).
  *
  *   out[m][n] = bf16( g_a * g_w * sum_k (v_a sc_a)[m][k] * (v_w sc_w)[n][k] ),
- *   i.e. out = A . W^T, A: M x K, W: N x K, out: M x N bf16 row-major.
+ *   i.e. out = A . W^T, A: M x K, W: N x K, out: M x N row-major.
  *
  *  a, a_format    FP4Q_F32 / FP4Q_BF16: A is a dense M x K tensor quantized here
  *                 (block 16, rule a_rule of ABSMAX/PREVENT_ZERO/FOUR_OVER_SIX/BRUTE_FORCE,
@@ -319,6 +339,9 @@ FP4Q_API int fp4_dequant_mse(const uint8_t* codes, const uint8_t* scales, int64_
  *  w_codes        device N*K/2 packed codes; w_scales E4M3 bytes in the MMA layout;
  *                 w_global_scale device g_w
  *  M % 128 == 0, N % 256 == 0, K % 256 == 0 (FP4Q_ERR_UNSUPPORTED otherwise)
+ *  out, out_dtype device M x N; FP4Q_BF16 (the W4A4 output) or FP4Q_F32: the fp32
+ *                 accumulator times g_a g_w without the bf16 rounding (for accuracy
+ *                 checks against an fp64 reference, or consumers that keep fp32)
  *  workspace      >= fp4q_workspace_size(FP4Q_OP_GEMM, M, K, N) bytes (at least 8 KiB
  *                 for packed A), 16-byte aligned; it also holds the error word read by
  *                 fp4q_gemm_status
@@ -327,7 +350,7 @@ FP4Q_API int fp4_dequant_mse(const uint8_t* codes, const uint8_t* scales, int64_
 FP4Q_API int w4a4_gemm(const void* a, int a_format, int a_rule, const uint8_t* a_scales,
                        const float* a_global_scale, const uint8_t* w_codes,
                        const uint8_t* w_scales, const float* w_global_scale, int64_t M,
-                       int64_t N, int64_t K, void* out, void* workspace,
+                       int64_t N, int64_t K, void* out, int out_dtype, void* workspace,
                        size_t workspace_bytes, void* stream);
 
 /*
@@ -372,14 +395,14 @@ FP4Q_API int razer_gemm_prepare(const uint8_t* codes, const uint8_t* meta, int64
  *                                a_global_scale device g_a
  *  w_codes, w_extra (nullable)   device N*K/2 bytes; w_scales E4M3 MMA layout;
  *                                w_global_scale device g_w
- *  shapes, out, workspace (>= 8 KiB) and errors as w4a4_gemm; fp4q_gemm_status
- *  reports a device timeout.
+ *  shapes, out / out_dtype, workspace (>= 8 KiB) and errors as w4a4_gemm;
+ *  fp4q_gemm_status reports a device timeout.
  */
 FP4Q_API int razer_w4a4_gemm(const uint8_t* a_codes, const uint8_t* a_extra, const uint8_t* a_scales,
                              const float* a_global_scale, const uint8_t* w_codes,
                              const uint8_t* w_extra, const uint8_t* w_scales,
                              const float* w_global_scale, int64_t M, int64_t N, int64_t K, void* out,
-                             void* workspace, size_t workspace_bytes, void* stream);
+                             int out_dtype, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Scale bytes from the row-major layout [rows][nscales] to FP4Q_SFLAYOUT_MMA
@@ -412,28 +435,35 @@ FP4Q_API int fp4_scales_to_mma(const uint8_t* scales, int64_t rows, int64_t nsca
  *  w_codes      device N*K/2 bytes; w_scales E8M0 bytes in FP4Q_SFLAYOUT_MMA
  *               (mxfp4_quantize + fp4_scales_to_mma)
  *  M % 128 == 0, N % 256 == 0, K % 256 == 0 (FP4Q_ERR_UNSUPPORTED otherwise)
+ *  out, out_dtype as w4a4_gemm (FP4Q_BF16 or FP4Q_F32)
  *  workspace    >= fp4q_workspace_size(FP4Q_OP_MX_GEMM, M, K, N) for dense A,
  *               8 KiB for packed A; 16-byte aligned; holds the error word read
  *               by fp4q_gemm_status
  */
 FP4Q_API int mxfp4_gemm(const void* a, int a_format, const uint8_t* a_scales, const float* chan_scale,
                         int hadamard32, const uint8_t* w_codes, const uint8_t* w_scales, int64_t M,
-                        int64_t N, int64_t K, void* out, void* workspace, size_t workspace_bytes,
-                        void* stream);
+                        int64_t N, int64_t K, void* out, int out_dtype, void* workspace,
+                        size_t workspace_bytes, void* stream);
 
 /*
- * Synchronizes `stream` and reports whether the last w4a4_gemm that used this
- * workspace finished normally (FP4Q_OK) or gave up a bounded device-side wait
- * (FP4Q_ERR_TIMEOUT; its output is then incomplete).
+ * Synchronizes `stream` and reports whether the last GEMM call (w4a4_gemm,
+ * razer_w4a4_gemm or mxfp4_gemm) that used this workspace finished normally
+ * (FP4Q_OK) or had a bounded device-side wait give up (FP4Q_ERR_TIMEOUT; its
+ * output is then incomplete).  Every GEMM call clears the word first.
  */
 FP4Q_API int fp4q_gemm_status(const void* workspace, void* stream);
 
 /*
- * The same report for any call that takes a GEMM workspace (w4a4_gemm,
- * razer_w4a4_gemm, mxfp4_gemm): synchronizes `stream`, then FP4Q_OK or
- * FP4Q_ERR_TIMEOUT.  Same semantics as fp4q_gemm_status.
+ * Debug: the limit, in SM clock cycles, after which the main-loop waits of the
+ * tensor-core kernels (the three GEMMs and the Hessian blocks) give up; 0 or a
+ * negative value restores the default (4e9 cycles, about 2 s at the boost
+ * clock).  Process-wide; read when a call launches its kernels.  Meant for
+ * tests of the timeout path: with a limit of 1 cycle a wait that is not
+ * satisfied at once gives up, the kernel winds down (letting its own copies
+ * and MMAs finish under the default limit), and the status call of that
+ * entry point reports FP4Q_ERR_TIMEOUT.  Returns the previous setting.
  */
-FP4Q_API int fp4q_sync_status(const void* workspace, void* stream);
+FP4Q_API int64_t fp4q_debug_set_wait_cycles(int64_t cycles);
 
 #ifdef __cplusplus
 }

@@ -52,7 +52,7 @@ def test_version_and_status_strings(L):
 def test_workspace_sizes(L):
     assert L.fp4q_workspace_size(0, 4096, 4096, 0) >= 592 * 4
     h = L.fp4q_workspace_size(1, 8192, 4096, 0)
-    assert h == (8192 // 256) * (4096 // 32) * 1024 * 4
+    assert h == 256 + (8192 // 256) * (4096 // 32) * 1024 * 4     # error word header + partials
     assert L.fp4q_workspace_size(1, 8192, 100, 0) == 0
     assert L.fp4q_workspace_size(2, 8192, 4096, 4096) > 0
 
@@ -105,6 +105,9 @@ def test_mx_and_dequant_argument_errors(L):
     assert L.fp4_dequant_mse(FAKE, FAKE, 4, 64, 16, 2, None, 0, None, None, 0, FAKE, None, None) == 1
     assert L.fp4_dequant_mse(FAKE, FAKE, 4, 64, 16, 0, None, 0, None, None, 0, FAKE, FAKE, None) == 1
     assert L.fp4_hessian_blocks(FAKE, 0, 64, 64, None, 1, FAKE, None, 0, None) == 6
+    need = L.fp4q_workspace_size(1, 64, 64, 0)
+    assert L.fp4_hessian_blocks(FAKE, 0, 64, 64, None, 1, FAKE, FAKE, need - 1, None) == 6
+    assert L.fp4_hessian_blocks(FAKE, 0, 64, 64, None, 1, FAKE, MIS, need, None) == 2
     assert L.mxfp4_channel_scale(FAKE, 0, 64, FAKE, 0, 64, 12, 0.75, FAKE, None, FAKE, 1 << 20, None) == 1
     # Flip-Refinement: bad width, budget, missing Hessian, misalignment, too wide,
     # missing workspace, empty
@@ -137,20 +140,25 @@ def test_gemm_family_argument_errors(L):
     assert L.razer_gemm_prepare(MIS, FAKE, 128, 64, 1, sp, 4, FAKE, FAKE, FAKE, None) == 2
     assert L.razer_gemm_prepare(None, None, 0, 64, 1, sp, 4, None, None, None, None) == 0
     # razer_w4a4_gemm: missing operands, shapes, alignment, workspace
-    assert L.razer_w4a4_gemm(None, None, FAKE, FAKE, FAKE, None, FAKE, FAKE, 128, 256, 256, FAKE, FAKE, 8192, None) == 1
-    assert L.razer_w4a4_gemm(FAKE, None, FAKE, FAKE, FAKE, None, FAKE, FAKE, 100, 256, 256, FAKE, FAKE, 8192, None) == 3
-    assert L.razer_w4a4_gemm(FAKE, MIS, FAKE, FAKE, FAKE, None, FAKE, FAKE, 128, 256, 256, FAKE, FAKE, 8192, None) == 2
-    assert L.razer_w4a4_gemm(FAKE, None, FAKE, FAKE, FAKE, None, FAKE, FAKE, 128, 256, 256, FAKE, FAKE, 100, None) == 6
+    assert L.razer_w4a4_gemm(None, None, FAKE, FAKE, FAKE, None, FAKE, FAKE, 128, 256, 256, FAKE, 1, FAKE, 8192, None) == 1
+    assert L.razer_w4a4_gemm(FAKE, None, FAKE, FAKE, FAKE, None, FAKE, FAKE, 100, 256, 256, FAKE, 1, FAKE, 8192, None) == 3
+    assert L.razer_w4a4_gemm(FAKE, MIS, FAKE, FAKE, FAKE, None, FAKE, FAKE, 128, 256, 256, FAKE, 1, FAKE, 8192, None) == 2
+    assert L.razer_w4a4_gemm(FAKE, None, FAKE, FAKE, FAKE, None, FAKE, FAKE, 128, 256, 256, FAKE, 1, FAKE, 100, None) == 6
     # mxfp4_gemm: format, packed A without scales or with a channel scale, shapes, workspace
-    assert L.mxfp4_gemm(FAKE, 2, FAKE, None, 1, FAKE, FAKE, 128, 256, 256, FAKE, FAKE, 1 << 20, None) == 1
-    assert L.mxfp4_gemm(FAKE, 3, None, None, 1, FAKE, FAKE, 128, 256, 256, FAKE, FAKE, 1 << 20, None) == 1
-    assert L.mxfp4_gemm(FAKE, 3, FAKE, FAKE, 1, FAKE, FAKE, 128, 256, 256, FAKE, FAKE, 1 << 20, None) == 1
-    assert L.mxfp4_gemm(FAKE, 1, None, None, 1, FAKE, FAKE, 128, 256, 100, FAKE, FAKE, 1 << 20, None) == 3
-    assert L.mxfp4_gemm(FAKE, 1, None, None, 1, FAKE, FAKE, 0, 256, 256, FAKE, FAKE, 1 << 20, None) == 1
+    assert L.mxfp4_gemm(FAKE, 2, FAKE, None, 1, FAKE, FAKE, 128, 256, 256, FAKE, 1, FAKE, 1 << 20, None) == 1
+    assert L.mxfp4_gemm(FAKE, 3, None, None, 1, FAKE, FAKE, 128, 256, 256, FAKE, 1, FAKE, 1 << 20, None) == 1
+    assert L.mxfp4_gemm(FAKE, 3, FAKE, FAKE, 1, FAKE, FAKE, 128, 256, 256, FAKE, 1, FAKE, 1 << 20, None) == 1
+    assert L.mxfp4_gemm(FAKE, 1, None, None, 1, FAKE, FAKE, 128, 256, 100, FAKE, 1, FAKE, 1 << 20, None) == 3
+    assert L.mxfp4_gemm(FAKE, 1, None, None, 1, FAKE, FAKE, 0, 256, 256, FAKE, 1, FAKE, 1 << 20, None) == 1
     need = L.fp4q_workspace_size(5, 128, 256, 256)
     assert need == 8192 + 128 * 256 // 2 + 128 * 256 // 32
-    assert L.mxfp4_gemm(FAKE, 1, None, None, 1, FAKE, FAKE, 128, 256, 256, FAKE, FAKE, need - 1, None) == 6
-    assert L.mxfp4_gemm(FAKE, 3, FAKE, None, 1, FAKE, FAKE, 128, 256, 256, FAKE, FAKE, 8191, None) == 6
+    assert L.mxfp4_gemm(FAKE, 1, None, None, 1, FAKE, FAKE, 128, 256, 256, FAKE, 1, FAKE, need - 1, None) == 6
+    assert L.mxfp4_gemm(FAKE, 3, FAKE, None, 1, FAKE, FAKE, 128, 256, 256, FAKE, 1, FAKE, 8191, None) == 6
+    # fp4_scales_to_mma
+    # every GEMM rejects an output type other than bf16 / fp32
+    assert L.razer_w4a4_gemm(FAKE, None, FAKE, FAKE, FAKE, None, FAKE, FAKE, 128, 256, 256, FAKE, 2, FAKE, 8192, None) == 1
+    assert L.mxfp4_gemm(FAKE, 1, None, None, 1, FAKE, FAKE, 128, 256, 256, FAKE, 3, FAKE, 1 << 20, None) == 1
+    assert L.w4a4_gemm(FAKE, 2, 0, FAKE, FAKE, FAKE, FAKE, FAKE, 128, 256, 256, FAKE, 2, FAKE, 1 << 20, None) == 1
     # fp4_scales_to_mma
     assert L.fp4_scales_to_mma(FAKE, 100, 8, FAKE, None) == 1
     assert L.fp4_scales_to_mma(FAKE, 128, 6, FAKE, None) == 1
@@ -179,4 +187,14 @@ def test_header_is_plain_c(tmp_path):
 
 def test_status_calls_reject_a_missing_workspace(L):
     assert L.fp4q_gemm_status(None, None) == 1
-    assert L.fp4q_sync_status(None, None) == 1
+
+
+def test_debug_wait_limit_setter_round_trips(L):
+    """The wait-limit knob is host state only: it stores and returns settings, 0 = default."""
+    prev = L.fp4q_debug_set_wait_cycles(1)
+    try:
+        assert L.fp4q_debug_set_wait_cycles(12345) == 1
+        assert L.fp4q_debug_set_wait_cycles(-5) == 12345
+        assert L.fp4q_debug_set_wait_cycles(0) == 0          # a negative value stored as the default
+    finally:
+        L.fp4q_debug_set_wait_cycles(prev)

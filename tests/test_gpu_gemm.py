@@ -1,9 +1,13 @@
-"""GPU parity of the tcgen05 W4A4 GEMM against the oracle's fp64 product of
-the exactly decoded NVFP4 operands.
+"""GPU parity of the tcgen05 W4A4 GEMM ("Why Gated DeltaNet Survives 4-Bit
+Quantization" review, section 1: NVFP4 W4A4) against the oracle's fp64 product
+of the exactly decoded NVFP4 operands.
 
-Bar: relative Frobenius error against the bf16-rounded fp64 reference
-<= 1e-3 (bf16 output rounding alone is ~1.5e-3 against the raw fp64 value,
-so the raw-reference error is reported, and bounded at 4e-3).
+Every checked element is held to a bound derived from fp32 accumulation (and,
+for bf16 output, the bf16 rounding): see tests/gemm_check.py.  The fp32 output
+mode is also held to a relative Frobenius error of 1e-5 against the raw fp64
+product, the bf16 output to 1e-3 against the bf16-rounded product.  The
+full-size case checks one row in every 128-row band over all columns, so every
+output tile of both kernels is sampled.
 """
 import ctypes
 
@@ -13,6 +17,7 @@ import torch
 
 from block_scaled_fp4_03_b200 import binding as fq
 from block_scaled_fp4_03_b200 import inputs
+from gemm_check import band_rows, check_gemm
 
 pytestmark = pytest.mark.gpu
 
@@ -28,23 +33,6 @@ def to_mma_layout(sc):
     return out
 
 
-def bf16_round(x64):
-    f = x64.astype(np.float32)
-    return inputs.bf16_bits_to_f32(inputs.f32_to_bf16_bits(f)).astype(np.float64)
-
-
-def check(gpu_bf16, ref64, tol=1e-3):
-    got = gpu_bf16.float().cpu().numpy().astype(np.float64)
-    ref_b = bf16_round(ref64)
-    den = np.linalg.norm(ref64)
-    e_b = np.linalg.norm(got - ref_b) / den
-    e_raw = np.linalg.norm(got - ref64) / den
-    assert np.isfinite(got).all()
-    assert e_b <= tol, (e_b, e_raw)
-    assert e_raw <= 4e-3, (e_b, e_raw)
-    return e_b, e_raw
-
-
 def dev(a):
     a = np.ascontiguousarray(a)
     if a.dtype == np.uint16:
@@ -58,19 +46,40 @@ def quantized_operand(O, x32, rule):
     return q, g
 
 
-@pytest.mark.parametrize("M,N,K", [(128, 256, 256), (256, 512, 512), (384, 768, 2048), (2048, 4096, 512)])
-def test_gemm_packed_operands(O, M, N, K):
+SHAPES = [(128, 256, 256), (256, 512, 512), (384, 768, 2048), (2048, 4096, 512)]
+
+
+@pytest.mark.parametrize("out_dtype", [fq.BF16, fq.F32])
+@pytest.mark.parametrize("M,N,K", SHAPES)
+def test_gemm_packed_operands(O, M, N, K, out_dtype):
     a32 = inputs.as_f32(inputs.generate("gemm_act", M, K, seed=M + K))
     w32 = inputs.as_f32(inputs.generate("gemm_weight", N, K, seed=N + K))
     qa, ga = quantized_operand(O, a32, O.RULE_FOUR_OVER_SIX)
     qw, gw = quantized_operand(O, w32, O.RULE_ABSMAX)
     out = fq.w4a4_gemm(dev(qa["codes"]), dev(qw["codes"]), dev(to_mma_layout(qw["scales"])),
                        dev(np.array([gw], np.float32)), a_scales=dev(to_mma_layout(qa["scales"])),
-                       a_global_scale=dev(np.array([ga], np.float32)))
+                       a_global_scale=dev(np.array([ga], np.float32)), out_dtype=out_dtype)
     torch.cuda.synchronize()
-    rows = np.arange(M) if M <= 512 else np.sort(np.random.default_rng(0).choice(M, 96, replace=False))
-    ref = O.gemm_ref(qa["codes"], qa["scales"], ga, qw["codes"], qw["scales"], gw, rows=rows)
-    check(out[torch.from_numpy(rows).cuda()], ref)
+    rows = np.arange(M) if M <= 512 else band_rows(M)
+    da = O.nvfp4_decode_exact(qa["codes"][rows], qa["scales"][rows])
+    dw = O.nvfp4_decode_exact(qw["codes"], qw["scales"])
+    check_gemm(out[torch.from_numpy(rows).cuda()], da, dw, float(ga) * float(gw), K,
+               "nvfp4 packed %dx%dx%d" % (M, N, K))
+
+
+def test_fp32_and_bf16_outputs_agree(O):
+    """The bf16 output is the round-to-nearest bf16 of the fp32 output, element for element."""
+    M, N, K = 256, 512, 1024
+    a32 = inputs.as_f32(inputs.generate("gemm_act", M, K, seed=3))
+    w32 = inputs.as_f32(inputs.generate("gemm_weight", N, K, seed=4))
+    qa, ga = quantized_operand(O, a32, O.RULE_FOUR_OVER_SIX)
+    qw, gw = quantized_operand(O, w32, O.RULE_ABSMAX)
+    args = (dev(qa["codes"]), dev(qw["codes"]), dev(to_mma_layout(qw["scales"])), dev(np.array([gw], np.float32)))
+    kw = dict(a_scales=dev(to_mma_layout(qa["scales"])), a_global_scale=dev(np.array([ga], np.float32)))
+    o16 = fq.w4a4_gemm(*args, **kw)
+    o32 = fq.w4a4_gemm(*args, out_dtype=fq.F32, **kw)
+    assert o32.dtype == torch.float32 and o16.dtype == torch.bfloat16
+    assert torch.equal(o32.to(torch.bfloat16).view(torch.int16), o16.view(torch.int16))
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
@@ -87,8 +96,8 @@ def test_gemm_fused_activation_quant(O, dtype):
                        dev(np.array([gw], np.float32)), a_rule=fq.FOUR_OVER_SIX, workspace=ws)
     assert fq.gemm_status(ws) == 0
     qa, ga = quantized_operand(O, a32, O.RULE_FOUR_OVER_SIX)
-    ref = O.gemm_ref(qa["codes"], qa["scales"], ga, qw["codes"], qw["scales"], gw)
-    check(out, ref)
+    check_gemm(out, O.nvfp4_decode_exact(qa["codes"], qa["scales"]), O.nvfp4_decode_exact(qw["codes"], qw["scales"]),
+               float(ga) * float(gw), K, "nvfp4 fused act quant " + dtype)
     # the fused quantizer's outputs in the workspace are the oracle's, bit for bit
     wsh = ws.cpu().numpy()
     assert wsh[4096:4100].view(np.float32)[0] == ga
@@ -100,27 +109,27 @@ def test_gemm_rejects_unsupported_shapes():
     L = fq.lib()
     fake = ctypes.c_void_p(0x10000)
     for M, N, K in ((100, 256, 256), (128, 200, 256), (128, 256, 100), (0, 256, 256)):
-        st = L.w4a4_gemm(fake, fq.NVFP4_PACKED, 0, fake, fake, fake, fake, fake, M, N, K, fake, fake, 1 << 20, None)
+        st = L.w4a4_gemm(fake, fq.NVFP4_PACKED, 0, fake, fake, fake, fake, fake, M, N, K, fake, fq.BF16, fake, 1 << 20, None)
         assert st in (1, 3), (M, N, K, st)
 
 
-def test_gemm_full_size_sampled(O):
-    """M=8192 tokens x K=4096 x N=14336: dynamic 4-over-6 activations, abs-max weights."""
+@pytest.mark.parametrize("out_dtype", [fq.BF16, fq.F32])
+def test_gemm_full_size_sampled(O, out_dtype):
+    """M=8192 tokens x K=4096 x N=14336: dynamic 4-over-6 activations, abs-max
+    weights; one row of every 128-row band against all 14336 columns."""
     M, N, K = 8192, 14336, 4096
     a = inputs.generate("gemm_act")
     w32 = inputs.as_f32(inputs.generate("gemm_weight"))
     qw, gw = quantized_operand(O, w32, O.RULE_ABSMAX)
     ws = torch.empty(fq.workspace_size(fq.OP_GEMM, M, K, N), dtype=torch.uint8, device="cuda")
     out = fq.w4a4_gemm(dev(a), dev(qw["codes"]), dev(to_mma_layout(qw["scales"])),
-                       dev(np.array([gw], np.float32)), a_rule=fq.FOUR_OVER_SIX, workspace=ws)
+                       dev(np.array([gw], np.float32)), a_rule=fq.FOUR_OVER_SIX, workspace=ws,
+                       out_dtype=out_dtype)
     assert fq.gemm_status(ws) == 0
     a32 = inputs.as_f32(a)
     ga = O.global_scale(O.amax(a32))
-    rows = np.sort(np.random.default_rng(1).choice(M, 48, replace=False))
+    rows = band_rows(M, salt=out_dtype)
     qa = O.nvfp4_quantize(a32[rows], 16, O.RULE_FOUR_OVER_SIX, g=ga, want_deq=False, want_mse=False)
-    ref = O.gemm_ref(qa["codes"], qa["scales"], ga, qw["codes"], qw["scales"], gw)
-    check(out[torch.from_numpy(rows).cuda()], ref)
-    # one full row tile and one full column tile, to cover every M and N tile position
-    cols = np.arange(0, N, 97)
-    ref_c = O.gemm_ref(qa["codes"], qa["scales"], ga, qw["codes"], qw["scales"], gw, cols=cols)
-    check(out[torch.from_numpy(rows).cuda()][:, torch.from_numpy(cols).cuda()], ref_c)
+    check_gemm(out[torch.from_numpy(rows).cuda()], O.nvfp4_decode_exact(qa["codes"], qa["scales"]),
+               O.nvfp4_decode_exact(qw["codes"], qw["scales"]), float(ga) * float(gw), K,
+               "nvfp4 full 8192x14336x4096")

@@ -264,8 +264,9 @@ def test_mxfp4_hessian_small(O, dtype):
 def test_hessian_blocks(O, dtype):
     x, x32 = make("mx_act", 700, 128, seed=9, dtype=dtype)
     t = inputs.positive_vector(128, seed=6)
-    h = fq.hessian_blocks(x, dev(t), True)
-    torch.cuda.synchronize()
+    ws = torch.empty(fq.workspace_size(fq.OP_HESSIAN, 700, 128), dtype=torch.uint8, device="cuda")
+    h = fq.hessian_blocks(x, dev(t), True, workspace=ws)
+    assert fq.hessian_status(ws) == 0
     ref = O.hessian_blocks(x32, t, True)
     got = host(h).astype(np.float64)
     for k in range(ref.shape[0]):
@@ -444,8 +445,8 @@ def test_full_mxfp4_prep_sampled(O):
     # H' from the GPU's own t, against the oracle on the same t
     href = O.hessian_blocks(x32, tg, True)
     hg = host(h).astype(np.float64)
-    for k in range(0, 128, 9):
-        assert np.linalg.norm(hg[k] - href[k]) / np.linalg.norm(href[k]) <= 1e-4
+    for k in range(128):                      # every 32 x 32 block, at the small cases' tolerance
+        assert np.linalg.norm(hg[k] - href[k]) / np.linalg.norm(href[k]) <= 1e-5, k
     # weight quantizer: decision parity on the oracle's H' (an input to both)
     hin = href.astype(np.float32)
     qw = fq.mxfp4_quantize(w, ti, True, fq.HESSIAN_EXP, hess=dev(hin), mse=True)

@@ -1,0 +1,116 @@
+"""Failure detection of the tensor-core kernels, exercised without a GPU fault.
+
+Every wait of the GEMM kernels (single-CTA and CTA-pair) and of the Hessian
+kernel on its own barriers is bounded.  With the process-wide debug limit set
+to one cycle (fp4q_debug_set_wait_cycles), the first wait that is not
+satisfied at once gives up: the kernel raises its abort flag, lets the copies
+and MMAs it already issued finish (those waits keep the default limit),
+releases its tensor memory and returns.  The host sees FP4Q_ERR_TIMEOUT from
+the entry point's status call.  A normal call on the same workspace
+afterwards must return FP4Q_OK with output bit-identical to a call made
+before: the context stays usable.
+"""
+import numpy as np
+import pytest
+import torch
+
+from block_scaled_fp4_03_b200 import binding as fq
+from block_scaled_fp4_03_b200 import inputs
+from test_gpu_gemm import dev, quantized_operand, to_mma_layout
+
+pytestmark = pytest.mark.gpu
+
+TIMEOUT = 5
+
+
+class short_waits:
+    """Context manager: every bounded device wait gives up after one cycle."""
+
+    def __enter__(self):
+        self.prev = fq.debug_set_wait_cycles(1)
+
+    def __exit__(self, *exc):
+        fq.debug_set_wait_cycles(self.prev)
+
+
+def gemm_operands(O, M, N, K):
+    a32 = inputs.as_f32(inputs.generate("gemm_act", M, K, seed=40))
+    w32 = inputs.as_f32(inputs.generate("gemm_weight", N, K, seed=41))
+    qa, ga = quantized_operand(O, a32, O.RULE_FOUR_OVER_SIX)
+    qw, gw = quantized_operand(O, w32, O.RULE_ABSMAX)
+    args = (dev(qa["codes"]), dev(qw["codes"]), dev(to_mma_layout(qw["scales"])), dev(np.array([gw], np.float32)))
+    kw = dict(a_scales=dev(to_mma_layout(qa["scales"])), a_global_scale=dev(np.array([ga], np.float32)))
+    return args, kw
+
+
+# M = 128: the single-CTA kernel; M = 256: the CTA-pair kernel.  K = 4096 gives
+# each tile a 16-step main loop, so the epilogue's wait for the accumulator
+# cannot be satisfied at its first test.
+@pytest.mark.parametrize("M", [128, 256])
+@pytest.mark.parametrize("mx", [False, True])
+def test_gemm_wait_gives_up_and_reports_timeout(O, M, mx):
+    N, K = 512, 4096
+    ws = torch.zeros(8192, dtype=torch.uint8, device="cuda")
+    if mx:
+        x32 = inputs.as_f32(inputs.generate("mx_act", M, K, seed=42))
+        w32 = inputs.as_f32(inputs.generate("mx_weight", N, K, seed=43))
+        qa = O.mxfp4_quantize(x32, None, True, O.RULE_ABSMAX, want_deq=False, want_mse=False)
+        qw = O.mxfp4_quantize(w32, None, True, O.RULE_ABSMAX, want_deq=False, want_mse=False)
+        args = (dev(qa["codes"]), dev(qw["codes"]), dev(to_mma_layout(qw["scales"])))
+
+        def run():
+            return fq.mxfp4_gemm(*args, a_scales=dev(to_mma_layout(qa["scales"])), workspace=ws)
+    else:
+        args, kw = gemm_operands(O, M, N, K)
+
+        def run():
+            return fq.w4a4_gemm(*args, workspace=ws, **kw)
+    ref = run()
+    assert fq.gemm_status(ws) == 0
+    with short_waits():
+        run()
+        st = fq.gemm_status(ws)
+    assert st == TIMEOUT, st
+    again = run()
+    assert fq.gemm_status(ws) == 0
+    assert torch.equal(again.view(torch.int16), ref.view(torch.int16))
+
+
+def test_razer_two_pass_gemm_wait_gives_up(O):
+    """The multi-pass K loop (RaZeR weights: two passes) winds down the same way."""
+    M, N, K = 256, 512, 2048
+    args, kw = gemm_operands(O, M, N, K)
+    a_codes, w_codes, w_sc, gw = args
+    ws = torch.zeros(8192, dtype=torch.uint8, device="cuda")
+
+    def run():
+        return fq.razer_w4a4_gemm(a_codes, kw["a_scales"], kw["a_global_scale"], w_codes, w_sc, gw,
+                                  w_extra=w_codes, workspace=ws)
+    ref = run()
+    assert fq.gemm_status(ws) == 0
+    with short_waits():
+        run()
+        st = fq.gemm_status(ws)
+    assert st == TIMEOUT, st
+    again = run()
+    assert fq.gemm_status(ws) == 0
+    assert torch.equal(again.view(torch.int16), ref.view(torch.int16))
+
+
+def test_hessian_wait_gives_up_and_reports_timeout():
+    """H' blocks: the CTAs that gave up leave NaN blocks and the error word set."""
+    rows, cols = 2048, 256
+    x = dev(inputs.generate("mx_act", rows, cols, seed=44))
+    t = dev(inputs.positive_vector(cols, seed=45))
+    ws = torch.empty(fq.workspace_size(fq.OP_HESSIAN, rows, cols), dtype=torch.uint8, device="cuda")
+    ref = fq.hessian_blocks(x, t, True, workspace=ws)
+    assert fq.hessian_status(ws) == 0
+    assert torch.isfinite(ref).all()
+    with short_waits():
+        bad = fq.hessian_blocks(x, t, True, workspace=ws)
+        st = fq.hessian_status(ws)
+    assert st == TIMEOUT, st
+    assert torch.isnan(bad).any()
+    again = fq.hessian_blocks(x, t, True, workspace=ws)
+    assert fq.hessian_status(ws) == 0
+    assert torch.equal(again.view(torch.int32), ref.view(torch.int32))
