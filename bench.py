@@ -96,15 +96,17 @@ class Row:
     """One hot-path row: how to launch it on device buffers and what it moves."""
 
     def __init__(self, name, kernel, units, bytes_, launches, fn, out, bound="hbm", flops=0.0, evals=0.0,
-                 eval_ws=None, block=0, extra=False):
+                 eval_ws=None, block=0, extra=False, standalone=False):
         self.name, self.kernel, self.units, self.bytes, self.launches = name, kernel, units, bytes_, launches
         self.fn, self.out, self.bound, self.flops, self.evals = fn, out, bound, flops, evals
         # brute force: workspace whose counter at FP4Q_WS_BF_EVALS receives the
         # number of (block, candidate) error evaluations a call performs
         self.eval_ws, self.block = eval_ws, block
-        # rows beyond the hot path proper (the next rows built on it): timed
-        # and reported per row, outside the step and its value
+        # rows beyond the hot path proper (the next rows built on it, and the
+        # standalone form of a step that the hot path runs fused): timed and
+        # reported per row, outside the step and its value
         self.extra = extra
+        self.standalone = standalone
         # the step's input tensors (keys of X) this row reads; set per workload
         self.inputs = []
 
@@ -139,6 +141,16 @@ def build_rows(torch, fq, inputs, dev, host_copies=None, groups=None):
             o1.update(fq.nvfp4_quantize(X["c1"], 16, fq.PREVENT_ZERO, gs_mode=fq.GS_AMAX, dequant=True,
                                         mse=True, out=o1, workspace=ws1))
         rows.append(Row("c1_nvfp4_pz_deq_mse", "nvfp4_quant_kernel<16, float, 1, 0>", n1, n1 * (4 + 0.5 + 1 / 16 + 4 + 4 / 16), 2, c1, o1))
+        # the standalone dequantizer (fp4_dequant_mse) on that output: codes,
+        # scales and g in, the reference x in for the MSE, dequant and MSE out
+        od1 = {"dequant": torch.empty(a1.shape, dtype=torch.float32, device=dev),
+               "mse": torch.empty((a1.shape[0], a1.shape[1] // 16), dtype=torch.float32, device=dev)}
+
+        def c1d():
+            fq.dequant_mse(o1["codes"], o1["scales"], a1.shape[0], a1.shape[1], 16, fq.SF_E4M3,
+                           global_scale=o1["global_scale"], ref=X["c1"], out=od1)
+        rows.append(Row("c1_dequant_mse", "dequant_kernel<16, 0, false, float>", n1,
+                        n1 * (0.5 + 1 / 16 + 4 + 4 + 4 / 16), 1, c1d, od1, extra=True, standalone=True))
     set_inputs(n0, [k for k in ("c1",) if k in X])
     n0 = len(rows)
     if groups is None or "c2" in groups:
@@ -156,9 +168,11 @@ def build_rows(torch, fq, inputs, dev, host_copies=None, groups=None):
                 def c2(B=B, rule=rule, o=o, wsr=wsr):
                     o.update(fq.nvfp4_quantize(X["c2"], B, rule, gs_mode=fq.GS_NONE, mse=True, out=o, workspace=wsr))
                 kern = ("nvfp4_bf_kernel<%d, float, 0>" % B) if bf else ("nvfp4_quant_kernel<%d, float, %d, 0>" % (B, rule))
+                # brute force is held to the HBM roofline like the other rules (the
+                # evaluations it performs are reported beside it, not as its bound)
                 rows.append(Row("c2_B%d_%s" % (B, names[rule]), kern,
                                 n2, n2 * (4 + 0.5 + 1 / B + 4 / B), 1, c2, o,
-                                bound="alu" if bf else "hbm", eval_ws=wsr, block=B))
+                                bound="hbm", eval_ws=wsr, block=B))
         # the summary's comparison: UE5M3 block scales without a global scale
         # against E4M3 with 4-over-6 and hierarchical (global) scaling
         wsh2 = torch.empty(fq.workspace_size(fq.OP_QUANTIZE, 1, 1), dtype=torch.uint8, device=dev)
@@ -663,7 +677,7 @@ def main():
             d["TFLOP_s"] = r.flops / (ms * 1e-3) / 1e12
         row_out[r.name] = d
     for r in extra:
-        row_out[r.name]["next_row"] = True
+        row_out[r.name]["standalone_call" if r.standalone else "next_row"] = True
     dom = max(hot, key=lambda r: row_out[r.name]["ms"])
     dms = row_out[dom.name]["ms"]
     # fp32 pipe: 148 SMs x 128 lanes x clock; one element-candidate evaluation of

@@ -259,11 +259,17 @@ def channel_scale(x: torch.Tensor, w: torch.Tensor, alpha: float = 0.75, out=Non
 
 def dequant_mse(codes: torch.Tensor, scales: torch.Tensor, rows: int, cols: int, block: int,
                 scale_fmt: int, specials=None, global_scale: torch.Tensor | None = None,
-                ref: torch.Tensor | None = None, want_dequant: bool = True, stream=None) -> dict:
+                ref: torch.Tensor | None = None, want_dequant: bool = True, stream=None,
+                out: dict | None = None) -> dict:
+    """Dequantized values (and, given the reference, per-block MSE) of packed codes;
+    returns dict(dequant, mse).  `out` may supply the output tensors."""
     _need_cuda(codes, scales, global_scale, ref)
     dev = codes.device
-    dq = torch.empty((rows, cols), dtype=torch.float32, device=dev) if want_dequant else None
-    ms = torch.empty((rows, cols // block), dtype=torch.float32, device=dev) if ref is not None else None
+    o = out or {}
+    dq = (o.get("dequant") if o.get("dequant") is not None else
+          torch.empty((rows, cols), dtype=torch.float32, device=dev)) if want_dequant else None
+    ms = (o.get("mse") if o.get("mse") is not None else
+          torch.empty((rows, cols // block), dtype=torch.float32, device=dev)) if ref is not None else None
     sp = None
     n_sp = 0
     if specials is not None:

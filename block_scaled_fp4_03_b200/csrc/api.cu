@@ -19,7 +19,13 @@ cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
 int from_cuda(cudaError_t e) { return e == cudaSuccess ? FP4Q_OK : FP4Q_ERR_CUDA; }
 
-constexpr size_t kQuantWs = 4096;   // >= kAmaxPartials floats, rounded up
+// Quantize workspace: [0, 4096) the partial maxima of a separate amax pass,
+// FP4Q_WS_BF_EVALS the brute-force evaluation counter, kQuantCounter the
+// fused amax's grid-barrier counter, [kQuantFused, +4 * kFusedMaxCtas) the
+// fused amax's per-CTA maxima.
+constexpr size_t kQuantWs = 8192;
+constexpr size_t kQuantCounter = 3584;
+constexpr size_t kQuantFused = 4096;
 // Flip-Refinement: a row's state lives in shared memory (5 bytes per column
 // per row, 4 rows per CTA), and a row's move budget is bounded
 constexpr int64_t kFlipMaxCols = 8192;
@@ -29,13 +35,53 @@ constexpr int kFlipMaxMoves = 1 << 20;
 constexpr size_t kGemmHeader = 8192;
 constexpr size_t kGemmGa = 4096;
 constexpr size_t kGemmErr = 4160;
+constexpr size_t kGemmCounter = 4168;   // fused amax of the dense A: barrier counter
+constexpr size_t kGemmFused = 4224;     // and per-CTA maxima
 // Hessian workspace: [0, 256) header (error word at 0), then the partial sums.
 constexpr size_t kHessHeader = 256;
 bool valid_out_dtype(int d) { return d == FP4Q_BF16 || d == FP4Q_F32; }
 size_t gemm_ws_bytes(int64_t M, int64_t K) { return kGemmHeader + (size_t)M * (size_t)K / 2 + (size_t)M * (size_t)K / 16; }
 size_t mx_gemm_ws_bytes(int64_t M, int64_t K) { return kGemmHeader + (size_t)M * (size_t)K / 2 + (size_t)M * (size_t)K / 32; }
-static_assert(kAmaxPartials * sizeof(float) <= FP4Q_WS_BF_EVALS && FP4Q_WS_BF_EVALS + 8 <= kQuantWs,
-              "amax partials and the evaluation counter must fit");
+static_assert(kAmaxPartials * sizeof(float) <= FP4Q_WS_BF_EVALS && FP4Q_WS_BF_EVALS + 8 <= kQuantCounter &&
+                  kQuantCounter + 4 <= kQuantFused && kQuantFused + 4 * kFusedMaxCtas <= kQuantWs,
+              "quantize workspace regions must not overlap");
+static_assert(kGemmErr + 4 <= kGemmCounter && kGemmCounter + 4 <= kGemmFused &&
+                  kGemmFused + 4 * kFusedMaxCtas <= kGemmHeader,
+              "GEMM workspace header regions must not overlap");
+
+// A fused global amax (GsArgs mode 3) whose partials and barrier counter live
+// in the workspace at the given offsets; the counter is cleared on `s`.
+cudaError_t fused_gs(GsArgs& gs, const void* x, int64_t n, uint8_t* ws, size_t fused_off, size_t counter_off,
+                     cudaStream_t s)
+{
+    gs.mode = 3;
+    gs.x = x;
+    gs.n = n;
+    gs.fused_partials = reinterpret_cast<float*>(ws + fused_off);
+    gs.counter = reinterpret_cast<unsigned int*>(ws + counter_off);
+    gs.wait_limit = wait_limit_cycles();
+    return cudaMemsetAsync(gs.counter, 0, sizeof(unsigned int), s);
+}
+
+// Run a quantizer launch; if its fused amax cannot be launched cooperatively
+// here (the device holds fewer resident CTAs than its grid, e.g. when shared
+// under MPS), fall back to a separate amax pass whose partials go to
+// ws[0, 4 * kAmaxPartials).
+template <typename F>
+cudaError_t launch_with_gs(GsArgs& gs, const void* x, int dtype, int64_t n, void* ws, cudaStream_t s, F&& launch)
+{
+    cudaError_t e = launch(gs);
+    if (e == cudaErrorCooperativeLaunchTooLarge && gs.mode == 3) {
+        (void)cudaGetLastError();
+        gs.mode = 1;
+        gs.partials = reinterpret_cast<const float*>(ws);
+        gs.n_partials = kAmaxPartials;
+        e = launch_amax(x, dtype, n, reinterpret_cast<float*>(ws), s);
+        if (e == cudaSuccess)
+            e = launch(gs);
+    }
+    return e;
+}
 
 // Resolve a global-scale request into launch arguments (running the amax
 // pre-pass for AMAX).  Returns FP4Q_OK or an error.
@@ -59,10 +105,8 @@ int prepare_gs(int gs_mode, float denom, const void* x, int dtype, int64_t n, fl
         return FP4Q_ERR_WORKSPACE;
     if (!aligned16(ws))
         return FP4Q_ERR_ALIGN;
-    gs.partials = reinterpret_cast<const float*>(ws);
-    gs.n_partials = kAmaxPartials;
     gs.out = global_scale;
-    return from_cuda(launch_amax(x, dtype, n, reinterpret_cast<float*>(ws), s));
+    return from_cuda(fused_gs(gs, x, n, static_cast<uint8_t*>(ws), kQuantFused, kQuantCounter, s));
 }
 
 }  // namespace
@@ -137,9 +181,10 @@ int fp4_block_quantize(const void* x, int dtype, int64_t rows, int64_t cols, int
         (workspace && workspace_bytes >= kQuantWs)
             ? reinterpret_cast<unsigned long long*>(static_cast<uint8_t*>(workspace) + FP4Q_WS_BF_EVALS)
             : nullptr;
-    return from_cuda(launch_nvfp4_quant(x, dtype, rows, cols, block, rule, gs, codes, scales,
-                                        sf_layout == FP4Q_SFLAYOUT_MMA, dequant, block_mse, evals, s,
-                                        ue5m3 ? 1 : 0));
+    return from_cuda(launch_with_gs(gs, x, dtype, rows * cols, workspace, s, [&](const GsArgs& g) {
+        return launch_nvfp4_quant(x, dtype, rows, cols, block, rule, g, codes, scales,
+                                  sf_layout == FP4Q_SFLAYOUT_MMA, dequant, block_mse, evals, s, ue5m3 ? 1 : 0);
+    }));
 }
 
 int nvfp4_quantize(const void* x, int dtype, int64_t rows, int64_t cols, int block, int rule,
@@ -190,8 +235,10 @@ int razer_quantize(const void* x, int dtype, int64_t rows, int64_t cols, int sca
                         workspace_bytes, s, gs);
     if (st != FP4Q_OK)
         return st;
-    return from_cuda(launch_razer_quant(x, dtype, rows, cols, scale_fmt, specials, n_special, gs,
-                                        codes, meta, dequant, block_mse, s));
+    return from_cuda(launch_with_gs(gs, x, dtype, rows * cols, workspace, s, [&](const GsArgs& g) {
+        return launch_razer_quant(x, dtype, rows, cols, scale_fmt, specials, n_special, g, codes, meta, dequant,
+                                  block_mse, s);
+    }));
 }
 
 int mxfp4_quantize(const void* x, int dtype, int64_t rows, int64_t cols,
@@ -357,15 +404,14 @@ int w4a4_gemm(const void* a, int a_format, int a_rule, const uint8_t* a_scales,
         uint8_t* qsf = qcodes + (size_t)M * (size_t)K / 2;
         float* g = reinterpret_cast<float*>(ws + kGemmGa);
         GsArgs gs{};
-        gs.mode = FP4Q_GS_AMAX;
         gs.denom = 2688.0f;
-        gs.partials = reinterpret_cast<const float*>(ws);
-        gs.n_partials = kAmaxPartials;
         gs.out = g;
-        cudaError_t e = launch_amax(a, a_format, M * K, reinterpret_cast<float*>(ws), s);
+        cudaError_t e = fused_gs(gs, a, M * K, ws, kGemmFused, kGemmCounter, s);
         if (e == cudaSuccess)
-            e = launch_nvfp4_quant(a, a_format, M, K, 16, a_rule, gs, qcodes, qsf, 1, nullptr,
-                                   nullptr, nullptr, s);
+            e = launch_with_gs(gs, a, a_format, M * K, ws, s, [&](const GsArgs& gg) {
+                return launch_nvfp4_quant(a, a_format, M, K, 16, a_rule, gg, qcodes, qsf, 1, nullptr, nullptr,
+                                          nullptr, s);
+            });
         if (e != cudaSuccess)
             return FP4Q_ERR_CUDA;
         a_codes = qcodes;

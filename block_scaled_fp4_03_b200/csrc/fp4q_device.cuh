@@ -298,6 +298,35 @@ __device__ __forceinline__ void warp_load_blocks(const T* __restrict__ x, int64_
     }
 }
 
+// The converse of warp_load_blocks for fp32 outputs of B elements per block
+// (B = 8, 16 or 32): the warp's lanes put their blocks into `buf` (this warp's
+// 32 * B * 4 bytes of shared memory) and the warp writes the 32 blocks as
+// whole rows, 512 consecutive bytes per store instruction; blocks at or past
+// nblk are not written.  A lane storing its own 32-128 contiguous bytes would
+// touch 16-32 different 32-byte sectors per warp instruction.
+template <int B>
+__device__ __forceinline__ void warp_store_f32_blocks(float* __restrict__ out, int64_t base, int64_t nblk,
+                                                      uint4* buf, const float (&v)[B])
+{
+    constexpr int CPB = B / 4;
+    const int lane = threadIdx.x & 31;
+    const int64_t left = nblk - base;
+    const int nb = left < 32 ? (int)left : 32;
+    __syncwarp();   // the buffer's previous contents have been read
+#pragma unroll
+    for (int p = 0; p < CPB; ++p)
+        buf[staged_slot<CPB>(lane, p)] = make_uint4(__float_as_uint(v[4 * p]), __float_as_uint(v[4 * p + 1]),
+                                                    __float_as_uint(v[4 * p + 2]), __float_as_uint(v[4 * p + 3]));
+    __syncwarp();
+    uint4* dst = reinterpret_cast<uint4*>(out + base * B);
+#pragma unroll
+    for (int k = 0; k < CPB; ++k) {
+        const int c = lane + 32 * k;
+        if (c / CPB < nb)
+            dst[c] = buf[staged_slot<CPB>(c / CPB, c % CPB)];
+    }
+}
+
 template <int N>
 __device__ __forceinline__ void store_f32(float* __restrict__ p, const float (&x)[N])
 {

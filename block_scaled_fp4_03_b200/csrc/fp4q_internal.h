@@ -18,16 +18,26 @@ long long wait_limit_cycles();
 
 // Global-scale source for a quantizer launch.
 struct GsArgs {
-    int mode;                 // 0 none (g = 1), 1 amax partials in ws, 2 given (device float)
+    int mode;                 // 0 none (g = 1), 1 amax partials in ws, 2 given (device float),
+                              // 3 amax computed in the quantizer launch itself (fused)
     const float* partials;    // mode 1: per-CTA block maxima written by launch_amax
     int n_partials;
-    float denom;              // mode 1: 6 * largest scale of the format (2688 or 180)
+    float denom;              // modes 1, 3: 6 * largest scale of the format (2688, 180, 6 * 114688)
     const float* given;       // mode 2
     float* out;               // nullable: where to write the g that was used
+    // mode 3: the whole input (n elements), one partial maximum per CTA, and the
+    // grid barrier's arrival counter (zero before the launch)
+    const void* x;
+    int64_t n;
+    float* fused_partials;
+    unsigned int* counter;
+    long long wait_limit;
 };
 
 // Number of partial maxima launch_amax writes (fixed; the workspace holds them).
 constexpr int kAmaxPartials = 592;   // 148 SMs x 4
+// Largest grid of a fused-amax quantizer launch (its partials area holds this many).
+constexpr int kFusedMaxCtas = 960;
 
 // SM count of the current device (cached per device).
 int num_sms();

@@ -16,7 +16,10 @@
 // packed in registers by the hardware e2m1x2 conversion and written with one
 // vector store per block.
 #include <cfloat>
+#include <cmath>
 #include <cstdint>
+#include <mutex>
+#include <utility>
 
 #include "fp4q_device.cuh"
 #include "fp4q_internal.h"
@@ -35,7 +38,132 @@ __device__ __forceinline__ float warp_max(float v)
     return v;
 }
 
+// max |x| over the 16-byte vectors [v0, v1) of x, this CTA's threads
+// striding by the block size with eight loads in flight per thread (the
+// quantizer grids hold only 2-5 CTAs per SM).
+template <typename T>
+__device__ float cta_amax_part(const T* __restrict__ x, int64_t v0, int64_t v1)
+{
+    const uint4* xv = reinterpret_cast<const uint4*>(x);
+    float m = 0.0f;
+    auto fold = [&](const uint4& w) {
+        if constexpr (sizeof(T) == 4) {
+            m = fmaxf(m, fmaxf(fmaxf(fabsf(__uint_as_float(w.x)), fabsf(__uint_as_float(w.y))),
+                               fmaxf(fabsf(__uint_as_float(w.z)), fabsf(__uint_as_float(w.w)))));
+        } else {
+            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                float lo, hi;
+                bf16x2_to_f32(ww[q], lo, hi);
+                m = fmaxf(m, fmaxf(fabsf(lo), fabsf(hi)));
+            }
+        }
+    };
+    const int64_t st = blockDim.x;
+    int64_t i = v0 + threadIdx.x;
+    for (; i + 7 * st < v1; i += 8 * st) {
+        uint4 w[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            w[u] = __ldg(xv + i + u * st);
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+            fold(w[u]);
+    }
+    for (; i < v1; i += st)
+        fold(__ldg(xv + i));
+    return m;
+}
+
+// max |x| of the elements past the last whole 16-byte vector.
+template <typename T>
+__device__ float amax_tail(const T* __restrict__ x, int64_t n)
+{
+    constexpr int V = 16 / sizeof(T);
+    float m = 0.0f;
+    for (int64_t i = n / V * V + threadIdx.x; i < n; i += blockDim.x) {
+        float f;
+        if constexpr (sizeof(T) == 4)
+            f = reinterpret_cast<const float*>(x)[i];
+        else
+            f = __uint_as_float((uint32_t)reinterpret_cast<const uint16_t*>(x)[i] << 16);
+        m = fmaxf(m, fabsf(f));
+    }
+    return m;
+}
+
+// Maximum over the CTA (every thread gets it).
+__device__ __forceinline__ float cta_max(float m)
+{
+    __shared__ float red[kThreads / 32];
+    __shared__ float s_m;
+    m = warp_max(m);
+    if ((threadIdx.x & 31) == 0)
+        red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        m = threadIdx.x < (int)(blockDim.x >> 5) ? red[threadIdx.x] : 0.0f;
+        m = warp_max(m);
+        if (threadIdx.x == 0)
+            s_m = m;
+    }
+    __syncthreads();
+    return s_m;
+}
+
+// Fused global maximum (GsArgs mode 3): every CTA takes the maximum of its own
+// contiguous slice of x, publishes it and meets the others at a grid barrier
+// (the launch is cooperative, so all CTAs are resident); then each reduces all
+// partials.  The maximum is exact and order-free, so g is the same as from a
+// separate pass.  The barrier wait is bounded: a CTA that gives up computes
+// the maximum of the whole tensor itself (slower, same result).
+template <typename T>
+__device__ float fused_global_amax(const GsArgs& gs)
+{
+    __shared__ int s_alone;
+    const T* x = reinterpret_cast<const T*>(gs.x);
+    constexpr int V = 16 / sizeof(T);
+    const int64_t nvec = gs.n / V;
+    const int64_t per = (nvec + gridDim.x - 1) / gridDim.x;
+    const int64_t v0 = (int64_t)blockIdx.x * per < nvec ? (int64_t)blockIdx.x * per : nvec;
+    const int64_t v1 = v0 + per < nvec ? v0 + per : nvec;
+    float m = cta_amax_part<T>(x, v0, v1);
+    if (blockIdx.x == 0)
+        m = fmaxf(m, amax_tail<T>(x, gs.n));
+    m = cta_max(m);
+    if (threadIdx.x == 0) {
+        gs.fused_partials[blockIdx.x] = m;
+        __threadfence();
+        atomicAdd(gs.counter, 1u);
+        int alone = 0;
+        const long long t0 = clock64();
+        for (;;) {
+            unsigned int c;
+            asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(c) : "l"(gs.counter) : "memory");
+            if (c >= gridDim.x)
+                break;
+            if (clock64() - t0 > gs.wait_limit) {
+                alone = 1;
+                break;
+            }
+        }
+        s_alone = alone;
+    }
+    __syncthreads();
+    if (s_alone) {
+        m = cta_amax_part<T>(x, 0, nvec);
+        m = fmaxf(m, amax_tail<T>(x, gs.n));
+    } else {
+        m = 0.0f;
+        for (int i = threadIdx.x; i < (int)gridDim.x; i += blockDim.x)
+            m = fmaxf(m, __ldcg(gs.fused_partials + i));
+    }
+    return cta_max(m);
+}
+
 // The per-tensor global scale for this launch (all threads of the CTA get it).
+template <typename T>
 __device__ float resolve_global_scale(const GsArgs& gs)
 {
     __shared__ float s_g;
@@ -43,6 +171,19 @@ __device__ float resolve_global_scale(const GsArgs& gs)
         return 1.0f;
     if (gs.mode == 2)
         return __ldg(gs.given);
+    if (gs.mode == 3) {
+        const float m = fused_global_amax<T>(gs);
+        if (threadIdx.x == 0) {
+            float g = __fdiv_rn(m, gs.denom);
+            if (!(g > 0.0f))
+                g = 1.0f;
+            s_g = g;
+            if (blockIdx.x == 0 && gs.out)
+                *gs.out = g;
+        }
+        __syncthreads();
+        return s_g;
+    }
     if (threadIdx.x < 32) {
         float m = 0.0f;
         for (int i = threadIdx.x; i < gs.n_partials; i += 32)
@@ -234,16 +375,22 @@ nvfp4_quant_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs
                    uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, int mma_layout,
                    float* __restrict__ deq, float* __restrict__ mse)
 {
-    const float g = resolve_global_scale(gs);
+    const float g = resolve_global_scale<T>(gs);
     const float g6 = __fmul_rn(6.0f, g);
     const float g4 = __fmul_rn(4.0f, g);
     const int lane = threadIdx.x & 31;
     const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
     const int64_t kb_atoms = (bpr + 3) >> 2;
-    // blocks of 128 bytes or more are loaded warp-cooperatively through shared memory
+    // blocks of 128 bytes or more are loaded warp-cooperatively through shared
+    // memory; dequantized blocks of 32 bytes or more are stored that way too
+    // (the same buffer, sized for the larger of the two)
     constexpr bool kStaged = B * sizeof(T) >= 128;
-    __shared__ uint4 stage_buf[kStaged ? kThreads / 32 : 1][kStaged ? 2 * B * (int)sizeof(T) : 1];
+    constexpr bool kStoreStaged = B >= 8;
+    constexpr int kBufChunks = (kStaged ? 2 * B * (int)sizeof(T) : 1) > (kStoreStaged ? 8 * B : 1)
+                                   ? (kStaged ? 2 * B * (int)sizeof(T) : 1)
+                                   : (kStoreStaged ? 8 * B : 1);
+    __shared__ uint4 stage_buf[kThreads / 32][kBufChunks];
     // small blocks (one or two 16-byte loads per lane): keep the next block's
     // load in flight while this one is quantized
     constexpr bool kPrefetch = !kStaged && B * sizeof(T) <= 32;
@@ -334,10 +481,14 @@ nvfp4_quant_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs
             store_codes<B>(codes + b * (B / 2), cw);
             const int64_t so = mma_layout ? mma_sf_offset(r_cur, kb_cur, kb_atoms) : b;
             scales[so] = (uint8_t)sc;
-            if (deq)
+            if (!kStoreStaged && deq)
                 store_f32<B>(deq + b * B, dq);
             if (mse)
                 mse[b] = __fmul_rn(sse, 1.0f / (float)B);
+        }
+        if constexpr (kStoreStaged) {
+            if (deq)
+                warp_store_f32_blocks<B>(deq, base, nblk, stage_buf[threadIdx.x >> 5], dq);
         }
         if (mma_layout) {
             kb_cur += step_kb;
@@ -377,7 +528,7 @@ razer_quant_kernel(const T* __restrict__ x, int64_t nblk, GsArgs gs, SpecialArgs
                    float* __restrict__ deq, float* __restrict__ mse)
 {
     constexpr int B = 16;
-    const float g = resolve_global_scale(gs);
+    const float g = resolve_global_scale<T>(gs);
     const float g6 = __fmul_rn(6.0f, g);
     const int lane = threadIdx.x & 31;
     const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -580,7 +731,7 @@ razer_paired_kernel(const T* __restrict__ x, int64_t nblk, GsArgs gs, SpecialArg
                     float* __restrict__ deq, float* __restrict__ mse)
 {
     constexpr int B = 16;
-    const float g = resolve_global_scale(gs);
+    const float g = resolve_global_scale<T>(gs);
     const float g6 = __fmul_rn(6.0f, g);
     const int lane = threadIdx.x & 31;
     const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -702,8 +853,8 @@ razer_paired_kernel(const T* __restrict__ x, int64_t nblk, GsArgs gs, SpecialArg
 
 // ------------------------------------------------------- brute-force scale
 // Brute force over the scale format's codes (E4M3 1..126, UE5M3 1..254): the
-// least in-order squared error, ties
-// to the lowest code.  Exact shortcuts (each provably skips only losers):
+// least in-order squared error, ties to the lowest code.  Exact shortcuts
+// (each provably skips only codes that cannot win):
 //  * from the first code at which the largest element rounds to zero
 //    (|y| <= 0.25; |y| falls as the code grows) every element does, so that
 //    code gives the all-zero error (the in-order sum of x^2) and every higher
@@ -712,45 +863,142 @@ razer_paired_kernel(const T* __restrict__ x, int64_t nblk, GsArgs gs, SpecialArg
 //    a - 6S grows as the code falls, and its square alone bounds the in-order
 //    fma chain from below (the chain only adds non-negative terms and
 //    rounding is monotone): the downward scan from c6 stops at the first
-//    code whose bound already loses against c6 or the all-zero code.
-// Every code left in between is evaluated in full.  Load balance: the ranges
-// of a warp's 32 blocks differ widely (a heavy-tailed block spans far more
-// codes), so the warp lays all (block, code) pairs end to end and every lane
-// takes every 32nd pair, reading the block from shared memory.  A block's
-// best (error, code) is one 64-bit key -- error bits (non-negative floats
-// order like their bits) above the code -- lowered with a shared-memory
-// atomic minimum, so the lowest code wins ties exactly as in a sequential
-// scan.
+//    code whose bound already loses against c6 or the all-zero code;
+//  * codes above c6 that no element can prefer: when g and the scale S_r of
+//    c6 are powers of two (so x / S_r is exact and c6's encode picks, for every
+//    element, the nearest point of its grid S_r G, G = {0, .5, 1, 1.5, 2, 3,
+//    4, 6}) and no element clips at c6 (a <= 6 S_r), a code c with grid S_c G
+//    can bring an element nearer only through a point p of S_c G in
+//    (0, 6 S_r) that S_r G lacks, and only for elements strictly inside the
+//    window between the midpoints of p and its two neighbours in S_r G (past
+//    6 S_r every point is farther than 6 S_r itself).  If no element of the
+//    block lies in any window of c, every |x_i - q_c(x_i)| >= |x_i -
+//    q_r(x_i)|; the rounded errors and their in-order fma chain keep that
+//    order, and a tie goes to the lower code c6, so c cannot win.  With
+//    k = S_c / S_r the windows depend on k alone, and k depends only on the
+//    offset of c from c6 and on whether c6 is a normal power of two or the
+//    subnormal code 1, 2 or 4 (the same in E4M3 and UE5M3, both with three
+//    mantissa bits).  BfWindows holds, per reference type and per 1/8-wide
+//    bin of |x| / S_r in [0, 6], the mask of code offsets whose windows meet
+//    the bin; a block ORs the masks of its elements' bins.  Codes with
+//    k in {2, 4, 6, 8, 12} or k >= 13 add no point below 6 S_r and never
+//    appear in a mask.
+// Every other code of [clo, all-zero code) is evaluated in full: each lane
+// takes the first kDirect of its block's codes from registers; the rest of
+// the warp's (block, code) pairs are laid end to end and every lane takes
+// every 32nd pair, reading the block from shared memory.  A block's best
+// (error, code) is one 64-bit key -- error bits (non-negative floats order
+// like their bits) above the code -- lowered with a shared-memory atomic
+// minimum, so the lowest code wins ties exactly as in a sequential scan.  The
+// seed c6 is evaluated with its codes kept: most blocks keep c6 and are
+// stored without a second encode.
 constexpr int kWarps = kThreads / 32;
 
+// Codes and in-order squared error of a block at the candidate t = (S, inv).
+template <int B>
+__device__ __forceinline__ float quant_codes_sse(const float (&x)[B], float2 t, uint32_t (&cw)[(B + 7) / 8])
+{
+    const float S = t.x;
+    const float inv = t.y;
+    float acc = 0.0f;
+    if constexpr (B == 4) {
+        const uint32_t w = e2m1x4_encode(__fmul_rn(x[0], inv), __fmul_rn(x[1], inv),
+                                         __fmul_rn(x[2], inv), __fmul_rn(x[3], inv));
+        float v[4];
+        e2m1x4_decode(w, v);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float e = __fsub_rn(x[i], __fmul_rn(v[i], S));
+            acc = __fmaf_rn(e, e, acc);
+        }
+        cw[0] = w;
+    } else {
+#pragma unroll
+        for (int j = 0; j < B / 8; ++j) {
+            const int o = 8 * j;
+            const uint32_t w = e2m1x8_encode(__fmul_rn(x[o], inv), __fmul_rn(x[o + 1], inv),
+                                             __fmul_rn(x[o + 2], inv), __fmul_rn(x[o + 3], inv),
+                                             __fmul_rn(x[o + 4], inv), __fmul_rn(x[o + 5], inv),
+                                             __fmul_rn(x[o + 6], inv), __fmul_rn(x[o + 7], inv));
+            float v[8];
+            e2m1x8_decode(w, v);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float e = __fsub_rn(x[o + i], __fmul_rn(v[i], S));
+                acc = __fmaf_rn(e, e, acc);
+            }
+            cw[j] = w;
+        }
+    }
+    return acc;
+}
+
+// True when a fp32 value is a normal power of two in [2^-100, 2^100].
+__device__ __forceinline__ bool pow2_in_range(float v)
+{
+    const uint32_t u = __float_as_uint(v);
+    const uint32_t e = u >> 23;                  // sign bit included: negatives fail
+    return (u & 0x007FFFFFu) == 0u && e >= 127u - 100u && e <= 127u + 100u;
+}
+
+// Per reference type (0 a normal power of two, 1-3 the subnormal codes 1, 2,
+// 4) and per bin b of |x| / S_r (width 1/8, b = 0..48): bit j set when code
+// c6 + 1 + j has a window meeting the bin.
+struct BfWindows {
+    unsigned long long m[4][49];
+};
+
+// Reference type of a scale code (3 mantissa bits): 1 + type, 0 when its
+// scale is not a power of two.
+__device__ __forceinline__ uint32_t ref_type(uint32_t c)
+{
+    if (c >= 8u)
+        return (c & 7u) == 0u ? 1u : 0u;
+    if (c == 0u || (c & (c - 1u)) != 0u)
+        return 0u;
+    return 33u - (uint32_t)__clz((int)c);   // subnormal 1, 2, 4 -> 2, 3, 4
+}
+
+// Resident CTAs per SM the brute-force kernel is compiled for (its register cap).
+template <int B>
+constexpr int bf_min_ctas() { return B <= 4 ? 5 : B <= 8 ? 4 : B <= 16 ? 3 : 2; }
+
 template <int B, typename T, int SFMT>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, bf_min_ctas<B>())
 nvfp4_bf_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs,
                 uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, int mma_layout,
-                float* __restrict__ deq, float* __restrict__ mse, unsigned long long* evals)
+                float* __restrict__ deq, float* __restrict__ mse, unsigned long long* evals,
+                const __grid_constant__ BfWindows win)
 {
     uint32_t n_eval = 0;   // this lane's error evaluations (seed, all-zero, scan)
     // the format's largest finite code, and the "no all-zero code" marker
     constexpr uint32_t kLast = SFMT == 1 ? 254u : 126u;
-    // codes each lane evaluates itself before the warp shares out the rest
-    // (measured on the Student-t block sweep: 3 for B <= 8, 5 above)
-    constexpr int kDirect = B <= 8 ? 3 : 5;
+    // codes each lane may evaluate itself before the warp shares out the rest
+    constexpr int kDirect = B <= 8 ? 2 : 3;
     constexpr uint32_t kNone = kLast + 1u;
     // (S, inv) of every code: S = sc * g, inv = min(1/S, FLT_MAX), 0 for S = 0
     __shared__ float2 tab[kNone + 1];
+    // the window masks, in shared memory: lanes index them by their own bins,
+    // which constant-space reads would serialize
+    __shared__ unsigned long long wmask[4 * 49];
     __shared__ __align__(16) float xs[kWarps][32 * B];
     __shared__ unsigned long long key[kWarps][32];
     __shared__ int pre[kWarps][32];
-    __shared__ uint32_t meta[kWarps][32];   // clo | c6 << 8
+    __shared__ uint32_t lowm[kWarps][32];            // next lower code | lower count << 8 | c6 << 16
+    __shared__ unsigned long long upm[kWarps][32];   // upper codes left: bit j = code c6 + 1 + j
 
-    const float g = resolve_global_scale(gs);
+    const float g = resolve_global_scale<T>(gs);
     const float g6 = __fmul_rn(6.0f, g);
     // only a starting point for the exact all-zero search below
     const float four_over_g = __fmul_rn(4.0f, __frcp_rn(g));
+    // every S = sc * g and every v * S is exact when g is a moderate power of two
+    const bool g_pow2 = pow2_in_range(g);
     for (int c = threadIdx.x; c <= (int)kNone; c += blockDim.x) {
         const float S = __fmul_rn(sf_decode<SFMT>((uint32_t)c < kNone ? (uint32_t)c : kLast), g);
         tab[c] = make_float2(S, (S == 0.0f) ? 0.0f : fminf(__frcp_rn(S), kFltMax));
     }
+    for (int i = threadIdx.x; i < 4 * 49; i += blockDim.x)
+        wmask[i] = win.m[i / 49][i % 49];
     __syncthreads();
 
     const int lane = threadIdx.x & 31;
@@ -789,7 +1037,9 @@ nvfp4_bf_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs,
         }
         uint32_t c6 = sf_encode<SFMT>(__fdiv_rn(a, g6));
         c6 = c6 == 0u ? 1u : c6;
-        float best = quant_sse<B>(xv, 0.0f, 0.0f, tab[c6]);
+        const float2 t6 = tab[c6];
+        uint32_t cw[(B + 7) / 8];
+        float best = quant_codes_sse<B>(xv, t6, cw);
         uint32_t bc = c6;
         n_eval += valid ? 1u : 0u;
         // first all-zero code (kNone = none): step from a nearby code to the
@@ -829,15 +1079,54 @@ nvfp4_bf_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs,
                 break;
             --clo;
         }
-        int chi = (int)(cz < kNone ? cz : kNone) - 1;   // last code to evaluate
-        // the first kDirect codes of the range other than c6 straight from
-        // registers (most blocks need no more); the rest is shared out across
-        // the warp.  Code list: clo, clo + 1, ... with c6 left out.
+        // the block's code list: clo .. c6 - 1, then the codes of (c6, chi]
+        // the lattice shortcut leaves, as a mask over c6 + 1 + j
+        const int chi = (int)(cz < kNone ? cz : kNone) - 1;   // last code to evaluate
+        const int nup = valid ? chi - (int)c6 : 0;
+        unsigned long long um = nup <= 0 ? 0ull : nup >= 64 ? ~0ull : ((1ull << nup) - 1ull);
+        // c6 is a usable reference: a power-of-two scale with an exact
+        // reciprocal at which no element clips; then only the codes whose
+        // windows hold an element stay
+        const uint32_t ty = ref_type(c6);
+        const bool use_ref = g_pow2 && ty != 0u && __fmul_rn(t6.x, t6.y) == 1.0f && __fmul_rn(a, t6.y) <= 6.0f;
+        if (use_ref) {
+            unsigned long long allow = 0ull;
+#pragma unroll
+            for (int i = 0; i < B; ++i) {
+                // |x| / S_r <= 6 exactly, so the bin is 0 .. 48
+                const int bin = __float2int_rz(__fmul_rn(__fmul_rn(fabsf(xv[i]), t6.y), 8.0f));
+                allow |= wmask[(ty - 1u) * 49u + (uint32_t)bin];
+            }
+            um &= allow;
+        }
+        int nlow = valid ? (int)(c6 - clo) : 0;
+        uint32_t lo_next = clo;
+        // codes past c6 + 64 (all with k >= 13, so never in a window, for a
+        // usable reference): in practice no block has any, its range above c6
+        // being at most about 40 codes in either format
+        for (int c = (int)c6 + 65; c <= chi && valid && !use_ref; ++c) {
+            const float sc_ = quant_sse<B>(xv, 0.0f, 0.0f, tab[c]);
+            n_eval += 1u;
+            if (sc_ < best || (sc_ == best && (uint32_t)c < bc)) {
+                best = sc_;
+                bc = (uint32_t)c;
+            }
+        }
+        // the first kDirect codes of the list straight from registers (most
+        // warps have none left after the shortcuts)
 #pragma unroll
         for (int s = 0; s < kDirect; ++s) {
-            uint32_t c = clo + (uint32_t)s;
-            c += c >= c6 ? 1u : 0u;
-            if (valid && (int)c <= chi) {
+            if (!__any_sync(0xffffffffu, nlow > 0 || um != 0ull))
+                break;
+            uint32_t c = 0u;
+            if (nlow > 0) {
+                c = lo_next++;
+                --nlow;
+            } else if (um != 0ull) {
+                c = c6 + (uint32_t)__ffsll((long long)um);
+                um &= um - 1ull;
+            }
+            if (c != 0u) {
                 const float sc_ = quant_sse<B>(xv, 0.0f, 0.0f, tab[c]);
                 n_eval += 1u;
                 if (sc_ < best || (sc_ == best && c < bc)) {
@@ -846,11 +1135,9 @@ nvfp4_bf_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs,
                 }
             }
         }
-        // codes left after the direct ones (c6 <= chi unless the block is all zero)
-        int span = chi - (int)clo + 1 - ((int)c6 <= chi ? 1 : 0) - kDirect;
-        span = (valid && span > 0) ? span : 0;
+        const int span = nlow + __popcll(um);
 
-        // lay the warp's candidates end to end
+        // lay the warp's remaining candidates end to end
         int incl = span;
 #pragma unroll
         for (int d = 1; d < 32; d <<= 1) {
@@ -866,7 +1153,8 @@ nvfp4_bf_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs,
                     make_float4(xv[i], xv[i + 1], xv[i + 2], xv[i + 3]);
             key[w][lane] = ((unsigned long long)__float_as_uint(best) << 32) | bc;
             pre[w][lane] = incl - span;
-            meta[w][lane] = clo | (c6 << 8);   // clo <= c6 <= kLast: 8 bits each
+            lowm[w][lane] = lo_next | ((uint32_t)nlow << 8) | (c6 << 16);   // 8 bits each
+            upm[w][lane] = um;
             __syncwarp();
             for (int t = lane; t < total; t += 32) {
                 // owner: the last block whose range starts at or before t
@@ -875,9 +1163,18 @@ nvfp4_bf_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs,
                 for (int st = 16; st > 0; st >>= 1)
                     if (pre[w][j + st] <= t)
                         j += st;
-                const uint32_t m = meta[w][j];
-                uint32_t c = (m & 0xFFu) + (uint32_t)(kDirect + t - pre[w][j]);
-                c += c >= (m >> 8) ? 1u : 0u;
+                const uint32_t lm = lowm[w][j];
+                const int k = t - pre[w][j];
+                const int nl = (int)((lm >> 8) & 0xFFu);
+                uint32_t c;
+                if (k < nl) {
+                    c = (lm & 0xFFu) + (uint32_t)k;
+                } else {
+                    unsigned long long m = upm[w][j];
+                    for (int i = nl; i < k; ++i)
+                        m &= m - 1ull;
+                    c = ((lm >> 16) & 0xFFu) + (uint32_t)__ffsll((long long)m);
+                }
                 float xj[B];
 #pragma unroll
                 for (int i = 0; i < B; i += 4) {
@@ -896,9 +1193,12 @@ nvfp4_bf_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs,
             __syncwarp();
         }
 
-        uint32_t cw[(B + 7) / 8];
+        // c6 kept: its codes and error are already in registers
+        float sse = best;
         float dq[B];
-        const float sse = quant_eval<B>(xv, sf_decode<SFMT>(bc), g, cw, dq);
+        if (bc != c6 || deq) {
+            sse = quant_eval<B>(xv, sf_decode<SFMT>(bc), g, cw, dq);
+        }
         if (valid) {
             store_codes<B>(codes + b * (B / 2), cw);
             const int64_t so = mma_layout ? mma_sf_offset(r_cur, kb_cur, kb_atoms) : b;
@@ -933,12 +1233,26 @@ dequant_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ sc
                int64_t nblk, SpecialArgs sp, const float* __restrict__ gs_dev,
                const TR* __restrict__ ref, float* __restrict__ deq, float* __restrict__ mse)
 {
+    // warps walk 32 consecutive blocks at a time (a warp-uniform trip count),
+    // so blocks of 32 bytes or more of the reference are read, and the
+    // dequantized blocks written, as whole rows through shared memory
+    constexpr bool kRefStaged = B * sizeof(TR) >= 32;
+    constexpr bool kStoreStaged = B >= 8;
+    __shared__ uint4 buf[kThreads / 32][(kRefStaged || kStoreStaged) ? 8 * B : 1];
     const float g = gs_dev ? __ldg(gs_dev) : 1.0f;
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblk; b += stride) {
-        const uint32_t sb = __ldg(scales + b);
+    const int lane = threadIdx.x & 31;
+    const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    for (int64_t base = warp0 * 32; base < nblk; base += nwarps * 32) {
+        const int64_t b = base + lane;
+        const bool valid = b < nblk;
+        const uint32_t sb = valid ? __ldg(scales + b) : 0u;
         uint32_t cw[(B + 7) / 8];
-        if constexpr (B == 4) {
+        if (!valid) {
+#pragma unroll
+            for (int j = 0; j < (B + 7) / 8; ++j)
+                cw[j] = 0u;
+        } else if constexpr (B == 4) {
             cw[0] = __ldg(reinterpret_cast<const uint16_t*>(codes + b * 2));
         } else if constexpr (B == 8) {
             cw[0] = __ldg(reinterpret_cast<const uint32_t*>(codes + b * 4));
@@ -994,21 +1308,41 @@ dequant_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ sc
                 dq[i] = __fmul_rn(vi, S);
             }
         }
-        if (deq)
-            store_f32<B>(deq + b * B, dq);
         if (mse) {
             float xr[B];
-            load_elems<TR, B>(ref + b * B, xr);
+            if constexpr (kRefStaged) {
+                warp_load_blocks<TR, B>(ref, base, nblk, buf[threadIdx.x >> 5], xr);
+            } else if (valid) {
+                load_elems<TR, B>(ref + b * B, xr);
+            } else {
+#pragma unroll
+                for (int i = 0; i < B; ++i)
+                    xr[i] = 0.0f;
+            }
             float acc = 0.0f;
 #pragma unroll
             for (int i = 0; i < B; ++i) {
                 float e = __fsub_rn(xr[i], dq[i]);
                 acc = __fmaf_rn(e, e, acc);
             }
-            mse[b] = __fmul_rn(acc, 1.0f / (float)B);
+            if (valid)
+                mse[b] = __fmul_rn(acc, 1.0f / (float)B);
+        }
+        if (deq) {
+            if constexpr (kStoreStaged)
+                warp_store_f32_blocks<B>(deq, base, nblk, buf[threadIdx.x >> 5], dq);
+            else if (valid)
+                store_f32<B>(deq + b * B, dq);
         }
     }
 }
+
+// Launch a quantizer kernel over nblk blocks (one thread each) on a grid sized
+// by grid_for; a fused global amax (gs.mode 3) needs every CTA resident at
+// once, so that launch is cooperative and its grid at most kFusedMaxCtas.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_quant_kernel(void (*kernel)(KArgs...), int64_t nblk, const GsArgs& gs, cudaStream_t s,
+                                Args&&... args);
 
 int grid_for(int64_t work_threads, const void* kernel)
 {
@@ -1023,6 +1357,71 @@ int grid_for(int64_t work_threads, const void* kernel)
     return (int)(want < 1 ? 1 : want);
 }
 
+// The brute-force window masks (see BfWindows), computed once in exact
+// (dyadic, so exact in double) arithmetic.  Scale values in units of the
+// subnormal step s of a 3-mantissa-bit format: code c < 8 is c s, code
+// 8 + 8 d + m is 2^d (8 + m) s; a normal power-of-two reference behaves like
+// code 8 (its offsets repeat the same ratios).
+const BfWindows& bf_windows()
+{
+    static BfWindows w;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        const double G[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+        auto value = [](int c) { return c < 8 ? (double)c : std::ldexp((double)(8 + ((c - 8) & 7)), (c - 8) >> 3); };
+        const int ref_code[4] = {8, 1, 2, 4};
+        for (int t = 0; t < 4; ++t) {
+            for (int b = 0; b < 49; ++b)
+                w.m[t][b] = 0ull;
+            const int r = ref_code[t];
+            for (int j = 0; j < 64; ++j) {
+                const double k = value(r + 1 + j) / value(r);
+                for (int i = 1; i < 8; ++i) {
+                    const double p = k * G[i];
+                    bool on_grid = false;
+                    for (int q = 0; q < 8; ++q)
+                        on_grid = on_grid || G[q] == p;
+                    if (p >= 6.0 || on_grid)
+                        continue;
+                    double q1 = 0.0, q2 = 6.0;
+                    for (int q = 0; q < 8; ++q) {
+                        if (G[q] < p && G[q] > q1)
+                            q1 = G[q];
+                        if (G[q] > p && G[q] < q2)
+                            q2 = G[q];
+                    }
+                    const double lo = 0.5 * (q1 + p), hi = 0.5 * (p + q2);   // open window
+                    for (int b = 0; b < 49; ++b)
+                        if (b / 8.0 < hi && (b + 1) / 8.0 > lo)
+                            w.m[t][b] |= 1ull << j;
+                }
+            }
+        }
+    });
+    return w;
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_quant_kernel(void (*kernel)(KArgs...), int64_t nblk, const GsArgs& gs, cudaStream_t s,
+                                Args&&... args)
+{
+    int grid = grid_for(nblk, (const void*)kernel);
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    if (gs.mode == 3) {
+        grid = grid < kFusedMaxCtas ? grid : kFusedMaxCtas;
+        attr[0].id = cudaLaunchAttributeCooperative;
+        attr[0].val.cooperative = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 template <int B, typename T, int RULE, int SFMT>
 cudaError_t nvfp4_launch_t(const void* x, int64_t rows, int64_t cols, const GsArgs& gs,
                            uint8_t* codes, uint8_t* scales, int mma, float* deq, float* mse,
@@ -1030,17 +1429,12 @@ cudaError_t nvfp4_launch_t(const void* x, int64_t rows, int64_t cols, const GsAr
 {
     const int64_t nblk = rows * (cols / B);
     if constexpr (RULE == R_BF) {
-        auto k = nvfp4_bf_kernel<B, T, SFMT>;
-        k<<<grid_for(nblk, (const void*)k), kThreads, 0, s>>>(reinterpret_cast<const T*>(x), nblk,
-                                                               cols / B, gs, codes, scales, mma,
-                                                               deq, mse, evals);
+        return launch_quant_kernel(nvfp4_bf_kernel<B, T, SFMT>, nblk, gs, s, reinterpret_cast<const T*>(x), nblk,
+                                   cols / B, gs, codes, scales, mma, deq, mse, evals, bf_windows());
     } else {
-        auto k = nvfp4_quant_kernel<B, T, RULE, SFMT>;
-        k<<<grid_for(nblk, (const void*)k), kThreads, 0, s>>>(reinterpret_cast<const T*>(x), nblk,
-                                                               cols / B, gs, codes, scales, mma,
-                                                               deq, mse);
+        return launch_quant_kernel(nvfp4_quant_kernel<B, T, RULE, SFMT>, nblk, gs, s, reinterpret_cast<const T*>(x),
+                                   nblk, cols / B, gs, codes, scales, mma, deq, mse);
     }
-    return cudaGetLastError();
 }
 
 template <int B, typename T, int SFMT>
@@ -1161,11 +1555,8 @@ cudaError_t launch_razer_quant(const void* x, int dtype, int64_t rows, int64_t c
     if (paired) {
         const int np = n_special / 2;
 #define FP4Q_RAZER_PAIRED(TT, SFV, NP)                                                                  \
-    {                                                                                                \
-        auto k = razer_paired_kernel<TT, SFV, NP>;                                                   \
-        k<<<grid_for(nblk, (const void*)k), kThreads, 0, s>>>(reinterpret_cast<const TT*>(x), nblk, gs, \
-                                                               sp, codes, meta, deq, mse);           \
-    }
+    return launch_quant_kernel(razer_paired_kernel<TT, SFV, NP>, nblk, gs, s, reinterpret_cast<const TT*>(x), \
+                               nblk, gs, sp, codes, meta, deq, mse);
         if (dtype == 1) {
             if (sf == 1) {
                 if (np == 1) FP4Q_RAZER_PAIRED(__nv_bfloat16, 1, 1) else FP4Q_RAZER_PAIRED(__nv_bfloat16, 1, 2)
@@ -1180,30 +1571,19 @@ cudaError_t launch_razer_quant(const void* x, int dtype, int64_t rows, int64_t c
             }
         }
 #undef FP4Q_RAZER_PAIRED
-        return cudaGetLastError();
     }
     if (dtype == 1) {
-        if (sf == 1) {
-            auto k = razer_quant_kernel<__nv_bfloat16, 1>;
-            k<<<grid_for(nblk, (const void*)k), kThreads, 0, s>>>(
-                reinterpret_cast<const __nv_bfloat16*>(x), nblk, gs, sp, codes, meta, deq, mse);
-        } else {
-            auto k = razer_quant_kernel<__nv_bfloat16, 0>;
-            k<<<grid_for(nblk, (const void*)k), kThreads, 0, s>>>(
-                reinterpret_cast<const __nv_bfloat16*>(x), nblk, gs, sp, codes, meta, deq, mse);
-        }
-    } else {
-        if (sf == 1) {
-            auto k = razer_quant_kernel<float, 1>;
-            k<<<grid_for(nblk, (const void*)k), kThreads, 0, s>>>(
-                reinterpret_cast<const float*>(x), nblk, gs, sp, codes, meta, deq, mse);
-        } else {
-            auto k = razer_quant_kernel<float, 0>;
-            k<<<grid_for(nblk, (const void*)k), kThreads, 0, s>>>(
-                reinterpret_cast<const float*>(x), nblk, gs, sp, codes, meta, deq, mse);
-        }
+        if (sf == 1)
+            return launch_quant_kernel(razer_quant_kernel<__nv_bfloat16, 1>, nblk, gs, s,
+                                       reinterpret_cast<const __nv_bfloat16*>(x), nblk, gs, sp, codes, meta, deq, mse);
+        return launch_quant_kernel(razer_quant_kernel<__nv_bfloat16, 0>, nblk, gs, s,
+                                   reinterpret_cast<const __nv_bfloat16*>(x), nblk, gs, sp, codes, meta, deq, mse);
     }
-    return cudaGetLastError();
+    if (sf == 1)
+        return launch_quant_kernel(razer_quant_kernel<float, 1>, nblk, gs, s, reinterpret_cast<const float*>(x),
+                                   nblk, gs, sp, codes, meta, deq, mse);
+    return launch_quant_kernel(razer_quant_kernel<float, 0>, nblk, gs, s, reinterpret_cast<const float*>(x), nblk,
+                               gs, sp, codes, meta, deq, mse);
 }
 
 cudaError_t launch_dequant_mse(const uint8_t* codes, const uint8_t* scales, int64_t rows,

@@ -100,8 +100,13 @@ typedef enum {
 /* Per-tensor FP32 global scale g of hierarchical scaling ([Finer] Methodology 2):
  *  NONE   g = 1
  *  AMAX   g = amax(x) / (6 * S_max), S_max = 448 (E4M3) or 30 (E3M3); g = 1 for
- *         an all-zero tensor.  Computed on the device by a pre-pass; needs a
- *         workspace; the g used is written to *global_scale if non-NULL.
+ *         an all-zero tensor.  Computed on the device inside the quantizer's
+ *         own launch: every CTA takes the maximum of its slice of x, the CTAs
+ *         meet at a bounded grid barrier (a cooperative launch; a CTA whose
+ *         wait runs out takes the maximum of all of x itself, same result),
+ *         and x is then read again for the quantization, mostly from L2.
+ *         Needs a workspace; the g used is written to *global_scale if
+ *         non-NULL.
  *  GIVEN  g read from *global_scale (device) -- e.g. one g shared by fused
  *         projections, the global-scale mismatch fix of [NVFP4] 3. */
 typedef enum { FP4Q_GS_NONE = 0, FP4Q_GS_AMAX = 1, FP4Q_GS_GIVEN = 2 } fp4q_gs_mode;

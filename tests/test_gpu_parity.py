@@ -210,6 +210,58 @@ def test_brute_force_evaluation_counter(O):
     assert int(host(ws)[fq.WS_BF_EVALS:fq.WS_BF_EVALS + 8].view(np.uint64)[0]) == 0
 
 
+def lattice_blocks(O, sf, B, g, rows, seed):
+    """Blocks built around power-of-two scales r (the brute-force kernel's
+    lattice shortcut): the largest element at 0.97-1.0 of 6 S_r (c6 = r, no
+    clipping) or 1.0-1.03 of it (c6 = r, clipping: the shortcut must stay off),
+    the others uniform in +-6 S_r, and some placed exactly on the grids of
+    neighbouring codes (k S_r v for k in 1..13), so that exact ties between
+    codes occur."""
+    rng = np.random.default_rng(seed)
+    val = O.ue5m3_value if sf == O.SF_UE5M3 else O.e4m3_value
+    last = 254 if sf == O.SF_UE5M3 else 126
+    pow2 = [c for c in range(1, last + 1) if float(np.frexp(val(c))[0]) == 0.5]
+    pow2 = [c for c in pow2 if c < last - 8]
+    grid = np.array([0.5, 1, 1.5, 2, 3, 4, 6], np.float64)
+    n = rows * 256 // B
+    x = np.empty((n, B), np.float64)
+    for i in range(n):
+        S = val(int(rng.choice(pow2))) * float(g)
+        u = rng.uniform(-6, 6, B)
+        top = rng.uniform(0.97, 1.0) if i % 4 else rng.uniform(1.0, 1.03)
+        u[rng.integers(B)] = 6 * top * rng.choice([-1, 1])
+        for j in np.nonzero(rng.random(B) < 0.4)[0]:
+            if abs(u[j]) < 6 * 0.97:
+                k = int(rng.integers(1, 14))
+                p = k * rng.choice(grid) * rng.choice([-1, 1])
+                if abs(p) < 5.8:
+                    u[j] = p
+        x[i] = u * S
+    return x.reshape(rows, 256).astype(np.float32)
+
+
+@pytest.mark.parametrize("sf", [0, 3])
+@pytest.mark.parametrize("B", [4, 8, 16, 32])
+@pytest.mark.parametrize("g", [1.0, 0.125])
+def test_brute_force_lattice_shortcut_cases(O, sf, B, g):
+    """Brute force on blocks whose abs-max scale is a power of two: codes, scale
+    bytes, dequant and MSE equal the oracle's full scan of every code, with g = 1
+    (GS_NONE) and with a power-of-two g given."""
+    x32 = lattice_blocks(O, O.SF_UE5M3 if sf == 3 else O.SF_E4M3, B, g, 48, seed=100 + B + sf)
+    given = torch.tensor([g], dtype=torch.float32, device="cuda")
+    gs_mode = fq.GS_NONE if g == 1.0 else fq.GS_GIVEN
+    r = fq.nvfp4_quantize(dev(x32), block=B, rule=fq.BRUTE_FORCE, gs_mode=gs_mode,
+                          global_scale=given if gs_mode == fq.GS_GIVEN else None,
+                          dequant=True, mse=True, scale_fmt=fq.SF_UE5M3 if sf == 3 else fq.SF_E4M3)
+    torch.cuda.synchronize()
+    ref = O.block_fp4_quantize(x32, B, O.RULE_BRUTE_FORCE, O.SF_UE5M3 if sf == 3 else O.SF_E4M3,
+                               g=np.float32(g))
+    assert_bits(r["codes"], ref["codes"], "codes")
+    assert_bits(r["scales"], ref["scales"], "scales")
+    assert_bits(r["dequant"], ref["deq"], "dequant")
+    assert_bits(r["mse"], ref["mse"], "mse")
+
+
 # ------------------------------------------------------------------ RaZeR
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("sf,kind,specials", [(fq.SF_E3M3, "razer_weight", [5.0, -5.0, 3.5, -3.5]),

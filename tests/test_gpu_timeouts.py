@@ -9,6 +9,10 @@ releases its tensor memory and returns.  The host sees FP4Q_ERR_TIMEOUT from
 the entry point's status call.  A normal call on the same workspace
 afterwards must return FP4Q_OK with output bit-identical to a call made
 before: the context stays usable.
+
+The quantizers' fused global amax waits at a grid barrier, also bounded: a
+CTA whose wait runs out computes the whole maximum itself, so its results do
+not change at all (tested with the same one-cycle limit).
 """
 import numpy as np
 import pytest
@@ -114,3 +118,25 @@ def test_hessian_wait_gives_up_and_reports_timeout():
     again = fq.hessian_blocks(x, t, True, workspace=ws)
     assert fq.hessian_status(ws) == 0
     assert torch.equal(again.view(torch.int32), ref.view(torch.int32))
+
+
+@pytest.mark.parametrize("kind,rule,B", [("gaussian", fq.PREVENT_ZERO, 16), ("gemm_act", fq.FOUR_OVER_SIX, 16),
+                                         ("student_t", fq.BRUTE_FORCE, 8)])
+def test_fused_amax_barrier_fallback_keeps_results(O, kind, rule, B):
+    """The hierarchical (AMAX) global scale is reduced inside the quantizer
+    launch behind a grid barrier.  With the barrier's wait limited to one cycle
+    the CTAs that give up take the maximum of the whole tensor themselves: g,
+    codes, scales and errors must not change."""
+    from test_gpu_parity import make, assert_bits
+    x, x32 = make(kind, 1000, 512, seed=7, dtype="bf16" if kind == "gemm_act" else "f32")
+    ref = O.nvfp4_quantize(x32, B, rule, g=O.global_scale(O.amax(x32)))
+    normal = fq.nvfp4_quantize(x, B, rule, gs_mode=fq.GS_AMAX, mse=True)
+    with short_waits():
+        alone = fq.nvfp4_quantize(x, B, rule, gs_mode=fq.GS_AMAX, mse=True)
+        torch.cuda.synchronize()
+    for r in (normal, alone):
+        assert_bits(r["global_scale"], np.array([O.global_scale(O.amax(x32))], np.float32), "g")
+        assert_bits(r["codes"], ref["codes"], "codes")
+        assert_bits(r["scales"], ref["scales"], "scales")
+        assert_bits(r["mse"], ref["mse"], "mse")
+
