@@ -511,6 +511,27 @@ def run_reference(args, rank, world):
 
 
 # ------------------------------------------------------------------ main arm
+def fp4_ceiling(torch, fq, mx, iters=16384, reps=3):
+    """Measured tensor-pipe ceiling (TFLOP/s) of the GEMMs' MMA stream: the library's probe
+    kernel (fp4q_mma_ceiling) issuing back-to-back 256x256x64 block-scaled FP4 MMAs on every SM
+    pair, timed with CUDA events on the launching stream (best of `reps`, after one warm-up)."""
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    fq.mma_ceiling(mx, 64, err)
+    best = None
+    flops = 0.0
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        flops = fq.mma_ceiling(mx, iters, err)
+        b.record()
+        torch.cuda.synchronize()
+        ms = a.elapsed_time(b)
+        best = ms if best is None else min(best, ms)
+    if int(err.item()) != 0:
+        raise RuntimeError("tensor-pipe ceiling probe: a bounded wait gave up")
+    return flops / (best * 1e-3) / 1e12
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -520,6 +541,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch the timed step eagerly, not as a CUDA graph")
+    ap.add_argument("--fp4-ceiling", action="store_true",
+                    help="measure the tensor-pipe ceiling of the GEMMs' FP4 MMA stream and print it (no JSON)")
     ap.add_argument("--no-next-rows", action="store_true",
                     help="time the hot-path step only (skip the rows built on top of it)")
     ap.add_argument("--profile-row", default=None,
@@ -547,6 +570,12 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     fq.lib(build_if_missing=True)
     hbm_peak, sm_max_mhz, bf16_peak, bf16_sust, peak_src = load_peaks()
+
+    if args.fp4_ceiling:
+        for mx in (False, True):
+            print("fp4 MMA ceiling (%s): %.1f TFLOP/s" % ("kind::mxf4 block32" if mx else "kind::mxf4nvf4 block16",
+                                                         fp4_ceiling(torch, fq, mx)))
+        return 0
 
     if args.profile_row:
         # the next rows f2 / f3 are built with the workloads they extend
@@ -741,9 +770,15 @@ def main():
     gemm = None
     if gem is not None:
         g = row_out[gem.name]
+        ceil = fp4_ceiling(torch, fq, False)
         gemm = {"TFLOP_s": g["TFLOP_s"], "frac_of_fp4_peak": g["tensor_frac"], "fp4_peak_TFLOP_s": fp4_peak,
                 "frac_of_9000_spec": g["TFLOP_s"] / 9000.0,
+                "fp4_mma_ceiling_TFLOP_s": ceil, "frac_of_mma_ceiling": g["TFLOP_s"] / ceil,
                 "ms": g["ms"], "shape": "M=8192 N=14336 K=4096", "traffic": profiled_traffic("c5_w4a4_gemm")}
+        for r in rows:
+            if r.name.startswith("f3_mx_gemm"):
+                row_out[r.name]["frac_of_mma_ceiling"] = row_out[r.name]["TFLOP_s"] / fp4_ceiling(torch, fq, True)
+                break
     line = {
         "metric": METRIC, "value": value, "unit": "Gelem/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",

@@ -44,6 +44,8 @@ SIGNATURES = {
     "fp4q_gemm_status": (_i, [_vp, _vp]),
     "fp4q_hessian_status": (_i, [_vp, _vp]),
     "fp4q_debug_set_wait_cycles": (_i64, [_i64]),
+    "fp4q_mma_ceiling": (_i, [_i, _i, _vp, _vp]),
+    "fp4q_mma_ceiling_flops": (ctypes.c_double, [_i]),
     "razer_gemm_prepare": (_i, [_vp, _vp, _i64, _i64, _i, _vp, _i, _vp, _vp, _vp, _vp]),
     "razer_w4a4_gemm": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _vp, _i, _vp, _sz, _vp]),
     "fp4_scales_to_mma": (_i, [_vp, _i64, _i64, _vp, _vp]),
@@ -402,3 +404,12 @@ def debug_set_wait_cycles(cycles: int) -> int:
     """Process-wide limit of the tensor-core kernels' bounded waits (0: the default);
     returns the previous setting.  For tests of the timeout path."""
     return int(lib().fp4q_debug_set_wait_cycles(int(cycles)))
+
+
+def mma_ceiling(mx: bool, iters: int, err: torch.Tensor, stream=None) -> float:
+    """Enqueue the tensor-pipe ceiling probe (fp4q_mma_ceiling); returns the flops the launch
+    performs.  err: a device int32 tensor the kernel sets to 1 if its final wait gave up."""
+    _need_cuda(err)
+    _check(lib().fp4q_mma_ceiling(int(bool(mx)), int(iters), _ptr(err), _stream(stream)), "fp4q_mma_ceiling")
+    return float(lib().fp4q_mma_ceiling_flops(int(iters)))
+

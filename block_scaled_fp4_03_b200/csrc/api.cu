@@ -435,6 +435,20 @@ int fp4q_gemm_status(const void* workspace, void* stream)
     return flag ? FP4Q_ERR_TIMEOUT : FP4Q_OK;
 }
 
+int fp4q_mma_ceiling(int mx, int iters, int* err, void* stream)
+{
+    if (!err || iters < 1 || iters > (1 << 20) || (mx != 0 && mx != 1))
+        return FP4Q_ERR_ARG;
+    if ((reinterpret_cast<uintptr_t>(err) & 3u) != 0)
+        return FP4Q_ERR_ALIGN;
+    return from_cuda(launch_mma_ceiling(mx, iters, err, as_stream(stream)));
+}
+
+double fp4q_mma_ceiling_flops(int iters)
+{
+    return iters < 1 ? 0.0 : (double)mma_ceiling_pairs() * (double)iters * 4.0 * 2.0 * 256.0 * 256.0 * 64.0;
+}
+
 int fp4q_hessian_status(const void* workspace, void* stream)
 {
     // NULL: the error word of fp4_hessian_blocks_noalloc on the current device

@@ -103,6 +103,12 @@ cudaError_t launch_w4a4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const 
                              const uint8_t* a1_codes = nullptr, const uint8_t* w1_codes = nullptr,
                              int mx = 0);
 
+// The tensor-pipe ceiling probe: every SM pair issues iters x 4 back-to-back
+// 256x256x64 block-scaled FP4 MMAs (mx: kind::mxf4) on resident operands;
+// *err (device) is set to 1 if a bounded wait gave up.
+cudaError_t launch_mma_ceiling(int mx, int iters, int* err, cudaStream_t s);
+int mma_ceiling_pairs();
+
 // Row-major scale bytes [rows][nscales] -> the MMA scale layout (rows % 128 == 0,
 // nscales % 4 == 0).
 cudaError_t launch_scales_to_mma(const uint8_t* scales, int64_t rows, int64_t nscales, uint8_t* out,

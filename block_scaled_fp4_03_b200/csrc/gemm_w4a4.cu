@@ -920,6 +920,101 @@ w4a4_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                      : "memory");
 }
 
+// ------------------------------------------------ tensor-pipe ceiling probe
+// Back-to-back block-scaled FP4 MMAs of the GEMM's shape (CTA pair, M = N =
+// 256, K = 64, four per 256-wide K step) on operand tiles parked in shared
+// memory and scale atoms copied into TMEM once: no global traffic and no
+// barrier wait inside the loop, so its rate is the most the tensor pipe gives
+// this instruction stream.  The leader thread of each pair issues `iters`
+// groups of four MMAs into one accumulator and commits; both CTAs then wait
+// (bounded) for completion and meet at the teardown handshake.  Operand bytes
+// are a fixed pattern (finite E2M1 values; scales 1.0 in UE4M3 or UE8M0).
+constexpr int kCeilTile = 128 * kBK / 2;                  // 16 KiB per operand tile
+// far more shared memory than the tiles need, so that one CTA holds an SM (and
+// its 512 TMEM columns) alone
+constexpr int kCeilSmem = 128 * 1024;
+static_assert(2 * kCeilTile + k2SfaStage + k2SfbStage + 1024 + 64 <= kCeilSmem, "ceiling probe shared memory");
+
+template <bool MX>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(128, 1)
+mma_ceiling_kernel(int iters, int* err)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sa_codes = smem;
+    uint8_t* sb_codes = smem + kCeilTile;
+    uint8_t* sa_sf = smem + 2 * kCeilTile;
+    uint8_t* sb_sf = sa_sf + k2SfaStage;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sb_sf + k2SfbStage);   // [0] done, [1] teardown
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2);
+    const int warp = threadIdx.x >> 5;
+    const uint32_t rank = cluster_rank();
+    const uint32_t done = smem_u32(bars);
+    const uint32_t bye = done + 8u;
+    constexpr int kAt = SfGeom<MX>::kAtoms;
+    {
+        uint32_t* c32 = reinterpret_cast<uint32_t*>(smem);
+        for (int i = threadIdx.x; i < 2 * kCeilTile / 4; i += blockDim.x)
+            c32[i] = 0x5A5A5A5Au;                                   // E2M1 codes 0xA and 0x5
+        const uint32_t one = MX ? 0x7F7F7F7Fu : 0x38383838u;        // 1.0 as UE8M0 / UE4M3
+        uint32_t* s32 = reinterpret_cast<uint32_t*>(sa_sf);
+        for (int i = threadIdx.x; i < (k2SfaStage + k2SfbStage) / 4; i += blockDim.x)
+            s32[i] = one;
+    }
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    if (threadIdx.x == 0) {
+        mbar_init(done, 1);
+        mbar_init(bye, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_holder)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+    tc_fence_after();
+    const uint32_t tmem = *tmem_holder;
+    if (threadIdx.x == 0 && rank == 0) {
+        const uint32_t tsfa = tmem + kSfCol0;
+        const uint32_t tsfb = tsfa + 16;
+        const uint32_t sa_s = smem_u32(sa_sf), sb_s = smem_u32(sb_sf);
+#pragma unroll
+        for (int s = 0; s < kAt; ++s) {
+            tc2_cp_sf(tsfa + 4 * s, sdesc_sf(sa_s + 512 * s));
+            tc2_cp_sf(tsfb + 8 * s, sdesc_sf(sb_s + 512 * s));
+            tc2_cp_sf(tsfb + 8 * s + 4, sdesc_sf(sb_s + 512 * kAt + 512 * s));
+        }
+        const uint32_t a_s = smem_u32(sa_codes), b_s = smem_u32(sb_codes);
+        for (int it = 0; it < iters; ++it) {
+#pragma unroll
+            for (int s = 0; s < 4; ++s) {
+                uint32_t sfa, sfb, id;
+                mma_scale_operands<MX>(s, tsfa, tsfb, MX ? (k2Idesc | kScaleUE8M0) : k2Idesc, sfa, sfb, id);
+                tc2_mma<MX>(tmem, sdesc_sw128(a_s + 32 * s), sdesc_sw128(b_s + 32 * s), id, (it | s) != 0, sfa, sfb);
+            }
+        }
+        tc2_commit_mc(done, (uint16_t)0x3);
+    }
+    if (threadIdx.x == 0 && !mbar_wait(done, 0, nullptr))
+        atomicExch(err, 1);
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        mbar_arrive_cluster(mapa_rank(bye, rank ^ 1u));
+        if (!mbar_wait_cluster(bye, 0, nullptr, kTeardownCycles))
+            atomicExch(err, 1);
+    }
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1)
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+                     : "memory");
+}
+
 // ------------------------------------------------------------ host side
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
 {
@@ -1027,6 +1122,22 @@ cudaError_t launch_gemm_t(const uint8_t* a_codes, const uint8_t* a_sf, const uin
     const int tiles = p.tiles_m * p.tiles_n;
     const int grid = tiles < num_sms() ? tiles : num_sms();
     w4a4_gemm_1sm_kernel<MX, OUTF32><<<grid, kThreads, kSmemBytes, s>>>(ta, tb, tsa, tsb, ta1, tb1, p);
+    return cudaGetLastError();
+}
+
+int mma_ceiling_pairs() { return num_sms() / 2; }
+
+cudaError_t launch_mma_ceiling(int mx, int iters, int* err, cudaStream_t s)
+{
+    const void* k = mx ? (const void*)mma_ceiling_kernel<true> : (const void*)mma_ceiling_kernel<false>;
+    const cudaError_t e = smem_opt_in(k, kCeilSmem);
+    if (e != cudaSuccess)
+        return e;
+    const int grid = 2 * mma_ceiling_pairs();
+    if (mx)
+        mma_ceiling_kernel<true><<<grid, 128, kCeilSmem, s>>>(iters, err);
+    else
+        mma_ceiling_kernel<false><<<grid, 128, kCeilSmem, s>>>(iters, err);
     return cudaGetLastError();
 }
 

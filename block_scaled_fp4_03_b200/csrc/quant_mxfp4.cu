@@ -232,6 +232,190 @@ mx_quant_absmax_kernel(const T* __restrict__ x, uint32_t nblk, uint32_t kb,
     }
 }
 
+// ------------------------------------- OCP exponent (activations), two lanes
+// per block.  Lanes 2j and 2j+1 hold the two 16-element halves of a warp's
+// block j (16 blocks per warp and step), which halves the registers a lane
+// needs and lets four CTAs share an SM.  The rotation's strides 1-8 stay
+// inside a half; stride 16 pairs element i of one half with element i of the
+// other, exchanged with one shuffle, and each lane applies the same add or
+// subtract (a + b on the first half, a - b on the second) as the one-lane
+// form.  The maximum is the maximum of the two halves' maxima; the ordered
+// squared error runs over the first half in one lane and continues over the
+// second half in the other.  The channel scale t is kept whole in shared
+// memory (16-byte chunks XOR-swizzled by column block, so a warp's reads are
+// conflict-free); the warp's 16 blocks are read as whole rows, parked in
+// shared memory and picked up by half, and the next group's loads are in
+// flight while the current one is transformed.
+constexpr int kMx2BlocksPerWarp = 16;
+// largest cols/32 whose t table fits the shared-memory budget of this kernel
+constexpr int kMx2MaxColBlocks = 512;
+
+template <typename T, bool ERR>
+__global__ void __launch_bounds__(kThreads, ERR ? 3 : 4)
+mx_quant_absmax2_kernel(const T* __restrict__ x, uint32_t nblk, uint32_t kb,
+                        const float* __restrict__ t, int had, uint8_t* __restrict__ codes,
+                        uint8_t* __restrict__ scales, float* __restrict__ deq,
+                        float* __restrict__ mse, int mma)
+{
+    constexpr int CPB = 32 * (int)sizeof(T) / 16;   // 16-byte chunks per block
+    constexpr int CPL = CPB / 2;                      // chunks per lane (its half)
+    constexpr int kStage = kMx2BlocksPerWarp * CPB;   // chunks per warp
+    extern __shared__ uint4 mx2_smem[];
+    uint4* ttab = mx2_smem;                                       // kb rows of 8 chunks
+    const int lane = threadIdx.x & 31;
+    const int w = threadIdx.x >> 5;
+    uint4* stage = mx2_smem + (t ? (size_t)kb * 8 : 0) + (size_t)w * kStage;
+    if (t) {
+        const uint4* t4 = reinterpret_cast<const uint4*>(t);
+        for (uint32_t i = threadIdx.x; i < kb * 8u; i += blockDim.x) {
+            const uint32_t r = i >> 3, p = i & 7u;
+            ttab[r * 8u + (p ^ (r & 7u))] = __ldg(t4 + i);
+        }
+        __syncthreads();
+    }
+    const int j = lane >> 1;          // this lane's block within the warp's group
+    const int h = lane & 1;           // and its half
+    const uint64_t warp0 = ((uint64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const uint64_t nwarps = ((uint64_t)gridDim.x * blockDim.x) >> 5;
+    const uint64_t step = nwarps * kMx2BlocksPerWarp;
+    uint4 v[CPL];
+    auto fetch = [&](uint64_t gbase) {
+        const uint64_t left = nblk - gbase;
+        const uint32_t nb = (uint32_t)(left < kMx2BlocksPerWarp ? left : kMx2BlocksPerWarp);
+        const uint4* src = reinterpret_cast<const uint4*>(x + gbase * 32);
+#pragma unroll
+        for (int k = 0; k < CPL; ++k) {
+            const int c = lane + 32 * k;
+            v[k] = (uint32_t)(c / CPB) < nb ? ldg_stream(src + c) : make_uint4(0u, 0u, 0u, 0u);
+        }
+    };
+    uint64_t base = warp0 * kMx2BlocksPerWarp;
+    if (base < nblk)
+        fetch(base);
+    for (; base < nblk; base += step) {
+        const uint64_t left = nblk - base;
+        const uint32_t nb = (uint32_t)(left < kMx2BlocksPerWarp ? left : kMx2BlocksPerWarp);
+        __syncwarp();   // the previous group has been read back
+#pragma unroll
+        for (int k = 0; k < CPL; ++k) {
+            const int c = lane + 32 * k;
+            stage[staged_slot<CPB>(c / CPB, c % CPB)] = v[k];
+        }
+        __syncwarp();
+        if (base + step < nblk)
+            fetch(base + step);        // the next group's loads, in flight meanwhile
+        float u[16];
+#pragma unroll
+        for (int p = 0; p < CPL; ++p) {
+            const uint4 q = stage[staged_slot<CPB>(j, h * CPL + p)];
+            if constexpr (sizeof(T) == 4) {
+                u[4 * p] = __uint_as_float(q.x);
+                u[4 * p + 1] = __uint_as_float(q.y);
+                u[4 * p + 2] = __uint_as_float(q.z);
+                u[4 * p + 3] = __uint_as_float(q.w);
+            } else {
+                bf16x2_to_f32(q.x, u[8 * p], u[8 * p + 1]);
+                bf16x2_to_f32(q.y, u[8 * p + 2], u[8 * p + 3]);
+                bf16x2_to_f32(q.z, u[8 * p + 4], u[8 * p + 5]);
+                bf16x2_to_f32(q.w, u[8 * p + 6], u[8 * p + 7]);
+            }
+        }
+        const uint64_t b = base + (uint64_t)j;
+        const uint32_t kbi = (uint32_t)(b % kb);
+        if (t) {
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+                const uint4 q = ttab[kbi * 8u + ((uint32_t)(4 * h + p) ^ (kbi & 7u))];
+                u[4 * p] = __fmul_rn(u[4 * p], __uint_as_float(q.x));
+                u[4 * p + 1] = __fmul_rn(u[4 * p + 1], __uint_as_float(q.y));
+                u[4 * p + 2] = __fmul_rn(u[4 * p + 2], __uint_as_float(q.z));
+                u[4 * p + 3] = __fmul_rn(u[4 * p + 3], __uint_as_float(q.w));
+            }
+        }
+        if (had) {
+#pragma unroll
+            for (int s = 1; s < 16; s <<= 1) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    if ((i & s) == 0) {
+                        const float p = u[i], q = u[i + s];
+                        u[i] = __fadd_rn(p, q);
+                        u[i + s] = __fsub_rn(p, q);
+                    }
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const float o = __shfl_xor_sync(0xffffffffu, u[i], 1);
+                u[i] = h == 0 ? __fadd_rn(u[i], o) : __fsub_rn(o, u[i]);
+            }
+            const float c = had_norm();
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                u[i] = __fmul_rn(u[i], c);
+        }
+        float a = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            a = fmaxf(a, fabsf(u[i]));
+        a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+        const int e = mx_exponent(a);
+        const float down = pow2f(-e);
+        uint32_t cw[2];
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            const int o = 8 * q;
+            cw[q] = e2m1x8_encode(__fmul_rn(u[o], down), __fmul_rn(u[o + 1], down),
+                                  __fmul_rn(u[o + 2], down), __fmul_rn(u[o + 3], down),
+                                  __fmul_rn(u[o + 4], down), __fmul_rn(u[o + 5], down),
+                                  __fmul_rn(u[o + 6], down), __fmul_rn(u[o + 7], down));
+        }
+        const bool valid = (uint32_t)j < nb;
+        if constexpr (ERR) {
+            const float up = pow2f(e);
+            float dq[16];
+            float acc0 = 0.0f;     // the first half's error chain ...
+            float acc = 0.0f;
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                float vv[8];
+                e2m1x8_decode(cw[q], vv);
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    dq[8 * q + i] = __fmul_rn(vv[i], up);
+            }
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const float er = __fsub_rn(u[i], dq[i]);
+                acc0 = __fmaf_rn(er, er, acc0);
+            }
+            // ... continued over the second half from where the first ended
+            acc = __shfl_xor_sync(0xffffffffu, acc0, 1);
+            if (h == 1) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float er = __fsub_rn(u[i], dq[i]);
+                    acc = __fmaf_rn(er, er, acc);
+                }
+            }
+            if (valid) {
+                if (deq)
+                    store_f32<16>(deq + b * 32 + 16 * h, dq);
+                if (mse && h == 1)
+                    mse[b] = __fmul_rn(acc, 1.0f / 32.0f);
+            }
+        }
+        if (valid) {
+            *reinterpret_cast<uint2*>(codes + b * 16 + 8 * h) = make_uint2(cw[0], cw[1]);
+            if (h == 0) {
+                const uint64_t r = b / kb;
+                scales[mma ? mma_sf_offset((int64_t)r, (int64_t)(b - r * kb), kb >> 2) : (int64_t)b] =
+                    (uint8_t)(e + 127);
+            }
+        }
+    }
+}
+
 // Block error d = u - deq(u, e) at exponent e.
 __device__ __forceinline__ void mx_err(const float (&u)[32], int e, float (&d)[32])
 {
@@ -735,6 +919,37 @@ cudaError_t launch_mxfp4_quant(const void* x, int dtype, int64_t rows, int64_t c
     if (nblk > (int64_t)0xFFFFFFFFu)
         return cudaErrorInvalidValue;
     const bool err = deq || mse;
+    if (kb <= kMx2MaxColBlocks) {
+        // two lanes per block; the t table and the warps' staging in dynamic shared memory
+        const int esz = dtype == 1 ? 2 : 4;
+        const int smem = (chan_scale ? (int)kb * 128 : 0) + kMxWarps * kMx2BlocksPerWarp * 32 * esz;
+        const void* kp = dtype == 1 ? (err ? (const void*)mx_quant_absmax2_kernel<__nv_bfloat16, true>
+                                           : (const void*)mx_quant_absmax2_kernel<__nv_bfloat16, false>)
+                                    : (err ? (const void*)mx_quant_absmax2_kernel<float, true>
+                                           : (const void*)mx_quant_absmax2_kernel<float, false>);
+        const cudaError_t ae = smem_opt_in(kp, kMx2MaxColBlocks * 128 + kMxWarps * kMx2BlocksPerWarp * 32 * 4);
+        if (ae != cudaSuccess)
+            return ae;
+        int per_sm = 0;
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kp, kThreads, smem);
+        per_sm = per_sm < 1 ? 1 : per_sm;
+        const int64_t groups = (nblk + kMx2BlocksPerWarp - 1) / kMx2BlocksPerWarp;
+        int64_t grid = (groups + kMxWarps - 1) / kMxWarps;
+        const int64_t cap = (int64_t)num_sms() * per_sm;
+        grid = grid > cap ? cap : grid;
+        grid = grid < 1 ? 1 : grid;
+        if (dtype == 1) {
+            auto k = err ? mx_quant_absmax2_kernel<__nv_bfloat16, true> : mx_quant_absmax2_kernel<__nv_bfloat16, false>;
+            k<<<(unsigned)grid, kThreads, smem, s>>>(reinterpret_cast<const __nv_bfloat16*>(x), (uint32_t)nblk,
+                                                     (uint32_t)kb, chan_scale, hadamard, codes, scales, deq, mse,
+                                                     mma_layout);
+        } else {
+            auto k = err ? mx_quant_absmax2_kernel<float, true> : mx_quant_absmax2_kernel<float, false>;
+            k<<<(unsigned)grid, kThreads, smem, s>>>(reinterpret_cast<const float*>(x), (uint32_t)nblk, (uint32_t)kb,
+                                                     chan_scale, hadamard, codes, scales, deq, mse, mma_layout);
+        }
+        return cudaGetLastError();
+    }
     if (dtype == 1) {
         auto k = err ? mx_quant_absmax_kernel<__nv_bfloat16, true> : mx_quant_absmax_kernel<__nv_bfloat16, false>;
         k<<<grid_for(nblk, (const void*)k), kThreads, 0, s>>>(

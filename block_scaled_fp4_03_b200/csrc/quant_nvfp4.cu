@@ -1016,12 +1016,33 @@ nvfp4_bf_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs,
         step_kb = step % bpr;
     }
     float* xw = xs[w];
+    // blocks of up to 32 bytes: the next block's load is in flight while this
+    // one is searched (one load round trip per block otherwise stalls the warp)
+    constexpr bool kPrefetch = B * sizeof(T) <= 32;
+    float xn[kPrefetch ? B : 1];
+    if constexpr (kPrefetch) {
+        const int64_t b0 = warp0 * 32 + lane;
+        if (b0 < nblk) {
+            load_elems<T, B>(x + b0 * B, xn);
+        } else {
+#pragma unroll
+            for (int i = 0; i < B; ++i)
+                xn[i] = 0.0f;
+        }
+    }
 
     for (int64_t base = warp0 * 32; base < nblk; base += nwarps * 32) {
         const int64_t b = base + lane;
         const bool valid = b < nblk;
         float xv[B];
-        if (valid) {
+        if constexpr (kPrefetch) {
+#pragma unroll
+            for (int i = 0; i < B; ++i)
+                xv[i] = xn[i];
+            const int64_t bn = b + nwarps * 32;
+            if (bn < nblk)
+                load_elems<T, B>(x + bn * B, xn);
+        } else if (valid) {
             load_elems<T, B>(x + b * B, xv);
         } else {
 #pragma unroll

@@ -459,6 +459,23 @@ FP4Q_API int mxfp4_gemm(const void* a, int a_format, const uint8_t* a_scales, co
 FP4Q_API int fp4q_gemm_status(const void* workspace, void* stream);
 
 /*
+ * Diagnostic: the tensor-pipe ceiling the GEMMs are measured against.  Launches
+ * a kernel in which every pair of SMs issues `iters` groups of four
+ * back-to-back block-scaled FP4 MMAs of the GEMMs' shape (CTA pair, 256 x 256
+ * x 64; mx = 0: kind::mxf4nvf4 with UE4M3 scales per 16, mx = 1: kind::mxf4
+ * with UE8M0 scales per 32) on operand tiles held in shared memory and scales
+ * copied into TMEM once -- no global traffic and no waits inside the loop.
+ * Enqueued on `stream`; time it with events on that stream and divide
+ * fp4q_mma_ceiling_flops(iters) (the flops one launch performs on the current
+ * device) by the time.  err: device int (4-byte aligned), set to 1 if the
+ * final bounded wait gave up (the caller clears it).  1 <= iters <= 2^20 (a
+ * launch then stays far inside the wait's bound).
+ * Errors: ERR_ARG, ERR_ALIGN, ERR_CUDA.
+ */
+FP4Q_API int fp4q_mma_ceiling(int mx, int iters, int* err, void* stream);
+FP4Q_API double fp4q_mma_ceiling_flops(int iters);
+
+/*
  * Debug: the limit, in SM clock cycles, after which the main-loop waits of the
  * tensor-core kernels (the three GEMMs and the Hessian blocks) give up; 0 or a
  * negative value restores the default (4e9 cycles, about 2 s at the boost

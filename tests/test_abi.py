@@ -189,6 +189,15 @@ def test_status_calls_reject_a_missing_workspace(L):
     assert L.fp4q_gemm_status(None, None) == 1
 
 
+def test_mma_ceiling_probe_argument_errors(L):
+    assert L.fp4q_mma_ceiling(0, 0, FAKE, None) == 1            # no iterations
+    assert L.fp4q_mma_ceiling(0, (1 << 20) + 1, FAKE, None) == 1
+    assert L.fp4q_mma_ceiling(2, 16, FAKE, None) == 1            # mx is 0 or 1
+    assert L.fp4q_mma_ceiling(0, 16, None, None) == 1
+    assert L.fp4q_mma_ceiling(0, 16, ctypes.c_void_p(0x10002), None) == 2
+    assert L.fp4q_mma_ceiling_flops(0) == 0.0
+
+
 def test_debug_wait_limit_setter_round_trips(L):
     """The wait-limit knob is host state only: it stores and returns settings, 0 = default."""
     prev = L.fp4q_debug_set_wait_cycles(1)

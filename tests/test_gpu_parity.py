@@ -295,6 +295,20 @@ def test_mxfp4_absmax_small(O, dtype, use_t, had):
     assert_bits(r["mse"], ref["mse"], "mse")
 
 
+def test_mxfp4_absmax_wide_rows(O):
+    """Rows of more than 512 column blocks (16416 columns): the one-lane-per-block
+    kernel, with t and the rotation, bit for bit."""
+    x, x32 = make("mx_act", 9, 16416, seed=17, dtype="bf16")
+    t = inputs.positive_vector(16416, seed=18)
+    r = fq.mxfp4_quantize(x, dev(t), True, fq.ABSMAX, dequant=True, mse=True)
+    torch.cuda.synchronize()
+    ref = O.mxfp4_quantize(x32, t, True, O.RULE_ABSMAX)
+    assert_bits(r["codes"], ref["codes"], "codes")
+    assert_bits(r["scales"], ref["scales"], "scales")
+    assert_bits(r["dequant"], ref["deq"], "dequant")
+    assert_bits(r["mse"], ref["mse"], "mse")
+
+
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 def test_mxfp4_hessian_small(O, dtype):
     w, w32 = make("mx_weight", 300, 256, seed=8, dtype=dtype)
