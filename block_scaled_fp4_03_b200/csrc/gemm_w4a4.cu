@@ -927,8 +927,9 @@ w4a4_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
 // barrier wait inside the loop, so its rate is the most the tensor pipe gives
 // this instruction stream.  The leader thread of each pair issues `iters`
 // groups of four MMAs into one accumulator and commits; both CTAs then wait
-// (bounded) for completion and meet at the teardown handshake.  Operand bytes
-// are a fixed pattern (finite E2M1 values; scales 1.0 in UE4M3 or UE8M0).
+// (bounded) for completion and meet at the teardown handshake.  Operand codes
+// are hashed bytes (every E2M1 code is finite; operand bits toggle as with real
+// data, which sets the power drawn), scales 1.0 in UE4M3 or UE8M0.
 constexpr int kCeilTile = 128 * kBK / 2;                  // 16 KiB per operand tile
 // far more shared memory than the tiles need, so that one CTA holds an SM (and
 // its 512 TMEM columns) alone
@@ -953,9 +954,16 @@ mma_ceiling_kernel(int iters, int* err)
     const uint32_t bye = done + 8u;
     constexpr int kAt = SfGeom<MX>::kAtoms;
     {
+        // operand codes: a hash of the word index, so the MMAs see data that
+        // toggles like real operands (every E2M1 code is finite)
         uint32_t* c32 = reinterpret_cast<uint32_t*>(smem);
-        for (int i = threadIdx.x; i < 2 * kCeilTile / 4; i += blockDim.x)
-            c32[i] = 0x5A5A5A5Au;                                   // E2M1 codes 0xA and 0x5
+        for (int i = threadIdx.x; i < 2 * kCeilTile / 4; i += blockDim.x) {
+            uint32_t h = (uint32_t)i * 0x9E3779B1u + 0x7F4A7C15u * (uint32_t)(blockIdx.x + 1);
+            h ^= h >> 15;
+            h *= 0x85EBCA6Bu;
+            h ^= h >> 13;
+            c32[i] = h;
+        }
         const uint32_t one = MX ? 0x7F7F7F7Fu : 0x38383838u;        // 1.0 as UE8M0 / UE4M3
         uint32_t* s32 = reinterpret_cast<uint32_t*>(sa_sf);
         for (int i = threadIdx.x; i < (k2SfaStage + k2SfbStage) / 4; i += blockDim.x)

@@ -1245,6 +1245,380 @@ nvfp4_bf_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs,
     }
 }
 
+// A block's search after the exact shortcuts: the better of c6 and the
+// all-zero code so far, and the codes still to evaluate (clo .. c6 - 1, then
+// the bits of um: code c6 + 1 + j; `over`: codes past c6 + 64 as well).
+struct BfPlan {
+    float best;
+    uint32_t bc, c6, clo;
+    int chi;
+    unsigned long long um;
+    bool over;
+};
+
+template <int B, int SFMT>
+__device__ __forceinline__ BfPlan bf_plan(const float (&xv)[B], bool valid, const float2* tab,
+                                          const unsigned long long* wmask, float g6, float four_over_g,
+                                          bool g_pow2, uint32_t (&cw)[(B + 7) / 8], uint32_t& n_eval)
+{
+    constexpr uint32_t kLast = SFMT == 1 ? 254u : 126u;
+    constexpr uint32_t kNone = kLast + 1u;
+    BfPlan pl;
+    float a = 0.0f;
+    float sse0 = 0.0f;
+#pragma unroll
+    for (int i = 0; i < B; ++i) {
+        a = fmaxf(a, fabsf(xv[i]));
+        sse0 = __fmaf_rn(xv[i], xv[i], sse0);
+    }
+    uint32_t c6 = sf_encode<SFMT>(__fdiv_rn(a, g6));
+    c6 = c6 == 0u ? 1u : c6;
+    const float2 t6 = tab[c6];
+    float best = quant_codes_sse<B>(xv, t6, cw);
+    uint32_t bc = c6;
+    n_eval += valid ? 1u : 0u;
+    // first all-zero code (kNone = none): step from a nearby code to the
+    // boundary (|y| is monotone in the code)
+    uint32_t cz = sf_encode<SFMT>(__fmul_rn(a, four_over_g));
+    cz = cz == 0u ? 1u : cz;
+    {
+        // usually the boundary is cz or cz + 1: test both without a loop
+        const bool f0 = cz > 1u && __fmul_rn(a, tab[cz - 1u].y) <= 0.25f;
+        const bool f1 = __fmul_rn(a, tab[cz].y) <= 0.25f;
+        const bool f2 = cz + 1u >= kNone || __fmul_rn(a, tab[cz + 1u].y) <= 0.25f;
+        if (f1 && !f0) {
+        } else if (!f1 && f2) {
+            ++cz;
+        } else if (f1) {
+            --cz;
+            while (cz > 1u && __fmul_rn(a, tab[cz - 1u].y) <= 0.25f)
+                --cz;
+        } else {
+            ++cz;
+            do {
+                ++cz;
+            } while (cz < kNone && __fmul_rn(a, tab[cz].y) > 0.25f);
+        }
+    }
+    n_eval += (valid && cz < kNone) ? 1u : 0u;
+    if (cz < kNone && (sse0 < best || (sse0 == best && cz < bc))) {
+        best = sse0;
+        bc = cz;
+    }
+    // downward: codes below c6 while the clipped bound can still win
+    uint32_t clo = c6;
+    while (clo > 1u) {
+        const float2 t = tab[clo - 1u];
+        const float em = elem_err(a, t.x, t.y);
+        if (__fmul_rn(em, em) > best)
+            break;
+        --clo;
+    }
+    const int chi = (int)(cz < kNone ? cz : kNone) - 1;   // last code to evaluate
+    const int nup = valid ? chi - (int)c6 : 0;
+    unsigned long long um = nup <= 0 ? 0ull : nup >= 64 ? ~0ull : ((1ull << nup) - 1ull);
+    // c6 is a usable reference: a power-of-two scale with an exact
+    // reciprocal at which no element clips; then only the codes whose
+    // windows hold an element stay
+    const uint32_t ty = ref_type(c6);
+    const bool use_ref = g_pow2 && ty != 0u && __fmul_rn(t6.x, t6.y) == 1.0f && __fmul_rn(a, t6.y) <= 6.0f;
+    if (use_ref) {
+        unsigned long long allow = 0ull;
+#pragma unroll
+        for (int i = 0; i < B; ++i) {
+            // |x| / S_r <= 6 exactly, so the bin is 0 .. 48
+            const int bin = __float2int_rz(__fmul_rn(__fmul_rn(fabsf(xv[i]), t6.y), 8.0f));
+            allow |= wmask[(ty - 1u) * 49u + (uint32_t)bin];
+        }
+        um &= allow;
+    }
+    pl.best = best;
+    pl.bc = bc;
+    pl.c6 = c6;
+    pl.clo = valid ? clo : c6;
+    pl.chi = chi;
+    pl.um = um;
+    // codes past c6 + 64 (all with k >= 13, so never in a window, for a usable
+    // reference): in practice no block has any, its range above c6 being at
+    // most about 40 codes in either format
+    pl.over = valid && !use_ref && chi > (int)c6 + 64;
+    return pl;
+}
+
+// Capacity of a warp's queue of blocks whose search continues after the
+// shortcuts (a flush takes 32 of them; one step adds at most 32).
+constexpr int kBfQueue = 64;
+
+// Resident CTAs per SM the queued kernel is compiled for (its register cap).
+template <int B>
+constexpr int bfq_min_ctas() { return B <= 4 ? 4 : 3; }
+
+template <int B, typename T, int SFMT>
+__global__ void __launch_bounds__(kThreads, bfq_min_ctas<B>())
+nvfp4_bf_queue_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs,
+                uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, int mma_layout,
+                float* __restrict__ deq, float* __restrict__ mse, unsigned long long* evals,
+                const __grid_constant__ BfWindows win)
+{
+    uint32_t n_eval = 0;   // this lane's error evaluations (seeds, all-zero codes, searches)
+    constexpr uint32_t kLast = SFMT == 1 ? 254u : 126u;
+    constexpr uint32_t kNone = kLast + 1u;
+    // (S, inv) of every code: S = sc * g, inv = min(1/S, FLT_MAX), 0 for S = 0
+    __shared__ float2 tab[kNone + 1];
+    // the window masks, in shared memory: lanes index them by their own bins,
+    // which constant-space reads would serialize
+    __shared__ unsigned long long wmask[4 * 49];
+    __shared__ __align__(16) float xs[kWarps][32 * B];
+    __shared__ unsigned long long key[kWarps][32];
+    __shared__ int pre[kWarps][32];
+    __shared__ uint32_t lowm[kWarps][32];            // next lower code | lower count << 8 | c6 << 16
+    __shared__ unsigned long long upm[kWarps][32];   // upper codes left: bit j = code c6 + 1 + j
+    // the warp's queue of blocks whose search continues: block index (the
+    // launcher keeps nblk below 2^32), the best error so far with `over` in
+    // its sign bit (errors are non-negative), codes (best | c6 << 8 | clo << 16
+    // | chi << 24), the upper-code mask
+    __shared__ uint32_t q_idx[kWarps][kBfQueue];
+    __shared__ unsigned long long q_um[kWarps][kBfQueue];
+    __shared__ uint32_t q_best[kWarps][kBfQueue];
+    __shared__ uint32_t q_codes[kWarps][kBfQueue];
+
+    const float g = resolve_global_scale<T>(gs);
+    const float g6 = __fmul_rn(6.0f, g);
+    // only a starting point for the exact all-zero search
+    const float four_over_g = __fmul_rn(4.0f, __frcp_rn(g));
+    // every S = sc * g and every v * S is exact when g is a moderate power of two
+    const bool g_pow2 = pow2_in_range(g);
+    for (int c = threadIdx.x; c <= (int)kNone; c += blockDim.x) {
+        const float S = __fmul_rn(sf_decode<SFMT>((uint32_t)c < kNone ? (uint32_t)c : kLast), g);
+        tab[c] = make_float2(S, (S == 0.0f) ? 0.0f : fminf(__frcp_rn(S), kFltMax));
+    }
+    for (int i = threadIdx.x; i < 4 * 49; i += blockDim.x)
+        wmask[i] = win.m[i / 49][i % 49];
+    __syncthreads();
+
+    const int lane = threadIdx.x & 31;
+    const int w = threadIdx.x >> 5;
+    const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+    const int64_t kb_atoms = (bpr + 3) >> 2;
+    int64_t r_cur = 0, kb_cur = 0, step_r = 0, step_kb = 0;
+    if (mma_layout) {
+        const int64_t b0 = warp0 * 32 + lane;
+        const int64_t step = nwarps * 32;
+        r_cur = b0 / bpr;
+        kb_cur = b0 % bpr;
+        step_r = step / bpr;
+        step_kb = step % bpr;
+    }
+    float* xw = xs[w];
+
+    // Store block b's result at code bc (its codes at c6 are cw and its error
+    // `best` when bc == c6 and no dequantized output is wanted).
+    auto store_block = [&](int64_t b, const float (&xv)[B], uint32_t bc, uint32_t c6, uint32_t (&cw)[(B + 7) / 8],
+                           float best, int64_t so) {
+        float sse = best;
+        float dq[B];
+        if (bc != c6 || deq)
+            sse = quant_eval<B>(xv, sf_decode<SFMT>(bc), g, cw, dq);
+        store_codes<B>(codes + b * (B / 2), cw);
+        scales[so] = (uint8_t)bc;
+        if (deq)
+            store_f32<B>(deq + b * B, dq);
+        if (mse)
+            mse[b] = __fmul_rn(sse, 1.0f / (float)B);
+    };
+
+    // Finish the first n queued blocks: every lane takes one (reloading its
+    // elements), the warp lays the blocks' remaining (block, code) pairs end to
+    // end and every lane takes every 32nd pair, reading the block from shared
+    // memory; a block's best (error, code) is a 64-bit key lowered with an
+    // atomic minimum (error bits above the code: the lowest code wins ties).
+    auto flush = [&](int n) {
+        const bool act = lane < n;
+        int64_t b = 0;
+        float best = 0.0f;
+        uint32_t bc = 0u, c6 = 1u, clo = 1u;
+        int chi = 0;
+        unsigned long long um = 0ull;
+        bool over = false;
+        float xv[B];
+        if (act) {
+            b = (int64_t)q_idx[w][lane];
+            const uint32_t qb = q_best[w][lane];
+            best = __uint_as_float(qb & 0x7FFFFFFFu);
+            over = (qb >> 31) != 0u;
+            const uint32_t qc = q_codes[w][lane];
+            bc = qc & 0xFFu;
+            c6 = (qc >> 8) & 0xFFu;
+            clo = (qc >> 16) & 0xFFu;
+            chi = (int)(qc >> 24);
+            um = q_um[w][lane];
+            load_elems<T, B>(x + b * B, xv);
+        } else {
+#pragma unroll
+            for (int i = 0; i < B; ++i)
+                xv[i] = 0.0f;
+        }
+        for (int c = (int)c6 + 65; c <= chi && over; ++c) {
+            const float sc_ = quant_sse<B>(xv, 0.0f, 0.0f, tab[c]);
+            n_eval += 1u;
+            if (sc_ < best || (sc_ == best && (uint32_t)c < bc)) {
+                best = sc_;
+                bc = (uint32_t)c;
+            }
+        }
+        const int nlow = act ? (int)(c6 - clo) : 0;
+        const int span = nlow + __popcll(um);
+        int incl = span;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, d);
+            if (lane >= d)
+                incl += v;
+        }
+        const int total = __shfl_sync(0xffffffffu, incl, 31);
+        if (total > 0) {
+#pragma unroll
+            for (int i = 0; i < B; i += 4)
+                *reinterpret_cast<float4*>(&xw[lane * B + i]) = make_float4(xv[i], xv[i + 1], xv[i + 2], xv[i + 3]);
+            key[w][lane] = ((unsigned long long)__float_as_uint(best) << 32) | bc;
+            pre[w][lane] = incl - span;
+            lowm[w][lane] = clo | ((uint32_t)nlow << 8) | (c6 << 16);
+            upm[w][lane] = um;
+            __syncwarp();
+            for (int t = lane; t < total; t += 32) {
+                // owner: the last block whose range starts at or before t
+                int j = 0;
+#pragma unroll
+                for (int st = 16; st > 0; st >>= 1)
+                    if (pre[w][j + st] <= t)
+                        j += st;
+                const uint32_t lm = lowm[w][j];
+                const int k = t - pre[w][j];
+                const int nl = (int)((lm >> 8) & 0xFFu);
+                uint32_t c;
+                if (k < nl) {
+                    c = (lm & 0xFFu) + (uint32_t)k;
+                } else {
+                    unsigned long long m = upm[w][j];
+                    for (int i = nl; i < k; ++i)
+                        m &= m - 1ull;
+                    c = ((lm >> 16) & 0xFFu) + (uint32_t)__ffsll((long long)m);
+                }
+                float xj[B];
+#pragma unroll
+                for (int i = 0; i < B; i += 4) {
+                    const float4 q = *reinterpret_cast<const float4*>(&xw[j * B + i]);
+                    xj[i] = q.x;
+                    xj[i + 1] = q.y;
+                    xj[i + 2] = q.z;
+                    xj[i + 3] = q.w;
+                }
+                const float sc_ = quant_sse<B>(xj, 0.0f, 0.0f, tab[c]);
+                atomicMin(&key[w][j], ((unsigned long long)__float_as_uint(sc_) << 32) | c);
+                ++n_eval;
+            }
+            __syncwarp();
+            bc = (uint32_t)key[w][lane];
+            __syncwarp();
+        }
+        if (act) {
+            uint32_t cw[(B + 7) / 8];
+            const int64_t so = mma_layout ? mma_sf_offset(b / bpr, b % bpr, kb_atoms) : b;
+            store_block(b, xv, bc, 0xFFFFu, cw, best, so);   // never c6: codes from bc
+        }
+    };
+
+    // blocks of up to 32 bytes: the next block's load is in flight while this
+    // one is searched (one load round trip per block otherwise stalls the warp)
+    constexpr bool kPrefetch = B * sizeof(T) <= 32;
+    float xn[kPrefetch ? B : 1];
+    if constexpr (kPrefetch) {
+        const int64_t b0 = warp0 * 32 + lane;
+        if (b0 < nblk) {
+            load_elems<T, B>(x + b0 * B, xn);
+        } else {
+#pragma unroll
+            for (int i = 0; i < B; ++i)
+                xn[i] = 0.0f;
+        }
+    }
+    int pcount = 0;   // queued blocks of this warp (the same in every lane)
+
+    for (int64_t base = warp0 * 32; base < nblk; base += nwarps * 32) {
+        const int64_t b = base + lane;
+        const bool valid = b < nblk;
+        float xv[B];
+        if constexpr (kPrefetch) {
+#pragma unroll
+            for (int i = 0; i < B; ++i)
+                xv[i] = xn[i];
+            const int64_t bn = b + nwarps * 32;
+            if (bn < nblk)
+                load_elems<T, B>(x + bn * B, xn);
+        } else if (valid) {
+            load_elems<T, B>(x + b * B, xv);
+        } else {
+#pragma unroll
+            for (int i = 0; i < B; ++i)
+                xv[i] = 0.0f;
+        }
+        uint32_t cw[(B + 7) / 8];
+        const BfPlan pl = bf_plan<B, SFMT>(xv, valid, tab, wmask, g6, four_over_g, g_pow2, cw, n_eval);
+        const bool pending = valid && (pl.clo < pl.c6 || pl.um != 0ull || pl.over);
+        const int64_t so = mma_layout ? mma_sf_offset(r_cur, kb_cur, kb_atoms) : b;
+        if (valid && !pending)
+            store_block(b, xv, pl.bc, pl.c6, cw, pl.best, so);
+        // queue the blocks whose search continues
+        const uint32_t bal = __ballot_sync(0xffffffffu, pending);
+        if (pending) {
+            const int slot = pcount + __popc(bal & ((1u << lane) - 1u));
+            q_idx[w][slot] = (uint32_t)b;
+            q_best[w][slot] = __float_as_uint(pl.best) | (pl.over ? 0x80000000u : 0u);
+            q_codes[w][slot] = pl.bc | (pl.c6 << 8) | (pl.clo << 16) | ((uint32_t)pl.chi << 24);
+            q_um[w][slot] = pl.um;
+        }
+        pcount += __popc(bal);
+        __syncwarp();
+        if (pcount >= 32) {
+            flush(32);
+            // move the rest of the queue to its front
+            pcount -= 32;
+            uint32_t t_idx = 0, t_best = 0, t_codes = 0;
+            unsigned long long t_um = 0;
+            if (lane < pcount) {
+                t_idx = q_idx[w][32 + lane];
+                t_um = q_um[w][32 + lane];
+                t_best = q_best[w][32 + lane];
+                t_codes = q_codes[w][32 + lane];
+            }
+            __syncwarp();
+            if (lane < pcount) {
+                q_idx[w][lane] = t_idx;
+                q_um[w][lane] = t_um;
+                q_best[w][lane] = t_best;
+                q_codes[w][lane] = t_codes;
+            }
+            __syncwarp();
+        }
+        if (mma_layout) {
+            kb_cur += step_kb;
+            r_cur += step_r;
+            if (kb_cur >= bpr) {
+                kb_cur -= bpr;
+                ++r_cur;
+            }
+        }
+    }
+    if (pcount > 0)
+        flush(pcount);
+    if (evals) {
+        const uint32_t wsum = __reduce_add_sync(0xffffffffu, n_eval);
+        if (lane == 0 && wsum)
+            atomicAdd(evals, (unsigned long long)wsum);
+    }
+}
+
 // ------------------------------------------------------ dequant + MSE
 // SF: 0 E4M3, 1 E3M3, 2 E8M0, 3 UE5M3.  RAZ: the -0 code decodes to the block's
 // special value (selector in the scale byte's top bits).
@@ -1450,6 +1824,13 @@ cudaError_t nvfp4_launch_t(const void* x, int64_t rows, int64_t cols, const GsAr
 {
     const int64_t nblk = rows * (cols / B);
     if constexpr (RULE == R_BF) {
+        // small blocks: the queued search (block indices are kept in 32 bits)
+        if constexpr (B <= 8) {
+            if (nblk < ((int64_t)1 << 32))
+                return launch_quant_kernel(nvfp4_bf_queue_kernel<B, T, SFMT>, nblk, gs, s,
+                                           reinterpret_cast<const T*>(x), nblk, cols / B, gs, codes, scales, mma, deq,
+                                           mse, evals, bf_windows());
+        }
         return launch_quant_kernel(nvfp4_bf_kernel<B, T, SFMT>, nblk, gs, s, reinterpret_cast<const T*>(x), nblk,
                                    cols / B, gs, codes, scales, mma, deq, mse, evals, bf_windows());
     } else {

@@ -463,8 +463,9 @@ FP4Q_API int fp4q_gemm_status(const void* workspace, void* stream);
  * a kernel in which every pair of SMs issues `iters` groups of four
  * back-to-back block-scaled FP4 MMAs of the GEMMs' shape (CTA pair, 256 x 256
  * x 64; mx = 0: kind::mxf4nvf4 with UE4M3 scales per 16, mx = 1: kind::mxf4
- * with UE8M0 scales per 32) on operand tiles held in shared memory and scales
- * copied into TMEM once -- no global traffic and no waits inside the loop.
+ * with UE8M0 scales per 32) on operand tiles held in shared memory (hashed
+ * code bytes, so the operands toggle like real data) and scales copied into
+ * TMEM once -- no global traffic and no waits inside the loop.
  * Enqueued on `stream`; time it with events on that stream and divide
  * fp4q_mma_ceiling_flops(iters) (the flops one launch performs on the current
  * device) by the time.  err: device int (4-byte aligned), set to 1 if the
