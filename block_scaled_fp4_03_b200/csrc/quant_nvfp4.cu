@@ -883,15 +883,16 @@ razer_paired_kernel(const T* __restrict__ x, int64_t nblk, GsArgs gs, SpecialArg
 //    the bin; a block ORs the masks of its elements' bins.  Codes with
 //    k in {2, 4, 6, 8, 12} or k >= 13 add no point below 6 S_r and never
 //    appear in a mask.
-// Every other code of [clo, all-zero code) is evaluated in full: each lane
-// takes the first kDirect of its block's codes from registers; the rest of
-// the warp's (block, code) pairs are laid end to end and every lane takes
-// every 32nd pair, reading the block from shared memory.  A block's best
-// (error, code) is one 64-bit key -- error bits (non-negative floats order
-// like their bits) above the code -- lowered with a shared-memory atomic
-// minimum, so the lowest code wins ties exactly as in a sequential scan.  The
-// seed c6 is evaluated with its codes kept: most blocks keep c6 and are
-// stored without a second encode.
+// Every other code of [clo, all-zero code) is evaluated in full.  A block
+// with none left (most blocks) is stored at once; the seed c6 is evaluated
+// with its codes kept, so a block that keeps c6 needs no second encode.  The
+// others wait in a per-warp queue; once 32 are queued the warp takes them
+// together: each lane reloads one, the (block, code) pairs still to evaluate
+// are laid end to end and every lane takes every 32nd pair, reading the block
+// from shared memory.  A block's best (error, code) is one 64-bit key --
+// error bits (non-negative floats order like their bits) above the code --
+// lowered with a shared-memory atomic minimum, so the lowest code wins ties
+// exactly as in a sequential scan.
 constexpr int kWarps = kThreads / 32;
 
 // Codes and in-order squared error of a block at the candidate t = (S, inv).
@@ -957,292 +958,6 @@ __device__ __forceinline__ uint32_t ref_type(uint32_t c)
     if (c == 0u || (c & (c - 1u)) != 0u)
         return 0u;
     return 33u - (uint32_t)__clz((int)c);   // subnormal 1, 2, 4 -> 2, 3, 4
-}
-
-// Resident CTAs per SM the brute-force kernel is compiled for (its register cap).
-template <int B>
-constexpr int bf_min_ctas() { return B <= 4 ? 5 : B <= 8 ? 4 : B <= 16 ? 3 : 2; }
-
-template <int B, typename T, int SFMT>
-__global__ void __launch_bounds__(kThreads, bf_min_ctas<B>())
-nvfp4_bf_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs,
-                uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, int mma_layout,
-                float* __restrict__ deq, float* __restrict__ mse, unsigned long long* evals,
-                const __grid_constant__ BfWindows win)
-{
-    uint32_t n_eval = 0;   // this lane's error evaluations (seed, all-zero, scan)
-    // the format's largest finite code, and the "no all-zero code" marker
-    constexpr uint32_t kLast = SFMT == 1 ? 254u : 126u;
-    // codes each lane may evaluate itself before the warp shares out the rest
-    constexpr int kDirect = B <= 8 ? 2 : 3;
-    constexpr uint32_t kNone = kLast + 1u;
-    // (S, inv) of every code: S = sc * g, inv = min(1/S, FLT_MAX), 0 for S = 0
-    __shared__ float2 tab[kNone + 1];
-    // the window masks, in shared memory: lanes index them by their own bins,
-    // which constant-space reads would serialize
-    __shared__ unsigned long long wmask[4 * 49];
-    __shared__ __align__(16) float xs[kWarps][32 * B];
-    __shared__ unsigned long long key[kWarps][32];
-    __shared__ int pre[kWarps][32];
-    __shared__ uint32_t lowm[kWarps][32];            // next lower code | lower count << 8 | c6 << 16
-    __shared__ unsigned long long upm[kWarps][32];   // upper codes left: bit j = code c6 + 1 + j
-
-    const float g = resolve_global_scale<T>(gs);
-    const float g6 = __fmul_rn(6.0f, g);
-    // only a starting point for the exact all-zero search below
-    const float four_over_g = __fmul_rn(4.0f, __frcp_rn(g));
-    // every S = sc * g and every v * S is exact when g is a moderate power of two
-    const bool g_pow2 = pow2_in_range(g);
-    for (int c = threadIdx.x; c <= (int)kNone; c += blockDim.x) {
-        const float S = __fmul_rn(sf_decode<SFMT>((uint32_t)c < kNone ? (uint32_t)c : kLast), g);
-        tab[c] = make_float2(S, (S == 0.0f) ? 0.0f : fminf(__frcp_rn(S), kFltMax));
-    }
-    for (int i = threadIdx.x; i < 4 * 49; i += blockDim.x)
-        wmask[i] = win.m[i / 49][i % 49];
-    __syncthreads();
-
-    const int lane = threadIdx.x & 31;
-    const int w = threadIdx.x >> 5;
-    const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
-    const int64_t kb_atoms = (bpr + 3) >> 2;
-    int64_t r_cur = 0, kb_cur = 0, step_r = 0, step_kb = 0;
-    if (mma_layout) {
-        const int64_t b0 = warp0 * 32 + lane;
-        const int64_t step = nwarps * 32;
-        r_cur = b0 / bpr;
-        kb_cur = b0 % bpr;
-        step_r = step / bpr;
-        step_kb = step % bpr;
-    }
-    float* xw = xs[w];
-    // blocks of up to 32 bytes: the next block's load is in flight while this
-    // one is searched (one load round trip per block otherwise stalls the warp)
-    constexpr bool kPrefetch = B * sizeof(T) <= 32;
-    float xn[kPrefetch ? B : 1];
-    if constexpr (kPrefetch) {
-        const int64_t b0 = warp0 * 32 + lane;
-        if (b0 < nblk) {
-            load_elems<T, B>(x + b0 * B, xn);
-        } else {
-#pragma unroll
-            for (int i = 0; i < B; ++i)
-                xn[i] = 0.0f;
-        }
-    }
-
-    for (int64_t base = warp0 * 32; base < nblk; base += nwarps * 32) {
-        const int64_t b = base + lane;
-        const bool valid = b < nblk;
-        float xv[B];
-        if constexpr (kPrefetch) {
-#pragma unroll
-            for (int i = 0; i < B; ++i)
-                xv[i] = xn[i];
-            const int64_t bn = b + nwarps * 32;
-            if (bn < nblk)
-                load_elems<T, B>(x + bn * B, xn);
-        } else if (valid) {
-            load_elems<T, B>(x + b * B, xv);
-        } else {
-#pragma unroll
-            for (int i = 0; i < B; ++i)
-                xv[i] = 0.0f;
-        }
-        float a = 0.0f;
-        float sse0 = 0.0f;
-#pragma unroll
-        for (int i = 0; i < B; ++i) {
-            a = fmaxf(a, fabsf(xv[i]));
-            sse0 = __fmaf_rn(xv[i], xv[i], sse0);
-        }
-        uint32_t c6 = sf_encode<SFMT>(__fdiv_rn(a, g6));
-        c6 = c6 == 0u ? 1u : c6;
-        const float2 t6 = tab[c6];
-        uint32_t cw[(B + 7) / 8];
-        float best = quant_codes_sse<B>(xv, t6, cw);
-        uint32_t bc = c6;
-        n_eval += valid ? 1u : 0u;
-        // first all-zero code (kNone = none): step from a nearby code to the
-        // boundary (|y| is monotone in the code)
-        uint32_t cz = sf_encode<SFMT>(__fmul_rn(a, four_over_g));
-        cz = cz == 0u ? 1u : cz;
-        {
-            // usually the boundary is cz or cz + 1: test both without a loop
-            const bool f0 = cz > 1u && __fmul_rn(a, tab[cz - 1u].y) <= 0.25f;
-            const bool f1 = __fmul_rn(a, tab[cz].y) <= 0.25f;
-            const bool f2 = cz + 1u >= kNone || __fmul_rn(a, tab[cz + 1u].y) <= 0.25f;
-            if (f1 && !f0) {
-            } else if (!f1 && f2) {
-                ++cz;
-            } else if (f1) {
-                --cz;
-                while (cz > 1u && __fmul_rn(a, tab[cz - 1u].y) <= 0.25f)
-                    --cz;
-            } else {
-                ++cz;
-                do {
-                    ++cz;
-                } while (cz < kNone && __fmul_rn(a, tab[cz].y) > 0.25f);
-            }
-        }
-        n_eval += (valid && cz < kNone) ? 1u : 0u;
-        if (cz < kNone && (sse0 < best || (sse0 == best && cz < bc))) {
-            best = sse0;
-            bc = cz;
-        }
-        // downward: codes below c6 while the clipped bound can still win
-        uint32_t clo = c6;
-        while (clo > 1u) {
-            const float2 t = tab[clo - 1u];
-            const float em = elem_err(a, t.x, t.y);
-            if (__fmul_rn(em, em) > best)
-                break;
-            --clo;
-        }
-        // the block's code list: clo .. c6 - 1, then the codes of (c6, chi]
-        // the lattice shortcut leaves, as a mask over c6 + 1 + j
-        const int chi = (int)(cz < kNone ? cz : kNone) - 1;   // last code to evaluate
-        const int nup = valid ? chi - (int)c6 : 0;
-        unsigned long long um = nup <= 0 ? 0ull : nup >= 64 ? ~0ull : ((1ull << nup) - 1ull);
-        // c6 is a usable reference: a power-of-two scale with an exact
-        // reciprocal at which no element clips; then only the codes whose
-        // windows hold an element stay
-        const uint32_t ty = ref_type(c6);
-        const bool use_ref = g_pow2 && ty != 0u && __fmul_rn(t6.x, t6.y) == 1.0f && __fmul_rn(a, t6.y) <= 6.0f;
-        if (use_ref) {
-            unsigned long long allow = 0ull;
-#pragma unroll
-            for (int i = 0; i < B; ++i) {
-                // |x| / S_r <= 6 exactly, so the bin is 0 .. 48
-                const int bin = __float2int_rz(__fmul_rn(__fmul_rn(fabsf(xv[i]), t6.y), 8.0f));
-                allow |= wmask[(ty - 1u) * 49u + (uint32_t)bin];
-            }
-            um &= allow;
-        }
-        int nlow = valid ? (int)(c6 - clo) : 0;
-        uint32_t lo_next = clo;
-        // codes past c6 + 64 (all with k >= 13, so never in a window, for a
-        // usable reference): in practice no block has any, its range above c6
-        // being at most about 40 codes in either format
-        for (int c = (int)c6 + 65; c <= chi && valid && !use_ref; ++c) {
-            const float sc_ = quant_sse<B>(xv, 0.0f, 0.0f, tab[c]);
-            n_eval += 1u;
-            if (sc_ < best || (sc_ == best && (uint32_t)c < bc)) {
-                best = sc_;
-                bc = (uint32_t)c;
-            }
-        }
-        // the first kDirect codes of the list straight from registers (most
-        // warps have none left after the shortcuts)
-#pragma unroll
-        for (int s = 0; s < kDirect; ++s) {
-            if (!__any_sync(0xffffffffu, nlow > 0 || um != 0ull))
-                break;
-            uint32_t c = 0u;
-            if (nlow > 0) {
-                c = lo_next++;
-                --nlow;
-            } else if (um != 0ull) {
-                c = c6 + (uint32_t)__ffsll((long long)um);
-                um &= um - 1ull;
-            }
-            if (c != 0u) {
-                const float sc_ = quant_sse<B>(xv, 0.0f, 0.0f, tab[c]);
-                n_eval += 1u;
-                if (sc_ < best || (sc_ == best && c < bc)) {
-                    best = sc_;
-                    bc = c;
-                }
-            }
-        }
-        const int span = nlow + __popcll(um);
-
-        // lay the warp's remaining candidates end to end
-        int incl = span;
-#pragma unroll
-        for (int d = 1; d < 32; d <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, incl, d);
-            if (lane >= d)
-                incl += v;
-        }
-        const int total = __shfl_sync(0xffffffffu, incl, 31);
-        if (total > 0) {
-#pragma unroll
-            for (int i = 0; i < B; i += 4)
-                *reinterpret_cast<float4*>(&xw[lane * B + i]) =
-                    make_float4(xv[i], xv[i + 1], xv[i + 2], xv[i + 3]);
-            key[w][lane] = ((unsigned long long)__float_as_uint(best) << 32) | bc;
-            pre[w][lane] = incl - span;
-            lowm[w][lane] = lo_next | ((uint32_t)nlow << 8) | (c6 << 16);   // 8 bits each
-            upm[w][lane] = um;
-            __syncwarp();
-            for (int t = lane; t < total; t += 32) {
-                // owner: the last block whose range starts at or before t
-                int j = 0;
-#pragma unroll
-                for (int st = 16; st > 0; st >>= 1)
-                    if (pre[w][j + st] <= t)
-                        j += st;
-                const uint32_t lm = lowm[w][j];
-                const int k = t - pre[w][j];
-                const int nl = (int)((lm >> 8) & 0xFFu);
-                uint32_t c;
-                if (k < nl) {
-                    c = (lm & 0xFFu) + (uint32_t)k;
-                } else {
-                    unsigned long long m = upm[w][j];
-                    for (int i = nl; i < k; ++i)
-                        m &= m - 1ull;
-                    c = ((lm >> 16) & 0xFFu) + (uint32_t)__ffsll((long long)m);
-                }
-                float xj[B];
-#pragma unroll
-                for (int i = 0; i < B; i += 4) {
-                    const float4 q = *reinterpret_cast<const float4*>(&xw[j * B + i]);
-                    xj[i] = q.x;
-                    xj[i + 1] = q.y;
-                    xj[i + 2] = q.z;
-                    xj[i + 3] = q.w;
-                }
-                const float sc_ = quant_sse<B>(xj, 0.0f, 0.0f, tab[c]);
-                atomicMin(&key[w][j], ((unsigned long long)__float_as_uint(sc_) << 32) | c);
-                ++n_eval;
-            }
-            __syncwarp();
-            bc = (uint32_t)key[w][lane];
-            __syncwarp();
-        }
-
-        // c6 kept: its codes and error are already in registers
-        float sse = best;
-        float dq[B];
-        if (bc != c6 || deq) {
-            sse = quant_eval<B>(xv, sf_decode<SFMT>(bc), g, cw, dq);
-        }
-        if (valid) {
-            store_codes<B>(codes + b * (B / 2), cw);
-            const int64_t so = mma_layout ? mma_sf_offset(r_cur, kb_cur, kb_atoms) : b;
-            scales[so] = (uint8_t)bc;
-            if (deq)
-                store_f32<B>(deq + b * B, dq);
-            if (mse)
-                mse[b] = __fmul_rn(sse, 1.0f / (float)B);
-        }
-        if (mma_layout) {
-            kb_cur += step_kb;
-            r_cur += step_r;
-            if (kb_cur >= bpr) {
-                kb_cur -= bpr;
-                ++r_cur;
-            }
-        }
-    }
-    if (evals) {
-        const uint32_t wsum = __reduce_add_sync(0xffffffffu, n_eval);
-        if (lane == 0 && wsum)
-            atomicAdd(evals, (unsigned long long)wsum);
-    }
 }
 
 // A block's search after the exact shortcuts: the better of c6 and the
@@ -1349,13 +1064,13 @@ __device__ __forceinline__ BfPlan bf_plan(const float (&xv)[B], bool valid, cons
 // shortcuts (a flush takes 32 of them; one step adds at most 32).
 constexpr int kBfQueue = 64;
 
-// Resident CTAs per SM the queued kernel is compiled for (its register cap).
+// Resident CTAs per SM the brute-force kernel is compiled for (its register cap).
 template <int B>
-constexpr int bfq_min_ctas() { return B <= 4 ? 4 : 3; }
+constexpr int bf_min_ctas() { return B <= 4 ? 4 : B <= 8 ? 3 : 2; }
 
 template <int B, typename T, int SFMT>
-__global__ void __launch_bounds__(kThreads, bfq_min_ctas<B>())
-nvfp4_bf_queue_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs,
+__global__ void __launch_bounds__(kThreads, bf_min_ctas<B>())
+nvfp4_bf_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs,
                 uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, int mma_layout,
                 float* __restrict__ deq, float* __restrict__ mse, unsigned long long* evals,
                 const __grid_constant__ BfWindows win)
@@ -1368,16 +1083,16 @@ nvfp4_bf_queue_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs
     // the window masks, in shared memory: lanes index them by their own bins,
     // which constant-space reads would serialize
     __shared__ unsigned long long wmask[4 * 49];
-    __shared__ __align__(16) float xs[kWarps][32 * B];
+    // each warp's 32 blocks being searched (dynamic: kWarps * 32 * B floats)
+    extern __shared__ __align__(16) float blk_xs[];
     __shared__ unsigned long long key[kWarps][32];
     __shared__ int pre[kWarps][32];
     __shared__ uint32_t lowm[kWarps][32];            // next lower code | lower count << 8 | c6 << 16
     __shared__ unsigned long long upm[kWarps][32];   // upper codes left: bit j = code c6 + 1 + j
-    // the warp's queue of blocks whose search continues: block index (the
-    // launcher keeps nblk below 2^32), the best error so far with `over` in
-    // its sign bit (errors are non-negative), codes (best | c6 << 8 | clo << 16
-    // | chi << 24), the upper-code mask
-    __shared__ uint32_t q_idx[kWarps][kBfQueue];
+    // the warp's queue of blocks whose search continues: block index, the
+    // best error so far with `over` in its sign bit (errors are non-negative),
+    // codes (best | c6 << 8 | clo << 16 | chi << 24), the upper-code mask
+    __shared__ unsigned long long q_idx[kWarps][kBfQueue];
     __shared__ unsigned long long q_um[kWarps][kBfQueue];
     __shared__ uint32_t q_best[kWarps][kBfQueue];
     __shared__ uint32_t q_codes[kWarps][kBfQueue];
@@ -1410,7 +1125,7 @@ nvfp4_bf_queue_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs
         step_r = step / bpr;
         step_kb = step % bpr;
     }
-    float* xw = xs[w];
+    float* xw = blk_xs + w * 32 * B;
 
     // Store block b's result at code bc (its codes at c6 are cw and its error
     // `best` when bc == c6 and no dequantized output is wanted).
@@ -1573,7 +1288,7 @@ nvfp4_bf_queue_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs
         const uint32_t bal = __ballot_sync(0xffffffffu, pending);
         if (pending) {
             const int slot = pcount + __popc(bal & ((1u << lane) - 1u));
-            q_idx[w][slot] = (uint32_t)b;
+            q_idx[w][slot] = (unsigned long long)b;
             q_best[w][slot] = __float_as_uint(pl.best) | (pl.over ? 0x80000000u : 0u);
             q_codes[w][slot] = pl.bc | (pl.c6 << 8) | (pl.clo << 16) | ((uint32_t)pl.chi << 24);
             q_um[w][slot] = pl.um;
@@ -1584,8 +1299,8 @@ nvfp4_bf_queue_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs
             flush(32);
             // move the rest of the queue to its front
             pcount -= 32;
-            uint32_t t_idx = 0, t_best = 0, t_codes = 0;
-            unsigned long long t_um = 0;
+            uint32_t t_best = 0, t_codes = 0;
+            unsigned long long t_idx = 0, t_um = 0;
             if (lane < pcount) {
                 t_idx = q_idx[w][32 + lane];
                 t_um = q_um[w][32 + lane];
@@ -1738,11 +1453,14 @@ dequant_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ sc
 template <typename... KArgs, typename... Args>
 cudaError_t launch_quant_kernel(void (*kernel)(KArgs...), int64_t nblk, const GsArgs& gs, cudaStream_t s,
                                 Args&&... args);
+template <typename... KArgs, typename... Args>
+cudaError_t launch_quant_kernel_smem(void (*kernel)(KArgs...), int64_t nblk, const GsArgs& gs, cudaStream_t s,
+                                     int dyn_smem, Args&&... args);
 
-int grid_for(int64_t work_threads, const void* kernel)
+int grid_for(int64_t work_threads, const void* kernel, size_t dyn_smem = 0)
 {
     int per_sm = 0;
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, 0);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, dyn_smem);
     if (per_sm < 1)
         per_sm = 1;
     int64_t want = (work_threads + kThreads - 1) / kThreads;
@@ -1800,7 +1518,20 @@ template <typename... KArgs, typename... Args>
 cudaError_t launch_quant_kernel(void (*kernel)(KArgs...), int64_t nblk, const GsArgs& gs, cudaStream_t s,
                                 Args&&... args)
 {
-    int grid = grid_for(nblk, (const void*)kernel);
+    return launch_quant_kernel_smem(kernel, nblk, gs, s, 0, std::forward<Args>(args)...);
+}
+
+// The same with `dyn_smem` bytes of dynamic shared memory per CTA.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_quant_kernel_smem(void (*kernel)(KArgs...), int64_t nblk, const GsArgs& gs, cudaStream_t s,
+                                     int dyn_smem, Args&&... args)
+{
+    if (dyn_smem > 0) {
+        const cudaError_t e = smem_opt_in((const void*)kernel, dyn_smem);
+        if (e != cudaSuccess)
+            return e;
+    }
+    int grid = grid_for(nblk, (const void*)kernel, (size_t)dyn_smem);
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     if (gs.mode == 3) {
@@ -1812,7 +1543,7 @@ cudaError_t launch_quant_kernel(void (*kernel)(KArgs...), int64_t nblk, const Gs
     }
     cfg.gridDim = dim3((unsigned)grid);
     cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = 0;
+    cfg.dynamicSmemBytes = (size_t)dyn_smem;
     cfg.stream = s;
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
@@ -1824,15 +1555,9 @@ cudaError_t nvfp4_launch_t(const void* x, int64_t rows, int64_t cols, const GsAr
 {
     const int64_t nblk = rows * (cols / B);
     if constexpr (RULE == R_BF) {
-        // small blocks: the queued search (block indices are kept in 32 bits)
-        if constexpr (B <= 8) {
-            if (nblk < ((int64_t)1 << 32))
-                return launch_quant_kernel(nvfp4_bf_queue_kernel<B, T, SFMT>, nblk, gs, s,
-                                           reinterpret_cast<const T*>(x), nblk, cols / B, gs, codes, scales, mma, deq,
-                                           mse, evals, bf_windows());
-        }
-        return launch_quant_kernel(nvfp4_bf_kernel<B, T, SFMT>, nblk, gs, s, reinterpret_cast<const T*>(x), nblk,
-                                   cols / B, gs, codes, scales, mma, deq, mse, evals, bf_windows());
+        return launch_quant_kernel_smem(nvfp4_bf_kernel<B, T, SFMT>, nblk, gs, s,
+                                        kWarps * 32 * B * (int)sizeof(float), reinterpret_cast<const T*>(x), nblk,
+                                        cols / B, gs, codes, scales, mma, deq, mse, evals, bf_windows());
     } else {
         return launch_quant_kernel(nvfp4_quant_kernel<B, T, RULE, SFMT>, nblk, gs, s, reinterpret_cast<const T*>(x),
                                    nblk, cols / B, gs, codes, scales, mma, deq, mse);
