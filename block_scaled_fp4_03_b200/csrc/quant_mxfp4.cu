@@ -542,19 +542,26 @@ hessian_reduce_kernel(const float* __restrict__ part, int64_t nchunk, int64_t to
 }
 
 // ------------------------------------------------------- channel scale
-// Column statistics in fp64 over a chunk of rows: sum and sum of squares.
-// One thread owns 8 consecutive columns (one 16-byte bf16 vector or two fp32
-// vectors) for every row of the chunk.
-constexpr int kStatRows = 64;
+// Column statistics in fp64 over a chunk of kStatRows rows: sum and sum of
+// squares.  A CTA covers 256 columns: lane l of every warp owns the 8
+// consecutive columns 8 l .. 8 l + 7 of the tile (one 16-byte bf16 vector or
+// two fp32 vectors per row), and warp w takes rows w, w + 8, w + 16, ... of the
+// chunk, 8 rows per batch with all 8 loads issued before the sums.  The 8
+// warps' partial sums are then added in warp order through shared memory.
+constexpr int kStatRows = 256;
+constexpr int kStatCols = 256;
+constexpr int kStatWarps = kThreads / 32;
 
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
 column_stats_kernel(const T* __restrict__ x, int64_t rows, int64_t cols, double* __restrict__ sum,
                     double* __restrict__ sumsq)
 {
-    const int64_t c0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 8;
-    if (c0 >= cols)
-        return;
+    __shared__ double red[2][kStatWarps][kStatCols];
+    const int lane = threadIdx.x & 31;
+    const int warp = threadIdx.x >> 5;
+    const int64_t c0 = (int64_t)blockIdx.x * kStatCols + 8 * lane;
+    const bool own = c0 < cols;
     const int64_t r0 = (int64_t)blockIdx.y * kStatRows;
     const int64_t r1 = (r0 + kStatRows) < rows ? (r0 + kStatRows) : rows;
     double s[8], q[8];
@@ -563,40 +570,53 @@ column_stats_kernel(const T* __restrict__ x, int64_t rows, int64_t cols, double*
         s[i] = 0.0;
         q[i] = 0.0;
     }
-    // rows in groups of 8 with all 8 loads issued before the sums, so each
-    // thread keeps 8 vectors in flight
-    int64_t r = r0;
-    for (; r + 8 <= r1; r += 8) {
-        float v[8][8];
+    int64_t r = r0 + warp;
+    if (own) {
+        for (; r + 7 * kStatWarps < r1; r += 8 * kStatWarps) {
+            float v[8][8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k)
-            load_elems<T, 8>(x + (r + k) * cols + c0, v[k]);
+            for (int k = 0; k < 8; ++k)
+                load_elems<T, 8>(x + (r + k * kStatWarps) * cols + c0, v[k]);
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
+            for (int k = 0; k < 8; ++k) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const double d = (double)v[k][i];
+                    s[i] += d;
+                    q[i] = fma(d, d, q[i]);
+                }
+            }
+        }
+        for (; r < r1; r += kStatWarps) {
+            float v[8];
+            load_elems<T, 8>(x + r * cols + c0, v);
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                const double d = (double)v[k][i];
+                const double d = (double)v[i];
                 s[i] += d;
                 q[i] = fma(d, d, q[i]);
             }
         }
     }
-    for (; r < r1; ++r) {
-        float v[8];
-        load_elems<T, 8>(x + r * cols + c0, v);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const double d = (double)v[i];
-            s[i] += d;
-            q[i] = fma(d, d, q[i]);
-        }
-    }
-    const int64_t o = (int64_t)blockIdx.y * cols + c0;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
+        red[0][warp][8 * lane + i] = s[i];
+        red[1][warp][8 * lane + i] = q[i];
+    }
+    __syncthreads();
+    // thread t finishes column t of the tile
+    const int64_t c = (int64_t)blockIdx.x * kStatCols + threadIdx.x;
+    if (c < cols) {
+        double ts = red[0][0][threadIdx.x], tq = red[1][0][threadIdx.x];
+#pragma unroll
+        for (int w = 1; w < kStatWarps; ++w) {
+            ts += red[0][w][threadIdx.x];
+            tq += red[1][w][threadIdx.x];
+        }
+        const int64_t o = (int64_t)blockIdx.y * cols + c;
         if (sum)
-            sum[o + i] = s[i];
-        sumsq[o + i] = q[i];
+            sum[o] = ts;
+        sumsq[o] = tq;
     }
 }
 
@@ -1002,7 +1022,7 @@ cudaError_t launch_mx_channel_scale(const void* x, int xdt, int64_t tokens, cons
     double* wsum = reinterpret_cast<double*>(ws);
     double* wsq = wsum + wch * cols;
     double* xsq = wsq + wch * cols;
-    const unsigned gx = (unsigned)((cols / 8 + kThreads - 1) / kThreads);
+    const unsigned gx = (unsigned)((cols + kStatCols - 1) / kStatCols);
     if (wdt == 1)
         column_stats_kernel<__nv_bfloat16><<<dim3(gx, (unsigned)wch), kThreads, 0, s>>>(
             reinterpret_cast<const __nv_bfloat16*>(w), n_out, cols, wsum, wsq);
