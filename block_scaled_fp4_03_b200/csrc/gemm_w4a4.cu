@@ -483,22 +483,28 @@ w4a4_gemm_1sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
 // issuer waits on that barrier and issues only the four MMAs.  One thread
 // issuing 12 copies and 4 MMAs per stage was the bound: the copies cost as
 // much issue time as the MMAs, and split across warps they overlap.
-// The epilogue stages bf16 32 x 64 boxes in 128B-swizzled shared memory (two
-// boxes, half a tile row, at a time) and writes them with TMA stores, handing
-// the accumulator back as soon as its TMEM reads are done, so the stores
-// overlap the next tile's main loop.  Five 38 KiB stages keep ~190 KiB of
-// operands in flight per SM.
+// Eight epilogue warps per CTA, two per TMEM lane quarter, each own 128 of the
+// 256 accumulator columns of its 32 rows: the TMEM reads of a tile take half
+// as long as with one warp per quarter, and the accumulator goes back to the
+// MMA issuer as soon as they are done (the next tile's MMAs wait on it; one
+// accumulator is all TMEM holds beside the scale slots).  A warp stages one
+// bf16 32 x 64 box in 128B-swizzled shared memory at a time and writes it with
+// a TMA store, so the stores overlap the next tile's main loop.  Five 38 KiB
+// stages keep ~190 KiB of operands in flight per SM.
 constexpr int k2Stages = 5;
 constexpr int k2AStage = 128 * kBK / 2;        // 16 KiB
 constexpr int k2BStage = 128 * kBK / 2;        // 16 KiB (this CTA's half of B)
 constexpr int k2SfaStage = 128 * kBK / 16;     // 2 KiB
 constexpr int k2SfbStage = 256 * kBK / 16;     // 4 KiB (both B row atoms)
 constexpr int k2StageBytes = k2AStage + k2BStage + k2SfaStage + k2SfbStage;
-constexpr int k2EpiWarpBytes = 32 * 128 * 2;   // 32 rows x 128 bf16 per epilogue warp (half a tile row)
-constexpr int k2EpiBytes = 4 * k2EpiWarpBytes;
+constexpr int k2EpiWarpBytes = 32 * 64 * 2;    // one 32-row x 64-column bf16 box per epilogue warp
+constexpr int k2EpiBytes = 8 * k2EpiWarpBytes;
 constexpr int k2SmemBytes = k2Stages * k2StageBytes + k2EpiBytes + 1024 + kBarBytes;
-// warp 0 producer, warp 1 MMA issuer, warps 2-5 epilogue, warps 6-8 scale copies
-constexpr int k2Threads = 288;
+// warp 0 producer, warp 1 MMA issuer, warps 2-5 and 9-12 epilogue (two per
+// TMEM lane quarter: accumulator columns 0-127 and 128-255), warps 6-8 scale
+// copies.  Thirteen warps: one sub-partition holds four of them, so a thread
+// may use at most 128 registers.
+constexpr int k2Threads = 416;
 static_assert(8 * (3 * k2Stages + 7) + 8 <= kBarBytes, "barrier area");
 static_assert(k2StageBytes % 1024 == 0 && (k2Stages * k2StageBytes) % 1024 == 0, "swizzle alignment");
 static_assert(k2SmemBytes <= 232448, "shared memory budget");
@@ -565,11 +571,11 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t sr
                  : "memory");
 }
 
-// Write 32 bf16 columns (chunk c of 8 across the 256-column row half-pair)
-// of row `lane` into the epilogue staging: box (c/2)%2 holds columns
-// [64 (c/2 % 2), +64) of a 128-column half; row `lane` of a box is 128 bytes
-// whose 16-byte chunks sit at (chunk ^ (row % 8)), the 128-byte swizzle the
-// output tensor map expects.
+// Write 32 bf16 columns (chunk c) of row `lane` into the epilogue staging:
+// box (c/2)%2 at offset 4096 holds chunks with (c/2)%2 set, and chunk c fills
+// half c%2 of the box's 128-byte row; row `lane` of a box is 128 bytes whose
+// 16-byte chunks sit at (chunk ^ (row % 8)), the 128-byte swizzle the output
+// tensor map expects.  The pair kernel's warps own one box (c = 0, 1).
 __device__ __forceinline__ void stage_row_chunk(uint8_t* stg, int c, int lane, const uint32_t (&h)[16])
 {
     uint8_t* rowp = stg + ((c >> 1) & 1) * 4096 + lane * 128;
@@ -618,7 +624,7 @@ w4a4_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
             mbar_init(sf_ready_bar(s), 3);
         }
         mbar_init(acc_full, 1);
-        mbar_init(acc_empty, 2 * 128);
+        mbar_init(acc_empty, 2 * 256);
         mbar_init(drain, 1);
         mbar_init(bye, 1);
         for (int w = 0; w < 3; ++w)
@@ -757,7 +763,7 @@ w4a4_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                     give_up();
             }
         }
-    } else if (warp >= 6) {
+    } else if (warp >= 6 && warp <= 8) {
         if (lane == 0 && leader) {
             // ------------------------------- scale-copy warps (leader), one
             // atom column each: 0 SFA, 1 SFB rows 0-127, 2 SFB rows 128-255
@@ -804,8 +810,12 @@ w4a4_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
         }
     } else {
         // ------------------------------------------------ epilogue (both CTAs)
+        // eight warps: warp w reads TMEM lane quarter w % 4, accumulator
+        // columns 128 * half .. 128 * half + 127, converts them to bf16 in
+        // registers and hands the accumulator back before staging and storing
         const int q = warp & 3;
-        uint8_t* stg = epi + q * k2EpiWarpBytes;
+        const int half = warp >= 9 ? 1 : 0;
+        uint8_t* stg = epi + (q + 4 * half) * k2EpiWarpBytes;
         const uint32_t leader_acc_empty = mapa_rank(acc_empty, 0);
         uint32_t acc_phase = 0;
         const float scale = p.ga ? __fmul_rn(__ldg(p.ga), __ldg(p.gw)) : 1.0f;
@@ -820,18 +830,19 @@ w4a4_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
             tc_fence_after();
             const int mt = tile % p.tiles_m;
             const int nt = tile / p.tiles_m;
-            const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16);
+            const uint32_t tq = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(128 * half);
             if constexpr (OUTF32) {
                 // fp32 output: each lane writes its own accumulator row directly
                 float* orow = static_cast<float*>(p.out) +
-                              (int64_t)(mt * 256 + (int)rank * 128 + q * 32 + lane) * p.N + (int64_t)nt * 256;
+                              (int64_t)(mt * 256 + (int)rank * 128 + q * 32 + lane) * p.N + (int64_t)nt * 256 +
+                              128 * half;
 #pragma unroll 1
-                for (int c2 = 0; c2 < 4; ++c2) {
-                    uint32_t r[64];
-                    tmem_ld64(tq + 64 * c2, r);
-                    float4* dst = reinterpret_cast<float4*>(orow + 64 * c2);
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t r[32];
+                    tmem_ld32(tq + 32 * c, r);
+                    float4* dst = reinterpret_cast<float4*>(orow + 32 * c);
 #pragma unroll
-                    for (int j = 0; j < 16; ++j)
+                    for (int j = 0; j < 8; ++j)
                         dst[j] = make_float4(__fmul_rn(__uint_as_float(r[4 * j]), scale),
                                              __fmul_rn(__uint_as_float(r[4 * j + 1]), scale),
                                              __fmul_rn(__uint_as_float(r[4 * j + 2]), scale),
@@ -842,59 +853,50 @@ w4a4_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
                 acc_phase ^= 1u;
                 continue;
             }
-            // the previous tile's stores have finished reading the staging buffer
+            // the warp's 128 columns, 32 per TMEM load: the first 64 go to the
+            // staging box, the other 64 stay in registers as bf16 pairs, and the
+            // accumulator goes back to the MMA issuer before any store is waited for
             if (lane == 0)
                 asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
             __syncwarp();
-            // columns [0, 128) of the accumulator row go to the staging buffer,
-            // columns [128, 256) stay in registers as bf16: the accumulator
-            // goes back to the MMA issuer before any store is waited for
-            uint32_t pk[4][16];
+            uint32_t pk[2][16];
 #pragma unroll
-            for (int c2 = 0; c2 < 4; ++c2) {
-                // two 32-column chunks per TMEM load: half the load round trips
-                uint32_t r[64];
-                tmem_ld64(tq + 64 * c2, r);
+            for (int c = 0; c < 4; ++c) {
+                uint32_t r[32];
+                tmem_ld32(tq + 32 * c, r);
+                uint32_t h16[16];
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int c = 2 * c2 + h;
-                    uint32_t h16[16];
+                for (int j = 0; j < 16; ++j) {
+                    __nv_bfloat162 b = __floats2bfloat162_rn(__fmul_rn(__uint_as_float(r[2 * j]), scale),
+                                                             __fmul_rn(__uint_as_float(r[2 * j + 1]), scale));
+                    h16[j] = *reinterpret_cast<uint32_t*>(&b);
+                }
+                if (c < 2) {
+                    stage_row_chunk(stg, c, lane, h16);
+                } else {
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        __nv_bfloat162 b = __floats2bfloat162_rn(
-                            __fmul_rn(__uint_as_float(r[32 * h + 2 * j]), scale),
-                            __fmul_rn(__uint_as_float(r[32 * h + 2 * j + 1]), scale));
-                        h16[j] = *reinterpret_cast<uint32_t*>(&b);
-                    }
-                    if (c < 4) {
-                        stage_row_chunk(stg, c, lane, h16);
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 16; ++j)
-                            pk[c - 4][j] = h16[j];
-                    }
+                    for (int j = 0; j < 16; ++j)
+                        pk[c - 2][j] = h16[j];
                 }
             }
             tc_fence_before();
             mbar_arrive_cluster(leader_acc_empty);
+            const int x0 = nt * 256 + 128 * half;
             const int y = mt * 256 + (int)rank * 128 + q * 32;
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             __syncwarp();
             if (lane == 0) {
-                tma_store_2d(&tmOut, smem_u32(stg), nt * 256, y);
-                tma_store_2d(&tmOut, smem_u32(stg + 4096), nt * 256 + 64, y);
+                tma_store_2d(&tmOut, smem_u32(stg), x0, y);
                 asm volatile("cp.async.bulk.commit_group;" ::: "memory");
                 asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
             }
             __syncwarp();
-#pragma unroll
-            for (int c = 4; c < 8; ++c)
-                stage_row_chunk(stg, c, lane, pk[c - 4]);
+            stage_row_chunk(stg, 0, lane, pk[0]);
+            stage_row_chunk(stg, 1, lane, pk[1]);
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             __syncwarp();
             if (lane == 0) {
-                tma_store_2d(&tmOut, smem_u32(stg), nt * 256 + 128, y);
-                tma_store_2d(&tmOut, smem_u32(stg + 4096), nt * 256 + 192, y);
+                tma_store_2d(&tmOut, smem_u32(stg), x0 + 64, y);
                 asm volatile("cp.async.bulk.commit_group;" ::: "memory");
             }
             acc_phase ^= 1u;
