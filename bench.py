@@ -63,17 +63,26 @@ def load_peaks():
 # Per-launch DRAM traffic of a row's kernel, from the committed ncu summary of
 # that kernel on the same workload (profiles/*.md); rows without one report null.
 PROFILE_OF_ROW = {
+    "c1_nvfp4_pz_deq_mse": "nvfp4_quant_kernel_B16_pz_deq_mse_gaussian_4096x4096.md",
+    "c1_dequant_mse": "dequant_kernel_B16_e4m3_gaussian_4096x4096.md",
     "c2_B4_bf": "nvfp4_bf_kernel_B4_student_t_8192x8192.md",
+    "c2_B8_bf": "nvfp4_bf_kernel_B8_student_t_8192x8192.md",
+    "c2_B16_bf": "nvfp4_bf_kernel_B16_student_t_8192x8192.md",
+    "c2_B32_bf": "nvfp4_bf_kernel_B32_student_t_8192x8192.md",
     "c2_B4_4o6": "nvfp4_quant_kernel_B4_4o6_student_t_8192x8192.md",
     "c2_B16_absmax": "nvfp4_quant_kernel_B16_absmax_student_t_8192x8192.md",
     "c3_razer_weight": "razer_paired_kernel_weights_8192x8192_bf16.md",
     "c3_razer_act": "razer_paired_kernel_acts_16384x4096_bf16.md",
-    "c4_mx_act": "mx_quant_absmax_kernel_acts_8192x4096_bf16.md",
+    "c4_channel_scale": "column_stats_kernel_acts_8192x4096_bf16.md",
+    "c4_mx_act": "mx_quant_absmax2_kernel_acts_8192x4096_bf16.md",
     "c4_mx_weight_hessian": "mx_quant_hessian_kernel_weights_4096x4096_bf16.md",
     "c4_hessian_blocks": "hessian_partial_tc_kernel_acts_8192x4096_bf16.md",
+    "c4_mx_weight_flip": "flip_blocks_kernel_weights_4096x4096_bf16.md",
     "c5_act_quant_4o6_mma": "nvfp4_quant_kernel_B16_4o6_bf16_mma_layout_8192x4096.md",
     "c5_w4a4_gemm": "w4a4_gemm_2sm_kernel_M8192_N14336_K4096.md",
-    "c1_nvfp4_pz_deq_mse": "nvfp4_quant_kernel_B16_pz_deq_mse_gaussian_4096x4096.md",
+    "f2_razer_prepare_weights": "razer_prepare_kernel_weights_14336x4096.md",
+    "f2_razer_gemm_w_2pass": "w4a4_gemm_2sm_kernel_razer_2pass_M8192_N14336_K4096.md",
+    "f3_mx_gemm_packed": "w4a4_gemm_2sm_kernel_mxf4_M8192_N16384_K4096.md",
 }
 
 
