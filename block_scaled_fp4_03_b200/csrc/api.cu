@@ -601,7 +601,8 @@ int mxfp4_gemm(const void* a, int a_format, const uint8_t* a_scales, const float
         a_sf = qsf;
     }
     return from_cuda(launch_w4a4_gemm(a_codes, a_sf, nullptr, w_codes, w_scales, nullptr, M, N, K, out,
-                                      out_dtype == FP4Q_F32, err, s, nullptr, nullptr, 1));
+                                      out_dtype == FP4Q_F32, err, s, nullptr, nullptr, 1,
+                                      a_format != FP4Q_MXFP4_PACKED));
 }
 
 }  // extern "C"

@@ -101,7 +101,11 @@ cudaError_t launch_w4a4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const 
                              const uint8_t* w_codes, const uint8_t* w_sf, const float* gw, int64_t M,
                              int64_t N, int64_t K, void* out, int out_f32, int* err, cudaStream_t s,
                              const uint8_t* a1_codes = nullptr, const uint8_t* w1_codes = nullptr,
-                             int mx = 0);
+                             int mx = 0, int after_prologue = 0);
+// after_prologue: the kernel before it on the stream is the operand prologue
+// (a kernel that executes griddepcontrol.launch_dependents); the GEMM is then
+// launched as its programmatic dependent, overlapping its setup with the
+// prologue's tail.
 
 // The tensor-pipe ceiling probe: every SM pair issues iters x 4 back-to-back
 // 256x256x64 block-scaled FP4 MMAs (mx: kind::mxf4) on resident operands;

@@ -302,6 +302,8 @@ w4a4_gemm_1sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
+    // a programmatic dependent of the operand prologue (see the pair kernel)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int num_tiles = p.tiles_m * p.tiles_n;
 
     auto give_up = [&]() {
@@ -644,6 +646,9 @@ w4a4_gemm_2sm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_const
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
+    // launched as a programmatic dependent of the operand prologue: the setup
+    // above overlapped its tail; A and its scales are read only after it is done
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int cluster = blockIdx.x >> 1;
     const int nclusters = gridDim.x >> 1;
     const int num_tiles = p.tiles_m * p.tiles_n;
@@ -1097,10 +1102,32 @@ bool gemm_shape_supported(int64_t M, int64_t N, int64_t K)
            N / kBN < (1 << 20);
 }
 
+// Launch with `pdl` set: the kernel may start while the previous kernel on the
+// stream (the operand prologue, which allows it) is still running, and waits
+// for it at griddepcontrol.wait.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_gemm_kernel(void (*kernel)(KArgs...), int grid, int threads, int smem, cudaStream_t s, bool pdl,
+                               Args&&... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3((unsigned)threads);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = s;
+    if (pdl) {
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 template <bool MX, bool OUTF32>
 cudaError_t launch_gemm_t(const uint8_t* a_codes, const uint8_t* a_sf, const uint8_t* w_codes,
                           const uint8_t* w_sf, const uint8_t* a1, const uint8_t* w1, int64_t M, int64_t N,
-                          int64_t K, void* out, GemmParams& p, cudaStream_t s)
+                          int64_t K, void* out, GemmParams& p, cudaStream_t s, bool pdl)
 {
     if (M % 256 == 0) {
         // CTA pairs: 256 x 256 tiles
@@ -1117,8 +1144,8 @@ cudaError_t launch_gemm_t(const uint8_t* a_codes, const uint8_t* a_sf, const uin
         const int tiles = p.tiles_m * p.tiles_n;
         const int pairs = num_sms() / 2;
         const int grid = 2 * (tiles < pairs ? tiles : pairs);
-        w4a4_gemm_2sm_kernel<MX, OUTF32><<<grid, k2Threads, k2SmemBytes, s>>>(ta, tb, tsa, tsb, to, ta1, tb1, p);
-        return cudaGetLastError();
+        return launch_gemm_kernel(w4a4_gemm_2sm_kernel<MX, OUTF32>, grid, k2Threads, k2SmemBytes, s, pdl, ta, tb, tsa,
+                                  tsb, to, ta1, tb1, p);
     }
     CUtensorMap ta, tb, tsa, tsb, ta1, tb1;
     if (!make_code_map(&ta, a_codes, M, K / 2, kBM) || !make_code_map(&tb, w_codes, N, K / 2, kBN) ||
@@ -1131,8 +1158,8 @@ cudaError_t launch_gemm_t(const uint8_t* a_codes, const uint8_t* a_sf, const uin
     p.tiles_m = (int)(M / kBM);
     const int tiles = p.tiles_m * p.tiles_n;
     const int grid = tiles < num_sms() ? tiles : num_sms();
-    w4a4_gemm_1sm_kernel<MX, OUTF32><<<grid, kThreads, kSmemBytes, s>>>(ta, tb, tsa, tsb, ta1, tb1, p);
-    return cudaGetLastError();
+    return launch_gemm_kernel(w4a4_gemm_1sm_kernel<MX, OUTF32>, grid, kThreads, kSmemBytes, s, pdl, ta, tb, tsa, tsb,
+                              ta1, tb1, p);
 }
 
 int mma_ceiling_pairs() { return num_sms() / 2; }
@@ -1154,7 +1181,7 @@ cudaError_t launch_mma_ceiling(int mx, int iters, int* err, cudaStream_t s)
 cudaError_t launch_w4a4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* ga,
                              const uint8_t* w_codes, const uint8_t* w_sf, const float* gw, int64_t M,
                              int64_t N, int64_t K, void* out, int out_f32, int* err, cudaStream_t s,
-                             const uint8_t* a1_codes, const uint8_t* w1_codes, int mx)
+                             const uint8_t* a1_codes, const uint8_t* w1_codes, int mx, int after_prologue)
 {
     GemmParams p;
     // passes in K-block order: (A, W), then (A, W1), (A1, W), (A1, W1) as present
@@ -1186,11 +1213,12 @@ cudaError_t launch_w4a4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const 
     p.kiters = p.kblocks << p.pass_shift;
     const uint8_t* a1 = a1_codes ? a1_codes : a_codes;
     const uint8_t* w1 = w1_codes ? w1_codes : w_codes;
+    const bool pdl = after_prologue != 0;
     if (mx)
-        return out_f32 ? launch_gemm_t<true, true>(a_codes, a_sf, w_codes, w_sf, a1, w1, M, N, K, out, p, s)
-                       : launch_gemm_t<true, false>(a_codes, a_sf, w_codes, w_sf, a1, w1, M, N, K, out, p, s);
-    return out_f32 ? launch_gemm_t<false, true>(a_codes, a_sf, w_codes, w_sf, a1, w1, M, N, K, out, p, s)
-                   : launch_gemm_t<false, false>(a_codes, a_sf, w_codes, w_sf, a1, w1, M, N, K, out, p, s);
+        return out_f32 ? launch_gemm_t<true, true>(a_codes, a_sf, w_codes, w_sf, a1, w1, M, N, K, out, p, s, pdl)
+                       : launch_gemm_t<true, false>(a_codes, a_sf, w_codes, w_sf, a1, w1, M, N, K, out, p, s, pdl);
+    return out_f32 ? launch_gemm_t<false, true>(a_codes, a_sf, w_codes, w_sf, a1, w1, M, N, K, out, p, s, pdl)
+                   : launch_gemm_t<false, false>(a_codes, a_sf, w_codes, w_sf, a1, w1, M, N, K, out, p, s, pdl);
 }
 
 }  // namespace fp4q

@@ -128,6 +128,10 @@ mx_quant_absmax_kernel(const T* __restrict__ x, uint32_t nblk, uint32_t kb,
                        uint8_t* __restrict__ scales, float* __restrict__ deq,
                        float* __restrict__ mse, int mma)
 {
+    // a GEMM launched after this kernel with programmatic stream serialization
+    // may start its setup now; it waits for this grid's completion (and the
+    // visibility of its writes) before reading A
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     constexpr int CPB = 32 * (int)sizeof(T) / 16;   // 16-byte chunks per block
     // one 4 KB buffer per warp: first the warp's blocks, then their t slices
     __shared__ uint4 buf[kMxWarps][32 * 8];
@@ -257,6 +261,10 @@ mx_quant_absmax2_kernel(const T* __restrict__ x, uint32_t nblk, uint32_t kb,
                         uint8_t* __restrict__ scales, float* __restrict__ deq,
                         float* __restrict__ mse, int mma)
 {
+    // a GEMM launched after this kernel with programmatic stream serialization
+    // may start its setup now; it waits for this grid's completion (and the
+    // visibility of its writes) before reading A
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     constexpr int CPB = 32 * (int)sizeof(T) / 16;   // 16-byte chunks per block
     constexpr int CPL = CPB / 2;                      // chunks per lane (its half)
     constexpr int kStage = kMx2BlocksPerWarp * CPB;   // chunks per warp
