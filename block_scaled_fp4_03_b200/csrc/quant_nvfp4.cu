@@ -275,12 +275,20 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const T* __restrict__ x,
 // ------------------------------------------------------- block evaluation
 // Quantize one block with decoded scale sc and global scale g: packed codes
 // (cw), dequantized values (dq) and the in-order fma squared error.
-template <int B>
-__device__ __forceinline__ float quant_eval(const float (&x)[B], float sc, float g,
-                                            uint32_t (&cw)[(B + 7) / 8], float (&dq)[B])
+// The candidate as t = (S, inv): S = sc * g and inv = min(1/S, FLT_MAX) (0 for
+// S = 0), both rounded to nearest, as quant_eval computes them.
+__device__ __forceinline__ float2 scale_pair(float sc, float g)
 {
     const float S = __fmul_rn(sc, g);
-    const float inv = (S == 0.0f) ? 0.0f : fminf(__frcp_rn(S), kFltMax);
+    return make_float2(S, (S == 0.0f) ? 0.0f : fminf(__frcp_rn(S), kFltMax));
+}
+
+template <int B>
+__device__ __forceinline__ float quant_eval_t(const float (&x)[B], float2 t, uint32_t (&cw)[(B + 7) / 8],
+                                              float (&dq)[B])
+{
+    const float S = t.x;
+    const float inv = t.y;
     float acc = 0.0f;
     if constexpr (B == 4) {
         uint32_t w = e2m1x4_encode(__fmul_rn(x[0], inv), __fmul_rn(x[1], inv),
@@ -316,6 +324,13 @@ __device__ __forceinline__ float quant_eval(const float (&x)[B], float sc, float
         }
     }
     return acc;
+}
+
+template <int B>
+__device__ __forceinline__ float quant_eval(const float (&x)[B], float sc, float g,
+                                            uint32_t (&cw)[(B + 7) / 8], float (&dq)[B])
+{
+    return quant_eval_t<B>(x, scale_pair(sc, g), cw, dq);
 }
 
 // Squared error only (brute-force search); t = (S, inv) of the candidate,
@@ -378,6 +393,13 @@ nvfp4_quant_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs
     const float g = resolve_global_scale<T>(gs);
     const float g6 = __fmul_rn(6.0f, g);
     const float g4 = __fmul_rn(4.0f, g);
+    // (S, inv) of every scale code, computed once per CTA (the encoders return
+    // at most 0xFE for UE5M3 and, for an all-NaN block, 0x7F for E4M3)
+    constexpr int kCodes = SFMT == 1 ? 256 : 128;
+    __shared__ float2 qtab[kCodes];
+    for (int c = threadIdx.x; c < kCodes; c += blockDim.x)
+        qtab[c] = scale_pair(sf_decode<SFMT>((uint32_t)c), g);
+    __syncthreads();
     const int lane = threadIdx.x & 31;
     const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
@@ -452,18 +474,18 @@ nvfp4_quant_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs
             sc = sf_encode<SFMT>(__fdiv_rn(a, g6));
             if (RULE == R_PZ && sc == 0u)
                 sc = 1u;
-            sse = quant_eval<B>(xv, sf_decode<SFMT>(sc), g, cw, dq);
+            sse = quant_eval_t<B>(xv, qtab[sc], cw, dq);
         } else if constexpr (RULE == R_46) {
             const uint32_t c6 = sf_encode<SFMT>(__fdiv_rn(a, g6));
             const uint32_t c4 = sf_encode<SFMT>(__fdiv_rn(a, g4));
-            const float s6 = quant_eval<B>(xv, sf_decode<SFMT>(c6), g, cw, dq);
+            const float s6 = quant_eval_t<B>(xv, qtab[c6], cw, dq);
             sc = c6;
             sse = s6;
             // equal codes give equal errors, and a tie keeps the 6-mapping
             if (c4 != c6) {
                 uint32_t cw4[(B + 7) / 8];
                 float dq4[B];
-                const float s4 = quant_eval<B>(xv, sf_decode<SFMT>(c4), g, cw4, dq4);
+                const float s4 = quant_eval_t<B>(xv, qtab[c4], cw4, dq4);
                 if (s4 < s6) {
                     sc = c4;
                     sse = s4;
