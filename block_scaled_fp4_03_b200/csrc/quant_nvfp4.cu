@@ -1156,7 +1156,7 @@ nvfp4_bf_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs,
         float sse = best;
         float dq[B];
         if (bc != c6 || deq)
-            sse = quant_eval<B>(xv, sf_decode<SFMT>(bc), g, cw, dq);
+            sse = quant_eval_t<B>(xv, tab[bc], cw, dq);
         store_codes<B>(codes + b * (B / 2), cw);
         scales[so] = (uint8_t)bc;
         if (deq)
@@ -1237,10 +1237,13 @@ nvfp4_bf_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs,
                 if (k < nl) {
                     c = (lm & 0xFFu) + (uint32_t)k;
                 } else {
-                    unsigned long long m = upm[w][j];
-                    for (int i = nl; i < k; ++i)
-                        m &= m - 1ull;
-                    c = ((lm >> 16) & 0xFFu) + (uint32_t)__ffsll((long long)m);
+                    // the (k - nl)-th set bit (from 0) of the upper-code mask
+                    const unsigned long long m = upm[w][j];
+                    const uint32_t lo = (uint32_t)m, hi = (uint32_t)(m >> 32);
+                    const int r = k - nl;
+                    const int nlo = __popc(lo);
+                    const uint32_t pos = r < nlo ? __fns(lo, 0u, r + 1) : 32u + __fns(hi, 0u, r - nlo + 1);
+                    c = ((lm >> 16) & 0xFFu) + pos + 1u;
                 }
                 float xj[B];
 #pragma unroll
