@@ -746,6 +746,34 @@ __device__ __forceinline__ uint32_t spread_bits_to_nibbles(uint32_t b)
     return b;
 }
 
+// A block's elements as raw 16-byte words (read-only path) and their fp32
+// values: bf16 is the high half of an fp32 (element 2i in the low half-word).
+template <typename T, int B>
+__device__ __forceinline__ void load_raw(const T* __restrict__ p, uint4 (&w)[B * sizeof(T) / 16])
+{
+#pragma unroll
+    for (int k = 0; k < (int)(B * sizeof(T) / 16); ++k)
+        w[k] = __ldg(reinterpret_cast<const uint4*>(p) + k);
+}
+
+template <typename T, int B>
+__device__ __forceinline__ void raw_to_f32(const uint4 (&w)[B * sizeof(T) / 16], float (&x)[B])
+{
+#pragma unroll
+    for (int k = 0; k < (int)(B * sizeof(T) / 16); ++k) {
+        const uint32_t v[4] = {w[k].x, w[k].y, w[k].z, w[k].w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            if constexpr (sizeof(T) == 4) {
+                x[4 * k + q] = __uint_as_float(v[q]);
+            } else {
+                x[8 * k + 2 * q] = __uint_as_float(v[q] << 16);
+                x[8 * k + 2 * q + 1] = __uint_as_float(v[q] & 0xFFFF0000u);
+            }
+        }
+    }
+}
+
 template <typename T, int SF, int NPAIR>
 __global__ void __launch_bounds__(kThreads, 3)
 razer_paired_kernel(const T* __restrict__ x, int64_t nblk, GsArgs gs, SpecialArgs sp,
@@ -753,6 +781,7 @@ razer_paired_kernel(const T* __restrict__ x, int64_t nblk, GsArgs gs, SpecialArg
                     float* __restrict__ deq, float* __restrict__ mse)
 {
     constexpr int B = 16;
+    static_assert(NPAIR >= 1 && NPAIR <= 2, "the scale table holds two special magnitudes");
     const float g = resolve_global_scale<T>(gs);
     const float g6 = __fmul_rn(6.0f, g);
     const int lane = threadIdx.x & 31;
@@ -762,17 +791,39 @@ razer_paired_kernel(const T* __restrict__ x, int64_t nblk, GsArgs gs, SpecialArg
 #pragma unroll
     for (int m = 0; m < NPAIR; ++m)
         mag[m] = sp.v[2 * m];
+    // per scale code, computed once per CTA: S = sc * g, inv = min(1/S, FLT_MAX)
+    // (0 for S = 0) and each special magnitude times S (E3M3 encodes to 0..63,
+    // E4M3 to 0..127)
+    constexpr int kCodes = SF == 1 ? 64 : 128;
+    __shared__ float4 rtab[kCodes];
+    for (int c = threadIdx.x; c < kCodes; c += blockDim.x) {
+        const float S = __fmul_rn(SF == 1 ? e3m3_decode((uint32_t)c) : e4m3_decode((uint32_t)c), g);
+        const float inv = (S == 0.0f) ? 0.0f : fminf(__frcp_rn(S), kFltMax);
+        rtab[c] = make_float4(S, inv, __fmul_rn(mag[0], S), NPAIR > 1 ? __fmul_rn(mag[NPAIR - 1], S) : 0.0f);
+    }
+    __syncthreads();
+
+    // the next block's raw words are in flight while this one is quantized
+    constexpr int kWords = B * (int)sizeof(T) / 16;
+    uint4 wn[kWords];
+#pragma unroll
+    for (int k = 0; k < kWords; ++k)
+        wn[k] = make_uint4(0u, 0u, 0u, 0u);
+    if (warp0 * 32 + lane < nblk)
+        load_raw<T, B>(x + (warp0 * 32 + lane) * B, wn);
 
     for (int64_t base = warp0 * 32; base < nblk; base += nwarps * 32) {
         const int64_t b = base + lane;
         const bool valid = b < nblk;
         float xv[B];
-        if (valid) {
-            load_elems<T, B>(x + b * B, xv);
-        } else {
+        raw_to_f32<T, B>(wn, xv);
+        {
+            const int64_t bn = b + nwarps * 32;
 #pragma unroll
-            for (int i = 0; i < B; ++i)
-                xv[i] = 0.0f;
+            for (int k = 0; k < kWords; ++k)
+                wn[k] = make_uint4(0u, 0u, 0u, 0u);
+            if (bn < nblk)
+                load_raw<T, B>(x + bn * B, wn);
         }
         float a = 0.0f;
 #pragma unroll
@@ -780,13 +831,13 @@ razer_paired_kernel(const T* __restrict__ x, int64_t nblk, GsArgs gs, SpecialArg
             a = fmaxf(a, fabsf(xv[i]));
         const float r = __fdiv_rn(a, g6);
         const uint32_t scc = SF == 1 ? e3m3_encode(r) : e4m3_encode(r);
-        const float scv = SF == 1 ? e3m3_decode(scc) : e4m3_decode(scc);
-        const float S = __fmul_rn(scv, g);
-        const float inv = (S == 0.0f) ? 0.0f : fminf(__frcp_rn(S), kFltMax);
+        const float4 st = rtab[scc];
+        const float S = st.x;
+        const float inv = st.y;
         float D[NPAIR];
-#pragma unroll
-        for (int m = 0; m < NPAIR; ++m)
-            D[m] = __fmul_rn(mag[m], S);
+        D[0] = st.z;
+        if constexpr (NPAIR > 1)
+            D[NPAIR - 1] = st.w;
 
         float acc[2 * NPAIR];
         uint32_t mask[2 * NPAIR];
