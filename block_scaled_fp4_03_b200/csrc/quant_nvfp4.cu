@@ -371,6 +371,45 @@ __device__ __forceinline__ float quant_sse(const float (&x)[B], float, float, fl
     return acc;
 }
 
+// Codes and in-order squared error of a block at the candidate t = (S, inv).
+template <int B>
+__device__ __forceinline__ float quant_codes_sse(const float (&x)[B], float2 t, uint32_t (&cw)[(B + 7) / 8])
+{
+    const float S = t.x;
+    const float inv = t.y;
+    float acc = 0.0f;
+    if constexpr (B == 4) {
+        const uint32_t w = e2m1x4_encode(__fmul_rn(x[0], inv), __fmul_rn(x[1], inv),
+                                         __fmul_rn(x[2], inv), __fmul_rn(x[3], inv));
+        float v[4];
+        e2m1x4_decode(w, v);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float e = __fsub_rn(x[i], __fmul_rn(v[i], S));
+            acc = __fmaf_rn(e, e, acc);
+        }
+        cw[0] = w;
+    } else {
+#pragma unroll
+        for (int j = 0; j < B / 8; ++j) {
+            const int o = 8 * j;
+            const uint32_t w = e2m1x8_encode(__fmul_rn(x[o], inv), __fmul_rn(x[o + 1], inv),
+                                             __fmul_rn(x[o + 2], inv), __fmul_rn(x[o + 3], inv),
+                                             __fmul_rn(x[o + 4], inv), __fmul_rn(x[o + 5], inv),
+                                             __fmul_rn(x[o + 6], inv), __fmul_rn(x[o + 7], inv));
+            float v[8];
+            e2m1x8_decode(w, v);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float e = __fsub_rn(x[o + i], __fmul_rn(v[i], S));
+                acc = __fmaf_rn(e, e, acc);
+            }
+            cw[j] = w;
+        }
+    }
+    return acc;
+}
+
 // Error of one element of magnitude a under scale S / reciprocal inv.
 __device__ __forceinline__ float elem_err(float a, float S, float inv)
 {
@@ -384,7 +423,7 @@ enum { R_ABSMAX = 0, R_PZ = 1, R_46 = 2, R_BF = 3 };
 
 // Abs-max, prevent-zero and 4-over-6 (brute force has its own kernel below).
 // SFMT: the block-scale format, 0 = E4M3 (NVFP4), 1 = UE5M3.
-template <int B, typename T, int RULE, int SFMT>
+template <int B, typename T, int RULE, int SFMT, bool DEQ>
 __global__ void __launch_bounds__(kThreads)
 nvfp4_quant_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs,
                    uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, int mma_layout,
@@ -478,24 +517,25 @@ nvfp4_quant_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs
         } else if constexpr (RULE == R_46) {
             const uint32_t c6 = sf_encode<SFMT>(__fdiv_rn(a, g6));
             const uint32_t c4 = sf_encode<SFMT>(__fdiv_rn(a, g4));
-            const float s6 = quant_eval_t<B>(xv, qtab[c6], cw, dq);
+            // codes and errors of both candidates; the dequantized values only
+            // for the chosen one, and only when they are wanted
+            sse = quant_codes_sse<B>(xv, qtab[c6], cw);
             sc = c6;
-            sse = s6;
             // equal codes give equal errors, and a tie keeps the 6-mapping
             if (c4 != c6) {
                 uint32_t cw4[(B + 7) / 8];
-                float dq4[B];
-                const float s4 = quant_eval_t<B>(xv, qtab[c4], cw4, dq4);
-                if (s4 < s6) {
+                const float s4 = quant_codes_sse<B>(xv, qtab[c4], cw4);
+                if (s4 < sse) {
                     sc = c4;
                     sse = s4;
 #pragma unroll
                     for (int j = 0; j < (B + 7) / 8; ++j)
                         cw[j] = cw4[j];
-#pragma unroll
-                    for (int i = 0; i < B; ++i)
-                        dq[i] = dq4[i];
                 }
+            }
+            if constexpr (DEQ) {
+                uint32_t cwd[(B + 7) / 8];
+                quant_eval_t<B>(xv, qtab[sc], cwd, dq);
             }
         }
 
@@ -503,13 +543,13 @@ nvfp4_quant_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs
             store_codes<B>(codes + b * (B / 2), cw);
             const int64_t so = mma_layout ? mma_sf_offset(r_cur, kb_cur, kb_atoms) : b;
             scales[so] = (uint8_t)sc;
-            if (!kStoreStaged && deq)
+            if (!kStoreStaged && DEQ)
                 store_f32<B>(deq + b * B, dq);
             if (mse)
                 mse[b] = __fmul_rn(sse, 1.0f / (float)B);
         }
         if constexpr (kStoreStaged) {
-            if (deq)
+            if constexpr (DEQ)
                 warp_store_f32_blocks<B>(deq, base, nblk, stage_buf[threadIdx.x >> 5], dq);
         }
         if (mma_layout) {
@@ -967,45 +1007,6 @@ razer_paired_kernel(const T* __restrict__ x, int64_t nblk, GsArgs gs, SpecialArg
 // lowered with a shared-memory atomic minimum, so the lowest code wins ties
 // exactly as in a sequential scan.
 constexpr int kWarps = kThreads / 32;
-
-// Codes and in-order squared error of a block at the candidate t = (S, inv).
-template <int B>
-__device__ __forceinline__ float quant_codes_sse(const float (&x)[B], float2 t, uint32_t (&cw)[(B + 7) / 8])
-{
-    const float S = t.x;
-    const float inv = t.y;
-    float acc = 0.0f;
-    if constexpr (B == 4) {
-        const uint32_t w = e2m1x4_encode(__fmul_rn(x[0], inv), __fmul_rn(x[1], inv),
-                                         __fmul_rn(x[2], inv), __fmul_rn(x[3], inv));
-        float v[4];
-        e2m1x4_decode(w, v);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const float e = __fsub_rn(x[i], __fmul_rn(v[i], S));
-            acc = __fmaf_rn(e, e, acc);
-        }
-        cw[0] = w;
-    } else {
-#pragma unroll
-        for (int j = 0; j < B / 8; ++j) {
-            const int o = 8 * j;
-            const uint32_t w = e2m1x8_encode(__fmul_rn(x[o], inv), __fmul_rn(x[o + 1], inv),
-                                             __fmul_rn(x[o + 2], inv), __fmul_rn(x[o + 3], inv),
-                                             __fmul_rn(x[o + 4], inv), __fmul_rn(x[o + 5], inv),
-                                             __fmul_rn(x[o + 6], inv), __fmul_rn(x[o + 7], inv));
-            float v[8];
-            e2m1x8_decode(w, v);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float e = __fsub_rn(x[o + i], __fmul_rn(v[i], S));
-                acc = __fmaf_rn(e, e, acc);
-            }
-            cw[j] = w;
-        }
-    }
-    return acc;
-}
 
 // True when a fp32 value is a normal power of two in [2^-100, 2^100].
 __device__ __forceinline__ bool pow2_in_range(float v)
@@ -1635,8 +1636,13 @@ cudaError_t nvfp4_launch_t(const void* x, int64_t rows, int64_t cols, const GsAr
                                         kWarps * 32 * B * (int)sizeof(float), reinterpret_cast<const T*>(x), nblk,
                                         cols / B, gs, codes, scales, mma, deq, mse, evals, bf_windows());
     } else {
-        return launch_quant_kernel(nvfp4_quant_kernel<B, T, RULE, SFMT>, nblk, gs, s, reinterpret_cast<const T*>(x),
-                                   nblk, cols / B, gs, codes, scales, mma, deq, mse);
+        // dequantized values are a compile-time option: without them the
+        // candidates' values need not stay live
+        if (deq)
+            return launch_quant_kernel(nvfp4_quant_kernel<B, T, RULE, SFMT, true>, nblk, gs, s,
+                                       reinterpret_cast<const T*>(x), nblk, cols / B, gs, codes, scales, mma, deq, mse);
+        return launch_quant_kernel(nvfp4_quant_kernel<B, T, RULE, SFMT, false>, nblk, gs, s,
+                                   reinterpret_cast<const T*>(x), nblk, cols / B, gs, codes, scales, mma, deq, mse);
     }
 }
 
