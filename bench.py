@@ -149,7 +149,7 @@ def build_rows(torch, fq, inputs, dev, host_copies=None, groups=None):
         def c1():
             o1.update(fq.nvfp4_quantize(X["c1"], 16, fq.PREVENT_ZERO, gs_mode=fq.GS_AMAX, dequant=True,
                                         mse=True, out=o1, workspace=ws1))
-        rows.append(Row("c1_nvfp4_pz_deq_mse", "nvfp4_quant_kernel<16, float, 1, 0>", n1, n1 * (4 + 0.5 + 1 / 16 + 4 + 4 / 16), 2, c1, o1))
+        rows.append(Row("c1_nvfp4_pz_deq_mse", "nvfp4_quant_kernel<16, float, 1, 0, true>", n1, n1 * (4 + 0.5 + 1 / 16 + 4 + 4 / 16), 2, c1, o1))
         # the standalone dequantizer (fp4_dequant_mse) on that output: codes,
         # scales and g in, the reference x in for the MSE, dequant and MSE out
         od1 = {"dequant": torch.empty(a1.shape, dtype=torch.float32, device=dev),
@@ -176,7 +176,7 @@ def build_rows(torch, fq, inputs, dev, host_copies=None, groups=None):
 
                 def c2(B=B, rule=rule, o=o, wsr=wsr):
                     o.update(fq.nvfp4_quantize(X["c2"], B, rule, gs_mode=fq.GS_NONE, mse=True, out=o, workspace=wsr))
-                kern = ("nvfp4_bf_kernel<%d, float, 0>" % B) if bf else ("nvfp4_quant_kernel<%d, float, %d, 0>" % (B, rule))
+                kern = ("nvfp4_bf_kernel<%d, float, 0>" % B) if bf else ("nvfp4_quant_kernel<%d, float, %d, 0, false>" % (B, rule))
                 # brute force is held to the HBM roofline like the other rules (the
                 # evaluations it performs are reported beside it, not as its bound)
                 rows.append(Row("c2_B%d_%s" % (B, names[rule]), kern,
@@ -195,7 +195,7 @@ def build_rows(torch, fq, inputs, dev, host_copies=None, groups=None):
                     o.update(fq.nvfp4_quantize(X["c2"], B, rule, gs_mode=gsm, mse=True, out=o, scale_fmt=sfmt,
                                                workspace=wsh2 if gsm == fq.GS_AMAX else None))
                 rows.append(Row("c2_B%d_%s" % (B, tag),
-                                "nvfp4_quant_kernel<%d, float, %d, %d>" % (B, rule, 1 if sfmt == fq.SF_UE5M3 else 0),
+                                "nvfp4_quant_kernel<%d, float, %d, %d, false>" % (B, rule, 1 if sfmt == fq.SF_UE5M3 else 0),
                                 n2, n2 * (4 + 0.5 + 1 / B + 4 / B), 2 if gsm == fq.GS_AMAX else 1, c2x, o, extra=True))
     set_inputs(n0, [k for k in ("c2",) if k in X])
     n0 = len(rows)
@@ -315,7 +315,7 @@ def build_rows(torch, fq, inputs, dev, host_copies=None, groups=None):
         def c5g():
             fq.w4a4_gemm(o5["codes"], qw5["codes"], qw5["scales"], qw5["global_scale"], a_scales=o5["scales"],
                          a_global_scale=o5["global_scale"], K=K5, out=y5, workspace=wsg)
-        rows.append(Row("c5_act_quant_4o6_mma", "nvfp4_quant_kernel<16, __nv_bfloat16, 2, 0>", a5.size, a5.size * (2 + 0.5 + 1 / 16), 2, c5, o5))
+        rows.append(Row("c5_act_quant_4o6_mma", "nvfp4_quant_kernel<16, __nv_bfloat16, 2, 0, false>", a5.size, a5.size * (2 + 0.5 + 1 / 16), 2, c5, o5))
         rows.append(Row("c5_w4a4_gemm", "w4a4_gemm_2sm_kernel<false>", 0, M5 * K5 * (0.5 + 1 / 16) + N5 * K5 * (0.5 + 1 / 16) + M5 * N5 * 2,
                         1, c5g, {"out": y5}, bound="tensor", flops=2.0 * M5 * N5 * K5))
 

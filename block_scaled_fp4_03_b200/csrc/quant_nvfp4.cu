@@ -1140,9 +1140,9 @@ constexpr int kBfQueue = 64;
 
 // Resident CTAs per SM the brute-force kernel is compiled for (its register cap).
 template <int B>
-constexpr int bf_min_ctas() { return B <= 4 ? 4 : B <= 8 ? 3 : 2; }
+constexpr int bf_min_ctas() { return B <= 4 ? 4 : B <= 16 ? 3 : 2; }
 
-template <int B, typename T, int SFMT>
+template <int B, typename T, int SFMT, bool DEQ>
 __global__ void __launch_bounds__(kThreads, bf_min_ctas<B>())
 nvfp4_bf_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs,
                 uint8_t* __restrict__ codes, uint8_t* __restrict__ scales, int mma_layout,
@@ -1207,11 +1207,11 @@ nvfp4_bf_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs,
                            float best, int64_t so) {
         float sse = best;
         float dq[B];
-        if (bc != c6 || deq)
+        if (bc != c6 || DEQ)
             sse = quant_eval_t<B>(xv, tab[bc], cw, dq);
         store_codes<B>(codes + b * (B / 2), cw);
         scales[so] = (uint8_t)bc;
-        if (deq)
+        if constexpr (DEQ)
             store_f32<B>(deq + b * B, dq);
         if (mse)
             mse[b] = __fmul_rn(sse, 1.0f / (float)B);
@@ -1632,9 +1632,14 @@ cudaError_t nvfp4_launch_t(const void* x, int64_t rows, int64_t cols, const GsAr
 {
     const int64_t nblk = rows * (cols / B);
     if constexpr (RULE == R_BF) {
-        return launch_quant_kernel_smem(nvfp4_bf_kernel<B, T, SFMT>, nblk, gs, s,
-                                        kWarps * 32 * B * (int)sizeof(float), reinterpret_cast<const T*>(x), nblk,
-                                        cols / B, gs, codes, scales, mma, deq, mse, evals, bf_windows());
+        const int dyn = kWarps * 32 * B * (int)sizeof(float);
+        if (deq)
+            return launch_quant_kernel_smem(nvfp4_bf_kernel<B, T, SFMT, true>, nblk, gs, s, dyn,
+                                            reinterpret_cast<const T*>(x), nblk, cols / B, gs, codes, scales, mma, deq,
+                                            mse, evals, bf_windows());
+        return launch_quant_kernel_smem(nvfp4_bf_kernel<B, T, SFMT, false>, nblk, gs, s, dyn,
+                                        reinterpret_cast<const T*>(x), nblk, cols / B, gs, codes, scales, mma, deq, mse,
+                                        evals, bf_windows());
     } else {
         // dequantized values are a compile-time option: without them the
         // candidates' values need not stay live
