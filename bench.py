@@ -176,7 +176,7 @@ def build_rows(torch, fq, inputs, dev, host_copies=None, groups=None):
 
                 def c2(B=B, rule=rule, o=o, wsr=wsr):
                     o.update(fq.nvfp4_quantize(X["c2"], B, rule, gs_mode=fq.GS_NONE, mse=True, out=o, workspace=wsr))
-                kern = ("nvfp4_bf_kernel<%d, float, 0>" % B) if bf else ("nvfp4_quant_kernel<%d, float, %d, 0, false>" % (B, rule))
+                kern = ("nvfp4_bf_kernel<%d, float, 0, false>" % B) if bf else ("nvfp4_quant_kernel<%d, float, %d, 0, false>" % (B, rule))
                 # brute force is held to the HBM roofline like the other rules (the
                 # evaluations it performs are reported beside it, not as its bound)
                 rows.append(Row("c2_B%d_%s" % (B, names[rule]), kern,
