@@ -433,7 +433,10 @@ FP4Q_API int fp4_scales_to_mma(const uint8_t* scales, int64_t rows, int64_t nsca
  *  a, a_format  FP4Q_F32 / FP4Q_BF16: A is a dense M x K tensor; the prologue
  *               (a * chan_scale, the 32-block rotation if hadamard32, OCP E8M0
  *               exponent, E2M1 codes) runs here into the workspace, scales
- *               written in the GEMM's layout; FP4Q_MXFP4_PACKED: a = codes
+ *               written in the GEMM's layout, and the GEMM kernel is launched
+ *               on the same stream as its programmatic dependent (its setup
+ *               overlaps the prologue's tail; it reads A only after the
+ *               prologue completed); FP4Q_MXFP4_PACKED: a = codes
  *               (M*K/2 bytes), a_scales = E8M0 bytes in FP4Q_SFLAYOUT_MMA
  *               (chan_scale must be NULL)
  *  chan_scale   device fp32 [K] (nullable): t for the dense A
