@@ -44,6 +44,7 @@ SIGNATURES = {
     "fp4q_gemm_status": (_i, [_vp, _vp]),
     "fp4q_hessian_status": (_i, [_vp, _vp]),
     "fp4q_debug_set_wait_cycles": (_i64, [_i64]),
+    "fp4q_debug_force_amax_pass": (_i, [_i]),
     "fp4q_mma_ceiling": (_i, [_i, _i, _vp, _vp]),
     "fp4q_mma_ceiling_flops": (ctypes.c_double, [_i]),
     "razer_gemm_prepare": (_i, [_vp, _vp, _i64, _i64, _i, _vp, _i, _vp, _vp, _vp, _vp]),
@@ -404,6 +405,12 @@ def debug_set_wait_cycles(cycles: int) -> int:
     """Process-wide limit of the tensor-core kernels' bounded waits (0: the default);
     returns the previous setting.  For tests of the timeout path."""
     return int(lib().fp4q_debug_set_wait_cycles(int(cycles)))
+
+
+def debug_force_amax_pass(on: bool) -> int:
+    """Process-wide: hierarchical global scales through the separate amax pass (the
+    non-cooperative fallback) instead of the fused one; returns the previous setting."""
+    return int(lib().fp4q_debug_force_amax_pass(int(bool(on))))
 
 
 def mma_ceiling(mx: bool, iters: int, err: torch.Tensor, stream=None) -> float:

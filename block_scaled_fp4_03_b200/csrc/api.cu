@@ -65,14 +65,16 @@ cudaError_t fused_gs(GsArgs& gs, const void* x, int64_t n, uint8_t* ws, size_t f
 
 // Run a quantizer launch; if its fused amax cannot be launched cooperatively
 // here (the device holds fewer resident CTAs than its grid, e.g. when shared
-// under MPS), fall back to a separate amax pass whose partials go to
-// ws[0, 4 * kAmaxPartials).
+// under MPS), or fp4q_debug_force_amax_pass asks for it, fall back to a
+// separate amax pass whose partials go to ws[0, 4 * kAmaxPartials).
 template <typename F>
 cudaError_t launch_with_gs(GsArgs& gs, const void* x, int dtype, int64_t n, void* ws, cudaStream_t s, F&& launch)
 {
-    cudaError_t e = launch(gs);
+    const bool forced = gs.mode == 3 && force_amax_pass();
+    cudaError_t e = forced ? cudaErrorCooperativeLaunchTooLarge : launch(gs);
     if (e == cudaErrorCooperativeLaunchTooLarge && gs.mode == 3) {
-        (void)cudaGetLastError();
+        if (!forced)
+            (void)cudaGetLastError();
         gs.mode = 1;
         gs.partials = reinterpret_cast<const float*>(ws);
         gs.n_partials = kAmaxPartials;

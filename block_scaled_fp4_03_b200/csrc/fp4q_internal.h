@@ -15,6 +15,8 @@ constexpr long long kDefaultWaitCycles = 4000000000LL;
 // The limit the next launch gives its main-loop waits: the process-wide
 // setting of fp4q_debug_set_wait_cycles, or kDefaultWaitCycles.
 long long wait_limit_cycles();
+// fp4q_debug_force_amax_pass: take the separate amax pass instead of the fused one
+bool force_amax_pass();
 
 // Global-scale source for a quantizer launch.
 struct GsArgs {

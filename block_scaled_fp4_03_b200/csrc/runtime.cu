@@ -20,8 +20,11 @@ std::atomic<int> g_sms[kMaxDevices];
 std::mutex g_opt_mu;
 std::set<std::pair<const void*, int>> g_opted;   // (kernel, device) pairs already opted in
 std::atomic<long long> g_wait_cycles{0};         // 0: kDefaultWaitCycles
+std::atomic<int> g_force_amax_pass{0};
 
 }  // namespace
+
+bool force_amax_pass() { return g_force_amax_pass.load(std::memory_order_relaxed) != 0; }
 
 long long wait_limit_cycles()
 {
@@ -63,4 +66,9 @@ cudaError_t smem_opt_in(const void* kernel, int bytes)
 extern "C" int64_t fp4q_debug_set_wait_cycles(int64_t cycles)
 {
     return fp4q::g_wait_cycles.exchange(cycles > 0 ? cycles : 0, std::memory_order_relaxed);
+}
+
+extern "C" int fp4q_debug_force_amax_pass(int on)
+{
+    return fp4q::g_force_amax_pass.exchange(on != 0 ? 1 : 0, std::memory_order_relaxed);
 }

@@ -31,7 +31,8 @@
  *    layout is requested.
  *  - "device" pointers are CUDA device memory owned by the caller; the library
  *    allocates and frees nothing and keeps no state between calls (apart from
- *    the debug wait limit of fp4q_debug_set_wait_cycles and the fixed scratch
+ *    the debug settings of fp4q_debug_set_wait_cycles and
+ *    fp4q_debug_force_amax_pass, and the fixed scratch
  *    of fp4_hessian_blocks_noalloc).  "host" pointers are read during the call
  *    only.
  *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
@@ -490,6 +491,16 @@ FP4Q_API double fp4q_mma_ceiling_flops(int iters);
  * entry point reports FP4Q_ERR_TIMEOUT.  Returns the previous setting.
  */
 FP4Q_API int64_t fp4q_debug_set_wait_cycles(int64_t cycles);
+
+/*
+ * Debug: with on != 0, every later call that computes a hierarchical global
+ * scale (FP4Q_GS_AMAX) takes the path used when the device cannot make the
+ * quantizer's launch cooperative: a separate amax pass over x writes partial
+ * maxima into the workspace, and the quantizer reduces them (the same exact
+ * maximum, so the same results).  Process-wide, for tests of that path.
+ * Returns the previous setting.
+ */
+FP4Q_API int fp4q_debug_force_amax_pass(int on);
 
 #ifdef __cplusplus
 }

@@ -207,3 +207,14 @@ def test_debug_wait_limit_setter_round_trips(L):
         assert L.fp4q_debug_set_wait_cycles(0) == 0          # a negative value stored as the default
     finally:
         L.fp4q_debug_set_wait_cycles(prev)
+
+
+def test_debug_force_amax_pass_setter_round_trips(L):
+    """The forced-amax-pass knob is host state only: any nonzero value reads back as 1."""
+    prev = L.fp4q_debug_force_amax_pass(1)
+    try:
+        assert L.fp4q_debug_force_amax_pass(7) == 1
+        assert L.fp4q_debug_force_amax_pass(0) == 1
+        assert L.fp4q_debug_force_amax_pass(0) == 0
+    finally:
+        L.fp4q_debug_force_amax_pass(prev)

@@ -140,3 +140,58 @@ def test_fused_amax_barrier_fallback_keeps_results(O, kind, rule, B):
         assert_bits(r["scales"], ref["scales"], "scales")
         assert_bits(r["mse"], ref["mse"], "mse")
 
+
+
+class separate_amax_pass:
+    """Context manager: hierarchical global scales through the separate amax pass."""
+
+    def __enter__(self):
+        self.prev = fq.debug_force_amax_pass(True)
+
+    def __exit__(self, *exc):
+        fq.debug_force_amax_pass(self.prev)
+
+
+@pytest.mark.parametrize("kind,rule,B", [("gaussian", fq.PREVENT_ZERO, 16), ("student_t", fq.FOUR_OVER_SIX, 4),
+                                         ("student_t", fq.BRUTE_FORCE, 32)])
+def test_separate_amax_pass_matches_fused(O, kind, rule, B):
+    """The path taken when the quantizer cannot be launched cooperatively: a
+    separate amax pass (amax_kernel) writes partial maxima, the quantizer
+    reduces them.  g, codes, scales and errors equal the fused path's and the
+    oracle's."""
+    from test_gpu_parity import make, assert_bits
+    x, x32 = make(kind, 777, 512, seed=11, dtype="f32")
+    g = np.array([O.global_scale(O.amax(x32))], np.float32)
+    ref = O.nvfp4_quantize(x32, B, rule, g=g[0])
+    fused = fq.nvfp4_quantize(x, B, rule, gs_mode=fq.GS_AMAX, mse=True)
+    with separate_amax_pass():
+        alone = fq.nvfp4_quantize(x, B, rule, gs_mode=fq.GS_AMAX, mse=True)
+        torch.cuda.synchronize()
+    for r in (fused, alone):
+        assert_bits(r["global_scale"], g, "g")
+        assert_bits(r["codes"], ref["codes"], "codes")
+        assert_bits(r["scales"], ref["scales"], "scales")
+        assert_bits(r["mse"], ref["mse"], "mse")
+
+
+def test_separate_amax_pass_razer_and_gemm_activations(O):
+    """The same fallback for a RaZeR quantizer and for the W4A4 GEMM's dense
+    activations: results equal the fused path's bit for bit."""
+    from test_gpu_parity import make
+    x, _ = make("razer_act", 512, 256, seed=12, dtype="bf16")
+    fused = fq.razer_quantize(x, fq.SF_E4M3, [5.0, -5.0], gs_mode=fq.GS_AMAX, mse=True)
+    with separate_amax_pass():
+        alone = fq.razer_quantize(x, fq.SF_E4M3, [5.0, -5.0], gs_mode=fq.GS_AMAX, mse=True)
+        torch.cuda.synchronize()
+    for k in ("codes", "meta", "mse", "global_scale"):
+        assert torch.equal(fused[k].view(torch.uint8), alone[k].view(torch.uint8)), k
+    M, N, K = 256, 512, 1024
+    a = torch.from_numpy(inputs.generate("gemm_act", M, K, seed=13).view(np.int16)).cuda().view(torch.bfloat16)
+    w32 = inputs.as_f32(inputs.generate("gemm_weight", N, K, seed=14))
+    qw, gw = quantized_operand(O, w32, O.RULE_ABSMAX)
+    wargs = (dev(qw["codes"]), dev(to_mma_layout(qw["scales"])), dev(np.array([gw], np.float32)))
+    y0 = fq.w4a4_gemm(a, *wargs)
+    with separate_amax_pass():
+        y1 = fq.w4a4_gemm(a, *wargs)
+        torch.cuda.synchronize()
+    assert torch.equal(y0.view(torch.int16), y1.view(torch.int16))
