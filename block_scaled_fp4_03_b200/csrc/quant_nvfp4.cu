@@ -452,9 +452,9 @@ nvfp4_quant_kernel(const T* __restrict__ x, int64_t nblk, int64_t bpr, GsArgs gs
                                    ? (kStaged ? 2 * B * (int)sizeof(T) : 1)
                                    : (kStoreStaged ? 8 * B : 1);
     __shared__ uint4 stage_buf[kThreads / 32][kBufChunks];
-    // small blocks (one or two 16-byte loads per lane): keep the next block's
+    // small blocks (up to four 16-byte loads per lane): keep the next block's
     // load in flight while this one is quantized
-    constexpr bool kPrefetch = !kStaged && B * sizeof(T) <= 32;
+    constexpr bool kPrefetch = !kStaged && B * sizeof(T) <= 64;
     float xn[B];
     if constexpr (kPrefetch) {
         const int64_t b0 = warp0 * 32 + lane;
