@@ -73,7 +73,7 @@ PROFILE_OF_ROW = {
     "c2_B16_absmax": "nvfp4_quant_kernel_B16_absmax_student_t_8192x8192.md",
     "c3_razer_weight": "razer_paired_kernel_weights_8192x8192_bf16.md",
     "c3_razer_act": "razer_paired_kernel_acts_16384x4096_bf16.md",
-    "c4_channel_scale": "column_stats_kernel_acts_8192x4096_bf16.md",
+    "c4_channel_scale": "column_stats_kernel_weights_4096x4096_acts_8192x4096_bf16.md",
     "c4_mx_act": "mx_quant_absmax2_kernel_acts_8192x4096_bf16.md",
     "c4_mx_weight_hessian": "mx_quant_hessian_kernel_weights_4096x4096_bf16.md",
     "c4_hessian_blocks": "hessian_partial_tc_kernel_acts_8192x4096_bf16.md",
@@ -244,7 +244,7 @@ def build_rows(torch, fq, inputs, dev, host_copies=None, groups=None):
 
         def c4w():
             o4w.update(fq.mxfp4_quantize(X["c4w"], ti4, True, fq.HESSIAN_EXP, hess=h4, out=o4w))
-        rows.append(Row("c4_channel_scale", "column_stats_kernel", 0, x4.size * 2 + w4.size * 2, 3, c4s, {"t": t4, "t_inv": ti4}))
+        rows.append(Row("c4_channel_scale", "column_stats_kernel", 0, x4.size * 2 + w4.size * 2, 2, c4s, {"t": t4, "t_inv": ti4}))
         rows.append(Row("c4_hessian_blocks", "hessian_partial_kernel", 0, x4.size * 2 + C * 32 * 4, 2, c4h,
                         {"hess": h4}, flops=2.0 * T * C * 32))
         rows.append(Row("c4_mx_act", "mx_quant_absmax_kernel", x4.size, x4.size * (2 + 0.5 + 1 / 32), 1, c4a, o4a))

@@ -551,7 +551,7 @@ hessian_reduce_kernel(const float* __restrict__ part, int64_t nchunk, int64_t to
 
 // ------------------------------------------------------- channel scale
 // Column statistics in fp64 over a chunk of kStatRows rows: sum and sum of
-// squares.  A CTA covers 256 columns: lane l of every warp owns the 8
+// squares.  A tile is one chunk x 256 columns: lane l of every warp owns the 8
 // consecutive columns 8 l .. 8 l + 7 of the tile (one 16-byte bf16 vector or
 // two fp32 vectors per row), and warp w takes rows w, w + 8, w + 16, ... of the
 // chunk, 8 rows per batch with all 8 loads issued before the sums.  The 8
@@ -561,16 +561,16 @@ constexpr int kStatCols = 256;
 constexpr int kStatWarps = kThreads / 32;
 
 template <typename T>
-__global__ void __launch_bounds__(kThreads)
-column_stats_kernel(const T* __restrict__ x, int64_t rows, int64_t cols, double* __restrict__ sum,
-                    double* __restrict__ sumsq)
+__device__ __forceinline__ void column_stats_tile(const T* __restrict__ x, int64_t rows, int64_t cols,
+                                                  double* __restrict__ sum, double* __restrict__ sumsq,
+                                                  int64_t tx, int64_t ty,
+                                                  double (&red)[2][kStatWarps][kStatCols])
 {
-    __shared__ double red[2][kStatWarps][kStatCols];
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
-    const int64_t c0 = (int64_t)blockIdx.x * kStatCols + 8 * lane;
+    const int64_t c0 = tx * kStatCols + 8 * lane;
     const bool own = c0 < cols;
-    const int64_t r0 = (int64_t)blockIdx.y * kStatRows;
+    const int64_t r0 = ty * kStatRows;
     const int64_t r1 = (r0 + kStatRows) < rows ? (r0 + kStatRows) : rows;
     double s[8], q[8];
 #pragma unroll
@@ -613,7 +613,7 @@ column_stats_kernel(const T* __restrict__ x, int64_t rows, int64_t cols, double*
     }
     __syncthreads();
     // thread t finishes column t of the tile
-    const int64_t c = (int64_t)blockIdx.x * kStatCols + threadIdx.x;
+    const int64_t c = tx * kStatCols + threadIdx.x;
     if (c < cols) {
         double ts = red[0][0][threadIdx.x], tq = red[1][0][threadIdx.x];
 #pragma unroll
@@ -621,10 +621,35 @@ column_stats_kernel(const T* __restrict__ x, int64_t rows, int64_t cols, double*
             ts += red[0][w][threadIdx.x];
             tq += red[1][w][threadIdx.x];
         }
-        const int64_t o = (int64_t)blockIdx.y * cols + c;
+        const int64_t o = ty * cols + c;
         if (sum)
             sum[o] = ts;
         sumsq[o] = tq;
+    }
+}
+
+// Both tensors' statistics in one persistent launch: the weight tiles (sum and
+// sum of squares, wch row chunks) come first, then the activation tiles (sum of
+// squares, xch row chunks), and CTA b takes tiles b, b + gridDim.x, ...  A
+// tile's partial sums do not depend on which CTA computes it or when.
+template <typename TW, typename TX>
+__global__ void __launch_bounds__(kThreads)
+column_stats_kernel(const TW* __restrict__ w, int64_t n_out, double* __restrict__ wsum,
+                    double* __restrict__ wsq, int64_t wch, const TX* __restrict__ x, int64_t tokens,
+                    double* __restrict__ xsq, int64_t xch, int64_t cols)
+{
+    __shared__ double red[2][kStatWarps][kStatCols];
+    const int64_t gx = (cols + kStatCols - 1) / kStatCols;
+    const int64_t nw = gx * wch;
+    const int64_t total = nw + gx * xch;
+    for (int64_t t = blockIdx.x; t < total; t += gridDim.x) {
+        if (t < nw) {
+            column_stats_tile<TW>(w, n_out, cols, wsum, wsq, t % gx, t / gx, red);
+        } else {
+            const int64_t u = t - nw;
+            column_stats_tile<TX>(x, tokens, cols, nullptr, xsq, u % gx, u / gx, red);
+        }
+        __syncthreads();   // the next tile reuses red
     }
 }
 
@@ -1030,19 +1055,26 @@ cudaError_t launch_mx_channel_scale(const void* x, int xdt, int64_t tokens, cons
     double* wsum = reinterpret_cast<double*>(ws);
     double* wsq = wsum + wch * cols;
     double* xsq = wsq + wch * cols;
-    const unsigned gx = (unsigned)((cols + kStatCols - 1) / kStatCols);
-    if (wdt == 1)
-        column_stats_kernel<__nv_bfloat16><<<dim3(gx, (unsigned)wch), kThreads, 0, s>>>(
-            reinterpret_cast<const __nv_bfloat16*>(w), n_out, cols, wsum, wsq);
+    const int64_t tiles = (cols + kStatCols - 1) / kStatCols * (wch + xch);
+    auto launch = [&](auto kernel, const auto* wp, const auto* xp) {
+        int per_sm = 0;
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kThreads, 0);
+        const int64_t cap = (int64_t)num_sms() * (per_sm < 1 ? 1 : per_sm);
+        const unsigned grid = (unsigned)(tiles < cap ? tiles : cap);
+        kernel<<<grid, kThreads, 0, s>>>(wp, n_out, wsum, wsq, wch, xp, tokens, xsq, xch, cols);
+    };
+    const auto* wb = reinterpret_cast<const __nv_bfloat16*>(w);
+    const auto* wf = reinterpret_cast<const float*>(w);
+    const auto* xb = reinterpret_cast<const __nv_bfloat16*>(x);
+    const auto* xf = reinterpret_cast<const float*>(x);
+    if (wdt == 1 && xdt == 1)
+        launch(column_stats_kernel<__nv_bfloat16, __nv_bfloat16>, wb, xb);
+    else if (wdt == 1)
+        launch(column_stats_kernel<__nv_bfloat16, float>, wb, xf);
+    else if (xdt == 1)
+        launch(column_stats_kernel<float, __nv_bfloat16>, wf, xb);
     else
-        column_stats_kernel<float><<<dim3(gx, (unsigned)wch), kThreads, 0, s>>>(
-            reinterpret_cast<const float*>(w), n_out, cols, wsum, wsq);
-    if (xdt == 1)
-        column_stats_kernel<__nv_bfloat16><<<dim3(gx, (unsigned)xch), kThreads, 0, s>>>(
-            reinterpret_cast<const __nv_bfloat16*>(x), tokens, cols, nullptr, xsq);
-    else
-        column_stats_kernel<float><<<dim3(gx, (unsigned)xch), kThreads, 0, s>>>(
-            reinterpret_cast<const float*>(x), tokens, cols, nullptr, xsq);
+        launch(column_stats_kernel<float, float>, wf, xf);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess)
         return e;
