@@ -553,12 +553,16 @@ hessian_reduce_kernel(const float* __restrict__ part, int64_t nchunk, int64_t to
 // Column statistics in fp64 over a chunk of kStatRows rows: sum and sum of
 // squares.  A tile is one chunk x 256 columns: lane l of every warp owns the 8
 // consecutive columns 8 l .. 8 l + 7 of the tile (one 16-byte bf16 vector or
-// two fp32 vectors per row), and warp w takes rows w, w + 8, w + 16, ... of the
-// chunk, 8 rows per batch with all 8 loads issued before the sums.  The 8
-// warps' partial sums are then added in warp order through shared memory.
+// two fp32 vectors per row), and warp w adds rows w, w + 8, w + 16, ... of the
+// chunk in that order, loading them in batches with the next batch in flight
+// while the current one is added.  The 8 warps' partial sums are then added in
+// warp order through shared memory.
 constexpr int kStatRows = 256;
 constexpr int kStatCols = 256;
 constexpr int kStatWarps = kThreads / 32;
+// 16-byte words a lane loads per batch: 4 rows of bf16 or 2 of fp32 (a deeper
+// batch raises the double-buffered registers past two CTAs per SM)
+constexpr int kStatBatchWords = 4;
 
 template <typename T>
 __device__ __forceinline__ void column_stats_tile(const T* __restrict__ x, int64_t rows, int64_t cols,
@@ -578,21 +582,64 @@ __device__ __forceinline__ void column_stats_tile(const T* __restrict__ x, int64
         s[i] = 0.0;
         q[i] = 0.0;
     }
+    // whole batches of kB rows are double-buffered, the rest go row by row
+    constexpr int kWd = (int)sizeof(T) / 2;        // 16-byte words per row slice
+    constexpr int kB = kStatBatchWords / kWd;      // rows per batch
+    auto load_batch = [&](int64_t rb, uint4 (&wv)[kB][kWd]) {
+#pragma unroll
+        for (int k = 0; k < kB; ++k)
+#pragma unroll
+            for (int h = 0; h < kWd; ++h)
+                wv[k][h] = __ldg(reinterpret_cast<const uint4*>(x + (rb + k * kStatWarps) * cols + c0) + h);
+    };
+    auto add_batch = [&](const uint4 (&wv)[kB][kWd]) {
+#pragma unroll
+        for (int k = 0; k < kB; ++k) {
+#pragma unroll
+            for (int h = 0; h < kWd; ++h) {
+                const uint32_t u[4] = {wv[k][h].x, wv[k][h].y, wv[k][h].z, wv[k][h].w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    if constexpr (sizeof(T) == 4) {
+                        const double d = (double)__uint_as_float(u[e]);
+                        s[4 * h + e] += d;
+                        q[4 * h + e] = fma(d, d, q[4 * h + e]);
+                    } else {
+                        const double d0 = (double)__uint_as_float(u[e] << 16);
+                        const double d1 = (double)__uint_as_float(u[e] & 0xFFFF0000u);
+                        s[2 * e] += d0;
+                        q[2 * e] = fma(d0, d0, q[2 * e]);
+                        s[2 * e + 1] += d1;
+                        q[2 * e + 1] = fma(d1, d1, q[2 * e + 1]);
+                    }
+                }
+            }
+        }
+    };
+    constexpr int64_t kSpan = (int64_t)(kB - 1) * kStatWarps;   // a batch's last row offset
+    constexpr int64_t kStep = (int64_t)kB * kStatWarps;
     int64_t r = r0 + warp;
     if (own) {
-        for (; r + 7 * kStatWarps < r1; r += 8 * kStatWarps) {
-            float v[8][8];
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-                load_elems<T, 8>(x + (r + k * kStatWarps) * cols + c0, v[k]);
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const double d = (double)v[k][i];
-                    s[i] += d;
-                    q[i] = fma(d, d, q[i]);
-                }
+        if (r + kSpan < r1) {
+            uint4 wa[kB][kWd], wb[kB][kWd];
+            load_batch(r, wa);
+            for (;;) {
+                const int64_t ra = r + kStep;
+                const bool more_a = ra + kSpan < r1;
+                if (more_a)
+                    load_batch(ra, wb);
+                add_batch(wa);
+                r = ra;
+                if (!more_a)
+                    break;
+                const int64_t rb = r + kStep;
+                const bool more_b = rb + kSpan < r1;
+                if (more_b)
+                    load_batch(rb, wa);
+                add_batch(wb);
+                r = rb;
+                if (!more_b)
+                    break;
             }
         }
         for (; r < r1; r += kStatWarps) {
