@@ -720,26 +720,25 @@ razer_quant_kernel(const T* __restrict__ x, int64_t nblk, GsArgs gs, SpecialArgs
 // is then nonzero with that sign), so with d = |y - v|:
 //   +m candidate: special iff v > 0 and |y - m| < d
 //   -m candidate: special iff v < 0 and |y + m| < d
-// (|y -/+ m| is the |(|y|) - m| of the general rule, written without |y|).
+// A nonzero v has the sign of y, so both distances are ||y| - m| (RN(-a) =
+// -RN(a)): one subtraction per magnitude serves the pair.
 // Each candidate's in-order fma chain takes either the grid error e or the
 // special error es; the choice is a predicated fma pair on the FMA pipe
 // rather than a select on the integer pipe, and the element's bit enters
 // that candidate's mask under the same predicate.
 // One pair's two candidates; operands: %0/%1 the +/- chains, %2/%3 their
-// masks, %4 y, %5 e, %6 m, %7 es, %8 the element's bit; d, pp, pn shared.
-#define FP4Q_RAZER_PAIR_PTX(A0, A1, M0, M1, Y, E, MAG, ES, BIT)        \
-    "sub.rn.f32 t, " Y ", " MAG ";\n\t"                                \
-    "abs.f32 t, t;\n\t"                                                \
-    "setp.lt.and.f32 q, t, d, pp;\n\t"                                 \
+// masks, e the grid error, m, es, the element's bit; ay = |y|, d, pp, pn shared.
+#define FP4Q_RAZER_PAIR_PTX(A0, A1, M0, M1, E, MAG, ES, BIT)           \
+    "sub.rn.f32 t, ay, " MAG ";\n\t"                                 \
+    "abs.f32 t, t;\n\t"                                              \
+    "setp.lt.and.f32 q, t, d, pp;\n\t"                               \
+    "setp.lt.and.f32 r, t, d, pn;\n\t"                               \
     "@!q fma.rn.f32 " A0 ", " E ", " E ", " A0 ";\n\t"                 \
     "@q fma.rn.f32 " A0 ", " ES ", " ES ", " A0 ";\n\t"                \
     "@q or.b32 " M0 ", " M0 ", " BIT ";\n\t"                           \
-    "add.rn.f32 t, " Y ", " MAG ";\n\t"                                \
-    "abs.f32 t, t;\n\t"                                                \
-    "setp.lt.and.f32 q, t, d, pn;\n\t"                                 \
-    "@!q fma.rn.f32 " A1 ", " E ", " E ", " A1 ";\n\t"                 \
-    "@q fma.rn.f32 " A1 ", " ES ", " ES ", " A1 ";\n\t"                \
-    "@q or.b32 " M1 ", " M1 ", " BIT ";\n\t"
+    "@!r fma.rn.f32 " A1 ", " E ", " E ", " A1 ";\n\t"                 \
+    "@r fma.rn.f32 " A1 ", " ES ", " ES ", " A1 ";\n\t"                \
+    "@r or.b32 " M1 ", " M1 ", " BIT ";\n\t"
 
 template <int NPAIR>
 __device__ __forceinline__ void razer_pair_step(float y, float v, float e, const float (&mag)[NPAIR],
@@ -749,26 +748,28 @@ __device__ __forceinline__ void razer_pair_step(float y, float v, float e, const
     static_assert(NPAIR == 1 || NPAIR == 2, "one or two pairs");
     if constexpr (NPAIR == 1) {
         asm("{\n\t"
-            ".reg .pred pp, pn, q;\n\t"
-            ".reg .f32 d, t;\n\t"
+            ".reg .pred pp, pn, q, r;\n\t"
+            ".reg .f32 d, t, ay;\n\t"
             "setp.gt.f32 pp, %5, 0f00000000;\n\t"
             "setp.lt.f32 pn, %5, 0f00000000;\n\t"
             "sub.rn.f32 d, %4, %5;\n\t"
             "abs.f32 d, d;\n\t"
-            FP4Q_RAZER_PAIR_PTX("%0", "%1", "%2", "%3", "%4", "%6", "%7", "%8", "%9")
+            "abs.f32 ay, %4;\n\t"
+            FP4Q_RAZER_PAIR_PTX("%0", "%1", "%2", "%3", "%6", "%7", "%8", "%9")
             "}"
             : "+f"(acc[0]), "+f"(acc[1]), "+r"(mask[0]), "+r"(mask[1])
             : "f"(y), "f"(v), "f"(e), "f"(mag[0]), "f"(es[0]), "r"(bit));
     } else {
         asm("{\n\t"
-            ".reg .pred pp, pn, q;\n\t"
-            ".reg .f32 d, t;\n\t"
+            ".reg .pred pp, pn, q, r;\n\t"
+            ".reg .f32 d, t, ay;\n\t"
             "setp.gt.f32 pp, %9, 0f00000000;\n\t"
             "setp.lt.f32 pn, %9, 0f00000000;\n\t"
             "sub.rn.f32 d, %8, %9;\n\t"
             "abs.f32 d, d;\n\t"
-            FP4Q_RAZER_PAIR_PTX("%0", "%1", "%4", "%5", "%8", "%10", "%11", "%13", "%15")
-            FP4Q_RAZER_PAIR_PTX("%2", "%3", "%6", "%7", "%8", "%10", "%12", "%14", "%15")
+            "abs.f32 ay, %8;\n\t"
+            FP4Q_RAZER_PAIR_PTX("%0", "%1", "%4", "%5", "%10", "%11", "%13", "%15")
+            FP4Q_RAZER_PAIR_PTX("%2", "%3", "%6", "%7", "%10", "%12", "%14", "%15")
             "}"
             : "+f"(acc[0]), "+f"(acc[1]), "+f"(acc[2]), "+f"(acc[3]), "+r"(mask[0]), "+r"(mask[1]),
               "+r"(mask[2]), "+r"(mask[3])
